@@ -1,0 +1,255 @@
+"""Thin Python binding of libsmuon.so (the C ABI in include/smuon.h).
+
+Argument marshalling only: every step of the optimizer runs in the library's
+CUDA kernels. PyTorch supplies device memory and the current stream. There is
+no fallback: if the shared library is missing, importing a function raises.
+
+Functions keep the C names: smuon_ns, smuon_sign_pack, smuon_vote,
+smuon_update, cachemuon_reuse_probe, lionmuon_step (plus the workspace
+queries). Matrices are 2-D torch tensors with unit column stride.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_float, c_int8, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsmuon.so")
+
+F32, BF16, I8 = 0, 1, 2
+NS_FP32_REF, NS_SPLIT_BF16, NS_NO_NORMALIZE, NS_EMIT_Q, NS_SIMT_BF16 = 1, 2, 4, 8, 16
+VOTE_POPCOUNT, VOTE_INT8 = 0, 1
+DEV_NONFINITE_NORM, DEV_WAIT_TIMEOUT = 1, 2
+
+STATUS_NAMES = {0: "OK", -1: "INVALID_ARG", -2: "SHAPE", -3: "DTYPE", -4: "UNSUPPORTED",
+                -5: "WORKSPACE", -6: "CUDA"}
+
+
+class SmuonError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"smuon status {code} ({STATUS_NAMES.get(code, '?')}): {msg}")
+        self.code = code
+
+
+class SmuonMat(ctypes.Structure):
+    _fields_ = [("data", c_void_p), ("rows", c_int32), ("cols", c_int32), ("ld", c_int64),
+                ("dtype", c_int32)]
+
+
+class CacheMuonCounters(ctypes.Structure):
+    _fields_ = [("hits", c_int64), ("misses", c_int64), ("probes", c_int64), ("reserved", c_int64)]
+
+
+class TraceRec(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 40), ("kind", c_int32), ("work", ctypes.c_double), ("ms", c_float)]
+
+
+class LionMuonState(ctypes.Structure):
+    _fields_ = [("n_layers", c_int32), ("workers", c_int32), ("W", POINTER(SmuonMat)),
+                ("mom", POINTER(SmuonMat)), ("t", c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libsmuon.so once; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m matrix_aware_sign_b200.build` (there is no fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        M = POINTER(SmuonMat)
+        sigs = {
+            "smuon_last_error": (ctypes.c_char_p, []),
+            "smuon_version": (c_int32, []),
+            "smuon_launch_count": (c_int64, []),
+            "smuon_trace_enable": (None, [c_int32]),
+            "smuon_trace_read": (c_int32, [POINTER(TraceRec), c_int32]),
+            "smuon_ns_workspace_bytes": (c_int32, [M, c_int32, c_int32, c_uint32, POINTER(c_size_t)]),
+            "smuon_ns": (c_int32, [M, M, c_int32, M, c_float, c_float, c_float, c_float, c_int32, c_float,
+                                   c_uint32, M, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+            "smuon_sign_pack": (c_int32, [M, c_int32, c_void_p, c_void_p, c_void_p]),
+            "smuon_vote": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int8, c_void_p, c_void_p]),
+            "smuon_update": (c_int32, [M, c_int32, M, M, M, c_int32, c_float, c_int8, c_uint32,
+                                       POINTER(c_void_p), POINTER(c_void_p), c_void_p]),
+            "cachemuon_workspace_bytes": (c_int32, [M, POINTER(c_size_t)]),
+            "cachemuon_reuse_probe": (c_int32, [M, M, M, c_float, c_float, c_void_p, c_void_p, c_void_p,
+                                                c_void_p, c_size_t, c_void_p, c_void_p]),
+            "lionmuon_workspace_bytes": (c_int32, [POINTER(LionMuonState), c_int32, c_uint32,
+                                                   POINTER(c_size_t)]),
+            "lionmuon_step": (c_int32, [POINTER(LionMuonState), c_int32, c_float, c_float, c_float, c_float,
+                                        c_float, c_float, c_int32, c_int8, c_uint32, M, c_void_p, c_size_t,
+                                        c_void_p, c_void_p]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(code: int) -> None:
+    if code != 0:
+        raise SmuonError(code, lib().smuon_last_error().decode())
+
+
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.int8: I8}
+
+
+def mat(t: torch.Tensor) -> SmuonMat:
+    """Describes a 2-D row-major tensor (unit column stride)."""
+    if t.dim() != 2 or (t.stride(1) != 1 and t.shape[1] > 1):
+        raise ValueError("matrices must be 2-D with unit column stride")
+    if t.dtype not in _DT:
+        raise ValueError(f"dtype {t.dtype} is not supported")
+    ld = t.stride(0) if t.shape[0] > 1 else t.shape[1]
+    return SmuonMat(t.data_ptr(), t.shape[0], t.shape[1], max(ld, t.shape[1]), _DT[t.dtype])
+
+
+def _mats(ts):
+    if ts is None:
+        return None
+    arr = (SmuonMat * len(ts))(*[mat(t) for t in ts])
+    return arr
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """Caller-owned workspace (torch allocation, 512-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+# ---------------------------------------------------------------- diagnostics
+WORK_FLOPS, WORK_BYTES = 0, 1
+
+
+def launch_count() -> int:
+    return lib().smuon_launch_count()
+
+
+def trace_enable(on: bool = True) -> None:
+    lib().smuon_trace_enable(1 if on else 0)
+
+
+def trace_read() -> list[dict]:
+    """Synchronises on the logged launch events and returns and clears them."""
+    n = lib().smuon_trace_read(None, 0)
+    if n == 0:
+        return []
+    buf = (TraceRec * n)()
+    got = lib().smuon_trace_read(buf, n)
+    return [dict(name=r.name.decode(), kind=r.kind, work=r.work, ms=r.ms) for r in buf[:got]]
+
+
+# ---------------------------------------------------------------- smuon_ns
+def smuon_ns_workspace_bytes(M_in, iters: int, flags: int = 0) -> int:
+    arr = _mats(M_in)
+    out = c_size_t(0)
+    _check(lib().smuon_ns_workspace_bytes(arr, len(M_in), iters, flags, ctypes.byref(out)))
+    return out.value
+
+
+def smuon_ns(M_in, U_out, a, b, c, iters, G=None, beta=0.0, eps=1e-7, flags=0, Q_out=None,
+             skip_if=None, ws=None, status=None, stream=None):
+    """Momentum (when G is given) + Frobenius normalisation + K Newton-Schulz steps."""
+    if ws is None:
+        ws = workspace(smuon_ns_workspace_bytes(M_in, iters, flags), M_in[0].device)
+    _check(lib().smuon_ns(_mats(M_in), _mats(U_out), len(M_in), _mats(G), beta, a, b, c, iters, eps, flags,
+                          _mats(Q_out), _ptr(skip_if), ws.data_ptr(), ws.numel(), _ptr(status),
+                          _stream(stream)))
+    return ws
+
+
+# ---------------------------------------------------------------- sign / vote / update
+def packed_words(n: int) -> int:
+    return ((n + 127) // 128) * 4
+
+
+def smuon_sign_pack(U, packed=None, signs_i8=None, stream=None):
+    _check(lib().smuon_sign_pack(_mats(U), len(U), _ptr(packed), _ptr(signs_i8), _stream(stream)))
+
+
+def smuon_vote(M: int, N: int, vote, packed=None, signs_i8=None, tie_value: int = 0, stream=None):
+    _check(lib().smuon_vote(_ptr(packed), _ptr(signs_i8), M, N, tie_value, vote.data_ptr(), _stream(stream)))
+
+
+def smuon_update(W, eta: float, U=None, votes=None, dense=None, M: int = 1, tie_value: int = 0,
+                 vote_kind: int = VOTE_POPCOUNT, packed_out=None, vote_out=None, stream=None):
+    """U is a list over layers of lists over workers (flattened worker-minor)."""
+    Uflat = None if U is None else [u for layer in U for u in layer]
+    n = len(W)
+    po = None if packed_out is None else (c_void_p * n)(*[_ptr(p) for p in packed_out])
+    vo = None if vote_out is None else (c_void_p * n)(*[_ptr(v) for v in vote_out])
+    _check(lib().smuon_update(_mats(W), n, _mats(Uflat), _mats(votes), _mats(dense), M, eta, tie_value,
+                              vote_kind, po, vo, _stream(stream)))
+
+
+# ---------------------------------------------------------------- CacheMuon
+def cachemuon_workspace_bytes(M_t) -> int:
+    out = c_size_t(0)
+    _check(lib().cachemuon_workspace_bytes(ctypes.byref(mat(M_t)), ctypes.byref(out)))
+    return out.value
+
+
+def new_counters(device=None) -> torch.Tensor:
+    """Device storage for cachemuon_counters (4 x int64)."""
+    return torch.zeros(4, dtype=torch.int64, device=device or "cuda")
+
+
+def cachemuon_reuse_probe(Q, M_t, D_hat, gamma, err, accept, counters=None, eps=1e-7, ws=None, status=None,
+                          stream=None):
+    if ws is None:
+        ws = workspace(cachemuon_workspace_bytes(M_t), M_t.device)
+    qm = None if Q is None else ctypes.byref(mat(Q))
+    _check(lib().cachemuon_reuse_probe(qm, ctypes.byref(mat(M_t)), ctypes.byref(mat(D_hat)), gamma, eps,
+                                       err.data_ptr(), accept.data_ptr(), _ptr(counters), ws.data_ptr(),
+                                       ws.numel(), _ptr(status), _stream(stream)))
+    return ws
+
+
+# ---------------------------------------------------------------- LionMuon
+class LionMuon:
+    """Holds the C lionmuon_state for lists W[layer] and mom[layer][worker]."""
+
+    def __init__(self, W, mom, t: int = 0):
+        self.W = list(W)
+        self.mom = [list(m) for m in mom]
+        self.workers = len(self.mom[0])
+        self._w = _mats(self.W)
+        self._m = _mats([m for layer in self.mom for m in layer])
+        self.state = LionMuonState(len(self.W), self.workers, self._w, self._m, t)
+
+    @property
+    def t(self) -> int:
+        return self.state.t
+
+    def workspace_bytes(self, iters: int, ns_flags: int = 0) -> int:
+        out = c_size_t(0)
+        _check(lib().lionmuon_workspace_bytes(ctypes.byref(self.state), iters, ns_flags, ctypes.byref(out)))
+        return out.value
+
+
+def lionmuon_step(opt: LionMuon, G, P, beta1, beta2, eta, a, b, c, iters, tie_value=0, ns_flags=0, ws=None,
+                  status=None, stream=None):
+    """G is a list over layers of lists over workers. Returns the workspace used."""
+    if ws is None:
+        ws = workspace(opt.workspace_bytes(iters, ns_flags), opt.W[0].device)
+    Gflat = _mats([g for layer in G for g in layer])
+    _check(lib().lionmuon_step(ctypes.byref(opt.state), P, beta1, beta2, eta, a, b, c, iters, tie_value, ns_flags,
+                               Gflat, ws.data_ptr(), ws.numel(), _ptr(status), _stream(stream)))
+    return ws

@@ -1,0 +1,1007 @@
+// abi.cu -- host side of the C ABI declared in include/smuon.h.
+//
+// Checks arguments before enqueueing anything, lays out the caller's
+// workspace, builds the device plan (groups, per-matrix descriptors, TMA
+// tensor maps, tile tables), uploads it with a kernel and launches the
+// stage kernels on the caller's stream. The host never reads device data.
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "kernels.cuh"
+
+using namespace smuon;
+
+namespace {
+
+thread_local std::string g_err;
+
+smuon_status fail(smuon_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                  \
+  do {                                                                                  \
+    cudaError_t e_ = (expr);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(SMUON_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));      \
+  } while (0)
+
+// ------------------------------------------------------------------ launch trace
+// Every kernel launch goes through a Launch guard: it counts the launch and,
+// while tracing is on, brackets it with CUDA events on the launch stream and
+// records the launch's algorithmic work (flops or bytes) for roofline reports.
+struct TraceRec {
+  const char* name;
+  int32_t kind;
+  double work;
+  cudaEvent_t a, b;
+};
+
+std::mutex g_tr_mu;
+bool g_tr_on = false;
+std::vector<TraceRec> g_tr;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_ev_free;
+std::atomic<long long> g_launches{0};
+
+struct Launch {
+  TraceRec r{};
+  bool on = false;
+  cudaStream_t s;
+  Launch(const char* name, int32_t kind, double work, cudaStream_t st) : s(st) {
+    g_launches.fetch_add(1);
+    std::lock_guard<std::mutex> lk(g_tr_mu);
+    if (!g_tr_on || g_tr.size() >= 1000000) return;
+    r.name = name; r.kind = kind; r.work = work;
+    if (!g_ev_free.empty()) {
+      r.a = g_ev_free.back().first; r.b = g_ev_free.back().second;
+      g_ev_free.pop_back();
+    } else if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) {
+      return;
+    }
+    on = true;
+    cudaEventRecord(r.a, s);
+  }
+  ~Launch() {
+    if (!on) return;
+    cudaEventRecord(r.b, s);
+    std::lock_guard<std::mutex> lk(g_tr_mu);
+    g_tr.push_back(r);
+  }
+};
+
+// ------------------------------------------------------------------ device info
+struct DevInfo {
+  int sms = 0;
+  int major = 0, minor = 0;
+  bool ok = false;
+};
+
+std::mutex g_dev_mu;
+std::map<int, DevInfo> g_dev;
+
+smuon_status device_info(DevInfo* out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  auto it = g_dev.find(dev);
+  if (it == g_dev.end()) {
+    DevInfo d;
+    CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    CUDA_TRY(cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev));
+    CUDA_TRY(cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev));
+    d.ok = (d.major == 10 && d.minor == 0);
+    it = g_dev.emplace(dev, d).first;
+  }
+  *out = it->second;
+  if (!out->ok)
+    return fail(SMUON_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", dev,
+                out->major, out->minor);
+  return SMUON_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+smuon_status get_encoder(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return fail(SMUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available (%s)", cudaGetErrorString(err));
+  *fn = cached;
+  return SMUON_OK;
+}
+
+// 3-D bf16 map over [count][rows][ld] with box {box0 (inner), box1, 1}, 128B swizzle
+smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, int64_t rows, int64_t count,
+                            int64_t ld, uint32_t box0, uint32_t box1) {
+  EncodeTiledFn enc;
+  smuon_status st = get_encoder(&enc);
+  if (st != SMUON_OK) return st;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)count};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(ld * 2 * rows)};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SMUON_OK;
+}
+
+// ------------------------------------------------------------------ validation
+int dtype_size(int32_t dt) { return dt == SMUON_F32 ? 4 : dt == SMUON_BF16 ? 2 : dt == SMUON_I8 ? 1 : 0; }
+
+smuon_status check_mat(const smuon_mat& m, const char* what, int i, bool allow_f32, bool allow_bf16,
+                       bool allow_i8) {
+  if (!m.data) return fail(SMUON_ERR_INVALID_ARG, "%s[%d].data is NULL", what, i);
+  if (m.rows < 1 || m.cols < 1 || m.rows > 65536 || m.cols > 65536)
+    return fail(SMUON_ERR_SHAPE, "%s[%d] has shape %dx%d (each side must be in 1..65536)", what, i, m.rows, m.cols);
+  if (m.ld < m.cols) return fail(SMUON_ERR_SHAPE, "%s[%d].ld=%lld < cols=%d", what, i, (long long)m.ld, m.cols);
+  const bool ok = (m.dtype == SMUON_F32 && allow_f32) || (m.dtype == SMUON_BF16 && allow_bf16) ||
+                  (m.dtype == SMUON_I8 && allow_i8);
+  if (!ok) return fail(SMUON_ERR_DTYPE, "%s[%d] has an unsupported dtype %d", what, i, m.dtype);
+  if (reinterpret_cast<uintptr_t>(m.data) % dtype_size(m.dtype) != 0)
+    return fail(SMUON_ERR_INVALID_ARG, "%s[%d].data is not aligned to its element size", what, i);
+  return SMUON_OK;
+}
+
+bool same_shape(const smuon_mat& a, const smuon_mat& b) { return a.rows == b.rows && a.cols == b.cols; }
+
+// ------------------------------------------------------------------ NS plan
+struct NsRequest {
+  const smuon_mat* M_in;
+  const smuon_mat* U_out;
+  int32_t n_mats;
+  const smuon_mat* G;
+  float beta, a, b, c;
+  int32_t iters;
+  float eps;
+  uint32_t flags;
+  const smuon_mat* Q_out;   // EMIT_Q outputs, or (probe) the user's cached Q
+  bool probe;               // build the CacheMuon REUSE + PROBE plan instead of the NS chain
+  float gamma;
+};
+
+struct Layout {
+  size_t plan_bytes = 0, total = 0;
+  size_t off_groups = 0, off_mats = 0, off_tmaps = 0;
+  size_t off_partials = 0, off_scale = 0, off_probe = 0;
+  int n_tmaps = 0;
+};
+
+struct Builder {
+  std::vector<GroupDesc> groups;
+  std::vector<MatDesc> mats;
+  std::vector<CUtensorMap> maps;
+  PlanHeader h{};
+  Layout L;
+  size_t cursor = 0;
+  char* base = nullptr;  // device workspace base (nullptr while sizing)
+
+  size_t take(size_t bytes) {
+    cursor = (size_t)round_up((int64_t)cursor, 256);
+    size_t o = cursor;
+    cursor += bytes;
+    return o;
+  }
+  template <class T>
+  T* ptr_at(size_t off) {
+    return base ? reinterpret_cast<T*>(base + off) : nullptr;
+  }
+};
+
+Mode pick_mode(uint32_t flags) {
+  if (flags & SMUON_NS_FP32_REF) return MODE_SIMT_F32;
+  if (flags & SMUON_NS_SIMT_BF16) return MODE_SIMT_BF16;
+  return MODE_TC_BF16;
+}
+
+// Builds groups, descriptors and the workspace layout. With base == nullptr it
+// only sizes the workspace; otherwise it also fills device pointers and maps.
+smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
+  B->base = base;
+  const Mode mode = pick_mode(rq.flags);
+  const bool bf = (mode != MODE_SIMT_F32);
+  const bool tc = (mode == MODE_TC_BF16);
+  const bool emit_q = (rq.flags & SMUON_NS_EMIT_Q) && !rq.probe;
+  const int K = rq.iters;
+  const int BM = tc ? kTcBM : kSimtBM, BN = tc ? kTcBN : kSimtBN;
+  const size_t esz = bf ? 2 : 4;
+  // split BF16: operand buffers hold [hi parts of all matrices][lo parts of all matrices]
+  const int parts = (tc && (rq.flags & SMUON_NS_SPLIT_BF16) && !rq.probe) ? 2 : 1;
+
+  // group by wide shape, biggest first
+  std::map<std::pair<int, int>, std::vector<int>> by_shape;
+  for (int i = 0; i < rq.n_mats; ++i) {
+    const smuon_mat& M = rq.M_in[i];
+    by_shape[{std::min(M.rows, M.cols), std::max(M.rows, M.cols)}].push_back(i);
+  }
+  std::vector<std::pair<std::pair<int, int>, std::vector<int>>> order(by_shape.begin(), by_shape.end());
+  std::stable_sort(order.begin(), order.end(), [](const auto& x, const auto& y) {
+    return (int64_t)x.first.first * x.first.second > (int64_t)y.first.first * y.first.second;
+  });
+
+  B->groups.clear();
+  B->mats.clear();
+  B->maps.clear();
+  int mom_tiles = 0;
+  for (auto& kv : order) {
+    GroupDesc g{};
+    g.m = kv.first.first;
+    g.n = kv.first.second;
+    g.count = (int32_t)kv.second.size();
+    g.first_mat = (int32_t)B->mats.size();
+    g.ldn = round_up(g.n, 128);
+    g.ldm = round_up(g.m, 128);
+    for (int z = 0; z < g.count; ++z) {
+      const int i = kv.second[z];
+      const smuon_mat& M = rq.M_in[i];
+      MatDesc d{};
+      d.m_ptr = M.data; d.m_ld = M.ld; d.m_dtype = M.dtype;
+      if (rq.G) { d.g_ptr = rq.G[i].data; d.g_ld = rq.G[i].ld; d.g_dtype = rq.G[i].dtype; }
+      d.u_ptr = rq.U_out[i].data; d.u_ld = rq.U_out[i].ld; d.u_dtype = rq.U_out[i].dtype;
+      if (rq.Q_out && (emit_q || rq.probe)) { d.q_ptr = rq.Q_out[i].data; d.q_ld = rq.Q_out[i].ld; }
+      d.rows = M.rows; d.cols = M.cols; d.tall = M.rows > M.cols ? 1 : 0;
+      d.group = (int32_t)B->groups.size();
+      d.z = z;
+      d.mom_tiles_c = ceil_div(M.cols, 64);
+      d.mom_count = ceil_div(M.rows, 64) * d.mom_tiles_c;
+      d.mom_begin = mom_tiles;
+      mom_tiles += d.mom_count;
+      B->mats.push_back(d);
+    }
+    B->groups.push_back(g);
+  }
+  // momentum tiles must be increasing along mats for the device binary search: they are.
+
+  // tile tables
+  int totals[ST_COUNT] = {0};
+  for (auto& g : B->groups) {
+    const int tmm = ceil_div(g.m, BM);
+    for (int st = 0; st < ST_COUNT; ++st) {
+      const int No = (st == ST_AXPY || st == ST_REUSE) ? g.n : g.m;
+      g.tiles_m[st] = tmm;
+      g.tiles_n[st] = ceil_div(No, BN);
+      g.tile_begin[st] = totals[st];
+      totals[st] += g.count * g.tiles_m[st] * g.tiles_n[st];
+    }
+  }
+
+  // layout: plan region first
+  Layout& L = B->L;
+  B->cursor = 0;
+  const size_t hdr = B->take(sizeof(Plan));
+  (void)hdr;
+  L.off_groups = B->take(sizeof(GroupDesc) * B->groups.size());
+  L.off_mats = B->take(sizeof(MatDesc) * B->mats.size());
+  // tensor maps: count them first
+  auto want_map = [&](int32_t& slot) { slot = L.n_tmaps++; };
+  L.n_tmaps = 0;
+  for (auto& g : B->groups) {
+    for (int i = 0; i < 2; ++i) { g.tm_x_k[i] = g.tm_x_mn[i] = g.tm_q_mn[i] = -1; }
+    g.tm_a_k = g.tm_b_k = g.tm_uq_k = -1;
+    if (!tc) continue;
+    if (!rq.probe) {
+      want_map(g.tm_x_k[0]);
+      want_map(g.tm_x_mn[0]);
+      if (K >= 2) { want_map(g.tm_x_k[1]); want_map(g.tm_x_mn[1]); }
+      if (rq.c != 0.f) want_map(g.tm_a_k);
+      want_map(g.tm_b_k);
+      if (emit_q && K >= 2) want_map(g.tm_q_mn[1]);
+      if (emit_q && K >= 3) want_map(g.tm_q_mn[0]);
+    } else {
+      want_map(g.tm_x_mn[0]);
+      want_map(g.tm_uq_k);
+      want_map(g.tm_x_k[1]);
+    }
+  }
+  L.off_tmaps = B->take(sizeof(CUtensorMap) * std::max(L.n_tmaps, 1));
+  L.plan_bytes = (size_t)round_up((int64_t)B->cursor, 256);
+  L.off_partials = B->take(sizeof(float) * std::max(mom_tiles, 1));
+  L.off_scale = B->take(sizeof(float) * B->mats.size());
+  L.off_probe = B->take(sizeof(float) * 4 * std::max(totals[ST_PROBE], 1));
+
+  // per-group buffers
+  for (auto& g : B->groups) {
+    const size_t nx = (size_t)g.count * g.m * g.ldn, nm = (size_t)g.count * g.m * g.ldm;
+    g.xop[0] = B->ptr_at<void>(B->take(nx * esz * parts));
+    g.xop[1] = nullptr;
+    g.xf[0] = g.xf[1] = nullptr;
+    g.af = nullptr; g.aop = nullptr; g.bop = nullptr;
+    g.qf[0] = g.qf[1] = nullptr; g.qop[0] = g.qop[1] = nullptr;
+    if (rq.probe) {
+      g.xop[1] = B->ptr_at<void>(B->take(nx * esz));
+      continue;
+    }
+    if (K >= 2) g.xop[1] = B->ptr_at<void>(B->take(nx * esz * parts));
+    if (bf && K >= 2) g.xf[1] = B->ptr_at<float>(B->take(nx * 4));
+    if (bf && K >= 3) g.xf[0] = B->ptr_at<float>(B->take(nx * 4));
+    if (rq.c != 0.f) {
+      g.af = B->ptr_at<float>(B->take(nm * 4));
+      g.aop = bf ? B->ptr_at<void>(B->take(nm * 2 * parts)) : (void*)g.af;
+    }
+    g.bop = B->ptr_at<void>(B->take(nm * esz * parts));
+    if (emit_q && K >= 2) {
+      g.qop[1] = B->ptr_at<void>(B->take(nm * esz * parts));
+      g.qf[1] = bf ? B->ptr_at<float>(B->take(nm * 4)) : reinterpret_cast<float*>(g.qop[1]);
+    }
+    if (emit_q && K >= 3) {
+      g.qop[0] = B->ptr_at<void>(B->take(nm * esz * parts));
+      g.qf[0] = bf ? B->ptr_at<float>(B->take(nm * 4)) : reinterpret_cast<float*>(g.qop[0]);
+    }
+  }
+  L.total = (size_t)round_up((int64_t)B->cursor, 256);
+
+  // header
+  PlanHeader& h = B->h;
+  h = PlanHeader{};
+  h.n_mats = (int32_t)B->mats.size();
+  h.n_groups = (int32_t)B->groups.size();
+  h.n_tmaps = L.n_tmaps;
+  h.mode = mode;
+  h.iters = K;
+  h.flags = rq.flags;
+  h.a = rq.a; h.b = rq.b; h.c = rq.c; h.eps = rq.eps; h.beta = rq.beta; h.gamma = rq.gamma;
+  h.total_mom_tiles = mom_tiles;
+  h.tile_bm = BM; h.tile_bn = BN;
+  for (int st = 0; st < ST_COUNT; ++st) h.total_tiles[st] = totals[st];
+  h.partials = B->ptr_at<float>(L.off_partials);
+  h.scale = B->ptr_at<float>(L.off_scale);
+  h.probe_partials = B->ptr_at<float>(L.off_probe);
+  h.groups = B->ptr_at<GroupDesc>(L.off_groups);
+  h.mats = B->ptr_at<MatDesc>(L.off_mats);
+  h.tmaps = B->ptr_at<CUtensorMap>(L.off_tmaps);
+
+  if (!base) return SMUON_OK;
+
+  // tensor maps
+  B->maps.assign(std::max(L.n_tmaps, 1), CUtensorMap{});
+  for (auto& g : B->groups) {
+    if (!tc) continue;
+    auto enc = [&](int32_t slot, const void* p, int64_t inner, int64_t rows, int64_t cnt, int64_t ld, uint32_t b0,
+                   uint32_t b1) -> smuon_status {
+      if (slot < 0) return SMUON_OK;
+      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, b0, b1);
+    };
+    smuon_status st;
+    const int64_t zc = (int64_t)g.count * parts;  // matrices in the map: hi parts, then lo parts
+    for (int i = 0; i < 2; ++i) {
+      if ((st = enc(g.tm_x_k[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 128)) != SMUON_OK) return st;
+      if ((st = enc(g.tm_x_mn[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 64)) != SMUON_OK) return st;
+      if ((st = enc(g.tm_q_mn[i], g.qop[i], g.m, g.m, zc, g.ldm, 64, 64)) != SMUON_OK) return st;
+    }
+    if ((st = enc(g.tm_a_k, g.aop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_b_k, g.bop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
+    if (g.tm_uq_k >= 0) {
+      const MatDesc& d = B->mats[g.first_mat];
+      if ((st = enc(g.tm_uq_k, d.q_ptr, g.m, g.m, 1, d.q_ld, 64, 128)) != SMUON_OK) return st;
+    }
+  }
+  return SMUON_OK;
+}
+
+smuon_status upload_plan(Builder& B, cudaStream_t s) {
+  std::vector<unsigned char> bytes(B.L.plan_bytes, 0);
+  Plan p;
+  p.h = B.h;
+  memcpy(bytes.data(), &p, sizeof(Plan));
+  memcpy(bytes.data() + B.L.off_groups, B.groups.data(), sizeof(GroupDesc) * B.groups.size());
+  memcpy(bytes.data() + B.L.off_mats, B.mats.data(), sizeof(MatDesc) * B.mats.size());
+  if (B.L.n_tmaps > 0) memcpy(bytes.data() + B.L.off_tmaps, B.maps.data(), sizeof(CUtensorMap) * B.L.n_tmaps);
+  static UploadChunk chunk;  // large parameter block; filled then launched by value
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  for (size_t off = 0; off < bytes.size(); off += kUploadBytes) {
+    const size_t n = std::min(bytes.size() - off, (size_t)kUploadBytes);
+    chunk.dst = B.base + off;
+    chunk.bytes = (int32_t)n;
+    memcpy(chunk.data, bytes.data() + off, n);
+    const int blocks = (int)std::min<size_t>(8, (n / 16 + 255) / 256);
+    Launch L("k_plan_upload", SMUON_WORK_BYTES, 2.0 * n, s);
+    k_plan_upload<<<std::max(blocks, 1), 256, 0, s>>>(chunk);
+    CUDA_TRY(cudaGetLastError());
+  }
+  return SMUON_OK;
+}
+
+// algorithmic flops of one stage over the whole batch: 2 * Mo * No * K per matrix
+double stage_flops(const Builder& B, int st) {
+  double f = 0;
+  for (const GroupDesc& g : B.groups) {
+    const double m = g.m, n = g.n;
+    double per = 0;
+    switch (st) {
+      case ST_GRAM: case ST_PROBE: per = 2 * m * m * n; break;
+      case ST_AXPY: case ST_REUSE: per = 2 * m * n * m; break;
+      default: per = 2 * m * m * m; break;
+    }
+    f += per * g.count;
+  }
+  return f;
+}
+
+// algorithmic bytes of the momentum / normalisation prologue
+double momentum_bytes(const NsRequest& rq, const PlanHeader& h) {
+  double b = 0;
+  const int op = (h.mode == MODE_SIMT_F32) ? 4 : ((h.flags & SMUON_NS_SPLIT_BF16) ? 4 : 2);
+  for (int i = 0; i < rq.n_mats; ++i) {
+    const double n = (double)rq.M_in[i].rows * rq.M_in[i].cols;
+    b += n * dtype_size(rq.M_in[i].dtype) + n * op;
+    if (rq.G) b += n * (dtype_size(rq.G[i].dtype) + 4);
+  }
+  return b;
+}
+
+smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int iter, const int32_t* skip,
+                         const DevInfo& di, cudaStream_t s, double stage_flops) {
+  const int total = h.total_tiles[st];
+  if (total == 0) return SMUON_OK;
+  static const char* tc_names[2] = {"k_gemm_tc", "k_gemm_tc_split"};
+  if (h.mode == MODE_TC_BF16) {
+    const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && st <= ST_QAXPY;
+    Launch L(tc_names[split], SMUON_WORK_FLOPS, stage_flops, s);
+    CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
+  } else {
+    const int grid = std::min(total, di.sms * 6);
+    Launch L(h.mode == MODE_SIMT_F32 ? "k_gemm_simt_f32" : "k_gemm_simt_bf16", SMUON_WORK_FLOPS, stage_flops, s);
+    if (h.mode == MODE_SIMT_F32) k_gemm_simt_f32<<<grid, 256, 0, s>>>(d_plan, st, iter, skip);
+    else k_gemm_simt_bf16<<<grid, 256, 0, s>>>(d_plan, st, iter, skip);
+    CUDA_TRY(cudaGetLastError());
+  }
+  return SMUON_OK;
+}
+
+smuon_status validate_ns(const NsRequest& rq) {
+  if (rq.n_mats < 1 || rq.n_mats > 4096) return fail(SMUON_ERR_INVALID_ARG, "n_mats=%d must be in 1..4096", rq.n_mats);
+  if (!rq.M_in || !rq.U_out) return fail(SMUON_ERR_INVALID_ARG, "M_in and U_out must not be NULL");
+  if (rq.iters < 1 || rq.iters > 64) return fail(SMUON_ERR_INVALID_ARG, "iters=%d must be in 1..64", rq.iters);
+  const uint32_t known =
+      SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_SIMT_BF16;
+  if (rq.flags & ~known) return fail(SMUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", rq.flags & ~known);
+  const uint32_t modes = rq.flags & (SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_SIMT_BF16);
+  if (modes & (modes - 1))
+    return fail(SMUON_ERR_INVALID_ARG, "SMUON_NS_FP32_REF, SMUON_NS_SPLIT_BF16 and SMUON_NS_SIMT_BF16 are exclusive");
+  if ((rq.flags & SMUON_NS_EMIT_Q) && !rq.Q_out)
+    return fail(SMUON_ERR_INVALID_ARG, "SMUON_NS_EMIT_Q needs Q_out");
+  for (int i = 0; i < rq.n_mats; ++i) {
+    smuon_status st;
+    const bool has_g = rq.G != nullptr;
+    if ((st = check_mat(rq.M_in[i], "M_in", i, true, !has_g, !has_g)) != SMUON_OK) return st;
+    if ((st = check_mat(rq.U_out[i], "U_out", i, true, true, false)) != SMUON_OK) return st;
+    if (!same_shape(rq.M_in[i], rq.U_out[i])) return fail(SMUON_ERR_SHAPE, "U_out[%d] shape differs from M_in", i);
+    if (has_g) {
+      if ((st = check_mat(rq.G[i], "G", i, true, true, false)) != SMUON_OK) return st;
+      if (!same_shape(rq.M_in[i], rq.G[i])) return fail(SMUON_ERR_SHAPE, "G[%d] shape differs from M_in", i);
+    }
+    if (rq.flags & SMUON_NS_EMIT_Q) {
+      const int m = std::min(rq.M_in[i].rows, rq.M_in[i].cols);
+      if ((st = check_mat(rq.Q_out[i], "Q_out", i, false, true, false)) != SMUON_OK) return st;
+      if (rq.Q_out[i].rows != m || rq.Q_out[i].cols != m)
+        return fail(SMUON_ERR_SHAPE, "Q_out[%d] must be %dx%d", i, m, m);
+    }
+  }
+  return SMUON_OK;
+}
+
+smuon_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(SMUON_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(SMUON_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(SMUON_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", ws_bytes, need);
+  return SMUON_OK;
+}
+
+// enqueue the whole momentum + NS chain for a validated request
+smuon_status enqueue_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t* d_status, const int32_t* skip,
+                        cudaStream_t s) {
+  DevInfo di;
+  smuon_status st = device_info(&di);
+  if (st != SMUON_OK) return st;
+  Builder B;
+  if ((st = build_plan(rq, nullptr, &B)) != SMUON_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, B.L.total)) != SMUON_OK) return st;
+  if ((st = build_plan(rq, reinterpret_cast<char*>(ws), &B)) != SMUON_OK) return st;
+  B.h.status = d_status;
+  if ((st = upload_plan(B, s)) != SMUON_OK) return st;
+  const Plan* d_plan = reinterpret_cast<const Plan*>(ws);
+  const PlanHeader& h = B.h;
+  {
+    const int grid = std::min(h.total_mom_tiles, di.sms * 8);
+    {
+      Launch L("k_momentum", SMUON_WORK_BYTES, momentum_bytes(rq, h), s);
+      k_momentum<<<std::max(grid, 1), 256, 0, s>>>(d_plan, skip);
+      CUDA_TRY(cudaGetLastError());
+    }
+    const int warps_per_block = 8;
+    Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * h.total_mom_tiles, s);
+    k_norm_finalize<<<(h.n_mats + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(d_plan, skip);
+    CUDA_TRY(cudaGetLastError());
+  }
+  const bool emit_q = (rq.flags & SMUON_NS_EMIT_Q) != 0;
+  for (int k = 0; k < rq.iters; ++k) {
+    if ((st = launch_gemm(d_plan, h, ST_GRAM, k, skip, di, s, stage_flops(B, ST_GRAM))) != SMUON_OK) return st;
+    if (rq.c != 0.f && (st = launch_gemm(d_plan, h, ST_POLY, k, skip, di, s, stage_flops(B, ST_POLY))) != SMUON_OK)
+      return st;
+    if ((st = launch_gemm(d_plan, h, ST_AXPY, k, skip, di, s, stage_flops(B, ST_AXPY))) != SMUON_OK) return st;
+    if (emit_q && k >= 1 &&
+        (st = launch_gemm(d_plan, h, ST_QAXPY, k, skip, di, s, stage_flops(B, ST_QAXPY))) != SMUON_OK)
+      return st;
+  }
+  return SMUON_OK;
+}
+
+// ------------------------------------------------------------------ elementwise tables
+struct EwBuild {
+  std::vector<EwLayer> layers;
+  std::vector<std::vector<EwSrc>> srcs;  // per layer
+};
+
+bool vec_ok(const void* p, int64_t ld, int32_t cols, int esz) {
+  return ld == cols && (reinterpret_cast<uintptr_t>(p) % 16 == 0) && esz > 0;
+}
+
+int ew_grid(int64_t chunks, const DevInfo& di) {
+  const int64_t want = (chunks + 255) / 256;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)di.sms * 16));
+}
+
+// splits layers into launches of at most kEwMaxLayers layers / kEwMaxSrcs sources
+template <class F>
+smuon_status for_each_ew_launch(const EwBuild& eb, const EwTable& proto, F&& launch) {
+  static EwTable tb;  // large parameter block, launched by value
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  size_t i = 0;
+  while (i < eb.layers.size()) {
+    tb = proto;
+    tb.n_layers = 0;
+    int nsrc = 0;
+    int64_t chunks = 0;
+    tb.any_packed = 0;
+    while (i < eb.layers.size() && tb.n_layers < kEwMaxLayers &&
+           nsrc + (int)eb.srcs[i].size() <= kEwMaxSrcs) {
+      EwLayer L = eb.layers[i];
+      L.chunk_begin = chunks;
+      L.src_first = nsrc;
+      for (const EwSrc& e : eb.srcs[i]) tb.srcs[nsrc++] = e;
+      chunks += 16 * ((L.n + 127) / 128);
+      if (L.packed_out) tb.any_packed = 1;
+      tb.layers[tb.n_layers++] = L;
+      ++i;
+    }
+    if (tb.n_layers == 0) return fail(SMUON_ERR_UNSUPPORTED, "a layer needs more than %d sources", kEwMaxSrcs);
+    tb.total_chunks = chunks;
+    smuon_status st = launch(tb);
+    if (st != SMUON_OK) return st;
+  }
+  return SMUON_OK;
+}
+
+}  // namespace
+
+// ======================================================================== ABI
+extern "C" {
+
+const char* smuon_last_error(void) { return g_err.c_str(); }
+
+int64_t smuon_launch_count(void) { return g_launches.load(); }
+
+void smuon_trace_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_tr_mu);
+  g_tr_on = on != 0;
+}
+
+int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs) {
+  std::vector<TraceRec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_tr_mu);
+    if (!out) return (int32_t)g_tr.size();
+    recs.swap(g_tr);
+  }
+  int32_t n = 0;
+  for (const TraceRec& r : recs) {
+    float ms = -1.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess) cudaEventElapsedTime(&ms, r.a, r.b);
+    if (out && n < max_recs) {
+      smuon_trace_rec& o = out[n];
+      memset(&o, 0, sizeof(o));
+      strncpy(o.name, r.name, sizeof(o.name) - 1);
+      o.kind = r.kind;
+      o.work = r.work;
+      o.ms = ms;
+    }
+    ++n;
+  }
+  std::lock_guard<std::mutex> lk(g_tr_mu);
+  for (const TraceRec& r : recs) g_ev_free.emplace_back(r.a, r.b);
+  return std::min(n, max_recs);
+}
+int32_t smuon_version(void) { return (1 << 16) | 0; }
+
+smuon_status smuon_ns_workspace_bytes(const smuon_mat* M_in, int32_t n_mats, int32_t iters, uint32_t flags,
+                                      size_t* bytes) {
+  if (!bytes || !M_in) return fail(SMUON_ERR_INVALID_ARG, "NULL argument");
+  if (n_mats < 1 || n_mats > 4096 || iters < 1 || iters > 64) return fail(SMUON_ERR_INVALID_ARG, "bad n_mats/iters");
+  std::vector<smuon_mat> fake(M_in, M_in + n_mats);
+  NsRequest rq{};
+  rq.M_in = fake.data(); rq.U_out = fake.data(); rq.n_mats = n_mats; rq.iters = iters; rq.flags = flags;
+  rq.c = 1.f;  // size for the quintic case (the cubic needs less)
+  std::vector<smuon_mat> q(n_mats);
+  rq.Q_out = (flags & SMUON_NS_EMIT_Q) ? q.data() : nullptr;
+  Builder B;
+  smuon_status st = build_plan(rq, nullptr, &B);
+  if (st != SMUON_OK) return st;
+  *bytes = B.L.total;
+  return SMUON_OK;
+}
+
+smuon_status smuon_ns(const smuon_mat* M_in, const smuon_mat* U_out, int32_t n_mats, const smuon_mat* G,
+                      float beta, float a, float b, float c, int32_t iters, float eps, uint32_t flags,
+                      const smuon_mat* Q_out, const int32_t* d_skip_if, void* ws, size_t ws_bytes,
+                      int32_t* d_status, void* stream) {
+  NsRequest rq{};
+  rq.M_in = M_in; rq.U_out = U_out; rq.n_mats = n_mats; rq.G = G; rq.beta = beta;
+  rq.a = a; rq.b = b; rq.c = c; rq.iters = iters; rq.eps = eps; rq.flags = flags; rq.Q_out = Q_out;
+  smuon_status st = validate_ns(rq);
+  if (st != SMUON_OK) return st;
+  return enqueue_ns(rq, ws, ws_bytes, d_status, d_skip_if, reinterpret_cast<cudaStream_t>(stream));
+}
+
+smuon_status smuon_sign_pack(const smuon_mat* U, int32_t M, uint32_t* packed, int8_t* signs_i8, void* stream) {
+  if (!U) return fail(SMUON_ERR_INVALID_ARG, "U is NULL");
+  if (M < 1 || M > kMaxWorkers) return fail(SMUON_ERR_UNSUPPORTED, "M=%d must be in 1..%d", M, kMaxWorkers);
+  if (!packed && !signs_i8) return fail(SMUON_ERR_INVALID_ARG, "give packed and/or signs_i8");
+  for (int k = 0; k < M; ++k) {
+    smuon_status st = check_mat(U[k], "U", k, true, true, false);
+    if (st != SMUON_OK) return st;
+    if (!same_shape(U[k], U[0]) || U[k].dtype != U[0].dtype)
+      return fail(SMUON_ERR_SHAPE, "U[%d] differs from U[0] in shape or dtype", k);
+  }
+  DevInfo di;
+  smuon_status st = device_info(&di);
+  if (st != SMUON_OK) return st;
+  EwBuild eb;
+  EwLayer L{};
+  L.rows = U[0].rows; L.cols = U[0].cols; L.n = (int64_t)L.rows * L.cols;
+  L.words = 4 * ((L.n + 127) / 128);
+  L.vec = 1;
+  std::vector<EwSrc> srcs;
+  for (int k = 0; k < M; ++k) {
+    srcs.push_back(EwSrc{U[k].data, U[k].ld});
+    if (!vec_ok(U[k].data, U[k].ld, U[k].cols, 1)) L.vec = 0;
+  }
+  eb.layers.push_back(L);
+  eb.srcs.push_back(srcs);
+  EwTable proto{};
+  proto.M = M; proto.src_dtype = U[0].dtype;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
+    const double n = (double)tb.layers[0].n;
+    Launch L("k_sign_pack", SMUON_WORK_BYTES,
+             n * M * dtype_size(U[0].dtype) + (packed ? n * M / 8.0 : 0.0) + (signs_i8 ? n * M : 0.0), s);
+    k_sign_pack<<<ew_grid(tb.total_chunks, di), 256, 0, s>>>(tb, packed, signs_i8);
+    CUDA_TRY(cudaGetLastError());
+    return SMUON_OK;
+  });
+}
+
+smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t M, int64_t N, int8_t tie_value,
+                        int8_t* vote, void* stream) {
+  if ((packed == nullptr) == (signs_i8 == nullptr))
+    return fail(SMUON_ERR_INVALID_ARG, "give exactly one of packed and signs_i8");
+  if (!vote) return fail(SMUON_ERR_INVALID_ARG, "vote is NULL");
+  if (M < 1 || M > kMaxWorkers) return fail(SMUON_ERR_UNSUPPORTED, "M=%d must be in 1..%d", M, kMaxWorkers);
+  if (N < 1) return fail(SMUON_ERR_SHAPE, "N=%lld must be positive", (long long)N);
+  if (tie_value < -1 || tie_value > 1) return fail(SMUON_ERR_INVALID_ARG, "tie_value must be -1, 0 or 1");
+  if (packed && reinterpret_cast<uintptr_t>(packed) % 16) return fail(SMUON_ERR_INVALID_ARG, "packed must be 16-byte aligned");
+  DevInfo di;
+  smuon_status st = device_info(&di);
+  if (st != SMUON_OK) return st;
+  const int64_t nw = (N + 31) / 32;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((nw + 255) / 256, (int64_t)di.sms * 16));
+  Launch L("k_vote", SMUON_WORK_BYTES, (double)N * (packed ? M / 8.0 : (double)M) + (double)N,
+           reinterpret_cast<cudaStream_t>(stream));
+  k_vote<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(packed, signs_i8, M, N, 4 * ((N + 127) / 128),
+                                                                    tie_value, vote);
+  CUDA_TRY(cudaGetLastError());
+  return SMUON_OK;
+}
+
+smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
+                          const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
+                          uint32_t* const* packed_out, int8_t* const* vote_out, void* stream) {
+  if (!W || n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "W is NULL or n_layers < 1");
+  const int nsrc = (U != nullptr) + (votes != nullptr) + (dense != nullptr);
+  if (nsrc != 1) return fail(SMUON_ERR_INVALID_ARG, "exactly one of U, votes, dense must be given");
+  if (U && (M < 1 || M > kMaxWorkers)) return fail(SMUON_ERR_UNSUPPORTED, "M=%d must be in 1..%d", M, kMaxWorkers);
+  if (tie_value < -1 || tie_value > 1) return fail(SMUON_ERR_INVALID_ARG, "tie_value must be -1, 0 or 1");
+  if (vote_kind > SMUON_VOTE_INT8) return fail(SMUON_ERR_INVALID_ARG, "unknown vote_kind %u", vote_kind);
+  if (!U && (packed_out || vote_out)) return fail(SMUON_ERR_INVALID_ARG, "packed_out/vote_out need the U source");
+  int32_t src_dtype = -1;
+  EwBuild eb;
+  for (int l = 0; l < n_layers; ++l) {
+    smuon_status st = check_mat(W[l], "W", l, true, true, false);
+    if (st != SMUON_OK) return st;
+    EwLayer L{};
+    L.w = W[l].data; L.w_ld = W[l].ld; L.w_dtype = W[l].dtype;
+    L.rows = W[l].rows; L.cols = W[l].cols; L.n = (int64_t)L.rows * L.cols;
+    L.words = 4 * ((L.n + 127) / 128);
+    L.vec = vec_ok(W[l].data, W[l].ld, W[l].cols, 1);
+    std::vector<EwSrc> srcs;
+    if (U) {
+      for (int k = 0; k < M; ++k) {
+        const smuon_mat& u = U[(int64_t)l * M + k];
+        if ((st = check_mat(u, "U", l * M + k, true, true, false)) != SMUON_OK) return st;
+        if (!same_shape(u, W[l])) return fail(SMUON_ERR_SHAPE, "U[%d] shape differs from W[%d]", l * M + k, l);
+        if (src_dtype >= 0 && u.dtype != src_dtype) return fail(SMUON_ERR_DTYPE, "all U must share one dtype");
+        src_dtype = u.dtype;
+        if (!vec_ok(u.data, u.ld, u.cols, 1)) L.vec = 0;
+        srcs.push_back(EwSrc{u.data, u.ld});
+      }
+      if (packed_out && packed_out[l]) {
+        if (reinterpret_cast<uintptr_t>(packed_out[l]) % 16) return fail(SMUON_ERR_INVALID_ARG, "packed_out[%d] must be 16-byte aligned", l);
+        L.packed_out = packed_out[l];
+      }
+      if (vote_out) L.vote_out = vote_out[l];
+    } else {
+      const smuon_mat& d = votes ? votes[l] : dense[l];
+      if ((st = check_mat(d, votes ? "votes" : "dense", l, !votes, !votes, votes != nullptr)) != SMUON_OK) return st;
+      if (!same_shape(d, W[l])) return fail(SMUON_ERR_SHAPE, "source %d shape differs from W", l);
+      if (src_dtype >= 0 && d.dtype != src_dtype) return fail(SMUON_ERR_DTYPE, "all sources must share one dtype");
+      src_dtype = d.dtype;
+      if (!vec_ok(d.data, d.ld, d.cols, 1)) L.vec = 0;
+      srcs.push_back(EwSrc{d.data, d.ld});
+    }
+    eb.layers.push_back(L);
+    eb.srcs.push_back(srcs);
+  }
+  DevInfo di;
+  smuon_status st = device_info(&di);
+  if (st != SMUON_OK) return st;
+  EwTable proto{};
+  proto.M = U ? M : 1;
+  proto.tie = tie_value;
+  proto.src_dtype = src_dtype;
+  proto.eta = eta;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
+    const int grid = ew_grid(tb.total_chunks, di);
+    double bytes = 0;
+    for (int l = 0; l < tb.n_layers; ++l) {
+      const EwLayer& Ly = tb.layers[l];
+      bytes += (double)Ly.n * (tb.M * dtype_size(src_dtype) + 2 * dtype_size(Ly.w_dtype));
+      if (Ly.packed_out) bytes += (double)Ly.n * tb.M / 8.0;
+      if (Ly.vote_out) bytes += (double)Ly.n;
+    }
+    if (U) {
+      Launch L(vote_kind == SMUON_VOTE_POPCOUNT ? "k_vote_update_popcount" : "k_vote_update_int8",
+               SMUON_WORK_BYTES, bytes, s);
+      if (vote_kind == SMUON_VOTE_POPCOUNT) k_vote_update_popcount<<<grid, 256, 0, s>>>(tb);
+      else k_vote_update_int8<<<grid, 256, 0, s>>>(tb);
+    } else {
+      Launch L("k_update_src", SMUON_WORK_BYTES, bytes, s);
+      k_update_src<<<grid, 256, 0, s>>>(tb);
+    }
+    CUDA_TRY(cudaGetLastError());
+    return SMUON_OK;
+  });
+}
+
+smuon_status cachemuon_workspace_bytes(const smuon_mat* M_t, size_t* bytes) {
+  if (!M_t || !bytes) return fail(SMUON_ERR_INVALID_ARG, "NULL argument");
+  NsRequest rq{};
+  rq.M_in = M_t; rq.U_out = M_t; rq.n_mats = 1; rq.iters = 1; rq.probe = true; rq.Q_out = M_t;
+  Builder B;
+  smuon_status st = build_plan(rq, nullptr, &B);
+  if (st != SMUON_OK) return st;
+  *bytes = B.L.total;
+  return SMUON_OK;
+}
+
+smuon_status cachemuon_reuse_probe(const smuon_mat* Q, const smuon_mat* M_t, const smuon_mat* D_hat, float gamma,
+                                   float eps, float* d_err, int32_t* d_accept, cachemuon_counters* d_counters,
+                                   void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (!M_t || !D_hat || !d_err || !d_accept) return fail(SMUON_ERR_INVALID_ARG, "M_t, D_hat, d_err, d_accept must not be NULL");
+  smuon_status st;
+  if ((st = check_mat(*M_t, "M_t", 0, true, false, false)) != SMUON_OK) return st;
+  if ((st = check_mat(*D_hat, "D_hat", 0, true, true, false)) != SMUON_OK) return st;
+  if (!same_shape(*M_t, *D_hat)) return fail(SMUON_ERR_SHAPE, "D_hat shape differs from M_t");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DevInfo di;
+  if ((st = device_info(&di)) != SMUON_OK) return st;
+  if (!Q) {
+    Launch L("k_probe_nocache", SMUON_WORK_BYTES, 8.0, s);
+    k_probe_nocache<<<1, 1, 0, s>>>(d_err, d_accept, d_counters);
+    CUDA_TRY(cudaGetLastError());
+    return SMUON_OK;
+  }
+  const int m = std::min(M_t->rows, M_t->cols);
+  if ((st = check_mat(*Q, "Q", 0, false, true, false)) != SMUON_OK) return st;
+  if (Q->rows != m || Q->cols != m) return fail(SMUON_ERR_SHAPE, "Q must be %dx%d", m, m);
+  if (reinterpret_cast<uintptr_t>(Q->data) % 16 || (Q->ld * 2) % 16)
+    return fail(SMUON_ERR_INVALID_ARG, "Q must be 16-byte aligned with ld a multiple of 8 (TMA operand)");
+  NsRequest rq{};
+  rq.M_in = M_t; rq.U_out = D_hat; rq.n_mats = 1; rq.iters = 1; rq.eps = eps; rq.flags = 0;
+  rq.Q_out = Q; rq.probe = true; rq.gamma = gamma;
+  Builder B;
+  if ((st = build_plan(rq, nullptr, &B)) != SMUON_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, B.L.total)) != SMUON_OK) return st;
+  if ((st = build_plan(rq, reinterpret_cast<char*>(ws), &B)) != SMUON_OK) return st;
+  B.h.status = d_status;
+  B.h.d_err = d_err;
+  B.h.d_accept = d_accept;
+  B.h.counters = d_counters;
+  if ((st = upload_plan(B, s)) != SMUON_OK) return st;
+  const Plan* d_plan = reinterpret_cast<const Plan*>(ws);
+  {
+    Launch L("k_momentum", SMUON_WORK_BYTES, momentum_bytes(rq, B.h), s);
+    k_momentum<<<std::max(1, std::min(B.h.total_mom_tiles, di.sms * 8)), 256, 0, s>>>(d_plan, nullptr);
+    CUDA_TRY(cudaGetLastError());
+  }
+  {
+    Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * B.h.total_mom_tiles, s);
+    k_norm_finalize<<<1, 32, 0, s>>>(d_plan, nullptr);
+    CUDA_TRY(cudaGetLastError());
+  }
+  if ((st = launch_gemm(d_plan, B.h, ST_REUSE, 0, nullptr, di, s, stage_flops(B, ST_REUSE))) != SMUON_OK) return st;
+  if ((st = launch_gemm(d_plan, B.h, ST_PROBE, 0, nullptr, di, s, stage_flops(B, ST_PROBE))) != SMUON_OK) return st;
+  Launch L("k_probe_finalize", SMUON_WORK_BYTES, 16.0 * B.h.total_tiles[ST_PROBE], s);
+  k_probe_finalize<<<1, 32, 0, s>>>(d_plan);
+  CUDA_TRY(cudaGetLastError());
+  return SMUON_OK;
+}
+
+// LionMuon workspace: the mean buffers and directions of a Muon step, then the NS workspace
+static smuon_status lion_layout(const lionmuon_state* st, int32_t iters, uint32_t ns_flags, size_t* mean_off, size_t* dir_off,
+                                size_t* ns_off, size_t* total, std::vector<smuon_mat>* means,
+                                std::vector<smuon_mat>* dirs, char* base) {
+  size_t cur = 0;
+  means->clear();
+  dirs->clear();
+  *mean_off = 0;
+  for (int l = 0; l < st->n_layers; ++l) {
+    const smuon_mat& w = st->W[l];
+    smuon_mat m{};
+    m.rows = w.rows; m.cols = w.cols; m.ld = w.cols; m.dtype = SMUON_F32;
+    m.data = base ? base + cur : nullptr;
+    cur = (size_t)round_up((int64_t)(cur + (size_t)w.rows * w.cols * 4), 256);
+    means->push_back(m);
+  }
+  *dir_off = cur;
+  for (int l = 0; l < st->n_layers; ++l) {
+    const smuon_mat& w = st->W[l];
+    smuon_mat d{};
+    d.rows = w.rows; d.cols = w.cols; d.ld = w.cols; d.dtype = SMUON_F32;
+    d.data = base ? base + cur : nullptr;
+    cur = (size_t)round_up((int64_t)(cur + (size_t)w.rows * w.cols * 4), 256);
+    dirs->push_back(d);
+  }
+  *ns_off = cur;
+  size_t ns_bytes = 0;
+  smuon_status s = smuon_ns_workspace_bytes(means->data(), st->n_layers, iters, ns_flags, &ns_bytes);
+  if (s != SMUON_OK) return s;
+  *total = cur + ns_bytes;
+  return SMUON_OK;
+}
+
+smuon_status lionmuon_workspace_bytes(const lionmuon_state* st, int32_t iters, uint32_t ns_flags, size_t* bytes) {
+  if (!st || !bytes || !st->W || st->n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "bad state");
+  size_t a, b, c, total;
+  std::vector<smuon_mat> means, dirs;
+  smuon_status s = lion_layout(st, iters, ns_flags, &a, &b, &c, &total, &means, &dirs, nullptr);
+  if (s != SMUON_OK) return s;
+  *bytes = total;
+  return SMUON_OK;
+}
+
+smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float beta2, float eta, float a, float b,
+                           float c, int32_t iters, int8_t tie_value, uint32_t ns_flags, const smuon_mat* G, void* ws,
+                           size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (!st || !st->W || !st->mom || !G) return fail(SMUON_ERR_INVALID_ARG, "state, W, mom and G must not be NULL");
+  if (st->n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "n_layers < 1");
+  const int M = st->workers;
+  if (M < 1 || M > kMaxWorkers) return fail(SMUON_ERR_UNSUPPORTED, "workers=%d must be in 1..%d", M, kMaxWorkers);
+  if (P < 0) return fail(SMUON_ERR_INVALID_ARG, "P must be >= 0 (0 = never a Muon step)");
+  if (tie_value < -1 || tie_value > 1) return fail(SMUON_ERR_INVALID_ARG, "tie_value must be -1, 0 or 1");
+  if (iters < 1 || iters > 64) return fail(SMUON_ERR_INVALID_ARG, "iters must be in 1..64");
+  smuon_status s;
+  EwBuild eb;
+  for (int l = 0; l < st->n_layers; ++l) {
+    if ((s = check_mat(st->W[l], "W", l, true, true, false)) != SMUON_OK) return s;
+    EwLayer L{};
+    L.w = st->W[l].data; L.w_ld = st->W[l].ld; L.w_dtype = st->W[l].dtype;
+    L.rows = st->W[l].rows; L.cols = st->W[l].cols; L.n = (int64_t)L.rows * L.cols;
+    L.vec = vec_ok(L.w, L.w_ld, L.cols, 1);
+    std::vector<EwSrc> srcs;
+    for (int k = 0; k < M; ++k) {
+      const smuon_mat& mo = st->mom[(int64_t)l * M + k];
+      const smuon_mat& g = G[(int64_t)l * M + k];
+      if ((s = check_mat(mo, "mom", l * M + k, true, false, false)) != SMUON_OK) return s;
+      if ((s = check_mat(g, "G", l * M + k, true, false, false)) != SMUON_OK) return s;
+      if (!same_shape(mo, st->W[l]) || !same_shape(g, st->W[l]))
+        return fail(SMUON_ERR_SHAPE, "mom/G of layer %d differ from W's shape", l);
+      if (!vec_ok(mo.data, mo.ld, mo.cols, 1) || !vec_ok(g.data, g.ld, g.cols, 1)) L.vec = 0;
+      srcs.push_back(EwSrc{mo.data, mo.ld});
+      srcs.push_back(EwSrc{g.data, g.ld});
+    }
+    eb.layers.push_back(L);
+    eb.srcs.push_back(srcs);
+  }
+  DevInfo di;
+  if ((s = device_info(&di)) != SMUON_OK) return s;
+  cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t t_next = st->t + 1;
+  const bool muon = P > 0 && (t_next % P) == 0;
+  EwTable proto{};
+  proto.M = M; proto.tie = tie_value; proto.src_dtype = SMUON_F32; proto.eta = eta;
+  proto.beta1 = beta1; proto.beta2 = beta2;
+  proto.c1 = 1.f - beta1;  // float32 (1 - beta), as in the reading of the EMA
+  proto.c2 = 1.f - beta2;
+  if (!muon) {
+    s = for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
+      double n = 0;
+      for (int l = 0; l < tb.n_layers; ++l) n += (double)tb.layers[l].n * (12.0 * M + 2 * dtype_size(tb.layers[l].w_dtype));
+      Launch L("k_lion_sign", SMUON_WORK_BYTES, n, strm);
+      k_lion_sign<<<ew_grid(tb.total_chunks, di), 256, 0, strm>>>(tb);
+      CUDA_TRY(cudaGetLastError());
+      return SMUON_OK;
+    });
+    if (s != SMUON_OK) return s;
+    st->t = t_next;
+    return SMUON_OK;
+  }
+  size_t mean_off, dir_off, ns_off, total;
+  std::vector<smuon_mat> means, dirs;
+  if ((s = lion_layout(st, iters, ns_flags, &mean_off, &dir_off, &ns_off, &total, &means, &dirs, nullptr)) != SMUON_OK)
+    return s;
+  if ((s = check_ws(ws, ws_bytes, total)) != SMUON_OK) return s;
+  char* base = reinterpret_cast<char*>(ws);
+  if ((s = lion_layout(st, iters, ns_flags, &mean_off, &dir_off, &ns_off, &total, &means, &dirs, base)) != SMUON_OK)
+    return s;
+  for (int l = 0; l < st->n_layers; ++l) {
+    eb.layers[l].aux = means[l].data;
+    eb.layers[l].vec_aux = (eb.layers[l].vec != 0);
+  }
+  s = for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
+    double n = 0;
+    for (int l = 0; l < tb.n_layers; ++l) n += (double)tb.layers[l].n * (12.0 * M + 4.0);
+    Launch L("k_lion_mean", SMUON_WORK_BYTES, n, strm);
+    k_lion_mean<<<ew_grid(tb.total_chunks, di), 256, 0, strm>>>(tb);
+    CUDA_TRY(cudaGetLastError());
+    return SMUON_OK;
+  });
+  if (s != SMUON_OK) return s;
+  NsRequest rq{};
+  rq.M_in = means.data(); rq.U_out = dirs.data(); rq.n_mats = st->n_layers; rq.iters = iters;
+  rq.a = a; rq.b = b; rq.c = c; rq.eps = 1e-7f; rq.flags = ns_flags;
+  if (ns_flags & SMUON_NS_EMIT_Q) return fail(SMUON_ERR_INVALID_ARG, "ns_flags may not ask for SMUON_NS_EMIT_Q");
+  if ((s = validate_ns(rq)) != SMUON_OK) return s;
+  if ((s = enqueue_ns(rq, base + ns_off, total - ns_off, d_status, nullptr, strm)) != SMUON_OK) return s;
+  s = smuon_update(st->W, st->n_layers, nullptr, nullptr, dirs.data(), 1, eta, 0, 0, nullptr, nullptr, stream);
+  if (s != SMUON_OK) return s;
+  st->t = t_next;
+  return SMUON_OK;
+}
+
+}  // extern "C"

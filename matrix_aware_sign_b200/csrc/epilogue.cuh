@@ -1,0 +1,259 @@
+// epilogue.cuh -- per-stage epilogues of the Newton-Schulz GEMM chain.
+//
+// Every GEMM kernel (tcgen05 or CUDA-core) hands its accumulator to
+// epi_chunk() as NV consecutive columns of one output row. The epilogue
+// applies the stage's scalar algebra in float32 and writes the stage's
+// outputs. Workspace buffers have leading dims padded to multiples of 128,
+// so full vector stores along a row are always in bounds there; user
+// buffers are written with bounds checks (and transposed for tall matrices).
+#pragma once
+
+#include "kernels.cuh"
+
+namespace smuon {
+
+struct TileCtx {
+  const GroupDesc* g;
+  const MatDesc* md;
+  int32_t stage, iter, last;  // last: this is the final Newton-Schulz step
+  int32_t z, Mo, No;
+  float s;                    // 1/(||M||_F + eps) of this matrix
+  float a, b, c;
+  uint32_t flags;
+  int32_t bf;                 // operands are bf16 (tcgen05 or SIMT-bf16 mode)
+  int32_t split;              // operands are stored as bf16 hi + lo parts
+  int64_t xlo, mlo;           // element offset of the lo part of an X (m x n) / m x m buffer
+};
+
+template <int NV>
+__device__ __forceinline__ void st_f32_vec(float* p, const float* v) {
+#pragma unroll
+  for (int q = 0; q < NV / 4; ++q)
+    reinterpret_cast<float4*>(p)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+template <int NV>
+__device__ __forceinline__ void st_bf16_vec(__nv_bfloat16* p, const float* v) {
+  if constexpr (NV % 8 == 0) {
+#pragma unroll
+    for (int q = 0; q < NV / 8; ++q) {
+      uint4 w;
+      w.x = pack_bf16x2_rn(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack_bf16x2_rn(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack_bf16x2_rn(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack_bf16x2_rn(v[8 * q + 6], v[8 * q + 7]);
+      reinterpret_cast<uint4*>(p)[q] = w;
+    }
+  } else {
+    static_assert(NV % 4 == 0, "chunk must be a multiple of 4");
+#pragma unroll
+    for (int q = 0; q < NV / 4; ++q) {
+      uint2 w;
+      w.x = pack_bf16x2_rn(v[4 * q + 0], v[4 * q + 1]);
+      w.y = pack_bf16x2_rn(v[4 * q + 2], v[4 * q + 3]);
+      reinterpret_cast<uint2*>(p)[q] = w;
+    }
+  }
+}
+
+template <int NV>
+__device__ __forceinline__ void st_op(void* base, int64_t off, int bf, const float* v) {
+  if (bf) st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
+  else st_f32_vec<NV>(reinterpret_cast<float*>(base) + off, v);
+}
+
+// operand store: f32, bf16, or bf16 hi at off and lo = bf16(v - hi) at off + lo_off
+template <int NV>
+__device__ __forceinline__ void st_operand(const TileCtx& t, void* base, int64_t off, int64_t lo_off,
+                                           const float* v) {
+  if (!t.bf) {
+    st_f32_vec<NV>(reinterpret_cast<float*>(base) + off, v);
+    return;
+  }
+  st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
+  if (t.split) {
+    float lo[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) lo[k] = v[k] - __bfloat162float(__float2bfloat16_rn(v[k]));
+    st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off + lo_off, lo);
+  }
+}
+
+template <int NV>
+__device__ __forceinline__ void ld_f32_vec(const float* p, float* v) {
+#pragma unroll
+  for (int q = 0; q < NV / 4; ++q) {
+    float4 t = reinterpret_cast<const float4*>(p)[q];
+    v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+  }
+}
+
+// user-orientation store of a wide-form row chunk (row i, cols j0..j0+NV-1)
+template <int NV>
+__device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int tall, int row,
+                                        int col0, int nvalid, const float* v) {
+  if (!tall) {
+    int64_t base = (int64_t)row * ld + col0;
+#pragma unroll
+    for (int q = 0; q < NV; ++q)
+      if (q < nvalid) store_from_f32(p, base + q, dtype, v[q]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < NV; ++q)
+      if (q < nvalid) store_from_f32(p, (int64_t)(col0 + q) * ld + row, dtype, v[q]);
+  }
+}
+
+// first cached transform Q_1 = aI + B_0 (CacheMuon fresh solve, reading R14)
+template <int NV>
+__device__ __forceinline__ void emit_q1(const TileCtx& t, int row, int col0, int nvalid, int64_t off,
+                                        const float* B) {
+  float q[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) q[k] = B[k] + ((row == col0 + k) ? t.a : 0.f);
+  if (t.iter == t.last) {  // K == 1: Q_1 is the final transform
+    st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, row, col0, nvalid, q);
+  } else {
+    if (t.bf) st_f32_vec<NV>(t.g->qf[1] + off, q);
+    st_operand<NV>(t, t.g->qop[1], off, t.mlo, q);
+  }
+}
+
+// v[] holds the raw accumulator of D = A_op * B_op at (row, col0..col0+NV-1)
+template <int NV>
+__device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, float* v,
+                                          float* probe_acc) {
+  if (row >= t.Mo || col0 >= t.No) return;
+  const int nvalid = min(NV, t.No - col0);
+  const GroupDesc& g = *t.g;
+  const int m = g.m;
+  switch (t.stage) {
+    case ST_GRAM: {
+      const float sc = (t.iter == 0 && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s * t.s : 1.f;
+      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
+      if (t.c != 0.f) {
+#pragma unroll
+        for (int k = 0; k < NV; ++k) v[k] *= sc;
+        st_f32_vec<NV>(g.af + off, v);
+        if (t.bf) st_operand<NV>(t, g.aop, off, t.mlo, v);
+      } else {
+#pragma unroll
+        for (int k = 0; k < NV; ++k) v[k] = t.b * (sc * v[k]);
+        st_operand<NV>(t, g.bop, off, t.mlo, v);
+        if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, off, v);
+      }
+      break;
+    }
+    case ST_POLY: {
+      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
+      float A[NV];
+      ld_f32_vec<NV>(g.af + off, A);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) v[k] = t.b * A[k] + t.c * v[k];
+      st_operand<NV>(t, g.bop, off, t.mlo, v);
+      if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, off, v);
+      break;
+    }
+    case ST_AXPY: {
+      const bool first = (t.iter == 0);
+      const float sc = (first && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s : 1.f;
+      const int64_t off = ((int64_t)t.z * m + row) * g.ldn + col0;
+      float x[NV];
+      if (first && t.bf) {
+        // X_0 read from the user's momentum in its own dtype and orientation
+        const MatDesc& md = *t.md;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+          float src = 0.f;
+          if (k < nvalid) {
+            const int64_t idx = md.tall ? (int64_t)(col0 + k) * md.m_ld + row
+                                        : (int64_t)row * md.m_ld + col0 + k;
+            src = load_as_f32(md.m_ptr, idx, md.m_dtype);
+          }
+          x[k] = src;
+        }
+      } else {
+        const float* src = t.bf ? g.xf[t.iter & 1] : reinterpret_cast<const float*>(g.xop[t.iter & 1]);
+        ld_f32_vec<NV>(src + off, x);
+      }
+#pragma unroll
+      for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sc * v[k];
+      if (t.iter != t.last) {
+        const int nb = (t.iter + 1) & 1;
+        if (t.bf) st_f32_vec<NV>(g.xf[nb] + off, x);
+        st_operand<NV>(t, g.xop[nb], off, t.xlo, x);
+      } else {
+        st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, row, col0, nvalid, x);
+      }
+      break;
+    }
+    case ST_QAXPY: {
+      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
+      float q[NV];
+      const float* src = t.bf ? g.qf[t.iter & 1] : reinterpret_cast<const float*>(g.qop[t.iter & 1]);
+      ld_f32_vec<NV>(src + off, q);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) q[k] = t.a * q[k] + v[k];
+      if (t.iter != t.last) {
+        const int nb = (t.iter + 1) & 1;
+        if (t.bf) st_f32_vec<NV>(g.qf[nb] + off, q);
+        st_operand<NV>(t, g.qop[nb], off, t.mlo, q);
+      } else {
+        st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, row, col0, nvalid, q);
+      }
+      break;
+    }
+    case ST_REUSE: {
+      const int64_t off = ((int64_t)t.z * m + row) * g.ldn + col0;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) v[k] *= t.s;
+      st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, row, col0, nvalid, v);
+      st_op<NV>(g.xop[1], off, t.bf, v);
+      break;
+    }
+    case ST_PROBE: {
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        if (k < nvalid) {
+          const float r = v[k] - ((row == col0 + k) ? 1.f : 0.f);
+          acc = fmaf(r, r, acc);
+        }
+      }
+      *probe_acc += acc;
+      break;
+    }
+    default: break;
+  }
+}
+
+// per-tile context from a linear tile index of stage st
+__device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int iter, int tile,
+                                            int& tm, int& tn) {
+  TileCtx t;
+  const int gi = find_group(h, st, tile);
+  const GroupDesc& g = h.groups[gi];
+  const int local = tile - g.tile_begin[st];
+  const int per = g.tiles_m[st] * g.tiles_n[st];
+  t.z = local / per;
+  const int rem = local - t.z * per;
+  tm = rem / g.tiles_n[st];
+  tn = rem - tm * g.tiles_n[st];
+  t.g = &h.groups[gi];
+  t.md = &h.mats[g.first_mat + t.z];
+  t.stage = st;
+  t.iter = iter;
+  t.last = h.iters - 1;
+  t.Mo = g.m;
+  t.No = (st == ST_AXPY || st == ST_REUSE) ? g.n : g.m;
+  t.s = h.scale[g.first_mat + t.z];
+  t.a = h.a; t.b = h.b; t.c = h.c;
+  t.flags = h.flags;
+  t.bf = (h.mode != MODE_SIMT_F32);
+  t.split = (h.flags & SMUON_NS_SPLIT_BF16) ? 1 : 0;
+  t.xlo = (int64_t)g.count * g.m * g.ldn;
+  t.mlo = (int64_t)g.count * g.m * g.ldm;
+  return t;
+}
+
+}  // namespace smuon

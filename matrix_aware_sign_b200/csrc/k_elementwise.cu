@@ -1,0 +1,497 @@
+// k_elementwise.cu -- bandwidth-bound kernels of the optimizer step.
+//
+//  * k_plan_upload     copies a Plan (carried in kernel parameters) into the workspace
+//  * k_momentum        M <- beta*M + G, per-tile sum of squares, X0 in wide form
+//  * k_norm_finalize   s = 1/(||M||_F + eps) per matrix (deterministic order)
+//  * k_vote_update     fused sign / pack / popcount (or int8) vote / W update
+//  * k_sign_pack       signs and 1-bit packing only
+//  * k_vote            vote from packed bits or int8 signs
+//  * k_update_src      W update from a vote matrix or a dense direction
+//  * k_lion_sign       LionMuon sign step (G_hat, vote, W and EMA update)
+//  * k_lion_mean       LionMuon Muon-step prologue (mean of G_hat, EMA update)
+//  * k_probe_finalize  CacheMuon residual, accept flag and counters
+#include "kernels.cuh"
+
+namespace smuon {
+
+// --------------------------------------------------------------------------
+__global__ void k_plan_upload(const __grid_constant__ UploadChunk c) {
+  const int n16 = c.bytes / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(c.data);
+  uint4* dst = reinterpret_cast<uint4*>(c.dst);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
+// X0 operand element: f32, bf16, or bf16 hi + lo (lo part count*m*ldn elements later)
+__device__ __forceinline__ void put_x0(const GroupDesc& g, int bf, int split, int64_t o, float v) {
+  if (!bf) {
+    reinterpret_cast<float*>(g.xop[0])[o] = v;
+    return;
+  }
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  reinterpret_cast<__nv_bfloat16*>(g.xop[0])[o] = hi;
+  if (split)
+    reinterpret_cast<__nv_bfloat16*>(g.xop[0])[o + (int64_t)g.count * g.m * g.ldn] =
+        __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+// --------------------------------------------------------------------------
+// SignMuon summary, algorithm flow step 1: momentum update (reading R1) fused
+// with the sum of squares for the Frobenius norm and the bf16/f32 operand
+// copy of X0 in the wide orientation (tall matrices transposed through smem).
+__global__ void __launch_bounds__(256) k_momentum(const Plan* plan, const int32_t* skip) {
+  if (skip && *skip) return;
+  const PlanHeader& h = plan->h;
+  __shared__ float tile[64][65];
+  __shared__ float red[8];
+  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+  for (int t = blockIdx.x; t < h.total_mom_tiles; t += gridDim.x) {
+    const int mi = find_mat_by_mom_tile(h, t);
+    const MatDesc& md = h.mats[mi];
+    const GroupDesc& g = h.groups[md.group];
+    const int local = t - md.mom_begin;
+    const int tr = local / md.mom_tiles_c, tc = local - (local / md.mom_tiles_c) * md.mom_tiles_c;
+    const int r0 = tr * 64, c0 = tc * 64;
+    float ss = 0.f;
+    for (int rr = ty; rr < 64; rr += 4) {
+      const int r = r0 + rr, c = c0 + tx;
+      float val = 0.f;
+      if (r < md.rows && c < md.cols) {
+        const int64_t idx = (int64_t)r * md.m_ld + c;
+        float mv = load_as_f32(md.m_ptr, idx, md.m_dtype);
+        if (md.g_ptr) {
+          const float gv = load_as_f32(md.g_ptr, (int64_t)r * md.g_ld + c, md.g_dtype);
+          mv = fmaf(h.beta, mv, gv);
+          reinterpret_cast<float*>(md.m_ptr)[idx] = mv;
+        }
+        val = mv;
+      }
+      ss = fmaf(val, val, ss);
+      tile[rr][tx] = val;
+    }
+    __syncthreads();
+    const int bf = (h.mode != MODE_SIMT_F32);
+    const int split = (h.flags & SMUON_NS_SPLIT_BF16) != 0;
+    const int m = g.m;
+    if (!md.tall) {
+      for (int rr = ty; rr < 64; rr += 4) {
+        const int r = r0 + rr, c = c0 + tx;
+        if (r < md.rows && c < md.cols) {
+          const int64_t o = ((int64_t)md.z * m + r) * g.ldn + c;
+          put_x0(g, bf, split, o, tile[rr][tx]);
+        }
+      }
+    } else {
+      // X0[c][r] = M[r][c]: wide row index = user column
+      for (int cc = ty; cc < 64; cc += 4) {
+        const int c = c0 + cc, r = r0 + tx;
+        if (r < md.rows && c < md.cols) {
+          const int64_t o = ((int64_t)md.z * m + c) * g.ldn + r;
+          put_x0(g, bf, split, o, tile[tx][cc]);
+        }
+      }
+    }
+    // deterministic block reduction of the tile's sum of squares
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) tot += red[w];
+      h.partials[t] = tot;
+    }
+    __syncthreads();
+  }
+}
+
+// s = 1 / (||M||_F + eps) (reading R4); one warp per matrix, fixed order.
+__global__ void k_norm_finalize(const Plan* plan, const int32_t* skip) {
+  if (skip && *skip) return;
+  const PlanHeader& h = plan->h;
+  const int mi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (mi >= h.n_mats) return;
+  const MatDesc& md = h.mats[mi];
+  float acc = 0.f;
+  for (int i = lane; i < md.mom_count; i += 32) acc += h.partials[md.mom_begin + i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    float s = 1.f;
+    if (!(h.flags & SMUON_NS_NO_NORMALIZE)) s = 1.f / (sqrtf(acc) + h.eps);
+    if (!isfinite(acc) && h.status) atomicOr(h.status, SMUON_DEV_NONFINITE_NORM);
+    h.scale[mi] = s;
+  }
+}
+
+// --------------------------------------------------------------------------
+// Sign / pack / vote / update. Work unit: a chunk of 8 consecutive entries of
+// one layer's row-major flattening; each layer's chunk range is padded to a
+// multiple of 16 chunks (128 entries = 4 packed words), so the four lanes that
+// build one packed word always belong to the same layer.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ int find_layer(const EwTable* tb, int64_t chunk) {
+  int lo = 0, hi = tb->n_layers - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tb->layers[mid].chunk_begin <= chunk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int64_t ew_index(const EwLayer& L, int64_t e, int64_t ld) {
+  // flat row-major entry -> element offset with a leading dimension
+  if (ld == L.cols) return e;
+  const int64_t r = e / L.cols;
+  return r * ld + (e - r * L.cols);
+}
+
+// load 8 entries starting at flat entry e0 as float (missing entries -> +0)
+__device__ __forceinline__ void load8(const void* p, int64_t ld, int32_t dtype, const EwLayer& L,
+                                      int64_t e0, int vec, float* out) {
+  if (vec && e0 + 8 <= L.n) {
+    if (dtype == SMUON_BF16) {
+      const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + e0);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        out[2 * k] = __uint_as_float(u[k] << 16);
+        out[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+      }
+    } else if (dtype == SMUON_F32) {
+      const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + e0);
+      const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + e0 + 4);
+      out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+      out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+    } else {
+      const uint2 w = *reinterpret_cast<const uint2*>(reinterpret_cast<const int8_t*>(p) + e0);
+      const int8_t* q = reinterpret_cast<const int8_t*>(&w);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) out[k] = (float)q[k];
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int64_t e = e0 + k;
+      out[k] = (e < L.n) ? load_as_f32(p, ew_index(L, e, ld), dtype) : 0.f;
+    }
+  }
+}
+
+__device__ __forceinline__ void store8(void* p, int64_t ld, int32_t dtype, const EwLayer& L,
+                                       int64_t e0, int vec, const float* v) {
+  if (vec && e0 + 8 <= L.n) {
+    if (dtype == SMUON_BF16) {
+      uint4 w;
+      w.x = pack_bf16x2_rn(v[0], v[1]); w.y = pack_bf16x2_rn(v[2], v[3]);
+      w.z = pack_bf16x2_rn(v[4], v[5]); w.w = pack_bf16x2_rn(v[6], v[7]);
+      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p) + e0) = w;
+    } else {
+      float* q = reinterpret_cast<float*>(p) + e0;
+      *reinterpret_cast<float4*>(q) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(q + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int64_t e = e0 + k;
+      if (e < L.n) store_from_f32(p, ew_index(L, e, ld), dtype, v[k]);
+    }
+  }
+}
+
+// combine the 8-bit sign bytes of lanes 4w..4w+3 into packed word w (reading R8)
+__device__ __forceinline__ uint32_t gather_word(uint32_t byte, int lane) {
+  uint32_t v = byte << (8 * (lane & 3));
+  v |= __shfl_xor_sync(0xffffffffu, v, 1);
+  v |= __shfl_xor_sync(0xffffffffu, v, 2);
+  return v;
+}
+
+__device__ __forceinline__ int8_t threshold(int total, int tie) {
+  return (int8_t)(total > 0 ? 1 : (total < 0 ? -1 : tie));
+}
+
+// SignMuon summary, flow steps 2-4 fused: sign (U >= 0), optional packed
+// message, majority vote (sum = 2*popcount - M, or integer sum of +-1), then
+// W <- W - eta*vote in float32, rounded to W's type.
+template <bool kPopcount>
+__device__ __forceinline__ void vote_update_body(const EwTable& tb) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t wbase = warp_global * 32; wbase < tb.total_chunks; wbase += warps_total * 32) {
+    const int64_t chunk = wbase + lane;
+    const bool active = chunk < tb.total_chunks;
+    const int li = find_layer(&tb, active ? chunk : tb.total_chunks - 1);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    const bool live = active && e0 < L.n;
+    uint64_t mask[8];
+    int sum[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { mask[k] = 0; sum[k] = 0; }
+    const int M = tb.M;
+    for (int wk = 0; wk < M; ++wk) {
+      const EwSrc& S = tb.srcs[L.src_first + wk];
+      float u[8];
+      if (live) load8(S.ptr, S.ld, tb.src_dtype, L, e0, L.vec, u);
+      uint32_t byte = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const bool pos = live && (e0 + k < L.n) && (u[k] >= 0.f);  // NaN -> negative
+        byte |= (uint32_t)pos << k;
+        if (kPopcount) mask[k] |= (uint64_t)pos << wk;
+        else sum[k] += pos ? 1 : -1;
+      }
+      if (tb.any_packed) {  // warp-uniform: every lane takes part in the shuffles
+        const uint32_t word = gather_word(byte, lane);
+        if (active && L.packed_out && (lane & 3) == 0)
+          L.packed_out[(int64_t)wk * L.words + ((chunk - L.chunk_begin) >> 2)] = word;
+      }
+    }
+    if (!live) continue;
+    int8_t v8[8];
+    float w[8];
+    load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int total = kPopcount ? 2 * __popcll(mask[k]) - M : sum[k];
+      v8[k] = threshold(total, tb.tie);
+      w[k] = __fsub_rn(w[k], tb.eta * (float)v8[k]);
+    }
+    store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+    if (L.vote_out) {
+      if (e0 + 8 <= L.n) {
+        uint2 pk;
+        memcpy(&pk, v8, 8);
+        if ((reinterpret_cast<uintptr_t>(L.vote_out + e0) & 7) == 0)
+          *reinterpret_cast<uint2*>(L.vote_out + e0) = pk;
+        else
+          for (int k = 0; k < 8; ++k) L.vote_out[e0 + k] = v8[k];
+      } else {
+        for (int k = 0; k < 8; ++k) if (e0 + k < L.n) L.vote_out[e0 + k] = v8[k];
+      }
+    }
+  }
+}
+__global__ void __launch_bounds__(256) k_vote_update_popcount(const __grid_constant__ EwTable tb) {
+  vote_update_body<true>(tb);
+}
+__global__ void __launch_bounds__(256) k_vote_update_int8(const __grid_constant__ EwTable tb) {
+  vote_update_body<false>(tb);
+}
+
+// SignMuon summary, flow steps 2-3: signs and the 1-bit message only.
+__global__ void __launch_bounds__(256) k_sign_pack(const __grid_constant__ EwTable tb,
+                                                   uint32_t* packed, int8_t* signs) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const EwLayer& L = tb.layers[0];
+  for (int64_t wbase = warp_global * 32; wbase < tb.total_chunks; wbase += warps_total * 32) {
+    const int64_t chunk = wbase + lane;
+    const bool active = chunk < tb.total_chunks;
+    const int64_t e0 = chunk * 8;
+    const bool live = active && e0 < L.n;
+    for (int wk = 0; wk < tb.M; ++wk) {
+      const EwSrc& S = tb.srcs[wk];
+      float u[8];
+      if (live) load8(S.ptr, S.ld, tb.src_dtype, L, e0, L.vec, u);
+      uint32_t byte = 0;
+      int8_t sg[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const bool pos = live && (e0 + k < L.n) && (u[k] >= 0.f);
+        byte |= (uint32_t)pos << k;
+        sg[k] = pos ? 1 : -1;
+      }
+      if (packed) {
+        const uint32_t word = gather_word(byte, lane);
+        if (active && (lane & 3) == 0) packed[(int64_t)wk * L.words + (chunk >> 2)] = word;
+      }
+      if (signs && live) {
+        int8_t* dst = signs + (int64_t)wk * L.n + e0;
+        if (e0 + 8 <= L.n && ((reinterpret_cast<uintptr_t>(dst) & 7) == 0)) {
+          uint2 pk;
+          memcpy(&pk, sg, 8);
+          *reinterpret_cast<uint2*>(dst) = pk;
+        } else {
+          for (int k = 0; k < 8; ++k) if (e0 + k < L.n) dst[k] = sg[k];
+        }
+      }
+    }
+  }
+}
+
+// SignMuon summary, flow steps 3-4: vote from the all-gathered bits (sum =
+// 2*popcount - M) or from the all-reduced int8 signs. One thread per 32
+// entries (one packed word per worker).
+__global__ void __launch_bounds__(256) k_vote(const uint32_t* packed, const int8_t* signs, int M,
+                                              int64_t N, int64_t words, int tie, int8_t* vote) {
+  const int64_t nw = (N + 31) / 32;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nw;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e0 = w * 32;
+    const int nvalid = (N - e0) < 32 ? (int)(N - e0) : 32;
+    int8_t out[32];
+    if (packed) {
+      uint32_t bits[kMaxWorkers];
+      for (int k = 0; k < M; ++k) bits[k] = packed[(int64_t)k * words + w];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        uint64_t mask = 0;
+        for (int k = 0; k < M; ++k) mask |= (uint64_t)((bits[k] >> j) & 1u) << k;
+        out[j] = threshold(2 * __popcll(mask) - M, tie);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) out[j] = 0;
+      for (int k = 0; k < M; ++k) {
+        const int8_t* src = signs + (int64_t)k * N + e0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) if (j < nvalid) out[j] += src[j];
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) out[j] = threshold(out[j], tie);
+    }
+    if (nvalid == 32 && ((reinterpret_cast<uintptr_t>(vote + e0) & 15) == 0)) {
+      uint4 a, b;
+      memcpy(&a, out, 16);
+      memcpy(&b, out + 16, 16);
+      reinterpret_cast<uint4*>(vote + e0)[0] = a;
+      reinterpret_cast<uint4*>(vote + e0)[1] = b;
+    } else {
+      for (int j = 0; j < nvalid; ++j) vote[e0 + j] = out[j];
+    }
+  }
+}
+
+// W <- W - eta * v (vote, exact product) or W - f32(eta * D) (dense), reading R9.
+__global__ void __launch_bounds__(256) k_update_src(const __grid_constant__ EwTable tb) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; chunk < tb.total_chunks;
+       chunk += stride) {
+    const int li = find_layer(&tb, chunk);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    if (e0 >= L.n) continue;
+    const EwSrc& S = tb.srcs[L.src_first];
+    float d[8], w[8];
+    load8(S.ptr, S.ld, tb.src_dtype, L, e0, L.vec, d);
+    load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w[k] = __fsub_rn(w[k], __fmul_rn(tb.eta, d[k]));
+    store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+  }
+}
+
+// LionMuon summary, methodology items 1-2, sign step: per worker
+// G_hat = f32(beta1*M) + f32((1-beta1)*G), bit = G_hat >= 0, then
+// EMA M <- f32(beta2*M) + f32((1-beta2)*G); majority vote; W update.
+__global__ void __launch_bounds__(256) k_lion_sign(const __grid_constant__ EwTable tb) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; chunk < tb.total_chunks;
+       chunk += stride) {
+    const int li = find_layer(&tb, chunk);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    if (e0 >= L.n) continue;
+    uint64_t mask[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mask[k] = 0;
+    for (int wk = 0; wk < tb.M; ++wk) {
+      const EwSrc& S = tb.srcs[L.src_first + 2 * wk];      // EMA (f32, in/out)
+      const EwSrc& Gs = tb.srcs[L.src_first + 2 * wk + 1]; // gradient (f32)
+      float mo[8], gr[8];
+      load8(S.ptr, S.ld, SMUON_F32, L, e0, L.vec, mo);
+      load8(Gs.ptr, Gs.ld, SMUON_F32, L, e0, L.vec, gr);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float gh = __fadd_rn(__fmul_rn(tb.beta1, mo[k]), __fmul_rn(tb.c1, gr[k]));
+        mask[k] |= (uint64_t)(gh >= 0.f) << wk;
+        mo[k] = __fadd_rn(__fmul_rn(tb.beta2, mo[k]), __fmul_rn(tb.c2, gr[k]));
+      }
+      store8(const_cast<void*>(S.ptr), S.ld, SMUON_F32, L, e0, L.vec, mo);
+    }
+    float w[8];
+    load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int8_t v = threshold(2 * __popcll(mask[k]) - tb.M, tb.tie);
+      w[k] = __fsub_rn(w[k], tb.eta * (float)v);
+    }
+    store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+  }
+}
+
+// LionMuon Muon step prologue (reading R11): mean over workers of G_hat into a
+// contiguous f32 buffer, and the EMA update of every worker.
+__global__ void __launch_bounds__(256) k_lion_mean(const __grid_constant__ EwTable tb) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const float invM = 1.f / (float)tb.M;
+  for (int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; chunk < tb.total_chunks;
+       chunk += stride) {
+    const int li = find_layer(&tb, chunk);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    if (e0 >= L.n) continue;
+    float acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+    for (int wk = 0; wk < tb.M; ++wk) {
+      const EwSrc& S = tb.srcs[L.src_first + 2 * wk];
+      const EwSrc& Gs = tb.srcs[L.src_first + 2 * wk + 1];
+      float mo[8], gr[8];
+      load8(S.ptr, S.ld, SMUON_F32, L, e0, L.vec, mo);
+      load8(Gs.ptr, Gs.ld, SMUON_F32, L, e0, L.vec, gr);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float gh = __fadd_rn(__fmul_rn(tb.beta1, mo[k]), __fmul_rn(tb.c1, gr[k]));
+        acc[k] = __fadd_rn(acc[k], gh);
+        mo[k] = __fadd_rn(__fmul_rn(tb.beta2, mo[k]), __fmul_rn(tb.c2, gr[k]));
+      }
+      store8(const_cast<void*>(S.ptr), S.ld, SMUON_F32, L, e0, L.vec, mo);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = __fmul_rn(acc[k], invM);
+    // the mean buffer is contiguous (ld == cols) f32 in the workspace
+    store8(L.aux, L.cols, SMUON_F32, L, e0, L.vec_aux, acc);
+  }
+}
+
+// CacheMuon summary, method item 3: err = sqrt(sum of squared residuals)/sqrt(m),
+// accept iff err <= gamma (NaN rejects), counters updated on the device.
+__global__ void k_probe_finalize(const Plan* plan) {
+  const PlanHeader& h = plan->h;
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  const int n = 4 * h.total_tiles[ST_PROBE];  // four partial sums per tile
+  float acc = 0.f;
+  for (int i = lane; i < n; i += 32) acc += h.probe_partials[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    const int m = h.groups[0].m;
+    const float err = sqrtf(acc) / sqrtf((float)m);
+    const int accept = (err <= h.gamma) ? 1 : 0;  // NaN compares false
+    *h.d_err = err;
+    *h.d_accept = accept;
+    if (h.counters) {
+      h.counters->probes += 1;
+      if (accept) h.counters->hits += 1; else h.counters->misses += 1;
+    }
+  }
+}
+
+// First CacheMuon step (no cached transform): reject without a probe.
+__global__ void k_probe_nocache(float* d_err, int32_t* d_accept, cachemuon_counters* counters) {
+  *d_err = __int_as_float(0x7f800000);
+  *d_accept = 0;
+  if (counters) counters->misses += 1;
+}
+
+}  // namespace smuon

@@ -1,0 +1,374 @@
+// k_gemm_tc.cu -- grouped Newton-Schulz GEMM stages on the sm_100a tensor cores.
+//
+// One persistent kernel per stage walks the plan's tile list (all layers x
+// workers in one launch). Per CTA:
+//   warp 0      TMA producer: 128B-swizzled tiles of A (K-major) and B
+//               (K-major, or MN-major for the X / Q right operand) into a
+//               6-deep shared-memory ring (full/empty mbarriers)
+//   warp 1      TMEM allocation and the single MMA-issuing thread:
+//               tcgen05.mma.cta_group::1.kind::f16, BF16 x BF16 -> FP32,
+//               M = N = 128, K = 16 per instruction, into one of two TMEM
+//               accumulators (128 columns each)
+//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns at a time, stage
+//               algebra in FP32 (epilogue.cuh), global stores
+// The two accumulators let the epilogue of tile i overlap the MMAs of tile
+// i+1. Every mbarrier wait is bounded; on expiry the CTA records
+// SMUON_DEV_WAIT_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
+#include "epilogue.cuh"
+
+namespace smuon {
+namespace tc {
+
+constexpr int BM = kTcBM, BN = kTcBN, BK = 64;
+constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x 64 k)
+constexpr int B_BYTES = BN * BK * 2;   // one bf16 tile of B
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int THREADS = 192;
+
+// plain BF16: one hi tile per operand; split BF16: hi and lo tiles per operand
+// (x = x_hi + x_lo, product ~ A_hi B_hi + A_hi B_lo + A_lo B_hi)
+template <bool kSplit>
+struct Cfg {
+  static constexpr int PARTS = kSplit ? 2 : 1;
+  static constexpr int STAGE_BYTES = PARTS * (A_BYTES + B_BYTES);
+  static constexpr int STAGES = kSplit ? 3 : 6;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// bounded wait: false when the budget ran out or another role aborted
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitCycles) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tensormap_acquire(const CUtensorMap* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(map))
+               : "memory");
+}
+
+// shared-memory matrix descriptors (tcgen05 format: version 1, 128B swizzle)
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;  // 8-row group stride
+  d |= (uint64_t)1 << 46;            // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
+  return d;
+}
+
+// instruction descriptor: BF16 x BF16 -> F32, A K-major, B K- or MN-major, 128 x 128
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// operands of one tile: tensor maps, coordinates, K extent
+struct TcOps {
+  const CUtensorMap* ma;
+  const CUtensorMap* mb;
+  int za, zb;
+  int zlo;   // split mode: the lo part of matrix z is matrix z + zlo of the same map
+  int K;
+  int b_mn;
+};
+
+__device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, int iter) {
+  const GroupDesc& g = *t.g;
+  TcOps o;
+  o.za = o.zb = t.z;
+  o.zlo = g.count;
+  switch (t.stage) {
+    case ST_GRAM: o.ma = o.mb = &h.tmaps[g.tm_x_k[iter & 1]]; o.K = g.n; o.b_mn = 0; break;
+    case ST_POLY: o.ma = o.mb = &h.tmaps[g.tm_a_k]; o.K = g.m; o.b_mn = 0; break;
+    case ST_AXPY: o.ma = &h.tmaps[g.tm_b_k]; o.mb = &h.tmaps[g.tm_x_mn[iter & 1]]; o.K = g.m; o.b_mn = 1; break;
+    case ST_QAXPY: o.ma = &h.tmaps[g.tm_b_k]; o.mb = &h.tmaps[g.tm_q_mn[iter & 1]]; o.K = g.m; o.b_mn = 1; break;
+    case ST_REUSE: o.ma = &h.tmaps[g.tm_uq_k]; o.za = 0; o.mb = &h.tmaps[g.tm_x_mn[0]]; o.K = g.m; o.b_mn = 1; break;
+    default: o.ma = o.mb = &h.tmaps[g.tm_x_k[1]]; o.K = g.n; o.b_mn = 0; break;  // ST_PROBE
+  }
+  return o;
+}
+
+template <bool kSplit>
+__device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int iter) {
+  constexpr int STAGES = Cfg<kSplit>::STAGES;
+  constexpr int STAGE_BYTES = Cfg<kSplit>::STAGE_BYTES;
+  constexpr int PARTS = Cfg<kSplit>::PARTS;
+  const PlanHeader& h = plan->h;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* base_ptr = smem_raw + (base - raw);
+  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+  // barrier layout (8 bytes each): full[S], empty[S], tfull[2], tempty[2], done
+  const uint32_t full_bar = bar0, empty_bar = bar0 + 8 * STAGES;
+  const uint32_t tfull_bar = bar0 + 16 * STAGES, tempty_bar = tfull_bar + 16, done_bar = tempty_bar + 16;
+  unsigned char* misc = base_ptr + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar + 8 * s, 1); mbar_init(empty_bar + 8 * s, 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar + 8 * a, 1); mbar_init(tempty_bar + 8 * a, 128); }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32((const void*)tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = h.total_tiles[stage];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t armed = 0, last_par = 0;  // per-stage bit sets for the exit drain
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int tm, tn;
+        const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+        const TcOps o = tc_ops(h, t, iter);
+        tensormap_acquire(o.ma);
+        tensormap_acquire(o.mb);
+        const int nk = (o.K + BK - 1) / BK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty_bar + 8 * s, ph ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t fb = full_bar + 8 * s;
+          mbar_expect_tx(fb, STAGE_BYTES);
+          armed |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          const uint32_t sa = base + s * STAGE_BYTES, sb = sa + PARTS * A_BYTES;
+#pragma unroll
+          for (int part = 0; part < PARTS; ++part) {
+            const int za = o.za + part * o.zlo, zb = o.zb + part * o.zlo;
+            const uint32_t da = sa + part * A_BYTES, db = sb + part * B_BYTES;
+            tma_load_3d(da, o.ma, kb * BK, tm * BM, za, fb);
+            if (o.b_mn) {
+              tma_load_3d(db, o.mb, tn * BN, kb * BK, zb, fb);
+              tma_load_3d(db + B_BYTES / 2, o.mb, tn * BN + 64, kb * BK, zb, fb);
+            } else {
+              tma_load_3d(db, o.mb, kb * BK, tn * BN, zb, fb);
+            }
+          }
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
+      }
+      // drain: every armed stage's last phase must have landed before exit
+      for (int q = 0; q < STAGES; ++q)
+        if (armed & (1u << q)) {
+          const uint32_t p = (last_par >> q) & 1u;
+          const unsigned long long t0 = clock64();
+          while (!mbar_try_wait(full_bar + 8 * q, p) && clock64() - t0 < kWaitCycles) {}
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int tm, tn;
+        const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+        const TcOps o = tc_ops(h, t, iter);
+        const uint32_t idesc = make_idesc((uint32_t)o.b_mn);
+        if (!mbar_wait(tempty_bar + 8 * acc, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
+        fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const int nk = (o.K + BK - 1) / BK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(full_bar + 8 * s, ph, abort_flag)) { ok = false; break; }
+          fence_after();
+          const uint32_t sa = base + s * STAGE_BYTES, sb = sa + PARTS * A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = desc_sw128(sa + kk * 32, 16);
+            const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, B_BYTES / 2) : desc_sw128(sb + kk * 32, 16);
+            mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            if constexpr (kSplit) {
+              const uint64_t adl = desc_sw128(sa + A_BYTES + kk * 32, 16);
+              const uint32_t sbl = sb + B_BYTES;
+              const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, B_BYTES / 2) : desc_sw128(sbl + kk * 32, 16);
+              mma_bf16(d_tmem, ad, bdl, idesc, 1u);   // A_hi * B_lo
+              mma_bf16(d_tmem, adl, bd, idesc, 1u);   // A_lo * B_hi
+            }
+          }
+          mma_commit(empty_bar + 8 * s);  // frees the smem slot once these MMAs have read it
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar + 8 * acc);  // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
+      }
+      // all MMAs issued by this thread complete before TMEM is released
+      mma_commit(done_bar);
+      const unsigned long long t0 = clock64();
+      while (!mbar_try_wait(done_bar, 0) && clock64() - t0 < kWaitCycles) {}
+    }
+  } else {
+    // ---------------- epilogue warps 2..5
+    const int ew = warp & 3;  // TMEM lane group this warp may access
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int tm, tn;
+      TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+      if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag)) {
+        *abort_flag = 1;
+        if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
+        break;
+      }
+      fence_after();
+      const int row = tm * BM + ew * 32 + lane;
+      float pacc = 0.f;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        float v[32];
+        tmem_ld32(tmem_base + (uint32_t)(acc * BN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
+        epi_chunk<32>(t, row, tn * BN + ch * 32, v, &pacc);
+      }
+      fence_before();
+      mbar_arrive(tempty_bar + 8 * acc);
+      if (stage == ST_PROBE) {  // one partial per epilogue warp: no barrier, fixed order later
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) pacc += __shfl_xor_sync(0xffffffffu, pacc, o2);
+        if (lane == 0) h.probe_partials[4 * tile + ew] = pacc;
+      }
+      if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS));
+}
+
+__global__ void __launch_bounds__(THREADS, 1) k_gemm_tc(const Plan* plan, int stage, int iter, const int32_t* skip) {
+  if (skip && *skip) return;
+  gemm_tc_body<false>(plan, stage, iter);
+}
+
+__global__ void __launch_bounds__(THREADS, 1) k_gemm_tc_split(const Plan* plan, int stage, int iter,
+                                                               const int32_t* skip) {
+  if (skip && *skip) return;
+  gemm_tc_body<true>(plan, stage, iter);
+}
+
+}  // namespace tc
+
+cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter, const int32_t* skip,
+                           int num_sms, cudaStream_t s) {
+  static bool attr_set[64][2] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && stage <= ST_QAXPY;
+  if (dev < 64 && !attr_set[dev][split]) {
+    cudaError_t e = split ? cudaFuncSetAttribute(tc::k_gemm_tc_split, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 tc::Cfg<true>::SMEM_BYTES)
+                          : cudaFuncSetAttribute(tc::k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 tc::Cfg<false>::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev][split] = true;
+  }
+  const int total = h.total_tiles[stage];
+  if (total == 0) return cudaSuccess;
+  const int grid = total < num_sms ? total : num_sms;
+  if (split)
+    tc::k_gemm_tc_split<<<grid, tc::THREADS, tc::Cfg<true>::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
+  else
+    tc::k_gemm_tc<<<grid, tc::THREADS, tc::Cfg<false>::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
+  return cudaGetLastError();
+}
+
+}  // namespace smuon

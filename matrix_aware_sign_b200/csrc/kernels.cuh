@@ -1,0 +1,83 @@
+// kernels.cuh -- declarations shared by the host ABI and the kernel files.
+#pragma once
+
+#include "plan.cuh"
+
+namespace smuon {
+
+// ---- plan upload: the plan bytes travel in kernel parameters
+constexpr int kUploadBytes = 16384;
+struct alignas(16) UploadChunk {
+  void* dst;
+  int32_t bytes;  // multiple of 16
+  int32_t pad[1];
+  alignas(16) unsigned char data[kUploadBytes];
+};
+
+// ---- elementwise tables (sign / vote / update / Lion), carried in kernel parameters
+constexpr int kEwMaxLayers = 64;
+constexpr int kEwMaxSrcs = 1024;
+
+struct EwSrc {
+  const void* ptr;
+  int64_t ld;
+};
+
+struct EwLayer {
+  void* w;                 // weights (in/out), or unused
+  int64_t w_ld;
+  int64_t n;               // entries = rows * cols
+  int64_t chunk_begin;     // first 8-entry chunk of this layer in the launch
+  uint32_t* packed_out;    // nullable [M][words]
+  int64_t words;           // packed words per worker
+  int8_t* vote_out;        // nullable [n]
+  void* aux;               // Lion mean output (f32, contiguous)
+  int32_t w_dtype;
+  int32_t vec;             // all operands contiguous and 16-byte aligned
+  int32_t vec_aux;
+  int32_t src_first;       // first entry of this layer in srcs[]
+  int32_t rows, cols;
+};
+
+struct EwTable {
+  int32_t n_layers, M, tie, src_dtype;
+  int32_t any_packed, pad;
+  float eta, beta1, beta2, c1, c2;
+  int64_t total_chunks;
+  EwLayer layers[kEwMaxLayers];
+  EwSrc srcs[kEwMaxSrcs];
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+// ---- kernels
+__global__ void k_plan_upload(const __grid_constant__ UploadChunk c);
+__global__ void k_momentum(const Plan* plan, const int32_t* skip);
+__global__ void k_norm_finalize(const Plan* plan, const int32_t* skip);
+__global__ void k_vote_update_popcount(const __grid_constant__ EwTable tb);
+__global__ void k_vote_update_int8(const __grid_constant__ EwTable tb);
+__global__ void k_sign_pack(const __grid_constant__ EwTable tb, uint32_t* packed, int8_t* signs);
+__global__ void k_vote(const uint32_t* packed, const int8_t* signs, int M, int64_t N, int64_t words,
+                       int tie, int8_t* vote);
+__global__ void k_update_src(const __grid_constant__ EwTable tb);
+__global__ void k_lion_sign(const __grid_constant__ EwTable tb);
+__global__ void k_lion_mean(const __grid_constant__ EwTable tb);
+__global__ void k_probe_finalize(const Plan* plan);
+__global__ void k_probe_nocache(float* d_err, int32_t* d_accept, cachemuon_counters* counters);
+
+// GEMM stage kernels (grouped, persistent)
+__global__ void k_gemm_simt_f32(const Plan* plan, int stage, int iter, const int32_t* skip);
+__global__ void k_gemm_simt_bf16(const Plan* plan, int stage, int iter, const int32_t* skip);
+
+// tcgen05 kernel entry (host-side launcher lives in k_gemm_tc.cu)
+cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter,
+                           const int32_t* skip, int num_sms, cudaStream_t s);
+constexpr int kTcBM = 128;
+constexpr int kTcBN = 128;
+constexpr int kSimtBM = 64;
+constexpr int kSimtBN = 64;
+
+}  // namespace smuon

@@ -1,0 +1,132 @@
+// plan.cuh -- device-resident description of one batched Newton-Schulz call.
+//
+// The host builds a Plan (groups of same-shape matrices, per-matrix user
+// pointers, workspace buffers, TMA tensor maps and per-stage tile tables),
+// uploads it into the head of the caller's workspace with a kernel whose
+// parameters carry the bytes (no host->device memcpy, so a call can be
+// captured in a CUDA graph), and every kernel of the call reads it from there.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "smuon.h"
+
+namespace smuon {
+
+constexpr int kMaxWorkers = 64;
+
+// Stages of the Newton-Schulz chain. Each is one grouped GEMM launch
+// D = A_op * B_op over every matrix of the batch, with its own epilogue.
+enum Stage : int32_t {
+  ST_GRAM = 0,   // A = s^2 X X^T                      (m x m, K = n)
+  ST_POLY = 1,   // B = b A + c A^2                      (m x m, K = m)
+  ST_AXPY = 2,   // X' = a s X + s B X                   (m x n, K = m)
+  ST_QAXPY = 3,  // Q' = a Q + B Q                       (m x m, K = m)
+  ST_REUSE = 4,  // D_hat = s Q X_t                      (m x n, K = m)
+  ST_PROBE = 5,  // sum (D_hat D_hat^T - I)^2 per tile   (m x m, K = n)
+  ST_COUNT = 6
+};
+
+enum Mode : int32_t { MODE_TC_BF16 = 0, MODE_SIMT_F32 = 1, MODE_SIMT_BF16 = 2 };
+
+// one user matrix (user orientation rows x cols); NS runs on the wide form
+// m x n with m = min(rows, cols): a tall matrix is read transposed.
+struct MatDesc {
+  void* m_ptr;      // momentum / input matrix
+  int64_t m_ld;
+  const void* g_ptr;  // gradient, nullable
+  int64_t g_ld;
+  void* u_ptr;      // polar-factor output (or D_hat for the probe)
+  int64_t u_ld;
+  void* q_ptr;      // bf16 m x m cached transform (EMIT_Q output, or REUSE input)
+  int64_t q_ld;
+  int32_t m_dtype, g_dtype, u_dtype, pad0;
+  int32_t rows, cols, tall, group;
+  int32_t z;              // index of this matrix inside its group
+  int32_t mom_begin;      // first momentum tile (= partial-sum slot)
+  int32_t mom_tiles_c;    // 64x64 tiles along cols (user orientation)
+  int32_t mom_count;      // number of momentum tiles
+};
+
+// matrices of one wide shape m x n, stored contiguously in the workspace
+struct GroupDesc {
+  int32_t m, n, count, first_mat;
+  int64_t ldn, ldm;       // padded leading dims (elements), multiples of 128
+  void* xop[2];           // X operand [count][m][ldn] (bf16, or f32 in FP32 mode)
+  float* xf[2];           // f32 master of X for iterations >= 1 (bf16 modes)
+  float* af;              // f32 A [count][m][ldm]
+  void* aop;              // A operand (bf16 modes; == af in FP32 mode)
+  void* bop;              // B operand [count][m][ldm]
+  float* qf[2];           // f32 master of Q (EMIT_Q)
+  void* qop[2];           // Q operand
+  int32_t tm_x_k[2];      // tensor-map indices: X K-major box {64,128}
+  int32_t tm_x_mn[2];     // X MN-major box {64,64}
+  int32_t tm_a_k, tm_b_k; // A / B K-major box {64,128}
+  int32_t tm_q_mn[2];     // Q MN-major box {64,64}
+  int32_t tm_uq_k;        // user Q K-major (REUSE A operand)
+  int32_t pad1;
+  int32_t tiles_m[ST_COUNT], tiles_n[ST_COUNT], tile_begin[ST_COUNT];
+};
+
+struct PlanHeader {
+  int32_t n_mats, n_groups, n_tmaps, mode;
+  int32_t iters;
+  uint32_t flags;
+  float a, b, c, eps;
+  float beta;
+  float gamma;              // probe threshold
+  int32_t total_mom_tiles;
+  int32_t tile_bm, tile_bn; // tile shape of the GEMM kernel the tables are built for
+  int32_t total_tiles[ST_COUNT];
+  float* partials;          // [total_mom_tiles] sum of squares per momentum tile
+  float* scale;             // [n_mats] s = 1/(||M||_F + eps)
+  float* probe_partials;    // [total PROBE tiles]
+  GroupDesc* groups;        // device pointers into the plan region
+  MatDesc* mats;
+  CUtensorMap* tmaps;
+  int32_t* status;          // nullable
+  float* d_err;             // probe outputs
+  int32_t* d_accept;
+  cachemuon_counters* counters;
+};
+
+struct Plan {
+  PlanHeader h;
+};
+
+// ---------------------------------------------------------------- helpers
+__host__ __device__ inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+__host__ __device__ inline int32_t ceil_div(int64_t x, int64_t m) { return (int32_t)((x + m - 1) / m); }
+
+__device__ inline float load_as_f32(const void* p, int64_t idx, int32_t dtype) {
+  if (dtype == SMUON_F32) return reinterpret_cast<const float*>(p)[idx];
+  if (dtype == SMUON_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[idx]);
+  return (float)reinterpret_cast<const int8_t*>(p)[idx];
+}
+
+__device__ inline void store_from_f32(void* p, int64_t idx, int32_t dtype, float v) {
+  if (dtype == SMUON_F32) reinterpret_cast<float*>(p)[idx] = v;
+  else reinterpret_cast<__nv_bfloat16*>(p)[idx] = __float2bfloat16_rn(v);
+}
+
+// locate the group of a linear tile index of stage st (groups are few: linear scan)
+__device__ inline int find_group(const PlanHeader& h, int st, int tile) {
+  int g = 0;
+  while (g + 1 < h.n_groups && h.groups[g + 1].tile_begin[st] <= tile) ++g;
+  return g;
+}
+
+// locate the matrix owning a momentum tile (binary search over mats)
+__device__ inline int find_mat_by_mom_tile(const PlanHeader& h, int tile) {
+  int lo = 0, hi = h.n_mats - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (h.mats[mid].mom_begin <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+}  // namespace smuon

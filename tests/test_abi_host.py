@@ -1,0 +1,90 @@
+"""Host-side checks of the C-ABI library (no GPU): it loads, exports every
+function that include/smuon.h declares, and rejects bad arguments before it
+would touch a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "smuon.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\**([a-z_][a-z0-9_]*)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import matrix_aware_sign_b200 as S
+    return S.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for want in ["smuon_ns", "smuon_sign_pack", "smuon_vote", "smuon_update", "cachemuon_reuse_probe",
+                 "lionmuon_step", "smuon_ns_workspace_bytes", "cachemuon_workspace_bytes",
+                 "lionmuon_workspace_bytes", "smuon_last_error", "smuon_version"]:
+        assert want in names, want
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), f"libsmuon.so does not export {name}"
+
+
+def test_version(L):
+    assert L.smuon_version() >> 16 == 1
+
+
+def test_vote_rejects_bad_arguments_before_launch(L):
+    import matrix_aware_sign_b200 as S
+    # neither source given
+    assert L.smuon_vote(None, None, 3, 10, 0, 1234, None) == -1
+    assert b"exactly one" in L.smuon_last_error()
+    # too many workers
+    assert L.smuon_vote(64, None, 65, 10, 0, 1234, None) == -4
+    # bad tie value
+    assert L.smuon_vote(64, None, 3, 10, 2, 1234, None) == -1
+
+
+def test_ns_rejects_bad_arguments_before_launch(L):
+    import matrix_aware_sign_b200 as S
+    m = S.SmuonMat(4096, 8, 8, 8, S.F32)
+    arr = (S.SmuonMat * 1)(m)
+    bad = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 8, 4, S.F32))  # ld < cols
+    assert L.smuon_ns(arr, arr, 0, None, 0.9, 1.5, -0.5, 0.0, 5, 1e-7, 0, None, None, None, 0, None, None) == -1
+    assert L.smuon_ns(arr, arr, 1, None, 0.9, 1.5, -0.5, 0.0, 0, 1e-7, 0, None, None, None, 0, None, None) == -1
+    assert L.smuon_ns(bad, arr, 1, None, 0.9, 1.5, -0.5, 0.0, 5, 1e-7, 0, None, None, None, 0, None, None) == -2
+    assert L.smuon_ns(arr, arr, 1, None, 0.9, 1.5, -0.5, 0.0, 5, 1e-7, 0x100, None, None, None, 0, None, None) == -1
+    assert L.smuon_ns(arr, arr, 1, None, 0.9, 1.5, -0.5, 0.0, 5, 1e-7, S.NS_EMIT_Q, None, None, None, 0, None,
+                      None) == -1
+    i8 = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 8, 8, S.I8))
+    g = (S.SmuonMat * 1)(m)
+    # int8 momentum cannot take a gradient
+    assert L.smuon_ns(i8, arr, 1, g, 0.9, 1.5, -0.5, 0.0, 5, 1e-7, 0, None, None, None, 0, None, None) == -3
+
+
+def test_workspace_query_runs_on_the_host(L):
+    import matrix_aware_sign_b200 as S
+    arr = (S.SmuonMat * 2)(S.SmuonMat(4096, 64, 147, 147, S.F32), S.SmuonMat(8192, 2048, 512, 512, S.F32))
+    out = ctypes.c_size_t(0)
+    assert L.smuon_ns_workspace_bytes(arr, 2, 5, 0, ctypes.byref(out)) == 0
+    # at least the bf16 X operands and f32 masters of both matrices
+    assert out.value > (64 * 256 + 512 * 2048) * (2 + 2 + 4 + 4)
+    out2 = ctypes.c_size_t(0)
+    assert L.smuon_ns_workspace_bytes(arr, 2, 1, 0, ctypes.byref(out2)) == 0
+    assert out2.value < out.value
+
+
+def test_update_rejects_bad_source_combinations(L):
+    import matrix_aware_sign_b200 as S
+    W = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 8, 8, S.F32))
+    assert L.smuon_update(W, 1, None, None, None, 1, 0.01, 0, 0, None, None, None) == -1
+    assert L.smuon_update(W, 1, W, W, None, 1, 0.01, 0, 0, None, None, None) == -1
+    assert L.smuon_update(W, 1, W, None, None, 1, 0.01, 0, 7, None, None, None) == -1

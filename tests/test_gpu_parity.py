@@ -1,0 +1,389 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
+on the same seeded inputs. Integer and rounding work (sign, pack, vote,
+update, LionMuon EMA) must be bit-exact; Newton-Schulz outputs must meet the
+path's tolerances (relative Frobenius error <= 1e-2 with BF16 tensor-core
+operands, <= 1e-4 in the FP32 reference mode; sign disagreements <= 1e-4 of
+entries and only where |U_oracle| < 1e-3 max|U_oracle|)."""
+import numpy as np
+import pytest
+import torch
+
+import matrix_aware_sign_b200 as S
+import oracle as O
+import workloads as WL
+from tests.gpu_util import check_ns_outputs, dev, host, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+SHAPES_SMALL = [(1, 1), (7, 13), (33, 65), (64, 147), (256, 256), (300, 130)]
+
+
+# ------------------------------------------------------------------ sign / pack / vote
+@pytest.mark.parametrize("shape", SHAPES_SMALL)
+@pytest.mark.parametrize("M", [1, 3, 4, 16])
+@pytest.mark.parametrize("udtype", ["bf16", "f32"])
+def test_sign_pack_vote_bit_exact(shape, M, udtype):
+    U = WL.synthetic_polar_outputs(shape, M, seed=hash((shape, M)) % 1000, dtype=udtype, zero_fraction=0.05)
+    tdt = torch.bfloat16 if udtype == "bf16" else torch.float32
+    Ud = [dev(u, tdt) for u in U]
+    n = shape[0] * shape[1]
+    words = S.packed_words(n)
+    packed = torch.full((M, words), 0xDEAD, dtype=torch.int32, device="cuda")
+    signs = torch.zeros((M, n), dtype=torch.int8, device="cuda")
+    S.smuon_sign_pack(Ud, packed=packed, signs_i8=signs)
+    torch.cuda.synchronize()
+    for k in range(M):
+        s_ref = O.sign_extract(U[k]).reshape(-1)
+        np.testing.assert_array_equal(host(signs[k]), s_ref)
+        np.testing.assert_array_equal(packed[k].cpu().numpy().view(np.uint32), O.pack_bits(s_ref))
+    for tie in (0, 1, -1):
+        v1 = torch.zeros(n, dtype=torch.int8, device="cuda")
+        v2 = torch.zeros(n, dtype=torch.int8, device="cuda")
+        S.smuon_vote(M, n, v1, packed=packed, tie_value=tie)
+        S.smuon_vote(M, n, v2, signs_i8=signs, tie_value=tie)
+        torch.cuda.synchronize()
+        ref = O.vote_from_signs([O.sign_extract(u).reshape(-1) for u in U], tie)
+        np.testing.assert_array_equal(host(v1), ref)
+        np.testing.assert_array_equal(host(v2), ref)
+
+
+@pytest.mark.parametrize("wdtype", ["f32", "bf16"])
+@pytest.mark.parametrize("kind", [S.VOTE_POPCOUNT, S.VOTE_INT8])
+@pytest.mark.parametrize("M,tie", [(3, 0), (4, 0), (4, 1), (8, -1), (33, 0)])
+def test_fused_vote_update_bit_exact(wdtype, kind, M, tie):
+    shapes = [(64, 147), (7, 13), (256, 256), (1, 1), (130, 300)]
+    W = WL.weights(shapes, "normal002", wdtype)
+    tw = torch.bfloat16 if wdtype == "bf16" else torch.float32
+    Wd = [dev(w, tw) for w in W]
+    U = [WL.synthetic_polar_outputs(s, M, seed=10 + i, dtype="bf16", zero_fraction=0.02)
+         for i, s in enumerate(shapes)]
+    Ud = [[dev(u, torch.bfloat16) for u in layer] for layer in U]
+    packed = [torch.zeros((M, S.packed_words(r * c)), dtype=torch.int32, device="cuda") for r, c in shapes]
+    votes = [torch.zeros(r * c, dtype=torch.int8, device="cuda") for r, c in shapes]
+    eta = 0.02
+    S.smuon_update(Wd, eta, U=Ud, M=M, tie_value=tie, vote_kind=kind, packed_out=packed, vote_out=votes)
+    torch.cuda.synchronize()
+    for i, s in enumerate(shapes):
+        signs = [O.sign_extract(u) for u in U[i]]
+        v = O.vote_from_signs(signs, tie)
+        np.testing.assert_array_equal(host(votes[i]).reshape(s), v)
+        for k in range(M):
+            np.testing.assert_array_equal(packed[i][k].cpu().numpy().view(np.uint32), O.pack_bits(signs[k]))
+        ref = O.update_with_vote(W[i], v, eta, wdtype)
+        np.testing.assert_array_equal(host(Wd[i]), ref)
+
+
+def test_fused_update_strided_matrices():
+    """Leading dimension larger than the width takes the scalar path."""
+    M, shape = 5, (37, 50)
+    W = WL.weights([shape], "normal002", "f32")[0]
+    Wbig = torch.zeros((37, 64), device="cuda")
+    Wbig[:, :50] = dev(W)
+    Wv = Wbig[:, :50]
+    U = WL.synthetic_polar_outputs(shape, M, seed=3, dtype="f32")
+    Ubig = [torch.zeros((37, 72), device="cuda") for _ in range(M)]
+    for k in range(M):
+        Ubig[k][:, :50] = dev(U[k])
+    S.smuon_update([Wv], 0.01, U=[[u[:, :50] for u in Ubig]], M=M)
+    torch.cuda.synchronize()
+    v = O.vote_from_signs([O.sign_extract(u) for u in U])
+    np.testing.assert_array_equal(host(Wv), O.update_with_vote(W, v, 0.01, "f32"))
+    assert torch.all(Wbig[:, 50:] == 0)
+
+
+@pytest.mark.parametrize("wdtype", ["f32", "bf16"])
+def test_update_from_votes_and_dense(wdtype):
+    shapes = [(65, 33), (128, 256)]
+    tw = torch.bfloat16 if wdtype == "bf16" else torch.float32
+    rng = np.random.default_rng(5)
+    W = WL.weights(shapes, "normal002", wdtype)
+    V = [rng.integers(-1, 2, s).astype(np.int8) for s in shapes]
+    D = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    Wd = [dev(w, tw) for w in W]
+    S.smuon_update(Wd, 0.01, votes=[dev(v, torch.int8) for v in V])
+    torch.cuda.synchronize()
+    for i in range(2):
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], V[i], 0.01, wdtype))
+    Wd = [dev(w, tw) for w in W]
+    S.smuon_update(Wd, 0.003, dense=[dev(d) for d in D])
+    torch.cuda.synchronize()
+    for i in range(2):
+        np.testing.assert_array_equal(host(Wd[i]), O.update_dense(W[i], D[i], 0.003, wdtype))
+
+
+# ------------------------------------------------------------------ Newton-Schulz
+NS_CASES = [
+    ((256, 256), WL.CUBIC, 5),
+    ((64, 147), WL.QUINTIC, 1),
+    ((147, 64), WL.QUINTIC, 2),
+    ((300, 130), WL.QUINTIC, 3),
+    ((129, 513), WL.CUBIC, 2),
+    ((1, 40), WL.QUINTIC, 1),
+    ((384, 1000), WL.QUINTIC, 5),
+]
+
+
+def _ns_run(mats, coeffs, iters, flags, G=None, beta=0.0, udtype=torch.float32, status=None):
+    Md = [dev(m) for m in mats]
+    Ud = [torch.full(m.shape, float("nan"), dtype=udtype, device="cuda") for m in mats]
+    Gd = None if G is None else [dev(g) for g in G]
+    S.smuon_ns(Md, Ud, *coeffs, iters, G=Gd, beta=beta, flags=flags, status=status)
+    torch.cuda.synchronize()
+    return Md, Ud
+
+
+@pytest.mark.parametrize("shape,coeffs,iters", NS_CASES)
+def test_ns_fp32_reference_mode(shape, coeffs, iters):
+    rng = np.random.default_rng(shape[0] * 7 + iters)
+    M = rng.standard_normal(shape).astype(np.float32)
+    _, Ud = _ns_run([M], coeffs, iters, S.NS_FP32_REF)
+    ref = O.newton_schulz(M, *coeffs, iters)
+    check_ns_outputs([(host(Ud[0]), ref)], 1e-4)
+
+
+@pytest.mark.parametrize("shape,coeffs,iters", NS_CASES)
+def test_ns_split_bf16_mode(shape, coeffs, iters):
+    """Accurate tensor-core mode: hi/lo bf16 operands meet the criteria for
+    every iteration count and coefficient set."""
+    rng = np.random.default_rng(shape[1] * 5 + iters)
+    M = rng.standard_normal(shape).astype(np.float32)
+    _, Ud = _ns_run([M], coeffs, iters, S.NS_SPLIT_BF16, udtype=torch.bfloat16)
+    ref = O.newton_schulz(M, *coeffs, iters)
+    check_ns_outputs([(host(Ud[0]), ref)], 1e-2)
+
+
+FAST_SETS = [
+    # the cubic and one-step quintic workloads run in plain BF16
+    ([(256, 256)] * 3, WL.CUBIC, 5),
+    ([(64, 147), (64, 576), (256, 64), (128, 1152), (512, 128), (256, 2304), (1024, 256), (512, 4608)],
+     WL.QUINTIC, 1),
+]
+
+
+@pytest.mark.parametrize("shapes,coeffs,iters", FAST_SETS)
+@pytest.mark.parametrize("mode", [0, S.NS_SIMT_BF16])
+def test_ns_plain_bf16_meets_criteria_where_used(shapes, coeffs, iters, mode):
+    rng = np.random.default_rng(len(shapes) + iters)
+    mats = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    _, Ud = _ns_run(mats, coeffs, iters, mode, udtype=torch.bfloat16)
+    check_ns_outputs([(host(u), O.newton_schulz(m, *coeffs, iters)) for u, m in zip(Ud, mats)], 1e-2)
+
+
+@pytest.mark.parametrize("shape", [(384, 1000), (768, 768)])
+def test_ns_plain_bf16_error_envelope_five_quintic(shape):
+    """Plain BF16 operands do not reach 1e-2 after five quintic steps (bf16
+    rounding of X, A and B amplified by the iteration); this records the
+    measured envelope, and the split mode above is the one that meets it."""
+    rng = np.random.default_rng(2)
+    M = rng.standard_normal(shape).astype(np.float32)
+    _, Ud = _ns_run([M], WL.QUINTIC, 5, 0, udtype=torch.bfloat16)
+    e = rel_fro(host(Ud[0]), O.newton_schulz(M, *WL.QUINTIC, 5))
+    assert 3e-3 < e < 3e-2, e
+
+
+def test_ns_tcgen05_matches_cuda_core_bf16():
+    """The tcgen05 kernel and the CUDA-core kernel see the same bf16 operands;
+    they differ only in float32 accumulation order."""
+    rng = np.random.default_rng(11)
+    mats = [rng.standard_normal(s).astype(np.float32) for s in [(256, 640), (640, 256), (128, 128), (200, 77)]]
+    _, U_tc = _ns_run(mats, WL.QUINTIC, 2, 0)
+    _, U_simt = _ns_run(mats, WL.QUINTIC, 2, S.NS_SIMT_BF16)
+    for a, b in zip(U_tc, U_simt):
+        assert rel_fro(host(a), host(b)) < 2e-3
+
+
+def test_ns_batched_groups_and_momentum():
+    """Many shapes in one call (several groups, tall and wide), with the
+    momentum update M <- beta*M + G fused in front."""
+    shapes = [(64, 147), (256, 64), (64, 256), (512, 128), (128, 512), (300, 200), (200, 300), (64, 147)]
+    rng = np.random.default_rng(21)
+    M0 = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    G = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    Md, Ud = _ns_run(M0, WL.QUINTIC, 1, 0, G=G, beta=0.9)
+    pairs = []
+    for i in range(len(shapes)):
+        Mref = O.momentum(M0[i], G[i], 0.9)
+        np.testing.assert_allclose(host(Md[i]), Mref, rtol=2e-6, atol=1e-6)
+        pairs.append((host(Ud[i]), O.newton_schulz(Mref, *WL.QUINTIC, 1)))
+    check_ns_outputs(pairs, 1e-2)
+
+
+def test_ns_int8_input_for_local_polar_step():
+    rng = np.random.default_rng(9)
+    V = rng.integers(-1, 2, (96, 200)).astype(np.int8)
+    Vd = dev(V, torch.int8)
+    Ud = torch.zeros((96, 200), device="cuda")
+    S.smuon_ns([Vd], [Ud], *WL.QUINTIC, 2, flags=S.NS_SPLIT_BF16)
+    torch.cuda.synchronize()
+    check_ns_outputs([(host(Ud), O.newton_schulz(V.astype(np.float64), *WL.QUINTIC, 2))], 1e-2)
+
+
+def test_ns_nonfinite_norm_sets_status():
+    M = np.ones((64, 64), np.float32)
+    M[3, 4] = np.nan
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _ns_run([M], WL.CUBIC, 1, 0, status=status)
+    assert int(status.item()) & S.DEV_NONFINITE_NORM
+
+
+def test_ns_skip_flag_leaves_outputs_untouched():
+    M = np.random.default_rng(1).standard_normal((64, 96)).astype(np.float32)
+    Md = [dev(M)]
+    Ud = [torch.full((64, 96), 7.0, device="cuda")]
+    flag = torch.ones(1, dtype=torch.int32, device="cuda")
+    S.smuon_ns(Md, Ud, *WL.QUINTIC, 5, G=[dev(M)], beta=0.9, skip_if=flag)
+    torch.cuda.synchronize()
+    assert torch.all(Ud[0] == 7.0)
+    np.testing.assert_array_equal(host(Md[0]), M)
+
+
+# ------------------------------------------------------------------ whole steps
+def test_config1_full_step():
+    cfg = WL.SIGN_MUON_WORKLOADS["c1_256sq"]
+    W = WL.weights(cfg.shapes, cfg.w_init, cfg.w_dtype)
+    grads = WL.GradientStreams(cfg.shapes, cfg.workers, cfg.grad_sigma).next_step()
+    Md = [torch.zeros(cfg.shapes[0], device="cuda") for _ in range(cfg.workers)]
+    Ud = [torch.zeros(cfg.shapes[0], dtype=torch.bfloat16, device="cuda") for _ in range(cfg.workers)]
+    S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=[dev(g) for g in grads[0]], beta=cfg.beta)
+    Wd = [dev(W[0])]
+    votes = torch.zeros(256 * 256, dtype=torch.int8, device="cuda")
+    S.smuon_update(Wd, cfg.eta, U=[Ud], M=cfg.workers, vote_out=[votes])
+    torch.cuda.synchronize()
+    ref = O.sign_muon_step(W, [[np.zeros(cfg.shapes[0])] * cfg.workers], grads, cfg.beta, cfg.coeffs,
+                           cfg.iters, cfg.eta, cfg.w_dtype)
+    check_ns_outputs([(host(u), r) for u, r in zip(Ud, ref["U"][0])], 1e-2)
+    v_gpu = host(votes).reshape(256, 256)
+    agree = v_gpu == ref["vote"][0]
+    assert (~agree).mean() <= 1e-4
+    np.testing.assert_array_equal(host(Wd[0])[agree], ref["W"][0][agree])
+
+
+def test_config2_resnet50_one_step():
+    cfg = WL.SIGN_MUON_WORKLOADS["c2_resnet50"]
+    W = WL.weights(cfg.shapes, cfg.w_init, cfg.w_dtype)
+    grads = WL.GradientStreams(cfg.shapes, cfg.workers, cfg.grad_sigma).next_step()
+    Md = [torch.zeros(s, device="cuda") for s in cfg.shapes for _ in range(cfg.workers)]
+    Ud = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in cfg.shapes for _ in range(cfg.workers)]
+    Gd = [dev(g) for layer in grads for g in layer]
+    S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=Gd, beta=cfg.beta)
+    Wd = [dev(w) for w in W]
+    L = len(cfg.shapes)
+    votes = [torch.zeros(r * c, dtype=torch.int8, device="cuda") for r, c in cfg.shapes]
+    S.smuon_update(Wd, cfg.eta, U=[Ud[l * cfg.workers:(l + 1) * cfg.workers] for l in range(L)], M=cfg.workers,
+                   vote_kind=S.VOTE_INT8, vote_out=votes)
+    torch.cuda.synchronize()
+    pairs, n_vdis, n_all = [], 0, 0
+    for l in range(L):
+        for k in range(cfg.workers):
+            ref_u = O.newton_schulz(grads[l][k].astype(np.float64), *cfg.coeffs, cfg.iters)
+            pairs.append((host(Ud[l * cfg.workers + k]), ref_u))
+        ref_v = O.vote_from_signs([O.sign_extract(p[1]) for p in pairs[-cfg.workers:]])
+        v_gpu = host(votes[l]).reshape(cfg.shapes[l])
+        agree = v_gpu == ref_v
+        n_vdis += int((~agree).sum())
+        n_all += agree.size
+        ref_w = O.update_with_vote(W[l], ref_v, cfg.eta, "f32")
+        np.testing.assert_array_equal(host(Wd[l])[agree], ref_w[agree])
+    check_ns_outputs(pairs, 1e-2)
+    assert n_vdis <= 1e-4 * n_all
+
+
+# ------------------------------------------------------------------ CacheMuon
+@pytest.mark.parametrize("shape", [(256, 384), (384, 256)])
+def test_cachemuon_fresh_q_and_probe(shape):
+    coeffs, K = WL.QUINTIC, 5
+    mom = list(WL.cachemuon_momenta(shape, 2, drift=0.01, seed0=77))
+    m = min(shape)
+    Md = dev(mom[0])
+    Ud = torch.zeros(shape, device="cuda")
+    Qd = torch.zeros((m, m), dtype=torch.bfloat16, device="cuda")
+    S.smuon_ns([Md], [Ud], *coeffs, K, flags=S.NS_EMIT_Q | S.NS_SPLIT_BF16, Q_out=[Qd])
+    torch.cuda.synchronize()
+    D_ref, Q_ref = O.newton_schulz_with_q(mom[0], *coeffs, K)
+    check_ns_outputs([(host(Ud), D_ref)], 1e-2)
+    assert rel_fro(host(Qd), Q_ref) < 1e-2
+    # probe the cached transform on the drifted momentum
+    err = torch.zeros(1, device="cuda")
+    acc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cnt = S.new_counters()
+    Dh = torch.zeros(shape, device="cuda")
+    S.cachemuon_reuse_probe(Qd, dev(mom[1]), Dh, 1e9, err, acc, cnt)
+    torch.cuda.synchronize()
+    Dh_ref, err_ref = O.cachemuon_probe(Q_ref, mom[1])
+    assert rel_fro(host(Dh), Dh_ref) < 1e-2
+    assert abs(err.item() - err_ref) <= 2e-2 * max(err_ref, 1e-3) + 1e-3
+    assert acc.item() == 1 and cnt.tolist()[:3] == [1, 0, 1]
+    # the same probe against a threshold below the residual rejects
+    S.cachemuon_reuse_probe(Qd, dev(mom[1]), Dh, err_ref / 4, err, acc, cnt)
+    torch.cuda.synchronize()
+    assert acc.item() == 0 and cnt.tolist()[:3] == [1, 1, 2]
+
+
+def test_cachemuon_first_step_and_skip():
+    shape = (128, 192)
+    M = next(WL.cachemuon_momenta(shape, 1, seed0=5))
+    err = torch.zeros(1, device="cuda")
+    acc = torch.ones(1, dtype=torch.int32, device="cuda")
+    cnt = S.new_counters()
+    Dh = torch.zeros(shape, device="cuda")
+    S.cachemuon_reuse_probe(None, dev(M), Dh, 15.0, err, acc, cnt)
+    Qd = torch.zeros((128, 128), dtype=torch.bfloat16, device="cuda")
+    S.smuon_ns([dev(M)], [Dh], *WL.QUINTIC, 5, flags=S.NS_EMIT_Q | S.NS_SPLIT_BF16, Q_out=[Qd], skip_if=acc)
+    torch.cuda.synchronize()
+    assert acc.item() == 0 and np.isinf(err.item()) and cnt.tolist()[:2] == [0, 1]
+    check_ns_outputs([(host(Dh), O.newton_schulz(M, *WL.QUINTIC, 5))], 1e-2)
+
+
+# ------------------------------------------------------------------ LionMuon
+def _lion_setup(shapes, workers, seed, wdtype="bf16"):
+    W = WL.weights(shapes, "normal002", wdtype)
+    rng = np.random.default_rng(seed)
+    mom = [[np.zeros(s, np.float32) for _ in range(workers)] for s in shapes]
+    return W, mom, rng
+
+
+def test_lionmuon_sign_steps_bit_exact():
+    shapes, M = [(64, 96), (96, 64), (33, 17)], 4
+    W, mom, rng = _lion_setup(shapes, M, 1)
+    Wd = [dev(w, torch.bfloat16) for w in W]
+    md = [[dev(x) for x in layer] for layer in mom]
+    opt = S.LionMuon(Wd, md)
+    for t in range(1, 4):
+        G = [[rng.standard_normal(s).astype(np.float32) for _ in range(M)] for s in shapes]
+        S.lionmuon_step(opt, [[dev(g) for g in layer] for layer in G], 0, 0.9, 0.99, 3e-4, *WL.QUINTIC, 5)
+        kind, W, mom = O.lionmuon_step(t, W, mom, G, 0, 0.9, 0.99, 3e-4, WL.QUINTIC, 5, "bf16")
+        assert kind == "sign"
+    torch.cuda.synchronize()
+    assert opt.t == 3
+    for l in range(len(shapes)):
+        np.testing.assert_array_equal(host(Wd[l]), W[l])
+        for k in range(M):
+            np.testing.assert_array_equal(host(md[l][k]), mom[l][k])
+
+
+def test_lionmuon_period_schedule():
+    shapes, M = [(64, 128), (128, 64)], 3
+    W, mom, rng = _lion_setup(shapes, M, 2, "f32")
+    Wd = [dev(w) for w in W]
+    md = [[dev(x) for x in layer] for layer in mom]
+    opt = S.LionMuon(Wd, md)
+    eta = 1e-2
+    for t in range(1, 3):  # P = 2: step 1 sign, step 2 Muon
+        G = [[rng.standard_normal(s).astype(np.float32) for _ in range(M)] for s in shapes]
+        S.lionmuon_step(opt, [[dev(g) for g in layer] for layer in G], 2, 0.9, 0.99, eta, *WL.QUINTIC, 5,
+                        ns_flags=S.NS_SPLIT_BF16)
+        torch.cuda.synchronize()
+        Wprev = [w.copy() for w in W]
+        kind, W, mom = O.lionmuon_step(t, W, mom, G, 2, 0.9, 0.99, eta, WL.QUINTIC, 5, "f32")
+        for l in range(len(shapes)):
+            for k in range(M):
+                np.testing.assert_array_equal(host(md[l][k]), mom[l][k])
+            if kind == "sign":
+                np.testing.assert_array_equal(host(Wd[l]), W[l])
+            else:
+                # float32 weights: the applied direction is the Muon direction,
+                # within the BF16 Newton-Schulz tolerance of the oracle's
+                d_gpu = (host(Wd[l]).astype(np.float64) - Wprev[l]) / -eta
+                d_ref = (W[l].astype(np.float64) - Wprev[l]) / -eta
+                assert rel_fro(d_gpu, d_ref) < 1e-2
+    assert opt.t == 2
