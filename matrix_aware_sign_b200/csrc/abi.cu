@@ -264,6 +264,16 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
       d.u_ptr = rq.U_out[i].data; d.u_ld = rq.U_out[i].ld; d.u_dtype = rq.U_out[i].dtype;
       if (rq.Q_out && (emit_q || rq.probe)) { d.q_ptr = rq.Q_out[i].data; d.q_ld = rq.Q_out[i].ld; }
       d.rows = M.rows; d.cols = M.cols; d.tall = M.rows > M.cols ? 1 : 0;
+      auto rows16 = [](const void* p, int64_t ld, int32_t dt) {
+        return p && reinterpret_cast<uintptr_t>(p) % 16 == 0 && (ld * dtype_size(dt)) % 16 == 0;
+      };
+      d.vec = 0;
+      if (M.dtype != SMUON_I8 && rows16(d.m_ptr, d.m_ld, d.m_dtype)) d.vec |= 1;
+      if (rows16(d.u_ptr, d.u_ld, d.u_dtype)) d.vec |= 2;
+      if (rows16(d.q_ptr, d.q_ld, SMUON_BF16)) d.vec |= 4;
+      if (M.dtype == SMUON_F32 && rows16(d.m_ptr, d.m_ld, SMUON_F32) && M.cols % 4 == 0 &&
+          (!d.g_ptr || (d.g_dtype == SMUON_F32 && rows16(d.g_ptr, d.g_ld, SMUON_F32))))
+        d.vec |= 8;
       d.group = (int32_t)B->groups.size();
       d.z = z;
       d.mom_tiles_c = ceil_div(M.cols, 64);
@@ -321,7 +331,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.plan_bytes = (size_t)round_up((int64_t)B->cursor, 256);
   L.off_partials = B->take(sizeof(float) * std::max(mom_tiles, 1));
   L.off_scale = B->take(sizeof(float) * B->mats.size());
-  L.off_probe = B->take(sizeof(float) * 4 * std::max(totals[ST_PROBE], 1));
+  L.off_probe = B->take(sizeof(float) * kProbeSlots * std::max(totals[ST_PROBE], 1));
 
   // per-group buffers
   for (auto& g : B->groups) {

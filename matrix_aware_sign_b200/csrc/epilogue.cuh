@@ -88,19 +88,82 @@ __device__ __forceinline__ void ld_f32_vec(const float* p, float* v) {
   }
 }
 
+__device__ __forceinline__ void unpack_bf16x8(const uint4 w, float* o) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    o[2 * k] = __uint_as_float(u[k] << 16);
+    o[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+  }
+}
+
+// read a wide-form row chunk (row i, cols j0..j0+NV-1) of a user matrix: a
+// wide matrix is read along its row (vector loads when rows are 16-byte
+// aligned), a tall one down its column (lanes hold consecutive rows, so each
+// warp access is contiguous)
+template <int NV>
+__device__ __forceinline__ void ld_user(const void* p, int64_t ld, int32_t dtype, int tall, int vec, int row,
+                                        int col0, int nvalid, float* out) {
+  if (!tall) {
+    const int64_t base = (int64_t)row * ld + col0;
+    if (vec && nvalid == NV) {
+      if (dtype == SMUON_F32) {
+        ld_f32_vec<NV>(reinterpret_cast<const float*>(p) + base, out);
+        return;
+      }
+      if (dtype == SMUON_BF16 && NV % 8 == 0) {
+        const uint4* q = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + base);
+#pragma unroll
+        for (int k = 0; k < NV / 8; ++k) unpack_bf16x8(q[k], out + 8 * k);
+        return;
+      }
+    }
+    if (dtype == SMUON_F32) {
+#pragma unroll
+      for (int k = 0; k < NV; ++k) out[k] = k < nvalid ? reinterpret_cast<const float*>(p)[base + k] : 0.f;
+    } else {
+#pragma unroll
+      for (int k = 0; k < NV; ++k) out[k] = k < nvalid ? load_as_f32(p, base + k, dtype) : 0.f;
+    }
+  } else {
+    if (dtype == SMUON_F32) {
+      const float* q = reinterpret_cast<const float*>(p) + row;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) out[k] = k < nvalid ? q[(int64_t)(col0 + k) * ld] : 0.f;
+    } else {
+#pragma unroll
+      for (int k = 0; k < NV; ++k) out[k] = k < nvalid ? load_as_f32(p, (int64_t)(col0 + k) * ld + row, dtype) : 0.f;
+    }
+  }
+}
+
 // user-orientation store of a wide-form row chunk (row i, cols j0..j0+NV-1)
 template <int NV>
-__device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int tall, int row,
+__device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int tall, int vec, int row,
                                         int col0, int nvalid, const float* v) {
   if (!tall) {
-    int64_t base = (int64_t)row * ld + col0;
+    const int64_t base = (int64_t)row * ld + col0;
+    if (vec && nvalid == NV) {
+      if (dtype == SMUON_F32) {
+        st_f32_vec<NV>(reinterpret_cast<float*>(p) + base, v);
+        return;
+      }
+      st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(p) + base, v);
+      return;
+    }
 #pragma unroll
     for (int q = 0; q < NV; ++q)
       if (q < nvalid) store_from_f32(p, base + q, dtype, v[q]);
-  } else {
+  } else if (dtype == SMUON_BF16) {
+    __nv_bfloat16* q = reinterpret_cast<__nv_bfloat16*>(p) + row;
 #pragma unroll
-    for (int q = 0; q < NV; ++q)
-      if (q < nvalid) store_from_f32(p, (int64_t)(col0 + q) * ld + row, dtype, v[q]);
+    for (int k = 0; k < NV; ++k)
+      if (k < nvalid) q[(int64_t)(col0 + k) * ld] = __float2bfloat16_rn(v[k]);
+  } else {
+    float* q = reinterpret_cast<float*>(p) + row;
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+      if (k < nvalid) q[(int64_t)(col0 + k) * ld] = v[k];
   }
 }
 
@@ -112,7 +175,7 @@ __device__ __forceinline__ void emit_q1(const TileCtx& t, int row, int col0, int
 #pragma unroll
   for (int k = 0; k < NV; ++k) q[k] = B[k] + ((row == col0 + k) ? t.a : 0.f);
   if (t.iter == t.last) {  // K == 1: Q_1 is the final transform
-    st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, row, col0, nvalid, q);
+    st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, (t.md->vec >> 2) & 1, row, col0, nvalid, q);
   } else {
     if (t.bf) st_f32_vec<NV>(t.g->qf[1] + off, q);
     st_operand<NV>(t, t.g->qop[1], off, t.mlo, q);
@@ -162,16 +225,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       if (first && t.bf) {
         // X_0 read from the user's momentum in its own dtype and orientation
         const MatDesc& md = *t.md;
-#pragma unroll
-        for (int k = 0; k < NV; ++k) {
-          float src = 0.f;
-          if (k < nvalid) {
-            const int64_t idx = md.tall ? (int64_t)(col0 + k) * md.m_ld + row
-                                        : (int64_t)row * md.m_ld + col0 + k;
-            src = load_as_f32(md.m_ptr, idx, md.m_dtype);
-          }
-          x[k] = src;
-        }
+        ld_user<NV>(md.m_ptr, md.m_ld, md.m_dtype, md.tall, md.vec & 1, row, col0, nvalid, x);
       } else {
         const float* src = t.bf ? g.xf[t.iter & 1] : reinterpret_cast<const float*>(g.xop[t.iter & 1]);
         ld_f32_vec<NV>(src + off, x);
@@ -183,7 +237,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
         if (t.bf) st_f32_vec<NV>(g.xf[nb] + off, x);
         st_operand<NV>(t, g.xop[nb], off, t.xlo, x);
       } else {
-        st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, row, col0, nvalid, x);
+        st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, x);
       }
       break;
     }
@@ -199,7 +253,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
         if (t.bf) st_f32_vec<NV>(g.qf[nb] + off, q);
         st_operand<NV>(t, g.qop[nb], off, t.mlo, q);
       } else {
-        st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, row, col0, nvalid, q);
+        st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, (t.md->vec >> 2) & 1, row, col0, nvalid, q);
       }
       break;
     }
@@ -207,7 +261,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       const int64_t off = ((int64_t)t.z * m + row) * g.ldn + col0;
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] *= t.s;
-      st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, row, col0, nvalid, v);
+      st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, v);
       st_op<NV>(g.xop[1], off, t.bf, v);
       break;
     }

@@ -40,12 +40,33 @@ __device__ __forceinline__ void put_x0(const GroupDesc& g, int bf, int split, in
 // SignMuon summary, algorithm flow step 1: momentum update (reading R1) fused
 // with the sum of squares for the Frobenius norm and the bf16/f32 operand
 // copy of X0 in the wide orientation (tall matrices transposed through smem).
+__device__ __forceinline__ void put_x0_4(const GroupDesc& g, int bf, int split, int64_t o, const float* v) {
+  if (!bf) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(g.xop[0]) + o) = make_float4(v[0], v[1], v[2], v[3]);
+    return;
+  }
+  uint2 hi;
+  hi.x = pack_bf16x2_rn(v[0], v[1]);
+  hi.y = pack_bf16x2_rn(v[2], v[3]);
+  *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(g.xop[0]) + o) = hi;
+  if (split) {
+    float lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) lo[k] = v[k] - __bfloat162float(__float2bfloat16_rn(v[k]));
+    uint2 l;
+    l.x = pack_bf16x2_rn(lo[0], lo[1]);
+    l.y = pack_bf16x2_rn(lo[2], lo[3]);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(g.xop[0]) + o + (int64_t)g.count * g.m * g.ldn) = l;
+  }
+}
+
 __global__ void __launch_bounds__(256) k_momentum(const Plan* plan, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
   __shared__ float tile[64][65];
   __shared__ float red[8];
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+  const int bf = (h.mode != MODE_SIMT_F32);
+  const int split = (h.flags & SMUON_NS_SPLIT_BF16) != 0;
   for (int t = blockIdx.x; t < h.total_mom_tiles; t += gridDim.x) {
     const int mi = find_mat_by_mom_tile(h, t);
     const MatDesc& md = h.mats[mi];
@@ -53,43 +74,74 @@ __global__ void __launch_bounds__(256) k_momentum(const Plan* plan, const int32_
     const int local = t - md.mom_begin;
     const int tr = local / md.mom_tiles_c, tc = local - (local / md.mom_tiles_c) * md.mom_tiles_c;
     const int r0 = tr * 64, c0 = tc * 64;
-    float ss = 0.f;
-    for (int rr = ty; rr < 64; rr += 4) {
-      const int r = r0 + rr, c = c0 + tx;
-      float val = 0.f;
-      if (r < md.rows && c < md.cols) {
-        const int64_t idx = (int64_t)r * md.m_ld + c;
-        float mv = load_as_f32(md.m_ptr, idx, md.m_dtype);
-        if (md.g_ptr) {
-          const float gv = load_as_f32(md.g_ptr, (int64_t)r * md.g_ld + c, md.g_dtype);
-          mv = fmaf(h.beta, mv, gv);
-          reinterpret_cast<float*>(md.m_ptr)[idx] = mv;
-        }
-        val = mv;
-      }
-      ss = fmaf(val, val, ss);
-      tile[rr][tx] = val;
-    }
-    __syncthreads();
-    const int bf = (h.mode != MODE_SIMT_F32);
-    const int split = (h.flags & SMUON_NS_SPLIT_BF16) != 0;
     const int m = g.m;
-    if (!md.tall) {
-      for (int rr = ty; rr < 64; rr += 4) {
-        const int r = r0 + rr, c = c0 + tx;
-        if (r < md.rows && c < md.cols) {
-          const int64_t o = ((int64_t)md.z * m + r) * g.ldn + c;
-          put_x0(g, bf, split, o, tile[rr][tx]);
+    float ss = 0.f;
+    if (md.vec & 8) {
+      // float32 rows, 16-byte aligned: each thread owns 4 consecutive columns of 4 rows
+      const int tx4 = threadIdx.x & 15, ty = threadIdx.x >> 4;
+      const int c = c0 + 4 * tx4;
+      const float* Mp = reinterpret_cast<const float*>(md.m_ptr);
+      const float* Gp = reinterpret_cast<const float*>(md.g_ptr);
+      float4 mv[4], gv[4];
+      bool ok[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int r = r0 + ty + 16 * p;
+        ok[p] = (r < md.rows) && (c < md.cols);
+        mv[p] = make_float4(0.f, 0.f, 0.f, 0.f);
+        gv[p] = mv[p];
+        if (ok[p]) {
+          mv[p] = *reinterpret_cast<const float4*>(Mp + (int64_t)r * md.m_ld + c);
+          if (Gp) gv[p] = *reinterpret_cast<const float4*>(Gp + (int64_t)r * md.g_ld + c);
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int rr = ty + 16 * p, r = r0 + rr;
+        float v[4] = {mv[p].x, mv[p].y, mv[p].z, mv[p].w};
+        if (ok[p] && Gp) {
+          const float gg[4] = {gv[p].x, gv[p].y, gv[p].z, gv[p].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) v[k] = fmaf(h.beta, v[k], gg[k]);
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(md.m_ptr) + (int64_t)r * md.m_ld + c) =
+              make_float4(v[0], v[1], v[2], v[3]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ss = fmaf(v[k], v[k], ss);
+        if (!md.tall) {
+          if (ok[p]) put_x0_4(g, bf, split, ((int64_t)md.z * m + r) * g.ldn + c, v);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) tile[rr][4 * tx4 + k] = v[k];
         }
       }
     } else {
-      // X0[c][r] = M[r][c]: wide row index = user column
+      const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+      for (int rr = ty; rr < 64; rr += 4) {
+        const int r = r0 + rr, c = c0 + tx;
+        float val = 0.f;
+        if (r < md.rows && c < md.cols) {
+          const int64_t idx = (int64_t)r * md.m_ld + c;
+          float mv = load_as_f32(md.m_ptr, idx, md.m_dtype);
+          if (md.g_ptr) {
+            const float gv = load_as_f32(md.g_ptr, (int64_t)r * md.g_ld + c, md.g_dtype);
+            mv = fmaf(h.beta, mv, gv);
+            reinterpret_cast<float*>(md.m_ptr)[idx] = mv;
+          }
+          val = mv;
+          if (!md.tall) put_x0(g, bf, split, ((int64_t)md.z * m + r) * g.ldn + c, val);
+        }
+        ss = fmaf(val, val, ss);
+        tile[rr][tx] = val;
+      }
+    }
+    if (md.tall) {
+      __syncthreads();
+      // X0[c][r] = M[r][c]: the wide row index is the user column; lanes walk user rows
+      const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
       for (int cc = ty; cc < 64; cc += 4) {
         const int c = c0 + cc, r = r0 + tx;
-        if (r < md.rows && c < md.cols) {
-          const int64_t o = ((int64_t)md.z * m + c) * g.ldn + r;
-          put_x0(g, bf, split, o, tile[tx][cc]);
-        }
+        if (r < md.rows && c < md.cols) put_x0(g, bf, split, ((int64_t)md.z * m + c) * g.ldn + r, tile[tx][cc]);
       }
     }
     // deterministic block reduction of the tile's sum of squares
@@ -235,28 +287,38 @@ __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) { mask[k] = 0; sum[k] = 0; }
     const int M = tb.M;
-    for (int wk = 0; wk < M; ++wk) {
-      const EwSrc& S = tb.srcs[L.src_first + wk];
-      float u[8];
-      if (live) load8(S.ptr, S.ld, tb.src_dtype, L, e0, L.vec, u);
-      uint32_t byte = 0;
+    float w[8];
+    if (live) load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+    // workers in groups of four: all loads of a group are issued before any use
+    for (int wk0 = 0; wk0 < M; wk0 += 4) {
+      float u[4][8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const bool pos = live && (e0 + k < L.n) && (u[k] >= 0.f);  // NaN -> negative
-        byte |= (uint32_t)pos << k;
-        if (kPopcount) mask[k] |= (uint64_t)pos << wk;
-        else sum[k] += pos ? 1 : -1;
+      for (int j = 0; j < 4; ++j) {
+        const int wk = wk0 + j;
+        if (wk < M && live) load8(tb.srcs[L.src_first + wk].ptr, tb.srcs[L.src_first + wk].ld, tb.src_dtype, L, e0,
+                                  L.vec, u[j]);
       }
-      if (tb.any_packed) {  // warp-uniform: every lane takes part in the shuffles
-        const uint32_t word = gather_word(byte, lane);
-        if (active && L.packed_out && (lane & 3) == 0)
-          L.packed_out[(int64_t)wk * L.words + ((chunk - L.chunk_begin) >> 2)] = word;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int wk = wk0 + j;
+        if (wk >= M) break;  // uniform across the warp
+        uint32_t byte = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const bool pos = live && (e0 + k < L.n) && (u[j][k] >= 0.f);  // NaN -> negative
+          byte |= (uint32_t)pos << k;
+          if (kPopcount) mask[k] |= (uint64_t)pos << wk;
+          else sum[k] += pos ? 1 : -1;
+        }
+        if (tb.any_packed) {  // warp-uniform: every lane takes part in the shuffles
+          const uint32_t word = gather_word(byte, lane);
+          if (active && L.packed_out && (lane & 3) == 0)
+            L.packed_out[(int64_t)wk * L.words + ((chunk - L.chunk_begin) >> 2)] = word;
+        }
       }
     }
     if (!live) continue;
     int8_t v8[8];
-    float w[8];
-    load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int total = kPopcount ? 2 * __popcll(mask[k]) - M : sum[k];
@@ -403,19 +465,30 @@ __global__ void __launch_bounds__(256) k_lion_sign(const __grid_constant__ EwTab
     uint64_t mask[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) mask[k] = 0;
-    for (int wk = 0; wk < tb.M; ++wk) {
-      const EwSrc& S = tb.srcs[L.src_first + 2 * wk];      // EMA (f32, in/out)
-      const EwSrc& Gs = tb.srcs[L.src_first + 2 * wk + 1]; // gradient (f32)
-      float mo[8], gr[8];
-      load8(S.ptr, S.ld, SMUON_F32, L, e0, L.vec, mo);
-      load8(Gs.ptr, Gs.ld, SMUON_F32, L, e0, L.vec, gr);
+    for (int wk0 = 0; wk0 < tb.M; wk0 += 2) {
+      float mo[2][8], gr[2][8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float gh = __fadd_rn(__fmul_rn(tb.beta1, mo[k]), __fmul_rn(tb.c1, gr[k]));
-        mask[k] |= (uint64_t)(gh >= 0.f) << wk;
-        mo[k] = __fadd_rn(__fmul_rn(tb.beta2, mo[k]), __fmul_rn(tb.c2, gr[k]));
+      for (int j = 0; j < 2; ++j) {
+        const int wk = wk0 + j;
+        if (wk < tb.M) {
+          load8(tb.srcs[L.src_first + 2 * wk].ptr, tb.srcs[L.src_first + 2 * wk].ld, SMUON_F32, L, e0, L.vec, mo[j]);
+          load8(tb.srcs[L.src_first + 2 * wk + 1].ptr, tb.srcs[L.src_first + 2 * wk + 1].ld, SMUON_F32, L, e0,
+                L.vec, gr[j]);
+        }
       }
-      store8(const_cast<void*>(S.ptr), S.ld, SMUON_F32, L, e0, L.vec, mo);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int wk = wk0 + j;
+        if (wk >= tb.M) break;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float gh = __fadd_rn(__fmul_rn(tb.beta1, mo[j][k]), __fmul_rn(tb.c1, gr[j][k]));
+          mask[k] |= (uint64_t)(gh >= 0.f) << wk;
+          mo[j][k] = __fadd_rn(__fmul_rn(tb.beta2, mo[j][k]), __fmul_rn(tb.c2, gr[j][k]));
+        }
+        const EwSrc& S = tb.srcs[L.src_first + 2 * wk];  // EMA (f32, in/out)
+        store8(const_cast<void*>(S.ptr), S.ld, SMUON_F32, L, e0, L.vec, mo[j]);
+      }
     }
     float w[8];
     load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
@@ -469,7 +542,7 @@ __global__ void k_probe_finalize(const Plan* plan) {
   const PlanHeader& h = plan->h;
   if (threadIdx.x >= 32) return;
   const int lane = threadIdx.x;
-  const int n = 4 * h.total_tiles[ST_PROBE];  // four partial sums per tile
+  const int n = kProbeSlots * h.total_tiles[ST_PROBE];
   float acc = 0.f;
   for (int i = lane; i < n; i += 32) acc += h.probe_partials[i];
 #pragma unroll

@@ -131,10 +131,8 @@ __device__ __forceinline__ void gemm_simt_body(const Plan* plan, int stage, int 
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) s += red[w];
-        h.probe_partials[4 * tile] = s;
-        h.probe_partials[4 * tile + 1] = 0.f;
-        h.probe_partials[4 * tile + 2] = 0.f;
-        h.probe_partials[4 * tile + 3] = 0.f;
+        h.probe_partials[kProbeSlots * tile] = s;
+        for (int q = 1; q < kProbeSlots; ++q) h.probe_partials[kProbeSlots * tile + q] = 0.f;
       }
       __syncthreads();
     }

@@ -23,7 +23,7 @@ constexpr int BM = kTcBM, BN = kTcBN, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x 64 k)
 constexpr int B_BYTES = BN * BK * 2;   // one bf16 tile of B
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
 
 // plain BF16: one hi tile per operand; split BF16: hi and lo tiles per operand
 // (x = x_hi + x_lo, product ~ A_hi B_hi + A_hi B_lo + A_lo B_hi)
@@ -182,7 +182,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar + 8 * s, 1); mbar_init(empty_bar + 8 * s, 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar + 8 * a, 1); mbar_init(tempty_bar + 8 * a, 128); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar + 8 * a, 1); mbar_init(tempty_bar + 8 * a, 256); }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -297,8 +297,9 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       while (!mbar_try_wait(done_bar, 0) && clock64() - t0 < kWaitCycles) {}
     }
   } else {
-    // ---------------- epilogue warps 2..5
-    const int ew = warp & 3;  // TMEM lane group this warp may access
+    // ---------------- epilogue warps 2..9: two warps per TMEM lane group, one per half of the columns
+    const int ew = warp & 3;         // TMEM lane group this warp may access
+    const int half = (warp - 2) >> 2;
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -313,7 +314,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       const int row = tm * BM + ew * 32 + lane;
       float pacc = 0.f;
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      for (int ch = half * (BN / 64); ch < (half + 1) * (BN / 64); ++ch) {
         float v[32];
         tmem_ld32(tmem_base + (uint32_t)(acc * BN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
         epi_chunk<32>(t, row, tn * BN + ch * 32, v, &pacc);
@@ -323,7 +324,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       if (stage == ST_PROBE) {  // one partial per epilogue warp: no barrier, fixed order later
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) pacc += __shfl_xor_sync(0xffffffffu, pacc, o2);
-        if (lane == 0) h.probe_partials[4 * tile + ew] = pacc;
+        if (lane == 0) h.probe_partials[kProbeSlots * tile + (warp - 2)] = pacc;
       }
       if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
     }

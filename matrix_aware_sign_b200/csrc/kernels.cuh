@@ -75,6 +75,7 @@ __global__ void k_gemm_simt_bf16(const Plan* plan, int stage, int iter, const in
 // tcgen05 kernel entry (host-side launcher lives in k_gemm_tc.cu)
 cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter,
                            const int32_t* skip, int num_sms, cudaStream_t s);
+constexpr int kProbeSlots = 8;  // residual partial sums per probe tile (one per epilogue warp)
 constexpr int kTcBM = 128;
 constexpr int kTcBN = 128;
 constexpr int kSimtBM = 64;

@@ -43,7 +43,9 @@ struct MatDesc {
   int64_t u_ld;
   void* q_ptr;      // bf16 m x m cached transform (EMIT_Q output, or REUSE input)
   int64_t q_ld;
-  int32_t m_dtype, g_dtype, u_dtype, pad0;
+  int32_t m_dtype, g_dtype, u_dtype;
+  int32_t vec;            // bit 0: M rows 16-byte aligned (vector reads); bit 1: U rows; bit 2: Q rows;
+                          // bit 3: M and G suit the vectorised momentum tile
   int32_t rows, cols, tall, group;
   int32_t z;              // index of this matrix inside its group
   int32_t mom_begin;      // first momentum tile (= partial-sum slot)
