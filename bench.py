@@ -237,9 +237,19 @@ def main():
     g_bytes = n_params * M * 4
     w_bytes = n_params * 4
 
+    # prepared calls (plan handles): each plan's descriptors are uploaded once into its workspace
+    ws2 = S.workspace(ws.numel())
+    ws_e2e = S.workspace(ws.numel()) if args.e2e_steps > 0 else None
+    ns_plans = [S.NsPlan(Md, Ud, *cfg.coeffs, cfg.iters, G=Gd[j], beta=cfg.beta, ws=[ws, ws2][j]) for j in range(2)]
+    upd_plan = S.UpdatePlan(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
+
     def step(i, G=None):
-        S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G if G is not None else Gd[i & 1], beta=cfg.beta, ws=ws)
-        S.smuon_update(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
+        if G is None:
+            ns_plans[i & 1].run()
+            upd_plan.run()
+        else:  # end to end: the one-shot public calls (own workspace, the plans keep theirs)
+            S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G, beta=cfg.beta, ws=ws_e2e)
+            S.smuon_update(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
 
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):

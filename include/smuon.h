@@ -197,6 +197,34 @@ smuon_status smuon_update(const smuon_mat* W, int32_t n_layers,
                           uint32_t* const* packed_out, int8_t* const* vote_out, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Plan handles: the same calls, prepared once and launched many times.
+ *
+ * smuon_ns_plan_create checks its arguments like smuon_ns, builds the plan
+ * and uploads it into ws on `stream`; smuon_ns_execute then enqueues only the
+ * kernels (d_skip_if as in smuon_ns). smuon_update_plan_create /
+ * smuon_update_execute do the same for smuon_update. Between executions the
+ * matrices' contents may change but not their addresses, and ws must hold
+ * the plan (do not use it for another call). A handle is a small host object
+ * owned by the caller; smuon_plan_destroy frees it (device memory is never
+ * allocated). Executing a plan is capturable in a CUDA graph.
+ * ---------------------------------------------------------------------- */
+typedef struct smuon_plan_s* smuon_plan;
+
+smuon_status smuon_ns_plan_create(const smuon_mat* M_in, const smuon_mat* U_out, int32_t n_mats,
+                                  const smuon_mat* G, float beta, float a, float b, float c,
+                                  int32_t iters, float eps, uint32_t flags, const smuon_mat* Q_out,
+                                  void* ws, size_t ws_bytes, int32_t* d_status, void* stream,
+                                  smuon_plan* out);
+smuon_status smuon_ns_execute(smuon_plan plan, const int32_t* d_skip_if, void* stream);
+smuon_status smuon_update_plan_create(const smuon_mat* W, int32_t n_layers, const smuon_mat* U,
+                                      const smuon_mat* votes, const smuon_mat* dense, int32_t M,
+                                      float eta, int8_t tie_value, uint32_t vote_kind,
+                                      uint32_t* const* packed_out, int8_t* const* vote_out,
+                                      smuon_plan* out);
+smuon_status smuon_update_execute(smuon_plan plan, void* stream);
+void         smuon_plan_destroy(smuon_plan plan);
+
+/* ------------------------------------------------------------------------
  * cachemuon_reuse_probe -- CacheMuon cached-transform reuse and residual
  * trigger, with the decision kept on the device.
  *

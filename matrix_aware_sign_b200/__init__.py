@@ -77,6 +77,14 @@ def lib() -> ctypes.CDLL:
             "smuon_vote": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int8, c_void_p, c_void_p]),
             "smuon_update": (c_int32, [M, c_int32, M, M, M, c_int32, c_float, c_int8, c_uint32,
                                        POINTER(c_void_p), POINTER(c_void_p), c_void_p]),
+            "smuon_ns_plan_create": (c_int32, [M, M, c_int32, M, c_float, c_float, c_float, c_float, c_int32,
+                                               c_float, c_uint32, M, c_void_p, c_size_t, c_void_p, c_void_p,
+                                               POINTER(c_void_p)]),
+            "smuon_ns_execute": (c_int32, [c_void_p, c_void_p, c_void_p]),
+            "smuon_update_plan_create": (c_int32, [M, c_int32, M, M, M, c_int32, c_float, c_int8, c_uint32,
+                                                   POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p)]),
+            "smuon_update_execute": (c_int32, [c_void_p, c_void_p]),
+            "smuon_plan_destroy": (None, [c_void_p]),
             "cachemuon_workspace_bytes": (c_int32, [M, POINTER(c_size_t)]),
             "cachemuon_reuse_probe": (c_int32, [M, M, M, c_float, c_float, c_void_p, c_void_p, c_void_p,
                                                 c_void_p, c_size_t, c_void_p, c_void_p]),
@@ -173,6 +181,56 @@ def smuon_ns(M_in, U_out, a, b, c, iters, G=None, beta=0.0, eps=1e-7, flags=0, Q
                           _mats(Q_out), _ptr(skip_if), ws.data_ptr(), ws.numel(), _ptr(status),
                           _stream(stream)))
     return ws
+
+
+class NsPlan:
+    """smuon_ns prepared once (plan uploaded into `ws`); run() enqueues only the kernels."""
+
+    def __init__(self, M_in, U_out, a, b, c, iters, G=None, beta=0.0, eps=1e-7, flags=0, Q_out=None, ws=None,
+                 status=None, stream=None):
+        self.tensors = (list(M_in), list(U_out), G, Q_out, status)  # keep the buffers alive
+        if ws is None:
+            ws = workspace(smuon_ns_workspace_bytes(M_in, iters, flags), M_in[0].device)
+        self.ws = ws
+        h = c_void_p()
+        _check(lib().smuon_ns_plan_create(_mats(M_in), _mats(U_out), len(M_in), _mats(G), beta, a, b, c, iters, eps,
+                                          flags, _mats(Q_out), ws.data_ptr(), ws.numel(), _ptr(status),
+                                          _stream(stream), ctypes.byref(h)))
+        self.handle = h
+
+    def run(self, skip_if=None, stream=None):
+        _check(lib().smuon_ns_execute(self.handle, _ptr(skip_if), _stream(stream)))
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h and _lib is not None:
+            _lib.smuon_plan_destroy(h)
+            self.handle = None
+
+
+class UpdatePlan:
+    """smuon_update prepared once; run() enqueues only the kernels."""
+
+    def __init__(self, W, eta, U=None, votes=None, dense=None, M=1, tie_value=0, vote_kind=VOTE_POPCOUNT,
+                 packed_out=None, vote_out=None):
+        Uflat = None if U is None else [u for layer in U for u in layer]
+        self.tensors = (list(W), Uflat, votes, dense, packed_out, vote_out)
+        n = len(W)
+        po = None if packed_out is None else (c_void_p * n)(*[_ptr(p) for p in packed_out])
+        vo = None if vote_out is None else (c_void_p * n)(*[_ptr(v) for v in vote_out])
+        h = c_void_p()
+        _check(lib().smuon_update_plan_create(_mats(W), n, _mats(Uflat), _mats(votes), _mats(dense), M, eta,
+                                              tie_value, vote_kind, po, vo, ctypes.byref(h)))
+        self.handle = h
+
+    def run(self, stream=None):
+        _check(lib().smuon_update_execute(self.handle, _stream(stream)))
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h and _lib is not None:
+            _lib.smuon_plan_destroy(h)
+            self.handle = None
 
 
 # ---------------------------------------------------------------- sign / vote / update

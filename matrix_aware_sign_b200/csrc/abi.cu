@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <memory>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -523,10 +524,21 @@ smuon_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 // enqueue the whole momentum + NS chain for a validated request
-smuon_status enqueue_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t* d_status, const int32_t* skip,
-                        cudaStream_t s) {
+// everything the host needs to launch the kernels of a plan that is already in the workspace
+struct NsExec {
+  PlanHeader h;
   DevInfo di;
-  smuon_status st = device_info(&di);
+  const Plan* d_plan = nullptr;
+  int iters = 1;
+  float c = 0.f;
+  uint32_t flags = 0;
+  double mom_bytes = 0;
+  double sflops[ST_COUNT] = {0};
+};
+
+smuon_status prepare_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t* d_status, cudaStream_t s,
+                        NsExec* ex) {
+  smuon_status st = device_info(&ex->di);
   if (st != SMUON_OK) return st;
   Builder B;
   if ((st = build_plan(rq, nullptr, &B)) != SMUON_OK) return st;
@@ -534,31 +546,52 @@ smuon_status enqueue_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t*
   if ((st = build_plan(rq, reinterpret_cast<char*>(ws), &B)) != SMUON_OK) return st;
   B.h.status = d_status;
   if ((st = upload_plan(B, s)) != SMUON_OK) return st;
-  const Plan* d_plan = reinterpret_cast<const Plan*>(ws);
-  const PlanHeader& h = B.h;
+  ex->h = B.h;
+  ex->d_plan = reinterpret_cast<const Plan*>(ws);
+  ex->iters = rq.iters;
+  ex->c = rq.c;
+  ex->flags = rq.flags;
+  ex->mom_bytes = momentum_bytes(rq, B.h);
+  for (int k = 0; k < ST_COUNT; ++k) ex->sflops[k] = stage_flops(B, k);
+  return SMUON_OK;
+}
+
+smuon_status run_ns(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
+  const PlanHeader& h = ex.h;
+  const DevInfo& di = ex.di;
+  smuon_status st;
   {
     const int grid = std::min(h.total_mom_tiles, di.sms * 8);
     {
-      Launch L("k_momentum", SMUON_WORK_BYTES, momentum_bytes(rq, h), s);
-      k_momentum<<<std::max(grid, 1), 256, 0, s>>>(d_plan, skip);
+      Launch L("k_momentum", SMUON_WORK_BYTES, ex.mom_bytes, s);
+      k_momentum<<<std::max(grid, 1), 256, 0, s>>>(ex.d_plan, skip);
       CUDA_TRY(cudaGetLastError());
     }
     const int warps_per_block = 8;
     Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * h.total_mom_tiles, s);
-    k_norm_finalize<<<(h.n_mats + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(d_plan, skip);
+    k_norm_finalize<<<(h.n_mats + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(ex.d_plan,
+                                                                                                          skip);
     CUDA_TRY(cudaGetLastError());
   }
-  const bool emit_q = (rq.flags & SMUON_NS_EMIT_Q) != 0;
-  for (int k = 0; k < rq.iters; ++k) {
-    if ((st = launch_gemm(d_plan, h, ST_GRAM, k, skip, di, s, stage_flops(B, ST_GRAM))) != SMUON_OK) return st;
-    if (rq.c != 0.f && (st = launch_gemm(d_plan, h, ST_POLY, k, skip, di, s, stage_flops(B, ST_POLY))) != SMUON_OK)
+  const bool emit_q = (ex.flags & SMUON_NS_EMIT_Q) != 0;
+  for (int k = 0; k < ex.iters; ++k) {
+    if ((st = launch_gemm(ex.d_plan, h, ST_GRAM, k, skip, di, s, ex.sflops[ST_GRAM])) != SMUON_OK) return st;
+    if (ex.c != 0.f && (st = launch_gemm(ex.d_plan, h, ST_POLY, k, skip, di, s, ex.sflops[ST_POLY])) != SMUON_OK)
       return st;
-    if ((st = launch_gemm(d_plan, h, ST_AXPY, k, skip, di, s, stage_flops(B, ST_AXPY))) != SMUON_OK) return st;
+    if ((st = launch_gemm(ex.d_plan, h, ST_AXPY, k, skip, di, s, ex.sflops[ST_AXPY])) != SMUON_OK) return st;
     if (emit_q && k >= 1 &&
-        (st = launch_gemm(d_plan, h, ST_QAXPY, k, skip, di, s, stage_flops(B, ST_QAXPY))) != SMUON_OK)
+        (st = launch_gemm(ex.d_plan, h, ST_QAXPY, k, skip, di, s, ex.sflops[ST_QAXPY])) != SMUON_OK)
       return st;
   }
   return SMUON_OK;
+}
+
+smuon_status enqueue_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t* d_status, const int32_t* skip,
+                        cudaStream_t s) {
+  NsExec ex;
+  smuon_status st = prepare_ns(rq, ws, ws_bytes, d_status, s, &ex);
+  if (st != SMUON_OK) return st;
+  return run_ns(ex, skip, s);
 }
 
 // ------------------------------------------------------------------ elementwise tables
@@ -579,9 +612,8 @@ int ew_grid(int64_t chunks, const DevInfo& di) {
 // splits layers into launches of at most kEwMaxLayers layers / kEwMaxSrcs sources
 template <class F>
 smuon_status for_each_ew_launch(const EwBuild& eb, const EwTable& proto, F&& launch) {
-  static EwTable tb;  // large parameter block, launched by value
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lk(mu);
+  std::unique_ptr<EwTable> holder(new EwTable());  // large parameter block, launched by value
+  EwTable& tb = *holder;
   size_t i = 0;
   while (i < eb.layers.size()) {
     tb = proto;
@@ -738,9 +770,21 @@ smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t 
   return SMUON_OK;
 }
 
-smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
-                          const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
-                          uint32_t* const* packed_out, int8_t* const* vote_out, void* stream) {
+}  // extern "C"
+
+namespace {
+
+struct UpdExec {
+  std::vector<EwTable> tables;   // one per launch
+  std::vector<double> bytes;
+  int source = 0;                // 0 = U (fused vote), 1 = votes / dense
+  uint32_t vote_kind = 0;
+  DevInfo di;
+};
+
+smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
+                            const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
+                            uint32_t* const* packed_out, int8_t* const* vote_out, UpdExec* ex) {
   if (!W || n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "W is NULL or n_layers < 1");
   const int nsrc = (U != nullptr) + (votes != nullptr) + (dense != nullptr);
   if (nsrc != 1) return fail(SMUON_ERR_INVALID_ARG, "exactly one of U, votes, dense must be given");
@@ -770,7 +814,8 @@ smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat*
         srcs.push_back(EwSrc{u.data, u.ld});
       }
       if (packed_out && packed_out[l]) {
-        if (reinterpret_cast<uintptr_t>(packed_out[l]) % 16) return fail(SMUON_ERR_INVALID_ARG, "packed_out[%d] must be 16-byte aligned", l);
+        if (reinterpret_cast<uintptr_t>(packed_out[l]) % 16)
+          return fail(SMUON_ERR_INVALID_ARG, "packed_out[%d] must be 16-byte aligned", l);
         L.packed_out = packed_out[l];
       }
       if (vote_out) L.vote_out = vote_out[l];
@@ -786,17 +831,18 @@ smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat*
     eb.layers.push_back(L);
     eb.srcs.push_back(srcs);
   }
-  DevInfo di;
-  smuon_status st = device_info(&di);
+  smuon_status st = device_info(&ex->di);
   if (st != SMUON_OK) return st;
   EwTable proto{};
   proto.M = U ? M : 1;
   proto.tie = tie_value;
   proto.src_dtype = src_dtype;
   proto.eta = eta;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ex->source = U ? 0 : 1;
+  ex->vote_kind = vote_kind;
+  ex->tables.clear();
+  ex->bytes.clear();
   return for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
-    const int grid = ew_grid(tb.total_chunks, di);
     double bytes = 0;
     for (int l = 0; l < tb.n_layers; ++l) {
       const EwLayer& Ly = tb.layers[l];
@@ -804,19 +850,100 @@ smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat*
       if (Ly.packed_out) bytes += (double)Ly.n * tb.M / 8.0;
       if (Ly.vote_out) bytes += (double)Ly.n;
     }
-    if (U) {
-      Launch L(vote_kind == SMUON_VOTE_POPCOUNT ? "k_vote_update_popcount" : "k_vote_update_int8",
-               SMUON_WORK_BYTES, bytes, s);
-      if (vote_kind == SMUON_VOTE_POPCOUNT) k_vote_update_popcount<<<grid, 256, 0, s>>>(tb);
-      else k_vote_update_int8<<<grid, 256, 0, s>>>(tb);
-    } else {
-      Launch L("k_update_src", SMUON_WORK_BYTES, bytes, s);
-      k_update_src<<<grid, 256, 0, s>>>(tb);
-    }
-    CUDA_TRY(cudaGetLastError());
+    ex->tables.push_back(tb);
+    ex->bytes.push_back(bytes);
     return SMUON_OK;
   });
 }
+
+smuon_status run_update(const UpdExec& ex, cudaStream_t s) {
+  for (size_t i = 0; i < ex.tables.size(); ++i) {
+    const EwTable& tb = ex.tables[i];
+    const int grid = ew_grid(tb.total_chunks, ex.di);
+    if (ex.source == 0) {
+      Launch L(ex.vote_kind == SMUON_VOTE_POPCOUNT ? "k_vote_update_popcount" : "k_vote_update_int8",
+               SMUON_WORK_BYTES, ex.bytes[i], s);
+      CUDA_TRY(launch_vote_update(tb, ex.vote_kind == SMUON_VOTE_POPCOUNT, grid, s));
+    } else {
+      Launch L("k_update_src", SMUON_WORK_BYTES, ex.bytes[i], s);
+      k_update_src<<<grid, 256, 0, s>>>(tb);
+    }
+    CUDA_TRY(cudaGetLastError());
+  }
+  return SMUON_OK;
+}
+
+}  // namespace
+
+// plan handles: host objects holding everything needed to relaunch a call
+struct smuon_plan_s {
+  int kind;  // 0 = Newton-Schulz, 1 = update
+  NsExec ns;
+  UpdExec upd;
+};
+
+extern "C" {
+
+smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
+                          const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
+                          uint32_t* const* packed_out, int8_t* const* vote_out, void* stream) {
+  UpdExec ex;
+  smuon_status st = prepare_update(W, n_layers, U, votes, dense, M, eta, tie_value, vote_kind, packed_out, vote_out, &ex);
+  if (st != SMUON_OK) return st;
+  return run_update(ex, reinterpret_cast<cudaStream_t>(stream));
+}
+
+smuon_status smuon_ns_plan_create(const smuon_mat* M_in, const smuon_mat* U_out, int32_t n_mats, const smuon_mat* G,
+                                  float beta, float a, float b, float c, int32_t iters, float eps, uint32_t flags,
+                                  const smuon_mat* Q_out, void* ws, size_t ws_bytes, int32_t* d_status, void* stream,
+                                  smuon_plan* out) {
+  if (!out) return fail(SMUON_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  NsRequest rq{};
+  rq.M_in = M_in; rq.U_out = U_out; rq.n_mats = n_mats; rq.G = G; rq.beta = beta;
+  rq.a = a; rq.b = b; rq.c = c; rq.iters = iters; rq.eps = eps; rq.flags = flags; rq.Q_out = Q_out;
+  smuon_status st = validate_ns(rq);
+  if (st != SMUON_OK) return st;
+  smuon_plan_s* p = new smuon_plan_s();
+  p->kind = 0;
+  st = prepare_ns(rq, ws, ws_bytes, d_status, reinterpret_cast<cudaStream_t>(stream), &p->ns);
+  if (st != SMUON_OK) {
+    delete p;
+    return st;
+  }
+  *out = p;
+  return SMUON_OK;
+}
+
+smuon_status smuon_ns_execute(smuon_plan plan, const int32_t* d_skip_if, void* stream) {
+  if (!plan || plan->kind != 0) return fail(SMUON_ERR_INVALID_ARG, "not a Newton-Schulz plan");
+  return run_ns(plan->ns, d_skip_if, reinterpret_cast<cudaStream_t>(stream));
+}
+
+smuon_status smuon_update_plan_create(const smuon_mat* W, int32_t n_layers, const smuon_mat* U,
+                                      const smuon_mat* votes, const smuon_mat* dense, int32_t M, float eta,
+                                      int8_t tie_value, uint32_t vote_kind, uint32_t* const* packed_out,
+                                      int8_t* const* vote_out, smuon_plan* out) {
+  if (!out) return fail(SMUON_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  smuon_plan_s* p = new smuon_plan_s();
+  p->kind = 1;
+  smuon_status st =
+      prepare_update(W, n_layers, U, votes, dense, M, eta, tie_value, vote_kind, packed_out, vote_out, &p->upd);
+  if (st != SMUON_OK) {
+    delete p;
+    return st;
+  }
+  *out = p;
+  return SMUON_OK;
+}
+
+smuon_status smuon_update_execute(smuon_plan plan, void* stream) {
+  if (!plan || plan->kind != 1) return fail(SMUON_ERR_INVALID_ARG, "not an update plan");
+  return run_update(plan->upd, reinterpret_cast<cudaStream_t>(stream));
+}
+
+void smuon_plan_destroy(smuon_plan plan) { delete plan; }
 
 smuon_status cachemuon_workspace_bytes(const smuon_mat* M_t, size_t* bytes) {
   if (!M_t || !bytes) return fail(SMUON_ERR_INVALID_ARG, "NULL argument");

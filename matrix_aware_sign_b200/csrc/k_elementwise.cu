@@ -267,51 +267,100 @@ __device__ __forceinline__ int8_t threshold(int total, int tie) {
   return (int8_t)(total > 0 ? 1 : (total < 0 ? -1 : tie));
 }
 
+// sign bits (u >= 0: +0, -0 and positives; NaN is not) of 8 consecutive entries
+__device__ __forceinline__ uint32_t pos_bits_bf16(const uint4 w) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  uint32_t r = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t b = (u[k] >> (16 * h)) & 0xffffu;
+      const uint32_t mag = b & 0x7fffu;
+      const bool pos = (mag == 0u) || (!(b & 0x8000u) && mag <= 0x7f80u);
+      r |= (uint32_t)pos << (2 * k + h);
+    }
+  }
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pos_bits_f32(const float* u) {
+  uint32_t r = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) r |= (uint32_t)(u[k] >= 0.f) << k;
+  return r;
+}
+
+// the 8 sign bits of one worker's entries e0..e0+7 (entries past the end -> 0)
+template <bool kBf16>
+__device__ __forceinline__ uint32_t worker_bits(const EwSrc& S, const EwLayer& L, int64_t e0, int32_t dtype) {
+  if (L.vec && e0 + 8 <= L.n) {
+    if (kBf16) return pos_bits_bf16(*reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(S.ptr) + e0));
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(S.ptr) + e0);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(S.ptr) + e0 + 4);
+    const float u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    return pos_bits_f32(u);
+  }
+  uint32_t r = 0;
+  for (int k = 0; k < 8; ++k) {
+    const int64_t e = e0 + k;
+    if (e < L.n) r |= (uint32_t)(load_as_f32(S.ptr, ew_index(L, e, S.ld), dtype) >= 0.f) << k;
+  }
+  return r;
+}
+
+// layer of each lane's chunk: one binary search per warp, then a short forward walk
+__device__ __forceinline__ int warp_layer(const EwTable& tb, int64_t wbase, int64_t chunk, int lane) {
+  int l0 = 0;
+  if (lane == 0) l0 = find_layer(&tb, wbase);
+  l0 = __shfl_sync(0xffffffffu, l0, 0);
+  int l = l0;
+  while (l + 1 < tb.n_layers && tb.layers[l + 1].chunk_begin <= chunk) ++l;
+  return l;
+}
+
 // SignMuon summary, flow steps 2-4 fused: sign (U >= 0), optional packed
-// message, majority vote (sum = 2*popcount - M, or integer sum of +-1), then
-// W <- W - eta*vote in float32, rounded to W's type.
-template <bool kPopcount>
+// message, majority vote (sum = 2*popcount - M over per-entry worker masks, or
+// the integer sum of +-1), then W <- W - eta*vote in float32, rounded to W's
+// type. Work unit: 8 consecutive entries per lane.
+template <bool kPopcount, bool kBf16, typename MaskT>
 __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int M = tb.M;
   for (int64_t wbase = warp_global * 32; wbase < tb.total_chunks; wbase += warps_total * 32) {
     const int64_t chunk = wbase + lane;
     const bool active = chunk < tb.total_chunks;
-    const int li = find_layer(&tb, active ? chunk : tb.total_chunks - 1);
+    const int li = warp_layer(tb, wbase, active ? chunk : tb.total_chunks - 1, lane);
     const EwLayer& L = tb.layers[li];
     const int64_t e0 = (chunk - L.chunk_begin) * 8;
     const bool live = active && e0 < L.n;
-    uint64_t mask[8];
+    float w[8];
+    if (live) load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+    MaskT mask[8];
     int sum[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) { mask[k] = 0; sum[k] = 0; }
-    const int M = tb.M;
-    float w[8];
-    if (live) load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
-    // workers in groups of four: all loads of a group are issued before any use
     for (int wk0 = 0; wk0 < M; wk0 += 4) {
-      float u[4][8];
+      uint32_t bits[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int wk = wk0 + j;
-        if (wk < M && live) load8(tb.srcs[L.src_first + wk].ptr, tb.srcs[L.src_first + wk].ld, tb.src_dtype, L, e0,
-                                  L.vec, u[j]);
+        bits[j] = (wk < M && live) ? worker_bits<kBf16>(tb.srcs[L.src_first + wk], L, e0, tb.src_dtype) : 0u;
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int wk = wk0 + j;
         if (wk >= M) break;  // uniform across the warp
-        uint32_t byte = 0;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const bool pos = live && (e0 + k < L.n) && (u[j][k] >= 0.f);  // NaN -> negative
-          byte |= (uint32_t)pos << k;
-          if (kPopcount) mask[k] |= (uint64_t)pos << wk;
+          const uint32_t pos = (bits[j] >> k) & 1u;
+          if (kPopcount) mask[k] |= (MaskT)pos << wk;
           else sum[k] += pos ? 1 : -1;
         }
         if (tb.any_packed) {  // warp-uniform: every lane takes part in the shuffles
-          const uint32_t word = gather_word(byte, lane);
+          const uint32_t word = gather_word(bits[j], lane);
           if (active && L.packed_out && (lane & 3) == 0)
             L.packed_out[(int64_t)wk * L.words + ((chunk - L.chunk_begin) >> 2)] = word;
         }
@@ -321,30 +370,44 @@ __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
     int8_t v8[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int total = kPopcount ? 2 * __popcll(mask[k]) - M : sum[k];
+      const int cnt = sizeof(MaskT) == 8 ? __popcll((unsigned long long)mask[k]) : __popc((unsigned)mask[k]);
+      const int total = kPopcount ? 2 * cnt - M : sum[k];
       v8[k] = threshold(total, tb.tie);
       w[k] = __fsub_rn(w[k], tb.eta * (float)v8[k]);
     }
     store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
     if (L.vote_out) {
-      if (e0 + 8 <= L.n) {
+      if (e0 + 8 <= L.n && ((reinterpret_cast<uintptr_t>(L.vote_out + e0) & 7) == 0)) {
         uint2 pk;
         memcpy(&pk, v8, 8);
-        if ((reinterpret_cast<uintptr_t>(L.vote_out + e0) & 7) == 0)
-          *reinterpret_cast<uint2*>(L.vote_out + e0) = pk;
-        else
-          for (int k = 0; k < 8; ++k) L.vote_out[e0 + k] = v8[k];
+        *reinterpret_cast<uint2*>(L.vote_out + e0) = pk;
       } else {
         for (int k = 0; k < 8; ++k) if (e0 + k < L.n) L.vote_out[e0 + k] = v8[k];
       }
     }
   }
 }
-__global__ void __launch_bounds__(256) k_vote_update_popcount(const __grid_constant__ EwTable tb) {
-  vote_update_body<true>(tb);
+
+template <bool kPopcount, bool kBf16, typename MaskT>
+__global__ void __launch_bounds__(256) k_vote_update(const __grid_constant__ EwTable tb) {
+  vote_update_body<kPopcount, kBf16, MaskT>(tb);
 }
-__global__ void __launch_bounds__(256) k_vote_update_int8(const __grid_constant__ EwTable tb) {
-  vote_update_body<false>(tb);
+
+cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, cudaStream_t s) {
+  const bool bf = tb.src_dtype == SMUON_BF16;
+  if (popcount) {
+    if (tb.M <= 32) {
+      if (bf) k_vote_update<true, true, uint32_t><<<grid, 256, 0, s>>>(tb);
+      else k_vote_update<true, false, uint32_t><<<grid, 256, 0, s>>>(tb);
+    } else {
+      if (bf) k_vote_update<true, true, uint64_t><<<grid, 256, 0, s>>>(tb);
+      else k_vote_update<true, false, uint64_t><<<grid, 256, 0, s>>>(tb);
+    }
+  } else {
+    if (bf) k_vote_update<false, true, uint32_t><<<grid, 256, 0, s>>>(tb);
+    else k_vote_update<false, false, uint32_t><<<grid, 256, 0, s>>>(tb);
+  }
+  return cudaGetLastError();
 }
 
 // SignMuon summary, flow steps 2-3: signs and the 1-bit message only.
