@@ -67,10 +67,19 @@ __global__ void __launch_bounds__(256) k_momentum(const Plan* plan, const int32_
   __shared__ float red[8];
   const int bf = (h.mode != MODE_SIMT_F32);
   const int split = (h.flags & SMUON_NS_SPLIT_BF16) != 0;
-  for (int t = blockIdx.x; t < h.total_mom_tiles; t += gridDim.x) {
+  const int total = h.total_mom_tiles;
+  float* __restrict__ partials = h.partials;
+  for (int t = blockIdx.x; t < total; t += gridDim.x) {
     const int mi = find_mat_by_mom_tile(h, t);
-    const MatDesc& md = h.mats[mi];
-    const GroupDesc& g = h.groups[md.group];
+    // descriptor fields live in registers: the stores below may not be assumed
+    // to leave global descriptors untouched, so nothing is re-read after them
+    const MatDesc md = h.mats[mi];
+    GroupDesc g;
+    {
+      const GroupDesc& gg = h.groups[md.group];
+      g.m = gg.m; g.count = gg.count; g.ldn = gg.ldn; g.xop[0] = gg.xop[0];
+    }
+    const float beta = h.beta;
     const int local = t - md.mom_begin;
     const int tr = local / md.mom_tiles_c, tc = local - (local / md.mom_tiles_c) * md.mom_tiles_c;
     const int r0 = tr * 64, c0 = tc * 64;
@@ -102,7 +111,7 @@ __global__ void __launch_bounds__(256) k_momentum(const Plan* plan, const int32_
         if (ok[p] && Gp) {
           const float gg[4] = {gv[p].x, gv[p].y, gv[p].z, gv[p].w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) v[k] = fmaf(h.beta, v[k], gg[k]);
+          for (int k = 0; k < 4; ++k) v[k] = fmaf(beta, v[k], gg[k]);
           *reinterpret_cast<float4*>(reinterpret_cast<float*>(md.m_ptr) + (int64_t)r * md.m_ld + c) =
               make_float4(v[0], v[1], v[2], v[3]);
         }
@@ -125,7 +134,7 @@ __global__ void __launch_bounds__(256) k_momentum(const Plan* plan, const int32_
           float mv = load_as_f32(md.m_ptr, idx, md.m_dtype);
           if (md.g_ptr) {
             const float gv = load_as_f32(md.g_ptr, (int64_t)r * md.g_ld + c, md.g_dtype);
-            mv = fmaf(h.beta, mv, gv);
+            mv = fmaf(beta, mv, gv);
             reinterpret_cast<float*>(md.m_ptr)[idx] = mv;
           }
           val = mv;
@@ -153,7 +162,7 @@ __global__ void __launch_bounds__(256) k_momentum(const Plan* plan, const int32_
       float tot = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) tot += red[w];
-      h.partials[t] = tot;
+      partials[t] = tot;
     }
     __syncthreads();
   }
