@@ -135,6 +135,36 @@ smuon_status smuon_ns(const smuon_mat* M_in, const smuon_mat* U_out, int32_t n_m
                       void* ws, size_t ws_bytes, int32_t* d_status, void* stream);
 
 /* ------------------------------------------------------------------------
+ * smuon_ns_static -- smuon_ns without a caller-provided workspace.
+ *
+ * The paper has no counterpart: this is a deployment convenience. It is for
+ * callers that cannot allocate device memory at the point of the call, for
+ * example code running under an external memory budget or allocator that
+ * forbids foreign allocations, or callers that must not enter the CUDA
+ * allocator (which may synchronise the device) in a latency-critical
+ * section. It computes exactly what smuon_ns computes, with the same
+ * arguments minus ws / ws_bytes; its scratch is a fixed array of
+ * SMUON_NS_STATIC_SCRATCH_BYTES in the library's device image, so every GPU
+ * that loads the library holds that memory until the process exits.
+ *  - Batches whose smuon_ns_workspace_bytes() exceeds the array are rejected
+ *    with SMUON_ERR_WORKSPACE before anything is enqueued.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents
+ *    (nothing in it needs to start at zero: every call rewrites what it
+ *    reads). Calls that may overlap on the GPU (other streams, other host
+ *    threads) race on it: serialise them, e.g. on one stream.
+ * ---------------------------------------------------------------------- */
+#define SMUON_NS_STATIC_SCRATCH_BYTES (32u << 20)
+
+smuon_status smuon_ns_static(const smuon_mat* M_in, const smuon_mat* U_out, int32_t n_mats,
+                             const smuon_mat* G, float beta,
+                             float a, float b, float c, int32_t iters, float eps, uint32_t flags,
+                             const smuon_mat* Q_out, const int32_t* d_skip_if,
+                             int32_t* d_status, void* stream);
+
+/* ------------------------------------------------------------------------
  * smuon_sign_pack -- entrywise sign and 1-bit packing of M workers' outputs.
  *
  * SignMuon summary, algorithm flow step 2 (S = sign(U)) and step 3 all-gather

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
             "smuon_vote": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int8, c_void_p, c_void_p]),
             "smuon_update": (c_int32, [M, c_int32, M, M, M, c_int32, c_float, c_int8, c_uint32,
                                        POINTER(c_void_p), POINTER(c_void_p), c_void_p]),
+            "smuon_ns_static": (c_int32, [M, M, c_int32, M, c_float, c_float, c_float, c_float, c_int32, c_float,
+                                          c_uint32, M, c_void_p, c_void_p, c_void_p]),
             "smuon_ns_plan_create": (c_int32, [M, M, c_int32, M, c_float, c_float, c_float, c_float, c_int32,
                                                c_float, c_uint32, M, c_void_p, c_size_t, c_void_p, c_void_p,
                                                POINTER(c_void_p)]),
@@ -181,6 +183,16 @@ def smuon_ns(M_in, U_out, a, b, c, iters, G=None, beta=0.0, eps=1e-7, flags=0, Q
                           _mats(Q_out), _ptr(skip_if), ws.data_ptr(), ws.numel(), _ptr(status),
                           _stream(stream)))
     return ws
+
+
+NS_STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def smuon_ns_static(M_in, U_out, a, b, c, iters, G=None, beta=0.0, eps=1e-7, flags=0, Q_out=None,
+                    skip_if=None, status=None, stream=None):
+    """smuon_ns with the library's fixed device scratch array (no workspace, no allocation)."""
+    _check(lib().smuon_ns_static(_mats(M_in), _mats(U_out), len(M_in), _mats(G), beta, a, b, c, iters, eps, flags,
+                                 _mats(Q_out), _ptr(skip_if), _ptr(status), _stream(stream)))
 
 
 class NsPlan:

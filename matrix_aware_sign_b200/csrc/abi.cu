@@ -1142,3 +1142,55 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
 }
 
 }  // extern "C"
+
+// ======================================================================== no-allocation variant
+// smuon_ns_static runs the same momentum + Newton-Schulz kernels as smuon_ns,
+// but its scratch (plan, norm partials, operand buffers) lives in this
+// file-scope device array instead of a caller-provided workspace. Every GPU
+// that loads the library holds the array until the process exits.
+static __device__ __align__(256) unsigned char g_ns_static_scratch[SMUON_NS_STATIC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_ptr[256] = {nullptr};
+
+// host code must not hand the symbol itself to a kernel: it is a host-side
+// stand-in, so the device address is looked up once per device
+smuon_status static_scratch(void** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 256) return fail(SMUON_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_ns_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(SMUON_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return SMUON_OK;
+}
+}  // namespace
+
+extern "C" smuon_status smuon_ns_static(const smuon_mat* M_in, const smuon_mat* U_out, int32_t n_mats,
+                                        const smuon_mat* G, float beta, float a, float b, float c, int32_t iters,
+                                        float eps, uint32_t flags, const smuon_mat* Q_out, const int32_t* d_skip_if,
+                                        int32_t* d_status, void* stream) {
+  NsRequest rq{};
+  rq.M_in = M_in; rq.U_out = U_out; rq.n_mats = n_mats; rq.G = G; rq.beta = beta;
+  rq.a = a; rq.b = b; rq.c = c; rq.iters = iters; rq.eps = eps; rq.flags = flags; rq.Q_out = Q_out;
+  smuon_status st = validate_ns(rq);
+  if (st != SMUON_OK) return st;
+  Builder B;
+  if ((st = build_plan(rq, nullptr, &B)) != SMUON_OK) return st;
+  if (B.L.total > (size_t)SMUON_NS_STATIC_SCRATCH_BYTES)
+    return fail(SMUON_ERR_WORKSPACE,
+                "this batch needs %zu bytes of scratch; smuon_ns_static holds at most %u bytes (use smuon_ns "
+                "with a workspace)",
+                B.L.total, (unsigned)SMUON_NS_STATIC_SCRATCH_BYTES);
+  void* ws = nullptr;
+  if ((st = static_scratch(&ws)) != SMUON_OK) return st;
+  return enqueue_ns(rq, ws, SMUON_NS_STATIC_SCRATCH_BYTES, d_status, d_skip_if,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
