@@ -45,6 +45,8 @@ def parse_args():
     p.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
     p.add_argument("--e2e-steps", type=int, default=30)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-ns4096", dest="ns4096", action="store_false",
+                   help="skip the extra 4096x4096 Newton-Schulz measurement")
     return p.parse_args()
 
 
@@ -162,6 +164,36 @@ class ClockSampler:
         reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower().startswith("active")})
         return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
                 "reasons": reasons, "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ Newton-Schulz on one large matrix
+def measure_ns_square(S, torch, peaks, n, iters, reps=10):
+    """Five quintic Newton-Schulz steps on one n x n matrix (plain BF16 mode),
+    as in a CacheMuon fresh solve without the transform. Issued and nominal
+    TFLOP/s of the GEMM stages, and the whole call's time."""
+    gen = torch.Generator(device="cuda").manual_seed(4242)
+    M = torch.randn((n, n), device="cuda", generator=gen)
+    U = torch.empty((n, n), dtype=torch.bfloat16, device="cuda")
+    plan = S.NsPlan([M], [U], *WL.QUINTIC, iters)
+    for _ in range(3):
+        plan.run()
+    torch.cuda.synchronize()
+    S.trace_enable(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        plan.run()
+    e1.record()
+    torch.cuda.synchronize()
+    S.trace_enable(False)
+    recs = [r for r in S.trace_read() if r["name"].startswith("k_gemm")]
+    ms_call = e0.elapsed_time(e1) / reps
+    t = sum(r["ms"] for r in recs) / 1e3
+    issued = sum(r["work"] for r in recs) / t / 1e12
+    nominal = sum(r["nominal"] for r in recs) / t / 1e12
+    return {"ms_per_call": ms_call, "gemm_tflops_issued": issued, "gemm_tflops_nominal": nominal,
+            "frac_of_peak": issued / peaks["bf16_tflops_sustained"], "nominal_tflop_per_call": 6 * n ** 3 * iters / 1e12}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -306,9 +338,10 @@ def main():
     peaks, peak_src = load_peaks()
     by = {}
     for r in recs:
-        d = by.setdefault(r["name"], {"ms": 0.0, "work": 0.0, "n": 0, "kind": r["kind"]})
+        d = by.setdefault(r["name"], {"ms": 0.0, "work": 0.0, "nominal": 0.0, "n": 0, "kind": r["kind"]})
         d["ms"] += max(r["ms"], 0.0)
         d["work"] += r["work"]
+        d["nominal"] += r["nominal"]
         d["n"] += 1
     roofline = None
     kernels = {}
@@ -385,9 +418,13 @@ def main():
     summary = {}
     if ns:
         fl = sum(by[k]["work"] for k in ns)
+        nom = sum(by[k]["nominal"] for k in ns)
         t = sum(by[k]["ms"] for k in ns)
         summary["ns_tflops"] = fl / (t / 1e3) / 1e12
+        summary["ns_tflops_nominal"] = nom / (t / 1e3) / 1e12
         summary["ns_frac_of_peak"] = summary["ns_tflops"] / peaks["bf16_tflops_sustained"]
+    if rank == 0 and world == 1 and args.ns4096:
+        summary["ns_4096sq_quintic5"] = measure_ns_square(S, torch, peaks, 4096, 5)
     vk = [k for k in kernels if k.startswith("k_vote_update")]
     if vk:
         summary["vote_gbs"] = kernels[vk[0]]["achieved"]

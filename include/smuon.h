@@ -69,9 +69,10 @@ int32_t     smuon_version(void);              /* (major << 16) | minor */
  * Launch counting and tracing (diagnostics; not part of the method).
  * smuon_launch_count: kernels launched by this library since it was loaded.
  * smuon_trace_enable(1): from then on every launch is bracketed by two CUDA
- * events on its stream and logged with its algorithmic work (flops of the
- * GEMM stages as 2*M*N*K; bytes of the bandwidth-bound kernels as the bytes
- * the method must move). smuon_trace_read synchronises on the logged events,
+ * events on its stream and logged with its work: for the GEMM stages the
+ * flops the tensor cores executed (padded tiles, three products in split
+ * mode) and the method's nominal 2*M*N*K flops; for the bandwidth-bound
+ * kernels the bytes the method must move. smuon_trace_read synchronises on the logged events,
  * copies up to max_recs records (oldest first), clears the log and returns
  * the number copied (with out == NULL: the number logged).
  * ---------------------------------------------------------------------- */
@@ -80,7 +81,8 @@ int32_t     smuon_version(void);              /* (major << 16) | minor */
 typedef struct {
   char    name[40];
   int32_t kind;     /* SMUON_WORK_FLOPS | SMUON_WORK_BYTES */
-  double  work;
+  double  work;     /* flops issued to the tensor (or CUDA) cores, tiles x tile flops; or bytes */
+  double  nominal;  /* the method's nominal flops (2*M*N*K per product); equals work for bytes */
   float   ms;       /* event-timed duration, -1 if unavailable */
 } smuon_trace_rec;
 

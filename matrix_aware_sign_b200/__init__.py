@@ -44,7 +44,8 @@ class CacheMuonCounters(ctypes.Structure):
 
 
 class TraceRec(ctypes.Structure):
-    _fields_ = [("name", ctypes.c_char * 40), ("kind", c_int32), ("work", ctypes.c_double), ("ms", c_float)]
+    _fields_ = [("name", ctypes.c_char * 40), ("kind", c_int32), ("work", ctypes.c_double),
+                ("nominal", ctypes.c_double), ("ms", c_float)]
 
 
 class LionMuonState(ctypes.Structure):
@@ -163,7 +164,7 @@ def trace_read() -> list[dict]:
         return []
     buf = (TraceRec * n)()
     got = lib().smuon_trace_read(buf, n)
-    return [dict(name=r.name.decode(), kind=r.kind, work=r.work, ms=r.ms) for r in buf[:got]]
+    return [dict(name=r.name.decode(), kind=r.kind, work=r.work, nominal=r.nominal, ms=r.ms) for r in buf[:got]]
 
 
 # ---------------------------------------------------------------- smuon_ns

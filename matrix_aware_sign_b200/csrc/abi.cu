@@ -15,7 +15,7 @@
 #include <string>
 #include <vector>
 
-#include "kernels.cuh"
+#include "epilogue.cuh"
 
 using namespace smuon;
 
@@ -47,7 +47,8 @@ smuon_status fail(smuon_status code, const char* fmt, ...) {
 struct TraceRec {
   const char* name;
   int32_t kind;
-  double work;
+  double work;      // issued work (flops the tensor cores executed, or bytes)
+  double nominal;   // the method's nominal count (equal to work for byte counts)
   cudaEvent_t a, b;
 };
 
@@ -61,11 +62,11 @@ struct Launch {
   TraceRec r{};
   bool on = false;
   cudaStream_t s;
-  Launch(const char* name, int32_t kind, double work, cudaStream_t st) : s(st) {
+  Launch(const char* name, int32_t kind, double work, cudaStream_t st, double nominal = -1.0) : s(st) {
     g_launches.fetch_add(1);
     std::lock_guard<std::mutex> lk(g_tr_mu);
     if (!g_tr_on || g_tr.size() >= 1000000) return;
-    r.name = name; r.kind = kind; r.work = work;
+    r.name = name; r.kind = kind; r.work = work; r.nominal = nominal < 0 ? work : nominal;
     if (!g_ev_free.empty()) {
       r.a = g_ev_free.back().first; r.b = g_ev_free.back().second;
       g_ev_free.pop_back();
@@ -228,7 +229,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   const bool tc = (mode == MODE_TC_BF16);
   const bool emit_q = (rq.flags & SMUON_NS_EMIT_Q) && !rq.probe;
   const int K = rq.iters;
-  const int BM = tc ? kTcBM : kSimtBM, BN = tc ? kTcBN : kSimtBN;
+  const int BM = tc ? kTcBM : kSimtBM;
   const size_t esz = bf ? 2 : 4;
   // split BF16: operand buffers hold [hi parts of all matrices][lo parts of all matrices]
   const int parts = (tc && (rq.flags & SMUON_NS_SPLIT_BF16) && !rq.probe) ? 2 : 1;
@@ -287,16 +288,24 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   }
   // momentum tiles must be increasing along mats for the device binary search: they are.
 
-  // tile tables
+  // tile tables: for the symmetric stages the tiles that reach the diagonal or
+  // lie above it (BN = ratio * BM), a full grid of BM x BN tiles otherwise
   int totals[ST_COUNT] = {0};
+  int ratios[ST_COUNT] = {0};
+  for (int st = 0; st < ST_COUNT; ++st) {
+    const int BN = tc ? tc_tile_n(st, rq.flags) : kSimtBN;
+    ratios[st] = BN / BM;
+  }
   for (auto& g : B->groups) {
     const int tmm = ceil_div(g.m, BM);
     for (int st = 0; st < ST_COUNT; ++st) {
+      const bool sym = sym_stage(st);
+      const int BN = BM * ratios[st];
       const int No = (st == ST_AXPY || st == ST_REUSE) ? g.n : g.m;
       g.tiles_m[st] = tmm;
       g.tiles_n[st] = ceil_div(No, BN);
       g.tile_begin[st] = totals[st];
-      totals[st] += g.count * g.tiles_m[st] * g.tiles_n[st];
+      totals[st] += g.count * (sym ? sym_start(tmm, g.tiles_n[st], ratios[st]) : g.tiles_m[st] * g.tiles_n[st]);
     }
   }
 
@@ -311,14 +320,23 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   auto want_map = [&](int32_t& slot) { slot = L.n_tmaps++; };
   L.n_tmaps = 0;
   for (auto& g : B->groups) {
-    for (int i = 0; i < 2; ++i) { g.tm_x_k[i] = g.tm_x_mn[i] = g.tm_q_mn[i] = -1; }
-    g.tm_a_k = g.tm_b_k = g.tm_uq_k = -1;
+    for (int i = 0; i < 2; ++i) { g.tm_x_k[i] = g.tm_x_mn[i] = g.tm_q_mn[i] = g.tm_x_kw[i] = -1; }
+    g.tm_a_k = g.tm_b_k = g.tm_uq_k = g.tm_a_kw = -1;
     if (!tc) continue;
+    const bool wide = tc_tile_n(ST_GRAM, rq.flags) == 256;
     if (!rq.probe) {
       want_map(g.tm_x_k[0]);
       want_map(g.tm_x_mn[0]);
-      if (K >= 2) { want_map(g.tm_x_k[1]); want_map(g.tm_x_mn[1]); }
-      if (rq.c != 0.f) want_map(g.tm_a_k);
+      if (wide) want_map(g.tm_x_kw[0]);
+      if (K >= 2) {
+        want_map(g.tm_x_k[1]);
+        want_map(g.tm_x_mn[1]);
+        if (wide) want_map(g.tm_x_kw[1]);
+      }
+      if (rq.c != 0.f) {
+        want_map(g.tm_a_k);
+        if (wide) want_map(g.tm_a_kw);
+      }
       want_map(g.tm_b_k);
       if (emit_q && K >= 2) want_map(g.tm_q_mn[1]);
       if (emit_q && K >= 3) want_map(g.tm_q_mn[0]);
@@ -326,6 +344,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
       want_map(g.tm_x_mn[0]);
       want_map(g.tm_uq_k);
       want_map(g.tm_x_k[1]);
+      if (wide) want_map(g.tm_x_kw[1]);
     }
   }
   L.off_tmaps = B->take(sizeof(CUtensorMap) * std::max(L.n_tmaps, 1));
@@ -376,8 +395,11 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   h.flags = rq.flags;
   h.a = rq.a; h.b = rq.b; h.c = rq.c; h.eps = rq.eps; h.beta = rq.beta; h.gamma = rq.gamma;
   h.total_mom_tiles = mom_tiles;
-  h.tile_bm = BM; h.tile_bn = BN;
-  for (int st = 0; st < ST_COUNT; ++st) h.total_tiles[st] = totals[st];
+  h.tile_bm = BM; h.tile_bn = tc ? tc_tile_n(ST_AXPY, rq.flags) : kSimtBN;
+  for (int st = 0; st < ST_COUNT; ++st) {
+    h.total_tiles[st] = totals[st];
+    h.sym_ratio[st] = ratios[st];
+  }
   h.partials = B->ptr_at<float>(L.off_partials);
   h.scale = B->ptr_at<float>(L.off_scale);
   h.probe_partials = B->ptr_at<float>(L.off_probe);
@@ -402,7 +424,9 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
       if ((st = enc(g.tm_x_k[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 128)) != SMUON_OK) return st;
       if ((st = enc(g.tm_x_mn[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 64)) != SMUON_OK) return st;
       if ((st = enc(g.tm_q_mn[i], g.qop[i], g.m, g.m, zc, g.ldm, 64, 64)) != SMUON_OK) return st;
+      if ((st = enc(g.tm_x_kw[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 256)) != SMUON_OK) return st;
     }
+    if ((st = enc(g.tm_a_kw, g.aop, g.m, g.m, zc, g.ldm, 64, 256)) != SMUON_OK) return st;
     if ((st = enc(g.tm_a_k, g.aop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
     if ((st = enc(g.tm_b_k, g.bop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
     if (g.tm_uq_k >= 0) {
@@ -453,6 +477,26 @@ double stage_flops(const Builder& B, int st) {
   return f;
 }
 
+// flops the tensor cores (or CUDA cores) actually execute for a stage: tiles
+// x 2 * BM * BN * (K rounded up to the k-block), three products in split mode
+double stage_issued(const Builder& B, int st) {
+  const PlanHeader& h = B.h;
+  const bool tc = h.mode == MODE_TC_BF16;
+  const int BM = tc ? kTcBM : kSimtBM, BK = tc ? 64 : 16;
+  const bool split = tc && (h.flags & SMUON_NS_SPLIT_BF16) && st <= ST_QAXPY;
+  double f = 0;
+  for (const GroupDesc& g : B.groups) {
+    const bool sym = sym_stage(st);
+    const int BN = sym ? BM : (tc ? tc_tile_n(st, h.flags) : kSimtBN);
+    const int T = g.tiles_m[st];
+    const double tiles = (double)g.count * (sym ? T * (T + 1) / 2 : T * g.tiles_n[st]);
+    const int K = (st == ST_GRAM || st == ST_PROBE) ? g.n : g.m;
+    const double kpad = (double)((K + BK - 1) / BK) * BK;
+    f += tiles * 2.0 * BM * BN * kpad;
+  }
+  return split ? 3 * f : f;
+}
+
 // algorithmic bytes of the momentum / normalisation prologue
 double momentum_bytes(const NsRequest& rq, const PlanHeader& h) {
   double b = 0;
@@ -466,17 +510,18 @@ double momentum_bytes(const NsRequest& rq, const PlanHeader& h) {
 }
 
 smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int iter, const int32_t* skip,
-                         const DevInfo& di, cudaStream_t s, double stage_flops) {
+                         const DevInfo& di, cudaStream_t s, double stage_flops, double issued_flops) {
   const int total = h.total_tiles[st];
   if (total == 0) return SMUON_OK;
   static const char* tc_names[2] = {"k_gemm_tc", "k_gemm_tc_split"};
   if (h.mode == MODE_TC_BF16) {
     const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && st <= ST_QAXPY;
-    Launch L(tc_names[split], SMUON_WORK_FLOPS, stage_flops, s);
+    Launch L(tc_names[split], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
     CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
   } else {
     const int grid = std::min(total, di.sms * 6);
-    Launch L(h.mode == MODE_SIMT_F32 ? "k_gemm_simt_f32" : "k_gemm_simt_bf16", SMUON_WORK_FLOPS, stage_flops, s);
+    Launch L(h.mode == MODE_SIMT_F32 ? "k_gemm_simt_f32" : "k_gemm_simt_bf16", SMUON_WORK_FLOPS, issued_flops, s,
+             stage_flops);
     if (h.mode == MODE_SIMT_F32) k_gemm_simt_f32<<<grid, 256, 0, s>>>(d_plan, st, iter, skip);
     else k_gemm_simt_bf16<<<grid, 256, 0, s>>>(d_plan, st, iter, skip);
     CUDA_TRY(cudaGetLastError());
@@ -534,6 +579,7 @@ struct NsExec {
   uint32_t flags = 0;
   double mom_bytes = 0;
   double sflops[ST_COUNT] = {0};
+  double sissued[ST_COUNT] = {0};
 };
 
 smuon_status prepare_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t* d_status, cudaStream_t s,
@@ -552,7 +598,10 @@ smuon_status prepare_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t*
   ex->c = rq.c;
   ex->flags = rq.flags;
   ex->mom_bytes = momentum_bytes(rq, B.h);
-  for (int k = 0; k < ST_COUNT; ++k) ex->sflops[k] = stage_flops(B, k);
+  for (int k = 0; k < ST_COUNT; ++k) {
+    ex->sflops[k] = stage_flops(B, k);
+    ex->sissued[k] = stage_issued(B, k);
+  }
   return SMUON_OK;
 }
 
@@ -575,12 +624,12 @@ smuon_status run_ns(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
   }
   const bool emit_q = (ex.flags & SMUON_NS_EMIT_Q) != 0;
   for (int k = 0; k < ex.iters; ++k) {
-    if ((st = launch_gemm(ex.d_plan, h, ST_GRAM, k, skip, di, s, ex.sflops[ST_GRAM])) != SMUON_OK) return st;
-    if (ex.c != 0.f && (st = launch_gemm(ex.d_plan, h, ST_POLY, k, skip, di, s, ex.sflops[ST_POLY])) != SMUON_OK)
+    if ((st = launch_gemm(ex.d_plan, h, ST_GRAM, k, skip, di, s, ex.sflops[ST_GRAM], ex.sissued[ST_GRAM])) != SMUON_OK) return st;
+    if (ex.c != 0.f && (st = launch_gemm(ex.d_plan, h, ST_POLY, k, skip, di, s, ex.sflops[ST_POLY], ex.sissued[ST_POLY])) != SMUON_OK)
       return st;
-    if ((st = launch_gemm(ex.d_plan, h, ST_AXPY, k, skip, di, s, ex.sflops[ST_AXPY])) != SMUON_OK) return st;
+    if ((st = launch_gemm(ex.d_plan, h, ST_AXPY, k, skip, di, s, ex.sflops[ST_AXPY], ex.sissued[ST_AXPY])) != SMUON_OK) return st;
     if (emit_q && k >= 1 &&
-        (st = launch_gemm(ex.d_plan, h, ST_QAXPY, k, skip, di, s, ex.sflops[ST_QAXPY])) != SMUON_OK)
+        (st = launch_gemm(ex.d_plan, h, ST_QAXPY, k, skip, di, s, ex.sflops[ST_QAXPY], ex.sissued[ST_QAXPY])) != SMUON_OK)
       return st;
   }
   return SMUON_OK;
@@ -671,6 +720,7 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs) {
       strncpy(o.name, r.name, sizeof(o.name) - 1);
       o.kind = r.kind;
       o.work = r.work;
+      o.nominal = r.nominal;
       o.ms = ms;
     }
     ++n;
@@ -1001,8 +1051,12 @@ smuon_status cachemuon_reuse_probe(const smuon_mat* Q, const smuon_mat* M_t, con
     k_norm_finalize<<<1, 32, 0, s>>>(d_plan, nullptr);
     CUDA_TRY(cudaGetLastError());
   }
-  if ((st = launch_gemm(d_plan, B.h, ST_REUSE, 0, nullptr, di, s, stage_flops(B, ST_REUSE))) != SMUON_OK) return st;
-  if ((st = launch_gemm(d_plan, B.h, ST_PROBE, 0, nullptr, di, s, stage_flops(B, ST_PROBE))) != SMUON_OK) return st;
+  if ((st = launch_gemm(d_plan, B.h, ST_REUSE, 0, nullptr, di, s, stage_flops(B, ST_REUSE),
+                        stage_issued(B, ST_REUSE))) != SMUON_OK)
+    return st;
+  if ((st = launch_gemm(d_plan, B.h, ST_PROBE, 0, nullptr, di, s, stage_flops(B, ST_PROBE),
+                        stage_issued(B, ST_PROBE))) != SMUON_OK)
+    return st;
   Launch L("k_probe_finalize", SMUON_WORK_BYTES, 16.0 * B.h.total_tiles[ST_PROBE], s);
   k_probe_finalize<<<1, 32, 0, s>>>(d_plan);
   CUDA_TRY(cudaGetLastError());

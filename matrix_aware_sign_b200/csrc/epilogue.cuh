@@ -22,8 +22,29 @@ struct TileCtx {
   uint32_t flags;
   int32_t bf;                 // operands are bf16 (tcgen05 or SIMT-bf16 mode)
   int32_t split;              // operands are stored as bf16 hi + lo parts
+  int32_t sym;                // symmetric m x m stage (Gram, A^2, probe)
   int64_t xlo, mlo;           // element offset of the lo part of an X (m x n) / m x m buffer
 };
+
+// Gram, A^2 and the probe produce symmetric m x m results. Only tiles that
+// reach the diagonal or lie above it are computed; in them an element
+// (i, j) is written if j >= i and also mirrored to (j, i) if j > i, so every
+// element is written exactly once (deterministically).
+__host__ __device__ inline bool sym_stage(int st) { return st == ST_GRAM || st == ST_POLY || st == ST_PROBE; }
+
+// Tiles are BM x BN with BN = r * BM (r = 1 or 2). Row tm of the tile grid
+// holds the column tiles tn >= floor(tm / r); sym_start(tm) counts the tiles
+// of the rows before tm, sym_start(T) the tiles of one matrix.
+__host__ __device__ inline int sym_start(int tm, int TN, int r) {
+  int f;
+  if (r == 1) {
+    f = tm * (tm - 1) / 2;
+  } else {
+    const int q = tm / 2;
+    f = (tm & 1) ? q * q : q * (q - 1);
+  }
+  return tm * TN - f;
+}
 
 template <int NV>
 __device__ __forceinline__ void st_f32_vec(float* p, const float* v) {
@@ -60,6 +81,17 @@ template <int NV>
 __device__ __forceinline__ void st_op(void* base, int64_t off, int bf, const float* v) {
   if (bf) st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
   else st_f32_vec<NV>(reinterpret_cast<float*>(base) + off, v);
+}
+
+// one operand element (same encodings as st_operand)
+__device__ __forceinline__ void st_operand1(const TileCtx& t, void* base, int64_t off, int64_t lo_off, float v) {
+  if (!t.bf) {
+    reinterpret_cast<float*>(base)[off] = v;
+    return;
+  }
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  reinterpret_cast<__nv_bfloat16*>(base)[off] = hi;
+  if (t.split) reinterpret_cast<__nv_bfloat16*>(base)[off + lo_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
 }
 
 // operand store: f32, bf16, or bf16 hi at off and lo = bf16(v - hi) at off + lo_off
@@ -167,18 +199,76 @@ __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int 
   }
 }
 
-// first cached transform Q_1 = aI + B_0 (CacheMuon fresh solve, reading R14)
+// symmetric-stage stores of a row chunk: elements k >= ds are written in
+// place (vector store when the whole chunk is, the row being padded), and
+// elements k >= ms (strictly above the diagonal) are also written transposed;
+// lanes hold consecutive rows, so each transposed store of a warp is contiguous
 template <int NV>
-__device__ __forceinline__ void emit_q1(const TileCtx& t, int row, int col0, int nvalid, int64_t off,
+__device__ __forceinline__ void sym_store_f32(const TileCtx& t, float* base, int row, int col0, int nvalid,
+                                              int ds, int ms, const float* v) {
+  const int64_t m = t.g->m, ld = t.g->ldm;
+  const int64_t off = ((int64_t)t.z * m + row) * ld + col0;
+  if (ds == 0) {
+    st_f32_vec<NV>(base + off, v);
+  } else {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+      if (k >= ds && k < nvalid) base[off + k] = v[k];
+  }
+  if (!t.sym) return;
+#pragma unroll
+  for (int k = 0; k < NV; ++k)
+    if (k >= ms && k < nvalid) base[((int64_t)t.z * m + col0 + k) * ld + row] = v[k];
+}
+
+template <int NV>
+__device__ __forceinline__ void sym_store_operand(const TileCtx& t, void* base, int row, int col0, int nvalid,
+                                                  int ds, int ms, const float* v) {
+  const int64_t m = t.g->m, ld = t.g->ldm;
+  const int64_t off = ((int64_t)t.z * m + row) * ld + col0;
+  if (ds == 0) {
+    st_operand<NV>(t, base, off, t.mlo, v);
+  } else {
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+      if (k >= ds && k < nvalid) st_operand1(t, base, off + k, t.mlo, v[k]);
+  }
+  if (!t.sym) return;
+#pragma unroll
+  for (int k = 0; k < NV; ++k)
+    if (k >= ms && k < nvalid) st_operand1(t, base, ((int64_t)t.z * m + col0 + k) * ld + row, t.mlo, v[k]);
+}
+
+// largest tm with sym_start(tm) <= r (binary search), then the column tile
+__device__ __forceinline__ void sym_decode(int r, int T, int TN, int ratio, int& tm, int& tn) {
+  int lo = 0, hi = T - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sym_start(mid, TN, ratio) <= r) lo = mid; else hi = mid - 1;
+  }
+  tm = lo;
+  tn = lo / ratio + (r - sym_start(lo, TN, ratio));
+}
+
+// first cached transform Q_1 = aI + B_0 (CacheMuon fresh solve, reading R14);
+// symmetric like B_0, stored with the same triangle rule
+template <int NV>
+__device__ __forceinline__ void emit_q1(const TileCtx& t, int row, int col0, int nvalid, int ds, int ms,
                                         const float* B) {
   float q[NV];
 #pragma unroll
   for (int k = 0; k < NV; ++k) q[k] = B[k] + ((row == col0 + k) ? t.a : 0.f);
-  if (t.iter == t.last) {  // K == 1: Q_1 is the final transform
-    st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, (t.md->vec >> 2) & 1, row, col0, nvalid, q);
+  if (t.iter == t.last) {  // K == 1: Q_1 is the final transform, in the user's bf16 buffer
+    __nv_bfloat16* Q = reinterpret_cast<__nv_bfloat16*>(t.md->q_ptr);
+    const int64_t ld = t.md->q_ld;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      if (k >= ds && k < nvalid) Q[(int64_t)row * ld + col0 + k] = __float2bfloat16_rn(q[k]);
+      if (k >= ms && k < nvalid) Q[(int64_t)(col0 + k) * ld + row] = __float2bfloat16_rn(q[k]);
+    }
   } else {
-    if (t.bf) st_f32_vec<NV>(t.g->qf[1] + off, q);
-    st_operand<NV>(t, t.g->qop[1], off, t.mlo, q);
+    if (t.bf) sym_store_f32<NV>(t, t.g->qf[1], row, col0, nvalid, ds, ms, q);
+    sym_store_operand<NV>(t, t.g->qop[1], row, col0, nvalid, ds, ms, q);
   }
 }
 
@@ -190,31 +280,35 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
   const int nvalid = min(NV, t.No - col0);
   const GroupDesc& g = *t.g;
   const int m = g.m;
+  // symmetric stages: elements k >= ds are on or above the diagonal, k >= ms strictly above
+  const int ds = t.sym ? max(0, row - col0) : 0;
+  const int ms = t.sym ? max(0, row - col0 + 1) : NV;
   switch (t.stage) {
     case ST_GRAM: {
+      if (ds >= nvalid) break;  // the chunk lies below the diagonal
       const float sc = (t.iter == 0 && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s * t.s : 1.f;
-      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
       if (t.c != 0.f) {
 #pragma unroll
         for (int k = 0; k < NV; ++k) v[k] *= sc;
-        st_f32_vec<NV>(g.af + off, v);
-        if (t.bf) st_operand<NV>(t, g.aop, off, t.mlo, v);
+        sym_store_f32<NV>(t, g.af, row, col0, nvalid, ds, ms, v);
+        if (t.bf) sym_store_operand<NV>(t, g.aop, row, col0, nvalid, ds, ms, v);
       } else {
 #pragma unroll
         for (int k = 0; k < NV; ++k) v[k] = t.b * (sc * v[k]);
-        st_operand<NV>(t, g.bop, off, t.mlo, v);
-        if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, off, v);
+        sym_store_operand<NV>(t, g.bop, row, col0, nvalid, ds, ms, v);
+        if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, ds, ms, v);
       }
       break;
     }
     case ST_POLY: {
+      if (ds >= nvalid) break;
       const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
       float A[NV];
       ld_f32_vec<NV>(g.af + off, A);
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] = t.b * A[k] + t.c * v[k];
-      st_operand<NV>(t, g.bop, off, t.mlo, v);
-      if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, off, v);
+      sym_store_operand<NV>(t, g.bop, row, col0, nvalid, ds, ms, v);
+      if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, ds, ms, v);
       break;
     }
     case ST_AXPY: {
@@ -269,9 +363,9 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       float acc = 0.f;
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
-        if (k < nvalid) {
+        if (k >= ds && k < nvalid) {
           const float r = v[k] - ((row == col0 + k) ? 1.f : 0.f);
-          acc = fmaf(r, r, acc);
+          acc = fmaf(k >= ms ? 2.f * r : r, r, acc);  // an element above the diagonal stands for its mirror too
         }
       }
       *probe_acc += acc;
@@ -288,11 +382,19 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
   const int gi = find_group(h, st, tile);
   const GroupDesc& g = h.groups[gi];
   const int local = tile - g.tile_begin[st];
-  const int per = g.tiles_m[st] * g.tiles_n[st];
-  t.z = local / per;
-  const int rem = local - t.z * per;
-  tm = rem / g.tiles_n[st];
-  tn = rem - tm * g.tiles_n[st];
+  if (sym_stage(st)) {
+    const int T = g.tiles_m[st], TN = g.tiles_n[st], ratio = h.sym_ratio[st];
+    const int per = sym_start(T, TN, ratio);
+    t.z = local / per;
+    sym_decode(local - t.z * per, T, TN, ratio, tm, tn);
+  } else {
+    const int per = g.tiles_m[st] * g.tiles_n[st];
+    t.z = local / per;
+    const int rem = local - t.z * per;
+    tm = rem / g.tiles_n[st];
+    tn = rem - tm * g.tiles_n[st];
+  }
+  t.sym = sym_stage(st) ? 1 : 0;
   t.g = &h.groups[gi];
   t.md = &h.mats[g.first_mat + t.z];
   t.stage = st;

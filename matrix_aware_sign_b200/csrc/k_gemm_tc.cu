@@ -19,19 +19,22 @@
 namespace smuon {
 namespace tc {
 
-constexpr int BM = kTcBM, BN = kTcBN, BK = 64;
+constexpr int BM = kTcBM, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x 64 k)
-constexpr int B_BYTES = BN * BK * 2;   // one bf16 tile of B
-constexpr int TMEM_COLS = 2 * BN;
 constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
 
 // plain BF16: one hi tile per operand; split BF16: hi and lo tiles per operand
-// (x = x_hi + x_lo, product ~ A_hi B_hi + A_hi B_lo + A_lo B_hi)
-template <bool kSplit>
+// (x = x_hi + x_lo, product ~ A_hi B_hi + A_hi B_lo + A_lo B_hi).
+// kBN = 128 in split mode, 256 in plain mode (the symmetric stages then use
+// 128 x 256 tiles over the triangle, the others a full grid).
+template <bool kSplit, int kBN>
 struct Cfg {
   static constexpr int PARTS = kSplit ? 2 : 1;
+  static constexpr int BN = kBN;
+  static constexpr int B_BYTES = kBN * BK * 2;
   static constexpr int STAGE_BYTES = PARTS * (A_BYTES + B_BYTES);
-  static constexpr int STAGES = kSplit ? 3 : 6;
+  static constexpr int STAGES = (192 * 1024) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = 2 * kBN;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz
@@ -95,9 +98,9 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
-// instruction descriptor: BF16 x BF16 -> F32, A K-major, B K- or MN-major, 128 x 128
-__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((uint32_t)(BN >> 3) << 17) |
+// instruction descriptor: BF16 x BF16 -> F32, A K-major, B K- or MN-major, 128 x n
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(BM >> 4) << 24);
 }
 
@@ -145,27 +148,71 @@ struct TcOps {
   int b_mn;
 };
 
-__device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, int iter) {
+__device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, int iter, int bn) {
   const GroupDesc& g = *t.g;
   TcOps o;
   o.za = o.zb = t.z;
   o.zlo = g.count;
+  const bool wide = bn == 256;  // K-major B tiles of 256 rows use the {64, 256} boxes
   switch (t.stage) {
-    case ST_GRAM: o.ma = o.mb = &h.tmaps[g.tm_x_k[iter & 1]]; o.K = g.n; o.b_mn = 0; break;
-    case ST_POLY: o.ma = o.mb = &h.tmaps[g.tm_a_k]; o.K = g.m; o.b_mn = 0; break;
+    case ST_GRAM:
+      o.ma = &h.tmaps[g.tm_x_k[iter & 1]];
+      o.mb = &h.tmaps[wide ? g.tm_x_kw[iter & 1] : g.tm_x_k[iter & 1]];
+      o.K = g.n; o.b_mn = 0; break;
+    case ST_POLY:
+      o.ma = &h.tmaps[g.tm_a_k];
+      o.mb = &h.tmaps[wide ? g.tm_a_kw : g.tm_a_k];
+      o.K = g.m; o.b_mn = 0; break;
     case ST_AXPY: o.ma = &h.tmaps[g.tm_b_k]; o.mb = &h.tmaps[g.tm_x_mn[iter & 1]]; o.K = g.m; o.b_mn = 1; break;
     case ST_QAXPY: o.ma = &h.tmaps[g.tm_b_k]; o.mb = &h.tmaps[g.tm_q_mn[iter & 1]]; o.K = g.m; o.b_mn = 1; break;
     case ST_REUSE: o.ma = &h.tmaps[g.tm_uq_k]; o.za = 0; o.mb = &h.tmaps[g.tm_x_mn[0]]; o.K = g.m; o.b_mn = 1; break;
-    default: o.ma = o.mb = &h.tmaps[g.tm_x_k[1]]; o.K = g.n; o.b_mn = 0; break;  // ST_PROBE
+    default:  // ST_PROBE
+      o.ma = &h.tmaps[g.tm_x_k[1]];
+      o.mb = &h.tmaps[wide ? g.tm_x_kw[1] : g.tm_x_k[1]];
+      o.K = g.n; o.b_mn = 0; break;
   }
   return o;
 }
 
-template <bool kSplit>
+// L2 prefetch of the row segments that the B X epilogue will read from its
+// X source (the user's momentum at the first step, the f32 master later),
+// issued by the producer warp while the tile's MMAs are still ahead
+__device__ __forceinline__ void prefetch_rows(const char* base, int64_t row_stride_bytes, int nrows, int bytes,
+                                              int lane) {
+  for (int r = lane; r < nrows; r += 32) {
+    const char* p = base + (int64_t)r * row_stride_bytes;
+    for (int b = 0; b < bytes; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + b));
+  }
+}
+
+template <int kBN>
+__device__ __forceinline__ void prefetch_axpy_source(const TileCtx& t, int tm, int tn, int lane) {
+  if (t.stage != ST_AXPY) return;
+  const int rows = min(BM, t.Mo - tm * BM), cols = min(kBN, t.No - tn * kBN);
+  if (rows <= 0 || cols <= 0) return;
+  if (t.iter == 0 && t.bf) {
+    const MatDesc& md = *t.md;
+    const int es = md.m_dtype == SMUON_F32 ? 4 : (md.m_dtype == SMUON_BF16 ? 2 : 1);
+    const char* p = reinterpret_cast<const char*>(md.m_ptr);
+    if (!md.tall)  // wide: X row i = user row i
+      prefetch_rows(p + ((int64_t)tm * BM * md.m_ld + (int64_t)tn * kBN) * es, md.m_ld * es, rows, cols * es, lane);
+    else           // tall: X column j = user row j
+      prefetch_rows(p + ((int64_t)tn * kBN * md.m_ld + (int64_t)tm * BM) * es, md.m_ld * es, cols, rows * es, lane);
+  } else {
+    const GroupDesc& g = *t.g;
+    const float* src = t.bf ? g.xf[t.iter & 1] : reinterpret_cast<const float*>(g.xop[t.iter & 1]);
+    const char* p = reinterpret_cast<const char*>(src + ((int64_t)t.z * g.m + (int64_t)tm * BM) * g.ldn + (int64_t)tn * kBN);
+    prefetch_rows(p, g.ldn * 4, rows, cols * 4, lane);
+  }
+}
+
+template <bool kSplit, int kBN>
 __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int iter) {
-  constexpr int STAGES = Cfg<kSplit>::STAGES;
-  constexpr int STAGE_BYTES = Cfg<kSplit>::STAGE_BYTES;
-  constexpr int PARTS = Cfg<kSplit>::PARTS;
+  using C = Cfg<kSplit, kBN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int STAGE_BYTES = C::STAGE_BYTES;
+  constexpr int PARTS = C::PARTS;
+  constexpr int B_BYTES = C::B_BYTES;
   const PlanHeader& h = plan->h;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -189,7 +236,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32((const void*)tmem_slot)),
-                 "r"(TMEM_COLS));
+                 "r"(C::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   fence_before();
@@ -199,16 +246,17 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   const int total = h.total_tiles[stage];
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer
-      int s = 0;
-      uint32_t ph = 0;
-      uint32_t armed = 0, last_par = 0;  // per-stage bit sets for the exit drain
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int tm, tn;
-        const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
-        const TcOps o = tc_ops(h, t, iter);
+    // ---------------- TMA producer (lane 0) + L2 prefetch of the epilogue source (all lanes)
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t armed = 0, last_par = 0;  // per-stage bit sets for the exit drain
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      int tm, tn;
+      const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+      prefetch_axpy_source<kBN>(t, tm, tn, lane);
+      if (lane == 0) {
+        const TcOps o = tc_ops(h, t, iter, kBN);
         tensormap_acquire(o.ma);
         tensormap_acquire(o.mb);
         const int nk = (o.K + BK - 1) / BK;
@@ -225,15 +273,18 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
             const uint32_t da = sa + part * A_BYTES, db = sb + part * B_BYTES;
             tma_load_3d(da, o.ma, kb * BK, tm * BM, za, fb);
             if (o.b_mn) {
-              tma_load_3d(db, o.mb, tn * BN, kb * BK, zb, fb);
-              tma_load_3d(db + B_BYTES / 2, o.mb, tn * BN + 64, kb * BK, zb, fb);
+#pragma unroll
+              for (int q = 0; q < kBN / 64; ++q) tma_load_3d(db + q * 8192, o.mb, tn * kBN + 64 * q, kb * BK, zb, fb);
             } else {
-              tma_load_3d(db, o.mb, kb * BK, tn * BN, zb, fb);
+              tma_load_3d(db, o.mb, kb * BK, tn * kBN, zb, fb);
             }
           }
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }
       }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0) {
       if (!ok) {
         *abort_flag = 1;
         if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
@@ -257,11 +308,11 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int tm, tn;
         const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
-        const TcOps o = tc_ops(h, t, iter);
-        const uint32_t idesc = make_idesc((uint32_t)o.b_mn);
+        const TcOps o = tc_ops(h, t, iter, kBN);
+        const uint32_t idesc = make_idesc((uint32_t)o.b_mn, kBN);
         if (!mbar_wait(tempty_bar + 8 * acc, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
         fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
         const int nk = (o.K + BK - 1) / BK;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(full_bar + 8 * s, ph, abort_flag)) { ok = false; break; }
@@ -270,12 +321,12 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_sw128(sa + kk * 32, 16);
-            const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, B_BYTES / 2) : desc_sw128(sb + kk * 32, 16);
+            const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, 8192) : desc_sw128(sb + kk * 32, 16);
             mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
             if constexpr (kSplit) {
               const uint64_t adl = desc_sw128(sa + A_BYTES + kk * 32, 16);
               const uint32_t sbl = sb + B_BYTES;
-              const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, B_BYTES / 2) : desc_sw128(sbl + kk * 32, 16);
+              const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, 8192) : desc_sw128(sbl + kk * 32, 16);
               mma_bf16(d_tmem, ad, bdl, idesc, 1u);   // A_hi * B_lo
               mma_bf16(d_tmem, adl, bd, idesc, 1u);   // A_lo * B_hi
             }
@@ -300,6 +351,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
     // ---------------- epilogue warps 2..9: two warps per TMEM lane group, one per half of the columns
     const int ew = warp & 3;         // TMEM lane group this warp may access
     const int half = (warp - 2) >> 2;
+    constexpr int CH = kBN / 64;     // 32-column chunks per warp
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -314,10 +366,10 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       const int row = tm * BM + ew * 32 + lane;
       float pacc = 0.f;
 #pragma unroll 1
-      for (int ch = half * (BN / 64); ch < (half + 1) * (BN / 64); ++ch) {
+      for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
         float v[32];
-        tmem_ld32(tmem_base + (uint32_t)(acc * BN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
-        epi_chunk<32>(t, row, tn * BN + ch * 32, v, &pacc);
+        tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
+        epi_chunk<32>(t, row, tn * kBN + ch * 32, v, &pacc);
       }
       fence_before();
       mbar_arrive(tempty_bar + 8 * acc);
@@ -332,44 +384,47 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   fence_before();
   __syncthreads();
   fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS));
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
 }
 
+template <bool kSplit, int kBN>
 __global__ void __launch_bounds__(THREADS, 1) k_gemm_tc(const Plan* plan, int stage, int iter, const int32_t* skip) {
   if (skip && *skip) return;
-  gemm_tc_body<false>(plan, stage, iter);
-}
-
-__global__ void __launch_bounds__(THREADS, 1) k_gemm_tc_split(const Plan* plan, int stage, int iter,
-                                                               const int32_t* skip) {
-  if (skip && *skip) return;
-  gemm_tc_body<true>(plan, stage, iter);
+  gemm_tc_body<kSplit, kBN>(plan, stage, iter);
 }
 
 }  // namespace tc
 
-cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter, const int32_t* skip,
-                           int num_sms, cudaStream_t s) {
-  static bool attr_set[64][2] = {};
+template <bool kSplit, int kBN>
+static cudaError_t launch_tc_variant(const Plan* d_plan, int stage, int iter, const int32_t* skip, int grid,
+                                     cudaStream_t s) {
+  static bool attr_set[256] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && stage <= ST_QAXPY;
-  if (dev < 64 && !attr_set[dev][split]) {
-    cudaError_t e = split ? cudaFuncSetAttribute(tc::k_gemm_tc_split, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 tc::Cfg<true>::SMEM_BYTES)
-                          : cudaFuncSetAttribute(tc::k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 tc::Cfg<false>::SMEM_BYTES);
+  if (dev < 256 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc<kSplit, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tc::Cfg<kSplit, kBN>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set[dev][split] = true;
+    attr_set[dev] = true;
   }
+  tc::k_gemm_tc<kSplit, kBN><<<grid, tc::THREADS, tc::Cfg<kSplit, kBN>::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
+  return cudaGetLastError();
+}
+
+int tc_tile_n(int stage, uint32_t flags) {
+  (void)stage;
+  return (flags & SMUON_NS_SPLIT_BF16) ? 128 : 256;  // split mode needs the smem for its lo tiles
+}
+
+cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter, const int32_t* skip,
+                           int num_sms, cudaStream_t s) {
   const int total = h.total_tiles[stage];
   if (total == 0) return cudaSuccess;
   const int grid = total < num_sms ? total : num_sms;
-  if (split)
-    tc::k_gemm_tc_split<<<grid, tc::THREADS, tc::Cfg<true>::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
-  else
-    tc::k_gemm_tc<<<grid, tc::THREADS, tc::Cfg<false>::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
-  return cudaGetLastError();
+  const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && stage <= ST_QAXPY;
+  if (split) return launch_tc_variant<true, 128>(d_plan, stage, iter, skip, grid, s);
+  if (tc_tile_n(stage, h.flags) == 128) return launch_tc_variant<false, 128>(d_plan, stage, iter, skip, grid, s);
+  return launch_tc_variant<false, 256>(d_plan, stage, iter, skip, grid, s);
 }
 
 }  // namespace smuon

@@ -76,7 +76,7 @@ cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, i
                            const int32_t* skip, int num_sms, cudaStream_t s);
 constexpr int kProbeSlots = 8;  // residual partial sums per probe tile (one per epilogue warp)
 constexpr int kTcBM = 128;
-constexpr int kTcBN = 128;
+int tc_tile_n(int stage, uint32_t flags);  // 128 (symmetric stages, split mode) or 256
 constexpr int kSimtBM = 64;
 constexpr int kSimtBN = 64;
 

@@ -69,6 +69,8 @@ struct GroupDesc {
   int32_t tm_a_k, tm_b_k; // A / B K-major box {64,128}
   int32_t tm_q_mn[2];     // Q MN-major box {64,64}
   int32_t tm_uq_k;        // user Q K-major (REUSE A operand)
+  int32_t tm_a_kw;        // A K-major box {64,256} (B operand of 256-wide tiles)
+  int32_t tm_x_kw[2];     // X K-major box {64,256}
   int32_t pad1;
   int32_t tiles_m[ST_COUNT], tiles_n[ST_COUNT], tile_begin[ST_COUNT];
 };
@@ -83,6 +85,7 @@ struct PlanHeader {
   int32_t total_mom_tiles;
   int32_t tile_bm, tile_bn; // tile shape of the GEMM kernel the tables are built for
   int32_t total_tiles[ST_COUNT];
+  int32_t sym_ratio[ST_COUNT];  // BN / BM of the symmetric stages' tiles (1 or 2)
   float* partials;          // [total_mom_tiles] sum of squares per momentum tile
   float* scale;             // [n_mats] s = 1/(||M||_F + eps)
   float* probe_partials;    // [total PROBE tiles]
