@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-ns4096", dest="ns4096", action="store_false",
                    help="skip the extra 4096x4096 Newton-Schulz measurement")
+    p.add_argument("--only-ns4096", action="store_true",
+                   help="run only the 4096x4096 Newton-Schulz measurement (for profiling)")
     return p.parse_args()
 
 
@@ -243,6 +245,10 @@ def main():
     import matrix_aware_sign_b200 as S
 
     torch.cuda.set_device(local)
+    if args.only_ns4096:
+        peaks, _ = load_peaks()
+        print(json.dumps({"ns_4096sq_quintic5": measure_ns_square(S, torch, peaks, 4096, 5, reps=args.steps)}))
+        return
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))

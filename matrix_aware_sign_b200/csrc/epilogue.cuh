@@ -388,11 +388,13 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
     t.z = local / per;
     sym_decode(local - t.z * per, T, TN, ratio, tm, tn);
   } else {
+    // column-major within a matrix: consecutive tiles share the right-hand
+    // operand's column panel (X or Q), which then stays in L2
     const int per = g.tiles_m[st] * g.tiles_n[st];
     t.z = local / per;
     const int rem = local - t.z * per;
-    tm = rem / g.tiles_n[st];
-    tn = rem - tm * g.tiles_n[st];
+    tn = rem / g.tiles_m[st];
+    tm = rem - tn * g.tiles_m[st];
   }
   t.sym = sym_stage(st) ? 1 : 0;
   t.g = &h.groups[gi];

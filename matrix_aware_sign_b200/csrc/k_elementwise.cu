@@ -332,6 +332,73 @@ __device__ __forceinline__ int warp_layer(const EwTable& tb, int64_t wbase, int6
 // message, majority vote (sum = 2*popcount - M over per-entry worker masks, or
 // the integer sum of +-1), then W <- W - eta*vote in float32, rounded to W's
 // type. Work unit: 8 consecutive entries per lane.
+// per 16-bit lane of w: 1 where the bf16 value is >= 0 (+0, -0, positives; not NaN)
+__device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
+  return (__vcmpleu2(w, 0x7f807f80u) | __vcmpeq2(w, 0x80008000u)) & 0x00010001u;
+}
+
+// int8 (integer-sum) vote on bf16 outputs: the count of positive signs of each
+// entry is accumulated two entries per 32-bit add (16-bit lanes), then
+// sum = 2 * count - M (the +-1 sum of the all-reduce variant)
+__device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int M = tb.M;
+  for (int64_t wbase = warp_global * 32; wbase < tb.total_chunks; wbase += warps_total * 32) {
+    const int64_t chunk = wbase + lane;
+    const bool active = chunk < tb.total_chunks;
+    const int li = warp_layer(tb, wbase, active ? chunk : tb.total_chunks - 1, lane);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    if (!(active && e0 < L.n)) continue;
+    float w[8];
+    load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+    uint32_t cnt[4] = {0u, 0u, 0u, 0u};
+    if (L.vec && e0 + 8 <= L.n) {
+      for (int wk0 = 0; wk0 < M; wk0 += 4) {
+        uint4 u[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (wk0 + j < M)
+            u[j] = *reinterpret_cast<const uint4*>(
+                reinterpret_cast<const __nv_bfloat16*>(tb.srcs[L.src_first + wk0 + j].ptr) + e0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (wk0 + j < M) {
+            cnt[0] += pos_halves_bf16(u[j].x);
+            cnt[1] += pos_halves_bf16(u[j].y);
+            cnt[2] += pos_halves_bf16(u[j].z);
+            cnt[3] += pos_halves_bf16(u[j].w);
+          }
+      }
+    } else {
+      for (int wk = 0; wk < M; ++wk) {
+        const uint32_t bits = worker_bits<true>(tb.srcs[L.src_first + wk], L, e0, tb.src_dtype);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cnt[k] += ((bits >> (2 * k)) & 1u) | (((bits >> (2 * k + 1)) & 1u) << 16);
+      }
+    }
+    int8_t v8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = (int)((cnt[k >> 1] >> (16 * (k & 1))) & 0xffffu);
+      v8[k] = threshold(2 * c - M, tb.tie);
+      w[k] = __fsub_rn(w[k], tb.eta * (float)v8[k]);
+    }
+    store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+    if (L.vote_out) {
+      if (e0 + 8 <= L.n && ((reinterpret_cast<uintptr_t>(L.vote_out + e0) & 7) == 0)) {
+        uint2 pk;
+        memcpy(&pk, v8, 8);
+        *reinterpret_cast<uint2*>(L.vote_out + e0) = pk;
+      } else {
+        for (int k = 0; k < 8; ++k) if (e0 + k < L.n) L.vote_out[e0 + k] = v8[k];
+      }
+    }
+  }
+}
+
 template <bool kPopcount, bool kBf16, typename MaskT>
 __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
   const int lane = threadIdx.x & 31;
@@ -402,6 +469,10 @@ __global__ void __launch_bounds__(256) k_vote_update(const __grid_constant__ EwT
   vote_update_body<kPopcount, kBf16, MaskT>(tb);
 }
 
+__global__ void __launch_bounds__(256) k_vote_update_i8_bf16(const __grid_constant__ EwTable tb) {
+  vote_update_int8_bf16(tb);
+}
+
 cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, cudaStream_t s) {
   const bool bf = tb.src_dtype == SMUON_BF16;
   if (popcount) {
@@ -413,7 +484,9 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, cudaS
       else k_vote_update<true, false, uint64_t><<<grid, 256, 0, s>>>(tb);
     }
   } else {
-    if (bf) k_vote_update<false, true, uint32_t><<<grid, 256, 0, s>>>(tb);
+    // the packed-counter kernel needs no packed message (it builds none)
+    if (bf && !tb.any_packed) k_vote_update_i8_bf16<<<grid, 256, 0, s>>>(tb);
+    else if (bf) k_vote_update<false, true, uint32_t><<<grid, 256, 0, s>>>(tb);
     else k_vote_update<false, false, uint32_t><<<grid, 256, 0, s>>>(tb);
   }
   return cudaGetLastError();
