@@ -49,6 +49,9 @@ def parse_args():
                    help="skip the extra 4096x4096 Newton-Schulz measurement")
     p.add_argument("--only-ns4096", action="store_true",
                    help="run only the 4096x4096 Newton-Schulz measurement (for profiling)")
+    p.add_argument("--cachemuon", nargs="*", metavar="RxC:GAMMA",
+                   help="CacheMuon sweep instead of the Sign-Muon step, e.g. 4096x4096:2 8192x8192:15 "
+                        "(no value: the three large shapes x gamma in {2, 15}); --steps sets the schedule length")
     return p.parse_args()
 
 
@@ -198,6 +201,44 @@ def measure_ns_square(S, torch, peaks, n, iters, reps=10):
             "frac_of_peak": issued / peaks["bf16_tflops_sustained"], "nominal_tflop_per_call": 6 * n ** 3 * iters / 1e12}
 
 
+# ------------------------------------------------------------------ CacheMuon sweep
+def run_cachemuon(S, torch, shape, gamma, steps, iters=5):
+    """M_0 ~ N(0,1); M_{t+1} = M_t + 0.01 N(0,1); every step probes the cached
+    transform on the device and runs the fresh solve only when the residual
+    exceeds gamma. Reports the hit rate and the orthogonalisation flops saved
+    against a fresh five-step quintic solve every step (nominal counts: Gram
+    2m^2n, A^2 2m^3, B X 2m^2n per step; Q accumulation 2m^3 for steps 2..K;
+    reuse Q X and probe D D^T 2m^2n each)."""
+    m, n = min(shape), max(shape)
+    gen = torch.Generator(device="cuda").manual_seed(4242)
+    M = torch.randn(shape, device="cuda", generator=gen)
+    D = torch.empty(shape, device="cuda")
+    cm = S.CacheMuon(M, D, gamma, WL.QUINTIC, iters)
+    noise = torch.empty_like(M)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(steps):
+        if t:
+            noise.normal_(generator=gen)
+            M.add_(noise, alpha=0.01)
+        cm.step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    c = cm.counters()
+    f_muon = iters * (4 * m * m * n + 2 * m ** 3)
+    f_q = (iters - 1) * 2 * m ** 3
+    f_probe = 4 * m * m * n
+    fresh = c["misses"]
+    cost = fresh * (f_muon + f_q) + c["probes"] * f_probe
+    return {"workload": "cachemuon", "shape": list(shape), "gamma": gamma, "steps": steps,
+            "hits": c["hits"], "misses": c["misses"], "hit_rate": c["hits"] / steps,
+            "orth_flops_saved_vs_fresh": 1.0 - cost / (steps * f_muon),
+            "ms_per_step": ms / steps, "note": "momentum drift generated on the device inside the timed loop"}
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, rank):
     cfg = WL.SIGN_MUON_WORKLOADS[WORKLOAD]
@@ -245,6 +286,14 @@ def main():
     import matrix_aware_sign_b200 as S
 
     torch.cuda.set_device(local)
+    if args.cachemuon is not None:
+        cases = args.cachemuon or [f"{r}x{c}:{g}" for (r, c) in ((4096, 4096), (8192, 8192), (4096, 16384))
+                                   for g in (2, 15)]
+        for case in cases:
+            shp, gam = case.split(":")
+            r, c = (int(x) for x in shp.split("x"))
+            print(json.dumps(run_cachemuon(S, torch, (r, c), float(gam), args.steps)), flush=True)
+        return
     if args.only_ns4096:
         peaks, _ = load_peaks()
         print(json.dumps({"ns_4096sq_quintic5": measure_ns_square(S, torch, peaks, 4096, 5, reps=args.steps)}))

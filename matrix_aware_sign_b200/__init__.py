@@ -293,6 +293,36 @@ def cachemuon_reuse_probe(Q, M_t, D_hat, gamma, err, accept, counters=None, eps=
     return ws
 
 
+class CacheMuon:
+    """CacheMuon schedule for one matrix, kept on the device: every step probes
+    the cached transform (reuse D_hat = Q X_t, residual, accept flag) and then
+    enqueues the fresh solve, whose kernels return at once when the flag says
+    the cached transform was accepted. The host never waits on the GPU; read
+    counters() at the end."""
+
+    def __init__(self, M_t, D_out, gamma, coeffs, iters, flags=NS_SPLIT_BF16, eps=1e-7):
+        dev = M_t.device
+        m = min(M_t.shape)
+        self.M, self.D, self.gamma, self.eps = M_t, D_out, float(gamma), eps
+        self.Q = torch.zeros((m, m), dtype=torch.bfloat16, device=dev)
+        self.err = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.accept = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.cnt = new_counters(dev)
+        self.ws_probe = workspace(cachemuon_workspace_bytes(M_t), dev)
+        self.fresh = NsPlan([M_t], [D_out], *coeffs, iters, flags=flags | NS_EMIT_Q, Q_out=[self.Q], eps=eps)
+        self.steps = 0
+
+    def step(self, stream=None):
+        cachemuon_reuse_probe(self.Q if self.steps > 0 else None, self.M, self.D, self.gamma, self.err, self.accept,
+                              self.cnt, eps=self.eps, ws=self.ws_probe, stream=stream)
+        self.fresh.run(skip_if=self.accept, stream=stream)
+        self.steps += 1
+
+    def counters(self) -> dict:
+        h, mi, pr, _ = self.cnt.tolist()
+        return {"hits": h, "misses": mi, "probes": pr}
+
+
 # ---------------------------------------------------------------- LionMuon
 class LionMuon:
     """Holds the C lionmuon_state for lists W[layer] and mom[layer][worker]."""
