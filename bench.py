@@ -171,6 +171,30 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
+# ------------------------------------------------------------------ multi-rank host logic
+def rank_seed_base(rank: int) -> int:
+    """Each rank updates its own layer set: its gradient streams are seeded
+    1000 * rank + worker, so no two ranks share a stream."""
+    return 1000 * rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(steps: int, ms_max: float, world: int) -> float:
+    """Whole-job layer-set steps per second: every rank ran `steps` steps of its
+    own layer set within the slowest rank's time."""
+    return world * steps / (ms_max / 1000.0)
+
+
 # ------------------------------------------------------------------ Newton-Schulz on one large matrix
 def measure_ns_square(S, torch, peaks, n, iters, reps=10):
     """Five quintic Newton-Schulz steps on one n x n matrix (plain BF16 mode),
@@ -312,7 +336,7 @@ def main():
     L = len(shapes)
     # --- inputs, resident in HBM (two gradient sets, so consecutive steps read different data)
     W = WL.weights(shapes, cfg.w_init, cfg.w_dtype)
-    streams = WL.GradientStreams(shapes, M, cfg.grad_sigma, seed_base=1000 * rank)
+    streams = WL.GradientStreams(shapes, M, cfg.grad_sigma, seed_base=rank_seed_base(rank))
     gsets = [streams.next_step(), streams.next_step()]
     Wd = [torch.from_numpy(w).cuda() for w in W]
     Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
@@ -379,15 +403,11 @@ def main():
     recs = S.trace_read()
     time.sleep(0.3)
     sampler.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ev0.elapsed_time(ev1), world, device="cuda")
     if graph is not None:
         launches = launches or 8 * args.steps  # graph replays launch the captured kernels
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1000.0)
+    value = job_throughput(args.steps, ms, world)
 
     # --- roofline of the dominant kernel (from the library's event trace)
     peaks, peak_src = load_peaks()
@@ -454,12 +474,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * args.e2e_steps / (ems / 1000.0), "unit": "steps/s",
+        ems = reduce_max(e0.elapsed_time(e1), world, device="cuda")
+        e2e = {"value": job_throughput(args.e2e_steps, ems, world), "unit": "steps/s",
                "h2d_bytes_per_step": g_bytes, "d2h_bytes_per_step": w_bytes}
 
     cpu = None
