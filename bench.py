@@ -442,10 +442,11 @@ def main():
                 with open(tf) as f:
                     tj = json.load(f)
                 ent = tj.get(dom)
-                if ent:
-                    src = os.path.join(ROOT, "matrix_aware_sign_b200", "csrc", ent["source"])
-                    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-                    if h == ent["sha256"]:
+                if ent:  # valid only while the kernel's sources are the ones the counters were taken on
+                    hs = hashlib.sha256()
+                    for f in ent["sources"]:
+                        hs.update(open(os.path.join(ROOT, "matrix_aware_sign_b200", "csrc", f), "rb").read())
+                    if hs.hexdigest() == ent["sha256"]:
                         traffic = ent["bytes_per_launch"]
             except Exception:
                 traffic = None

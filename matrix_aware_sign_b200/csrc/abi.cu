@@ -913,7 +913,7 @@ smuon_status run_update(const UpdExec& ex, cudaStream_t s) {
     if (ex.source == 0) {
       Launch L(ex.vote_kind == SMUON_VOTE_POPCOUNT ? "k_vote_update_popcount" : "k_vote_update_int8",
                SMUON_WORK_BYTES, ex.bytes[i], s);
-      CUDA_TRY(launch_vote_update(tb, ex.vote_kind == SMUON_VOTE_POPCOUNT, grid, s));
+      CUDA_TRY(launch_vote_update(tb, ex.vote_kind == SMUON_VOTE_POPCOUNT, grid, ex.di.sms, s));
     } else {
       Launch L("k_update_src", SMUON_WORK_BYTES, ex.bytes[i], s);
       k_update_src<<<grid, 256, 0, s>>>(tb);

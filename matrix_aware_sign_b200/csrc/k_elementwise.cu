@@ -10,6 +10,8 @@
 //  * k_lion_sign       LionMuon sign step (G_hat, vote, W and EMA update)
 //  * k_lion_mean       LionMuon Muon-step prologue (mean of G_hat, EMA update)
 //  * k_probe_finalize  CacheMuon residual, accept flag and counters
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace smuon {
@@ -339,61 +341,87 @@ __device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
 
 // int8 (integer-sum) vote on bf16 outputs: the count of positive signs of each
 // entry is accumulated two entries per 32-bit add (16-bit lanes), then
-// sum = 2 * count - M (the +-1 sum of the all-reduce variant)
+// sum = 2 * count - M (the +-1 sum of the all-reduce variant). Each lane takes
+// two consecutive 8-entry chunks (16 entries, 16-byte loads per worker); layer
+// chunk ranges are multiples of 16 chunks, so a pair never straddles layers.
+__device__ __forceinline__ void vote_i8_finish16(const EwTable& tb, const EwLayer& L, int64_t e0,
+                                                 const uint32_t* cnt, float* w) {
+  int8_t v8[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int c = (int)((cnt[k >> 1] >> (16 * (k & 1))) & 0xffffu);
+    v8[k] = threshold(2 * c - tb.M, tb.tie);
+    w[k] = __fsub_rn(w[k], tb.eta * (float)v8[k]);
+  }
+  store8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+  store8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
+  if (L.vote_out) {
+    int8_t* dst = L.vote_out + e0;
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      uint4 pk;
+      memcpy(&pk, v8, 16);
+      *reinterpret_cast<uint4*>(dst) = pk;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) dst[k] = v8[k];
+    }
+  }
+}
+
 __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int M = tb.M;
-  for (int64_t wbase = warp_global * 32; wbase < tb.total_chunks; wbase += warps_total * 32) {
-    const int64_t chunk = wbase + lane;
+  for (int64_t wbase = warp_global * 64; wbase < tb.total_chunks; wbase += warps_total * 64) {
+    const int64_t chunk = wbase + 2 * lane;
     const bool active = chunk < tb.total_chunks;
     const int li = warp_layer(tb, wbase, active ? chunk : tb.total_chunks - 1, lane);
     const EwLayer& L = tb.layers[li];
     const int64_t e0 = (chunk - L.chunk_begin) * 8;
     if (!(active && e0 < L.n)) continue;
-    float w[8];
-    load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
-    uint32_t cnt[4] = {0u, 0u, 0u, 0u};
-    if (L.vec && e0 + 8 <= L.n) {
+    if (L.vec && e0 + 16 <= L.n) {
+      float w[16];
+      uint32_t cnt[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+      load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
       for (int wk0 = 0; wk0 < M; wk0 += 4) {
-        uint4 u[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (wk0 + j < M)
-            u[j] = *reinterpret_cast<const uint4*>(
-                reinterpret_cast<const __nv_bfloat16*>(tb.srcs[L.src_first + wk0 + j].ptr) + e0);
+        uint4 u[4][2];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (wk0 + j < M) {
-            cnt[0] += pos_halves_bf16(u[j].x);
-            cnt[1] += pos_halves_bf16(u[j].y);
-            cnt[2] += pos_halves_bf16(u[j].z);
-            cnt[3] += pos_halves_bf16(u[j].w);
+            const uint4* p = reinterpret_cast<const uint4*>(
+                reinterpret_cast<const __nv_bfloat16*>(tb.srcs[L.src_first + wk0 + j].ptr) + e0);
+            u[j][0] = p[0];
+            u[j][1] = p[1];
+          }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (wk0 + j < M) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              cnt[4 * hh + 0] += pos_halves_bf16(u[j][hh].x);
+              cnt[4 * hh + 1] += pos_halves_bf16(u[j][hh].y);
+              cnt[4 * hh + 2] += pos_halves_bf16(u[j][hh].z);
+              cnt[4 * hh + 3] += pos_halves_bf16(u[j][hh].w);
+            }
           }
       }
+      vote_i8_finish16(tb, L, e0, cnt, w);
     } else {
-      for (int wk = 0; wk < M; ++wk) {
-        const uint32_t bits = worker_bits<true>(tb.srcs[L.src_first + wk], L, e0, tb.src_dtype);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) cnt[k] += ((bits >> (2 * k)) & 1u) | (((bits >> (2 * k + 1)) & 1u) << 16);
-      }
-    }
-    int8_t v8[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int c = (int)((cnt[k >> 1] >> (16 * (k & 1))) & 0xffffu);
-      v8[k] = threshold(2 * c - M, tb.tie);
-      w[k] = __fsub_rn(w[k], tb.eta * (float)v8[k]);
-    }
-    store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
-    if (L.vote_out) {
-      if (e0 + 8 <= L.n && ((reinterpret_cast<uintptr_t>(L.vote_out + e0) & 7) == 0)) {
-        uint2 pk;
-        memcpy(&pk, v8, 8);
-        *reinterpret_cast<uint2*>(L.vote_out + e0) = pk;
-      } else {
-        for (int k = 0; k < 8; ++k) if (e0 + k < L.n) L.vote_out[e0 + k] = v8[k];
+      // ragged or strided layers: entry by entry
+      const int nent = (int)min((int64_t)16, L.n - e0);
+      for (int k = 0; k < nent; ++k) {
+        const int64_t e = e0 + k;
+        int c = 0;
+        for (int wk = 0; wk < M; ++wk) {
+          const EwSrc& S = tb.srcs[L.src_first + wk];
+          c += load_as_f32(S.ptr, ew_index(L, e, S.ld), SMUON_BF16) >= 0.f ? 1 : 0;
+        }
+        const int8_t v = threshold(2 * c - M, tb.tie);
+        const int64_t wi = ew_index(L, e, L.w_ld);
+        store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+        if (L.vote_out) L.vote_out[e] = v;
       }
     }
   }
@@ -473,7 +501,7 @@ __global__ void __launch_bounds__(256) k_vote_update_i8_bf16(const __grid_consta
   vote_update_int8_bf16(tb);
 }
 
-cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, cudaStream_t s) {
+cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s) {
   const bool bf = tb.src_dtype == SMUON_BF16;
   if (popcount) {
     if (tb.M <= 32) {
@@ -485,7 +513,11 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, cudaS
     }
   } else {
     // the packed-counter kernel needs no packed message (it builds none)
-    if (bf && !tb.any_packed) k_vote_update_i8_bf16<<<grid, 256, 0, s>>>(tb);
+    if (bf && !tb.any_packed) {
+      // 16 entries per lane; measured best with 2-4 resident CTAs per SM
+      const int64_t want = (tb.total_chunks + 511) / 512;
+      k_vote_update_i8_bf16<<<(int)std::max<int64_t>(1, std::min<int64_t>(want, 4 * sms)), 256, 0, s>>>(tb);
+    }
     else if (bf) k_vote_update<false, true, uint32_t><<<grid, 256, 0, s>>>(tb);
     else k_vote_update<false, false, uint32_t><<<grid, 256, 0, s>>>(tb);
   }

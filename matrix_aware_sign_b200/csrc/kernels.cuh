@@ -57,7 +57,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
 __global__ void k_plan_upload(const __grid_constant__ UploadChunk c);
 __global__ void k_momentum(const Plan* plan, const int32_t* skip);
 __global__ void k_norm_finalize(const Plan* plan, const int32_t* skip);
-cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, cudaStream_t s);
+cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s);
 __global__ void k_sign_pack(const __grid_constant__ EwTable tb, uint32_t* packed, int8_t* signs);
 __global__ void k_vote(const uint32_t* packed, const int8_t* signs, int M, int64_t N, int64_t words,
                        int tie, int8_t* vote);
