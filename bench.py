@@ -43,6 +43,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
+    p.add_argument("--no-graph-compare", dest="graph_compare", action="store_false",
+                   help="skip the extra CUDA-graph replay measurement")
     p.add_argument("--e2e-steps", type=int, default=30)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-ns4096", dest="ns4096", action="store_false",
@@ -455,6 +457,29 @@ def main():
                     else peaks["hbm_gbs"], "unit": kd["unit"], "frac": kd["frac"], "traffic": traffic,
                     "peak_source": f"{peak_src} ({'bf16 sustained' if kd['unit'] == 'TFLOP/s' else 'HBM copy'})"}
 
+    # --- the same step replayed as a CUDA graph (launch overhead removed), reported beside `value`
+    graph_value = None
+    if graph is None and args.graph_compare and world == 1:
+        g2 = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+        side = torch.cuda.Stream()
+        with torch.cuda.stream(side):
+            for j in range(2):
+                with torch.cuda.graph(g2[j], stream=side):
+                    step(j)
+        torch.cuda.synchronize()
+        for j in range(4):
+            g2[j & 1].replay()
+        torch.cuda.synchronize()
+        q0 = torch.cuda.Event(enable_timing=True)
+        q1 = torch.cuda.Event(enable_timing=True)
+        q0.record(stream)
+        for i in range(args.steps):
+            g2[i & 1].replay()
+        q1.record(stream)
+        torch.cuda.synchronize()
+        graph_value = args.steps / (q0.elapsed_time(q1) / 1000.0)
+        del g2
+
     # --- end to end through the public API with host buffers
     e2e = None
     if args.e2e_steps > 0:
@@ -514,7 +539,8 @@ def main():
                        "global_batch": None, "seq_len": None, "parallelism": f"replicas x{world}",
                        "launch": "cuda_graph" if graph is not None else "eager",
                        "l2": "inputs larger than L2: 375 MB of gradients per step, two resident sets alternate"},
-            "roofline": roofline, "kernels": kernels, **summary, "clocks": clocks, "e2e": e2e,
+            "roofline": roofline, "kernels": kernels, **summary, "steps_per_s_cuda_graph": graph_value,
+            "clocks": clocks, "e2e": e2e,
             "gpu_launches": launches, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -189,7 +189,7 @@ struct NsRequest {
 struct Layout {
   size_t plan_bytes = 0, total = 0;
   size_t off_groups = 0, off_mats = 0, off_tmaps = 0;
-  size_t off_partials = 0, off_scale = 0, off_probe = 0;
+  size_t off_partials = 0, off_scale = 0, off_probe = 0, off_mom_begin = 0;
   int n_tmaps = 0;
 };
 
@@ -316,6 +316,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   (void)hdr;
   L.off_groups = B->take(sizeof(GroupDesc) * B->groups.size());
   L.off_mats = B->take(sizeof(MatDesc) * B->mats.size());
+  L.off_mom_begin = B->take(sizeof(int32_t) * (B->mats.size() + 1));
   // tensor maps: count them first
   auto want_map = [&](int32_t& slot) { slot = L.n_tmaps++; };
   L.n_tmaps = 0;
@@ -403,6 +404,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   h.partials = B->ptr_at<float>(L.off_partials);
   h.scale = B->ptr_at<float>(L.off_scale);
   h.probe_partials = B->ptr_at<float>(L.off_probe);
+  h.mom_begin = B->ptr_at<int32_t>(L.off_mom_begin);
   h.groups = B->ptr_at<GroupDesc>(L.off_groups);
   h.mats = B->ptr_at<MatDesc>(L.off_mats);
   h.tmaps = B->ptr_at<CUtensorMap>(L.off_tmaps);
@@ -444,6 +446,12 @@ smuon_status upload_plan(Builder& B, cudaStream_t s) {
   memcpy(bytes.data(), &p, sizeof(Plan));
   memcpy(bytes.data() + B.L.off_groups, B.groups.data(), sizeof(GroupDesc) * B.groups.size());
   memcpy(bytes.data() + B.L.off_mats, B.mats.data(), sizeof(MatDesc) * B.mats.size());
+  {
+    std::vector<int32_t> mb(B.mats.size() + 1);
+    for (size_t i = 0; i < B.mats.size(); ++i) mb[i] = B.mats[i].mom_begin;
+    mb[B.mats.size()] = B.h.total_mom_tiles;
+    memcpy(bytes.data() + B.L.off_mom_begin, mb.data(), sizeof(int32_t) * mb.size());
+  }
   if (B.L.n_tmaps > 0) memcpy(bytes.data() + B.L.off_tmaps, B.maps.data(), sizeof(CUtensorMap) * B.L.n_tmaps);
   static UploadChunk chunk;  // large parameter block; filled then launched by value
   static std::mutex mu;

@@ -89,6 +89,7 @@ struct PlanHeader {
   float* partials;          // [total_mom_tiles] sum of squares per momentum tile
   float* scale;             // [n_mats] s = 1/(||M||_F + eps)
   float* probe_partials;    // [total PROBE tiles]
+  const int32_t* mom_begin; // [n_mats + 1] first momentum tile of each matrix (compact, for the tile search)
   GroupDesc* groups;        // device pointers into the plan region
   MatDesc* mats;
   CUtensorMap* tmaps;
@@ -124,12 +125,14 @@ __device__ inline int find_group(const PlanHeader& h, int st, int tile) {
   return g;
 }
 
-// locate the matrix owning a momentum tile (binary search over mats)
+// locate the matrix owning a momentum tile (binary search over a compact
+// array of first tiles, which stays in L1 across the tiles of a CTA)
 __device__ inline int find_mat_by_mom_tile(const PlanHeader& h, int tile) {
+  const int32_t* __restrict__ b = h.mom_begin;
   int lo = 0, hi = h.n_mats - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
-    if (h.mats[mid].mom_begin <= tile) lo = mid; else hi = mid - 1;
+    if (__ldg(b + mid) <= tile) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
