@@ -387,3 +387,89 @@ def test_lionmuon_period_schedule():
                 d_ref = (W[l].astype(np.float64) - Wprev[l]) / -eta
                 assert rel_fro(d_gpu, d_ref) < 1e-2
     assert opt.t == 2
+
+
+# ------------------------------------------------------------------ more layouts and modes
+@pytest.mark.parametrize("shape", [(96, 200), (200, 96)])
+@pytest.mark.parametrize("flags", [0, S.NS_SPLIT_BF16, S.NS_FP32_REF])
+def test_ns_strided_user_matrices(shape, flags):
+    """Momentum, gradient and output with leading dimensions larger than the
+    width (scalar user I/O paths), wide and tall."""
+    rng = np.random.default_rng(shape[0])
+    M0 = rng.standard_normal(shape).astype(np.float32)
+    G = rng.standard_normal(shape).astype(np.float32)
+    r, c = shape
+    Mbig = torch.zeros((r, c + 13), device="cuda")
+    Gbig = torch.zeros((r, c + 7), device="cuda")
+    Ubig = torch.full((r, c + 5), 9.0, device="cuda")
+    Mbig[:, :c] = dev(M0)
+    Gbig[:, :c] = dev(G)
+    K = 1 if flags == 0 else 2  # plain BF16 is used (and meets the criteria) with one quintic step
+    S.smuon_ns([Mbig[:, :c]], [Ubig[:, :c]], *WL.QUINTIC, K, G=[Gbig[:, :c]], beta=0.9, flags=flags)
+    torch.cuda.synchronize()
+    Mref = O.momentum(M0, G, 0.9)
+    np.testing.assert_allclose(host(Mbig[:, :c]), Mref, rtol=2e-6, atol=1e-6)
+    assert torch.all(Mbig[:, c:] == 0) and torch.all(Ubig[:, c:] == 9.0)
+    tol = 1e-4 if flags == S.NS_FP32_REF else 1e-2
+    check_ns_outputs([(host(Ubig[:, :c]), O.newton_schulz(Mref, *WL.QUINTIC, K))], tol)
+
+
+def test_ns_bf16_input_f32_output():
+    rng = np.random.default_rng(4)
+    M = WL._to_bf16_values(rng.standard_normal((130, 384)).astype(np.float32))
+    Md = dev(M, torch.bfloat16)
+    Ud = torch.zeros((130, 384), device="cuda")
+    S.smuon_ns([Md], [Ud], *WL.CUBIC, 5)
+    torch.cuda.synchronize()
+    check_ns_outputs([(host(Ud), O.newton_schulz(M.astype(np.float64), *WL.CUBIC, 5))], 1e-2)
+
+
+@pytest.mark.parametrize("iters", [1, 2, 3])
+@pytest.mark.parametrize("flags", [S.NS_SPLIT_BF16, S.NS_FP32_REF])
+def test_emit_q_iteration_counts(iters, flags):
+    """The cached transform after K = 1, 2, 3 steps (Q_1 from the first
+    epilogue, then Q <- aQ + BQ) against the oracle's product of multipliers."""
+    rng = np.random.default_rng(iters)
+    for shape in [(160, 300), (300, 160)]:
+        M = rng.standard_normal(shape).astype(np.float32)
+        m = min(shape)
+        Ud = torch.zeros(shape, device="cuda")
+        Qd = torch.zeros((m, m), dtype=torch.bfloat16, device="cuda")
+        S.smuon_ns([dev(M)], [Ud], *WL.QUINTIC, iters, flags=flags | S.NS_EMIT_Q, Q_out=[Qd])
+        torch.cuda.synchronize()
+        D_ref, Q_ref = O.newton_schulz_with_q(M, *WL.QUINTIC, iters)
+        assert rel_fro(host(Qd), Q_ref) < 1e-2
+        check_ns_outputs([(host(Ud), D_ref)], 1e-2 if flags != S.NS_FP32_REF else 1e-4)
+
+
+@pytest.mark.parametrize("kind", [S.VOTE_POPCOUNT, S.VOTE_INT8])
+def test_fused_vote_update_64_workers_and_f32_outputs(kind):
+    shapes = [(33, 70), (128, 128)]
+    M = 64
+    W = WL.weights(shapes, "normal002", "f32")
+    Wd = [dev(w) for w in W]
+    U = [WL.synthetic_polar_outputs(s, M, seed=40 + i, dtype="f32", zero_fraction=0.03) for i, s in enumerate(shapes)]
+    Ud = [[dev(u) for u in layer] for layer in U]
+    votes = [torch.zeros(r * c, dtype=torch.int8, device="cuda") for r, c in shapes]
+    S.smuon_update(Wd, 0.01, U=Ud, M=M, vote_kind=kind, vote_out=votes)
+    torch.cuda.synchronize()
+    for i, s in enumerate(shapes):
+        v = O.vote_from_signs([O.sign_extract(u) for u in U[i]])
+        np.testing.assert_array_equal(host(votes[i]).reshape(s), v)
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, 0.01, "f32"))
+
+
+def test_nan_outputs_vote_negative():
+    """A NaN in a worker's output counts as a negative sign (u >= 0 is false)."""
+    M, shape = 3, (8, 40)
+    U = WL.synthetic_polar_outputs(shape, M, seed=7, dtype="f32")
+    U[0][2, 5] = np.nan
+    U[1][2, 5] = np.nan
+    U[2][2, 5] = 1.0
+    W = np.zeros(shape, np.float32)
+    Wd = [dev(W)]
+    S.smuon_update(Wd, 0.5, U=[[dev(u) for u in U]], M=M)
+    torch.cuda.synchronize()
+    v = O.vote_from_signs([O.sign_extract(u) for u in U])
+    assert v[2, 5] == -1
+    np.testing.assert_array_equal(host(Wd[0]), O.update_with_vote(W, v, 0.5, "f32"))
