@@ -219,11 +219,15 @@ def measure_ns_square(S, torch, peaks, n, iters, reps=10):
     torch.cuda.synchronize()
     S.trace_enable(False)
     recs = [r for r in S.trace_read() if r["name"].startswith("k_gemm")]
+    stage_ms = {}
+    for r in recs:
+        stage_ms[r["name"]] = stage_ms.get(r["name"], 0.0) + r["ms"] / reps
     ms_call = e0.elapsed_time(e1) / reps
     t = sum(r["ms"] for r in recs) / 1e3
     issued = sum(r["work"] for r in recs) / t / 1e12
     nominal = sum(r["nominal"] for r in recs) / t / 1e12
-    return {"ms_per_call": ms_call, "gemm_tflops_issued": issued, "gemm_tflops_nominal": nominal,
+    return {"ms_per_call": ms_call, "gemm_ms_per_call_by_stage": stage_ms,
+            "gemm_tflops_issued": issued, "gemm_tflops_nominal": nominal,
             "frac_of_peak": issued / peaks["bf16_tflops_sustained"], "nominal_tflop_per_call": 6 * n ** 3 * iters / 1e12}
 
 
@@ -413,13 +417,15 @@ def main():
 
     # --- roofline of the dominant kernel (from the library's event trace)
     peaks, peak_src = load_peaks()
-    by = {}
+    by, stages = {}, {}
     for r in recs:
-        d = by.setdefault(r["name"], {"ms": 0.0, "work": 0.0, "nominal": 0.0, "n": 0, "kind": r["kind"]})
-        d["ms"] += max(r["ms"], 0.0)
-        d["work"] += r["work"]
-        d["nominal"] += r["nominal"]
-        d["n"] += 1
+        kname = r["name"].split(".")[0]  # stage-qualified names ("k_gemm_tc.axpy") roll up into their kernel
+        for key, table in ((kname, by), (r["name"], stages)):
+            d = table.setdefault(key, {"ms": 0.0, "work": 0.0, "nominal": 0.0, "n": 0, "kind": r["kind"]})
+            d["ms"] += max(r["ms"], 0.0)
+            d["work"] += r["work"]
+            d["nominal"] += r["nominal"]
+            d["n"] += 1
     roofline = None
     kernels = {}
     total_ms = sum(d["ms"] for d in by.values()) or 1.0
@@ -433,6 +439,9 @@ def main():
             unit, peak = "GB/s", peaks["hbm_gbs"]
         kernels[name] = {"launches": d["n"], "share": d["ms"] / total_ms, "ms_per_launch": per_launch_ms,
                          "achieved": ach, "unit": unit, "frac": ach / peak}
+    stage_detail = {k: {"launches": d["n"], "ms_per_launch": d["ms"] / max(d["n"], 1),
+                        "tflops_issued": d["work"] / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0}
+                    for k, d in stages.items() if "." in k}
     if by:
         dom = max(by, key=lambda k: by[k]["ms"])
         kd = kernels[dom]
@@ -539,7 +548,8 @@ def main():
                        "global_batch": None, "seq_len": None, "parallelism": f"replicas x{world}",
                        "launch": "cuda_graph" if graph is not None else "eager",
                        "l2": "inputs larger than L2: 375 MB of gradients per step, two resident sets alternate"},
-            "roofline": roofline, "kernels": kernels, **summary, "steps_per_s_cuda_graph": graph_value,
+            "roofline": roofline, "kernels": kernels, "gemm_stages": stage_detail, **summary,
+            "steps_per_s_cuda_graph": graph_value,
             "clocks": clocks, "e2e": e2e,
             "gpu_launches": launches, "cpu_baseline": cpu,
         }

@@ -521,10 +521,14 @@ smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int it
                          const DevInfo& di, cudaStream_t s, double stage_flops, double issued_flops) {
   const int total = h.total_tiles[st];
   if (total == 0) return SMUON_OK;
-  static const char* tc_names[2] = {"k_gemm_tc", "k_gemm_tc_split"};
+  // trace names: kernel, then the stage after a dot
+  static const char* tc_names[2][ST_COUNT] = {
+      {"k_gemm_tc.gram", "k_gemm_tc.poly", "k_gemm_tc.axpy", "k_gemm_tc.qaxpy", "k_gemm_tc.reuse", "k_gemm_tc.probe"},
+      {"k_gemm_tc_split.gram", "k_gemm_tc_split.poly", "k_gemm_tc_split.axpy", "k_gemm_tc_split.qaxpy",
+       "k_gemm_tc_split.reuse", "k_gemm_tc_split.probe"}};
   if (h.mode == MODE_TC_BF16) {
     const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && st <= ST_QAXPY;
-    Launch L(tc_names[split], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
+    Launch L(tc_names[split][st], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
     CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
   } else {
     const int grid = std::min(total, di.sms * 6);

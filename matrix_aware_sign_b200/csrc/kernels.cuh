@@ -16,7 +16,7 @@ struct alignas(16) UploadChunk {
 
 // ---- elementwise tables (sign / vote / update / Lion), carried in kernel parameters
 constexpr int kEwMaxLayers = 64;
-constexpr int kEwMaxSrcs = 1024;
+constexpr int kEwMaxSrcs = 256;  // keeps the parameter block near 10 KB (launch cost grows with it)
 
 struct EwSrc {
   const void* ptr;
