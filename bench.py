@@ -7,6 +7,12 @@ M = 4 simulated workers: momentum update + Frobenius normalisation + one
 quintic Newton-Schulz step per worker and layer (212 matrices, tcgen05), then
 the fused sign / int8-sum vote / update of the 53 weight matrices.
 
+`--workload c3_gpt2s` times the GPT-2-small set instead (48 matrices, M = 8,
+five quintic steps, 1-bit packed popcount vote, optionally the local polar
+step); `--workload c5_gpt2l` times the LionMuon schedule on the GPT-2-Large
+set (144 matrices, M = 16, P = 4: a step is one step of the schedule, averaged
+over whole periods when --steps is a multiple of 4).
+
 Prints one JSON line (rank 0). `value` is layer-set steps per second over all
 ranks (each rank updates its own layer set: weak scaling, no data-path
 collective). `--impl reference` times the CPU oracle on the same workload.
@@ -51,6 +57,16 @@ def parse_args():
                    help="skip the extra 4096x4096 Newton-Schulz measurement")
     p.add_argument("--only-ns4096", action="store_true",
                    help="run only the 4096x4096 Newton-Schulz measurement (for profiling)")
+    p.add_argument("--workload", choices=["c2_resnet50", "c3_gpt2s", "c5_gpt2l"], default=WORKLOAD,
+                   help="layer set: ResNet-50 Sign-Muon (default), GPT-2-small Sign-Muon (M=8, popcount vote, "
+                        "5 quintic steps), GPT-2-Large LionMuon (M=16, P=4)")
+    p.add_argument("--ns-mode", choices=["plain", "split"], default=None,
+                   help="Newton-Schulz operand precision (default: plain for one quintic step, split BF16 for "
+                        "five, the mode that meets the 1e-2 tolerance there)")
+    p.add_argument("--layers", type=int, default=0,
+                   help="use only the first LAYERS matrices of the set (a smaller case for profiler captures)")
+    p.add_argument("--local-polar", action="store_true",
+                   help="GPT-2-small set: orthogonalise the voted matrix before the update")
     p.add_argument("--cachemuon", nargs="*", metavar="RxC:GAMMA",
                    help="CacheMuon sweep instead of the Sign-Muon step, e.g. 4096x4096:2 8192x8192:15 "
                         "(no value: the three large shapes x gamma in {2, 15}); --steps sets the schedule length")
@@ -269,35 +285,288 @@ def run_cachemuon(S, torch, shape, gamma, steps, iters=5):
             "ms_per_step": ms / steps, "note": "momentum drift generated on the device inside the timed loop"}
 
 
+# ------------------------------------------------------------------ oracle timing of the other layer sets
+_LION_INPUTS = {}
+
+
+def time_oracle_lion(cfg, budget_s):
+    """Oracle steps/s of the LionMuon schedule, from two bounded samples on one
+    transformer block (the blocks are identical): a sign step on the first rows
+    of the block's four matrices (elementwise: scaled by the entries), and a
+    Muon step on a square slice of the 1280 x 1280 matrix (scaled by the
+    Newton-Schulz flops of the block). Period time = (P-1) sign steps + one
+    Muon step."""
+    import oracle as O
+    block = cfg.shapes[:4]
+    n_blocks = len(cfg.shapes) // 4
+    if cfg.name not in _LION_INPUTS:
+        rng = np.random.default_rng(7)
+        W = WL.weights(block, "normal002", cfg.w_dtype)
+        G = [[rng.standard_normal(s, dtype=np.float32) for _ in range(cfg.workers)] for s in block]
+        _LION_INPUTS[cfg.name] = (W, G)
+    W, G = _LION_INPUTS[cfg.name]
+    args = (cfg.period, cfg.beta1, cfg.beta2, cfg.eta, cfg.coeffs, cfg.iters, cfg.w_dtype, cfg.tie_value)
+
+    def timed(t, Ws, Gs):
+        Ms = [[np.zeros(w.shape, np.float32) for _ in range(cfg.workers)] for w in Ws]
+        t0 = time.perf_counter()
+        O.lionmuon_step(t, Ws, Ms, Gs, *args)
+        return time.perf_counter() - t0
+
+    def sign_sample(rows):
+        return timed(1, [w[:rows] for w in W], [[g[:rows] for g in gl] for gl in G])
+
+    probe = sign_sample(16)
+    rows = int(min(1280, max(16, 16 * 0.5 * budget_s / max(probe, 1e-6))))
+    t_rows = sign_sample(rows)
+    frac = sum(min(rows, r) * c for r, c in block) / sum(r * c for r, c in block)
+    t_sign = t_rows / frac
+    side = 1280 if budget_s >= 4.0 else 320
+    t_sq = timed(cfg.period, [W[1][:side, :side]], [[g[:side, :side] for g in G[1]]])
+    ns = lambda m, n: 4 * m * m * n + 2 * m ** 3
+    t_muon = t_sq * sum(ns(min(r, c), max(r, c)) for r, c in block) / ns(side, side)
+    period = (cfg.period - 1) * t_sign + t_muon
+    return cfg.period / (period * n_blocks), rows, side, probe + t_rows + t_sq
+
+
+def oracle_rate(name, budget_s):
+    """(steps/s of the oracle, sample description) for a layer set."""
+    if name in WL.LION_MUON_WORKLOADS:
+        cfg = WL.LION_MUON_WORKLOADS[name]
+        v, rows, side, used = time_oracle_lion(cfg, budget_s)
+        return v, (f"one transformer block x {cfg.workers} workers: a sign step on the first {rows} rows, a Muon "
+                   f"step on a {side}x{side} slice ({used:.1f} s); period = {cfg.period - 1} sign + 1 Muon, "
+                   f"scaled by entries and NS flops to the {len(cfg.shapes) // 4} identical blocks")
+    cfg = WL.SIGN_MUON_WORKLOADS[name]
+    v, ids, share, used = time_oracle(cfg, budget_s)
+    return v, (f"{len(ids)} largest of {len(cfg.shapes)} layers x {cfg.workers} workers ({100 * share:.1f}% of "
+               f"the NS flops, {used:.1f} s), scaled to the full layer set")
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, rank):
-    cfg = WL.SIGN_MUON_WORKLOADS[WORKLOAD]
     if rank != 0:
         return
+    desc = describe(args.workload, default_ns_mode(args), args.local_polar)
     budget = max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        time_oracle(cfg, budget)
+        oracle_rate(args.workload, budget)
     vals = []
-    info = None
+    sample = None
     for _ in range(args.steps):
-        v, ids, share, used = time_oracle(cfg, budget)
+        v, sample = oracle_rate(args.workload, budget)
         vals.append(v)
-        info = (ids, share, used)
     value = float(np.median(vals))
     cores = blas_threads()
     line = {
         "impl": "reference", "metric": "Muon steps/s per layer set", "value": value, "unit": "steps/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded Gaussian gradients, He-normal weights)",
-        "config": {"workload": "resnet50_conv_set_53_layers_M4_quintic1_int8_vote", "global_batch": None,
-                   "seq_len": None, "parallelism": "cpu"},
-        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
-                         "sample": f"per step: {len(info[0])} largest layers x 4 workers "
-                                   f"({100 * info[1]:.1f}% of the NS flops), scaled to the full set"},
+        "data": "synthetic (seeded Gaussian gradients and weights of the same distributions, drawn on the host)",
+        "config": {"workload": desc["workload"], "global_batch": None, "seq_len": None, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the layer sets
+def default_ns_mode(args):
+    if args.ns_mode:
+        return args.ns_mode
+    return "plain" if args.workload == "c2_resnet50" else "split"
+
+
+def describe(name, ns_mode, local_polar):
+    if name == "c2_resnet50":
+        return {"workload": "resnet50_conv_set_53_layers_M4_quintic1_int8_vote",
+                "data": "synthetic (seeded Gaussian gradients N(0,1e-4), He-normal weights)"}
+    if name == "c3_gpt2s":
+        return {"workload": "gpt2_small_set_48_matrices_M8_quintic5_popcount_vote"
+                            + ("_local_polar" if local_polar else "") + f"_{ns_mode}_bf16",
+                "data": "synthetic (seeded Gaussian gradients N(0,1) drawn on the device, weights N(0,0.02^2) bf16)"}
+    return {"workload": f"gpt2_large_set_144_matrices_M16_lionmuon_P4_quintic5_{ns_mode}_bf16",
+            "data": "synthetic (seeded Gaussian gradients N(0,1) drawn on the device, weights N(0,0.02^2) bf16)"}
+
+
+def subset(shapes, layers):
+    return shapes[:layers] if layers > 0 else shapes
+
+
+def setup_c2(S, torch, rank, ns_flags, e2e, layers=0):
+    """ResNet-50 layer set, M = 4: momentum + one quintic NS step (prepared
+    plans on two resident gradient sets) + fused sign / int8-sum vote / update."""
+    cfg = WL.SIGN_MUON_WORKLOADS["c2_resnet50"]
+    M, shapes = cfg.workers, subset(cfg.shapes, layers)
+    L = len(shapes)
+    W = WL.weights(shapes, cfg.w_init, cfg.w_dtype)
+    streams = WL.GradientStreams(shapes, M, cfg.grad_sigma, seed_base=rank_seed_base(rank))
+    gsets = [streams.next_step(), streams.next_step()]
+    Wd = [torch.from_numpy(w).cuda() for w in W]
+    Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
+    Ud = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in shapes for _ in range(M)]
+    Gd = [[torch.from_numpy(g).cuda() for layer in gs for g in layer] for gs in gsets]
+    Ul = [Ud[l * M:(l + 1) * M] for l in range(L)]
+    nbytes = S.smuon_ns_workspace_bytes(Md, cfg.iters, ns_flags)
+    wss = [S.workspace(nbytes), S.workspace(nbytes)]
+    ws_e2e = S.workspace(nbytes) if e2e else None
+    ns_plans = [S.NsPlan(Md, Ud, *cfg.coeffs, cfg.iters, G=Gd[j], beta=cfg.beta, flags=ns_flags, ws=wss[j])
+                for j in range(2)]
+    upd_plan = S.UpdatePlan(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
+    n_params = sum(r * c for r, c in shapes)
+
+    def step(i, G=None):
+        if G is None:
+            ns_plans[i & 1].run()
+            upd_plan.run()
+        else:  # end to end: the one-shot public calls (own workspace, the plans keep theirs)
+            S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G, beta=cfg.beta, flags=ns_flags, ws=ws_e2e)
+            S.smuon_update(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
+
+    def e2e_io():
+        hostG = [[torch.from_numpy(g).pin_memory() for layer in gs for g in layer] for gs in gsets]
+        hostW = [torch.empty(w.shape, dtype=torch.float32).pin_memory() for w in W]
+        return hostG, [torch.empty_like(g) for g in Gd[0]], hostW, Wd
+
+    return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None,
+            "g_bytes": n_params * M * 4, "w_bytes": n_params * 4,
+            "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters, "vote": "int8 sum",
+                       "l2": "inputs larger than L2: 375 MB of gradients per step, two resident sets alternate"}}
+
+
+def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0):
+    """GPT-2-small layer set, M = 8: momentum + five quintic NS steps (prepared
+    plans on two resident gradient sets), then either the fused sign / 1-bit
+    pack / popcount vote / update with the packed payload written out, or
+    (local polar step) sign-pack + popcount vote, NS on the 48 voted matrices
+    and the dense update."""
+    cfg = WL.SIGN_MUON_WORKLOADS["c3_gpt2s"]
+    M, shapes = cfg.workers, subset(cfg.shapes, layers)
+    L = len(shapes)
+    Wd = [torch.from_numpy(w).to(torch.bfloat16).cuda() for w in WL.weights(shapes, cfg.w_init, cfg.w_dtype)]
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed_base(rank) + 3)
+    Gd = [[torch.randn(s, device="cuda", generator=gen) * cfg.grad_sigma for s in shapes for _ in range(M)]
+          for _ in range(2)]
+    Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
+    Ud = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in shapes for _ in range(M)]
+    Ul = [Ud[l * M:(l + 1) * M] for l in range(L)]
+    nbytes = S.smuon_ns_workspace_bytes(Md, cfg.iters, ns_flags)
+    wss = [S.workspace(nbytes), S.workspace(nbytes)]
+    ns_plans = [S.NsPlan(Md, Ud, *cfg.coeffs, cfg.iters, G=Gd[j], beta=cfg.beta, flags=ns_flags, ws=wss[j])
+                for j in range(2)]
+    packed = [torch.zeros((M, S.packed_words(r * c)), dtype=torch.int32, device="cuda") for r, c in shapes]
+    if not local_polar:
+        upd = S.UpdatePlan(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_POPCOUNT,
+                           packed_out=packed)
+
+        def tail():
+            upd.run()
+    else:
+        votes = [torch.zeros(s, dtype=torch.int8, device="cuda") for s in shapes]
+        dirs = [torch.zeros(s, device="cuda") for s in shapes]
+        polar = S.NsPlan(votes, dirs, *cfg.coeffs, cfg.iters, flags=ns_flags)
+        upd = S.UpdatePlan(Wd, cfg.eta, dense=dirs)
+
+        def tail():
+            for l, (r, c) in enumerate(shapes):
+                S.smuon_sign_pack(Ul[l], packed=packed[l])
+                S.smuon_vote(M, r * c, votes[l], packed=packed[l], tie_value=cfg.tie_value)
+            polar.run()
+            upd.run()
+    n_params = sum(r * c for r, c in shapes)
+    ws_e2e = S.workspace(nbytes) if e2e else None
+
+    def step(i, G=None):
+        if G is None:
+            ns_plans[i & 1].run()
+        else:
+            S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G, beta=cfg.beta, flags=ns_flags, ws=ws_e2e)
+        tail()
+
+    def e2e_io():
+        hostG = [[g.cpu().pin_memory() for g in Gd[0]]]
+        hostW = [torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for w in Wd]
+        return hostG, [torch.empty_like(g) for g in Gd[0]], hostW, Wd
+
+    return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None,
+            "g_bytes": n_params * M * 4, "w_bytes": n_params * 2,
+            "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters,
+                       "vote": "1-bit packed, popcount" + (", local polar step" if local_polar else ""),
+                       "l2": "inputs larger than L2: 2.7 GB of gradients per step, two resident sets alternate"}}
+
+
+def setup_c5(S, torch, rank, ns_flags, layers=0):
+    """GPT-2-Large LionMuon, M = 16, P = 4: three sign steps (vote of the
+    workers' sign(G_hat)) and one Muon step (NS of the worker mean) per period.
+    One resident gradient set (45 GB, far larger than L2)."""
+    cfg = WL.LION_MUON_WORKLOADS["c5_gpt2l"]
+    M, shapes = cfg.workers, subset(cfg.shapes, layers)
+    n_params = sum(r * c for r, c in shapes)
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed_base(rank) + 5)
+    Wd = [(torch.randn(s, device="cuda", generator=gen) * 0.02).to(torch.bfloat16) for s in shapes]
+    mom = [[torch.zeros(s, device="cuda") for _ in range(M)] for s in shapes]
+    G = [[torch.randn(s, device="cuda", generator=gen) for _ in range(M)] for s in shapes]
+    opt = S.LionMuon(Wd, mom)
+    ws = S.workspace(opt.workspace_bytes(cfg.iters, ns_flags))
+
+    def step(i, G_=None):
+        S.lionmuon_step(opt, G, cfg.period, cfg.beta1, cfg.beta2, cfg.eta, *cfg.coeffs, cfg.iters,
+                        tie_value=cfg.tie_value, ns_flags=ns_flags, ws=ws)
+
+    return {"step": step, "graphable": False, "e2e_io": None, "g_bytes": n_params * M * 4, "w_bytes": n_params * 2,
+            "period": cfg.period,
+            "config": {"layers": len(shapes), "params": n_params, "workers": M, "ns_iters": cfg.iters,
+                       "period": cfg.period, "vote": "1-bit majority on sign steps",
+                       "l2": "inputs larger than L2: 45 GB of gradients and 45 GB of EMA per step"}}
+
+
+def rollup(S, recs, peaks):
+    """Per-kernel time, work and roofline fraction from the library's trace."""
+    by, stages = {}, {}
+    for r in recs:
+        kname = r["name"].split(".")[0]  # stage-qualified names ("k_gemm_tc.axpy") roll up into their kernel
+        for key, table in ((kname, by), (r["name"], stages)):
+            d = table.setdefault(key, {"ms": 0.0, "work": 0.0, "nominal": 0.0, "n": 0, "kind": r["kind"]})
+            d["ms"] += max(r["ms"], 0.0)
+            d["work"] += r["work"]
+            d["nominal"] += r["nominal"]
+            d["n"] += 1
+    kernels = {}
+    total_ms = sum(d["ms"] for d in by.values()) or 1.0
+    for name, d in by.items():
+        per_launch_ms = d["ms"] / max(d["n"], 1)
+        if d["kind"] == S.WORK_FLOPS:
+            ach = d["work"] / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0
+            unit, peak = "TFLOP/s", peaks["bf16_tflops_sustained"]
+        else:
+            ach = d["work"] / (d["ms"] / 1e3) / 1e9 if d["ms"] > 0 else 0.0
+            unit, peak = "GB/s", peaks["hbm_gbs"]
+        kernels[name] = {"launches": d["n"], "share": d["ms"] / total_ms, "ms_per_launch": per_launch_ms,
+                         "achieved": ach, "unit": unit, "frac": ach / peak}
+    stage_detail = {k: {"launches": d["n"], "ms_per_launch": d["ms"] / max(d["n"], 1),
+                        "tflops_issued": d["work"] / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0}
+                    for k, d in stages.items() if "." in k}
+    return by, kernels, stage_detail
+
+
+def load_traffic(dom):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, valid
+    only while the kernel's sources are the ones the counters were taken on."""
+    tf = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(tf):
+        return None
+    try:
+        import hashlib
+        with open(tf) as f:
+            ent = json.load(f).get(dom)
+        if not ent:
+            return None
+        hs = hashlib.sha256()
+        for f in ent["sources"]:
+            hs.update(open(os.path.join(ROOT, "matrix_aware_sign_b200", "csrc", f), "rb").read())
+        return ent["bytes_per_launch"] if hs.hexdigest() == ent["sha256"] else None
+    except Exception:
+        return None
 
 
 # ------------------------------------------------------------------ our arm
@@ -336,37 +605,17 @@ def main():
         if world > 1:
             dist.barrier()
 
-    cfg = WL.SIGN_MUON_WORKLOADS[WORKLOAD]
-    M = cfg.workers
-    shapes = cfg.shapes
-    L = len(shapes)
-    # --- inputs, resident in HBM (two gradient sets, so consecutive steps read different data)
-    W = WL.weights(shapes, cfg.w_init, cfg.w_dtype)
-    streams = WL.GradientStreams(shapes, M, cfg.grad_sigma, seed_base=rank_seed_base(rank))
-    gsets = [streams.next_step(), streams.next_step()]
-    Wd = [torch.from_numpy(w).cuda() for w in W]
-    Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
-    Ud = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in shapes for _ in range(M)]
-    Gd = [[torch.from_numpy(g).cuda() for layer in gs for g in layer] for gs in gsets]
-    Ul = [Ud[l * M:(l + 1) * M] for l in range(L)]
-    ws = S.workspace(S.smuon_ns_workspace_bytes(Md, cfg.iters, 0))
-    n_params = sum(r * c for r, c in shapes)
-    g_bytes = n_params * M * 4
-    w_bytes = n_params * 4
-
-    # prepared calls (plan handles): each plan's descriptors are uploaded once into its workspace
-    ws2 = S.workspace(ws.numel())
-    ws_e2e = S.workspace(ws.numel()) if args.e2e_steps > 0 else None
-    ns_plans = [S.NsPlan(Md, Ud, *cfg.coeffs, cfg.iters, G=Gd[j], beta=cfg.beta, ws=[ws, ws2][j]) for j in range(2)]
-    upd_plan = S.UpdatePlan(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
-
-    def step(i, G=None):
-        if G is None:
-            ns_plans[i & 1].run()
-            upd_plan.run()
-        else:  # end to end: the one-shot public calls (own workspace, the plans keep theirs)
-            S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G, beta=cfg.beta, ws=ws_e2e)
-            S.smuon_update(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
+    ns_mode = default_ns_mode(args)
+    ns_flags = S.NS_SPLIT_BF16 if ns_mode == "split" else 0
+    desc = describe(args.workload, ns_mode, args.local_polar)
+    e2e_on = args.e2e_steps > 0
+    if args.workload == "c2_resnet50":
+        wl = setup_c2(S, torch, rank, ns_flags, e2e_on, args.layers)
+    elif args.workload == "c3_gpt2s":
+        wl = setup_c3(S, torch, rank, ns_flags, e2e_on, args.local_polar, args.layers)
+    else:
+        wl = setup_c5(S, torch, rank, ns_flags, args.layers)
+    step = wl["step"]
 
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
@@ -374,7 +623,7 @@ def main():
     torch.cuda.synchronize()
 
     graph = None
-    if args.graph:
+    if args.graph and wl["graphable"]:
         graph = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
         side = torch.cuda.Stream()
         with torch.cuda.stream(side):
@@ -387,7 +636,7 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    S.trace_enable(not args.graph)
+    S.trace_enable(graph is None)
     n0 = S.launch_count()
     barrier()
     torch.cuda.synchronize()
@@ -417,58 +666,19 @@ def main():
 
     # --- roofline of the dominant kernel (from the library's event trace)
     peaks, peak_src = load_peaks()
-    by, stages = {}, {}
-    for r in recs:
-        kname = r["name"].split(".")[0]  # stage-qualified names ("k_gemm_tc.axpy") roll up into their kernel
-        for key, table in ((kname, by), (r["name"], stages)):
-            d = table.setdefault(key, {"ms": 0.0, "work": 0.0, "nominal": 0.0, "n": 0, "kind": r["kind"]})
-            d["ms"] += max(r["ms"], 0.0)
-            d["work"] += r["work"]
-            d["nominal"] += r["nominal"]
-            d["n"] += 1
+    by, kernels, stage_detail = rollup(S, recs, peaks)
     roofline = None
-    kernels = {}
-    total_ms = sum(d["ms"] for d in by.values()) or 1.0
-    for name, d in by.items():
-        per_launch_ms = d["ms"] / max(d["n"], 1)
-        if d["kind"] == S.WORK_FLOPS:
-            ach = d["work"] / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0
-            unit, peak = "TFLOP/s", peaks["bf16_tflops_sustained"]
-        else:
-            ach = d["work"] / (d["ms"] / 1e3) / 1e9 if d["ms"] > 0 else 0.0
-            unit, peak = "GB/s", peaks["hbm_gbs"]
-        kernels[name] = {"launches": d["n"], "share": d["ms"] / total_ms, "ms_per_launch": per_launch_ms,
-                         "achieved": ach, "unit": unit, "frac": ach / peak}
-    stage_detail = {k: {"launches": d["n"], "ms_per_launch": d["ms"] / max(d["n"], 1),
-                        "tflops_issued": d["work"] / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0}
-                    for k, d in stages.items() if "." in k}
     if by:
         dom = max(by, key=lambda k: by[k]["ms"])
         kd = kernels[dom]
-        traffic = None
-        tf = os.path.join(ROOT, "profiles", "traffic.json")
-        if os.path.exists(tf):
-            try:
-                import hashlib
-                with open(tf) as f:
-                    tj = json.load(f)
-                ent = tj.get(dom)
-                if ent:  # valid only while the kernel's sources are the ones the counters were taken on
-                    hs = hashlib.sha256()
-                    for f in ent["sources"]:
-                        hs.update(open(os.path.join(ROOT, "matrix_aware_sign_b200", "csrc", f), "rb").read())
-                    if hs.hexdigest() == ent["sha256"]:
-                        traffic = ent["bytes_per_launch"]
-            except Exception:
-                traffic = None
         roofline = {"bound": "tensor" if kd["unit"] == "TFLOP/s" else "hbm", "kernel": dom,
                     "achieved": kd["achieved"], "peak": peaks["bf16_tflops_sustained"] if kd["unit"] == "TFLOP/s"
-                    else peaks["hbm_gbs"], "unit": kd["unit"], "frac": kd["frac"], "traffic": traffic,
+                    else peaks["hbm_gbs"], "unit": kd["unit"], "frac": kd["frac"], "traffic": load_traffic(dom),
                     "peak_source": f"{peak_src} ({'bf16 sustained' if kd['unit'] == 'TFLOP/s' else 'HBM copy'})"}
 
     # --- the same step replayed as a CUDA graph (launch overhead removed), reported beside `value`
     graph_value = None
-    if graph is None and args.graph_compare and world == 1:
+    if graph is None and args.graph_compare and world == 1 and wl["graphable"]:
         g2 = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
         side = torch.cuda.Stream()
         with torch.cuda.stream(side):
@@ -491,17 +701,15 @@ def main():
 
     # --- end to end through the public API with host buffers
     e2e = None
-    if args.e2e_steps > 0:
-        hostG = [[torch.from_numpy(g).pin_memory() for layer in gs for g in layer] for gs in gsets]
-        hostW = [torch.empty(w.shape, dtype=torch.float32).pin_memory() for w in W]
-        devG = [torch.empty_like(g) for g in Gd[0]]
+    if e2e_on and wl["e2e_io"] is not None:
+        hostG, devG, hostW, Wd = wl["e2e_io"]()
         torch.cuda.synchronize()
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(args.e2e_steps):
-            for d, h in zip(devG, hostG[i & 1]):
+            for d, h in zip(devG, hostG[i % len(hostG)]):
                 d.copy_(h, non_blocking=True)
             step(i, devG)
             for h, d in zip(hostW, Wd):
@@ -511,14 +719,16 @@ def main():
         barrier()
         ems = reduce_max(e0.elapsed_time(e1), world, device="cuda")
         e2e = {"value": job_throughput(args.e2e_steps, ems, world), "unit": "steps/s",
-               "h2d_bytes_per_step": g_bytes, "d2h_bytes_per_step": w_bytes}
+               "h2d_bytes_per_step": wl["g_bytes"], "d2h_bytes_per_step": wl["w_bytes"]}
+    elif e2e_on:
+        e2e = {"value": None, "unit": "steps/s", "h2d_bytes_per_step": wl["g_bytes"],
+               "d2h_bytes_per_step": wl["w_bytes"],
+               "note": "not measured: the layer set's gradients do not fit a pinned host copy per step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, ids, share, used = time_oracle(cfg, budget_s=15.0)
-        cpu = {"value": v, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{len(ids)} largest of 53 layers x 4 workers ({100 * share:.1f}% of the NS flops, "
-                         f"{used:.1f} s), scaled to the full layer set"}
+        v, sample = oracle_rate(args.workload, 15.0)
+        cpu = {"value": v, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle", "sample": sample}
 
     ns = [k for k in kernels if k.startswith("k_gemm")]
     summary = {}
@@ -529,25 +739,24 @@ def main():
         summary["ns_tflops"] = fl / (t / 1e3) / 1e12
         summary["ns_tflops_nominal"] = nom / (t / 1e3) / 1e12
         summary["ns_frac_of_peak"] = summary["ns_tflops"] / peaks["bf16_tflops_sustained"]
-    if rank == 0 and world == 1 and args.ns4096:
+    if rank == 0 and world == 1 and args.ns4096 and args.workload == "c2_resnet50":
         summary["ns_4096sq_quintic5"] = measure_ns_square(S, torch, peaks, 4096, 5)
-    vk = [k for k in kernels if k.startswith("k_vote_update")]
+    vk = [k for k in kernels if k.startswith("k_vote_update") or k == "k_lion_sign"]
     if vk:
+        summary["vote_kernel"] = vk[0]
         summary["vote_gbs"] = kernels[vk[0]]["achieved"]
         summary["vote_frac_of_hbm"] = kernels[vk[0]]["frac"]
 
     if rank == 0:
         clocks = sampler.summary(t_wall0, t_wall1)
+        wname = desc["workload"] + (f"_first_{args.layers}_matrices" if args.layers > 0 else "")
+        config = {"workload": wname, **wl["config"], "ns_mode": ns_mode,
+                  "global_batch": None, "seq_len": None, "parallelism": f"replicas x{world}",
+                  "launch": "cuda_graph" if graph is not None else "eager"}
         line = {
             "metric": "Muon steps/s per layer set", "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded Gaussian gradients N(0,1e-4), He-normal weights)",
-            "config": {"workload": "resnet50_conv_set_53_layers_M4_quintic1_int8_vote", "layers": L,
-                       "params": n_params, "workers": M, "ns_iters": cfg.iters, "vote": "int8 sum",
-                       "global_batch": None, "seq_len": None, "parallelism": f"replicas x{world}",
-                       "launch": "cuda_graph" if graph is not None else "eager",
-                       "l2": "inputs larger than L2: 375 MB of gradients per step, two resident sets alternate"},
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": desc["data"], "config": config,
             "roofline": roofline, "kernels": kernels, "gemm_stages": stage_detail, **summary,
             "steps_per_s_cuda_graph": graph_value,
             "clocks": clocks, "e2e": e2e,
