@@ -63,6 +63,13 @@ def parse_args():
     p.add_argument("--ns-mode", choices=["plain", "split"], default=None,
                    help="Newton-Schulz operand precision (default: plain for one quintic step, split BF16 for "
                         "five, the mode that meets the 1e-2 tolerance there)")
+    p.add_argument("--grad-source", choices=["hbm", "counter"], default="hbm",
+                   help="LionMuon set: read a resident 45 GB gradient set (default), or draw the workers' "
+                        "gradients inside the kernels from the counter-based streams (no gradient bytes, more ALU)")
+    p.add_argument("--period", type=int, default=None,
+                   help="LionMuon set: period P (default 4; 1 = Muon steps only, 0 = never a Muon step)")
+    p.add_argument("--beta2", type=float, default=None,
+                   help="LionMuon set: EMA rate beta2 (default 0.99; beta2 = beta1 = 0.9 gives Signum-type sign steps)")
     p.add_argument("--layers", type=int, default=0,
                    help="use only the first LAYERS matrices of the set (a smaller case for profiler captures)")
     p.add_argument("--local-polar", action="store_true",
@@ -386,7 +393,8 @@ def describe(name, ns_mode, local_polar):
                             + ("_local_polar" if local_polar else "") + f"_{ns_mode}_bf16",
                 "data": "synthetic (seeded Gaussian gradients N(0,1) drawn on the device, weights N(0,0.02^2) bf16)"}
     return {"workload": f"gpt2_large_set_144_matrices_M16_lionmuon_P4_quintic5_{ns_mode}_bf16",
-            "data": "synthetic (seeded Gaussian gradients N(0,1) drawn on the device, weights N(0,0.02^2) bf16)"}
+            "data": "synthetic (seeded Gaussian gradients N(0,1) resident on the device, or with --grad-source "
+                    "counter drawn in-kernel from Philox4x32-10 streams; weights N(0,0.02^2) bf16)"}
 
 
 def subset(shapes, layers):
@@ -495,29 +503,36 @@ def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0):
                        "l2": "inputs larger than L2: 2.7 GB of gradients per step, two resident sets alternate"}}
 
 
-def setup_c5(S, torch, rank, ns_flags, layers=0):
+def setup_c5(S, torch, rank, ns_flags, layers=0, grad_source="hbm", period=None, beta2=None):
     """GPT-2-Large LionMuon, M = 16, P = 4: three sign steps (vote of the
     workers' sign(G_hat)) and one Muon step (NS of the worker mean) per period.
-    One resident gradient set (45 GB, far larger than L2)."""
+    Gradients: drawn inside the kernels from the counter-based streams (each
+    step new numbers), or one resident 45 GB set read every step."""
     cfg = WL.LION_MUON_WORKLOADS["c5_gpt2l"]
+    P = cfg.period if period is None else period
+    b2 = cfg.beta2 if beta2 is None else beta2
     M, shapes = cfg.workers, subset(cfg.shapes, layers)
     n_params = sum(r * c for r, c in shapes)
     gen = torch.Generator(device="cuda").manual_seed(rank_seed_base(rank) + 5)
     Wd = [(torch.randn(s, device="cuda", generator=gen) * 0.02).to(torch.bfloat16) for s in shapes]
     mom = [[torch.zeros(s, device="cuda") for _ in range(M)] for s in shapes]
-    G = [[torch.randn(s, device="cuda", generator=gen) for _ in range(M)] for s in shapes]
-    opt = S.LionMuon(Wd, mom)
+    if grad_source == "hbm":
+        G = [[torch.randn(s, device="cuda", generator=gen) for _ in range(M)] for s in shapes]
+        opt = S.LionMuon(Wd, mom)
+    else:
+        G = None
+        opt = S.LionMuon(Wd, mom, grad=S.GradStream(rank_seed_base(rank), 0, 1.0, 0))
     ws = S.workspace(opt.workspace_bytes(cfg.iters, ns_flags))
 
     def step(i, G_=None):
-        S.lionmuon_step(opt, G, cfg.period, cfg.beta1, cfg.beta2, cfg.eta, *cfg.coeffs, cfg.iters,
+        S.lionmuon_step(opt, G, P, cfg.beta1, b2, cfg.eta, *cfg.coeffs, cfg.iters,
                         tie_value=cfg.tie_value, ns_flags=ns_flags, ws=ws)
 
     return {"step": step, "graphable": False, "e2e_io": None, "g_bytes": n_params * M * 4, "w_bytes": n_params * 2,
-            "period": cfg.period,
+            "period": P,
             "config": {"layers": len(shapes), "params": n_params, "workers": M, "ns_iters": cfg.iters,
-                       "period": cfg.period, "vote": "1-bit majority on sign steps",
-                       "l2": "inputs larger than L2: 45 GB of gradients and 45 GB of EMA per step"}}
+                       "period": P, "beta1": cfg.beta1, "beta2": b2, "vote": "1-bit majority on sign steps", "gradients": grad_source,
+                       "l2": "inputs larger than L2: 45 GB of EMA (and 45 GB of gradients when read) per step"}}
 
 
 def rollup(S, recs, peaks):
@@ -614,7 +629,7 @@ def main():
     elif args.workload == "c3_gpt2s":
         wl = setup_c3(S, torch, rank, ns_flags, e2e_on, args.local_polar, args.layers)
     else:
-        wl = setup_c5(S, torch, rank, ns_flags, args.layers)
+        wl = setup_c5(S, torch, rank, ns_flags, args.layers, args.grad_source, args.period, args.beta2)
     step = wl["step"]
 
     stream = torch.cuda.current_stream()

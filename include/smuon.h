@@ -291,6 +291,36 @@ smuon_status cachemuon_reuse_probe(const smuon_mat* Q, const smuon_mat* M_t, con
                                    int32_t* d_status, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Counter-based gradient streams of the simulated workers (harness: the
+ * pages describe no generator; this one makes a worker's gradient a pure
+ * function of its coordinates so kernels can draw it instead of reading it).
+ *
+ * Entry i (row-major, whatever the leading dimension) of worker k's gradient
+ * of matrix j at step t is sigma times Gaussian number i % 4 drawn from
+ * Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+ * Easy as 1, 2, 3", SC 2011) at counter (i/4 low word, i/4 high word, t, 0)
+ * and key (seed_base + k, matrix_base + j): the counter's four output words
+ * give two Box-Muller pairs, evaluated in float32 with every operation
+ * rounded on its own (u1 = ((x0 >> 8) + 1) 2^-24, radius sqrt(-2 ln u1),
+ * angle (x1 >> 30) pi/2 + ((x1 >> 8) & 0x3fffff) 2^-22 pi/2, ln, sin and cos
+ * from fixed series), so any IEEE float32 evaluation of the same steps
+ * reproduces the bits.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  uint32_t seed_base;
+  uint32_t matrix_base;
+  float    sigma;
+  uint32_t reserved;    /* 0 */
+} smuon_grad_stream;
+
+/* G[l*workers + k] (F32, rows x cols, any ld >= cols) <- worker k's gradient
+ * of matrix matrix_base + l at step `step`. Enqueued on `stream`; errors:
+ * SMUON_ERR_INVALID_ARG (NULL G or gs, workers < 1, n_layers < 1),
+ * SMUON_ERR_SHAPE, SMUON_ERR_DTYPE (not F32). */
+smuon_status smuon_harness_gaussian(const smuon_mat* G, int32_t n_layers, int32_t workers,
+                                    const smuon_grad_stream* gs, uint32_t step, void* stream);
+
+/* ------------------------------------------------------------------------
  * lionmuon_step -- one step of the LionMuon period-P schedule.
  *
  * LionMuon summary, section "Methodology" item 1 (a Muon step every P-th
@@ -307,17 +337,20 @@ smuon_status cachemuon_reuse_probe(const smuon_mat* Q, const smuon_mat* M_t, con
  *  st->W[n_layers]          F32 or BF16 weights, updated in place
  *  st->mom[n_layers*M]      F32 EMA per worker (worker-minor), updated in place
  *  st->t                    steps taken; the call runs step t+1 and increments it
- *  G[n_layers*M]            F32 gradients (worker-minor)
+ *  G[n_layers*M]            F32 gradients (worker-minor), or NULL to draw them in-kernel from
+ *                           st->grad (see smuon_harness_gaussian; no gradient bytes are read)
  *  ns_flags                 SMUON_NS_* flags of the Muon steps' Newton-Schulz call
  *                           (e.g. SMUON_NS_SPLIT_BF16)
  * Workers 1..64.
  * ---------------------------------------------------------------------- */
 typedef struct {
-  int32_t          n_layers;
-  int32_t          workers;
-  const smuon_mat* W;
-  const smuon_mat* mom;
-  int64_t          t;
+  int32_t                  n_layers;
+  int32_t                  workers;
+  const smuon_mat*         W;
+  const smuon_mat*         mom;
+  int64_t                  t;
+  const smuon_grad_stream* grad;  /* nullable: with G == NULL, worker k's gradient of layer l at step
+                                     t + 1 is drawn inside the kernels from stream (k, matrix_base + l) */
 } lionmuon_state;
 
 smuon_status lionmuon_workspace_bytes(const lionmuon_state* st, int32_t iters, uint32_t ns_flags,

@@ -48,9 +48,14 @@ class TraceRec(ctypes.Structure):
                 ("nominal", ctypes.c_double), ("ms", c_float)]
 
 
+class GradStream(ctypes.Structure):
+    """smuon_grad_stream: worker k's gradient of matrix j is keyed (seed_base + k, matrix_base + j)."""
+    _fields_ = [("seed_base", c_uint32), ("matrix_base", c_uint32), ("sigma", c_float), ("reserved", c_uint32)]
+
+
 class LionMuonState(ctypes.Structure):
     _fields_ = [("n_layers", c_int32), ("workers", c_int32), ("W", POINTER(SmuonMat)),
-                ("mom", POINTER(SmuonMat)), ("t", c_int64)]
+                ("mom", POINTER(SmuonMat)), ("t", c_int64), ("grad", POINTER(GradStream))]
 
 
 _lib = None
@@ -91,6 +96,7 @@ def lib() -> ctypes.CDLL:
             "cachemuon_workspace_bytes": (c_int32, [M, POINTER(c_size_t)]),
             "cachemuon_reuse_probe": (c_int32, [M, M, M, c_float, c_float, c_void_p, c_void_p, c_void_p,
                                                 c_void_p, c_size_t, c_void_p, c_void_p]),
+            "smuon_harness_gaussian": (c_int32, [M, c_int32, c_int32, POINTER(GradStream), c_uint32, c_void_p]),
             "lionmuon_workspace_bytes": (c_int32, [POINTER(LionMuonState), c_int32, c_uint32,
                                                    POINTER(c_size_t)]),
             "lionmuon_step": (c_int32, [POINTER(LionMuonState), c_int32, c_float, c_float, c_float, c_float,
@@ -325,15 +331,19 @@ class CacheMuon:
 
 # ---------------------------------------------------------------- LionMuon
 class LionMuon:
-    """Holds the C lionmuon_state for lists W[layer] and mom[layer][worker]."""
+    """Holds the C lionmuon_state for lists W[layer] and mom[layer][worker].
+    With `grad` (a GradStream), lionmuon_step may be called with G=None: the
+    kernels then draw the workers' gradients from the counter-based streams."""
 
-    def __init__(self, W, mom, t: int = 0):
+    def __init__(self, W, mom, t: int = 0, grad: GradStream | None = None):
         self.W = list(W)
         self.mom = [list(m) for m in mom]
         self.workers = len(self.mom[0])
         self._w = _mats(self.W)
         self._m = _mats([m for layer in self.mom for m in layer])
-        self.state = LionMuonState(len(self.W), self.workers, self._w, self._m, t)
+        self.grad = grad
+        self.state = LionMuonState(len(self.W), self.workers, self._w, self._m, t,
+                                   None if grad is None else ctypes.pointer(grad))
 
     @property
     def t(self) -> int:
@@ -347,10 +357,21 @@ class LionMuon:
 
 def lionmuon_step(opt: LionMuon, G, P, beta1, beta2, eta, a, b, c, iters, tie_value=0, ns_flags=0, ws=None,
                   status=None, stream=None):
-    """G is a list over layers of lists over workers. Returns the workspace used."""
+    """G is a list over layers of lists over workers, or None to draw the
+    gradients in-kernel from opt.grad at step t + 1. Returns the workspace used."""
     if ws is None:
         ws = workspace(opt.workspace_bytes(iters, ns_flags), opt.W[0].device)
-    Gflat = _mats([g for layer in G for g in layer])
+    Gflat = None if G is None else _mats([g for layer in G for g in layer])
     _check(lib().lionmuon_step(ctypes.byref(opt.state), P, beta1, beta2, eta, a, b, c, iters, tie_value, ns_flags,
                                Gflat, ws.data_ptr(), ws.numel(), _ptr(status), _stream(stream)))
     return ws
+
+
+def smuon_harness_gaussian(G, workers: int, stream_desc: GradStream, step: int, stream=None):
+    """G: flat list [layer * workers + worker] of float32 matrices, filled
+    with the counter-based gradient streams at `step`."""
+    n = len(G)
+    if n % workers:
+        raise ValueError("len(G) must be a multiple of workers")
+    _check(lib().smuon_harness_gaussian(_mats(G), n // workers, workers, ctypes.byref(stream_desc), step,
+                                        _stream(stream)))

@@ -9,9 +9,11 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <map>
 #include <memory>
 #include <mutex>
+#include <queue>
 #include <string>
 #include <vector>
 
@@ -190,6 +192,7 @@ struct Layout {
   size_t plan_bytes = 0, total = 0;
   size_t off_groups = 0, off_mats = 0, off_tmaps = 0;
   size_t off_partials = 0, off_scale = 0, off_probe = 0, off_mom_begin = 0;
+  size_t off_sched = 0, off_sched_begin = 0;
   int n_tmaps = 0;
 };
 
@@ -197,6 +200,7 @@ struct Builder {
   std::vector<GroupDesc> groups;
   std::vector<MatDesc> mats;
   std::vector<CUtensorMap> maps;
+  std::vector<int32_t> sched, sched_begin;  // tensor-core tile schedule (filled when base is set)
   PlanHeader h{};
   Layout L;
   size_t cursor = 0;
@@ -218,6 +222,57 @@ Mode pick_mode(uint32_t flags) {
   if (flags & SMUON_NS_FP32_REF) return MODE_SIMT_F32;
   if (flags & SMUON_NS_SIMT_BF16) return MODE_SIMT_BF16;
   return MODE_TC_BF16;
+}
+
+// Tile schedule of one tensor-core stage. The stages whose K is the long side
+// n (Gram, probe) mix tiles of very different lengths across groups (a 512 x
+// 4608 Gram tile runs 72 k-blocks, a 64 x 576 one 9): there, longest
+// processing time first -- tiles in decreasing cost (ties in tile order) each
+// onto the CTA with the least work so far. Cost of a tile in units of one
+// 64-deep k-block of MMAs: its k-blocks (three MMAs each in split mode) plus
+// about eight for the epilogue of a full 128 x 256 tile, scaled by the share
+// of the tile that lies inside the matrix. The other stages (K = m) keep the
+// round-robin order, tile t on CTA t mod ctas: their tiles are short and
+// epilogue-bound, so a count-balanced order does better than the cost model.
+bool lpt_stage(int st) { return st == ST_GRAM || st == ST_PROBE; }
+
+void schedule_stage(const std::vector<GroupDesc>& groups, int st, int total, int ctas, int bn, bool split,
+                    int32_t* ids, int32_t* begin) {
+  std::vector<std::vector<int32_t>> per(ctas);
+  if (!lpt_stage(st)) {
+    for (int t = 0; t < total; ++t) per[t % ctas].push_back(t);
+  } else {
+    std::vector<std::pair<double, int32_t>> cost_tile;  // (cost, tile)
+    cost_tile.reserve(total);
+    for (const GroupDesc& g : groups) {
+      const int tiles = sym_stage(st) ? sym_start(g.tiles_m[st], g.tiles_n[st], bn / kTcBM)
+                                      : g.tiles_m[st] * g.tiles_n[st];
+      const int K = (st == ST_GRAM || st == ST_PROBE) ? g.n : g.m;
+      const int No = (st == ST_AXPY || st == ST_REUSE) ? g.n : g.m;
+      const double kb = (double)((K + 63) / 64) * (split && st <= ST_QAXPY ? 3 : 1) * bn / 256.0;
+      const double fill = (double)g.m * No / ((double)g.tiles_m[st] * kTcBM * g.tiles_n[st] * bn);
+      const double cost = kb + 8.0 * fill * bn / 256.0;
+      for (int t = g.tile_begin[st]; t < g.tile_begin[st] + g.count * tiles; ++t) cost_tile.push_back({cost, t});
+    }
+    std::stable_sort(cost_tile.begin(), cost_tile.end(),
+                     [](const auto& x, const auto& y) { return x.first > y.first; });
+    // least-loaded CTA first (ties: lowest index)
+    using Load = std::pair<double, int32_t>;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < ctas; ++c) heap.push({0.0, c});
+    for (const auto& ct : cost_tile) {
+      Load l = heap.top();
+      heap.pop();
+      per[l.second].push_back(ct.second);
+      heap.push({l.first + ct.first, l.second});
+    }
+  }
+  int pos = 0;
+  for (int c = 0; c < ctas; ++c) {
+    begin[c] = pos;
+    for (int32_t t : per[c]) ids[pos++] = t;
+  }
+  begin[ctas] = pos;
 }
 
 // Builds groups, descriptors and the workspace layout. With base == nullptr it
@@ -309,6 +364,17 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     }
   }
 
+  // tile schedule sizes (tensor-core mode): every tile id once, a begin array per stage
+  int sched_off[ST_COUNT] = {0}, sched_boff[ST_COUNT] = {0};
+  int sched_n = 0, begin_n = 0;
+  for (int st = 0; st < ST_COUNT; ++st) {
+    sched_off[st] = sched_n;
+    sched_boff[st] = begin_n;
+    if (!tc) continue;
+    sched_n += totals[st];
+    begin_n += std::min(totals[st], kMaxSchedCtas) + 1;
+  }
+
   // layout: plan region first
   Layout& L = B->L;
   B->cursor = 0;
@@ -317,6 +383,8 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.off_groups = B->take(sizeof(GroupDesc) * B->groups.size());
   L.off_mats = B->take(sizeof(MatDesc) * B->mats.size());
   L.off_mom_begin = B->take(sizeof(int32_t) * (B->mats.size() + 1));
+  L.off_sched = B->take(sizeof(int32_t) * std::max(sched_n, 1));
+  L.off_sched_begin = B->take(sizeof(int32_t) * std::max(begin_n, 1));
   // tensor maps: count them first
   auto want_map = [&](int32_t& slot) { slot = L.n_tmaps++; };
   L.n_tmaps = 0;
@@ -405,11 +473,35 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   h.scale = B->ptr_at<float>(L.off_scale);
   h.probe_partials = B->ptr_at<float>(L.off_probe);
   h.mom_begin = B->ptr_at<int32_t>(L.off_mom_begin);
+  h.sched = B->ptr_at<int32_t>(L.off_sched);
+  h.sched_begin = B->ptr_at<int32_t>(L.off_sched_begin);
+  for (int st = 0; st < ST_COUNT; ++st) {
+    h.sched_off[st] = sched_off[st];
+    h.sched_boff[st] = sched_boff[st];
+    h.sched_ctas[st] = 0;
+  }
   h.groups = B->ptr_at<GroupDesc>(L.off_groups);
   h.mats = B->ptr_at<MatDesc>(L.off_mats);
   h.tmaps = B->ptr_at<CUtensorMap>(L.off_tmaps);
 
   if (!base) return SMUON_OK;
+
+  // tile schedules over this device's SMs (one persistent CTA per SM)
+  B->sched.assign(std::max(sched_n, 1), 0);
+  B->sched_begin.assign(std::max(begin_n, 1), 0);
+  if (tc) {
+    DevInfo di;
+    smuon_status dst = device_info(&di);
+    if (dst != SMUON_OK) return dst;
+    const bool split = (rq.flags & SMUON_NS_SPLIT_BF16) != 0 && parts == 2;
+    for (int st = 0; st < ST_COUNT; ++st) {
+      if (totals[st] == 0) continue;
+      const int ctas = std::min(std::min(totals[st], di.sms), kMaxSchedCtas);
+      h.sched_ctas[st] = ctas;
+      schedule_stage(B->groups, st, totals[st], ctas, BM * ratios[st], split, B->sched.data() + sched_off[st],
+                     B->sched_begin.data() + sched_boff[st]);
+    }
+  }
 
   // tensor maps
   B->maps.assign(std::max(L.n_tmaps, 1), CUtensorMap{});
@@ -452,6 +544,8 @@ smuon_status upload_plan(Builder& B, cudaStream_t s) {
     mb[B.mats.size()] = B.h.total_mom_tiles;
     memcpy(bytes.data() + B.L.off_mom_begin, mb.data(), sizeof(int32_t) * mb.size());
   }
+  memcpy(bytes.data() + B.L.off_sched, B.sched.data(), sizeof(int32_t) * B.sched.size());
+  memcpy(bytes.data() + B.L.off_sched_begin, B.sched_begin.data(), sizeof(int32_t) * B.sched_begin.size());
   if (B.L.n_tmaps > 0) memcpy(bytes.data() + B.L.off_tmaps, B.maps.data(), sizeof(CUtensorMap) * B.L.n_tmaps);
   static UploadChunk chunk;  // large parameter block; filled then launched by value
   static std::mutex mu;
@@ -1118,10 +1212,49 @@ smuon_status lionmuon_workspace_bytes(const lionmuon_state* st, int32_t iters, u
   return SMUON_OK;
 }
 
+smuon_status smuon_harness_gaussian(const smuon_mat* G, int32_t n_layers, int32_t workers,
+                                    const smuon_grad_stream* gs, uint32_t step, void* stream) {
+  if (!G || !gs) return fail(SMUON_ERR_INVALID_ARG, "G and gs must not be NULL");
+  if (n_layers < 1 || workers < 1) return fail(SMUON_ERR_INVALID_ARG, "n_layers and workers must be >= 1");
+  if ((int64_t)n_layers * workers > (1 << 20)) return fail(SMUON_ERR_INVALID_ARG, "too many matrices");
+  smuon_status s;
+  EwBuild eb;
+  for (int l = 0; l < n_layers; ++l)
+    for (int k = 0; k < workers; ++k) {
+      const int i = l * workers + k;
+      const smuon_mat& g = G[i];
+      if ((s = check_mat(g, "G", i, true, false, false)) != SMUON_OK) return s;
+      EwLayer L{};
+      L.w = g.data; L.w_ld = g.ld; L.w_dtype = SMUON_F32;
+      L.rows = g.rows; L.cols = g.cols; L.n = (int64_t)g.rows * g.cols;
+      L.vec = vec_ok(g.data, g.ld, g.cols, 1);
+      L.key0 = gs->seed_base + (uint32_t)k;
+      L.key1 = gs->matrix_base + (uint32_t)l;
+      eb.layers.push_back(L);
+      eb.srcs.push_back({});
+    }
+  DevInfo di;
+  if ((s = device_info(&di)) != SMUON_OK) return s;
+  cudaStream_t strm = reinterpret_cast<cudaStream_t>(stream);
+  EwTable proto{};
+  proto.gen_step = step;
+  proto.gen_sigma = gs->sigma;
+  return for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
+    double n = 0;
+    for (int l = 0; l < tb.n_layers; ++l) n += 4.0 * (double)tb.layers[l].n;
+    Launch L("k_harness_gaussian", SMUON_WORK_BYTES, n, strm);
+    k_harness_gaussian<<<ew_grid(tb.total_chunks, di), 256, 0, strm>>>(tb);
+    CUDA_TRY(cudaGetLastError());
+    return SMUON_OK;
+  });
+}
+
 smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float beta2, float eta, float a, float b,
                            float c, int32_t iters, int8_t tie_value, uint32_t ns_flags, const smuon_mat* G, void* ws,
                            size_t ws_bytes, int32_t* d_status, void* stream) {
-  if (!st || !st->W || !st->mom || !G) return fail(SMUON_ERR_INVALID_ARG, "state, W, mom and G must not be NULL");
+  if (!st || !st->W || !st->mom) return fail(SMUON_ERR_INVALID_ARG, "state, W and mom must not be NULL");
+  if (!G && !st->grad) return fail(SMUON_ERR_INVALID_ARG, "G is NULL and the state has no gradient stream");
+  const bool gen = (G == nullptr);
   if (st->n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "n_layers < 1");
   const int M = st->workers;
   if (M < 1 || M > kMaxWorkers) return fail(SMUON_ERR_UNSUPPORTED, "workers=%d must be in 1..%d", M, kMaxWorkers);
@@ -1137,15 +1270,21 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
     L.rows = st->W[l].rows; L.cols = st->W[l].cols; L.n = (int64_t)L.rows * L.cols;
     L.vec = vec_ok(L.w, L.w_ld, L.cols, 1);
     std::vector<EwSrc> srcs;
+    if (gen) L.key1 = st->grad->matrix_base + (uint32_t)l;
     for (int k = 0; k < M; ++k) {
       const smuon_mat& mo = st->mom[(int64_t)l * M + k];
-      const smuon_mat& g = G[(int64_t)l * M + k];
       if ((s = check_mat(mo, "mom", l * M + k, true, false, false)) != SMUON_OK) return s;
-      if ((s = check_mat(g, "G", l * M + k, true, false, false)) != SMUON_OK) return s;
-      if (!same_shape(mo, st->W[l]) || !same_shape(g, st->W[l]))
-        return fail(SMUON_ERR_SHAPE, "mom/G of layer %d differ from W's shape", l);
-      if (!vec_ok(mo.data, mo.ld, mo.cols, 1) || !vec_ok(g.data, g.ld, g.cols, 1)) L.vec = 0;
+      if (!same_shape(mo, st->W[l])) return fail(SMUON_ERR_SHAPE, "mom of layer %d differs from W's shape", l);
+      if (!vec_ok(mo.data, mo.ld, mo.cols, 1)) L.vec = 0;
       srcs.push_back(EwSrc{mo.data, mo.ld});
+      if (gen) {
+        srcs.push_back(EwSrc{nullptr, 0});  // drawn in-kernel
+        continue;
+      }
+      const smuon_mat& g = G[(int64_t)l * M + k];
+      if ((s = check_mat(g, "G", l * M + k, true, false, false)) != SMUON_OK) return s;
+      if (!same_shape(g, st->W[l])) return fail(SMUON_ERR_SHAPE, "G of layer %d differs from W's shape", l);
+      if (!vec_ok(g.data, g.ld, g.cols, 1)) L.vec = 0;
       srcs.push_back(EwSrc{g.data, g.ld});
     }
     eb.layers.push_back(L);
@@ -1161,10 +1300,18 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
   proto.beta1 = beta1; proto.beta2 = beta2;
   proto.c1 = 1.f - beta1;  // float32 (1 - beta), as in the reading of the EMA
   proto.c2 = 1.f - beta2;
+  if (gen) {
+    proto.gen_on = 1;
+    proto.gen_seed = st->grad->seed_base;
+    proto.gen_step = (uint32_t)t_next;
+    proto.gen_sigma = st->grad->sigma;
+  }
+  const double g_bytes = gen ? 0.0 : 4.0;  // gradient bytes read per entry and worker
   if (!muon) {
     s = for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
       double n = 0;
-      for (int l = 0; l < tb.n_layers; ++l) n += (double)tb.layers[l].n * (12.0 * M + 2 * dtype_size(tb.layers[l].w_dtype));
+      for (int l = 0; l < tb.n_layers; ++l)
+        n += (double)tb.layers[l].n * ((8.0 + g_bytes) * M + 2 * dtype_size(tb.layers[l].w_dtype));
       Launch L("k_lion_sign", SMUON_WORK_BYTES, n, strm);
       k_lion_sign<<<ew_grid(tb.total_chunks, di), 256, 0, strm>>>(tb);
       CUDA_TRY(cudaGetLastError());
@@ -1188,7 +1335,7 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
   }
   s = for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
     double n = 0;
-    for (int l = 0; l < tb.n_layers; ++l) n += (double)tb.layers[l].n * (12.0 * M + 4.0);
+    for (int l = 0; l < tb.n_layers; ++l) n += (double)tb.layers[l].n * ((8.0 + g_bytes) * M + 4.0);
     Launch L("k_lion_mean", SMUON_WORK_BYTES, n, strm);
     k_lion_mean<<<ew_grid(tb.total_chunks, di), 256, 0, strm>>>(tb);
     CUDA_TRY(cudaGetLastError());

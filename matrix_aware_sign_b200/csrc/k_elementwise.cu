@@ -10,8 +10,10 @@
 //  * k_lion_sign       LionMuon sign step (G_hat, vote, W and EMA update)
 //  * k_lion_mean       LionMuon Muon-step prologue (mean of G_hat, EMA update)
 //  * k_probe_finalize  CacheMuon residual, accept flag and counters
+//  * k_harness_gaussian  counter-based gradient streams written out (harness)
 #include <algorithm>
 
+#include "counter_rng.cuh"
 #include "kernels.cuh"
 
 namespace smuon {
@@ -335,8 +337,15 @@ __device__ __forceinline__ int warp_layer(const EwTable& tb, int64_t wbase, int6
 // the integer sum of +-1), then W <- W - eta*vote in float32, rounded to W's
 // type. Work unit: 8 consecutive entries per lane.
 // per 16-bit lane of w: 1 where the bf16 value is >= 0 (+0, -0, positives; not NaN)
+// Plain integer arithmetic on both halves at once (no carries cross the halves):
+// with mag = h & 0x7fff, u >= 0 holds iff (sign clear and mag <= 0x7f80, i.e.
+// not a NaN) or mag == 0 (-0). Bit 15 of mag + 0x7f is clear iff mag <= 0x7f80;
+// bit 15 of mag + 0x7fff is clear iff mag == 0.
 __device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
-  return (__vcmpleu2(w, 0x7f807f80u) | __vcmpeq2(w, 0x80008000u)) & 0x00010001u;
+  const uint32_t mag = w & 0x7fff7fffu;
+  const uint32_t le = mag + 0x007f007fu;
+  const uint32_t nz = mag + 0x7fff7fffu;
+  return (((~le & ~w) | ~nz) >> 15) & 0x00010001u;
 }
 
 // int8 (integer-sum) vote on bf16 outputs: the count of positive signs of each
@@ -347,11 +356,13 @@ __device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
 __device__ __forceinline__ void vote_i8_finish16(const EwTable& tb, const EwLayer& L, int64_t e0,
                                                  const uint32_t* cnt, float* w) {
   int8_t v8[16];
+  // eta * v for v = +1, -1 and the tie value: exact products, chosen per entry
+  const float up = tb.eta, down = -tb.eta, tied = tb.eta * (float)tb.tie;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    const int c = (int)((cnt[k >> 1] >> (16 * (k & 1))) & 0xffffu);
-    v8[k] = threshold(2 * c - tb.M, tb.tie);
-    w[k] = __fsub_rn(w[k], tb.eta * (float)v8[k]);
+    const int c2 = 2 * (int)((cnt[k >> 1] >> (16 * (k & 1))) & 0xffffu);
+    v8[k] = (int8_t)(c2 > tb.M ? 1 : (c2 < tb.M ? -1 : tb.tie));
+    w[k] = __fsub_rn(w[k], c2 > tb.M ? up : (c2 < tb.M ? down : tied));
   }
   store8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
   store8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
@@ -423,6 +434,114 @@ __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
         store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
         if (L.vote_out) L.vote_out[e] = v;
       }
+    }
+  }
+}
+
+// the 16 message bits of one lane (bit j = entry e0 + j is >= 0) from the
+// per-half flags of its 8 words (bit 0: entry 2i, bit 16: entry 2i + 1)
+__device__ __forceinline__ uint32_t mask16_from_halves(const uint32_t* p) {
+  uint32_t y = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y |= p[i] << (2 * i);
+  return (y | (y >> 15)) & 0xffffu;
+}
+
+// per-half sign flags of entries e, e + 1 (only those below `left` entries), one by one
+__device__ __noinline__ uint32_t pos_halves_scalar(const EwSrc& S, const EwLayer& L, int64_t e, int left) {
+  uint32_t f = 0;
+  if (left > 0) f |= (uint32_t)(load_as_f32(S.ptr, ew_index(L, e, S.ld), SMUON_BF16) >= 0.f);
+  if (left > 1) f |= (uint32_t)(load_as_f32(S.ptr, ew_index(L, e + 1, S.ld), SMUON_BF16) >= 0.f) << 16;
+  return f;
+}
+
+// vote and update of entries e, e + 1 (only those below `left`) from their packed counts
+__device__ __noinline__ void finish_pair_scalar(const EwTable& tb, const EwLayer& L, int64_t e, int left,
+                                                uint32_t cnt) {
+  for (int k = 0; k < 2 && k < left; ++k) {
+    const int c = (int)((cnt >> (16 * k)) & 0xffffu);
+    const int8_t v = threshold(2 * c - tb.M, tb.tie);
+    const int64_t wi = ew_index(L, e + k, L.w_ld);
+    store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+    if (L.vote_out) L.vote_out[e + k] = v;
+  }
+}
+
+// Fused sign / 1-bit message / majority vote / update for bf16 outputs, any
+// M up to 64, 16 entries per lane. Per worker, the lane's 16 sign flags (U >= 0)
+// are kept as 8 words of per-half flags. Their sum over the workers is, per
+// entry, the number of set bits among the M workers' message bits (two 16-bit
+// counters per add): the popcount of the entry's bits, and sum = 2*count - M.
+// The same flags are the lane's 16 message bits; two neighbouring lanes join
+// theirs into one packed word (entry i -> bit i%32 of word i/32) with one
+// shuffle. Layer chunk ranges are multiples of 16 chunks (128 entries), so a
+// lane pair never straddles a layer and the even lane's e0 is a multiple of 32.
+__device__ __forceinline__ void vote_update_bf16x16(const EwTable& tb) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int M = tb.M;
+  const bool any_packed = tb.any_packed != 0;  // uniform: the shuffles below involve every lane
+  for (int64_t wbase = warp_global * 64; wbase < tb.total_chunks; wbase += warps_total * 64) {
+    const int64_t chunk = wbase + 2 * lane;
+    const bool active = chunk < tb.total_chunks;
+    const int li = warp_layer(tb, wbase, active ? chunk : tb.total_chunks - 1, lane);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    const bool live = active && e0 < L.n;
+    const bool fast = live && L.vec && e0 + 16 <= L.n;
+    const int nent = live ? (int)min((int64_t)16, L.n - e0) : 0;
+    float w[16];
+    uint32_t cnt[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (fast) {
+      load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+      load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
+    }
+    for (int wk0 = 0; wk0 < M; wk0 += 4) {
+      uint4 u[4][2];
+      if (fast) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (wk0 + j < M) {
+            const uint4* q = reinterpret_cast<const uint4*>(
+                reinterpret_cast<const __nv_bfloat16*>(tb.srcs[L.src_first + wk0 + j].ptr) + e0);
+            u[j][0] = q[0];
+            u[j][1] = q[1];
+          }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int wk = wk0 + j;
+        if (wk >= M) break;  // uniform across the warp
+        uint32_t f[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (fast) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            f[4 * hh + 0] = pos_halves_bf16(u[j][hh].x);
+            f[4 * hh + 1] = pos_halves_bf16(u[j][hh].y);
+            f[4 * hh + 2] = pos_halves_bf16(u[j][hh].z);
+            f[4 * hh + 3] = pos_halves_bf16(u[j][hh].w);
+          }
+        } else if (live) {  // ragged tail or strided layer: entry by entry
+          const EwSrc& S = tb.srcs[L.src_first + wk];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] = pos_halves_scalar(S, L, e0 + 2 * i, nent - 2 * i);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cnt[i] += f[i];
+        if (any_packed) {
+          uint32_t v = mask16_from_halves(f) << (16 * (lane & 1));
+          v |= __shfl_xor_sync(0xffffffffu, v, 1);
+          if (active && L.packed_out && (lane & 1) == 0) L.packed_out[(int64_t)wk * L.words + (e0 >> 5)] = v;
+        }
+      }
+    }
+    if (!live) continue;
+    if (fast) {
+      vote_i8_finish16(tb, L, e0, cnt, w);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) finish_pair_scalar(tb, L, e0 + 2 * i, nent - 2 * i, cnt[i]);
     }
   }
 }
@@ -501,8 +620,19 @@ __global__ void __launch_bounds__(256) k_vote_update_i8_bf16(const __grid_consta
   vote_update_int8_bf16(tb);
 }
 
+__global__ void __launch_bounds__(256) k_vote_update_bf16x16(const __grid_constant__ EwTable tb) {
+  vote_update_bf16x16(tb);
+}
+
 cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s) {
   const bool bf = tb.src_dtype == SMUON_BF16;
+  // 16 entries per lane; measured best with 2-4 resident CTAs per SM
+  const int64_t want16 = (tb.total_chunks + 511) / 512;
+  const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 4 * sms));
+  if (bf && (popcount || tb.any_packed) && tb.M <= kMaxWorkers) {
+    k_vote_update_bf16x16<<<grid16, 256, 0, s>>>(tb);
+    return cudaGetLastError();
+  }
   if (popcount) {
     if (tb.M <= 32) {
       if (bf) k_vote_update<true, true, uint32_t><<<grid, 256, 0, s>>>(tb);
@@ -513,11 +643,7 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
     }
   } else {
     // the packed-counter kernel needs no packed message (it builds none)
-    if (bf && !tb.any_packed) {
-      // 16 entries per lane; measured best with 2-4 resident CTAs per SM
-      const int64_t want = (tb.total_chunks + 511) / 512;
-      k_vote_update_i8_bf16<<<(int)std::max<int64_t>(1, std::min<int64_t>(want, 4 * sms)), 256, 0, s>>>(tb);
-    }
+    if (bf && !tb.any_packed) k_vote_update_i8_bf16<<<grid16, 256, 0, s>>>(tb);
     else if (bf) k_vote_update<false, true, uint32_t><<<grid, 256, 0, s>>>(tb);
     else k_vote_update<false, false, uint32_t><<<grid, 256, 0, s>>>(tb);
   }
@@ -649,8 +775,11 @@ __global__ void __launch_bounds__(256) k_lion_sign(const __grid_constant__ EwTab
         const int wk = wk0 + j;
         if (wk < tb.M) {
           load8(tb.srcs[L.src_first + 2 * wk].ptr, tb.srcs[L.src_first + 2 * wk].ld, SMUON_F32, L, e0, L.vec, mo[j]);
-          load8(tb.srcs[L.src_first + 2 * wk + 1].ptr, tb.srcs[L.src_first + 2 * wk + 1].ld, SMUON_F32, L, e0,
-                L.vec, gr[j]);
+          if (tb.gen_on)
+            crng::gaussian8(tb.gen_seed + (uint32_t)wk, L.key1, tb.gen_step, e0, tb.gen_sigma, gr[j]);
+          else
+            load8(tb.srcs[L.src_first + 2 * wk + 1].ptr, tb.srcs[L.src_first + 2 * wk + 1].ld, SMUON_F32, L, e0,
+                  L.vec, gr[j]);
         }
       }
 #pragma unroll
@@ -697,7 +826,10 @@ __global__ void __launch_bounds__(256) k_lion_mean(const __grid_constant__ EwTab
       const EwSrc& Gs = tb.srcs[L.src_first + 2 * wk + 1];
       float mo[8], gr[8];
       load8(S.ptr, S.ld, SMUON_F32, L, e0, L.vec, mo);
-      load8(Gs.ptr, Gs.ld, SMUON_F32, L, e0, L.vec, gr);
+      if (tb.gen_on)
+        crng::gaussian8(tb.gen_seed + (uint32_t)wk, L.key1, tb.gen_step, e0, tb.gen_sigma, gr);
+      else
+        load8(Gs.ptr, Gs.ld, SMUON_F32, L, e0, L.vec, gr);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float gh = __fadd_rn(__fmul_rn(tb.beta1, mo[k]), __fmul_rn(tb.c1, gr[k]));
@@ -742,6 +874,22 @@ __global__ void k_probe_nocache(float* d_err, int32_t* d_accept, cachemuon_count
   *d_err = __int_as_float(0x7f800000);
   *d_accept = 0;
   if (counters) counters->misses += 1;
+}
+
+// Harness: sigma * N(0, 1) from the counter-based stream of each matrix
+// (key words per matrix, counter word 2 = the step), written as float32.
+__global__ void __launch_bounds__(256) k_harness_gaussian(const __grid_constant__ EwTable tb) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; chunk < tb.total_chunks;
+       chunk += stride) {
+    const int li = find_layer(&tb, chunk);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    if (e0 >= L.n) continue;
+    float v[8];
+    crng::gaussian8(L.key0, L.key1, tb.gen_step, e0, tb.gen_sigma, v);
+    store8(L.w, L.w_ld, SMUON_F32, L, e0, L.vec, v);
+  }
 }
 
 }  // namespace smuon

@@ -1,15 +1,20 @@
 // k_gemm_tc.cu -- grouped Newton-Schulz GEMM stages on the sm_100a tensor cores.
 //
-// One persistent kernel per stage walks the plan's tile list (all layers x
-// workers in one launch). Per CTA:
+// One persistent kernel per stage (all layers x workers in one launch); each
+// CTA walks its own list of tiles from the plan's schedule. Per CTA (320
+// threads, one per SM):
 //   warp 0      TMA producer: 128B-swizzled tiles of A (K-major) and B
 //               (K-major, or MN-major for the X / Q right operand) into a
-//               6-deep shared-memory ring (full/empty mbarriers)
+//               shared-memory ring (full/empty mbarriers): 4 stages of
+//               128 x 64 + 256 x 64 bf16 in plain mode, 3 stages of hi and
+//               lo parts of 128 x 64 + 128 x 64 in split mode
 //   warp 1      TMEM allocation and the single MMA-issuing thread:
 //               tcgen05.mma.cta_group::1.kind::f16, BF16 x BF16 -> FP32,
-//               M = N = 128, K = 16 per instruction, into one of two TMEM
-//               accumulators (128 columns each)
-//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns at a time, stage
+//               M = 128, N = BN (256 plain, 128 split), K = 16 per
+//               instruction (three per step in split mode: hi*hi, hi*lo,
+//               lo*hi), into one of two TMEM accumulators of BN columns
+//   warps 2-9   epilogue, two warps per TMEM lane group (one per half of the
+//               columns): tcgen05.ld 32 lanes x 32 columns at a time, stage
 //               algebra in FP32 (epilogue.cuh), global stores
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
 // i+1. Every mbarrier wait is bounded; on expiry the CTA records
@@ -174,38 +179,6 @@ __device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, i
   return o;
 }
 
-// L2 prefetch of the row segments that the B X epilogue will read from its
-// X source (the user's momentum at the first step, the f32 master later),
-// issued by the producer warp while the tile's MMAs are still ahead
-__device__ __forceinline__ void prefetch_rows(const char* base, int64_t row_stride_bytes, int nrows, int bytes,
-                                              int lane) {
-  for (int r = lane; r < nrows; r += 32) {
-    const char* p = base + (int64_t)r * row_stride_bytes;
-    for (int b = 0; b < bytes; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + b));
-  }
-}
-
-template <int kBN>
-__device__ __forceinline__ void prefetch_axpy_source(const TileCtx& t, int tm, int tn, int lane) {
-  if (t.stage != ST_AXPY) return;
-  const int rows = min(BM, t.Mo - tm * BM), cols = min(kBN, t.No - tn * kBN);
-  if (rows <= 0 || cols <= 0) return;
-  if (t.iter == 0 && t.bf) {
-    const MatDesc& md = *t.md;
-    const int es = md.m_dtype == SMUON_F32 ? 4 : (md.m_dtype == SMUON_BF16 ? 2 : 1);
-    const char* p = reinterpret_cast<const char*>(md.m_ptr);
-    if (!md.tall)  // wide: X row i = user row i
-      prefetch_rows(p + ((int64_t)tm * BM * md.m_ld + (int64_t)tn * kBN) * es, md.m_ld * es, rows, cols * es, lane);
-    else           // tall: X column j = user row j
-      prefetch_rows(p + ((int64_t)tn * kBN * md.m_ld + (int64_t)tm * BM) * es, md.m_ld * es, cols, rows * es, lane);
-  } else {
-    const GroupDesc& g = *t.g;
-    const float* src = t.bf ? g.xf[t.iter & 1] : reinterpret_cast<const float*>(g.xop[t.iter & 1]);
-    const char* p = reinterpret_cast<const char*>(src + ((int64_t)t.z * g.m + (int64_t)tm * BM) * g.ldn + (int64_t)tn * kBN);
-    prefetch_rows(p, g.ldn * 4, rows, cols * 4, lane);
-  }
-}
-
 template <bool kSplit, int kBN>
 __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int iter) {
   using C = Cfg<kSplit, kBN>;
@@ -243,18 +216,21 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = h.total_tiles[stage];
+  // this CTA's tiles (host-balanced list; every role walks the same one)
+  const int32_t* tiles = h.sched + h.sched_off[stage];
+  const int t_begin = h.sched_begin[h.sched_boff[stage] + blockIdx.x];
+  const int t_end = h.sched_begin[h.sched_boff[stage] + blockIdx.x + 1];
 
   if (warp == 0) {
-    // ---------------- TMA producer (lane 0) + L2 prefetch of the epilogue source (all lanes)
+    // ---------------- TMA producer (lane 0)
     int s = 0;
     uint32_t ph = 0;
     uint32_t armed = 0, last_par = 0;  // per-stage bit sets for the exit drain
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+    for (int i = t_begin; i < t_end && ok; ++i) {
+      const int tile = tiles[i];
       int tm, tn;
       const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
-      prefetch_axpy_source<kBN>(t, tm, tn, lane);
       if (lane == 0) {
         const TcOps o = tc_ops(h, t, iter, kBN);
         tensormap_acquire(o.ma);
@@ -305,7 +281,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       int acc = 0;
       uint32_t acc_ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int i = t_begin; i < t_end && ok; ++i) {
+        const int tile = tiles[i];
         int tm, tn;
         const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
         const TcOps o = tc_ops(h, t, iter, kBN);
@@ -354,7 +331,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
     constexpr int CH = kBN / 64;     // 32-column chunks per warp
     int acc = 0;
     uint32_t acc_ph = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int i = t_begin; i < t_end; ++i) {
+      const int tile = tiles[i];
       int tm, tn;
       TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
       if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag)) {
@@ -418,9 +396,9 @@ int tc_tile_n(int stage, uint32_t flags) {
 
 cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter, const int32_t* skip,
                            int num_sms, cudaStream_t s) {
-  const int total = h.total_tiles[stage];
-  if (total == 0) return cudaSuccess;
-  const int grid = total < num_sms ? total : num_sms;
+  (void)num_sms;  // the plan's schedule fixed the grid: one CTA per scheduled tile list
+  const int grid = h.sched_ctas[stage];
+  if (h.total_tiles[stage] == 0 || grid <= 0) return cudaSuccess;
   const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && stage <= ST_QAXPY;
   if (split) return launch_tc_variant<true, 128>(d_plan, stage, iter, skip, grid, s);
   if (tc_tile_n(stage, h.flags) == 128) return launch_tc_variant<false, 128>(d_plan, stage, iter, skip, grid, s);

@@ -37,12 +37,17 @@ struct EwLayer {
   int32_t vec_aux;
   int32_t src_first;       // first entry of this layer in srcs[]
   int32_t rows, cols;
+  uint32_t key0, key1;     // counter-based gradient stream keys (harness draws; key1 also for LionMuon)
 };
 
 struct EwTable {
   int32_t n_layers, M, tie, src_dtype;
   int32_t any_packed, pad;
   float eta, beta1, beta2, c1, c2;
+  int32_t gen_on;          // LionMuon: gradients drawn in-kernel instead of read (srcs hold no G)
+  uint32_t gen_seed;       // key word 0 of worker k = gen_seed + k
+  uint32_t gen_step;       // counter word 2
+  float gen_sigma;
   int64_t total_chunks;
   EwLayer layers[kEwMaxLayers];
   EwSrc srcs[kEwMaxSrcs];
@@ -62,6 +67,7 @@ __global__ void k_sign_pack(const __grid_constant__ EwTable tb, uint32_t* packed
 __global__ void k_vote(const uint32_t* packed, const int8_t* signs, int M, int64_t N, int64_t words,
                        int tie, int8_t* vote);
 __global__ void k_update_src(const __grid_constant__ EwTable tb);
+__global__ void k_harness_gaussian(const __grid_constant__ EwTable tb);
 __global__ void k_lion_sign(const __grid_constant__ EwTable tb);
 __global__ void k_lion_mean(const __grid_constant__ EwTable tb);
 __global__ void k_probe_finalize(const Plan* plan);

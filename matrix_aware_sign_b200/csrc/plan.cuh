@@ -17,6 +17,7 @@
 namespace smuon {
 
 constexpr int kMaxWorkers = 64;
+constexpr int kMaxSchedCtas = 1024;  // most CTAs a tensor-core stage is scheduled over
 
 // Stages of the Newton-Schulz chain. Each is one grouped GEMM launch
 // D = A_op * B_op over every matrix of the batch, with its own epilogue.
@@ -90,6 +91,13 @@ struct PlanHeader {
   float* scale;             // [n_mats] s = 1/(||M||_F + eps)
   float* probe_partials;    // [total PROBE tiles]
   const int32_t* mom_begin; // [n_mats + 1] first momentum tile of each matrix (compact, for the tile search)
+  // tensor-core stages: each CTA walks its own list of tiles, balanced on the
+  // host by tile cost (longest first onto the least loaded CTA)
+  const int32_t* sched;             // tile ids of every stage, CTA after CTA
+  const int32_t* sched_begin;       // per stage: first list entry of each CTA (sched_ctas + 1 entries)
+  int32_t sched_off[ST_COUNT];      // offset of each stage's tile ids in sched
+  int32_t sched_boff[ST_COUNT];     // offset of each stage's begin array in sched_begin
+  int32_t sched_ctas[ST_COUNT];     // CTAs of each stage's launch
   GroupDesc* groups;        // device pointers into the plan region
   MatDesc* mats;
   CUtensorMap* tmaps;

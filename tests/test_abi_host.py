@@ -88,3 +88,21 @@ def test_update_rejects_bad_source_combinations(L):
     assert L.smuon_update(W, 1, None, None, None, 1, 0.01, 0, 0, None, None, None) == -1
     assert L.smuon_update(W, 1, W, W, None, 1, 0.01, 0, 0, None, None, None) == -1
     assert L.smuon_update(W, 1, W, None, None, 1, 0.01, 0, 7, None, None, None) == -1
+
+
+def test_gradient_streams_reject_bad_arguments_before_launch(L):
+    import matrix_aware_sign_b200 as S
+    G = (S.SmuonMat * 2)(S.SmuonMat(4096, 8, 8, 8, S.F32), S.SmuonMat(4096, 8, 8, 8, S.BF16))
+    gs = S.GradStream(0, 0, 1.0, 0)
+    assert L.smuon_harness_gaussian(None, 1, 1, ctypes.byref(gs), 1, None) == -1
+    assert L.smuon_harness_gaussian(G, 1, 1, None, 1, None) == -1
+    assert L.smuon_harness_gaussian(G, 0, 1, ctypes.byref(gs), 1, None) == -1
+    assert L.smuon_harness_gaussian(G, 1, 2, ctypes.byref(gs), 1, None) == -3  # the second is not F32
+    # a LionMuon step without gradients needs a stream in its state
+    W = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 8, 8, S.F32))
+    mom = (S.SmuonMat * 1)(S.SmuonMat(8192, 8, 8, 8, S.F32))
+    st = S.LionMuonState(1, 1, W, mom, 0, None)
+    assert L.lionmuon_step(ctypes.byref(st), 4, 0.9, 0.99, 0.01, 1.5, -0.5, 0.0, 5, 0, 0, None, None, 0, None,
+                           None) == -1
+    assert b"no gradient stream" in L.smuon_last_error()
+    assert st.t == 0

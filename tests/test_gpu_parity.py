@@ -473,3 +473,163 @@ def test_nan_outputs_vote_negative():
     v = O.vote_from_signs([O.sign_extract(u) for u in U])
     assert v[2, 5] == -1
     np.testing.assert_array_equal(host(Wd[0]), O.update_with_vote(W, v, 0.5, "f32"))
+
+
+@pytest.mark.parametrize("kind", [S.VOTE_POPCOUNT, S.VOTE_INT8])
+@pytest.mark.parametrize("M,with_packed,with_votes", [(1, True, False), (5, False, False), (8, True, True),
+                                                      (64, True, True), (7, False, True)])
+def test_fused_vote_update_bf16_many_layers(kind, M, with_packed, with_votes):
+    """bf16 outputs, 16 entries per lane: many ragged layers in one call (more
+    than one launch once the sources pass the table size), zeros of both signs
+    and NaNs, with and without the packed message and the vote output."""
+    rng = np.random.default_rng(M)
+    shapes = [(int(rng.integers(1, 90)), int(rng.integers(1, 200))) for _ in range(70 if M <= 8 else 6)]
+    shapes[0] = (512, 768)  # several warps and CTAs on one layer
+    W = WL.weights(shapes, "normal002", "bf16")
+    Wd = [dev(w, torch.bfloat16) for w in W]
+    U = []
+    for i, s in enumerate(shapes):
+        layer = WL.synthetic_polar_outputs(s, M, seed=100 + i, dtype="bf16", zero_fraction=0.03)
+        for k, u in enumerate(layer):
+            flat = u.reshape(-1)
+            flat[rng.integers(0, flat.size, 3)] = -0.0
+            if (i + k) % 5 == 0:
+                flat[rng.integers(0, flat.size)] = np.nan
+        U.append(layer)
+    Ud = [[dev(u, torch.bfloat16) for u in layer] for layer in U]
+    packed = [torch.full((M, S.packed_words(r * c)), 0x5A5A, dtype=torch.int32, device="cuda")
+              for r, c in shapes] if with_packed else None
+    votes = [torch.full((r * c,), 9, dtype=torch.int8, device="cuda") for r, c in shapes] if with_votes else None
+    S.smuon_update(Wd, 0.02, U=Ud, M=M, tie_value=1, vote_kind=kind, packed_out=packed, vote_out=votes)
+    torch.cuda.synchronize()
+    for i, s in enumerate(shapes):
+        signs = [O.sign_extract(u) for u in U[i]]
+        v = O.vote_from_signs(signs, 1)
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, 0.02, "bf16"))
+        if with_votes:
+            np.testing.assert_array_equal(host(votes[i]).reshape(s), v)
+        if with_packed:
+            for k in range(M):
+                np.testing.assert_array_equal(packed[i][k].cpu().numpy().view(np.uint32), O.pack_bits(signs[k]))
+
+
+def test_fused_vote_update_bf16_strided():
+    """bf16 outputs whose rows are strided take the entry-by-entry path of the
+    16-entry kernel; the packed message is still the dense bit layout."""
+    M, shape = 6, (37, 50)
+    W = WL.weights([shape], "normal002", "bf16")[0]
+    Wd = dev(W, torch.bfloat16)
+    U = WL.synthetic_polar_outputs(shape, M, seed=5, dtype="bf16", zero_fraction=0.05)
+    Ubig = [torch.zeros((37, 72), dtype=torch.bfloat16, device="cuda") for _ in range(M)]
+    for k in range(M):
+        Ubig[k][:, :50] = dev(U[k], torch.bfloat16)
+    packed = torch.zeros((M, S.packed_words(37 * 50)), dtype=torch.int32, device="cuda")
+    S.smuon_update([Wd], 0.01, U=[[u[:, :50] for u in Ubig]], M=M, packed_out=[packed])
+    torch.cuda.synchronize()
+    signs = [O.sign_extract(u) for u in U]
+    v = O.vote_from_signs(signs)
+    np.testing.assert_array_equal(host(Wd), O.update_with_vote(W, v, 0.01, "bf16"))
+    for k in range(M):
+        np.testing.assert_array_equal(packed[k].cpu().numpy().view(np.uint32), O.pack_bits(signs[k]))
+
+
+# ------------------------------------------------------------------ counter-based gradient streams
+from workloads import counter_rng as CR  # noqa: E402
+
+
+def test_harness_gaussian_matches_the_stream_definition_bit_for_bit():
+    """The in-kernel draws equal the float32 stream definition computed on
+    the host, for ragged, strided and multi-launch (more than 64 matrices) calls."""
+    shapes = [(1, 1), (7, 13), (64, 147), (300, 130)] + [(3, 5)] * 30
+    M = 3
+    gs = S.GradStream(11, 40, 0.25, 0)
+    G, views = [], []
+    for r, c in shapes:
+        for k in range(M):
+            big = torch.full((r, c + 9), 7.0, device="cuda")
+            G.append(big)
+            views.append(big[:, :c] if (r * c) % 2 else big[:, :c].contiguous())
+    S.smuon_harness_gaussian(views, M, gs, step=6)
+    torch.cuda.synchronize()
+    for l, s in enumerate(shapes):
+        for k in range(M):
+            ref = CR.gaussian_matrix(11, k, 40 + l, 6, s, 0.25)
+            np.testing.assert_array_equal(views[l * M + k].cpu().numpy(), ref)
+    # strided views leave the padding alone
+    assert torch.all(G[M * 1][:, 13:] == 7.0)
+
+
+def test_lionmuon_with_in_kernel_gradients():
+    """G = None: every step draws the workers' gradients from the streams
+    (step t + 1). Sign steps and the EMA stay bit-exact against the oracle fed
+    with the same streams; the Muon step's direction within tolerance."""
+    shapes, M, P = [(64, 96), (96, 64), (33, 17)], 5, 3
+    W = WL.weights(shapes, "normal002", "bf16")
+    mom = [[np.zeros(s, np.float32) for _ in range(M)] for s in shapes]
+    Wd = [dev(w, torch.bfloat16) for w in W]
+    md = [[dev(x) for x in layer] for layer in mom]
+    gs = S.GradStream(500, 7, 1.0, 0)
+    opt = S.LionMuon(Wd, md, grad=gs)
+    eta = 3e-3
+    ws = S.workspace(opt.workspace_bytes(5, S.NS_SPLIT_BF16))
+    for t in range(1, 5):
+        S.lionmuon_step(opt, None, P, 0.9, 0.99, eta, *WL.QUINTIC, 5, ns_flags=S.NS_SPLIT_BF16, ws=ws)
+        torch.cuda.synchronize()
+        G = [[CR.gaussian_matrix(500, k, 7 + l, t, s, 1.0) for k in range(M)] for l, s in enumerate(shapes)]
+        Wprev = [w.copy() for w in W]
+        kind, W, mom = O.lionmuon_step(t, W, mom, G, P, 0.9, 0.99, eta, WL.QUINTIC, 5, "bf16")
+        assert kind == ("muon" if t % P == 0 else "sign")
+        for l in range(len(shapes)):
+            for k in range(M):
+                np.testing.assert_array_equal(host(md[l][k]), mom[l][k])
+            if kind == "sign":
+                np.testing.assert_array_equal(host(Wd[l]), W[l])
+            else:  # bf16 weights: compare the applied steps where both sides moved
+                moved = np.mean(host(Wd[l]) != W[l])
+                assert moved < 0.05
+                W[l] = host(Wd[l]).astype(np.float32)  # continue from the GPU's weights
+    assert opt.t == 4
+
+
+def test_lionmuon_special_cases_p1_and_equal_betas():
+    """P = 1: every step is a Muon step (dense update along the worker-mean
+    direction). P = 0 with beta1 = beta2: sign steps only, G_hat is the EMA
+    itself (Signum with a vote), bit-exact."""
+    shapes, M = [(48, 80), (80, 48)], 3
+    W = WL.weights(shapes, "normal002", "f32")
+    rng = np.random.default_rng(9)
+    # P = 1
+    mom = [[np.zeros(s, np.float32) for _ in range(M)] for s in shapes]
+    Wd = [dev(w) for w in W]
+    md = [[dev(x) for x in layer] for layer in mom]
+    opt = S.LionMuon(Wd, md)
+    Wc = [w.copy() for w in W]
+    for t in (1, 2):
+        G = [[rng.standard_normal(s).astype(np.float32) for _ in range(M)] for s in shapes]
+        S.lionmuon_step(opt, [[dev(g) for g in layer] for layer in G], 1, 0.9, 0.99, 1e-2, *WL.QUINTIC, 5,
+                        ns_flags=S.NS_SPLIT_BF16)
+        torch.cuda.synchronize()
+        Wprev = [w.copy() for w in Wc]
+        kind, Wc, mom = O.lionmuon_step(t, Wc, mom, G, 1, 0.9, 0.99, 1e-2, WL.QUINTIC, 5, "f32")
+        assert kind == "muon"
+        for l in range(len(shapes)):
+            for k in range(M):
+                np.testing.assert_array_equal(host(md[l][k]), mom[l][k])
+            d_gpu = (host(Wd[l]).astype(np.float64) - Wprev[l]) / -1e-2
+            d_ref = (Wc[l].astype(np.float64) - Wprev[l]) / -1e-2
+            assert rel_fro(d_gpu, d_ref) < 1e-2
+            Wc[l] = host(Wd[l]).astype(np.float32)
+    # P = 0, beta1 = beta2
+    mom = [[np.zeros(s, np.float32) for _ in range(M)] for s in shapes]
+    Wd = [dev(w) for w in W]
+    md = [[dev(x) for x in layer] for layer in mom]
+    opt = S.LionMuon(Wd, md)
+    Wc = [w.copy() for w in W]
+    for t in (1, 2, 3):
+        G = [[rng.standard_normal(s).astype(np.float32) for _ in range(M)] for s in shapes]
+        S.lionmuon_step(opt, [[dev(g) for g in layer] for layer in G], 0, 0.9, 0.9, 1e-2, *WL.QUINTIC, 5)
+        kind, Wc, mom = O.lionmuon_step(t, Wc, mom, G, 0, 0.9, 0.9, 1e-2, WL.QUINTIC, 5, "f32")
+        assert kind == "sign"
+    torch.cuda.synchronize()
+    for l in range(len(shapes)):
+        np.testing.assert_array_equal(host(Wd[l]), Wc[l])
