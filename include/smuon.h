@@ -340,9 +340,17 @@ smuon_status smuon_harness_gaussian(const smuon_mat* G, int32_t n_layers, int32_
  *  G[n_layers*M]            F32 gradients (worker-minor), or NULL to draw them in-kernel from
  *                           st->grad (see smuon_harness_gaussian; no gradient bytes are read)
  *  ns_flags                 SMUON_NS_* flags of the Muon steps' Newton-Schulz call
- *                           (e.g. SMUON_NS_SPLIT_BF16)
+ *                           (e.g. SMUON_NS_SPLIT_BF16), plus optionally
+ *                           SMUON_LION_MUON_VOTE: the other reading of a Muon step
+ *                           with M workers -- every worker orthogonalises its own
+ *                           G_hat and the step is a Sign-Muon step, W -= eta *
+ *                           vote(sign(NS(G_hat^(m)))) (SignMuon summary, flow
+ *                           steps 2-5, applied to G_hat); M x n_layers Newton-Schulz
+ *                           problems instead of n_layers, and a larger workspace
  * Workers 1..64.
  * ---------------------------------------------------------------------- */
+#define SMUON_LION_MUON_VOTE 0x100u
+
 typedef struct {
   int32_t                  n_layers;
   int32_t                  workers;

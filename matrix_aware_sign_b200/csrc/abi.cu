@@ -479,6 +479,9 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     h.sched_off[st] = sched_off[st];
     h.sched_boff[st] = sched_boff[st];
     h.sched_ctas[st] = 0;
+    h.max_k[st] = 0;
+    for (const GroupDesc& g : B->groups)
+      h.max_k[st] = std::max(h.max_k[st], (st == ST_GRAM || st == ST_PROBE) ? g.n : g.m);
   }
   h.groups = B->ptr_at<GroupDesc>(L.off_groups);
   h.mats = B->ptr_at<MatDesc>(L.off_mats);
@@ -1170,33 +1173,47 @@ smuon_status cachemuon_reuse_probe(const smuon_mat* Q, const smuon_mat* M_t, con
 }
 
 // LionMuon workspace: the mean buffers and directions of a Muon step, then the NS workspace
-static smuon_status lion_layout(const lionmuon_state* st, int32_t iters, uint32_t ns_flags, size_t* mean_off, size_t* dir_off,
-                                size_t* ns_off, size_t* total, std::vector<smuon_mat>* means,
+// LionMuon Muon-step workspace. Mean reading: per layer the f32 mean of G_hat
+// and the f32 direction, then the Newton-Schulz workspace of n_layers
+// problems. Vote reading (SMUON_LION_MUON_VOTE): per layer the M workers' f32
+// G_hat back to back (worker k at k * rows * cols), per (layer, worker) a bf16
+// polar factor, then the workspace of n_layers * M problems. `means` and
+// `dirs` are the Newton-Schulz inputs and outputs (worker-minor in the vote reading).
+static smuon_status lion_layout(const lionmuon_state* st, int32_t iters, uint32_t ns_flags, size_t* mean_off,
+                                size_t* dir_off, size_t* ns_off, size_t* total, std::vector<smuon_mat>* means,
                                 std::vector<smuon_mat>* dirs, char* base) {
+  const bool vote = (ns_flags & SMUON_LION_MUON_VOTE) != 0;
+  const int per = vote ? st->workers : 1;
   size_t cur = 0;
   means->clear();
   dirs->clear();
   *mean_off = 0;
   for (int l = 0; l < st->n_layers; ++l) {
     const smuon_mat& w = st->W[l];
-    smuon_mat m{};
-    m.rows = w.rows; m.cols = w.cols; m.ld = w.cols; m.dtype = SMUON_F32;
-    m.data = base ? base + cur : nullptr;
-    cur = (size_t)round_up((int64_t)(cur + (size_t)w.rows * w.cols * 4), 256);
-    means->push_back(m);
+    for (int k = 0; k < per; ++k) {
+      smuon_mat m{};
+      m.rows = w.rows; m.cols = w.cols; m.ld = w.cols; m.dtype = SMUON_F32;
+      m.data = base ? base + cur : nullptr;
+      cur += (size_t)w.rows * w.cols * 4;
+      means->push_back(m);
+    }
+    cur = (size_t)round_up((int64_t)cur, 256);
   }
   *dir_off = cur;
   for (int l = 0; l < st->n_layers; ++l) {
     const smuon_mat& w = st->W[l];
-    smuon_mat d{};
-    d.rows = w.rows; d.cols = w.cols; d.ld = w.cols; d.dtype = SMUON_F32;
-    d.data = base ? base + cur : nullptr;
-    cur = (size_t)round_up((int64_t)(cur + (size_t)w.rows * w.cols * 4), 256);
-    dirs->push_back(d);
+    for (int k = 0; k < per; ++k) {
+      smuon_mat d{};
+      d.rows = w.rows; d.cols = w.cols; d.ld = w.cols; d.dtype = vote ? SMUON_BF16 : SMUON_F32;
+      d.data = base ? base + cur : nullptr;
+      cur = (size_t)round_up((int64_t)(cur + (size_t)w.rows * w.cols * dtype_size(d.dtype)), 256);
+      dirs->push_back(d);
+    }
   }
   *ns_off = cur;
   size_t ns_bytes = 0;
-  smuon_status s = smuon_ns_workspace_bytes(means->data(), st->n_layers, iters, ns_flags, &ns_bytes);
+  smuon_status s = smuon_ns_workspace_bytes(means->data(), (int32_t)means->size(), iters,
+                                            ns_flags & ~SMUON_LION_MUON_VOTE, &ns_bytes);
   if (s != SMUON_OK) return s;
   *total = cur + ns_bytes;
   return SMUON_OK;
@@ -1261,6 +1278,9 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
   if (P < 0) return fail(SMUON_ERR_INVALID_ARG, "P must be >= 0 (0 = never a Muon step)");
   if (tie_value < -1 || tie_value > 1) return fail(SMUON_ERR_INVALID_ARG, "tie_value must be -1, 0 or 1");
   if (iters < 1 || iters > 64) return fail(SMUON_ERR_INVALID_ARG, "iters must be in 1..64");
+  if (ns_flags & SMUON_NS_EMIT_Q) return fail(SMUON_ERR_INVALID_ARG, "ns_flags may not ask for SMUON_NS_EMIT_Q");
+  if ((ns_flags & SMUON_LION_MUON_VOTE) && (int64_t)st->n_layers * M > 4096)
+    return fail(SMUON_ERR_UNSUPPORTED, "the vote reading orthogonalises n_layers * workers <= 4096 matrices");
   smuon_status s;
   EwBuild eb;
   for (int l = 0; l < st->n_layers; ++l) {
@@ -1329,13 +1349,15 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
   char* base = reinterpret_cast<char*>(ws);
   if ((s = lion_layout(st, iters, ns_flags, &mean_off, &dir_off, &ns_off, &total, &means, &dirs, base)) != SMUON_OK)
     return s;
+  const bool vote = (ns_flags & SMUON_LION_MUON_VOTE) != 0;
   for (int l = 0; l < st->n_layers; ++l) {
-    eb.layers[l].aux = means[l].data;
+    eb.layers[l].aux = means[(size_t)l * (vote ? M : 1)].data;
     eb.layers[l].vec_aux = (eb.layers[l].vec != 0);
   }
+  proto.ghat_out = vote ? 1 : 0;
   s = for_each_ew_launch(eb, proto, [&](const EwTable& tb) -> smuon_status {
     double n = 0;
-    for (int l = 0; l < tb.n_layers; ++l) n += (double)tb.layers[l].n * ((8.0 + g_bytes) * M + 4.0);
+    for (int l = 0; l < tb.n_layers; ++l) n += (double)tb.layers[l].n * ((8.0 + g_bytes) * M + (vote ? 4.0 * M : 4.0));
     Launch L("k_lion_mean", SMUON_WORK_BYTES, n, strm);
     k_lion_mean<<<ew_grid(tb.total_chunks, di), 256, 0, strm>>>(tb);
     CUDA_TRY(cudaGetLastError());
@@ -1343,12 +1365,15 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
   });
   if (s != SMUON_OK) return s;
   NsRequest rq{};
-  rq.M_in = means.data(); rq.U_out = dirs.data(); rq.n_mats = st->n_layers; rq.iters = iters;
-  rq.a = a; rq.b = b; rq.c = c; rq.eps = 1e-7f; rq.flags = ns_flags;
-  if (ns_flags & SMUON_NS_EMIT_Q) return fail(SMUON_ERR_INVALID_ARG, "ns_flags may not ask for SMUON_NS_EMIT_Q");
+  rq.M_in = means.data(); rq.U_out = dirs.data(); rq.n_mats = (int32_t)means.size(); rq.iters = iters;
+  rq.a = a; rq.b = b; rq.c = c; rq.eps = 1e-7f; rq.flags = ns_flags & ~SMUON_LION_MUON_VOTE;
   if ((s = validate_ns(rq)) != SMUON_OK) return s;
   if ((s = enqueue_ns(rq, base + ns_off, total - ns_off, d_status, nullptr, strm)) != SMUON_OK) return s;
-  s = smuon_update(st->W, st->n_layers, nullptr, nullptr, dirs.data(), 1, eta, 0, 0, nullptr, nullptr, stream);
+  if (vote)  // Sign-Muon step on the orthogonalised G_hat: fused sign / popcount vote / update
+    s = smuon_update(st->W, st->n_layers, dirs.data(), nullptr, nullptr, M, eta, tie_value, SMUON_VOTE_POPCOUNT,
+                     nullptr, nullptr, stream);
+  else
+    s = smuon_update(st->W, st->n_layers, nullptr, nullptr, dirs.data(), 1, eta, 0, 0, nullptr, nullptr, stream);
   if (s != SMUON_OK) return s;
   st->t = t_next;
   return SMUON_OK;

@@ -808,7 +808,9 @@ __global__ void __launch_bounds__(256) k_lion_sign(const __grid_constant__ EwTab
 }
 
 // LionMuon Muon step prologue (reading R11): mean over workers of G_hat into a
-// contiguous f32 buffer, and the EMA update of every worker.
+// contiguous f32 buffer, and the EMA update of every worker. With ghat_out (the
+// vote reading of the Muon step) every worker's G_hat is written instead, to
+// the contiguous f32 block aux + k * n.
 __global__ void __launch_bounds__(256) k_lion_mean(const __grid_constant__ EwTable tb) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const float invM = 1.f / (float)tb.M;
@@ -830,14 +832,17 @@ __global__ void __launch_bounds__(256) k_lion_mean(const __grid_constant__ EwTab
         crng::gaussian8(tb.gen_seed + (uint32_t)wk, L.key1, tb.gen_step, e0, tb.gen_sigma, gr);
       else
         load8(Gs.ptr, Gs.ld, SMUON_F32, L, e0, L.vec, gr);
+      float gh[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float gh = __fadd_rn(__fmul_rn(tb.beta1, mo[k]), __fmul_rn(tb.c1, gr[k]));
-        acc[k] = __fadd_rn(acc[k], gh);
+        gh[k] = __fadd_rn(__fmul_rn(tb.beta1, mo[k]), __fmul_rn(tb.c1, gr[k]));
+        acc[k] = __fadd_rn(acc[k], gh[k]);
         mo[k] = __fadd_rn(__fmul_rn(tb.beta2, mo[k]), __fmul_rn(tb.c2, gr[k]));
       }
       store8(const_cast<void*>(S.ptr), S.ld, SMUON_F32, L, e0, L.vec, mo);
+      if (tb.ghat_out) store8(reinterpret_cast<float*>(L.aux) + (int64_t)wk * L.n, L.cols, SMUON_F32, L, e0, L.vec_aux, gh);
     }
+    if (tb.ghat_out) continue;
 #pragma unroll
     for (int k = 0; k < 8; ++k) acc[k] = __fmul_rn(acc[k], invM);
     // the mean buffer is contiguous (ld == cols) f32 in the workspace

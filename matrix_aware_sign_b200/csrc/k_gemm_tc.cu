@@ -31,14 +31,17 @@ constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
 // plain BF16: one hi tile per operand; split BF16: hi and lo tiles per operand
 // (x = x_hi + x_lo, product ~ A_hi B_hi + A_hi B_lo + A_lo B_hi).
 // kBN = 128 in split mode, 256 in plain mode (the symmetric stages then use
-// 128 x 256 tiles over the triangle, the others a full grid).
-template <bool kSplit, int kBN>
+// 128 x 256 tiles over the triangle, the others a full grid). The ring takes
+// 192 KB of shared memory, or about 144 KB (kShallow) for stages whose K is
+// short: a tile then needs few k-blocks in flight, and the shared memory left
+// to the L1 cache serves the epilogue's row-per-lane global accesses.
+template <bool kSplit, int kBN, bool kShallow>
 struct Cfg {
   static constexpr int PARTS = kSplit ? 2 : 1;
   static constexpr int BN = kBN;
   static constexpr int B_BYTES = kBN * BK * 2;
   static constexpr int STAGE_BYTES = PARTS * (A_BYTES + B_BYTES);
-  static constexpr int STAGES = (192 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = ((kShallow ? 144 : 192) * 1024) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * kBN;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
@@ -179,9 +182,9 @@ __device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, i
   return o;
 }
 
-template <bool kSplit, int kBN>
+template <bool kSplit, int kBN, bool kShallow>
 __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int iter) {
-  using C = Cfg<kSplit, kBN>;
+  using C = Cfg<kSplit, kBN, kShallow>;
   constexpr int STAGES = C::STAGES;
   constexpr int STAGE_BYTES = C::STAGE_BYTES;
   constexpr int PARTS = C::PARTS;
@@ -365,28 +368,36 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
 }
 
-template <bool kSplit, int kBN>
+template <bool kSplit, int kBN, bool kShallow>
 __global__ void __launch_bounds__(THREADS, 1) k_gemm_tc(const Plan* plan, int stage, int iter, const int32_t* skip) {
   if (skip && *skip) return;
-  gemm_tc_body<kSplit, kBN>(plan, stage, iter);
+  gemm_tc_body<kSplit, kBN, kShallow>(plan, stage, iter);
 }
 
 }  // namespace tc
 
-template <bool kSplit, int kBN>
+template <bool kSplit, int kBN, bool kShallow>
 static cudaError_t launch_tc_variant(const Plan* d_plan, int stage, int iter, const int32_t* skip, int grid,
                                      cudaStream_t s) {
+  using C = tc::Cfg<kSplit, kBN, kShallow>;
   static bool attr_set[256] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 256 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc<kSplit, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         tc::Cfg<kSplit, kBN>::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc<kSplit, kBN, kShallow>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  tc::k_gemm_tc<kSplit, kBN><<<grid, tc::THREADS, tc::Cfg<kSplit, kBN>::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
+  tc::k_gemm_tc<kSplit, kBN, kShallow><<<grid, tc::THREADS, C::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
   return cudaGetLastError();
+}
+
+template <bool kSplit, int kBN>
+static cudaError_t launch_tc_depth(const PlanHeader& h, const Plan* d_plan, int stage, int iter,
+                                   const int32_t* skip, int grid, cudaStream_t s) {
+  if (h.max_k[stage] <= kShallowMaxK) return launch_tc_variant<kSplit, kBN, true>(d_plan, stage, iter, skip, grid, s);
+  return launch_tc_variant<kSplit, kBN, false>(d_plan, stage, iter, skip, grid, s);
 }
 
 int tc_tile_n(int stage, uint32_t flags) {
@@ -400,9 +411,9 @@ cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, i
   const int grid = h.sched_ctas[stage];
   if (h.total_tiles[stage] == 0 || grid <= 0) return cudaSuccess;
   const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && stage <= ST_QAXPY;
-  if (split) return launch_tc_variant<true, 128>(d_plan, stage, iter, skip, grid, s);
-  if (tc_tile_n(stage, h.flags) == 128) return launch_tc_variant<false, 128>(d_plan, stage, iter, skip, grid, s);
-  return launch_tc_variant<false, 256>(d_plan, stage, iter, skip, grid, s);
+  if (split) return launch_tc_depth<true, 128>(h, d_plan, stage, iter, skip, grid, s);
+  if (tc_tile_n(stage, h.flags) == 128) return launch_tc_depth<false, 128>(h, d_plan, stage, iter, skip, grid, s);
+  return launch_tc_depth<false, 256>(h, d_plan, stage, iter, skip, grid, s);
 }
 
 }  // namespace smuon

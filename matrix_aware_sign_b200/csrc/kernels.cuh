@@ -48,6 +48,7 @@ struct EwTable {
   uint32_t gen_seed;       // key word 0 of worker k = gen_seed + k
   uint32_t gen_step;       // counter word 2
   float gen_sigma;
+  int32_t ghat_out;        // LionMuon vote-based Muon step: write each worker's G_hat (aux + k * n), no mean
   int64_t total_chunks;
   EwLayer layers[kEwMaxLayers];
   EwSrc srcs[kEwMaxSrcs];

@@ -18,6 +18,7 @@ namespace smuon {
 
 constexpr int kMaxWorkers = 64;
 constexpr int kMaxSchedCtas = 1024;  // most CTAs a tensor-core stage is scheduled over
+constexpr int kShallowMaxK = 1024;    // stages with K up to this use the shallow smem ring
 
 // Stages of the Newton-Schulz chain. Each is one grouped GEMM launch
 // D = A_op * B_op over every matrix of the batch, with its own epilogue.
@@ -98,6 +99,7 @@ struct PlanHeader {
   int32_t sched_off[ST_COUNT];      // offset of each stage's tile ids in sched
   int32_t sched_boff[ST_COUNT];     // offset of each stage's begin array in sched_begin
   int32_t sched_ctas[ST_COUNT];     // CTAs of each stage's launch
+  int32_t max_k[ST_COUNT];          // longest K of each stage over the groups (picks the smem ring depth)
   GroupDesc* groups;        // device pointers into the plan region
   MatDesc* mats;
   CUtensorMap* tmaps;

@@ -38,6 +38,8 @@ Readings where the pages are silent (each is listed in the design doc):
       subtraction, then one round-to-nearest-even to bf16 for bf16 weights.
       The dense form (local polar step, Muon step) is f32(W) - f32(f32(eta)*D).
   R11 LionMuon Muon steps orthogonalise the mean over workers of G_hat.
+      Alternative (muon_vote): each worker orthogonalises its own G_hat and
+      the Muon step votes on the signs, as a Sign-Muon step.
   R12 LionMuon EMA update M <- beta2*M + (1-beta2)*G after G_hat is formed.
   R13 Steps are 1-indexed; step t is a Muon step iff P > 0 and t % P == 0.
   R14 CacheMuon's cached left transform is Q = P_{K-1} ... P_1 P_0 with
@@ -333,12 +335,15 @@ def lion_ema(M: np.ndarray, G: np.ndarray, beta2: float) -> np.ndarray:
 
 
 def lionmuon_step(t, W_layers, M_layers, G_layers, period, beta1, beta2, eta, coeffs,
-                  iters, w_dtype, tie_value=0, eps=1e-7):
+                  iters, w_dtype, tie_value=0, eps=1e-7, muon_vote=False):
     """Step t (1-indexed) of LionMuon with M simulated workers.
 
     Muon step iff period > 0 and t % period == 0 ([LM] methodology item 1;
     reading R13): W <- W - eta * NS(mean_m G_hat^(m)) (reading R11, dense
-    update). Otherwise a Lion sign step: W <- W - eta * vote(sign(G_hat^(m)))
+    update). With muon_vote, the alternative reading of R11: every worker
+    orthogonalises its own G_hat^(m) and the Muon step is a Sign-Muon step,
+    W <- W - eta * vote(sign(NS(G_hat^(m)))) ([SM] flow steps 2-5 applied to
+    G_hat). Otherwise a Lion sign step: W <- W - eta * vote(sign(G_hat^(m)))
     ([LM] problem section; the vote follows [SM]). Both kinds then update the
     shared EMA (reading R12). Returns (kind, W list, M lists)."""
     a, b, c = coeffs
@@ -346,7 +351,11 @@ def lionmuon_step(t, W_layers, M_layers, G_layers, period, beta1, beta2, eta, co
     W_out, M_out = [], []
     for W, Ms, Gs in zip(W_layers, M_layers, G_layers):
         Gh = [lion_interpolate(Mm, Gm, beta1) for Mm, Gm in zip(Ms, Gs)]
-        if muon:
+        if muon and muon_vote:
+            U = [newton_schulz(g.astype(np.float64), a, b, c, iters, eps) for g in Gh]
+            v = vote_from_signs([sign_extract(u) for u in U], tie_value)
+            Wn = update_with_vote(W, v, eta, w_dtype)
+        elif muon:
             mean = np.mean(np.stack([g.astype(np.float64) for g in Gh]), axis=0)
             D = newton_schulz(mean, a, b, c, iters, eps)
             Wn = update_dense(W, D, eta, w_dtype)

@@ -633,3 +633,34 @@ def test_lionmuon_special_cases_p1_and_equal_betas():
     torch.cuda.synchronize()
     for l in range(len(shapes)):
         np.testing.assert_array_equal(host(Wd[l]), Wc[l])
+
+
+def test_lionmuon_vote_reading_of_the_muon_step():
+    """SMUON_LION_MUON_VOTE: every worker orthogonalises its own G_hat and the
+    Muon step votes on the signs. The EMA stays bit-exact; the voted update
+    agrees with the oracle except where a worker's polar factor is near zero."""
+    shapes, M = [(64, 96), (96, 64), (33, 40)], 3
+    W = WL.weights(shapes, "normal002", "f32")
+    mom = [[np.zeros(s, np.float32) for _ in range(M)] for s in shapes]
+    Wd = [dev(w) for w in W]
+    md = [[dev(x) for x in layer] for layer in mom]
+    opt = S.LionMuon(Wd, md)
+    flags = S.NS_SPLIT_BF16 | S.LION_MUON_VOTE
+    ws = S.workspace(opt.workspace_bytes(5, flags))
+    assert ws.numel() > S.LionMuon(Wd, md).workspace_bytes(5, S.NS_SPLIT_BF16)
+    rng = np.random.default_rng(12)
+    for t in (1, 2):
+        G = [[rng.standard_normal(s).astype(np.float32) for _ in range(M)] for s in shapes]
+        S.lionmuon_step(opt, [[dev(g) for g in layer] for layer in G], 2, 0.9, 0.99, 1e-2, *WL.QUINTIC, 5,
+                        tie_value=0, ns_flags=flags, ws=ws)
+        torch.cuda.synchronize()
+        kind, W, mom = O.lionmuon_step(t, W, mom, G, 2, 0.9, 0.99, 1e-2, WL.QUINTIC, 5, "f32", muon_vote=True)
+        for l in range(len(shapes)):
+            for k in range(M):
+                np.testing.assert_array_equal(host(md[l][k]), mom[l][k])
+            if kind == "sign":
+                np.testing.assert_array_equal(host(Wd[l]), W[l])
+            else:
+                assert np.mean(host(Wd[l]) != W[l]) < 2e-3
+                W[l] = host(Wd[l]).astype(np.float32)
+    assert opt.t == 2

@@ -358,3 +358,30 @@ def test_ns_flops_counts():
     assert O.ns_flops(256, 256, 5, 0.0) == 5 * 4 * 256 ** 3
     assert O.ns_flops(4096, 4096, 5, 2.0) == 5 * 6 * 4096 ** 3
     assert O.ns_flops(3072, 768, 1, 2.0) == 4 * 768 ** 2 * 3072 + 2 * 768 ** 3
+
+
+def test_lionmuon_muon_vote_is_sign_muon_on_g_hat():
+    """The vote reading of the Muon step: each worker's G_hat is orthogonalised
+    and the signs are voted. Written with the singular-value closed form of
+    the iteration and a direct count of the signs, independent of the oracle's
+    iteration and vote functions; three workers, odd count, so no ties."""
+    W, Gs = _lion_inputs(seed=31)
+    M = [[np.zeros(w.shape, np.float32) for _ in range(3)] for w in W]
+    kind, Wn, Mn = O.lionmuon_step(1, W, M, Gs[0], 1, 0.9, 0.99, 1e-3, WL.QUINTIC, 2, "f32", muon_vote=True)
+    assert kind == "muon"
+    for i, w in enumerate(W):
+        count = np.zeros(w.shape, np.int64)
+        for m in range(3):
+            gh = (np.float32(np.float32(1) - np.float32(0.9)) * Gs[0][i][m]).astype(np.float64)  # M = 0
+            U, S, Vt = np.linalg.svd(gh, full_matrices=False)
+            s = S / (np.sqrt(np.sum(S ** 2)) + 1e-7)
+            ns = (U * _poly(s, WL.QUINTIC, 2)) @ Vt
+            count += (ns >= 0)
+        v = np.where(2 * count > 3, 1, -1)
+        expect = (w.astype(np.float32) - np.float32(1e-3) * v.astype(np.float32)).astype(np.float32)
+        np.testing.assert_array_equal(Wn[i], expect)
+    # the EMA does not depend on the kind of step
+    _, _, Md = O.lionmuon_step(1, W, M, Gs[0], 1, 0.9, 0.99, 1e-3, WL.QUINTIC, 2, "f32")
+    for a, b in zip(Mn, Md):
+        for x, y in zip(a, b):
+            np.testing.assert_array_equal(x, y)
