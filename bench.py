@@ -57,9 +57,11 @@ def parse_args():
                    help="skip the extra 4096x4096 Newton-Schulz measurement")
     p.add_argument("--only-ns4096", action="store_true",
                    help="run only the 4096x4096 Newton-Schulz measurement (for profiling)")
-    p.add_argument("--workload", choices=["c2_resnet50", "c3_gpt2s", "c5_gpt2l"], default=WORKLOAD,
+    p.add_argument("--workload", choices=["c2_resnet50", "c3_gpt2s", "c5_gpt2l", "resnet18", "llama124m",
+                                          "llama355m", "llama720m"], default=WORKLOAD,
                    help="layer set: ResNet-50 Sign-Muon (default), GPT-2-small Sign-Muon (M=8, popcount vote, "
-                        "5 quintic steps), GPT-2-Large LionMuon (M=16, P=4)")
+                        "5 quintic steps), GPT-2-Large LionMuon (M=16, P=4); ResNet-18 with the ResNet-50 "
+                        "set's settings, LLaMA-style 124M/355M/720M sets with the GPT-2-small set's")
     p.add_argument("--ns-mode", choices=["plain", "split"], default=None,
                    help="Newton-Schulz operand precision (default: plain for one quintic step, split BF16 for "
                         "five, the mode that meets the 1e-2 tolerance there)")
@@ -381,7 +383,7 @@ def run_reference(args, rank):
 def default_ns_mode(args):
     if args.ns_mode:
         return args.ns_mode
-    return "plain" if args.workload == "c2_resnet50" else "split"
+    return "plain" if args.workload in ("c2_resnet50", "resnet18") else "split"
 
 
 def describe(name, ns_mode, local_polar):
@@ -390,6 +392,14 @@ def describe(name, ns_mode, local_polar):
                 "data": "synthetic (seeded Gaussian gradients N(0,1e-4), He-normal weights)"}
     if name == "c3_gpt2s":
         return {"workload": "gpt2_small_set_48_matrices_M8_quintic5_popcount_vote"
+                            + ("_local_polar" if local_polar else "") + f"_{ns_mode}_bf16",
+                "data": "synthetic (seeded Gaussian gradients N(0,1) drawn on the device, weights N(0,0.02^2) bf16)"}
+    if name == "resnet18":
+        return {"workload": "resnet18_conv_set_20_layers_M4_quintic1_int8_vote",
+                "data": "synthetic (seeded Gaussian gradients N(0,1e-4), He-normal weights)"}
+    if name.startswith("llama"):
+        n = len(WL.SIGN_MUON_WORKLOADS[name].shapes)
+        return {"workload": f"{name}_style_set_{n}_matrices_M8_quintic5_popcount_vote"
                             + ("_local_polar" if local_polar else "") + f"_{ns_mode}_bf16",
                 "data": "synthetic (seeded Gaussian gradients N(0,1) drawn on the device, weights N(0,0.02^2) bf16)"}
     return {"workload": f"gpt2_large_set_144_matrices_M16_lionmuon_P4_quintic5_{ns_mode}_bf16",
@@ -401,10 +411,10 @@ def subset(shapes, layers):
     return shapes[:layers] if layers > 0 else shapes
 
 
-def setup_c2(S, torch, rank, ns_flags, e2e, layers=0):
-    """ResNet-50 layer set, M = 4: momentum + one quintic NS step (prepared
+def setup_c2(S, torch, rank, ns_flags, e2e, layers=0, name="c2_resnet50"):
+    """ResNet layer sets, M = 4: momentum + one quintic NS step (prepared
     plans on two resident gradient sets) + fused sign / int8-sum vote / update."""
-    cfg = WL.SIGN_MUON_WORKLOADS["c2_resnet50"]
+    cfg = WL.SIGN_MUON_WORKLOADS[name]
     M, shapes = cfg.workers, subset(cfg.shapes, layers)
     L = len(shapes)
     W = WL.weights(shapes, cfg.w_init, cfg.w_dtype)
@@ -438,34 +448,42 @@ def setup_c2(S, torch, rank, ns_flags, e2e, layers=0):
 
     return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None,
             "g_bytes": n_params * M * 4, "w_bytes": n_params * 4,
+            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], ns_flags != 0, 2),
             "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters, "vote": "int8 sum",
-                       "l2": "inputs larger than L2: 375 MB of gradients per step, two resident sets alternate"}}
+                       "l2": f"inputs larger than L2: {n_params * M * 4 / 1e6:.0f} MB of gradients per step, "
+                             "two resident sets alternate"}}
 
 
-def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0):
+def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0, name="c3_gpt2s"):
     """GPT-2-small layer set, M = 8: momentum + five quintic NS steps (prepared
     plans on two resident gradient sets), then either the fused sign / 1-bit
     pack / popcount vote / update with the packed payload written out, or
     (local polar step) sign-pack + popcount vote, NS on the 48 voted matrices
     and the dense update."""
-    cfg = WL.SIGN_MUON_WORKLOADS["c3_gpt2s"]
+    cfg = WL.SIGN_MUON_WORKLOADS[name]
     M, shapes = cfg.workers, subset(cfg.shapes, layers)
     L = len(shapes)
     Wd = [torch.from_numpy(w).to(torch.bfloat16).cuda() for w in WL.weights(shapes, cfg.w_init, cfg.w_dtype)]
     gen = torch.Generator(device="cuda").manual_seed(rank_seed_base(rank) + 3)
+    n_params = sum(r * c for r, c in shapes)
+    # two resident gradient sets alternate while they are small; one set (and one
+    # workspace) once a set alone is far larger than L2
+    n_sets = 2 if n_params * M * 4 <= 4e9 else 1
     Gd = [[torch.randn(s, device="cuda", generator=gen) * cfg.grad_sigma for s in shapes for _ in range(M)]
-          for _ in range(2)]
+          for _ in range(n_sets)]
     Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
     Ud = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in shapes for _ in range(M)]
     Ul = [Ud[l * M:(l + 1) * M] for l in range(L)]
     nbytes = S.smuon_ns_workspace_bytes(Md, cfg.iters, ns_flags)
-    wss = [S.workspace(nbytes), S.workspace(nbytes)]
+    wss = [S.workspace(nbytes) for _ in range(n_sets)]
     ns_plans = [S.NsPlan(Md, Ud, *cfg.coeffs, cfg.iters, G=Gd[j], beta=cfg.beta, flags=ns_flags, ws=wss[j])
-                for j in range(2)]
+                for j in range(n_sets)]
     packed = [torch.zeros((M, S.packed_words(r * c)), dtype=torch.int32, device="cuda") for r, c in shapes]
+    vote_plan = None
     if not local_polar:
         upd = S.UpdatePlan(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_POPCOUNT,
                            packed_out=packed)
+        vote_plan = upd
 
         def tail():
             upd.run()
@@ -481,12 +499,11 @@ def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0):
                 S.smuon_vote(M, r * c, votes[l], packed=packed[l], tie_value=cfg.tie_value)
             polar.run()
             upd.run()
-    n_params = sum(r * c for r, c in shapes)
     ws_e2e = S.workspace(nbytes) if e2e else None
 
     def step(i, G=None):
         if G is None:
-            ns_plans[i & 1].run()
+            ns_plans[i % n_sets].run()
         else:
             S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G, beta=cfg.beta, flags=ns_flags, ws=ws_e2e)
         tail()
@@ -496,11 +513,15 @@ def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0):
         hostW = [torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for w in Wd]
         return hostG, [torch.empty_like(g) for g in Gd[0]], hostW, Wd
 
+    vote_bytes = n_params * (M * 2 + 2 * 2 + M / 8)
     return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None,
             "g_bytes": n_params * M * 4, "w_bytes": n_params * 2,
+            "vote_alone": (vote_plan, vote_bytes) if vote_plan is not None else None,
+            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], ns_flags != 0, 2),
             "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters,
                        "vote": "1-bit packed, popcount" + (", local polar step" if local_polar else ""),
-                       "l2": "inputs larger than L2: 2.7 GB of gradients per step, two resident sets alternate"}}
+                       "l2": f"inputs larger than L2: {n_params * M * 4 / 1e9:.1f} GB of gradients per step"
+                             + (", two resident sets alternate" if n_sets == 2 else "")}}
 
 
 def setup_c5(S, torch, rank, ns_flags, layers=0, grad_source="hbm", period=None, beta2=None):
@@ -564,6 +585,27 @@ def rollup(S, recs, peaks):
     return by, kernels, stage_detail
 
 
+def gemm_stage_bytes(shapes, workers, iters, c, split, u_bytes):
+    """Algorithmic HBM bytes per launch of each Newton-Schulz GEMM stage
+    (averaged over the iterations), from the shapes alone: every operand read
+    once, the epilogue's source read and its outputs written once. X is the
+    wide m x n form; operands are bf16 (hi and lo parts in split mode), masters
+    and A are f32; the first step's X source is the f32 momentum, the last
+    step writes U (u_bytes per entry)."""
+    op = 4 if split else 2
+    tot = {"gram": 0.0, "poly": 0.0, "axpy": 0.0}
+    for r, cc in shapes:
+        m, n = min(r, cc), max(r, cc)
+        for k in range(iters):
+            last = k == iters - 1
+            tot["gram"] += workers * (op * m * n + (4 * m * m + op * m * m if c != 0 else op * m * m))
+            if c != 0:
+                tot["poly"] += workers * (op * m * m + 4 * m * m + op * m * m)
+            out = u_bytes * m * n if last else (4 + op) * m * n
+            tot["axpy"] += workers * (op * m * m + op * m * n + 4 * m * n + out)
+    return {k: v / iters for k, v in tot.items()}
+
+
 def load_traffic(dom):
     """Per-launch DRAM bytes of a kernel from the committed ncu summary, valid
     only while the kernel's sources are the ones the counters were taken on."""
@@ -624,10 +666,11 @@ def main():
     ns_flags = S.NS_SPLIT_BF16 if ns_mode == "split" else 0
     desc = describe(args.workload, ns_mode, args.local_polar)
     e2e_on = args.e2e_steps > 0
-    if args.workload == "c2_resnet50":
-        wl = setup_c2(S, torch, rank, ns_flags, e2e_on, args.layers)
-    elif args.workload == "c3_gpt2s":
-        wl = setup_c3(S, torch, rank, ns_flags, e2e_on, args.local_polar, args.layers)
+    if args.workload in ("c2_resnet50", "resnet18"):
+        wl = setup_c2(S, torch, rank, ns_flags, e2e_on, args.layers, args.workload)
+    elif args.workload == "c3_gpt2s" or args.workload.startswith("llama"):
+        wl = setup_c3(S, torch, rank, ns_flags, e2e_on and args.workload == "c3_gpt2s", args.local_polar,
+                      args.layers, args.workload)
     else:
         wl = setup_c5(S, torch, rank, ns_flags, args.layers, args.grad_source, args.period, args.beta2)
     step = wl["step"]
@@ -682,6 +725,12 @@ def main():
     # --- roofline of the dominant kernel (from the library's event trace)
     peaks, peak_src = load_peaks()
     by, kernels, stage_detail = rollup(S, recs, peaks)
+    if "stage_bytes" in wl:  # the GEMM stages of small matrices move bytes more than flops: their HBM view
+        for name, d in stage_detail.items():
+            b = wl["stage_bytes"].get(name.split(".")[1])
+            if b and d["ms_per_launch"] > 0:
+                d["gbs_algorithmic"] = b / (d["ms_per_launch"] / 1e3) / 1e9
+                d["frac_of_hbm"] = d["gbs_algorithmic"] / peaks["hbm_gbs"]
     roofline = None
     if by:
         dom = max(by, key=lambda k: by[k]["ms"])
@@ -761,6 +810,24 @@ def main():
         summary["vote_kernel"] = vk[0]
         summary["vote_gbs"] = kernels[vk[0]]["achieved"]
         summary["vote_frac_of_hbm"] = kernels[vk[0]]["frac"]
+    if wl.get("vote_alone") and world == 1:
+        # the fused sign / pack / popcount vote / update timed alone (burst), next to its in-step rate above,
+        # which runs at the clocks the tensor-core stages leave under the power cap
+        plan, vb = wl["vote_alone"]
+        for _ in range(3):
+            plan.run()
+        torch.cuda.synchronize()
+        v0 = torch.cuda.Event(enable_timing=True)
+        v1 = torch.cuda.Event(enable_timing=True)
+        v0.record(stream)
+        for _ in range(20):
+            plan.run()
+        v1.record(stream)
+        torch.cuda.synchronize()
+        vms = v0.elapsed_time(v1) / 20
+        summary["vote_alone"] = {"ms_per_call": vms, "gbs": vb / (vms / 1e3) / 1e9,
+                                 "frac_of_hbm": vb / (vms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                                 "bytes_per_call": vb}
 
     if rank == 0:
         clocks = sampler.summary(t_wall0, t_wall1)

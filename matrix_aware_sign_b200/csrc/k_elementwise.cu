@@ -348,37 +348,40 @@ __device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
   return (((~le & ~w) | ~nz) >> 15) & 0x00010001u;
 }
 
-// int8 (integer-sum) vote on bf16 outputs: the count of positive signs of each
-// entry is accumulated two entries per 32-bit add (16-bit lanes), then
-// sum = 2 * count - M (the +-1 sum of the all-reduce variant). Each lane takes
-// two consecutive 8-entry chunks (16 entries, 16-byte loads per worker); layer
-// chunk ranges are multiples of 16 chunks, so a pair never straddles layers.
-__device__ __forceinline__ void vote_i8_finish16(const EwTable& tb, const EwLayer& L, int64_t e0,
-                                                 const uint32_t* cnt, float* w) {
-  int8_t v8[16];
+// vote and update of 8 entries e0..e0+7 from their 4 packed count words
+__device__ __forceinline__ void vote_finish8(const EwTable& tb, const EwLayer& L, int64_t e0, const uint32_t* cnt) {
+  // W is loaded only here, after the workers' loads: fewer live registers, so
+  // three CTAs fit per SM (more loads in flight hide more latency)
+  float w[8];
+  load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+  int8_t v8[8];
   // eta * v for v = +1, -1 and the tie value: exact products, chosen per entry
   const float up = tb.eta, down = -tb.eta, tied = tb.eta * (float)tb.tie;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
+  for (int k = 0; k < 8; ++k) {
     const int c2 = 2 * (int)((cnt[k >> 1] >> (16 * (k & 1))) & 0xffffu);
     v8[k] = (int8_t)(c2 > tb.M ? 1 : (c2 < tb.M ? -1 : tb.tie));
     w[k] = __fsub_rn(w[k], c2 > tb.M ? up : (c2 < tb.M ? down : tied));
   }
   store8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
-  store8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
   if (L.vote_out) {
     int8_t* dst = L.vote_out + e0;
-    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-      uint4 pk;
-      memcpy(&pk, v8, 16);
-      *reinterpret_cast<uint4*>(dst) = pk;
+    if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
+      uint2 pk;
+      memcpy(&pk, v8, 8);
+      *reinterpret_cast<uint2*>(dst) = pk;
     } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) dst[k] = v8[k];
+      for (int k = 0; k < 8; ++k) dst[k] = v8[k];
     }
   }
 }
 
+// int8 (integer-sum) vote on bf16 outputs: the count of positive signs of each
+// entry is accumulated two entries per 32-bit add (16-bit lanes), then
+// sum = 2 * count - M (the +-1 sum of the all-reduce variant). Each lane takes
+// two consecutive 8-entry chunks (16 entries, 16-byte loads per worker); layer
+// chunk ranges are multiples of 16 chunks, so a pair never straddles layers.
 __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -392,10 +395,7 @@ __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
     const int64_t e0 = (chunk - L.chunk_begin) * 8;
     if (!(active && e0 < L.n)) continue;
     if (L.vec && e0 + 16 <= L.n) {
-      float w[16];
       uint32_t cnt[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-      load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
-      load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
       for (int wk0 = 0; wk0 < M; wk0 += 4) {
         uint4 u[4][2];
 #pragma unroll
@@ -418,7 +418,8 @@ __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
             }
           }
       }
-      vote_i8_finish16(tb, L, e0, cnt, w);
+      vote_finish8(tb, L, e0, cnt);
+      vote_finish8(tb, L, e0 + 8, cnt + 4);
     } else {
       // ragged or strided layers: entry by entry
       const int nent = (int)min((int64_t)16, L.n - e0);
@@ -491,12 +492,7 @@ __device__ __forceinline__ void vote_update_bf16x16(const EwTable& tb) {
     const bool live = active && e0 < L.n;
     const bool fast = live && L.vec && e0 + 16 <= L.n;
     const int nent = live ? (int)min((int64_t)16, L.n - e0) : 0;
-    float w[16];
     uint32_t cnt[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    if (fast) {
-      load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
-      load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
-    }
     for (int wk0 = 0; wk0 < M; wk0 += 4) {
       uint4 u[4][2];
       if (fast) {
@@ -538,7 +534,8 @@ __device__ __forceinline__ void vote_update_bf16x16(const EwTable& tb) {
     }
     if (!live) continue;
     if (fast) {
-      vote_i8_finish16(tb, L, e0, cnt, w);
+      vote_finish8(tb, L, e0, cnt);
+      vote_finish8(tb, L, e0 + 8, cnt + 4);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) finish_pair_scalar(tb, L, e0 + 2 * i, nent - 2 * i, cnt[i]);
@@ -616,19 +613,19 @@ __global__ void __launch_bounds__(256) k_vote_update(const __grid_constant__ EwT
   vote_update_body<kPopcount, kBf16, MaskT>(tb);
 }
 
-__global__ void __launch_bounds__(256) k_vote_update_i8_bf16(const __grid_constant__ EwTable tb) {
+__global__ void __launch_bounds__(256, 3) k_vote_update_i8_bf16(const __grid_constant__ EwTable tb) {
   vote_update_int8_bf16(tb);
 }
 
-__global__ void __launch_bounds__(256) k_vote_update_bf16x16(const __grid_constant__ EwTable tb) {
+__global__ void __launch_bounds__(256, 3) k_vote_update_bf16x16(const __grid_constant__ EwTable tb) {
   vote_update_bf16x16(tb);
 }
 
 cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s) {
   const bool bf = tb.src_dtype == SMUON_BF16;
-  // 16 entries per lane; measured best with 2-4 resident CTAs per SM
+  // 16 entries per lane, three resident CTAs per SM (launch bounds), one wave
   const int64_t want16 = (tb.total_chunks + 511) / 512;
-  const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 4 * sms));
+  const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
   if (bf && (popcount || tb.any_packed) && tb.M <= kMaxWorkers) {
     k_vote_update_bf16x16<<<grid16, 256, 0, s>>>(tb);
     return cudaGetLastError();

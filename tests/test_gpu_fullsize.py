@@ -179,3 +179,43 @@ def test_lionmuon_gpt2_large_sampled():
     D_ref = O.newton_schulz(np.mean(np.stack([g.astype(np.float64) for g in gh]), 0), *cfg.coeffs, cfg.iters)
     W_ref = O.update_dense(Wprev_layer1, D_ref, cfg.eta, "bf16")
     assert np.mean(host(Wd[1]) != W_ref) < 0.05
+
+
+# ------------------------------------------------------------------ LLaMA-style sets
+@pytest.mark.parametrize("name", ["llama124m", "llama355m"])
+def test_llama_style_set_one_step_sampled(name):
+    """The LLaMA-style layer sets (same kernels, other shapes): one Sign-Muon
+    step in the accurate split-BF16 mode with the fused popcount vote; the
+    oracle follows one matrix of each distinct shape (all workers)."""
+    cfg = WL.SIGN_MUON_WORKLOADS[name]
+    M, shapes = cfg.workers, cfg.shapes
+    n_params = sum(r * c for r, c in shapes)
+    if _free_gb() < n_params * M * 4 * 5 / 2 ** 30 + 8:
+        pytest.skip("not enough device memory")
+    W = WL.weights(shapes, cfg.w_init, cfg.w_dtype)
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    Gd = [torch.randn(s, device="cuda", generator=gen) for s in shapes for _ in range(M)]
+    Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
+    Ud = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in shapes for _ in range(M)]
+    S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=Gd, beta=cfg.beta, flags=S.NS_SPLIT_BF16)
+    Wd = [dev(w, torch.bfloat16) for w in W]
+    packed = [torch.zeros((M, S.packed_words(r * c)), dtype=torch.int32, device="cuda") for r, c in shapes]
+    S.smuon_update(Wd, cfg.eta, U=[Ud[l * M:(l + 1) * M] for l in range(len(shapes))], M=M,
+                   packed_out=packed)
+    torch.cuda.synchronize()
+    pairs, n_dis, n_all = [], 0, 0
+    for l in (4, 5, 6):  # one matrix of each shape (d x d, h x d, d x h)
+        G = [Gd[l * M + k].cpu().numpy() for k in range(M)]
+        ref_u = [O.newton_schulz(g.astype(np.float64), *cfg.coeffs, cfg.iters) for g in G]
+        pairs += [(host(Ud[l * M + k]), ref_u[k]) for k in range(M)]
+        signs = [O.sign_extract(u) for u in ref_u]
+        v = O.vote_from_signs(signs, cfg.tie_value)
+        agree_w = host(Wd[l]) == O.update_with_vote(W[l], v, cfg.eta, "bf16")
+        n_dis += int((~agree_w).sum())
+        n_all += agree_w.size
+        # the packed message carries the oracle's signs wherever the vote inputs agree
+        for k in range(M):
+            bits = np.unpackbits(packed[l][k].cpu().numpy().view(np.uint8), bitorder="little")[:signs[k].size]
+            assert np.mean(bits.astype(np.int8) * 2 - 1 != signs[k].reshape(-1)) <= 1e-4
+    check_ns_outputs(pairs, 1e-2)
+    assert n_dis <= 1e-4 * n_all

@@ -258,8 +258,11 @@ def test_config1_full_step():
     np.testing.assert_array_equal(host(Wd[0])[agree], ref["W"][0][agree])
 
 
-def test_config2_resnet50_one_step():
-    cfg = WL.SIGN_MUON_WORKLOADS["c2_resnet50"]
+@pytest.mark.parametrize("name", ["c2_resnet50", "resnet18"])
+def test_resnet_sets_one_step(name):
+    """ResNet-50 (and the ResNet-18 set, same settings): one full step, every
+    layer and worker against the oracle."""
+    cfg = WL.SIGN_MUON_WORKLOADS[name]
     W = WL.weights(cfg.shapes, cfg.w_init, cfg.w_dtype)
     grads = WL.GradientStreams(cfg.shapes, cfg.workers, cfg.grad_sigma).next_step()
     Md = [torch.zeros(s, device="cuda") for s in cfg.shapes for _ in range(cfg.workers)]

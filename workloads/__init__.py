@@ -54,6 +54,40 @@ def gpt2_large_shapes() -> list[tuple[int, int]]:
     return [s for _ in range(36) for s in ((1280, 3840), (1280, 1280), (1280, 5120), (5120, 1280))]
 
 
+def resnet18_conv_shapes() -> list[tuple[int, int]]:
+    """The 20 convolution weights of ResNet-18 as C_out x (C_in*k_h*k_w) (the
+    vision run of the "CacheMuon" experiments): the 7x7 stem, then four stages
+    of two basic blocks (two 3x3 convolutions each) with 64, 128, 256, 512
+    channels, and a 1x1 projection in the first block of stages 2-4.
+    11,166,912 parameters."""
+    shapes = [(64, 3 * 7 * 7)]
+    c_in = 64
+    for stage, c in enumerate((64, 128, 256, 512)):
+        for blk in range(2):
+            shapes.append((c, c_in * 9))
+            shapes.append((c, c * 9))
+            if blk == 0 and stage > 0:
+                shapes.append((c, c_in))
+            c_in = c
+    return shapes
+
+
+# LLaMA-style decoder blocks at the 124M / 355M / 720M scales the "LionMuon"
+# summary trains at: per block the attention projections q, k, v, o (d x d)
+# and the gated MLP gate, up (h x d) and down (d x h). The pages give only the
+# parameter counts; the widths are a reading: GPT-2's d and depth at 124M and
+# 355M, d = 1536 with 24 blocks at 720M, and h = 8/3 d rounded up to a multiple
+# of 256. Embeddings are not matrices the optimizer orthogonalises here.
+LLAMA_DIMS = {"124m": (768, 12), "355m": (1024, 24), "720m": (1536, 24)}
+
+
+def llama_shapes(size: str) -> list[tuple[int, int]]:
+    d, layers = LLAMA_DIMS[size]
+    h = -(-(8 * d // 3) // 256) * 256
+    block = [(d, d)] * 4 + [(h, d), (h, d), (d, h)]
+    return [s for _ in range(layers) for s in block]
+
+
 @dataclass
 class SignMuonWorkload:
     name: str
@@ -80,6 +114,16 @@ SIGN_MUON_WORKLOADS = {
                                     "f32", "he", 1e-2, "int8", 0, False, 10),
     "c3_gpt2s": SignMuonWorkload("c3_gpt2s", gpt2_small_shapes(), 8, 0.95, QUINTIC, 5, 0.02, "bf16",
                                  "normal002", 1.0, "popcount", 0, True, 20),
+    # more layer sets for the same kernels: ResNet-18 with the ResNet-50 set's
+    # hyper-parameters, the LLaMA-style sets with the GPT-2-small set's
+    "resnet18": SignMuonWorkload("resnet18", resnet18_conv_shapes(), 4, 0.9, QUINTIC, 1, 0.02,
+                                 "f32", "he", 1e-2, "int8", 0, False, 10),
+    "llama124m": SignMuonWorkload("llama124m", llama_shapes("124m"), 8, 0.95, QUINTIC, 5, 0.02, "bf16",
+                                  "normal002", 1.0, "popcount", 0, False, 20),
+    "llama355m": SignMuonWorkload("llama355m", llama_shapes("355m"), 8, 0.95, QUINTIC, 5, 0.02, "bf16",
+                                  "normal002", 1.0, "popcount", 0, False, 20),
+    "llama720m": SignMuonWorkload("llama720m", llama_shapes("720m"), 8, 0.95, QUINTIC, 5, 0.02, "bf16",
+                                  "normal002", 1.0, "popcount", 0, False, 20),
 }
 
 
