@@ -76,6 +76,8 @@ def parse_args():
                    help="use only the first LAYERS matrices of the set (a smaller case for profiler captures)")
     p.add_argument("--local-polar", action="store_true",
                    help="GPT-2-small set: orthogonalise the voted matrix before the update")
+    p.add_argument("--gram-only", action="store_true",
+                   help="CacheMuon sweep: fresh solves iterated on the m x m Gram (SMUON_NS_GRAM_ONLY)")
     p.add_argument("--cachemuon", nargs="*", metavar="RxC:GAMMA",
                    help="CacheMuon sweep instead of the Sign-Muon step, e.g. 4096x4096:2 8192x8192:15 "
                         "(no value: the three large shapes x gamma in {2, 15}); --steps sets the schedule length")
@@ -257,7 +259,7 @@ def measure_ns_square(S, torch, peaks, n, iters, reps=10):
 
 
 # ------------------------------------------------------------------ CacheMuon sweep
-def run_cachemuon(S, torch, shape, gamma, steps, iters=5):
+def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False):
     """M_0 ~ N(0,1); M_{t+1} = M_t + 0.01 N(0,1); every step probes the cached
     transform on the device and runs the fresh solve only when the residual
     exceeds gamma. Reports the hit rate and the orthogonalisation flops saved
@@ -268,7 +270,8 @@ def run_cachemuon(S, torch, shape, gamma, steps, iters=5):
     gen = torch.Generator(device="cuda").manual_seed(4242)
     M = torch.randn(shape, device="cuda", generator=gen)
     D = torch.empty(shape, device="cuda")
-    cm = S.CacheMuon(M, D, gamma, WL.QUINTIC, iters)
+    cm = S.CacheMuon(M, D, gamma, WL.QUINTIC, iters,
+                     flags=S.NS_SPLIT_BF16 | (S.NS_GRAM_ONLY if gram_only else 0))
     noise = torch.empty_like(M)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -286,12 +289,15 @@ def run_cachemuon(S, torch, shape, gamma, steps, iters=5):
     f_muon = iters * (4 * m * m * n + 2 * m ** 3)
     f_q = (iters - 1) * 2 * m ** 3
     f_probe = 4 * m * m * n
+    # Gram-only fresh solve: X_0 X_0^T and Q_K X_0 once, per step A^2 and, but for the last, Q and two A updates
+    f_gram_only = 4 * m * m * n + iters * 2 * m ** 3 + (iters - 1) * 3 * 2 * m ** 3
     fresh = c["misses"]
-    cost = fresh * (f_muon + f_q) + c["probes"] * f_probe
+    cost = fresh * (f_gram_only if gram_only else f_muon + f_q) + c["probes"] * f_probe
     return {"workload": "cachemuon", "shape": list(shape), "gamma": gamma, "steps": steps,
             "hits": c["hits"], "misses": c["misses"], "hit_rate": c["hits"] / steps,
             "orth_flops_saved_vs_fresh": 1.0 - cost / (steps * f_muon),
-            "ms_per_step": ms / steps, "note": "momentum drift generated on the device inside the timed loop"}
+            "ms_per_step": ms / steps, "fresh_solve": "gram_only" if gram_only else "x_iteration",
+            "note": "momentum drift generated on the device inside the timed loop"}
 
 
 # ------------------------------------------------------------------ oracle timing of the other layer sets
@@ -648,7 +654,8 @@ def main():
         for case in cases:
             shp, gam = case.split(":")
             r, c = (int(x) for x in shp.split("x"))
-            print(json.dumps(run_cachemuon(S, torch, (r, c), float(gam), args.steps)), flush=True)
+            print(json.dumps(run_cachemuon(S, torch, (r, c), float(gam), args.steps, gram_only=args.gram_only)),
+                  flush=True)
         return
     if args.only_ns4096:
         peaks, _ = load_peaks()

@@ -126,6 +126,13 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
 #define SMUON_NS_NO_NORMALIZE  4u  /* skip the Frobenius normalisation (s = 1) */
 #define SMUON_NS_EMIT_Q        8u  /* also write the CacheMuon transform Q */
 #define SMUON_NS_SIMT_BF16    16u  /* diagnostic: BF16 operands on CUDA cores instead of tcgen05 */
+#define SMUON_NS_GRAM_ONLY    32u  /* CacheMuon fresh solve iterated on the m x m Gram ("Gram
+                                      Newton-Schulz", CacheMuon summary, method item 1): A_0 = X_0 X_0^T once,
+                                      then per step P_k = aI + bA_k + cA_k^2, Q_{k+1} = P_k Q_k and
+                                      A_{k+1} = P_k A_k P_k (= P_k^2 A_k; the P_k commute with A_k), and
+                                      finally U = Q_K X_0: 4 m^2 n once plus about 8 m^3 per step,
+                                      instead of 4 m^2 n + 4 m^3 per step; fewer flops when m < n. Needs
+                                      SMUON_NS_EMIT_Q, one matrix, c != 0 and the tensor-core modes */
 
 smuon_status smuon_ns_workspace_bytes(const smuon_mat* M_in, int32_t n_mats, int32_t iters,
                                       uint32_t flags, size_t* bytes);

@@ -248,8 +248,8 @@ void schedule_stage(const std::vector<GroupDesc>& groups, int st, int total, int
       const int tiles = sym_stage(st) ? sym_start(g.tiles_m[st], g.tiles_n[st], bn / kTcBM)
                                       : g.tiles_m[st] * g.tiles_n[st];
       const int K = (st == ST_GRAM || st == ST_PROBE) ? g.n : g.m;
-      const int No = (st == ST_AXPY || st == ST_REUSE) ? g.n : g.m;
-      const double kb = (double)((K + 63) / 64) * (split && st <= ST_QAXPY ? 3 : 1) * bn / 256.0;
+      const int No = wide_out_stage(st) ? g.n : g.m;
+      const double kb = (double)((K + 63) / 64) * (split && split_stage(st) ? 3 : 1) * bn / 256.0;
       const double fill = (double)g.m * No / ((double)g.tiles_m[st] * kTcBM * g.tiles_n[st] * bn);
       const double cost = kb + 8.0 * fill * bn / 256.0;
       for (int t = g.tile_begin[st]; t < g.tile_begin[st] + g.count * tiles; ++t) cost_tile.push_back({cost, t});
@@ -283,6 +283,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   const bool bf = (mode != MODE_SIMT_F32);
   const bool tc = (mode == MODE_TC_BF16);
   const bool emit_q = (rq.flags & SMUON_NS_EMIT_Q) && !rq.probe;
+  const bool gram_only = (rq.flags & SMUON_NS_GRAM_ONLY) && !rq.probe;
   const int K = rq.iters;
   const int BM = tc ? kTcBM : kSimtBM;
   const size_t esz = bf ? 2 : 4;
@@ -356,10 +357,11 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     for (int st = 0; st < ST_COUNT; ++st) {
       const bool sym = sym_stage(st);
       const int BN = BM * ratios[st];
-      const int No = (st == ST_AXPY || st == ST_REUSE) ? g.n : g.m;
+      const int No = wide_out_stage(st) ? g.n : g.m;
       g.tiles_m[st] = tmm;
       g.tiles_n[st] = ceil_div(No, BN);
       g.tile_begin[st] = totals[st];
+      if ((st == ST_AA1 || st == ST_AA2 || st == ST_QX) && !gram_only) continue;  // the Gram-only solve's own
       totals[st] += g.count * (sym ? sym_start(tmm, g.tiles_n[st], ratios[st]) : g.tiles_m[st] * g.tiles_n[st]);
     }
   }
@@ -389,15 +391,20 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   auto want_map = [&](int32_t& slot) { slot = L.n_tmaps++; };
   L.n_tmaps = 0;
   for (auto& g : B->groups) {
-    for (int i = 0; i < 2; ++i) { g.tm_x_k[i] = g.tm_x_mn[i] = g.tm_q_mn[i] = g.tm_x_kw[i] = -1; }
-    g.tm_a_k = g.tm_b_k = g.tm_uq_k = g.tm_a_kw = -1;
+    for (int i = 0; i < 2; ++i) { g.tm_x_k[i] = g.tm_x_mn[i] = g.tm_q_mn[i] = g.tm_x_kw[i] = g.tm_q_k[i] = -1; }
+    g.tm_a_k = g.tm_b_k = g.tm_uq_k = g.tm_a_kw = g.tm_t_k = g.tm_t_kw = -1;
     if (!tc) continue;
     const bool wide = tc_tile_n(ST_GRAM, rq.flags) == 256;
     if (!rq.probe) {
       want_map(g.tm_x_k[0]);
       want_map(g.tm_x_mn[0]);
       if (wide) want_map(g.tm_x_kw[0]);
-      if (K >= 2) {
+      if (gram_only) {  // T operand (right operand of B T) and Q_K as the left operand of Q_K X_0
+        want_map(g.tm_t_k);
+        if (wide) want_map(g.tm_t_kw);
+        want_map(g.tm_q_k[K & 1]);
+      }
+      if (K >= 2 && !gram_only) {
         want_map(g.tm_x_k[1]);
         want_map(g.tm_x_mn[1]);
         if (wide) want_map(g.tm_x_kw[1]);
@@ -429,24 +436,29 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     g.xop[1] = nullptr;
     g.xf[0] = g.xf[1] = nullptr;
     g.af = nullptr; g.aop = nullptr; g.bop = nullptr;
+    g.af2 = nullptr; g.aop2 = nullptr;
     g.qf[0] = g.qf[1] = nullptr; g.qop[0] = g.qop[1] = nullptr;
     if (rq.probe) {
       g.xop[1] = B->ptr_at<void>(B->take(nx * esz));
       continue;
     }
-    if (K >= 2) g.xop[1] = B->ptr_at<void>(B->take(nx * esz * parts));
-    if (bf && K >= 2) g.xf[1] = B->ptr_at<float>(B->take(nx * 4));
-    if (bf && K >= 3) g.xf[0] = B->ptr_at<float>(B->take(nx * 4));
+    if (gram_only) {  // no X iterates: T between the two updates of A instead
+      g.af2 = B->ptr_at<float>(B->take(nm * 4));
+      g.aop2 = B->ptr_at<void>(B->take(nm * 2 * parts));
+    }
+    if (K >= 2 && !gram_only) g.xop[1] = B->ptr_at<void>(B->take(nx * esz * parts));
+    if (bf && K >= 2 && !gram_only) g.xf[1] = B->ptr_at<float>(B->take(nx * 4));
+    if (bf && K >= 3 && !gram_only) g.xf[0] = B->ptr_at<float>(B->take(nx * 4));
     if (rq.c != 0.f) {
       g.af = B->ptr_at<float>(B->take(nm * 4));
       g.aop = bf ? B->ptr_at<void>(B->take(nm * 2 * parts)) : (void*)g.af;
     }
     g.bop = B->ptr_at<void>(B->take(nm * esz * parts));
-    if (emit_q && K >= 2) {
+    if (emit_q && (K >= 2 || gram_only)) {
       g.qop[1] = B->ptr_at<void>(B->take(nm * esz * parts));
       g.qf[1] = bf ? B->ptr_at<float>(B->take(nm * 4)) : reinterpret_cast<float*>(g.qop[1]);
     }
-    if (emit_q && K >= 3) {
+    if (emit_q && (K >= 3 || (gram_only && K >= 2))) {
       g.qop[0] = B->ptr_at<void>(B->take(nm * esz * parts));
       g.qf[0] = bf ? B->ptr_at<float>(B->take(nm * 4)) : reinterpret_cast<float*>(g.qop[0]);
     }
@@ -521,9 +533,12 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
       if ((st = enc(g.tm_x_k[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 128)) != SMUON_OK) return st;
       if ((st = enc(g.tm_x_mn[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 64)) != SMUON_OK) return st;
       if ((st = enc(g.tm_q_mn[i], g.qop[i], g.m, g.m, zc, g.ldm, 64, 64)) != SMUON_OK) return st;
+      if ((st = enc(g.tm_q_k[i], g.qop[i], g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
       if ((st = enc(g.tm_x_kw[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 256)) != SMUON_OK) return st;
     }
     if ((st = enc(g.tm_a_kw, g.aop, g.m, g.m, zc, g.ldm, 64, 256)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_t_k, g.aop2, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_t_kw, g.aop2, g.m, g.m, zc, g.ldm, 64, 256)) != SMUON_OK) return st;
     if ((st = enc(g.tm_a_k, g.aop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
     if ((st = enc(g.tm_b_k, g.bop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
     if (g.tm_uq_k >= 0) {
@@ -574,7 +589,7 @@ double stage_flops(const Builder& B, int st) {
     double per = 0;
     switch (st) {
       case ST_GRAM: case ST_PROBE: per = 2 * m * m * n; break;
-      case ST_AXPY: case ST_REUSE: per = 2 * m * n * m; break;
+      case ST_AXPY: case ST_REUSE: case ST_QX: per = 2 * m * n * m; break;
       default: per = 2 * m * m * m; break;
     }
     f += per * g.count;
@@ -588,7 +603,7 @@ double stage_issued(const Builder& B, int st) {
   const PlanHeader& h = B.h;
   const bool tc = h.mode == MODE_TC_BF16;
   const int BM = tc ? kTcBM : kSimtBM, BK = tc ? 64 : 16;
-  const bool split = tc && (h.flags & SMUON_NS_SPLIT_BF16) && st <= ST_QAXPY;
+  const bool split = tc && (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
   double f = 0;
   for (const GroupDesc& g : B.groups) {
     const bool sym = sym_stage(st);
@@ -620,11 +635,12 @@ smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int it
   if (total == 0) return SMUON_OK;
   // trace names: kernel, then the stage after a dot
   static const char* tc_names[2][ST_COUNT] = {
-      {"k_gemm_tc.gram", "k_gemm_tc.poly", "k_gemm_tc.axpy", "k_gemm_tc.qaxpy", "k_gemm_tc.reuse", "k_gemm_tc.probe"},
+      {"k_gemm_tc.gram", "k_gemm_tc.poly", "k_gemm_tc.axpy", "k_gemm_tc.qaxpy", "k_gemm_tc.reuse", "k_gemm_tc.probe",
+       "k_gemm_tc.aa1", "k_gemm_tc.aa2"},
       {"k_gemm_tc_split.gram", "k_gemm_tc_split.poly", "k_gemm_tc_split.axpy", "k_gemm_tc_split.qaxpy",
-       "k_gemm_tc_split.reuse", "k_gemm_tc_split.probe"}};
+       "k_gemm_tc_split.reuse", "k_gemm_tc_split.probe", "k_gemm_tc_split.aa1", "k_gemm_tc_split.aa2"}};
   if (h.mode == MODE_TC_BF16) {
-    const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && st <= ST_QAXPY;
+    const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
     Launch L(tc_names[split][st], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
     CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
   } else {
@@ -643,13 +659,22 @@ smuon_status validate_ns(const NsRequest& rq) {
   if (!rq.M_in || !rq.U_out) return fail(SMUON_ERR_INVALID_ARG, "M_in and U_out must not be NULL");
   if (rq.iters < 1 || rq.iters > 64) return fail(SMUON_ERR_INVALID_ARG, "iters=%d must be in 1..64", rq.iters);
   const uint32_t known =
-      SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_SIMT_BF16;
+      SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_SIMT_BF16 |
+      SMUON_NS_GRAM_ONLY;
   if (rq.flags & ~known) return fail(SMUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", rq.flags & ~known);
   const uint32_t modes = rq.flags & (SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_SIMT_BF16);
   if (modes & (modes - 1))
     return fail(SMUON_ERR_INVALID_ARG, "SMUON_NS_FP32_REF, SMUON_NS_SPLIT_BF16 and SMUON_NS_SIMT_BF16 are exclusive");
   if ((rq.flags & SMUON_NS_EMIT_Q) && !rq.Q_out)
     return fail(SMUON_ERR_INVALID_ARG, "SMUON_NS_EMIT_Q needs Q_out");
+  if (rq.flags & SMUON_NS_GRAM_ONLY) {
+    if (!(rq.flags & SMUON_NS_EMIT_Q))
+      return fail(SMUON_ERR_INVALID_ARG, "SMUON_NS_GRAM_ONLY needs SMUON_NS_EMIT_Q (U = Q_K X_0)");
+    if (rq.flags & (SMUON_NS_FP32_REF | SMUON_NS_SIMT_BF16))
+      return fail(SMUON_ERR_UNSUPPORTED, "SMUON_NS_GRAM_ONLY runs on the tensor cores only");
+    if (rq.n_mats != 1) return fail(SMUON_ERR_UNSUPPORTED, "SMUON_NS_GRAM_ONLY takes one matrix per call");
+    if (rq.c == 0.f) return fail(SMUON_ERR_UNSUPPORTED, "SMUON_NS_GRAM_ONLY needs c != 0");
+  }
   for (int i = 0; i < rq.n_mats; ++i) {
     smuon_status st;
     const bool has_g = rq.G != nullptr;
@@ -732,6 +757,24 @@ smuon_status run_ns(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
     CUDA_TRY(cudaGetLastError());
   }
   const bool emit_q = (ex.flags & SMUON_NS_EMIT_Q) != 0;
+  if (ex.flags & SMUON_NS_GRAM_ONLY) {
+    // A_0 = X_0 X_0^T; per step B_k = bA_k + cA_k^2 (Q_1 = aI + B_0 from its epilogue),
+    // Q_{k+1} = aQ_k + B_k Q_k, and A_{k+1} = P_k (P_k A_k) except after the last step; then
+    // U = s Q_K X_0 from the f32-accumulated Q_K in the workspace (split operands in split mode)
+    auto run = [&](int stg, int k) {
+      return launch_gemm(ex.d_plan, h, stg, k, skip, di, s, ex.sflops[stg], ex.sissued[stg]);
+    };
+    if ((st = run(ST_GRAM, 0)) != SMUON_OK) return st;
+    for (int k = 0; k < ex.iters; ++k) {
+      if ((st = run(ST_POLY, k)) != SMUON_OK) return st;
+      if (k >= 1 && (st = run(ST_QAXPY, k)) != SMUON_OK) return st;
+      if (k + 1 < ex.iters) {
+        if ((st = run(ST_AA1, k)) != SMUON_OK) return st;
+        if ((st = run(ST_AA2, k)) != SMUON_OK) return st;
+      }
+    }
+    return run(ST_QX, ex.iters);
+  }
   for (int k = 0; k < ex.iters; ++k) {
     if ((st = launch_gemm(ex.d_plan, h, ST_GRAM, k, skip, di, s, ex.sflops[ST_GRAM], ex.sissued[ST_GRAM])) != SMUON_OK) return st;
     if (ex.c != 0.f && (st = launch_gemm(ex.d_plan, h, ST_POLY, k, skip, di, s, ex.sflops[ST_POLY], ex.sissued[ST_POLY])) != SMUON_OK)

@@ -30,7 +30,9 @@ struct TileCtx {
 // reach the diagonal or lie above it are computed; in them an element
 // (i, j) is written if j >= i and also mirrored to (j, i) if j > i, so every
 // element is written exactly once (deterministically).
-__host__ __device__ inline bool sym_stage(int st) { return st == ST_GRAM || st == ST_POLY || st == ST_PROBE; }
+__host__ __device__ inline bool sym_stage(int st) {
+  return st == ST_GRAM || st == ST_POLY || st == ST_PROBE || st == ST_AA1 || st == ST_AA2;
+}
 
 // Tiles are BM x BN with BN = r * BM (r = 1 or 2). Row tm of the tile grid
 // holds the column tiles tn >= floor(tm / r); sym_start(tm) counts the tiles
@@ -266,7 +268,8 @@ __device__ __forceinline__ void emit_q1(const TileCtx& t, int row, int col0, int
       if (k >= ds && k < nvalid) Q[(int64_t)row * ld + col0 + k] = __float2bfloat16_rn(q[k]);
       if (k >= ms && k < nvalid) Q[(int64_t)(col0 + k) * ld + row] = __float2bfloat16_rn(q[k]);
     }
-  } else {
+  }
+  if (t.iter != t.last || (t.flags & SMUON_NS_GRAM_ONLY)) {  // the Gram-only solve also multiplies by it
     if (t.bf) sym_store_f32<NV>(t, t.g->qf[1], row, col0, nvalid, ds, ms, q);
     sym_store_operand<NV>(t, t.g->qop[1], row, col0, nvalid, ds, ms, q);
   }
@@ -342,13 +345,19 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       ld_f32_vec<NV>(src + off, q);
 #pragma unroll
       for (int k = 0; k < NV; ++k) q[k] = t.a * q[k] + v[k];
-      if (t.iter != t.last) {
+      if (t.iter == t.last)
+        st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, (t.md->vec >> 2) & 1, row, col0, nvalid, q);
+      if (t.iter != t.last || (t.flags & SMUON_NS_GRAM_ONLY)) {  // Q_K X_0 reads the workspace copy
         const int nb = (t.iter + 1) & 1;
         if (t.bf) st_f32_vec<NV>(g.qf[nb] + off, q);
         st_operand<NV>(t, g.qop[nb], off, t.mlo, q);
-      } else {
-        st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, (t.md->vec >> 2) & 1, row, col0, nvalid, q);
       }
+      break;
+    }
+    case ST_QX: {  // Gram-only fresh solve: U = s Q_K X_0
+#pragma unroll
+      for (int k = 0; k < NV; ++k) v[k] *= t.s;
+      st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, v);
       break;
     }
     case ST_REUSE: {
@@ -356,7 +365,22 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] *= t.s;
       st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, v);
-      st_op<NV>(g.xop[1], off, t.bf, v);
+      if (!(t.flags & SMUON_NS_GRAM_ONLY)) st_op<NV>(g.xop[1], off, t.bf, v);  // the probe's operand
+      break;
+    }
+    case ST_AA1:
+    case ST_AA2: {
+      // Gram-only fresh solve: Y' = a Y + B Y with Y = A_k (first) or T = P_k A_k
+      // (second); both are symmetric (polynomials in A_k), stored by the triangle rule
+      if (ds >= nvalid) break;
+      const bool first = t.stage == ST_AA1;
+      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
+      float y[NV];
+      ld_f32_vec<NV>((first ? g.af : g.af2) + off, y);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) v[k] = t.a * y[k] + v[k];
+      sym_store_f32<NV>(t, first ? g.af2 : g.af, row, col0, nvalid, ds, ms, v);
+      sym_store_operand<NV>(t, first ? g.aop2 : g.aop, row, col0, nvalid, ds, ms, v);
       break;
     }
     case ST_PROBE: {
@@ -403,7 +427,7 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
   t.iter = iter;
   t.last = h.iters - 1;
   t.Mo = g.m;
-  t.No = (st == ST_AXPY || st == ST_REUSE) ? g.n : g.m;
+  t.No = wide_out_stage(st) ? g.n : g.m;
   t.s = h.scale[g.first_mat + t.z];
   t.a = h.a; t.b = h.b; t.c = h.c;
   t.flags = h.flags;

@@ -174,6 +174,18 @@ __device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, i
     case ST_AXPY: o.ma = &h.tmaps[g.tm_b_k]; o.mb = &h.tmaps[g.tm_x_mn[iter & 1]]; o.K = g.m; o.b_mn = 1; break;
     case ST_QAXPY: o.ma = &h.tmaps[g.tm_b_k]; o.mb = &h.tmaps[g.tm_q_mn[iter & 1]]; o.K = g.m; o.b_mn = 1; break;
     case ST_REUSE: o.ma = &h.tmaps[g.tm_uq_k]; o.za = 0; o.mb = &h.tmaps[g.tm_x_mn[0]]; o.K = g.m; o.b_mn = 1; break;
+    case ST_AA1:  // B * A with A symmetric: its rows are the K-major right operand
+      o.ma = &h.tmaps[g.tm_b_k];
+      o.mb = &h.tmaps[wide ? g.tm_a_kw : g.tm_a_k];
+      o.K = g.m; o.b_mn = 0; break;
+    case ST_QX:  // Q_K (K-major rows, hi and lo parts) times X_0 (MN-major)
+      o.ma = &h.tmaps[g.tm_q_k[iter & 1]];
+      o.mb = &h.tmaps[g.tm_x_mn[0]];
+      o.K = g.m; o.b_mn = 1; break;
+    case ST_AA2:  // B * T, T symmetric
+      o.ma = &h.tmaps[g.tm_b_k];
+      o.mb = &h.tmaps[wide ? g.tm_t_kw : g.tm_t_k];
+      o.K = g.m; o.b_mn = 0; break;
     default:  // ST_PROBE
       o.ma = &h.tmaps[g.tm_x_k[1]];
       o.mb = &h.tmaps[wide ? g.tm_x_kw[1] : g.tm_x_k[1]];
@@ -410,7 +422,7 @@ cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, i
   (void)num_sms;  // the plan's schedule fixed the grid: one CTA per scheduled tile list
   const int grid = h.sched_ctas[stage];
   if (h.total_tiles[stage] == 0 || grid <= 0) return cudaSuccess;
-  const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && stage <= ST_QAXPY;
+  const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(stage);
   if (split) return launch_tc_depth<true, 128>(h, d_plan, stage, iter, skip, grid, s);
   if (tc_tile_n(stage, h.flags) == 128) return launch_tc_depth<false, 128>(h, d_plan, stage, iter, skip, grid, s);
   return launch_tc_depth<false, 256>(h, d_plan, stage, iter, skip, grid, s);

@@ -29,8 +29,18 @@ enum Stage : int32_t {
   ST_QAXPY = 3,  // Q' = a Q + B Q                       (m x m, K = m)
   ST_REUSE = 4,  // D_hat = s Q X_t                      (m x n, K = m)
   ST_PROBE = 5,  // sum (D_hat D_hat^T - I)^2 per tile   (m x m, K = n)
-  ST_COUNT = 6
+  ST_AA1 = 6,    // T = a A + B A = P A                  (m x m, K = m)  Gram-only fresh solve
+  ST_AA2 = 7,    // A' = a T + B T = P^2 A               (m x m, K = m)  Gram-only fresh solve
+  ST_QX = 8,     // U = s Q_K X_0                        (m x n, K = m)  Gram-only fresh solve
+  ST_COUNT = 9
 };
+
+// stages whose output is the m x n wide form (the others are m x m)
+__host__ __device__ inline bool wide_out_stage(int st) { return st == ST_AXPY || st == ST_REUSE || st == ST_QX; }
+
+// stages whose operands carry hi and lo parts in split mode (all but the
+// CacheMuon reuse and probe products, which read the cached bf16 transform)
+__host__ __device__ inline bool split_stage(int st) { return st != ST_REUSE && st != ST_PROBE; }
 
 enum Mode : int32_t { MODE_TC_BF16 = 0, MODE_SIMT_F32 = 1, MODE_SIMT_BF16 = 2 };
 
@@ -66,6 +76,8 @@ struct GroupDesc {
   void* bop;              // B operand [count][m][ldm]
   float* qf[2];           // f32 master of Q (EMIT_Q)
   void* qop[2];           // Q operand
+  float* af2;             // Gram-only fresh solve: f32 T = P A between the two A updates
+  void* aop2;             // T operand
   int32_t tm_x_k[2];      // tensor-map indices: X K-major box {64,128}
   int32_t tm_x_mn[2];     // X MN-major box {64,64}
   int32_t tm_a_k, tm_b_k; // A / B K-major box {64,128}
@@ -73,6 +85,8 @@ struct GroupDesc {
   int32_t tm_uq_k;        // user Q K-major (REUSE A operand)
   int32_t tm_a_kw;        // A K-major box {64,256} (B operand of 256-wide tiles)
   int32_t tm_x_kw[2];     // X K-major box {64,256}
+  int32_t tm_t_k, tm_t_kw; // T K-major boxes {64,128} and {64,256}
+  int32_t tm_q_k[2];      // Q K-major box {64,128} (left operand of Q_K X_0)
   int32_t pad1;
   int32_t tiles_m[ST_COUNT], tiles_n[ST_COUNT], tile_begin[ST_COUNT];
 };

@@ -58,7 +58,7 @@ __all__ = [
     "momentum", "frobenius_scale", "newton_schulz", "newton_schulz_with_q",
     "sign_extract", "pack_bits", "unpack_bits", "packed_words", "vote_from_signs",
     "vote_from_packed", "bf16_round", "update_with_vote", "update_dense",
-    "sign_muon_step", "cachemuon_probe", "cachemuon_run", "lion_interpolate",
+    "newton_schulz_gram_only", "sign_muon_step", "cachemuon_probe", "cachemuon_run", "lion_interpolate",
     "lion_ema", "lionmuon_step", "ns_flops", "cachemuon_flops",
 ]
 
@@ -126,6 +126,28 @@ def newton_schulz_with_q(M: np.ndarray, a: float, b: float, c: float, iters: int
     tall = M.shape[0] > M.shape[1]
     X = (M.T if tall else M) * frobenius_scale(M, eps)
     X, Q = _ns_core(X, a, b, c, iters, True)
+    return (X.T if tall else X), Q
+
+
+def newton_schulz_gram_only(M: np.ndarray, a: float, b: float, c: float, iters: int,
+                            eps: float = 1e-7):
+    """The fresh solve iterated on the m x m Gram matrix ("Gram Newton-Schulz",
+    [CM] method item 1): A_0 = X_0 X_0^T, then per step P_k = aI + bA_k + cA_k^2,
+    Q_{k+1} = P_k Q_k and A_{k+1} = P_k A_k P_k; finally X_K = Q_K X_0. In exact
+    arithmetic this is the iteration of newton_schulz_with_q (P_k is a
+    polynomial in A_k, so X_{k+1} X_{k+1}^T = P_k A_k P_k). Returns (D, Q) like it."""
+    M = np.asarray(M, np.float64)
+    tall = M.shape[0] > M.shape[1]
+    X0 = (M.T if tall else M) * frobenius_scale(M, eps)
+    m = X0.shape[0]
+    I = np.eye(m)
+    A = X0 @ X0.T
+    Q = I.copy()
+    for _ in range(iters):
+        P = a * I + b * A + c * (A @ A)
+        Q = P @ Q
+        A = P @ A @ P
+    X = Q @ X0
     return (X.T if tall else X), Q
 
 

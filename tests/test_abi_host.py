@@ -106,3 +106,22 @@ def test_gradient_streams_reject_bad_arguments_before_launch(L):
                            None) == -1
     assert b"no gradient stream" in L.smuon_last_error()
     assert st.t == 0
+
+
+def test_gram_only_rejects_unsupported_requests(L):
+    import matrix_aware_sign_b200 as S
+    m = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 16, 16, S.F32))
+    q = (S.SmuonMat * 1)(S.SmuonMat(8192, 8, 8, 8, S.BF16))
+    two = (S.SmuonMat * 2)(S.SmuonMat(4096, 8, 16, 16, S.F32), S.SmuonMat(4096, 8, 16, 16, S.F32))
+    q2 = (S.SmuonMat * 2)(S.SmuonMat(8192, 8, 8, 8, S.BF16), S.SmuonMat(8192, 8, 8, 8, S.BF16))
+    g = S.NS_GRAM_ONLY
+    args = lambda c: (c, 5, 1e-7)
+    # needs EMIT_Q
+    assert L.smuon_ns(m, m, 1, None, 0.0, 3.4445, -4.775, *args(2.0315), g, q, None, None, 0, None, None) == -1
+    # one matrix only, tensor cores only, c != 0
+    assert L.smuon_ns(two, two, 2, None, 0.0, 3.4445, -4.775, *args(2.0315), g | S.NS_EMIT_Q, q2, None, None, 0,
+                      None, None) == -4
+    assert L.smuon_ns(m, m, 1, None, 0.0, 3.4445, -4.775, *args(2.0315), g | S.NS_EMIT_Q | S.NS_FP32_REF, q, None,
+                      None, 0, None, None) == -4
+    assert L.smuon_ns(m, m, 1, None, 0.0, 1.5, -0.5, *args(0.0), g | S.NS_EMIT_Q, q, None, None, 0, None,
+                      None) == -4

@@ -667,3 +667,38 @@ def test_lionmuon_vote_reading_of_the_muon_step():
                 assert np.mean(host(Wd[l]) != W[l]) < 2e-3
                 W[l] = host(Wd[l]).astype(np.float32)
     assert opt.t == 2
+
+
+# ------------------------------------------------------------------ Gram-only fresh solve
+@pytest.mark.parametrize("shape", [(256, 1024), (1024, 256), (384, 1536), (512, 512), (200, 700)])
+@pytest.mark.parametrize("iters", [1, 2, 5])
+def test_ns_gram_only_fresh_solve(shape, iters):
+    """SMUON_NS_GRAM_ONLY: the fresh solve iterated on the Gram matrix gives
+    the polar-factor approximation and the transform Q of the X iteration
+    (within the split-BF16 tolerance), with U = Q_K X_0 written to U."""
+    rng = np.random.default_rng(iters * 100 + shape[0])
+    M = rng.standard_normal(shape).astype(np.float32)
+    m = min(shape)
+    U = torch.zeros(shape, device="cuda")
+    Q = torch.zeros((m, m), dtype=torch.bfloat16, device="cuda")
+    S.smuon_ns([dev(M)], [U], *WL.QUINTIC, iters, flags=S.NS_SPLIT_BF16 | S.NS_EMIT_Q | S.NS_GRAM_ONLY, Q_out=[Q])
+    torch.cuda.synchronize()
+    D_ref, Q_ref = O.newton_schulz_with_q(M.astype(np.float64), *WL.QUINTIC, iters)
+    check_ns_outputs([(host(U), D_ref)], 1e-2)
+    assert rel_fro(host(Q), Q_ref) < 1e-2
+
+
+def test_cachemuon_with_gram_only_fresh_solves():
+    shape = (512, 2048)
+    mom = list(WL.cachemuon_momenta(shape, 3, drift=0.01))
+    Md = dev(mom[0])
+    D = torch.zeros(shape, device="cuda")
+    cm = S.CacheMuon(Md, D, -1.0, WL.QUINTIC, 5, flags=S.NS_SPLIT_BF16 | S.NS_GRAM_ONLY)  # gamma < 0: always fresh
+    for t in range(3):
+        if t:
+            Md.copy_(dev(mom[t]))
+        cm.step()
+        torch.cuda.synchronize()
+        D_ref, _ = O.newton_schulz_with_q(mom[t], *WL.QUINTIC, 5)
+        check_ns_outputs([(host(D), D_ref)], 1e-2)
+    assert cm.counters() == {"hits": 0, "misses": 3, "probes": 2}

@@ -385,3 +385,21 @@ def test_lionmuon_muon_vote_is_sign_muon_on_g_hat():
     for a, b in zip(Mn, Md):
         for x, y in zip(a, b):
             np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("shape", [(8, 40), (40, 8), (24, 24)])
+@pytest.mark.parametrize("iters", [1, 3, 5])
+def test_gram_only_solve_matches_the_x_iteration(shape, iters):
+    """Iterating on the Gram matrix reaches the same X_K and Q as iterating on
+    X: both equal the singular-value closed form."""
+    rng = np.random.default_rng(11)
+    M = rng.standard_normal(shape)
+    D1, Q1 = O.newton_schulz_with_q(M, *WL.QUINTIC, iters)
+    D2, Q2 = O.newton_schulz_gram_only(M, *WL.QUINTIC, iters)
+    U, S, Vt = np.linalg.svd(M, full_matrices=False)
+    s = S / (np.sqrt(np.sum(S ** 2)) + 1e-7)
+    closed = (U * _poly(s, WL.QUINTIC, iters)) @ Vt
+    assert _rel(D2, closed) < 1e-10
+    assert _rel(D2, D1) < 1e-10 and _rel(Q2, Q1) < 1e-10
+    # Q is a product of commuting symmetric factors: symmetric
+    assert _rel(Q2, Q2.T) < 1e-12
