@@ -154,6 +154,23 @@ smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, in
   return SMUON_OK;
 }
 
+// float32 3-D map (B X epilogue source): 128-byte swizzle for 32-float-wide boxes, none for wider ones
+smuon_status encode_f32_3d(CUtensorMap* out, const void* ptr, int64_t inner, int64_t rows, int64_t count,
+                           int64_t ld, uint32_t box0, uint32_t box1) {
+  EncodeTiledFn enc;
+  smuon_status st = get_encoder(&enc);
+  if (st != SMUON_OK) return st;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)count};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 4), (cuuint64_t)(ld * 4 * rows)};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, box0 * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SMUON_ERR_CUDA, "cuTensorMapEncodeTiled (f32) failed (%d)", (int)r);
+  return SMUON_OK;
+}
+
 // ------------------------------------------------------------------ validation
 int dtype_size(int32_t dt) { return dt == SMUON_F32 ? 4 : dt == SMUON_BF16 ? 2 : dt == SMUON_I8 ? 1 : 0; }
 
@@ -387,11 +404,25 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.off_mom_begin = B->take(sizeof(int32_t) * (B->mats.size() + 1));
   L.off_sched = B->take(sizeof(int32_t) * std::max(sched_n, 1));
   L.off_sched_begin = B->take(sizeof(int32_t) * std::max(begin_n, 1));
+  // the B X epilogue reads its X source through a TMA-fed shared-memory ring when every matrix's
+  // momentum is f32 with 16-byte aligned rows (later steps read the f32 masters, always aligned)
+  bool axpy_tma = tc && !rq.probe && !gram_only;
+  for (const MatDesc& d : B->mats)
+    if (!(d.m_dtype == SMUON_F32 && reinterpret_cast<uintptr_t>(d.m_ptr) % 16 == 0 && (d.m_ld * 4) % 16 == 0))
+      axpy_tma = false;
   // tensor maps: count them first
   auto want_map = [&](int32_t& slot) { slot = L.n_tmaps++; };
   L.n_tmaps = 0;
+  for (auto& d : B->mats) {
+    d.tm_src = -1;
+    if (axpy_tma) want_map(d.tm_src);
+  }
   for (auto& g : B->groups) {
-    for (int i = 0; i < 2; ++i) { g.tm_x_k[i] = g.tm_x_mn[i] = g.tm_q_mn[i] = g.tm_x_kw[i] = g.tm_q_k[i] = -1; }
+    for (int i = 0; i < 2; ++i) {
+      g.tm_x_k[i] = g.tm_x_mn[i] = g.tm_q_mn[i] = g.tm_x_kw[i] = g.tm_q_k[i] = g.tm_xf[i] = -1;
+    }
+    if (axpy_tma && bf && K >= 2) want_map(g.tm_xf[1]);
+    if (axpy_tma && bf && K >= 3) want_map(g.tm_xf[0]);
     g.tm_a_k = g.tm_b_k = g.tm_uq_k = g.tm_a_kw = g.tm_t_k = g.tm_t_kw = -1;
     if (!tc) continue;
     const bool wide = tc_tile_n(ST_GRAM, rq.flags) == 256;
@@ -492,6 +523,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     h.sched_boff[st] = sched_boff[st];
     h.sched_ctas[st] = 0;
     h.max_k[st] = 0;
+    h.axpy_tma = axpy_tma ? 1 : 0;
     for (const GroupDesc& g : B->groups)
       h.max_k[st] = std::max(h.max_k[st], (st == ST_GRAM || st == ST_PROBE) ? g.n : g.m);
   }
@@ -545,6 +577,16 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
       const MatDesc& d = B->mats[g.first_mat];
       if ((st = enc(g.tm_uq_k, d.q_ptr, g.m, g.m, 1, d.q_ld, 64, 128)) != SMUON_OK) return st;
     }
+    for (int i = 0; i < 2; ++i)  // f32 masters [count][m][ldn], 32 x 128 boxes
+      if (g.tm_xf[i] >= 0 &&
+          (st = encode_f32_3d(&B->maps[g.tm_xf[i]], g.xf[i], g.n, g.m, g.count, g.ldn, 32, 128)) != SMUON_OK)
+        return st;
+  }
+  for (const MatDesc& d : B->mats) {  // the momentum as the first B X step's source
+    if (d.tm_src < 0) continue;
+    smuon_status st = d.tall ? encode_f32_3d(&B->maps[d.tm_src], d.m_ptr, d.cols, d.rows, 1, d.m_ld, 128, 32)
+                             : encode_f32_3d(&B->maps[d.tm_src], d.m_ptr, d.cols, d.rows, 1, d.m_ld, 32, 128);
+    if (st != SMUON_OK) return st;
   }
   return SMUON_OK;
 }

@@ -399,6 +399,27 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
   }
 }
 
+// B X epilogue with its X source already read (x[]): X' = a s X + s B X (first
+// step) or a X + B X, written as the next step's f32 master and operand, or
+// into the user's U after the last step
+template <int NV>
+__device__ __forceinline__ void epi_axpy_src(const TileCtx& t, int row, int col0, const float* v, float* x) {
+  if (row >= t.Mo || col0 >= t.No) return;
+  const int nvalid = min(NV, t.No - col0);
+  const GroupDesc& g = *t.g;
+  const float sc = (t.iter == 0 && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s : 1.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sc * v[k];
+  if (t.iter != t.last) {
+    const int64_t off = ((int64_t)t.z * g.m + row) * g.ldn + col0;
+    const int nb = (t.iter + 1) & 1;
+    st_f32_vec<NV>(g.xf[nb] + off, x);
+    st_operand<NV>(t, g.xop[nb], off, t.xlo, x);
+  } else {
+    st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, x);
+  }
+}
+
 // per-tile context from a linear tile index of stage st
 __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int iter, int tile,
                                             int& tm, int& tn) {

@@ -26,7 +26,9 @@ namespace tc {
 
 constexpr int BM = kTcBM, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x 64 k)
-constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
+constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps (+ one source warp for B X)
+constexpr int SRC_SLOTS = 2;                // B X epilogue source ring
+constexpr int SRC_BYTES = BM * 32 * 4;      // one 128 x 32 f32 chunk of X (or its transpose)
 
 // plain BF16: one hi tile per operand; split BF16: hi and lo tiles per operand
 // (x = x_hi + x_lo, product ~ A_hi B_hi + A_hi B_lo + A_lo B_hi).
@@ -35,7 +37,7 @@ constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
 // 192 KB of shared memory, or about 144 KB (kShallow) for stages whose K is
 // short: a tile then needs few k-blocks in flight, and the shared memory left
 // to the L1 cache serves the epilogue's row-per-lane global accesses.
-template <bool kSplit, int kBN, bool kShallow>
+template <bool kSplit, int kBN, bool kShallow, bool kSrc>
 struct Cfg {
   static constexpr int PARTS = kSplit ? 2 : 1;
   static constexpr int BN = kBN;
@@ -43,7 +45,9 @@ struct Cfg {
   static constexpr int STAGE_BYTES = PARTS * (A_BYTES + B_BYTES);
   static constexpr int STAGES = ((kShallow ? 144 : 192) * 1024) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * kBN;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int NTHREADS = THREADS + (kSrc ? 32 : 0);
+  static constexpr int SRC_RING = kSrc ? SRC_SLOTS * SRC_BYTES : 0;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SRC_RING + 1024 /*align*/ + 256 /*barriers*/;
 };
 constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz
 
@@ -146,6 +150,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // operands of one tile: tensor maps, coordinates, K extent
 struct TcOps {
   const CUtensorMap* ma;
@@ -194,9 +210,9 @@ __device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, i
   return o;
 }
 
-template <bool kSplit, int kBN, bool kShallow>
+template <bool kSplit, int kBN, bool kShallow, bool kSrc>
 __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int iter) {
-  using C = Cfg<kSplit, kBN, kShallow>;
+  using C = Cfg<kSplit, kBN, kShallow, kSrc>;
   constexpr int STAGES = C::STAGES;
   constexpr int STAGE_BYTES = C::STAGE_BYTES;
   constexpr int PARTS = C::PARTS;
@@ -206,11 +222,13 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* base_ptr = smem_raw + (base - raw);
-  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
-  // barrier layout (8 bytes each): full[S], empty[S], tfull[2], tempty[2], done
+  const uint32_t src_base = base + STAGES * STAGE_BYTES;  // B X source ring (kSrc), 1024-aligned
+  const uint32_t bar0 = src_base + C::SRC_RING;
+  // barrier layout (8 bytes each): full[S], empty[S], tfull[2], tempty[2], done, sfull[2], sempty[2]
   const uint32_t full_bar = bar0, empty_bar = bar0 + 8 * STAGES;
   const uint32_t tfull_bar = bar0 + 16 * STAGES, tempty_bar = tfull_bar + 16, done_bar = tempty_bar + 16;
-  unsigned char* misc = base_ptr + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  const uint32_t sfull_bar = done_bar + 8, sempty_bar = sfull_bar + 8 * SRC_SLOTS;
+  unsigned char* misc = base_ptr + STAGES * STAGE_BYTES + C::SRC_RING + 8 * (2 * STAGES + 5 + 2 * SRC_SLOTS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
 
@@ -219,6 +237,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar + 8 * s, 1); mbar_init(empty_bar + 8 * s, 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar + 8 * a, 1); mbar_init(tempty_bar + 8 * a, 256); }
     mbar_init(done_bar, 1);
+    for (int q = 0; q < SRC_SLOTS; ++q) { mbar_init(sfull_bar + 8 * q, 1); mbar_init(sempty_bar + 8 * q, 8); }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -339,6 +358,97 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       const unsigned long long t0 = clock64();
       while (!mbar_try_wait(done_bar, 0) && clock64() - t0 < kWaitCycles) {}
     }
+  } else if (kSrc && warp == 10) {
+    if (lane == 0) {
+      // ---------------- B X source producer: the tile's X (f32, 128 rows x 32 columns per chunk, in
+      // chunk order) into a two-slot ring that all eight epilogue warps drain together
+      int k = 0;
+      uint32_t armed = 0, last_par = 0;
+      bool ok = true;
+      for (int i = t_begin; i < t_end && ok; ++i) {
+        const int tile = tiles[i];
+        int tm, tn;
+        const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+        const bool first = iter == 0;
+        const CUtensorMap* map = first ? &h.tmaps[t.md->tm_src] : &h.tmaps[t.g->tm_xf[iter & 1]];
+        const bool tall = first && t.md->tall;
+        tensormap_acquire(map);
+        for (int c = 0; c < kBN / 32; ++c, ++k) {
+          const int slot = k & 1;
+          const uint32_t ph = (uint32_t)(k >> 1) & 1u;
+          if (!mbar_wait(sempty_bar + 8 * slot, ph ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t fb = sfull_bar + 8 * slot;
+          mbar_expect_tx(fb, SRC_BYTES);
+          armed |= 1u << slot;
+          last_par = (last_par & ~(1u << slot)) | (ph << slot);
+          const uint32_t dst = src_base + slot * SRC_BYTES;
+          const int col = tn * kBN + c * 32;  // wide-form column of the chunk
+          if (!first) tma_load_3d(dst, map, col, tm * BM, t.z, fb);
+          else if (!tall) tma_load_3d(dst, map, col, tm * BM, 0, fb);   // user rows = wide rows
+          else tma_load_3d(dst, map, tm * BM, col, 0, fb);              // user rows = wide columns
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
+      }
+      for (int q = 0; q < SRC_SLOTS; ++q)
+        if (armed & (1u << q)) {
+          const uint32_t p = (last_par >> q) & 1u;
+          const unsigned long long t0 = clock64();
+          while (!mbar_try_wait(sfull_bar + 8 * q, p) && clock64() - t0 < kWaitCycles) {}
+        }
+    }
+  } else if (kSrc) {
+    // ---------------- B X epilogue, warps 2..9: every warp takes each 32-column chunk in turn (its
+    // lane group's 32 rows, one 16-column half), with the X source from the shared-memory ring
+    const int ew = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int lrow = ew * 32 + lane;   // row within the tile
+    const float* ring = reinterpret_cast<const float*>(base_ptr + STAGES * STAGE_BYTES);
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    int kc = 0;
+    bool ok = true;
+    for (int i = t_begin; i < t_end && ok; ++i) {
+      const int tile = tiles[i];
+      int tm, tn;
+      TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+      if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag)) { ok = false; break; }
+      fence_after();
+      const bool tall = iter == 0 && t.md->tall;
+      for (int c = 0; c < kBN / 32; ++c, ++kc) {
+        const int slot = kc & 1;
+        if (!mbar_wait(sfull_bar + 8 * slot, (uint32_t)(kc >> 1) & 1u, abort_flag)) { ok = false; break; }
+        float v[16], x[16];
+        tmem_ld16(tmem_base + (uint32_t)(acc * kBN + c * 32 + 16 * half) + ((uint32_t)(ew * 32) << 16), v);
+        const float* sp = ring + slot * (SRC_BYTES / 4);
+        if (!tall) {
+          // [128 rows][32 f32] with the 128-byte swizzle: 16-byte unit u of row r sits at u ^ (r & 7)
+          const unsigned char* rp = reinterpret_cast<const unsigned char*>(sp) + lrow * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 f = *reinterpret_cast<const float4*>(rp + (((4 * half + q) ^ (lrow & 7)) << 4));
+            x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+          }
+        } else {
+          // [32 user rows = wide columns][128 f32 = wide rows], no swizzle: lanes read along a row
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[j] = sp[(16 * half + j) * BM + lrow];
+        }
+        epi_axpy_src<16>(t, tm * BM + lrow, tn * kBN + c * 32 + 16 * half, v, x);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sempty_bar + 8 * slot);
+      }
+      if (!ok) break;
+      fence_before();
+      mbar_arrive(tempty_bar + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
+    }
   } else {
     // ---------------- epilogue warps 2..9: two warps per TMEM lane group, one per half of the columns
     const int ew = warp & 3;         // TMEM lane group this warp may access
@@ -380,36 +490,49 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
 }
 
-template <bool kSplit, int kBN, bool kShallow>
-__global__ void __launch_bounds__(THREADS, 1) k_gemm_tc(const Plan* plan, int stage, int iter, const int32_t* skip) {
+template <bool kSplit, int kBN, bool kShallow, bool kSrc>
+__global__ void __launch_bounds__(Cfg<kSplit, kBN, kShallow, kSrc>::NTHREADS, 1)
+    k_gemm_tc(const Plan* plan, int stage, int iter, const int32_t* skip) {
   if (skip && *skip) return;
-  gemm_tc_body<kSplit, kBN, kShallow>(plan, stage, iter);
+  gemm_tc_body<kSplit, kBN, kShallow, kSrc>(plan, stage, iter);
 }
 
 }  // namespace tc
 
-template <bool kSplit, int kBN, bool kShallow>
+template <bool kSplit, int kBN, bool kShallow, bool kSrc>
 static cudaError_t launch_tc_variant(const Plan* d_plan, int stage, int iter, const int32_t* skip, int grid,
                                      cudaStream_t s) {
-  using C = tc::Cfg<kSplit, kBN, kShallow>;
+  using C = tc::Cfg<kSplit, kBN, kShallow, kSrc>;
   static bool attr_set[256] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 256 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc<kSplit, kBN, kShallow>,
+    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc<kSplit, kBN, kShallow, kSrc>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  tc::k_gemm_tc<kSplit, kBN, kShallow><<<grid, tc::THREADS, C::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
+  tc::k_gemm_tc<kSplit, kBN, kShallow, kSrc><<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
   return cudaGetLastError();
+}
+
+template <bool kSplit, int kBN, bool kSrc>
+static cudaError_t launch_tc_src(const PlanHeader& h, const Plan* d_plan, int stage, int iter,
+                                 const int32_t* skip, int grid, cudaStream_t s) {
+  if (h.max_k[stage] <= kShallowMaxK)
+    return launch_tc_variant<kSplit, kBN, true, kSrc>(d_plan, stage, iter, skip, grid, s);
+  return launch_tc_variant<kSplit, kBN, false, kSrc>(d_plan, stage, iter, skip, grid, s);
 }
 
 template <bool kSplit, int kBN>
 static cudaError_t launch_tc_depth(const PlanHeader& h, const Plan* d_plan, int stage, int iter,
                                    const int32_t* skip, int grid, cudaStream_t s) {
-  if (h.max_k[stage] <= kShallowMaxK) return launch_tc_variant<kSplit, kBN, true>(d_plan, stage, iter, skip, grid, s);
-  return launch_tc_variant<kSplit, kBN, false>(d_plan, stage, iter, skip, grid, s);
+  // the B X stage takes its X source through the shared-memory ring when the plan has the maps and
+  // runs several steps (measured: with a single step the direct loads of the row-per-lane epilogue,
+  // served by L1, were 4% faster on the ResNet-50 set; from two steps on the ring wins, 5-12%)
+  if (stage == ST_AXPY && h.axpy_tma && h.iters >= 2)
+    return launch_tc_src<kSplit, kBN, true>(h, d_plan, stage, iter, skip, grid, s);
+  return launch_tc_src<kSplit, kBN, false>(h, d_plan, stage, iter, skip, grid, s);
 }
 
 int tc_tile_n(int stage, uint32_t flags) {

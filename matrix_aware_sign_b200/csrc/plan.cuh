@@ -63,6 +63,8 @@ struct MatDesc {
   int32_t mom_begin;      // first momentum tile (= partial-sum slot)
   int32_t mom_tiles_c;    // 64x64 tiles along cols (user orientation)
   int32_t mom_count;      // number of momentum tiles
+  int32_t tm_src;         // f32 map of M for the first B X epilogue's source (-1: none)
+  int32_t pad0;
 };
 
 // matrices of one wide shape m x n, stored contiguously in the workspace
@@ -87,7 +89,7 @@ struct GroupDesc {
   int32_t tm_x_kw[2];     // X K-major box {64,256}
   int32_t tm_t_k, tm_t_kw; // T K-major boxes {64,128} and {64,256}
   int32_t tm_q_k[2];      // Q K-major box {64,128} (left operand of Q_K X_0)
-  int32_t pad1;
+  int32_t tm_xf[2];       // f32 masters, box {32,128}, 128B swizzle (B X epilogue source, steps >= 1)
   int32_t tiles_m[ST_COUNT], tiles_n[ST_COUNT], tile_begin[ST_COUNT];
 };
 
@@ -114,6 +116,7 @@ struct PlanHeader {
   int32_t sched_boff[ST_COUNT];     // offset of each stage's begin array in sched_begin
   int32_t sched_ctas[ST_COUNT];     // CTAs of each stage's launch
   int32_t max_k[ST_COUNT];          // longest K of each stage over the groups (picks the smem ring depth)
+  int32_t axpy_tma;                 // the B X epilogue's X source is staged in shared memory by TMA
   GroupDesc* groups;        // device pointers into the plan region
   MatDesc* mats;
   CUtensorMap* tmaps;

@@ -702,3 +702,21 @@ def test_cachemuon_with_gram_only_fresh_solves():
         D_ref, _ = O.newton_schulz_with_q(mom[t], *WL.QUINTIC, 5)
         check_ns_outputs([(host(D), D_ref)], 1e-2)
     assert cm.counters() == {"hits": 0, "misses": 3, "probes": 2}
+
+
+@pytest.mark.parametrize("offset", [0, 1])
+@pytest.mark.parametrize("shape", [(96, 200), (200, 96)])
+def test_ns_source_ring_and_unaligned_fallback(shape, offset):
+    """The B X epilogue reads its X source through the TMA-fed shared-memory
+    ring when every momentum is f32 with 16-byte aligned rows (offset 0); a
+    matrix that starts 4 bytes off (offset 1) sends the whole call to the
+    direct global loads. Both give the oracle's result, over several steps."""
+    rng = np.random.default_rng(41 + offset)
+    M = rng.standard_normal(shape).astype(np.float32)
+    big = torch.zeros((shape[0], shape[1] + 8), device="cuda")
+    big[:, offset:offset + shape[1]] = dev(M)
+    Mv = big[:, offset:offset + shape[1]]
+    U = torch.zeros(shape, device="cuda")
+    S.smuon_ns([Mv], [U], *WL.QUINTIC, 3, flags=S.NS_SPLIT_BF16)
+    torch.cuda.synchronize()
+    check_ns_outputs([(host(U), O.newton_schulz(M.astype(np.float64), *WL.QUINTIC, 3))], 1e-2)
