@@ -496,13 +496,14 @@ def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0, name="c3_gpt2
     else:
         votes = [torch.zeros(s, dtype=torch.int8, device="cuda") for s in shapes]
         dirs = [torch.zeros(s, device="cuda") for s in shapes]
+        # one fused launch for the signs, the packed message and the votes of every layer (no W)
+        signs_votes = S.UpdatePlan(None, 0.0, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_POPCOUNT,
+                                   packed_out=packed, vote_out=votes)
         polar = S.NsPlan(votes, dirs, *cfg.coeffs, cfg.iters, flags=ns_flags)
         upd = S.UpdatePlan(Wd, cfg.eta, dense=dirs)
 
         def tail():
-            for l, (r, c) in enumerate(shapes):
-                S.smuon_sign_pack(Ul[l], packed=packed[l])
-                S.smuon_vote(M, r * c, votes[l], packed=packed[l], tie_value=cfg.tie_value)
+            signs_votes.run()
             polar.run()
             upd.run()
     ws_e2e = S.workspace(nbytes) if e2e else None

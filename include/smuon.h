@@ -223,7 +223,10 @@ smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t 
  *                    all-gather payload), vote_out[l] ([N] int8).
  *  votes[n_layers]   I8 matrices of -1/0/+1 (e.g. from smuon_vote).
  *  dense[n_layers]   F32 or BF16 direction D of W's shape.
- *  W[n_layers]       F32 or BF16, updated in place.
+ *  W[n_layers]       F32 or BF16, updated in place. With the U source W may be
+ *                    NULL when packed_out or vote_out is given: the call then
+ *                    only writes the message and the votes (the input of the
+ *                    local polar step, step 5; shapes are taken from U).
  * packed_out and vote_out are host arrays of n_layers device pointers
  * (entries may be NULL) or NULL. M in 1..64.
  * ---------------------------------------------------------------------- */

@@ -235,8 +235,8 @@ class UpdatePlan:
     def __init__(self, W, eta, U=None, votes=None, dense=None, M=1, tie_value=0, vote_kind=VOTE_POPCOUNT,
                  packed_out=None, vote_out=None):
         Uflat = None if U is None else [u for layer in U for u in layer]
-        self.tensors = (list(W), Uflat, votes, dense, packed_out, vote_out)
-        n = len(W)
+        self.tensors = (None if W is None else list(W), Uflat, votes, dense, packed_out, vote_out)
+        n = len(U) if W is None else len(W)  # W None: signs, message and votes only
         po = None if packed_out is None else (c_void_p * n)(*[_ptr(p) for p in packed_out])
         vo = None if vote_out is None else (c_void_p * n)(*[_ptr(v) for v in vote_out])
         h = c_void_p()
@@ -269,9 +269,10 @@ def smuon_vote(M: int, N: int, vote, packed=None, signs_i8=None, tie_value: int 
 
 def smuon_update(W, eta: float, U=None, votes=None, dense=None, M: int = 1, tie_value: int = 0,
                  vote_kind: int = VOTE_POPCOUNT, packed_out=None, vote_out=None, stream=None):
-    """U is a list over layers of lists over workers (flattened worker-minor)."""
+    """U is a list over layers of lists over workers (flattened worker-minor).
+    W may be None with U and packed_out / vote_out: signs, message and votes only."""
     Uflat = None if U is None else [u for layer in U for u in layer]
-    n = len(W)
+    n = len(U) if W is None else len(W)
     po = None if packed_out is None else (c_void_p * n)(*[_ptr(p) for p in packed_out])
     vo = None if vote_out is None else (c_void_p * n)(*[_ptr(v) for v in vote_out])
     _check(lib().smuon_update(_mats(W), n, _mats(Uflat), _mats(votes), _mats(dense), M, eta, tie_value,

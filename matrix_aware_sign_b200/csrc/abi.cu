@@ -1029,9 +1029,12 @@ struct UpdExec {
 smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
                             const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
                             uint32_t* const* packed_out, int8_t* const* vote_out, UpdExec* ex) {
-  if (!W || n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "W is NULL or n_layers < 1");
+  if (n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "n_layers < 1");
   const int nsrc = (U != nullptr) + (votes != nullptr) + (dense != nullptr);
   if (nsrc != 1) return fail(SMUON_ERR_INVALID_ARG, "exactly one of U, votes, dense must be given");
+  // W == NULL: signs, message and vote only (the local polar step's input, or an exchange's payload)
+  if (!W && !(U && (packed_out || vote_out)))
+    return fail(SMUON_ERR_INVALID_ARG, "W may be NULL only with the U source and packed_out or vote_out");
   if (U && (M < 1 || M > kMaxWorkers)) return fail(SMUON_ERR_UNSUPPORTED, "M=%d must be in 1..%d", M, kMaxWorkers);
   if (tie_value < -1 || tie_value > 1) return fail(SMUON_ERR_INVALID_ARG, "tie_value must be -1, 0 or 1");
   if (vote_kind > SMUON_VOTE_INT8) return fail(SMUON_ERR_INVALID_ARG, "unknown vote_kind %u", vote_kind);
@@ -1039,19 +1042,20 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
   int32_t src_dtype = -1;
   EwBuild eb;
   for (int l = 0; l < n_layers; ++l) {
-    smuon_status st = check_mat(W[l], "W", l, true, true, false);
-    if (st != SMUON_OK) return st;
+    smuon_status st = SMUON_OK;
+    const smuon_mat& shape = W ? W[l] : U[(int64_t)l * M];  // layer shape (the first worker's U without W)
+    if (W && (st = check_mat(W[l], "W", l, true, true, false)) != SMUON_OK) return st;
     EwLayer L{};
-    L.w = W[l].data; L.w_ld = W[l].ld; L.w_dtype = W[l].dtype;
-    L.rows = W[l].rows; L.cols = W[l].cols; L.n = (int64_t)L.rows * L.cols;
+    if (W) { L.w = W[l].data; L.w_ld = W[l].ld; L.w_dtype = W[l].dtype; }
+    L.rows = shape.rows; L.cols = shape.cols; L.n = (int64_t)L.rows * L.cols;
     L.words = 4 * ((L.n + 127) / 128);
-    L.vec = vec_ok(W[l].data, W[l].ld, W[l].cols, 1);
+    L.vec = W ? vec_ok(W[l].data, W[l].ld, W[l].cols, 1) : 1;
     std::vector<EwSrc> srcs;
     if (U) {
       for (int k = 0; k < M; ++k) {
         const smuon_mat& u = U[(int64_t)l * M + k];
         if ((st = check_mat(u, "U", l * M + k, true, true, false)) != SMUON_OK) return st;
-        if (!same_shape(u, W[l])) return fail(SMUON_ERR_SHAPE, "U[%d] shape differs from W[%d]", l * M + k, l);
+        if (!same_shape(u, shape)) return fail(SMUON_ERR_SHAPE, "U[%d] shape differs from W[%d]", l * M + k, l);
         if (src_dtype >= 0 && u.dtype != src_dtype) return fail(SMUON_ERR_DTYPE, "all U must share one dtype");
         src_dtype = u.dtype;
         if (!vec_ok(u.data, u.ld, u.cols, 1)) L.vec = 0;
@@ -1090,7 +1094,7 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
     double bytes = 0;
     for (int l = 0; l < tb.n_layers; ++l) {
       const EwLayer& Ly = tb.layers[l];
-      bytes += (double)Ly.n * (tb.M * dtype_size(src_dtype) + 2 * dtype_size(Ly.w_dtype));
+      bytes += (double)Ly.n * (tb.M * dtype_size(src_dtype) + (Ly.w ? 2 * dtype_size(Ly.w_dtype) : 0));
       if (Ly.packed_out) bytes += (double)Ly.n * tb.M / 8.0;
       if (Ly.vote_out) bytes += (double)Ly.n;
     }

@@ -351,11 +351,12 @@ __device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
 }
 
 // vote and update of 8 entries e0..e0+7 from their 4 packed count words
+template <bool kHasW>
 __device__ __forceinline__ void vote_finish8(const EwTable& tb, const EwLayer& L, int64_t e0, const uint32_t* cnt) {
   // W is loaded only here, after the workers' loads: fewer live registers, so
   // three CTAs fit per SM (more loads in flight hide more latency)
   float w[8];
-  load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+  if (kHasW) load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
   int8_t v8[8];
   // eta * v for v = +1, -1 and the tie value: exact products, chosen per entry
   const float up = tb.eta, down = -tb.eta, tied = tb.eta * (float)tb.tie;
@@ -365,7 +366,7 @@ __device__ __forceinline__ void vote_finish8(const EwTable& tb, const EwLayer& L
     v8[k] = (int8_t)(c2 > tb.M ? 1 : (c2 < tb.M ? -1 : tb.tie));
     w[k] = __fsub_rn(w[k], c2 > tb.M ? up : (c2 < tb.M ? down : tied));
   }
-  store8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+  if (kHasW) store8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);  // no W: signs, message and vote only
   if (L.vote_out) {
     int8_t* dst = L.vote_out + e0;
     if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
@@ -384,6 +385,7 @@ __device__ __forceinline__ void vote_finish8(const EwTable& tb, const EwLayer& L
 // sum = 2 * count - M (the +-1 sum of the all-reduce variant). Each lane takes
 // two consecutive 8-entry chunks (16 entries, 16-byte loads per worker); layer
 // chunk ranges are multiples of 16 chunks, so a pair never straddles layers.
+template <bool kHasW>
 __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -420,8 +422,8 @@ __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
             }
           }
       }
-      vote_finish8(tb, L, e0, cnt);
-      vote_finish8(tb, L, e0 + 8, cnt + 4);
+      vote_finish8<kHasW>(tb, L, e0, cnt);
+      vote_finish8<kHasW>(tb, L, e0 + 8, cnt + 4);
     } else {
       // ragged or strided layers: entry by entry
       const int nent = (int)min((int64_t)16, L.n - e0);
@@ -433,8 +435,10 @@ __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
           c += load_as_f32(S.ptr, ew_index(L, e, S.ld), SMUON_BF16) >= 0.f ? 1 : 0;
         }
         const int8_t v = threshold(2 * c - M, tb.tie);
-        const int64_t wi = ew_index(L, e, L.w_ld);
-        store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+        if (L.w) {
+          const int64_t wi = ew_index(L, e, L.w_ld);
+          store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+        }
         if (L.vote_out) L.vote_out[e] = v;
       }
     }
@@ -464,8 +468,10 @@ __device__ __noinline__ void finish_pair_scalar(const EwTable& tb, const EwLayer
   for (int k = 0; k < 2 && k < left; ++k) {
     const int c = (int)((cnt >> (16 * k)) & 0xffffu);
     const int8_t v = threshold(2 * c - tb.M, tb.tie);
-    const int64_t wi = ew_index(L, e + k, L.w_ld);
-    store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+    if (L.w) {
+      const int64_t wi = ew_index(L, e + k, L.w_ld);
+      store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+    }
     if (L.vote_out) L.vote_out[e + k] = v;
   }
 }
@@ -479,6 +485,7 @@ __device__ __noinline__ void finish_pair_scalar(const EwTable& tb, const EwLayer
 // theirs into one packed word (entry i -> bit i%32 of word i/32) with one
 // shuffle. Layer chunk ranges are multiples of 16 chunks (128 entries), so a
 // lane pair never straddles a layer and the even lane's e0 is a multiple of 32.
+template <bool kHasW>
 __device__ __forceinline__ void vote_update_bf16x16(const EwTable& tb) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -536,8 +543,8 @@ __device__ __forceinline__ void vote_update_bf16x16(const EwTable& tb) {
     }
     if (!live) continue;
     if (fast) {
-      vote_finish8(tb, L, e0, cnt);
-      vote_finish8(tb, L, e0 + 8, cnt + 4);
+      vote_finish8<kHasW>(tb, L, e0, cnt);
+      vote_finish8<kHasW>(tb, L, e0 + 8, cnt + 4);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) finish_pair_scalar(tb, L, e0 + 2 * i, nent - 2 * i, cnt[i]);
@@ -559,7 +566,7 @@ __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
     const int64_t e0 = (chunk - L.chunk_begin) * 8;
     const bool live = active && e0 < L.n;
     float w[8];
-    if (live) load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+    if (live && L.w) load8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
     MaskT mask[8];
     int sum[8];
 #pragma unroll
@@ -597,7 +604,7 @@ __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
       v8[k] = threshold(total, tb.tie);
       w[k] = __fsub_rn(w[k], tb.eta * (float)v8[k]);
     }
-    store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
+    if (L.w) store8(L.w, L.w_ld, L.w_dtype, L, e0, L.vec, w);
     if (L.vote_out) {
       if (e0 + 8 <= L.n && ((reinterpret_cast<uintptr_t>(L.vote_out + e0) & 7) == 0)) {
         uint2 pk;
@@ -615,12 +622,14 @@ __global__ void __launch_bounds__(256) k_vote_update(const __grid_constant__ EwT
   vote_update_body<kPopcount, kBf16, MaskT>(tb);
 }
 
+template <bool kHasW>
 __global__ void __launch_bounds__(256, 3) k_vote_update_i8_bf16(const __grid_constant__ EwTable tb) {
-  vote_update_int8_bf16(tb);
+  vote_update_int8_bf16<kHasW>(tb);
 }
 
+template <bool kHasW>
 __global__ void __launch_bounds__(256, 3) k_vote_update_bf16x16(const __grid_constant__ EwTable tb) {
-  vote_update_bf16x16(tb);
+  vote_update_bf16x16<kHasW>(tb);
 }
 
 cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s) {
@@ -628,8 +637,10 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
   // 16 entries per lane, three resident CTAs per SM (launch bounds), one wave
   const int64_t want16 = (tb.total_chunks + 511) / 512;
   const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
+  const bool has_w = tb.layers[0].w != nullptr;  // all layers or none (signs and votes only)
   if (bf && (popcount || tb.any_packed) && tb.M <= kMaxWorkers) {
-    k_vote_update_bf16x16<<<grid16, 256, 0, s>>>(tb);
+    if (has_w) k_vote_update_bf16x16<true><<<grid16, 256, 0, s>>>(tb);
+    else k_vote_update_bf16x16<false><<<grid16, 256, 0, s>>>(tb);
     return cudaGetLastError();
   }
   if (popcount) {
@@ -642,7 +653,10 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
     }
   } else {
     // the packed-counter kernel needs no packed message (it builds none)
-    if (bf && !tb.any_packed) k_vote_update_i8_bf16<<<grid16, 256, 0, s>>>(tb);
+    if (bf && !tb.any_packed) {
+      if (has_w) k_vote_update_i8_bf16<true><<<grid16, 256, 0, s>>>(tb);
+      else k_vote_update_i8_bf16<false><<<grid16, 256, 0, s>>>(tb);
+    }
     else if (bf) k_vote_update<false, true, uint32_t><<<grid, 256, 0, s>>>(tb);
     else k_vote_update<false, false, uint32_t><<<grid, 256, 0, s>>>(tb);
   }

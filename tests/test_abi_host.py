@@ -88,6 +88,9 @@ def test_update_rejects_bad_source_combinations(L):
     assert L.smuon_update(W, 1, None, None, None, 1, 0.01, 0, 0, None, None, None) == -1
     assert L.smuon_update(W, 1, W, W, None, 1, 0.01, 0, 0, None, None, None) == -1
     assert L.smuon_update(W, 1, W, None, None, 1, 0.01, 0, 7, None, None, None) == -1
+    # no W: only with the U source and an output to write
+    assert L.smuon_update(None, 1, W, None, None, 1, 0.01, 0, 0, None, None, None) == -1
+    assert L.smuon_update(None, 1, None, W, None, 1, 0.01, 0, 0, None, None, None) == -1
 
 
 def test_gradient_streams_reject_bad_arguments_before_launch(L):

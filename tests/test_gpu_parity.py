@@ -720,3 +720,25 @@ def test_ns_source_ring_and_unaligned_fallback(shape, offset):
     S.smuon_ns([Mv], [U], *WL.QUINTIC, 3, flags=S.NS_SPLIT_BF16)
     torch.cuda.synchronize()
     check_ns_outputs([(host(U), O.newton_schulz(M.astype(np.float64), *WL.QUINTIC, 3))], 1e-2)
+
+
+@pytest.mark.parametrize("udtype,kind,with_packed", [("bf16", S.VOTE_POPCOUNT, True), ("bf16", S.VOTE_INT8, False),
+                                                     ("f32", S.VOTE_POPCOUNT, True)])
+def test_signs_and_votes_without_weights(udtype, kind, with_packed):
+    """smuon_update with W = NULL: one fused pass writes the packed message and
+    the votes of every layer (the local polar step's input) and touches no W."""
+    shapes, M = [(64, 147), (7, 13), (256, 256), (130, 300)], 5
+    tdt = torch.bfloat16 if udtype == "bf16" else torch.float32
+    U = [WL.synthetic_polar_outputs(s, M, seed=60 + i, dtype=udtype, zero_fraction=0.03) for i, s in enumerate(shapes)]
+    Ud = [[dev(u, tdt) for u in layer] for layer in U]
+    votes = [torch.full((r * c,), 7, dtype=torch.int8, device="cuda") for r, c in shapes]
+    packed = [torch.full((M, S.packed_words(r * c)), 0x33, dtype=torch.int32, device="cuda")
+              for r, c in shapes] if with_packed else None
+    S.smuon_update(None, 0.0, U=Ud, M=M, tie_value=0, vote_kind=kind, packed_out=packed, vote_out=votes)
+    torch.cuda.synchronize()
+    for i, s in enumerate(shapes):
+        signs = [O.sign_extract(u) for u in U[i]]
+        np.testing.assert_array_equal(host(votes[i]).reshape(s), O.vote_from_signs(signs))
+        if with_packed:
+            for k in range(M):
+                np.testing.assert_array_equal(packed[i][k].cpu().numpy().view(np.uint32), O.pack_bits(signs[k]))
