@@ -452,7 +452,13 @@ def setup_c2(S, torch, rank, ns_flags, e2e, layers=0, name="c2_resnet50"):
         hostW = [torch.empty(w.shape, dtype=torch.float32).pin_memory() for w in W]
         return hostG, [torch.empty_like(g) for g in Gd[0]], hostW, Wd
 
-    return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None,
+    def e2e_ns(G):  # the one-shot public calls (own workspace; the prepared plans keep theirs)
+        S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G, beta=cfg.beta, flags=ns_flags, ws=ws_e2e)
+
+    def e2e_tail():
+        S.smuon_update(Wd, cfg.eta, U=Ul, M=M, tie_value=cfg.tie_value, vote_kind=S.VOTE_INT8)
+
+    return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None, "e2e_ns": e2e_ns, "e2e_tail": e2e_tail,
             "g_bytes": n_params * M * 4, "w_bytes": n_params * 4,
             "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], ns_flags != 0, 2),
             "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters, "vote": "int8 sum",
@@ -520,8 +526,11 @@ def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0, name="c3_gpt2
         hostW = [torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for w in Wd]
         return hostG, [torch.empty_like(g) for g in Gd[0]], hostW, Wd
 
+    def e2e_ns(G):
+        S.smuon_ns(Md, Ud, *cfg.coeffs, cfg.iters, G=G, beta=cfg.beta, flags=ns_flags, ws=ws_e2e)
+
     vote_bytes = n_params * (M * 2 + 2 * 2 + M / 8)
-    return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None,
+    return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None, "e2e_ns": e2e_ns, "e2e_tail": tail,
             "g_bytes": n_params * M * 4, "w_bytes": n_params * 2,
             "vote_alone": (vote_plan, vote_bytes) if vote_plan is not None else None,
             "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], ns_flags != 0, 2),
@@ -774,18 +783,48 @@ def main():
     # --- end to end through the public API with host buffers
     e2e = None
     if e2e_on and wl["e2e_io"] is not None:
-        hostG, devG, hostW, Wd = wl["e2e_io"]()
+        # every step copies its gradients from pinned host memory and reads the updated weights back; the
+        # copies run on their own streams, double-buffered, so that step i+1's gradients cross PCIe while
+        # step i computes and step i's weights come back while step i+1's Newton-Schulz runs
+        hostG, devG0, hostW, Wd = wl["e2e_io"]()
+        devG = [devG0, [torch.empty_like(g) for g in devG0]]
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_copied = [torch.cuda.Event(), torch.cuda.Event()]
+        ev_free = [torch.cuda.Event(), torch.cuda.Event()]
+        ev_done, ev_read = torch.cuda.Event(), torch.cuda.Event()
+        n = args.e2e_steps
         torch.cuda.synchronize()
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(args.e2e_steps):
-            for d, h in zip(devG, hostG[i % len(hostG)]):
-                d.copy_(h, non_blocking=True)
-            step(i, devG)
-            for h, d in zip(hostW, Wd):
-                h.copy_(d, non_blocking=True)
+        h2d.wait_stream(stream)
+        with torch.cuda.stream(h2d):
+            for d, hg in zip(devG[0], hostG[0]):
+                d.copy_(hg, non_blocking=True)
+            ev_copied[0].record(h2d)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:
+                with torch.cuda.stream(h2d):
+                    if i >= 1:
+                        h2d.wait_event(ev_free[1 - b])  # step i-1's Newton-Schulz has read that buffer
+                    for d, hg in zip(devG[1 - b], hostG[(i + 1) % len(hostG)]):
+                        d.copy_(hg, non_blocking=True)
+                    ev_copied[1 - b].record(h2d)
+            stream.wait_event(ev_copied[b])
+            wl["e2e_ns"](devG[b])
+            ev_free[b].record(stream)
+            if i >= 1:
+                stream.wait_event(ev_read)  # step i-1's weights are on the host before W changes again
+            wl["e2e_tail"]()
+            ev_done.record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ev_done)
+                for hw, d in zip(hostW, Wd):
+                    hw.copy_(d, non_blocking=True)
+                ev_read.record(d2h)
+        stream.wait_event(ev_read)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
