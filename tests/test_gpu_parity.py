@@ -742,3 +742,42 @@ def test_signs_and_votes_without_weights(udtype, kind, with_packed):
         if with_packed:
             for k in range(M):
                 np.testing.assert_array_equal(packed[i][k].cpu().numpy().view(np.uint32), O.pack_bits(signs[k]))
+
+
+# ------------------------------------------------------------------ one worker per GPU (host-side exchange)
+@pytest.mark.parametrize("exchange", ["allgather", "allreduce_int8"])
+def test_distributed_sign_muon_single_rank(exchange):
+    """DistributedSignMuon on one NCCL rank: sign-pack, exchange, vote and update
+    give exactly the single-process fused step with one worker."""
+    import socket
+
+    import torch.distributed as dist
+
+    from matrix_aware_sign_b200.distributed import DistributedSignMuon
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    import datetime
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        shapes = [(64, 147), (96, 40), (33, 70)]
+        rng = np.random.default_rng(4)
+        W = WL.weights(shapes, "normal002", "f32")
+        G = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+        # distributed path
+        Wd = [dev(w) for w in W]
+        opt = DistributedSignMuon(Wd, [torch.zeros(s, device="cuda") for s in shapes], WL.QUINTIC, 1, 0.9, 0.01,
+                                  exchange=exchange)
+        opt.step([dev(g) for g in G])
+        # single process, one worker
+        Ws = [dev(w) for w in W]
+        Ms = [torch.zeros(s, device="cuda") for s in shapes]
+        Us = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in shapes]
+        S.smuon_ns(Ms, Us, *WL.QUINTIC, 1, G=[dev(g) for g in G], beta=0.9)
+        S.smuon_update(Ws, 0.01, U=[[u] for u in Us], M=1)
+        torch.cuda.synchronize()
+        for a, b in zip(Wd, Ws):
+            assert torch.equal(a, b)
+    finally:
+        dist.destroy_process_group()

@@ -46,3 +46,47 @@ def test_two_ranks_max_time_and_throughput():
     assert ms0 == ms1 == 150.0                      # both ranks report the slowest time
     assert v0 == v1 == pytest.approx(2 * 10 / 0.150)
     assert len({a0, b0, a1, b1}) == 4               # four distinct gradient streams
+
+
+def _exchange_worker(rank, world, port, out):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle as O
+    import workloads as WL
+    from matrix_aware_sign_b200.distributed import exchange_packed, exchange_signs_int8
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        shape = (37, 29)                      # 1073 entries: a ragged last word
+        U = WL.synthetic_polar_outputs(shape, world, seed=5, dtype="f32", zero_fraction=0.05)
+        signs = [O.sign_extract(u).reshape(-1) for u in U]   # every rank knows all, sends its own
+        mine = torch.from_numpy(O.pack_bits(signs[rank]).view(np.int32))
+        gathered = exchange_packed(mine).numpy().view(np.uint32)
+        ok_gather = all(np.array_equal(gathered[k], O.pack_bits(signs[k])) for k in range(world))
+        ok_vote = np.array_equal(O.vote_from_packed(list(gathered), world, signs[0].size),
+                                 O.vote_from_signs(signs))
+        total = exchange_signs_int8(torch.from_numpy(signs[rank].copy())).numpy()
+        ok_sum = np.array_equal(total, np.sum(np.stack(signs).astype(np.int64), axis=0))
+        out.put((rank, ok_gather, ok_vote, ok_sum))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_exchange_the_messages():
+    """The pages' deployment (one worker per rank): the 1-bit messages are
+    all-gathered in rank order and vote like the signs they carry; the int8
+    signs all-reduce to their sum."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_exchange_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, True, True, True), (1, True, True, True)]
