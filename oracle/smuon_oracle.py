@@ -28,7 +28,8 @@ Readings where the pages are silent (each is listed in the design doc):
       given per workload (cubic (1.5,-0.5,0), quintic (3.4445,-4.7750,2.0315)).
   R3  The iteration runs on the smaller Gram side: a tall matrix is
       transposed, iterated, and transposed back.
-  R4  Frobenius normalisation X0 = M / (||M||_F + eps), eps = 1e-7.
+  R4  Frobenius normalisation X0 = M / (||M||_F + eps), eps = 1e-7 (the spectral
+      norm ||M||_2 in its place is the option the same section allows).
   R5  sign(u) = +1 if u >= 0 else -1 (so -0.0 -> +1, NaN -> -1).
   R6  Vote ties (even number of workers) give ``tie_value`` (0 by default).
   R8  Packed bits: entry i of the row-major flattening goes to bit i % 32 of
@@ -55,7 +56,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "momentum", "frobenius_scale", "newton_schulz", "newton_schulz_with_q",
+    "momentum", "frobenius_scale", "spectral_scale", "newton_schulz", "newton_schulz_with_q",
     "sign_extract", "pack_bits", "unpack_bits", "packed_words", "vote_from_signs",
     "vote_from_packed", "bf16_round", "update_with_vote", "update_dense",
     "newton_schulz_gram_only", "sign_muon_step", "cachemuon_probe", "cachemuon_run", "lion_interpolate",
@@ -100,19 +101,26 @@ def _ns_core(X: np.ndarray, a: float, b: float, c: float, iters: int, track_q: b
     return X, Q
 
 
+def spectral_scale(M: np.ndarray, eps: float) -> float:
+    """s = 1 / (||M||_2 + eps): the spectral-norm normalisation, the other choice
+    [SM] section 4 allows (largest singular value from LAPACK's SVD)."""
+    return 1.0 / (np.linalg.norm(np.asarray(M, np.float64), 2) + eps)
+
+
 def newton_schulz(M: np.ndarray, a: float, b: float, c: float, iters: int,
-                  eps: float = 1e-7, normalize: bool = True) -> np.ndarray:
+                  eps: float = 1e-7, normalize: bool = True, spectral: bool = False) -> np.ndarray:
     """Polar-factor approximation U = NS_K(M) in float64, same orientation as M.
 
     [SM] core mechanism 1 and flow step 1 (each worker orthogonalises its
     momentum with a Newton-Schulz iteration); [CM] problem statement (the
-    iteration replaces an SVD). Readings R2, R3, R4.
+    iteration replaces an SVD). Readings R2, R3, R4 (spectral: the spectral
+    norm instead of the Frobenius norm).
     """
     M = np.asarray(M, np.float64)
     tall = M.shape[0] > M.shape[1]
     X = M.T if tall else M
     if normalize:
-        X = X * frobenius_scale(M, eps)
+        X = X * (spectral_scale(M, eps) if spectral else frobenius_scale(M, eps))
     X, _ = _ns_core(X, a, b, c, iters, False)
     return X.T if tall else X
 

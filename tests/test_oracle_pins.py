@@ -403,3 +403,20 @@ def test_gram_only_solve_matches_the_x_iteration(shape, iters):
     assert _rel(D2, D1) < 1e-10 and _rel(Q2, Q1) < 1e-10
     # Q is a product of commuting symmetric factors: symmetric
     assert _rel(Q2, Q2.T) < 1e-12
+
+
+@pytest.mark.parametrize("shape", [(6, 10), (10, 6), (12, 12)])
+@pytest.mark.parametrize("coeffs,iters", [(WL.QUINTIC, 1), (WL.QUINTIC, 5), (WL.CUBIC, 5)])
+def test_ns_spectral_scaling_closed_form(shape, coeffs, iters):
+    """Spectral normalisation divides by the largest singular value, so the
+    largest scaled singular value is (almost) exactly 1."""
+    rng = np.random.default_rng(13)
+    M = rng.standard_normal(shape)
+    U, S, Vt = np.linalg.svd(M, full_matrices=False)
+    s = S / (S.max() + 1e-7)
+    assert abs(s.max() - 1.0) < 1e-6
+    expect = (U * _poly(s, coeffs, iters)) @ Vt
+    assert _rel(O.newton_schulz(M, *coeffs, iters, spectral=True), expect) < 1e-10
+    # a rank-one matrix: spectral and Frobenius norms agree
+    r1 = np.outer(rng.standard_normal(shape[0]), rng.standard_normal(shape[1]))
+    assert _rel(O.newton_schulz(r1, *coeffs, iters, spectral=True), O.newton_schulz(r1, *coeffs, iters)) < 1e-12
