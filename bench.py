@@ -76,6 +76,9 @@ def parse_args():
                    help="use only the first LAYERS matrices of the set (a smaller case for profiler captures)")
     p.add_argument("--local-polar", action="store_true",
                    help="GPT-2-small set: orthogonalise the voted matrix before the update")
+    p.add_argument("--spectral", action="store_true",
+                   help="Sign-Muon sets: normalise by the spectral norm (SMUON_NS_SPECTRAL, Lanczos estimate on "
+                        "the device) instead of the Frobenius norm")
     p.add_argument("--gram-only", action="store_true",
                    help="CacheMuon sweep: fresh solves iterated on the m x m Gram (SMUON_NS_GRAM_ONLY)")
     p.add_argument("--cachemuon", nargs="*", metavar="RxC:GAMMA",
@@ -102,7 +105,7 @@ def oracle_step_sample(cfg, W, grads, layer_ids):
     Ms = [[np.zeros(cfg.shapes[i]) for _ in range(cfg.workers)] for i in layer_ids]
     Gs = [grads[i] for i in layer_ids]
     return O.sign_muon_step(Ws, Ms, Gs, cfg.beta, cfg.coeffs, cfg.iters, cfg.eta, cfg.w_dtype,
-                            cfg.tie_value, cfg.vote)
+                            cfg.tie_value, cfg.vote, spectral=_SPECTRAL[0])
 
 
 def layer_cost(shape, cfg):
@@ -121,6 +124,7 @@ def blas_threads():
 
 
 _ORACLE_INPUTS = {}
+_SPECTRAL = [False]  # --spectral: both arms normalise by the spectral norm
 
 
 def time_oracle(cfg, budget_s):
@@ -362,7 +366,8 @@ def oracle_rate(name, budget_s):
 def run_reference(args, rank):
     if rank != 0:
         return
-    desc = describe(args.workload, default_ns_mode(args), args.local_polar)
+    _SPECTRAL[0] = args.spectral
+    desc = describe(args.workload, default_ns_mode(args), args.local_polar, args.spectral)
     budget = max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_rate(args.workload, budget)
@@ -392,7 +397,14 @@ def default_ns_mode(args):
     return "plain" if args.workload in ("c2_resnet50", "resnet18") else "split"
 
 
-def describe(name, ns_mode, local_polar):
+def describe(name, ns_mode, local_polar, spectral=False):
+    d = _describe(name, ns_mode, local_polar)
+    if spectral:
+        d["workload"] += "_spectral_norm"
+    return d
+
+
+def _describe(name, ns_mode, local_polar):
     if name == "c2_resnet50":
         return {"workload": "resnet50_conv_set_53_layers_M4_quintic1_int8_vote",
                 "data": "synthetic (seeded Gaussian gradients N(0,1e-4), He-normal weights)"}
@@ -460,7 +472,7 @@ def setup_c2(S, torch, rank, ns_flags, e2e, layers=0, name="c2_resnet50"):
 
     return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None, "e2e_ns": e2e_ns, "e2e_tail": e2e_tail,
             "g_bytes": n_params * M * 4, "w_bytes": n_params * 4,
-            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], ns_flags != 0, 2),
+            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], bool(ns_flags & S.NS_SPLIT_BF16), 2),
             "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters, "vote": "int8 sum",
                        "l2": f"inputs larger than L2: {n_params * M * 4 / 1e6:.0f} MB of gradients per step, "
                              "two resident sets alternate"}}
@@ -533,7 +545,7 @@ def setup_c3(S, torch, rank, ns_flags, e2e, local_polar, layers=0, name="c3_gpt2
     return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None, "e2e_ns": e2e_ns, "e2e_tail": tail,
             "g_bytes": n_params * M * 4, "w_bytes": n_params * 2,
             "vote_alone": (vote_plan, vote_bytes) if vote_plan is not None else None,
-            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], ns_flags != 0, 2),
+            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], bool(ns_flags & S.NS_SPLIT_BF16), 2),
             "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters,
                        "vote": "1-bit packed, popcount" + (", local polar step" if local_polar else ""),
                        "l2": f"inputs larger than L2: {n_params * M * 4 / 1e9:.1f} GB of gradients per step"
@@ -680,8 +692,11 @@ def main():
             dist.barrier()
 
     ns_mode = default_ns_mode(args)
-    ns_flags = S.NS_SPLIT_BF16 if ns_mode == "split" else 0
-    desc = describe(args.workload, ns_mode, args.local_polar)
+    ns_flags = (S.NS_SPLIT_BF16 if ns_mode == "split" else 0) | (S.NS_SPECTRAL if args.spectral else 0)
+    _SPECTRAL[0] = args.spectral
+    if args.spectral and args.workload == "c5_gpt2l":
+        raise SystemExit("--spectral applies to the Sign-Muon sets")
+    desc = describe(args.workload, ns_mode, args.local_polar, args.spectral)
     e2e_on = args.e2e_steps > 0
     if args.workload in ("c2_resnet50", "resnet18"):
         wl = setup_c2(S, torch, rank, ns_flags, e2e_on, args.layers, args.workload)

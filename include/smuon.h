@@ -51,7 +51,7 @@ typedef int32_t smuon_status;
 #define SMUON_I8   2
 
 /* bits OR-ed into *d_status by device code */
-#define SMUON_DEV_NONFINITE_NORM 1  /* a Frobenius norm was NaN or Inf */
+#define SMUON_DEV_NONFINITE_NORM 1  /* a Frobenius norm (or a spectral-norm estimate) was NaN or Inf */
 #define SMUON_DEV_WAIT_TIMEOUT   2  /* a bounded pipeline wait ran out; results invalid */
 
 /* a row-major matrix in device memory */
@@ -126,6 +126,11 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
 #define SMUON_NS_NO_NORMALIZE  4u  /* skip the Frobenius normalisation (s = 1) */
 #define SMUON_NS_EMIT_Q        8u  /* also write the CacheMuon transform Q */
 #define SMUON_NS_SIMT_BF16    16u  /* diagnostic: BF16 operands on CUDA cores instead of tcgen05 */
+#define SMUON_NS_SPECTRAL     64u  /* normalise by the spectral norm instead: X_0 = M / (||M||_2 + eps)
+                                      (SignMuon summary, section 4: either norm will do); ||M||_2 from a
+                                      24-step Lanczos estimate of the largest eigenvalue of the first Gram
+                                      matrix, per matrix, on the device. Not with SMUON_NS_NO_NORMALIZE,
+                                      SMUON_NS_EMIT_Q or SMUON_NS_GRAM_ONLY */
 #define SMUON_NS_GRAM_ONLY    32u  /* CacheMuon fresh solve iterated on the m x m Gram ("Gram
                                       Newton-Schulz", CacheMuon summary, method item 1): A_0 = X_0 X_0^T once,
                                       then per step P_k = aI + bA_k + cA_k^2, Q_{k+1} = P_k Q_k and

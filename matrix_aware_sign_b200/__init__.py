@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libsmuon.so")
 F32, BF16, I8 = 0, 1, 2
 NS_FP32_REF, NS_SPLIT_BF16, NS_NO_NORMALIZE, NS_EMIT_Q, NS_SIMT_BF16 = 1, 2, 4, 8, 16
 NS_GRAM_ONLY = 32  # CacheMuon fresh solve iterated on the m x m Gram (with NS_EMIT_Q, one matrix)
+NS_SPECTRAL = 64  # spectral-norm normalisation X_0 = M / (||M||_2 + eps) (Lanczos estimate on the device)
 VOTE_POPCOUNT, VOTE_INT8 = 0, 1
 LION_MUON_VOTE = 0x100  # lionmuon_step ns_flags: Muon steps as Sign-Muon steps (per-worker NS + vote)
 DEV_NONFINITE_NORM, DEV_WAIT_TIMEOUT = 1, 2

@@ -210,6 +210,7 @@ struct Layout {
   size_t off_groups = 0, off_mats = 0, off_tmaps = 0;
   size_t off_partials = 0, off_scale = 0, off_probe = 0, off_mom_begin = 0;
   size_t off_sched = 0, off_sched_begin = 0;
+  size_t off_lz_rows = 0, off_rscale = 0, off_lz = 0, off_lz_ab = 0;
   int n_tmaps = 0;
 };
 
@@ -301,6 +302,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   const bool tc = (mode == MODE_TC_BF16);
   const bool emit_q = (rq.flags & SMUON_NS_EMIT_Q) && !rq.probe;
   const bool gram_only = (rq.flags & SMUON_NS_GRAM_ONLY) && !rq.probe;
+  const bool spectral = (rq.flags & SMUON_NS_SPECTRAL) && !rq.probe;
   const int K = rq.iters;
   const int BM = tc ? kTcBM : kSimtBM;
   const size_t esz = bf ? 2 : 4;
@@ -360,6 +362,12 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     B->groups.push_back(g);
   }
   // momentum tiles must be increasing along mats for the device binary search: they are.
+  // spectral scaling: Lanczos vectors v_0 .. v_K and the work vector w of each matrix, m floats each
+  int64_t lz_floats = 0;
+  for (MatDesc& d : B->mats) {
+    d.lz_off = lz_floats;
+    if (spectral) lz_floats += (int64_t)(kLanczosSteps + 2) * B->groups[d.group].m;
+  }
 
   // tile tables: for the symmetric stages the tiles that reach the diagonal or
   // lie above it (BN = ratio * BM), a full grid of BM x BN tiles otherwise
@@ -404,6 +412,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.off_mom_begin = B->take(sizeof(int32_t) * (B->mats.size() + 1));
   L.off_sched = B->take(sizeof(int32_t) * std::max(sched_n, 1));
   L.off_sched_begin = B->take(sizeof(int32_t) * std::max(begin_n, 1));
+  L.off_lz_rows = B->take(sizeof(int32_t) * (B->mats.size() + 1));
   // the B X epilogue reads its X source through a TMA-fed shared-memory ring when every matrix's
   // momentum is f32 with 16-byte aligned rows (later steps read the f32 masters, always aligned)
   bool axpy_tma = tc && !rq.probe && !gram_only;
@@ -459,6 +468,9 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.off_partials = B->take(sizeof(float) * std::max(mom_tiles, 1));
   L.off_scale = B->take(sizeof(float) * B->mats.size());
   L.off_probe = B->take(sizeof(float) * kProbeSlots * std::max(totals[ST_PROBE], 1));
+  L.off_rscale = B->take(sizeof(float) * B->mats.size());
+  L.off_lz = spectral ? B->take(sizeof(float) * lz_floats) : 0;
+  L.off_lz_ab = spectral ? B->take(sizeof(float) * 2 * kLanczosSteps * B->mats.size()) : 0;
 
   // per-group buffers
   for (auto& g : B->groups) {
@@ -480,10 +492,8 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     if (K >= 2 && !gram_only) g.xop[1] = B->ptr_at<void>(B->take(nx * esz * parts));
     if (bf && K >= 2 && !gram_only) g.xf[1] = B->ptr_at<float>(B->take(nx * 4));
     if (bf && K >= 3 && !gram_only) g.xf[0] = B->ptr_at<float>(B->take(nx * 4));
-    if (rq.c != 0.f) {
-      g.af = B->ptr_at<float>(B->take(nm * 4));
-      g.aop = bf ? B->ptr_at<void>(B->take(nm * 2 * parts)) : (void*)g.af;
-    }
+    if (rq.c != 0.f || spectral) g.af = B->ptr_at<float>(B->take(nm * 4));  // f32 A_0 (Lanczos input)
+    if (rq.c != 0.f) g.aop = bf ? B->ptr_at<void>(B->take(nm * 2 * parts)) : (void*)g.af;
     g.bop = B->ptr_at<void>(B->take(nm * esz * parts));
     if (emit_q && (K >= 2 || gram_only)) {
       g.qop[1] = B->ptr_at<void>(B->take(nm * esz * parts));
@@ -515,6 +525,10 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   h.partials = B->ptr_at<float>(L.off_partials);
   h.scale = B->ptr_at<float>(L.off_scale);
   h.probe_partials = B->ptr_at<float>(L.off_probe);
+  h.rscale = B->ptr_at<float>(L.off_rscale);
+  h.lz = spectral ? B->ptr_at<float>(L.off_lz) : nullptr;
+  h.lz_ab = spectral ? B->ptr_at<float>(L.off_lz_ab) : nullptr;
+  h.lz_rows = B->ptr_at<int32_t>(L.off_lz_rows);
   h.mom_begin = B->ptr_at<int32_t>(L.off_mom_begin);
   h.sched = B->ptr_at<int32_t>(L.off_sched);
   h.sched_begin = B->ptr_at<int32_t>(L.off_sched_begin);
@@ -605,6 +619,11 @@ smuon_status upload_plan(Builder& B, cudaStream_t s) {
     memcpy(bytes.data() + B.L.off_mom_begin, mb.data(), sizeof(int32_t) * mb.size());
   }
   memcpy(bytes.data() + B.L.off_sched, B.sched.data(), sizeof(int32_t) * B.sched.size());
+  {  // first row of each matrix's A in the flattened row space of the Lanczos products
+    std::vector<int32_t> lr(B.mats.size() + 1, 0);
+    for (size_t i = 0; i < B.mats.size(); ++i) lr[i + 1] = lr[i] + B.groups[B.mats[i].group].m;
+    memcpy(bytes.data() + B.L.off_lz_rows, lr.data(), sizeof(int32_t) * lr.size());
+  }
   memcpy(bytes.data() + B.L.off_sched_begin, B.sched_begin.data(), sizeof(int32_t) * B.sched_begin.size());
   if (B.L.n_tmaps > 0) memcpy(bytes.data() + B.L.off_tmaps, B.maps.data(), sizeof(CUtensorMap) * B.L.n_tmaps);
   static UploadChunk chunk;  // large parameter block; filled then launched by value
@@ -678,9 +697,10 @@ smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int it
   // trace names: kernel, then the stage after a dot
   static const char* tc_names[2][ST_COUNT] = {
       {"k_gemm_tc.gram", "k_gemm_tc.poly", "k_gemm_tc.axpy", "k_gemm_tc.qaxpy", "k_gemm_tc.reuse", "k_gemm_tc.probe",
-       "k_gemm_tc.aa1", "k_gemm_tc.aa2"},
+       "k_gemm_tc.aa1", "k_gemm_tc.aa2", "k_gemm_tc.qx"},
       {"k_gemm_tc_split.gram", "k_gemm_tc_split.poly", "k_gemm_tc_split.axpy", "k_gemm_tc_split.qaxpy",
-       "k_gemm_tc_split.reuse", "k_gemm_tc_split.probe", "k_gemm_tc_split.aa1", "k_gemm_tc_split.aa2"}};
+       "k_gemm_tc_split.reuse", "k_gemm_tc_split.probe", "k_gemm_tc_split.aa1", "k_gemm_tc_split.aa2",
+       "k_gemm_tc_split.qx"}};
   if (h.mode == MODE_TC_BF16) {
     const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
     Launch L(tc_names[split][st], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
@@ -702,7 +722,7 @@ smuon_status validate_ns(const NsRequest& rq) {
   if (rq.iters < 1 || rq.iters > 64) return fail(SMUON_ERR_INVALID_ARG, "iters=%d must be in 1..64", rq.iters);
   const uint32_t known =
       SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_SIMT_BF16 |
-      SMUON_NS_GRAM_ONLY;
+      SMUON_NS_GRAM_ONLY | SMUON_NS_SPECTRAL;
   if (rq.flags & ~known) return fail(SMUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", rq.flags & ~known);
   const uint32_t modes = rq.flags & (SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_SIMT_BF16);
   if (modes & (modes - 1))
@@ -717,6 +737,9 @@ smuon_status validate_ns(const NsRequest& rq) {
     if (rq.n_mats != 1) return fail(SMUON_ERR_UNSUPPORTED, "SMUON_NS_GRAM_ONLY takes one matrix per call");
     if (rq.c == 0.f) return fail(SMUON_ERR_UNSUPPORTED, "SMUON_NS_GRAM_ONLY needs c != 0");
   }
+  if ((rq.flags & SMUON_NS_SPECTRAL) && (rq.flags & (SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_GRAM_ONLY)))
+    return fail(SMUON_ERR_UNSUPPORTED,
+                "SMUON_NS_SPECTRAL excludes SMUON_NS_NO_NORMALIZE, SMUON_NS_EMIT_Q and SMUON_NS_GRAM_ONLY");
   for (int i = 0; i < rq.n_mats; ++i) {
     smuon_status st;
     const bool has_g = rq.G != nullptr;
@@ -756,6 +779,8 @@ struct NsExec {
   double mom_bytes = 0;
   double sflops[ST_COUNT] = {0};
   double sissued[ST_COUNT] = {0};
+  int64_t lz_rows = 0;          // spectral scaling: rows of all A_0 together
+  double lz_matvec_bytes = 0;   // bytes of one A v product over the batch
 };
 
 smuon_status prepare_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t* d_status, cudaStream_t s,
@@ -774,10 +799,42 @@ smuon_status prepare_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t*
   ex->c = rq.c;
   ex->flags = rq.flags;
   ex->mom_bytes = momentum_bytes(rq, B.h);
+  for (const MatDesc& d : B.mats) {
+    const int m = B.groups[d.group].m;
+    ex->lz_rows += m;
+    ex->lz_matvec_bytes += 4.0 * ((double)m * m + 2.0 * m);
+  }
   for (int k = 0; k < ST_COUNT; ++k) {
     ex->sflops[k] = stage_flops(B, k);
     ex->sissued[k] = stage_issued(B, k);
   }
+  return SMUON_OK;
+}
+
+// spectral scaling: largest eigenvalue of each A_0 by Lanczos, then r = 1/(sqrt(lambda) + eps s)
+smuon_status run_lanczos(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
+  const PlanHeader& h = ex.h;
+  const int sms = ex.di.sms;
+  const int mat_grid = std::max(1, std::min(h.n_mats, sms * 4));
+  {
+    Launch L("k_lz_start", SMUON_WORK_BYTES, 4.0 * ex.lz_rows, s);
+    k_lz_start<<<mat_grid, 256, 0, s>>>(ex.d_plan, skip);
+    CUDA_TRY(cudaGetLastError());
+  }
+  const int row_grid = (int)std::max<int64_t>(1, std::min<int64_t>((ex.lz_rows + 7) / 8, (int64_t)sms * 8));
+  for (int j = 0; j < kLanczosSteps; ++j) {
+    {
+      Launch L("k_lz_matvec", SMUON_WORK_BYTES, ex.lz_matvec_bytes, s);
+      k_lz_matvec<<<row_grid, 256, 0, s>>>(ex.d_plan, j, skip);
+      CUDA_TRY(cudaGetLastError());
+    }
+    Launch L("k_lz_step", SMUON_WORK_BYTES, 4.0 * ex.lz_rows * (j + 6), s);
+    k_lz_step<<<mat_grid, 256, 0, s>>>(ex.d_plan, j, skip);
+    CUDA_TRY(cudaGetLastError());
+  }
+  Launch L("k_lz_finish", SMUON_WORK_BYTES, 8.0 * kLanczosSteps * h.n_mats, s);
+  k_lz_finish<<<(h.n_mats + 127) / 128, 128, 0, s>>>(ex.d_plan, skip);
+  CUDA_TRY(cudaGetLastError());
   return SMUON_OK;
 }
 
@@ -819,6 +876,7 @@ smuon_status run_ns(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
   }
   for (int k = 0; k < ex.iters; ++k) {
     if ((st = launch_gemm(ex.d_plan, h, ST_GRAM, k, skip, di, s, ex.sflops[ST_GRAM], ex.sissued[ST_GRAM])) != SMUON_OK) return st;
+    if (k == 0 && (ex.flags & SMUON_NS_SPECTRAL) && (st = run_lanczos(ex, skip, s)) != SMUON_OK) return st;
     if (ex.c != 0.f && (st = launch_gemm(ex.d_plan, h, ST_POLY, k, skip, di, s, ex.sflops[ST_POLY], ex.sissued[ST_POLY])) != SMUON_OK)
       return st;
     if ((st = launch_gemm(ex.d_plan, h, ST_AXPY, k, skip, di, s, ex.sflops[ST_AXPY], ex.sissued[ST_AXPY])) != SMUON_OK) return st;

@@ -18,6 +18,7 @@ struct TileCtx {
   int32_t stage, iter, last;  // last: this is the final Newton-Schulz step
   int32_t z, Mo, No;
   float s;                    // 1/(||M||_F + eps) of this matrix
+  float r;                    // spectral scaling: s r = 1/(||M||_2 + eps); 1 otherwise
   float a, b, c;
   uint32_t flags;
   int32_t bf;                 // operands are bf16 (tcgen05 or SIMT-bf16 mode)
@@ -296,6 +297,12 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
         sym_store_f32<NV>(t, g.af, row, col0, nvalid, ds, ms, v);
         if (t.bf) sym_store_operand<NV>(t, g.aop, row, col0, nvalid, ds, ms, v);
       } else {
+        if (t.flags & SMUON_NS_SPECTRAL) {  // f32 A_0 for the largest-eigenvalue estimate
+          float a0[NV];
+#pragma unroll
+          for (int k = 0; k < NV; ++k) a0[k] = sc * v[k];
+          sym_store_f32<NV>(t, g.af, row, col0, nvalid, ds, ms, a0);
+        }
 #pragma unroll
         for (int k = 0; k < NV; ++k) v[k] = t.b * (sc * v[k]);
         sym_store_operand<NV>(t, g.bop, row, col0, nvalid, ds, ms, v);
@@ -308,15 +315,20 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
       float A[NV];
       ld_f32_vec<NV>(g.af + off, A);
+      // spectral scaling at the first step: A' = r^2 A, so B = b r^2 A + c r^4 A^2 (r = 1 otherwise)
+      const float r2 = t.iter == 0 ? t.r * t.r : 1.f;
 #pragma unroll
-      for (int k = 0; k < NV; ++k) v[k] = t.b * A[k] + t.c * v[k];
+      for (int k = 0; k < NV; ++k) v[k] = t.b * (r2 * A[k]) + t.c * ((r2 * r2) * v[k]);
       sym_store_operand<NV>(t, g.bop, row, col0, nvalid, ds, ms, v);
       if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, ds, ms, v);
       break;
     }
     case ST_AXPY: {
       const bool first = (t.iter == 0);
-      const float sc = (first && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s : 1.f;
+      // s r: the Frobenius scale, times r for spectral scaling; with c = 0 the first B = b A was
+      // written before r was known, so its product takes the r^2 of A' = r^2 A here
+      const float sc = (first && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s * t.r : 1.f;
+      const float sv = (first && t.c == 0.f) ? sc * (t.r * t.r) : sc;
       const int64_t off = ((int64_t)t.z * m + row) * g.ldn + col0;
       float x[NV];
       if (first && t.bf) {
@@ -328,7 +340,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
         ld_f32_vec<NV>(src + off, x);
       }
 #pragma unroll
-      for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sc * v[k];
+      for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sv * v[k];
       if (t.iter != t.last) {
         const int nb = (t.iter + 1) & 1;
         if (t.bf) st_f32_vec<NV>(g.xf[nb] + off, x);
@@ -407,9 +419,10 @@ __device__ __forceinline__ void epi_axpy_src(const TileCtx& t, int row, int col0
   if (row >= t.Mo || col0 >= t.No) return;
   const int nvalid = min(NV, t.No - col0);
   const GroupDesc& g = *t.g;
-  const float sc = (t.iter == 0 && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s : 1.f;
+  const float sc = (t.iter == 0 && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s * t.r : 1.f;
+  const float sv = (t.iter == 0 && t.c == 0.f) ? sc * (t.r * t.r) : sc;
 #pragma unroll
-  for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sc * v[k];
+  for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sv * v[k];
   if (t.iter != t.last) {
     const int64_t off = ((int64_t)t.z * g.m + row) * g.ldn + col0;
     const int nb = (t.iter + 1) & 1;
@@ -450,6 +463,7 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
   t.Mo = g.m;
   t.No = wide_out_stage(st) ? g.n : g.m;
   t.s = h.scale[g.first_mat + t.z];
+  t.r = (h.flags & SMUON_NS_SPECTRAL) ? h.rscale[g.first_mat + t.z] : 1.f;
   t.a = h.a; t.b = h.b; t.c = h.c;
   t.flags = h.flags;
   t.bf = (h.mode != MODE_SIMT_F32);

@@ -69,6 +69,13 @@ __global__ void k_vote(const uint32_t* packed, const int8_t* signs, int M, int64
                        int tie, int8_t* vote);
 __global__ void k_update_src(const __grid_constant__ EwTable tb);
 __global__ void k_harness_gaussian(const __grid_constant__ EwTable tb);
+
+// spectral scaling (k_spectral.cu)
+constexpr int kLanczosSteps = 24;
+__global__ void k_lz_start(const Plan* plan, const int32_t* skip);
+__global__ void k_lz_matvec(const Plan* plan, int j, const int32_t* skip);
+__global__ void k_lz_step(const Plan* plan, int j, const int32_t* skip);
+__global__ void k_lz_finish(const Plan* plan, const int32_t* skip);
 __global__ void k_lion_sign(const __grid_constant__ EwTable tb);
 __global__ void k_lion_mean(const __grid_constant__ EwTable tb);
 __global__ void k_probe_finalize(const Plan* plan);

@@ -65,6 +65,7 @@ struct MatDesc {
   int32_t mom_count;      // number of momentum tiles
   int32_t tm_src;         // f32 map of M for the first B X epilogue's source (-1: none)
   int32_t pad0;
+  int64_t lz_off;         // spectral scaling: this matrix's Lanczos vectors in PlanHeader::lz
 };
 
 // matrices of one wide shape m x n, stored contiguously in the workspace
@@ -117,6 +118,10 @@ struct PlanHeader {
   int32_t sched_ctas[ST_COUNT];     // CTAs of each stage's launch
   int32_t max_k[ST_COUNT];          // longest K of each stage over the groups (picks the smem ring depth)
   int32_t axpy_tma;                 // the B X epilogue's X source is staged in shared memory by TMA
+  float* rscale;                    // spectral scaling: r per matrix (X_0 = s r M), or null
+  float* lz;                        // Lanczos vectors of every matrix (kLanczosSteps + 2 vectors of m each)
+  float* lz_ab;                     // [n_mats][2 kLanczosSteps] Lanczos alpha, beta
+  const int32_t* lz_rows;           // [n_mats + 1] first row of each matrix in the flattened row range
   GroupDesc* groups;        // device pointers into the plan region
   MatDesc* mats;
   CUtensorMap* tmaps;

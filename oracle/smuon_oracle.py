@@ -273,18 +273,19 @@ def update_dense(W: np.ndarray, D: np.ndarray, eta: float, dtype: str) -> np.nda
 # whole Sign-Muon step ([SM] flow steps 1-5)
 # --------------------------------------------------------------------------
 def sign_muon_step(W_layers, M_layers, G_layers, beta, coeffs, iters, eta, w_dtype,
-                   tie_value=0, vote_kind="popcount", local_polar=False, eps=1e-7):
+                   tie_value=0, vote_kind="popcount", local_polar=False, eps=1e-7, spectral=False):
     """One distributed Sign-Muon step over a set of layers, with the M workers
     simulated: per layer and worker, momentum -> Newton-Schulz polar factor ->
     sign; then the vote over workers and the update; optionally a local polar
-    step on the voted matrix ([SM] flow steps 1-5).
+    step on the voted matrix ([SM] flow steps 1-5). spectral: the spectral-norm
+    normalisation of reading R4 in every Newton-Schulz call.
 
     Returns dict(W=[...], M=[[...]], U=[[...]], vote=[...]) (new lists)."""
     a, b, c = coeffs
     W_out, M_out, U_out, V_out = [], [], [], []
     for W, Ms, Gs in zip(W_layers, M_layers, G_layers):
         Ms_new = [momentum(Mm, Gm, beta) for Mm, Gm in zip(Ms, Gs)]
-        Us = [newton_schulz(Mm, a, b, c, iters, eps) for Mm in Ms_new]
+        Us = [newton_schulz(Mm, a, b, c, iters, eps, spectral=spectral) for Mm in Ms_new]
         signs = [sign_extract(U) for U in Us]
         if vote_kind == "int8":
             v = vote_from_signs(signs, tie_value)
@@ -293,7 +294,7 @@ def sign_muon_step(W_layers, M_layers, G_layers, beta, coeffs, iters, eta, w_dty
             v = vote_from_packed([pack_bits(s) for s in signs], len(signs), n,
                                  tie_value).reshape(signs[0].shape)
         if local_polar:
-            D = newton_schulz(v.astype(np.float64), a, b, c, iters, eps)
+            D = newton_schulz(v.astype(np.float64), a, b, c, iters, eps, spectral=spectral)
             Wn = update_dense(W, D, eta, w_dtype)
         else:
             Wn = update_with_vote(W, v, eta, w_dtype)

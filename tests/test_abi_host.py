@@ -128,3 +128,24 @@ def test_gram_only_rejects_unsupported_requests(L):
                       None, 0, None, None) == -4
     assert L.smuon_ns(m, m, 1, None, 0.0, 1.5, -0.5, *args(0.0), g | S.NS_EMIT_Q, q, None, None, 0, None,
                       None) == -4
+
+
+def test_spectral_flag_validation_and_workspace(L):
+    """SMUON_NS_SPECTRAL excludes NO_NORMALIZE, EMIT_Q and GRAM_ONLY; its
+    workspace adds the Lanczos vectors (26 vectors of m floats per matrix, the
+    tridiagonal coefficients and the f32 Gram matrix even for c = 0)."""
+    import torch
+    import matrix_aware_sign_b200 as S
+    m = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 16, 16, S.F32))
+    q = (S.SmuonMat * 1)(S.SmuonMat(8192, 8, 8, 8, S.BF16))
+    sp = S.NS_SPECTRAL
+    for extra in (S.NS_NO_NORMALIZE, S.NS_EMIT_Q, S.NS_GRAM_ONLY | S.NS_EMIT_Q):
+        assert L.smuon_ns(m, m, 1, None, 0.0, 3.4445, -4.775, 2.0315, 5, 1e-7, sp | extra, q, None, None, 0, None,
+                          None) == -4
+        assert b"SMUON_NS_SPECTRAL" in L.smuon_last_error()
+    mats = [torch.zeros(s) for s in [(256, 1024), (64, 147), (300, 200)]]
+    for flags in (0, S.NS_SPLIT_BF16, S.NS_FP32_REF):
+        base = S.smuon_ns_workspace_bytes(mats, 5, flags)
+        spec = S.smuon_ns_workspace_bytes(mats, 5, flags | sp)
+        lz = 4 * 26 * (256 + 64 + 200) + 4 * 2 * 24 * 3
+        assert base + lz <= spec <= base + lz + 4 * 256 * 4, (base, spec)

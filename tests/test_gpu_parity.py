@@ -226,6 +226,80 @@ def test_ns_nonfinite_norm_sets_status():
     assert int(status.item()) & S.DEV_NONFINITE_NORM
 
 
+SPECTRAL_CASES = [
+    ((256, 1024), WL.QUINTIC, 5),
+    ((1024, 256), WL.QUINTIC, 1),
+    ((512, 512), WL.CUBIC, 5),
+    ((129, 513), WL.CUBIC, 2),
+    ((200, 700), WL.QUINTIC, 5),
+    ((1, 40), WL.QUINTIC, 1),
+]
+
+
+@pytest.mark.parametrize("shape,coeffs,iters", SPECTRAL_CASES)
+@pytest.mark.parametrize("mode,tol", [(S.NS_FP32_REF, 1e-4), (S.NS_SPLIT_BF16, 1e-2)])
+def test_ns_spectral_scaling(shape, coeffs, iters, mode, tol):
+    """SMUON_NS_SPECTRAL: X_0 = M / (||M||_2 + eps) with ||M||_2 from the
+    device's Lanczos estimate; the oracle takes ||M||_2 from an SVD."""
+    rng = np.random.default_rng(shape[0] * 3 + iters)
+    M = rng.standard_normal(shape).astype(np.float32)
+    _, Ud = _ns_run([M], coeffs, iters, mode | S.NS_SPECTRAL)
+    ref = O.newton_schulz(M, *coeffs, iters, spectral=True)
+    check_ns_outputs([(host(Ud[0]), ref)], tol)
+
+
+@pytest.mark.parametrize("mode", [0, S.NS_SIMT_BF16, S.NS_SPLIT_BF16, S.NS_FP32_REF])
+def test_ns_spectral_scaling_batched_groups(mode):
+    """Spectral scaling over a batch of several groups, tall and wide, one
+    Lanczos run per matrix (the flattened row space spans all of them), with
+    the momentum update fused in front and one zero matrix (status stays 0).
+    Plain BF16 operands keep the Frobenius error under 1e-2 but not the sign
+    criterion here: X_0 has its largest singular value at 1, so the rounding
+    of A and B enters the first step at full weight (about 4e-4 of the signs
+    flip); the split mode meets both."""
+    shapes = [(64, 147), (256, 64), (300, 200), (128, 512), (64, 147), (512, 128), (96, 96)]
+    rng = np.random.default_rng(41)
+    M0 = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    G = [rng.standard_normal(s).astype(np.float32) for s in shapes]
+    M0[4][:] = 0.0
+    G[4][:] = 0.0
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Md, Ud = _ns_run(M0, WL.QUINTIC, 1, mode | S.NS_SPECTRAL, G=G, beta=0.9, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    pairs = []
+    for m0, g, md, u in zip(M0, G, Md, Ud):
+        Mn = O.momentum(m0, g, 0.9)
+        np.testing.assert_allclose(host(md), Mn, rtol=2e-6, atol=1e-6)
+        pairs.append((host(u), O.newton_schulz(Mn, *WL.QUINTIC, 1, spectral=True)))
+    assert np.all(pairs[4][0] == 0.0)
+    rest = pairs[:4] + pairs[5:]
+    if mode in (0, S.NS_SIMT_BF16):
+        assert max(rel_fro(u, r) for u, r in rest) < 1e-2
+    else:
+        check_ns_outputs(rest, 1e-4 if mode == S.NS_FP32_REF else 1e-2)
+
+
+def test_ns_spectral_rank_two_closed_form():
+    """Closed form: M = 3 u1 v1^T + 1.2 u2 v2^T (orthonormal u, v). Spectral
+    scaling gives X_0 singular values 1 and rho = 0.4, and one cubic step
+    (c = 0) maps them to a + b = 1 and a rho + b rho^3; the Frobenius scaling
+    would give 1/sqrt(1 + rho^2) for the first. The Lanczos run breaks down
+    after two steps here, so this also covers its early stop."""
+    rng = np.random.default_rng(5)
+    Uo, _ = np.linalg.qr(rng.standard_normal((96, 2)))
+    Vo, _ = np.linalg.qr(rng.standard_normal((300, 2)))
+    M = (3.0 * np.outer(Uo[:, 0], Vo[:, 0]) + 1.2 * np.outer(Uo[:, 1], Vo[:, 1])).astype(np.float32)
+    a, b = WL.CUBIC[0], WL.CUBIC[1]
+    rho = 0.4
+    want = np.outer(Uo[:, 0], Vo[:, 0]) * (a + b) + np.outer(Uo[:, 1], Vo[:, 1]) * (a * rho + b * rho ** 3)
+    for mode, tol in [(S.NS_FP32_REF, 1e-5), (S.NS_SPLIT_BF16, 2e-3)]:
+        _, Ud = _ns_run([M], WL.CUBIC, 1, mode | S.NS_SPECTRAL)
+        assert rel_fro(host(Ud[0]), want) < tol
+        _, Uf = _ns_run([M], WL.CUBIC, 1, mode)  # the Frobenius scaling differs by far more
+        assert rel_fro(host(Uf[0]), want) > 0.02
+
+
 def test_ns_skip_flag_leaves_outputs_untouched():
     M = np.random.default_rng(1).standard_normal((64, 96)).astype(np.float32)
     Md = [dev(M)]
