@@ -76,6 +76,8 @@ def parse_args():
                    help="use only the first LAYERS matrices of the set (a smaller case for profiler captures)")
     p.add_argument("--local-polar", action="store_true",
                    help="GPT-2-small set: orthogonalise the voted matrix before the update")
+    p.add_argument("--sign-out", choices=["i8", "bf16"], default="i8",
+                   help="ResNet sets: the NS epilogue writes the int8 signs (default) or bf16 U for the vote kernel")
     p.add_argument("--spectral", action="store_true",
                    help="Sign-Muon sets: normalise by the spectral norm (SMUON_NS_SPECTRAL, Lanczos estimate on "
                         "the device) instead of the Frobenius norm")
@@ -429,9 +431,12 @@ def subset(shapes, layers):
     return shapes[:layers] if layers > 0 else shapes
 
 
-def setup_c2(S, torch, rank, ns_flags, e2e, layers=0, name="c2_resnet50"):
+def setup_c2(S, torch, rank, ns_flags, e2e, layers=0, name="c2_resnet50", sign_out="i8"):
     """ResNet layer sets, M = 4: momentum + one quintic NS step (prepared
-    plans on two resident gradient sets) + fused sign / int8-sum vote / update."""
+    plans on two resident gradient sets) + int8-sum vote / update. With
+    sign_out = "i8" the NS epilogue writes the workers' int8 sign matrices
+    (no U in memory) and the vote kernel sums them; with "bf16" it writes U
+    and the vote kernel takes the signs."""
     cfg = WL.SIGN_MUON_WORKLOADS[name]
     M, shapes = cfg.workers, subset(cfg.shapes, layers)
     L = len(shapes)
@@ -440,7 +445,8 @@ def setup_c2(S, torch, rank, ns_flags, e2e, layers=0, name="c2_resnet50"):
     gsets = [streams.next_step(), streams.next_step()]
     Wd = [torch.from_numpy(w).cuda() for w in W]
     Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
-    Ud = [torch.zeros(s, dtype=torch.bfloat16, device="cuda") for s in shapes for _ in range(M)]
+    u_dtype = torch.int8 if sign_out == "i8" else torch.bfloat16
+    Ud = [torch.zeros(s, dtype=u_dtype, device="cuda") for s in shapes for _ in range(M)]
     Gd = [[torch.from_numpy(g).cuda() for layer in gs for g in layer] for gs in gsets]
     Ul = [Ud[l * M:(l + 1) * M] for l in range(L)]
     nbytes = S.smuon_ns_workspace_bytes(Md, cfg.iters, ns_flags)
@@ -472,8 +478,10 @@ def setup_c2(S, torch, rank, ns_flags, e2e, layers=0, name="c2_resnet50"):
 
     return {"step": step, "graphable": True, "e2e_io": e2e_io if e2e else None, "e2e_ns": e2e_ns, "e2e_tail": e2e_tail,
             "g_bytes": n_params * M * 4, "w_bytes": n_params * 4,
-            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], bool(ns_flags & S.NS_SPLIT_BF16), 2),
+            "stage_bytes": gemm_stage_bytes(shapes, M, cfg.iters, cfg.coeffs[2], bool(ns_flags & S.NS_SPLIT_BF16),
+                                            1 if sign_out == "i8" else 2),
             "config": {"layers": L, "params": n_params, "workers": M, "ns_iters": cfg.iters, "vote": "int8 sum",
+                       "ns_output": "int8 signs from the NS epilogue" if sign_out == "i8" else "bf16 U",
                        "l2": f"inputs larger than L2: {n_params * M * 4 / 1e6:.0f} MB of gradients per step, "
                              "two resident sets alternate"}}
 
@@ -699,7 +707,7 @@ def main():
     desc = describe(args.workload, ns_mode, args.local_polar, args.spectral)
     e2e_on = args.e2e_steps > 0
     if args.workload in ("c2_resnet50", "resnet18"):
-        wl = setup_c2(S, torch, rank, ns_flags, e2e_on, args.layers, args.workload)
+        wl = setup_c2(S, torch, rank, ns_flags, e2e_on, args.layers, args.workload, args.sign_out)
     elif args.workload == "c3_gpt2s" or args.workload.startswith("llama"):
         wl = setup_c3(S, torch, rank, ns_flags, e2e_on and args.workload == "c3_gpt2s", args.local_polar,
                       args.layers, args.workload)

@@ -102,7 +102,11 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
  *
  *  M_in[n_mats]   momentum matrices (F32; BF16 or I8 accepted when G == NULL).
  *                 Updated in place when G != NULL.
- *  U_out[n_mats]  polar-factor outputs, same shape as M_in[i] (F32 or BF16).
+ *  U_out[n_mats]  polar-factor outputs, same shape as M_in[i] (F32 or BF16),
+ *                 or I8: then only the entrywise sign of U is written, +1 for
+ *                 u >= 0 (-0 included) and -1 otherwise (NaN included), taken on
+ *                 the float32 value in the last step's epilogue (SignMuon
+ *                 summary, flow step 2: the sign matrix without U in memory).
  *  G[n_mats]      nullable gradients (F32 or BF16), same shapes.
  *  beta           momentum coefficient (ignored when G == NULL).
  *  a, b, c        Newton-Schulz coefficients; c == 0 skips the A^2 product.
@@ -222,6 +226,8 @@ smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t 
  *
  * Exactly one source per call:
  *  U[n_layers*M]     (worker-minor) -> fused sign / vote / update in one pass;
+ *                    F32, BF16, or I8 sign matrices (entry >= 0 counts as +1;
+ *                    I8 takes no packed_out: pack with smuon_sign_pack);
  *                    vote_kind SMUON_VOTE_POPCOUNT (bit masks + popcount) or
  *                    SMUON_VOTE_INT8 (integer sum); both give the same vote.
  *                    Optional outputs: packed_out[l] ([M][words] message, the

@@ -744,7 +744,7 @@ smuon_status validate_ns(const NsRequest& rq) {
     smuon_status st;
     const bool has_g = rq.G != nullptr;
     if ((st = check_mat(rq.M_in[i], "M_in", i, true, !has_g, !has_g)) != SMUON_OK) return st;
-    if ((st = check_mat(rq.U_out[i], "U_out", i, true, true, false)) != SMUON_OK) return st;
+    if ((st = check_mat(rq.U_out[i], "U_out", i, true, true, true)) != SMUON_OK) return st;
     if (!same_shape(rq.M_in[i], rq.U_out[i])) return fail(SMUON_ERR_SHAPE, "U_out[%d] shape differs from M_in", i);
     if (has_g) {
       if ((st = check_mat(rq.G[i], "G", i, true, true, false)) != SMUON_OK) return st;
@@ -1112,7 +1112,7 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
     if (U) {
       for (int k = 0; k < M; ++k) {
         const smuon_mat& u = U[(int64_t)l * M + k];
-        if ((st = check_mat(u, "U", l * M + k, true, true, false)) != SMUON_OK) return st;
+        if ((st = check_mat(u, "U", l * M + k, true, true, true)) != SMUON_OK) return st;
         if (!same_shape(u, shape)) return fail(SMUON_ERR_SHAPE, "U[%d] shape differs from W[%d]", l * M + k, l);
         if (src_dtype >= 0 && u.dtype != src_dtype) return fail(SMUON_ERR_DTYPE, "all U must share one dtype");
         src_dtype = u.dtype;
@@ -1120,6 +1120,8 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
         srcs.push_back(EwSrc{u.data, u.ld});
       }
       if (packed_out && packed_out[l]) {
+        if (src_dtype == SMUON_I8)
+          return fail(SMUON_ERR_UNSUPPORTED, "packed_out needs F32 or BF16 U (pack I8 signs with smuon_sign_pack)");
         if (reinterpret_cast<uintptr_t>(packed_out[l]) % 16)
           return fail(SMUON_ERR_INVALID_ARG, "packed_out[%d] must be 16-byte aligned", l);
         L.packed_out = packed_out[l];

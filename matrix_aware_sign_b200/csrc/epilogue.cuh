@@ -183,6 +183,23 @@ __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int 
         st_f32_vec<NV>(reinterpret_cast<float*>(p) + base, v);
         return;
       }
+      if (dtype == SMUON_I8) {  // the signs only: four entries per 32-bit word
+        uint32_t pk[NV / 4];
+#pragma unroll
+        for (int k = 0; k < NV / 4; ++k)
+          pk[k] = (uint32_t)(uint8_t)sign_i8(v[4 * k]) | ((uint32_t)(uint8_t)sign_i8(v[4 * k + 1]) << 8) |
+                  ((uint32_t)(uint8_t)sign_i8(v[4 * k + 2]) << 16) | ((uint32_t)(uint8_t)sign_i8(v[4 * k + 3]) << 24);
+        uint32_t* q = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(p) + base);
+        if (NV % 16 == 0) {
+#pragma unroll
+          for (int k = 0; k < NV / 16; ++k)
+            reinterpret_cast<uint4*>(q)[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < NV / 4; ++k) q[k] = pk[k];
+        }
+        return;
+      }
       st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(p) + base, v);
       return;
     }
@@ -194,6 +211,11 @@ __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int 
 #pragma unroll
     for (int k = 0; k < NV; ++k)
       if (k < nvalid) q[(int64_t)(col0 + k) * ld] = __float2bfloat16_rn(v[k]);
+  } else if (dtype == SMUON_I8) {
+    int8_t* q = reinterpret_cast<int8_t*>(p) + row;
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+      if (k < nvalid) q[(int64_t)(col0 + k) * ld] = sign_i8(v[k]);
   } else {
     float* q = reinterpret_cast<float*>(p) + row;
 #pragma unroll

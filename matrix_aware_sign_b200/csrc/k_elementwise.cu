@@ -445,6 +445,70 @@ __device__ __forceinline__ void vote_update_int8_bf16(const EwTable& tb) {
   }
 }
 
+// int8 sum-then-sign vote on int8 sign matrices (the signs written by a
+// Newton-Schulz call with an I8 output): an entry counts as positive when its
+// sign bit is clear (+1, and 0 by the u >= 0 rule). Each lane takes 16
+// consecutive entries, one 16-byte load per worker; the positive flags add
+// up per byte (M <= 64, no carries), and the byte counts are spread into the
+// 16-bit lanes vote_finish8 takes.
+template <bool kHasW>
+__device__ __forceinline__ void vote_update_i8src(const EwTable& tb) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int M = tb.M;
+  for (int64_t wbase = warp_global * 64; wbase < tb.total_chunks; wbase += warps_total * 64) {
+    const int64_t chunk = wbase + 2 * lane;
+    const bool active = chunk < tb.total_chunks;
+    const int li = warp_layer(tb, wbase, active ? chunk : tb.total_chunks - 1, lane);
+    const EwLayer& L = tb.layers[li];
+    const int64_t e0 = (chunk - L.chunk_begin) * 8;
+    if (!(active && e0 < L.n)) continue;
+    if (L.vec && e0 + 16 <= L.n) {
+      uint32_t b[4] = {0u, 0u, 0u, 0u};  // per byte: positive signs of entries e0 + 4i .. e0 + 4i + 3
+      for (int wk0 = 0; wk0 < M; wk0 += 8) {
+        uint4 u[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (wk0 + j < M) u[j] = *reinterpret_cast<const uint4*>(
+                               reinterpret_cast<const int8_t*>(tb.srcs[L.src_first + wk0 + j].ptr) + e0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (wk0 + j < M) {
+            b[0] += (~u[j].x >> 7) & 0x01010101u;
+            b[1] += (~u[j].y >> 7) & 0x01010101u;
+            b[2] += (~u[j].z >> 7) & 0x01010101u;
+            b[3] += (~u[j].w >> 7) & 0x01010101u;
+          }
+      }
+      uint32_t cnt[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        cnt[2 * i] = __byte_perm(b[i], 0u, 0x4140);      // entries 4i, 4i + 1 in the low and high halves
+        cnt[2 * i + 1] = __byte_perm(b[i], 0u, 0x4342);  // entries 4i + 2, 4i + 3
+      }
+      vote_finish8<kHasW>(tb, L, e0, cnt);
+      vote_finish8<kHasW>(tb, L, e0 + 8, cnt + 4);
+    } else {
+      const int nent = (int)min((int64_t)16, L.n - e0);
+      for (int k = 0; k < nent; ++k) {
+        const int64_t e = e0 + k;
+        int c = 0;
+        for (int wk = 0; wk < M; ++wk) {
+          const EwSrc& S = tb.srcs[L.src_first + wk];
+          c += reinterpret_cast<const int8_t*>(S.ptr)[ew_index(L, e, S.ld)] >= 0 ? 1 : 0;
+        }
+        const int8_t v = threshold(2 * c - M, tb.tie);
+        if (L.w) {
+          const int64_t wi = ew_index(L, e, L.w_ld);
+          store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+        }
+        if (L.vote_out) L.vote_out[e] = v;
+      }
+    }
+  }
+}
+
 // the 16 message bits of one lane (bit j = entry e0 + j is >= 0) from the
 // per-half flags of its 8 words (bit 0: entry 2i, bit 16: entry 2i + 1)
 __device__ __forceinline__ uint32_t mask16_from_halves(const uint32_t* p) {
@@ -632,12 +696,22 @@ __global__ void __launch_bounds__(256, 3) k_vote_update_bf16x16(const __grid_con
   vote_update_bf16x16<kHasW>(tb);
 }
 
+template <bool kHasW>
+__global__ void __launch_bounds__(256, 3) k_vote_update_i8src(const __grid_constant__ EwTable tb) {
+  vote_update_i8src<kHasW>(tb);
+}
+
 cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s) {
   const bool bf = tb.src_dtype == SMUON_BF16;
   // 16 entries per lane, three resident CTAs per SM (launch bounds), one wave
   const int64_t want16 = (tb.total_chunks + 511) / 512;
   const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
   const bool has_w = tb.layers[0].w != nullptr;  // all layers or none (signs and votes only)
+  if (tb.src_dtype == SMUON_I8) {  // sign matrices: both vote kinds count the same positives
+    if (has_w) k_vote_update_i8src<true><<<grid16, 256, 0, s>>>(tb);
+    else k_vote_update_i8src<false><<<grid16, 256, 0, s>>>(tb);
+    return cudaGetLastError();
+  }
   if (bf && (popcount || tb.any_packed) && tb.M <= kMaxWorkers) {
     if (has_w) k_vote_update_bf16x16<true><<<grid16, 256, 0, s>>>(tb);
     else k_vote_update_bf16x16<false><<<grid16, 256, 0, s>>>(tb);

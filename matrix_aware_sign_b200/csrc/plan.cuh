@@ -145,8 +145,12 @@ __device__ inline float load_as_f32(const void* p, int64_t idx, int32_t dtype) {
   return (float)reinterpret_cast<const int8_t*>(p)[idx];
 }
 
+// an I8 destination receives the entrywise sign: +1 for v >= 0 (-0 included), -1 otherwise (NaN included)
+__device__ inline int8_t sign_i8(float v) { return v >= 0.f ? (int8_t)1 : (int8_t)-1; }
+
 __device__ inline void store_from_f32(void* p, int64_t idx, int32_t dtype, float v) {
   if (dtype == SMUON_F32) reinterpret_cast<float*>(p)[idx] = v;
+  else if (dtype == SMUON_I8) reinterpret_cast<int8_t*>(p)[idx] = sign_i8(v);
   else reinterpret_cast<__nv_bfloat16*>(p)[idx] = __float2bfloat16_rn(v);
 }
 

@@ -149,3 +149,15 @@ def test_spectral_flag_validation_and_workspace(L):
         spec = S.smuon_ns_workspace_bytes(mats, 5, flags | sp)
         lz = 4 * 26 * (256 + 64 + 200) + 4 * 2 * 24 * 3
         assert base + lz <= spec <= base + lz + 4 * 256 * 4, (base, spec)
+
+
+def test_int8_sign_sources_reject_packed_message(L):
+    """I8 sign matrices are accepted as the U source of smuon_update, but not
+    with packed_out (the message is packed by smuon_sign_pack)."""
+    import ctypes
+    import matrix_aware_sign_b200 as S
+    W = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 32, 32, S.F32))
+    U = (S.SmuonMat * 2)(S.SmuonMat(8192, 8, 32, 32, S.I8), S.SmuonMat(12288, 8, 32, 32, S.I8))
+    packed = (ctypes.c_void_p * 1)(16384)
+    assert L.smuon_update(W, 1, U, None, None, 2, 0.01, 0, S.VOTE_INT8, packed, None, None) == -4
+    assert b"packed_out needs F32 or BF16 U" in L.smuon_last_error()

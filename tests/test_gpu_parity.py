@@ -92,6 +92,36 @@ def test_fused_update_strided_matrices():
 
 
 @pytest.mark.parametrize("wdtype", ["f32", "bf16"])
+@pytest.mark.parametrize("kind", [S.VOTE_POPCOUNT, S.VOTE_INT8])
+@pytest.mark.parametrize("M,tie", [(1, 0), (3, 0), (4, 0), (4, -1), (8, 1), (64, 0)])
+def test_fused_vote_update_from_int8_signs(wdtype, kind, M, tie):
+    """I8 sign matrices as the U source (what a Newton-Schulz call with I8
+    outputs writes): entries >= 0 count as +1, so a 0 votes like +1; ragged,
+    tiny and strided layers take the entry-by-entry path. Bit-exact W and votes."""
+    shapes = [(64, 147), (7, 13), (256, 256), (1, 1), (130, 300), (37, 50)]
+    W = WL.weights(shapes, "normal002", wdtype)
+    tw = torch.bfloat16 if wdtype == "bf16" else torch.float32
+    Wd = [dev(w, tw) for w in W]
+    rng = np.random.default_rng(M * 7 + tie + 3)
+    U = [[rng.choice(np.array([-1, 0, 1], np.int8), size=sh, p=[0.48, 0.04, 0.48]) for _ in range(M)]
+         for sh in shapes]
+    Ud = [[dev(u, torch.int8) for u in layer] for layer in U]
+    # the last layer strided: ld 64 > cols 50
+    big = [torch.zeros((37, 64), dtype=torch.int8, device="cuda") for _ in range(M)]
+    for k in range(M):
+        big[k][:, :50] = Ud[-1][k]
+    Ud[-1] = [b[:, :50] for b in big]
+    votes = [torch.zeros(r * c, dtype=torch.int8, device="cuda") for r, c in shapes]
+    eta = 0.02
+    S.smuon_update(Wd, eta, U=Ud, M=M, tie_value=tie, vote_kind=kind, vote_out=votes)
+    torch.cuda.synchronize()
+    for i, sh in enumerate(shapes):
+        v = O.vote_from_signs([O.sign_extract(u.astype(np.float64)) for u in U[i]], tie)
+        np.testing.assert_array_equal(host(votes[i]).reshape(sh), v)
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, eta, wdtype))
+
+
+@pytest.mark.parametrize("wdtype", ["f32", "bf16"])
 def test_update_from_votes_and_dense(wdtype):
     shapes = [(65, 33), (128, 256)]
     tw = torch.bfloat16 if wdtype == "bf16" else torch.float32
@@ -125,7 +155,8 @@ NS_CASES = [
 
 def _ns_run(mats, coeffs, iters, flags, G=None, beta=0.0, udtype=torch.float32, status=None):
     Md = [dev(m) for m in mats]
-    Ud = [torch.full(m.shape, float("nan"), dtype=udtype, device="cuda") for m in mats]
+    fill = 85 if udtype == torch.int8 else float("nan")  # unwritten entries stay visible
+    Ud = [torch.full(m.shape, fill, dtype=udtype, device="cuda") for m in mats]
     Gd = None if G is None else [dev(g) for g in G]
     S.smuon_ns(Md, Ud, *coeffs, iters, G=Gd, beta=beta, flags=flags, status=status)
     torch.cuda.synchronize()
@@ -298,6 +329,67 @@ def test_ns_spectral_rank_two_closed_form():
         assert rel_fro(host(Ud[0]), want) < tol
         _, Uf = _ns_run([M], WL.CUBIC, 1, mode)  # the Frobenius scaling differs by far more
         assert rel_fro(host(Uf[0]), want) > 0.02
+
+
+I8_OUT_CASES = [
+    ((256, 1024), WL.QUINTIC, 1, 0),
+    ((1024, 256), WL.QUINTIC, 1, 0),
+    ((200, 700), WL.QUINTIC, 5, S.NS_SPLIT_BF16),
+    ((300, 130), WL.CUBIC, 2, S.NS_FP32_REF),
+    ((96, 160), WL.QUINTIC, 1, S.NS_SIMT_BF16),
+    ((33, 65), WL.QUINTIC, 1, 0),
+]
+
+
+@pytest.mark.parametrize("shape,coeffs,iters,mode", I8_OUT_CASES)
+def test_ns_int8_sign_output(shape, coeffs, iters, mode):
+    """An I8 U_out receives sign(U) from the last step's epilogue: equal to the
+    sign of the F32 output of the same call (same kernels, same order), and
+    within the sign criterion of the oracle. Ragged widths and odd leading
+    sizes (65, 130) take the element stores."""
+    rng = np.random.default_rng(shape[0] + 17 * iters)
+    M = rng.standard_normal(shape).astype(np.float32)
+    _, Uf = _ns_run([M], coeffs, iters, mode)
+    _, Ui = _ns_run([M], coeffs, iters, mode, udtype=torch.int8)
+    si = host(Ui[0])
+    np.testing.assert_array_equal(si, O.sign_extract(host(Uf[0])))
+    ref = O.newton_schulz(M, *coeffs, iters)
+    dis = (si >= 0) != (ref >= 0)
+    assert dis.sum() <= 1e-4 * dis.size
+    if dis.any():
+        assert np.abs(ref[dis]).max() < 1e-3 * np.abs(ref).max()
+
+
+def test_ns_int8_sign_output_batched_with_vote():
+    """The ResNet-style chain with int8 signs: momentum + one quintic step
+    writing I8 signs for M = 4 workers, then the int8-sum vote and update on
+    them, against the oracle's Sign-Muon step (votes where no worker's U is
+    near zero must agree; W bit-exact where the votes agree)."""
+    shapes = [(64, 147), (256, 64), (128, 576), (512, 128)]
+    Mw = 4
+    rng = np.random.default_rng(77)
+    W = WL.weights(shapes, "he", "f32")
+    G = [[(1e-2 * rng.standard_normal(sh)).astype(np.float32) for _ in range(Mw)] for sh in shapes]
+    Md = [torch.zeros(sh, device="cuda") for sh in shapes for _ in range(Mw)]
+    Ud = [torch.zeros(sh, dtype=torch.int8, device="cuda") for sh in shapes for _ in range(Mw)]
+    Gd = [dev(g) for layer in G for g in layer]
+    Wd = [dev(w) for w in W]
+    S.smuon_ns(Md, Ud, *WL.QUINTIC, 1, G=Gd, beta=0.9)
+    S.smuon_update(Wd, 0.02, U=[Ud[l * Mw:(l + 1) * Mw] for l in range(len(shapes))], M=Mw,
+                   vote_kind=S.VOTE_INT8)
+    torch.cuda.synchronize()
+    ref = O.sign_muon_step(W, [[np.zeros(sh) for _ in range(Mw)] for sh in shapes], G, 0.9, WL.QUINTIC, 1,
+                           0.02, "f32", vote_kind="int8")
+    for l, sh in enumerate(shapes):
+        Us = ref["U"][l]
+        scale = max(np.abs(u).max() for u in Us)
+        near0 = np.any([np.abs(u) < 1e-3 * scale for u in Us], axis=0)
+        for k in range(Mw):
+            s_gpu = host(Ud[l * Mw + k])
+            dis = s_gpu != O.sign_extract(Us[k])
+            assert not np.any(dis & ~near0)
+        sure = ~near0
+        np.testing.assert_array_equal(host(Wd[l])[sure], ref["W"][l][sure])
 
 
 def test_ns_skip_flag_leaves_outputs_untouched():
