@@ -366,7 +366,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   int64_t lz_floats = 0;
   for (MatDesc& d : B->mats) {
     d.lz_off = lz_floats;
-    if (spectral) lz_floats += (int64_t)(kLanczosSteps + 2) * B->groups[d.group].m;
+    if (spectral) lz_floats += (int64_t)(kLanczosSteps + 2) * lz_stride(B->groups[d.group].m);
   }
 
   // tile tables: for the symmetric stages the tiles that reach the diagonal or
@@ -802,7 +802,9 @@ smuon_status prepare_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t*
   for (const MatDesc& d : B.mats) {
     const int m = B.groups[d.group].m;
     ex->lz_rows += m;
-    ex->lz_matvec_bytes += 4.0 * ((double)m * m + 2.0 * m);
+    const double a_bytes = (B.h.mode != MODE_SIMT_F32 && rq.c != 0.f && !(rq.flags & SMUON_NS_SPLIT_BF16))
+                               ? 2.0 : 4.0;  // bf16 operand copy or f32 A
+    ex->lz_matvec_bytes += a_bytes * m * m + 8.0 * m;
   }
   for (int k = 0; k < ST_COUNT; ++k) {
     ex->sflops[k] = stage_flops(B, k);
@@ -821,19 +823,19 @@ smuon_status run_lanczos(const NsExec& ex, const int32_t* skip, cudaStream_t s) 
     k_lz_start<<<mat_grid, 256, 0, s>>>(ex.d_plan, skip);
     CUDA_TRY(cudaGetLastError());
   }
-  const int row_grid = (int)std::max<int64_t>(1, std::min<int64_t>((ex.lz_rows + 7) / 8, (int64_t)sms * 8));
+  const int row_grid = (int)std::max<int64_t>(1, std::min<int64_t>((ex.lz_rows + 7) / 8, (int64_t)sms * 4));
   for (int j = 0; j < kLanczosSteps; ++j) {
     {
       Launch L("k_lz_matvec", SMUON_WORK_BYTES, ex.lz_matvec_bytes, s);
       k_lz_matvec<<<row_grid, 256, 0, s>>>(ex.d_plan, j, skip);
       CUDA_TRY(cudaGetLastError());
     }
-    Launch L("k_lz_step", SMUON_WORK_BYTES, 4.0 * ex.lz_rows * (j + 6), s);
+    Launch L("k_lz_step", SMUON_WORK_BYTES, 4.0 * ex.lz_rows * (4.0 * (j + 1) + 6.0), s);
     k_lz_step<<<mat_grid, 256, 0, s>>>(ex.d_plan, j, skip);
     CUDA_TRY(cudaGetLastError());
   }
   Launch L("k_lz_finish", SMUON_WORK_BYTES, 8.0 * kLanczosSteps * h.n_mats, s);
-  k_lz_finish<<<(h.n_mats + 127) / 128, 128, 0, s>>>(ex.d_plan, skip);
+  k_lz_finish<<<(h.n_mats * 32 + 255) / 256, 256, 0, s>>>(ex.d_plan, skip);  // one warp per matrix
   CUDA_TRY(cudaGetLastError());
   return SMUON_OK;
 }

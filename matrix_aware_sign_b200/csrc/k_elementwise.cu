@@ -350,13 +350,11 @@ __device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
   return (((~le & ~w) | ~nz) >> 15) & 0x00010001u;
 }
 
-// vote and update of 8 entries e0..e0+7 from their 4 packed count words
+// vote and update of 8 entries e0..e0+7 from their 4 packed count words, W
+// already loaded into w (when kHasW)
 template <bool kHasW>
-__device__ __forceinline__ void vote_finish8(const EwTable& tb, const EwLayer& L, int64_t e0, const uint32_t* cnt) {
-  // W is loaded only here, after the workers' loads: fewer live registers, so
-  // three CTAs fit per SM (more loads in flight hide more latency)
-  float w[8];
-  if (kHasW) load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+__device__ __forceinline__ void vote_apply8(const EwTable& tb, const EwLayer& L, int64_t e0, const uint32_t* cnt,
+                                            float* w) {
   int8_t v8[8];
   // eta * v for v = +1, -1 and the tie value: exact products, chosen per entry
   const float up = tb.eta, down = -tb.eta, tied = tb.eta * (float)tb.tie;
@@ -378,6 +376,15 @@ __device__ __forceinline__ void vote_finish8(const EwTable& tb, const EwLayer& L
       for (int k = 0; k < 8; ++k) dst[k] = v8[k];
     }
   }
+}
+
+template <bool kHasW>
+__device__ __forceinline__ void vote_finish8(const EwTable& tb, const EwLayer& L, int64_t e0, const uint32_t* cnt) {
+  // W is loaded only here, after the workers' loads: fewer live registers, so
+  // three CTAs fit per SM (more loads in flight hide more latency)
+  float w[8];
+  if (kHasW) load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+  vote_apply8<kHasW>(tb, L, e0, cnt, w);
 }
 
 // int8 (integer-sum) vote on bf16 outputs: the count of positive signs of each
@@ -465,6 +472,12 @@ __device__ __forceinline__ void vote_update_i8src(const EwTable& tb) {
     const int64_t e0 = (chunk - L.chunk_begin) * 8;
     if (!(active && e0 < L.n)) continue;
     if (L.vec && e0 + 16 <= L.n) {
+      // W first: the int8 signs need few registers, so W's loads go out together with the workers'
+      float w[16];
+      if (kHasW) {
+        load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
+        load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
+      }
       uint32_t b[4] = {0u, 0u, 0u, 0u};  // per byte: positive signs of entries e0 + 4i .. e0 + 4i + 3
       for (int wk0 = 0; wk0 < M; wk0 += 8) {
         uint4 u[8];
@@ -487,8 +500,8 @@ __device__ __forceinline__ void vote_update_i8src(const EwTable& tb) {
         cnt[2 * i] = __byte_perm(b[i], 0u, 0x4140);      // entries 4i, 4i + 1 in the low and high halves
         cnt[2 * i + 1] = __byte_perm(b[i], 0u, 0x4342);  // entries 4i + 2, 4i + 3
       }
-      vote_finish8<kHasW>(tb, L, e0, cnt);
-      vote_finish8<kHasW>(tb, L, e0 + 8, cnt + 4);
+      vote_apply8<kHasW>(tb, L, e0, cnt, w);
+      vote_apply8<kHasW>(tb, L, e0 + 8, cnt + 4, w + 8);
     } else {
       const int nent = (int)min((int64_t)16, L.n - e0);
       for (int k = 0; k < nent; ++k) {

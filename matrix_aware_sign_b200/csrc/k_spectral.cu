@@ -8,10 +8,15 @@
 // r = 1 / (sqrt(lambda_max) + eps s), so that X_0 = s r M = M / (||M||_2 + eps).
 //
 // Per Lanczos step j: w = A v_j (k_lz_matvec: one warp per row, all matrices),
-// then alpha_j = w.v_j, w -= alpha_j v_j + beta_{j-1} v_{j-1}, w is
-// orthogonalised against every earlier v, beta_j = ||w||, v_{j+1} = w / beta_j
-// (k_lz_step: one CTA per matrix). The largest eigenvalue of the tridiagonal
-// (alpha, beta) matrix is found by bisection on its Sturm counts (k_lz_finish).
+// then w is orthogonalised against v_0 .. v_j by classical Gram-Schmidt done
+// twice (all j + 1 coefficients of a pass in one block reduction); alpha_j is
+// the v_j coefficient of the two passes together, beta_j = ||w|| and
+// v_{j+1} = w / beta_j (k_lz_step: one CTA per matrix). In exact arithmetic the
+// coefficients of v_0 .. v_{j-2} vanish and that of v_{j-1} is beta_{j-1}, the
+// three-term recurrence; the full passes keep the basis orthogonal in float32.
+// The largest eigenvalue of the tridiagonal (alpha, beta) matrix is found by
+// bisection on its Sturm counts (k_lz_finish). Vectors are stored with a
+// stride of m rounded up to 4 floats, so rows of A and vectors load as float4.
 #include "kernels.cuh"
 
 namespace smuon {
@@ -20,7 +25,7 @@ namespace {
 
 __device__ __forceinline__ float* lz_vec(const PlanHeader& h, const MatDesc& md, int j) {
   const GroupDesc& g = h.groups[md.group];
-  return h.lz + md.lz_off + (int64_t)j * g.m;
+  return h.lz + md.lz_off + (int64_t)j * lz_stride(g.m);
 }
 
 // block-wide sum (256 threads); every thread gets the result
@@ -72,65 +77,134 @@ __global__ void __launch_bounds__(256) k_lz_start(const Plan* plan, const int32_
   }
 }
 
-// w = A v_j for every matrix: one warp per row of A (f32, in its group's buffer)
+// w = A v_j for every matrix: one warp per row of A, each warp over a
+// contiguous range of the flattened rows (one matrix lookup per range). A is
+// the f32 A_0, or in the plain BF16 modes with c != 0 the bf16 operand copy
+// of it: half the bytes, for a relative perturbation of lambda_max near
+// 2^-9 / sqrt(m), inside those modes' own rounding. The split mode keeps the
+// f32 A_0: its sign criterion is tight enough to notice that perturbation.
 __global__ void __launch_bounds__(256) k_lz_matvec(const Plan* plan, int j, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t total = h.lz_rows[h.n_mats];
-  for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < total; row += warps) {
-    const int i = lz_mat_of_row(h, row);
+  const int64_t per = (total + warps - 1) / warps;
+  int64_t row = warp * per;
+  const int64_t end = min(total, row + per);
+  if (row >= end) return;
+  const bool use_bf = h.mode != MODE_SIMT_F32 && h.c != 0.f && !(h.flags & SMUON_NS_SPLIT_BF16);
+  int i = lz_mat_of_row(h, row);
+  while (row < end) {
     const MatDesc& md = h.mats[i];
     const GroupDesc& g = h.groups[md.group];
-    const int r = (int)(row - h.lz_rows[i]);
-    const float* a = g.af + ((int64_t)md.z * g.m + r) * g.ldm;
-    const float* v = lz_vec(h, md, j);
-    float acc = 0.f;
-    for (int k = lane; k < g.m; k += 32) acc += a[k] * v[k];
+    const int m = g.m;
+    const int64_t ldm = g.ldm;
+    const int64_t r_first = h.lz_rows[i];
+    const int64_t r_stop = min(end, (int64_t)h.lz_rows[i + 1]);
+    const float* __restrict__ v = h.lz + md.lz_off + (int64_t)j * lz_stride(m);  // 16-byte aligned
+    float* __restrict__ w = h.lz + md.lz_off + (int64_t)(kLanczosSteps + 1) * lz_stride(m);
+    const float* af = g.af + (int64_t)md.z * m * ldm;
+    const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(g.aop) + (int64_t)md.z * m * ldm;
+    for (; row < r_stop; ++row) {
+      const int r = (int)(row - r_first);
+      float acc = 0.f;
+      if (use_bf) {  // rows 256-byte aligned (ldm % 128 == 0): 8 bf16 per 16-byte load
+        const uint4* a = reinterpret_cast<const uint4*>(ab + (int64_t)r * ldm);
+        const int m8 = m >> 3;
+        for (int k = lane; k < m8; k += 32) {
+          const uint4 q = a[k];
+          const float4 y0 = reinterpret_cast<const float4*>(v)[2 * k];
+          const float4 y1 = reinterpret_cast<const float4*>(v)[2 * k + 1];
+          acc += __uint_as_float(q.x << 16) * y0.x + __uint_as_float(q.x & 0xffff0000u) * y0.y +
+                 __uint_as_float(q.y << 16) * y0.z + __uint_as_float(q.y & 0xffff0000u) * y0.w +
+                 __uint_as_float(q.z << 16) * y1.x + __uint_as_float(q.z & 0xffff0000u) * y1.y +
+                 __uint_as_float(q.w << 16) * y1.z + __uint_as_float(q.w & 0xffff0000u) * y1.w;
+        }
+        for (int k = 8 * m8 + lane; k < m; k += 32) acc += __bfloat162float(ab[(int64_t)r * ldm + k]) * v[k];
+      } else {  // rows 512-byte aligned
+        const float* a = af + (int64_t)r * ldm;
+        const int m4 = m >> 2;
+        for (int k = lane; k < m4; k += 32) {
+          const float4 x = reinterpret_cast<const float4*>(a)[k];
+          const float4 y = reinterpret_cast<const float4*>(v)[k];
+          acc += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+        }
+        for (int k = 4 * m4 + lane; k < m; k += 32) acc += a[k] * v[k];
+      }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) lz_vec(h, md, kLanczosSteps + 1)[r] = acc;  // the work vector w
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) w[r] = acc;
+    }
+    ++i;
   }
 }
 
-// one Lanczos step per matrix (one CTA each)
+// one classical Gram-Schmidt pass of w against v_0 .. v_j: every coefficient
+// from one block reduction, then w -= sum_t c_t v_t; returns c_j
+__device__ __forceinline__ float cgs_pass(const float* __restrict__ V, int64_t st, int m, int j,
+                                          float* __restrict__ w, float (*red)[kLanczosSteps], float* coef) {
+  float c[kLanczosSteps];
+#pragma unroll
+  for (int t = 0; t < kLanczosSteps; ++t) c[t] = 0.f;
+  for (int k = threadIdx.x; k < m; k += blockDim.x) {
+    const float wk = w[k];
+#pragma unroll
+    for (int t = 0; t < kLanczosSteps; ++t)
+      if (t <= j) c[t] += wk * V[t * st + k];
+  }
+  const int wi = threadIdx.x >> 5, l = threadIdx.x & 31;
+#pragma unroll
+  for (int t = 0; t < kLanczosSteps; ++t) {
+    if (t > j) break;
+    float x = c[t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (l == 0) red[wi][t] = x;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x <= j) {
+    float x = 0.f;
+    for (int q = 0; q < (int)(blockDim.x >> 5); ++q) x += red[q][threadIdx.x];
+    coef[threadIdx.x] = x;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < m; k += blockDim.x) {
+    float wk = w[k];
+    for (int t = 0; t <= j; ++t) wk -= coef[t] * V[t * st + k];
+    w[k] = wk;
+  }
+  const float cj = coef[j];
+  __syncthreads();  // coef and red are reused by the next pass
+  return cj;
+}
+
+// one Lanczos step per matrix (one CTA of 256 threads each)
 __global__ void __launch_bounds__(256) k_lz_step(const Plan* plan, int j, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
-  __shared__ float red[8];
+  __shared__ float red[8][kLanczosSteps];
+  __shared__ float coef[kLanczosSteps];
+  __shared__ float red1[8];
   for (int i = blockIdx.x; i < h.n_mats; i += gridDim.x) {
     const MatDesc& md = h.mats[i];
     const int m = h.groups[md.group].m;
     float* ab = h.lz_ab + (int64_t)i * 2 * kLanczosSteps;  // alpha[0..K), beta[K..2K)
-    float* w = lz_vec(h, md, kLanczosSteps + 1);
-    const float* vj = lz_vec(h, md, j);
     if (j > 0 && ab[kLanczosSteps + j - 1] == 0.f) {  // an earlier step broke down: nothing to add
       if (threadIdx.x == 0) { ab[j] = 0.f; ab[kLanczosSteps + j] = 0.f; }
       continue;
     }
-    float p = 0.f;
-    for (int k = threadIdx.x; k < m; k += blockDim.x) p += w[k] * vj[k];
-    const float alpha = block_sum(p, red);
-    const float bprev = j > 0 ? ab[kLanczosSteps + j - 1] : 0.f;
-    const float* vp = j > 0 ? lz_vec(h, md, j - 1) : vj;
-    for (int k = threadIdx.x; k < m; k += blockDim.x) w[k] -= alpha * vj[k] + bprev * vp[k];
-    __syncthreads();
-    // full reorthogonalisation against v_0 .. v_j
-    for (int t = 0; t <= j; ++t) {
-      const float* vt = lz_vec(h, md, t);
-      float q = 0.f;
-      for (int k = threadIdx.x; k < m; k += blockDim.x) q += w[k] * vt[k];
-      const float c = block_sum(q, red);
-      for (int k = threadIdx.x; k < m; k += blockDim.x) w[k] -= c * vt[k];
-      __syncthreads();
-    }
+    const int64_t st = lz_stride(m);
+    float* V = h.lz + md.lz_off;  // v_0 .. v_K, then w
+    float* w = V + (int64_t)(kLanczosSteps + 1) * st;
+    const float alpha = cgs_pass(V, st, m, j, w, red, coef) + cgs_pass(V, st, m, j, w, red, coef);
     float ss = 0.f;
     for (int k = threadIdx.x; k < m; k += blockDim.x) ss += w[k] * w[k];
-    const float beta = sqrtf(block_sum(ss, red));
+    const float beta = sqrtf(block_sum(ss, red1));
     const bool ok = beta > 1e-6f * fabsf(alpha) && beta > 1e-30f && j + 1 < kLanczosSteps;
     if (ok) {
-      float* vn = lz_vec(h, md, j + 1);
+      float* vn = V + (int64_t)(j + 1) * st;
       const float inv = 1.f / beta;
       for (int k = threadIdx.x; k < m; k += blockDim.x) vn[k] = w[k] * inv;
     }
@@ -139,47 +213,71 @@ __global__ void __launch_bounds__(256) k_lz_step(const Plan* plan, int j, const 
   }
 }
 
-// Sturm count: eigenvalues of the k x k tridiagonal matrix below x
-__device__ __forceinline__ int sturm_below(const float* alpha, const float* beta, int k, double x) {
+// Sturm count: eigenvalues of the k x k tridiagonal matrix below x (float32:
+// the count is exact for a matrix within a few ulps of T, which bounds the
+// bisection's error near 1e-7 of ||T||)
+__device__ __forceinline__ int sturm_below(const float* alpha, const float* beta, int k, float x) {
   int count = 0;
-  double d = 1.0;
-  for (int i = 0; i < k; ++i) {
-    const double b2 = i > 0 ? (double)beta[i - 1] * beta[i - 1] : 0.0;
-    d = ((double)alpha[i] - x) - (i > 0 ? b2 / d : 0.0);
-    if (d == 0.0) d = -1e-300;
-    if (d < 0.0) ++count;
+  float d = 1.f;
+#pragma unroll
+  for (int i = 0; i < kLanczosSteps; ++i) {  // fully unrolled: alpha and beta stay in registers
+    if (i < k) {
+      const float b2 = i > 0 ? beta[i - 1] * beta[i - 1] : 0.f;
+      d = (alpha[i] - x) - (i > 0 ? __fdiv_rn(b2, d) : 0.f);
+      if (d == 0.f) d = -1e-30f;
+      if (d < 0.f) ++count;
+    }
   }
   return count;
 }
 
-// lambda_max of each matrix's tridiagonal matrix by bisection, then r = 1 / (sqrt(lambda) + eps s)
-__global__ void k_lz_finish(const Plan* plan, const int32_t* skip) {
+// lambda_max of each matrix's tridiagonal matrix, one warp per matrix: each
+// round the 32 lanes take Sturm counts at 32 interior points of [lo, hi] and
+// the interval shrinks to the gap where the count reaches k (33x per round);
+// then r = 1 / (sqrt(lambda) + eps s)
+__global__ void __launch_bounds__(256) k_lz_finish(const Plan* plan, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < h.n_mats; i += gridDim.x * blockDim.x) {
-    const float* alpha = h.lz_ab + (int64_t)i * 2 * kLanczosSteps;
-    const float* beta = alpha + kLanczosSteps;
-    int k = 1;  // the Krylov dimension actually built: steps up to the first breakdown
-    while (k < kLanczosSteps && beta[k - 1] != 0.f) ++k;
-    double lo = 0.0, hi = 0.0;
-    for (int t = 0; t < k; ++t) {
-      const double rad = (t > 0 ? fabs((double)beta[t - 1]) : 0.0) + (t + 1 < k ? fabs((double)beta[t]) : 0.0);
-      hi = fmax(hi, (double)alpha[t] + rad);
-      lo = fmin(lo, (double)alpha[t] - rad);
-    }
-    for (int it = 0; it < 100 && hi - lo > 1e-12 * fmax(1.0, fabs(hi)); ++it) {
-      const double mid = 0.5 * (lo + hi);
-      if (sturm_below(alpha, beta, k, mid) == k) hi = mid; else lo = mid;
-    }
-    const float lam = (float)hi;  // 0 for a zero matrix: then s r = 1/eps, as in the Frobenius case
-    const float s = h.scale[i];
-    float r = 1.f / (sqrtf(fmaxf(lam, 0.f)) + h.eps * s);
-    if (!isfinite(lam) || !isfinite(r)) {
-      r = 1.f;
-      if (h.status) atomicOr(h.status, SMUON_DEV_NONFINITE_NORM);
-    }
-    h.rscale[i] = r;
+  const int lane = threadIdx.x & 31;
+  const int i = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if (i >= h.n_mats) return;
+  const float* alpha = h.lz_ab + (int64_t)i * 2 * kLanczosSteps;
+  const float* beta = alpha + kLanczosSteps;
+  int k = 1;  // the Krylov dimension actually built: steps up to the first breakdown
+  while (k < kLanczosSteps && beta[k - 1] != 0.f) ++k;
+  float a[kLanczosSteps], b[kLanczosSteps];  // the tridiagonal matrix, in registers (uniform over the warp)
+  float lo = 0.f, hi = 0.f;  // Gershgorin bounds (lo <= 0: A_0 is positive semidefinite)
+#pragma unroll
+  for (int t = 0; t < kLanczosSteps; ++t) {
+    a[t] = t < k ? alpha[t] : 0.f;
+    b[t] = t + 1 < k ? beta[t] : 0.f;
   }
+  for (int t = 0; t < k; ++t) {
+    const float rad = (t > 0 ? fabsf(beta[t - 1]) : 0.f) + (t + 1 < k ? fabsf(beta[t]) : 0.f);
+    hi = fmaxf(hi, alpha[t] + rad);
+    lo = fminf(lo, alpha[t] - rad);
+  }
+  for (int round = 0; round < 8 && hi - lo > 2e-7f * fmaxf(fabsf(hi), 1e-30f); ++round) {
+    const float x = lo + (hi - lo) * (float)(lane + 1) * (1.f / 33.f);
+    const unsigned above = __ballot_sync(0xffffffffu, sturm_below(a, b, k, x) == k);
+    if (above) {  // lowest point with every eigenvalue below it
+      const int f = __ffs(above) - 1;
+      const float nhi = lo + (hi - lo) * (float)(f + 1) * (1.f / 33.f);
+      lo = f > 0 ? lo + (hi - lo) * (float)f * (1.f / 33.f) : lo;
+      hi = nhi;
+    } else {
+      lo = lo + (hi - lo) * (32.f / 33.f);
+    }
+  }
+  if (lane != 0) return;
+  const float lam = (float)hi;  // 0 for a zero matrix: then s r = 1/eps, as in the Frobenius case
+  const float s = h.scale[i];
+  float r = 1.f / (sqrtf(fmaxf(lam, 0.f)) + h.eps * s);
+  if (!isfinite(lam) || !isfinite(r)) {
+    r = 1.f;
+    if (h.status) atomicOr(h.status, SMUON_DEV_NONFINITE_NORM);
+  }
+  h.rscale[i] = r;
 }
 
 }  // namespace smuon
