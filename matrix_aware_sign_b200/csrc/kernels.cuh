@@ -71,7 +71,7 @@ __global__ void k_update_src(const __grid_constant__ EwTable tb);
 __global__ void k_harness_gaussian(const __grid_constant__ EwTable tb);
 
 // spectral scaling (k_spectral.cu)
-constexpr int kLanczosSteps = 24;
+constexpr int kLanczosSteps = 64;  // at most; a matrix stops once its largest Ritz value has converged
 __host__ __device__ constexpr int64_t lz_stride(int m) { return (m + 3) & ~3; }  // floats per Lanczos vector
 __global__ void k_lz_start(const Plan* plan, const int32_t* skip);
 __global__ void k_lz_matvec(const Plan* plan, int j, const int32_t* skip);

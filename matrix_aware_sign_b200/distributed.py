@@ -6,10 +6,14 @@ momentum (flow steps 1-2), turns the polar factor into signs, and the ranks
 exchange them in one of the two forms of flow step 3:
 
 * ``"allgather"``: 1 bit per parameter (the packed message of smuon_sign_pack,
-  entry i at bit i % 32 of word i / 32); every rank gathers all ranks'
-  messages and counts the set bits (sum = 2 * popcount - M, flow step 4);
+  entry i at bit i % 32 of word i / 32, packed from the int8 signs); every
+  rank gathers all ranks' messages and counts the set bits (sum =
+  2 * popcount - M, flow step 4);
 * ``"allreduce_int8"``: the +-1 signs as int8, summed by an all-reduce; the
   vote is the sign of the sum.
+
+On both paths the Newton-Schulz call writes the int8 signs itself (an int8
+output), so U never reaches memory.
 
 Every rank then applies the same vote to its replica of W (flow step 4), so
 the replicas stay identical. The exchange itself is torch.distributed (NCCL
@@ -62,13 +66,13 @@ class DistributedSignMuon:
         self.exchange, self.tie, self.flags, self.group = exchange, tie_value, ns_flags, group
         self.world = dist.get_world_size(group)
         dev = self.W[0].device
-        self.U = [torch.empty(w.shape, dtype=torch.bfloat16, device=dev) for w in self.W]
+        self.U = [torch.empty(w.shape, dtype=torch.int8, device=dev) for w in self.W]  # the signs themselves
         self.votes = [torch.empty(w.numel(), dtype=torch.int8, device=dev) for w in self.W]
         self.ws = workspace(smuon_ns_workspace_bytes(self.M, iters, ns_flags), dev)
         if exchange == "allgather":
             self.local = [torch.empty(packed_words(w.numel()), dtype=torch.int32, device=dev) for w in self.W]
         else:
-            self.local = [torch.empty((1, w.numel()), dtype=torch.int8, device=dev) for w in self.W]
+            self.local = [u.view(1, -1) for u in self.U]
 
     def step(self, G):
         # flow steps 1-2: momentum and polar factor of this worker
@@ -79,8 +83,7 @@ class DistributedSignMuon:
                 smuon_sign_pack([self.U[l]], packed=self.local[l].view(1, -1))
                 gathered = exchange_packed(self.local[l], self.group)
                 smuon_vote(self.world, n, self.votes[l], packed=gathered, tie_value=self.tie)
-            else:
-                smuon_sign_pack([self.U[l]], signs_i8=self.local[l])
+            else:  # the int8 signs came straight from the Newton-Schulz epilogue
                 total = exchange_signs_int8(self.local[l], self.group)
                 smuon_vote(1, n, self.votes[l], signs_i8=total, tie_value=self.tie)  # sign of the summed signs
         # flow step 4: the same update on every replica

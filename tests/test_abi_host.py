@@ -132,7 +132,7 @@ def test_gram_only_rejects_unsupported_requests(L):
 
 def test_spectral_flag_validation_and_workspace(L):
     """SMUON_NS_SPECTRAL excludes NO_NORMALIZE, EMIT_Q and GRAM_ONLY; its
-    workspace adds the Lanczos vectors (26 vectors of m floats per matrix, the
+    workspace adds the Lanczos vectors (66 vectors of m floats per matrix, the
     tridiagonal coefficients and the f32 Gram matrix even for c = 0)."""
     import torch
     import matrix_aware_sign_b200 as S
@@ -147,7 +147,7 @@ def test_spectral_flag_validation_and_workspace(L):
     for flags in (0, S.NS_SPLIT_BF16, S.NS_FP32_REF):
         base = S.smuon_ns_workspace_bytes(mats, 5, flags)
         spec = S.smuon_ns_workspace_bytes(mats, 5, flags | sp)
-        lz = 4 * 26 * (256 + 64 + 200) + 4 * 2 * 24 * 3
+        lz = 4 * 66 * (256 + 64 + 200) + 4 * 2 * 64 * 3  # at most 64 Lanczos steps: 65 vectors and w
         assert base + lz <= spec <= base + lz + 4 * 256 * 4, (base, spec)
 
 

@@ -114,7 +114,15 @@ def test_fused_vote_update_from_int8_signs(wdtype, kind, M, tie):
     votes = [torch.zeros(r * c, dtype=torch.int8, device="cuda") for r, c in shapes]
     eta = 0.02
     S.smuon_update(Wd, eta, U=Ud, M=M, tie_value=tie, vote_kind=kind, vote_out=votes)
+    # the same int8 signs through smuon_sign_pack: message bits and +-1 bytes
+    packed = torch.zeros((M, S.packed_words(64 * 147)), dtype=torch.int32, device="cuda")
+    signs = torch.zeros((M, 64 * 147), dtype=torch.int8, device="cuda")
+    S.smuon_sign_pack(Ud[0], packed=packed, signs_i8=signs)
     torch.cuda.synchronize()
+    for k in range(M):
+        s_ref = O.sign_extract(U[0][k].astype(np.float64)).reshape(-1)
+        np.testing.assert_array_equal(host(signs[k]), s_ref)
+        np.testing.assert_array_equal(packed[k].cpu().numpy().view(np.uint32), O.pack_bits(s_ref))
     for i, sh in enumerate(shapes):
         v = O.vote_from_signs([O.sign_extract(u.astype(np.float64)) for u in U[i]], tie)
         np.testing.assert_array_equal(host(votes[i]).reshape(sh), v)
@@ -277,6 +285,16 @@ def test_ns_spectral_scaling(shape, coeffs, iters, mode, tol):
     _, Ud = _ns_run([M], coeffs, iters, mode | S.NS_SPECTRAL)
     ref = O.newton_schulz(M, *coeffs, iters, spectral=True)
     check_ns_outputs([(host(Ud[0]), ref)], tol)
+
+
+@pytest.mark.parametrize("shape", [(512, 4608), (3072, 768)])
+def test_ns_spectral_scaling_slow_lanczos_convergence(shape):
+    """Gaussian matrices whose largest singular values lie close together: a
+    fixed 24-step Lanczos run left sigma_max 1.6e-3 low on these seeds; the
+    residual-stopped run meets the FP32 mode's 1e-4."""
+    M = np.random.default_rng(shape[0] + shape[1]).standard_normal(shape).astype(np.float32)
+    _, Ud = _ns_run([M], WL.QUINTIC, 1, S.NS_FP32_REF | S.NS_SPECTRAL)
+    check_ns_outputs([(host(Ud[0]), O.newton_schulz(M, *WL.QUINTIC, 1, spectral=True))], 1e-4)
 
 
 @pytest.mark.parametrize("mode", [0, S.NS_SIMT_BF16, S.NS_SPLIT_BF16, S.NS_FP32_REF])
