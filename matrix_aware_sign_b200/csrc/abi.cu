@@ -210,7 +210,7 @@ struct Layout {
   size_t off_groups = 0, off_mats = 0, off_tmaps = 0;
   size_t off_partials = 0, off_scale = 0, off_probe = 0, off_mom_begin = 0;
   size_t off_sched = 0, off_sched_begin = 0;
-  size_t off_lz_rows = 0, off_rscale = 0, off_lz = 0, off_lz_ab = 0;
+  size_t off_lz_rows = 0, off_rscale = 0, off_lz = 0, off_lz_ab = 0, off_lz_act = 0;
   int n_tmaps = 0;
 };
 
@@ -471,6 +471,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.off_rscale = B->take(sizeof(float) * B->mats.size());
   L.off_lz = spectral ? B->take(sizeof(float) * lz_floats) : 0;
   L.off_lz_ab = spectral ? B->take(sizeof(float) * 2 * kLanczosSteps * B->mats.size()) : 0;
+  L.off_lz_act = spectral ? B->take(sizeof(int32_t) * (2 * B->mats.size() + 2)) : 0;
 
   // per-group buffers
   for (auto& g : B->groups) {
@@ -529,6 +530,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   h.lz = spectral ? B->ptr_at<float>(L.off_lz) : nullptr;
   h.lz_ab = spectral ? B->ptr_at<float>(L.off_lz_ab) : nullptr;
   h.lz_rows = B->ptr_at<int32_t>(L.off_lz_rows);
+  h.lz_act = spectral ? B->ptr_at<int32_t>(L.off_lz_act) : nullptr;
   h.mom_begin = B->ptr_at<int32_t>(L.off_mom_begin);
   h.sched = B->ptr_at<int32_t>(L.off_sched);
   h.sched_begin = B->ptr_at<int32_t>(L.off_sched_begin);
@@ -825,8 +827,13 @@ smuon_status run_lanczos(const NsExec& ex, const int32_t* skip, cudaStream_t s) 
   }
   const int row_grid = (int)std::max<int64_t>(1, std::min<int64_t>((ex.lz_rows + 7) / 8, (int64_t)sms * 4));
   for (int j = 0; j < kLanczosSteps; ++j) {
-    {
-      Launch L("k_lz_matvec", SMUON_WORK_BYTES, ex.lz_matvec_bytes, s);
+    {  // the list of matrices still iterating (all of them before the first step)
+      Launch L("k_lz_compact", SMUON_WORK_BYTES, 12.0 * h.n_mats, s);
+      k_lz_compact<<<1, 1024, 0, s>>>(ex.d_plan, j - 1, skip);
+      CUDA_TRY(cudaGetLastError());
+    }
+    {  // only the first launch's bytes are known on the host (later ones skip stopped matrices)
+      Launch L("k_lz_matvec", SMUON_WORK_BYTES, j == 0 ? ex.lz_matvec_bytes : 0.0, s);
       k_lz_matvec<<<row_grid, 256, 0, s>>>(ex.d_plan, j, skip);
       CUDA_TRY(cudaGetLastError());
     }

@@ -90,19 +90,21 @@ __device__ __forceinline__ float tri_lambda_max(const float* a, const float* b, 
 }
 
 // |last component| of the unit eigenvector of (a, b) for its largest
-// eigenvalue theta, by the forward recurrence from y_0 = 1. theta lies above
-// every eigenvalue of the leading blocks (interlacing), so the components keep
-// one sign and do not cancel; a running rescale keeps them finite.
+// eigenvalue theta, by the recurrence of the rows run backward from
+// y_{k-1} = 1. The eigenvector of a converged Ritz value decays toward its
+// last index, so backward is the direction in which it grows: the stable one
+// (forward, the tiny last component would come out of a cancellation that
+// theta's own rounding swamps). A running rescale keeps the values finite.
 __device__ __forceinline__ float tri_last_component(const float* a, const float* b, int k, float theta) {
-  float yp = 0.f, y = 1.f, nrm = 1.f;
-  for (int i = 0; i + 1 < k; ++i) {
-    const float yn = ((theta - a[i]) * y - (i > 0 ? b[i - 1] * yp : 0.f)) / b[i];
-    yp = y;
-    y = yn;
-    nrm += yn * yn;
-    if (nrm > 1e30f) { y *= 1e-15f; yp *= 1e-15f; nrm *= 1e-30f; }
+  float y1 = 0.f, y = 1.f, last = 1.f, nrm = 1.f;  // y = y_i, y1 = y_{i+1}
+  for (int i = k - 1; i >= 1; --i) {
+    const float ym = ((theta - a[i]) * y - (i + 1 < k ? b[i] * y1 : 0.f)) / b[i - 1];
+    y1 = y;
+    y = ym;
+    nrm += ym * ym;
+    if (nrm > 1e30f) { y *= 1e-15f; y1 *= 1e-15f; last *= 1e-15f; nrm *= 1e-30f; }
   }
-  return fabsf(y) * rsqrtf(nrm);
+  return last * rsqrtf(nrm);
 }
 
 // matrix of a flattened Lanczos row (binary search over the compact row prefix)
@@ -149,27 +151,34 @@ __global__ void __launch_bounds__(256) k_lz_matvec(const Plan* plan, int j, cons
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
   const int lane = threadIdx.x & 31;
+  const int n_act = h.lz_act[0];
+  const int32_t* act_rows = h.lz_act + 1;              // [n_act + 1] prefix of the active matrices' rows
+  const int32_t* act_mat = h.lz_act + 2 + h.n_mats;    // [n_act] their indices
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t total = h.lz_rows[h.n_mats];
+  const int64_t total = n_act > 0 ? act_rows[n_act] : 0;
   const int64_t per = (total + warps - 1) / warps;
   int64_t row = warp * per;
   const int64_t end = min(total, row + per);
   if (row >= end) return;
   const bool use_bf = h.mode != MODE_SIMT_F32 && h.c != 0.f && !(h.flags & SMUON_NS_SPLIT_BF16);
-  int i = lz_mat_of_row(h, row);
+  int q;  // active entry holding `row`: the last with act_rows[q] <= row
+  {
+    int lo = 0, hi = n_act - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (act_rows[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    q = lo;
+  }
   while (row < end) {
+    const int i = act_mat[q];
     const MatDesc& md = h.mats[i];
     const GroupDesc& g = h.groups[md.group];
     const int m = g.m;
     const int64_t ldm = g.ldm;
-    const int64_t r_first = h.lz_rows[i];
-    const int64_t r_stop = min(end, (int64_t)h.lz_rows[i + 1]);
-    if (j > 0 && h.lz_ab[(int64_t)i * 2 * kLanczosSteps + kLanczosSteps + j - 1] == 0.f) {  // stopped
-      row = r_stop;
-      ++i;
-      continue;
-    }
+    const int64_t r_first = act_rows[q];
+    const int64_t r_stop = min(end, (int64_t)act_rows[q + 1]);
     const float* __restrict__ v = h.lz + md.lz_off + (int64_t)j * lz_stride(m);  // 16-byte aligned
     float* __restrict__ w = h.lz + md.lz_off + (int64_t)(kLanczosSteps + 1) * lz_stride(m);
     const float* af = g.af + (int64_t)md.z * m * ldm;
@@ -181,13 +190,13 @@ __global__ void __launch_bounds__(256) k_lz_matvec(const Plan* plan, int j, cons
         const uint4* a = reinterpret_cast<const uint4*>(ab + (int64_t)r * ldm);
         const int m8 = m >> 3;
         for (int k = lane; k < m8; k += 32) {
-          const uint4 q = a[k];
+          const uint4 x = a[k];
           const float4 y0 = reinterpret_cast<const float4*>(v)[2 * k];
           const float4 y1 = reinterpret_cast<const float4*>(v)[2 * k + 1];
-          acc += __uint_as_float(q.x << 16) * y0.x + __uint_as_float(q.x & 0xffff0000u) * y0.y +
-                 __uint_as_float(q.y << 16) * y0.z + __uint_as_float(q.y & 0xffff0000u) * y0.w +
-                 __uint_as_float(q.z << 16) * y1.x + __uint_as_float(q.z & 0xffff0000u) * y1.y +
-                 __uint_as_float(q.w << 16) * y1.z + __uint_as_float(q.w & 0xffff0000u) * y1.w;
+          acc += __uint_as_float(x.x << 16) * y0.x + __uint_as_float(x.x & 0xffff0000u) * y0.y +
+                 __uint_as_float(x.y << 16) * y0.z + __uint_as_float(x.y & 0xffff0000u) * y0.w +
+                 __uint_as_float(x.z << 16) * y1.x + __uint_as_float(x.z & 0xffff0000u) * y1.y +
+                 __uint_as_float(x.w << 16) * y1.z + __uint_as_float(x.w & 0xffff0000u) * y1.w;
         }
         for (int k = 8 * m8 + lane; k < m; k += 32) acc += __bfloat162float(ab[(int64_t)r * ldm + k]) * v[k];
       } else {  // rows 512-byte aligned
@@ -204,7 +213,62 @@ __global__ void __launch_bounds__(256) k_lz_matvec(const Plan* plan, int j, cons
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) w[r] = acc;
     }
-    ++i;
+    ++q;
+  }
+}
+
+// the matrices still iterating after step j (all of them for j < 0: before
+// the first step): a matrix continues while its last beta is nonzero. One CTA
+// of 1024 threads scans the batch (up to 4096 matrices, four per thread).
+__global__ void __launch_bounds__(1024) k_lz_compact(const Plan* plan, int j, const int32_t* skip) {
+  if (skip && *skip) return;
+  const PlanHeader& h = plan->h;
+  const int n = h.n_mats;
+  const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int first = (int)threadIdx.x * per;
+  int cnt = 0, rows = 0;
+  for (int i = first; i < min(n, first + per); ++i) {
+    const bool act = j < 0 || h.lz_ab[(int64_t)i * 2 * kLanczosSteps + kLanczosSteps + j] != 0.f;
+    if (act) { ++cnt; rows += h.lz_rows[i + 1] - h.lz_rows[i]; }
+  }
+  // block-wide exclusive scan of (cnt, rows)
+  __shared__ int s_cnt[32], s_rows[32];
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  int ic = cnt, ir = rows;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int c = __shfl_up_sync(0xffffffffu, ic, o), r = __shfl_up_sync(0xffffffffu, ir, o);
+    if (lane >= o) { ic += c; ir += r; }
+  }
+  if (lane == 31) { s_cnt[wi] = ic; s_rows[wi] = ir; }
+  __syncthreads();
+  if (wi == 0) {
+    int c = lane < (int)(blockDim.x >> 5) ? s_cnt[lane] : 0, r = lane < (int)(blockDim.x >> 5) ? s_rows[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int c2 = __shfl_up_sync(0xffffffffu, c, o), r2 = __shfl_up_sync(0xffffffffu, r, o);
+      if (lane >= o) { c += c2; r += r2; }
+    }
+    s_cnt[lane] = c;  // inclusive over warps
+    s_rows[lane] = r;
+  }
+  __syncthreads();
+  int pc = ic - cnt + (wi > 0 ? s_cnt[wi - 1] : 0);    // exclusive prefix of this thread
+  int pr = ir - rows + (wi > 0 ? s_rows[wi - 1] : 0);
+  int32_t* act_rows = h.lz_act + 1;
+  int32_t* act_mat = h.lz_act + 2 + n;
+  for (int i = first; i < min(n, first + per); ++i) {
+    const bool act = j < 0 || h.lz_ab[(int64_t)i * 2 * kLanczosSteps + kLanczosSteps + j] != 0.f;
+    if (act) {
+      act_mat[pc] = i;
+      act_rows[pc] = pr;
+      ++pc;
+      pr += h.lz_rows[i + 1] - h.lz_rows[i];
+    }
+  }
+  if (threadIdx.x == blockDim.x - 1) {  // the last thread ends with the totals
+    h.lz_act[0] = pc;
+    act_rows[pc] = pr;
   }
 }
 

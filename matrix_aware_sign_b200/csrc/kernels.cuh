@@ -77,6 +77,7 @@ __global__ void k_lz_start(const Plan* plan, const int32_t* skip);
 __global__ void k_lz_matvec(const Plan* plan, int j, const int32_t* skip);
 __global__ void k_lz_step(const Plan* plan, int j, const int32_t* skip);
 __global__ void k_lz_finish(const Plan* plan, const int32_t* skip);
+__global__ void k_lz_compact(const Plan* plan, int j, const int32_t* skip);
 __global__ void k_lion_sign(const __grid_constant__ EwTable tb);
 __global__ void k_lion_mean(const __grid_constant__ EwTable tb);
 __global__ void k_probe_finalize(const Plan* plan);

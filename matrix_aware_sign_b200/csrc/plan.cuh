@@ -122,6 +122,7 @@ struct PlanHeader {
   float* lz;                        // Lanczos vectors of every matrix (kLanczosSteps + 2 vectors of m each)
   float* lz_ab;                     // [n_mats][2 kLanczosSteps] Lanczos alpha, beta
   const int32_t* lz_rows;           // [n_mats + 1] first row of each matrix in the flattened row range
+  int32_t* lz_act;                  // matrices still iterating: [count][rows prefix, n_mats + 1][matrix, n_mats]
   GroupDesc* groups;        // device pointers into the plan region
   MatDesc* mats;
   CUtensorMap* tmaps;
