@@ -22,7 +22,7 @@ Sources (page title, section):
         schedule, shared double-EMA momentum, special cases; section "Problem"
         for the two update kinds.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   R1  Sign-Muon momentum is heavy-ball M <- beta*M + G from zero, no Nesterov.
   R2  Newton-Schulz step X <- aX + b(XX^T)X + c(XX^T)^2 X with the coefficients
       given per workload (cubic (1.5,-0.5,0), quintic (3.4445,-4.7750,2.0315)).
