@@ -7,7 +7,8 @@
 // the batch at once; the first step's epilogues then rescale by
 // r = 1 / (sqrt(lambda_max) + eps s), so that X_0 = s r M = M / (||M||_2 + eps).
 //
-// Per Lanczos step j: w = A v_j (k_lz_matvec: one warp per row, all matrices),
+// Per Lanczos step j: k_lz_compact lists the matrices still iterating, and
+// w = A v_j for them (k_lz_matvec: one warp per row, their rows spread evenly),
 // then w is orthogonalised against v_0 .. v_j by classical Gram-Schmidt done
 // twice (one warp per basis vector for the coefficients); alpha_j is the v_j
 // coefficient of the two passes together, beta_j = ||w|| and
@@ -105,16 +106,6 @@ __device__ __forceinline__ float tri_last_component(const float* a, const float*
     if (nrm > 1e30f) { y *= 1e-15f; y1 *= 1e-15f; last *= 1e-15f; nrm *= 1e-30f; }
   }
   return last * rsqrtf(nrm);
-}
-
-// matrix of a flattened Lanczos row (binary search over the compact row prefix)
-__device__ __forceinline__ int lz_mat_of_row(const PlanHeader& h, int64_t row) {
-  int lo = 0, hi = h.n_mats - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (h.lz_rows[mid] <= row) lo = mid; else hi = mid - 1;
-  }
-  return lo;
 }
 
 }  // namespace
