@@ -471,7 +471,8 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.off_rscale = B->take(sizeof(float) * B->mats.size());
   L.off_lz = spectral ? B->take(sizeof(float) * lz_floats) : 0;
   L.off_lz_ab = spectral ? B->take(sizeof(float) * 2 * kLanczosSteps * B->mats.size()) : 0;
-  L.off_lz_act = spectral ? B->take(sizeof(int32_t) * (2 * B->mats.size() + 2)) : 0;
+  // the active list ([count][rows prefix][matrices]) and the step launches' ticket
+  L.off_lz_act = spectral ? B->take(sizeof(int32_t) * (2 * B->mats.size() + 3)) : 0;
 
   // per-group buffers
   for (auto& g : B->groups) {
@@ -826,12 +827,12 @@ smuon_status run_lanczos(const NsExec& ex, const int32_t* skip, cudaStream_t s) 
     CUDA_TRY(cudaGetLastError());
   }
   const int row_grid = (int)std::max<int64_t>(1, std::min<int64_t>((ex.lz_rows + 7) / 8, (int64_t)sms * 4));
+  {  // every matrix iterates at first; each step's last block then writes the next list
+    Launch L("k_lz_compact", SMUON_WORK_BYTES, 12.0 * h.n_mats, s);
+    k_lz_compact<<<1, 1024, 0, s>>>(ex.d_plan, -1, skip);
+    CUDA_TRY(cudaGetLastError());
+  }
   for (int j = 0; j < kLanczosSteps; ++j) {
-    {  // the list of matrices still iterating (all of them before the first step)
-      Launch L("k_lz_compact", SMUON_WORK_BYTES, 12.0 * h.n_mats, s);
-      k_lz_compact<<<1, 1024, 0, s>>>(ex.d_plan, j - 1, skip);
-      CUDA_TRY(cudaGetLastError());
-    }
     {  // only the first launch's bytes are known on the host (later ones skip stopped matrices)
       Launch L("k_lz_matvec", SMUON_WORK_BYTES, j == 0 ? ex.lz_matvec_bytes : 0.0, s);
       k_lz_matvec<<<row_grid, 256, 0, s>>>(ex.d_plan, j, skip);

@@ -7,8 +7,9 @@
 // the batch at once; the first step's epilogues then rescale by
 // r = 1 / (sqrt(lambda_max) + eps s), so that X_0 = s r M = M / (||M||_2 + eps).
 //
-// Per Lanczos step j: k_lz_compact lists the matrices still iterating, and
-// w = A v_j for them (k_lz_matvec: one warp per row, their rows spread evenly),
+// Per Lanczos step j: w = A v_j for the matrices still iterating
+// (k_lz_matvec: one warp per row, their rows spread evenly; the list comes
+// from the previous step's last block, or k_lz_compact before the first),
 // then w is orthogonalised against v_0 .. v_j by classical Gram-Schmidt done
 // twice (one warp per basis vector for the coefficients); alpha_j is the v_j
 // coefficient of the two passes together, beta_j = ||w|| and
@@ -209,22 +210,23 @@ __global__ void __launch_bounds__(256) k_lz_matvec(const Plan* plan, int j, cons
 }
 
 // the matrices still iterating after step j (all of them for j < 0: before
-// the first step): a matrix continues while its last beta is nonzero. One CTA
-// of 1024 threads scans the batch (up to 4096 matrices, four per thread).
-__global__ void __launch_bounds__(1024) k_lz_compact(const Plan* plan, int j, const int32_t* skip) {
-  if (skip && *skip) return;
-  const PlanHeader& h = plan->h;
+// the first step), written into h.lz_act by the calling block (a multiple of
+// 32 threads, up to 1024; up to 4096 matrices): a matrix continues while its
+// last beta is nonzero. The betas come from other blocks of the same launch
+// when the last block of k_lz_step calls this, so they are read past L1.
+__device__ void lz_compact_block(const PlanHeader& h, int j) {
   const int n = h.n_mats;
   const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
   const int first = (int)threadIdx.x * per;
+  auto active = [&](int i) {
+    return j < 0 || __ldcg(h.lz_ab + (int64_t)i * 2 * kLanczosSteps + kLanczosSteps + j) != 0.f;
+  };
   int cnt = 0, rows = 0;
-  for (int i = first; i < min(n, first + per); ++i) {
-    const bool act = j < 0 || h.lz_ab[(int64_t)i * 2 * kLanczosSteps + kLanczosSteps + j] != 0.f;
-    if (act) { ++cnt; rows += h.lz_rows[i + 1] - h.lz_rows[i]; }
-  }
+  for (int i = first; i < min(n, first + per); ++i)
+    if (active(i)) { ++cnt; rows += h.lz_rows[i + 1] - h.lz_rows[i]; }
   // block-wide exclusive scan of (cnt, rows)
   __shared__ int s_cnt[32], s_rows[32];
-  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
   int ic = cnt, ir = rows;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(1024) k_lz_compact(const Plan* plan, int j, co
   if (lane == 31) { s_cnt[wi] = ic; s_rows[wi] = ir; }
   __syncthreads();
   if (wi == 0) {
-    int c = lane < (int)(blockDim.x >> 5) ? s_cnt[lane] : 0, r = lane < (int)(blockDim.x >> 5) ? s_rows[lane] : 0;
+    int c = lane < nw ? s_cnt[lane] : 0, r = lane < nw ? s_rows[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int c2 = __shfl_up_sync(0xffffffffu, c, o), r2 = __shfl_up_sync(0xffffffffu, r, o);
@@ -244,23 +246,31 @@ __global__ void __launch_bounds__(1024) k_lz_compact(const Plan* plan, int j, co
     s_rows[lane] = r;
   }
   __syncthreads();
-  int pc = ic - cnt + (wi > 0 ? s_cnt[wi - 1] : 0);    // exclusive prefix of this thread
+  int pc = ic - cnt + (wi > 0 ? s_cnt[wi - 1] : 0);  // exclusive prefix of this thread
   int pr = ir - rows + (wi > 0 ? s_rows[wi - 1] : 0);
   int32_t* act_rows = h.lz_act + 1;
   int32_t* act_mat = h.lz_act + 2 + n;
-  for (int i = first; i < min(n, first + per); ++i) {
-    const bool act = j < 0 || h.lz_ab[(int64_t)i * 2 * kLanczosSteps + kLanczosSteps + j] != 0.f;
-    if (act) {
+  for (int i = first; i < min(n, first + per); ++i)
+    if (active(i)) {
       act_mat[pc] = i;
       act_rows[pc] = pr;
       ++pc;
       pr += h.lz_rows[i + 1] - h.lz_rows[i];
     }
-  }
   if (threadIdx.x == blockDim.x - 1) {  // the last thread ends with the totals
     h.lz_act[0] = pc;
     act_rows[pc] = pr;
   }
+  __syncthreads();
+}
+
+// the first active list (every matrix) and a zero ticket for the step launches;
+// later lists come from the last block of each k_lz_step launch
+__global__ void __launch_bounds__(1024) k_lz_compact(const Plan* plan, int j, const int32_t* skip) {
+  if (skip && *skip) return;
+  const PlanHeader& h = plan->h;
+  lz_compact_block(h, j);
+  if (threadIdx.x == 0) h.lz_act[2 * h.n_mats + 2] = 0;
 }
 
 // one classical Gram-Schmidt pass of w against v_0 .. v_j: the coefficients
@@ -339,6 +349,19 @@ __global__ void __launch_bounds__(256) k_lz_step(const Plan* plan, int j, const 
     }
     if (threadIdx.x == 0) { ab[j] = alpha; ab[kLanczosSteps + j] = ok ? beta : 0.f; }
     __syncthreads();
+  }
+  // the last block to finish lists the matrices still iterating for the next A v launch (no block waits:
+  // the ticket only tells the last one that every other block's betas are written and fenced)
+  __shared__ int s_last;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(h.lz_act + 2 * h.n_mats + 2, 1) == (int)gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    lz_compact_block(h, j);
+    if (threadIdx.x == 0) h.lz_act[2 * h.n_mats + 2] = 0;  // ready for the next step's launch
   }
 }
 
