@@ -132,9 +132,10 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
 #define SMUON_NS_SIMT_BF16    16u  /* diagnostic: BF16 operands on CUDA cores instead of tcgen05 */
 #define SMUON_NS_SPECTRAL     64u  /* normalise by the spectral norm instead: X_0 = M / (||M||_2 + eps)
                                       (SignMuon summary, section 4: either norm will do); ||M||_2 from a
-                                      24-step Lanczos estimate of the largest eigenvalue of the first Gram
-                                      matrix, per matrix, on the device. Not with SMUON_NS_NO_NORMALIZE,
-                                      SMUON_NS_EMIT_Q or SMUON_NS_GRAM_ONLY */
+                                      Lanczos estimate of the largest eigenvalue of the first Gram matrix,
+                                      per matrix, on the device: at most 64 steps, each matrix stopped once
+                                      the residual of its largest Ritz pair is below 1e-4 of it. Not with
+                                      SMUON_NS_NO_NORMALIZE, SMUON_NS_EMIT_Q or SMUON_NS_GRAM_ONLY */
 #define SMUON_NS_GRAM_ONLY    32u  /* CacheMuon fresh solve iterated on the m x m Gram ("Gram
                                       Newton-Schulz", CacheMuon summary, method item 1): A_0 = X_0 X_0^T once,
                                       then per step P_k = aI + bA_k + cA_k^2, Q_{k+1} = P_k Q_k and
