@@ -420,3 +420,25 @@ def test_ns_spectral_scaling_closed_form(shape, coeffs, iters):
     # a rank-one matrix: spectral and Frobenius norms agree
     r1 = np.outer(rng.standard_normal(shape[0]), rng.standard_normal(shape[1]))
     assert _rel(O.newton_schulz(r1, *coeffs, iters, spectral=True), O.newton_schulz(r1, *coeffs, iters)) < 1e-12
+
+
+def test_sign_muon_step_spectral_passes_the_scaling_through():
+    """sign_muon_step(spectral=True) orthogonalises every worker's momentum
+    with the spectral scaling: with one quintic step its U is the singular-
+    value closed form p(s_i / s_max), a different matrix from the Frobenius
+    step's, and the vote and update follow from those signs."""
+    rng = np.random.default_rng(31)
+    shape, M = (6, 9), 3
+    W = [np.zeros(shape)]
+    Ms = [[np.zeros(shape) for _ in range(M)]]
+    G = [[rng.standard_normal(shape) for _ in range(M)]]
+    out = O.sign_muon_step(W, Ms, G, 0.9, WL.QUINTIC, 1, 0.01, "f32", spectral=True)
+    plain = O.sign_muon_step(W, Ms, G, 0.9, WL.QUINTIC, 1, 0.01, "f32")
+    for k in range(M):
+        Uk, S, Vt = np.linalg.svd(G[0][k], full_matrices=False)
+        expect = (Uk * _poly(S / (S.max() + 1e-7), WL.QUINTIC, 1)) @ Vt
+        assert _rel(out["U"][0][k], expect) < 1e-10
+        assert _rel(out["U"][0][k], plain["U"][0][k]) > 1e-3
+    v = O.vote_from_packed([O.pack_bits(O.sign_extract(u)) for u in out["U"][0]], M, 54).reshape(shape)
+    np.testing.assert_array_equal(out["vote"][0], v)
+    np.testing.assert_array_equal(out["W"][0], O.update_with_vote(W[0], v, 0.01, "f32"))
