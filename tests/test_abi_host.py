@@ -161,3 +161,21 @@ def test_int8_sign_sources_reject_packed_message(L):
     packed = (ctypes.c_void_p * 1)(16384)
     assert L.smuon_update(W, 1, U, None, None, 2, 0.01, 0, S.VOTE_INT8, packed, None, None) == -4
     assert b"packed_out needs F32 or BF16 U" in L.smuon_last_error()
+
+
+def test_size_limits_are_checked_on_the_host(L):
+    """Each side in 1..65536 and at most 4096 matrices per call: the limits
+    are rejected (or, at the limit, sized) before anything is enqueued."""
+    import ctypes
+    import matrix_aware_sign_b200 as S
+    out = ctypes.c_size_t(0)
+    edge = (S.SmuonMat * 1)(S.SmuonMat(4096, 1, 65536, 65536, S.F32))
+    assert L.smuon_ns_workspace_bytes(edge, 1, 1, 0, ctypes.byref(out)) == 0 and out.value > 0
+    for rows, cols in [(1, 65537), (65537, 1), (0, 8), (8, 0)]:
+        big = (S.SmuonMat * 1)(S.SmuonMat(4096, rows, cols, max(cols, 1), S.F32))
+        assert L.smuon_ns(big, big, 1, None, 0.9, 1.5, -0.5, 0.0, 1, 1e-7, 0, None, None, None, 0, None,
+                          None) == -2, (rows, cols)
+    many = (S.SmuonMat * 4097)(*[S.SmuonMat(4096, 8, 8, 8, S.F32)] * 4097)
+    assert L.smuon_ns(many, many, 4097, None, 0.9, 1.5, -0.5, 0.0, 1, 1e-7, 0, None, None, None, 0, None,
+                      None) == -1
+    assert b"n_mats" in L.smuon_last_error()
