@@ -333,25 +333,84 @@ def test_lionmuon_p1_is_pure_muon():
         np.testing.assert_array_equal(a, b)
 
 
+def test_lion_interpolate_and_ema_golden():
+    """Hand-derived float32 cases of the interpolation G_hat = beta1 M + (1-beta1) G
+    and of the EMA update (same arithmetic with beta2), bit for bit, including
+    two ties to even and the coefficient taken from f32(beta)."""
+    g = _golden("lion_f32.json")
+    for case in g["cases"]:
+        M = np.array([case["M"]], np.float32)
+        G = np.array([case["G"]], np.float32)
+        want = int(case["expect_bits"], 16)
+        for fn in (O.lion_interpolate, O.lion_ema):
+            got = fn(M, G, case["beta"])
+            assert got.dtype == np.float32
+            assert int(got.view(np.uint32)[0]) == want, (fn.__name__, case)
+
+
+def _bf16_torch(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).float().numpy()
+
+
 def test_lionmuon_pinf_equal_betas_is_signum():
-    """P = infinity with beta1 = beta2: pure sign steps on the EMA itself, i.e.
-    Signum with a majority vote (LionMuon summary, special cases)."""
+    """P = infinity with beta1 = beta2 and the EMA from zero: every step is a sign
+    step on the EMA itself, i.e. Signum with a majority vote (LionMuon summary,
+    special cases). The reference loop is written here with numpy float32
+    arithmetic, a direct count of the positive signs and torch's bf16
+    conversion, calling nothing of the oracle."""
     W, Gs = _lion_inputs(seed=22)
-    beta = 0.9
-    M = [[np.zeros(w.shape, np.float32) for _ in range(3)] for w in W]
+    beta, eta, workers = 0.9, 1e-3, 3
+    M = [[np.zeros(w.shape, np.float32) for _ in range(workers)] for w in W]
     Ws = [w.copy() for w in W]
     Ms = [[m.copy() for m in ms] for ms in M]
+    b32 = np.float32(beta)
+    c32 = np.float32(np.float32(1.0) - b32)
     for t in range(1, 6):
-        _, W, M = O.lionmuon_step(t, W, M, Gs[t - 1], 0, beta, beta, 1e-3, WL.QUINTIC, 2, "bf16")
+        kind, W, M = O.lionmuon_step(t, W, M, Gs[t - 1], 0, beta, beta, eta, WL.QUINTIC, 2, "bf16")
+        assert kind == "sign"
         for i in range(len(Ws)):
-            Ms[i] = [O.lion_ema(Ms[i][m], Gs[t - 1][i][m], beta) for m in range(3)]
-            v = O.vote_from_signs([np.where(Ms[i][m] >= 0, 1, -1) for m in range(3)])
-            Ws[i] = O.update_with_vote(Ws[i], v, 1e-3, "bf16")
+            new = []
+            for m in range(workers):
+                prod_m = np.multiply(b32, Ms[i][m], dtype=np.float32)
+                prod_g = np.multiply(c32, Gs[t - 1][i][m], dtype=np.float32)
+                new.append(np.add(prod_m, prod_g, dtype=np.float32))
+            Ms[i] = new
+            positives = sum((x >= 0).astype(np.int64) for x in new)
+            v = np.where(2 * positives > workers, 1.0, -1.0).astype(np.float32)  # odd count: no ties
+            Ws[i] = _bf16_torch(np.subtract(Ws[i], np.float32(eta) * v, dtype=np.float32))
     for a, b in zip(W, Ws):
         np.testing.assert_array_equal(a, b)
     for a, b in zip(M, Ms):
         for x, y in zip(a, b):
             np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("workers", [1, 2, 3, 4])
+@pytest.mark.parametrize("shape", [(6, 10), (10, 6)])
+def test_sign_muon_local_polar_identical_workers(workers, shape):
+    """The local polar step (SignMuon summary, algorithm flow step 5) with M
+    identical workers: the vote is the workers' common sign matrix S itself
+    (no ties: the sum is M S), and the direction is the Newton-Schulz map of S,
+    written here by its singular-value closed form; with W = 0 the update is
+    -f32(f32(eta) D) exactly."""
+    rng = np.random.default_rng(40 + workers)
+    G = rng.standard_normal(shape)
+    W = [np.zeros(shape, np.float32)]
+    Ms = [[np.zeros(shape) for _ in range(workers)]]
+    Gs = [[G.copy() for _ in range(workers)]]
+    eta, iters = 0.02, 3
+    out = O.sign_muon_step(W, Ms, Gs, 0.9, WL.QUINTIC, iters, eta, "f32", local_polar=True)
+    # every worker orthogonalised the same momentum G: its sign matrix by the closed form
+    Ug, Sg, Vgt = np.linalg.svd(G, full_matrices=False)
+    Ug_ns = (Ug * _poly(Sg / (np.sqrt(np.sum(Sg ** 2)) + 1e-7), WL.QUINTIC, iters)) @ Vgt
+    S = np.where(Ug_ns >= 0, 1.0, -1.0)
+    np.testing.assert_array_equal(out["vote"][0], S.astype(np.int8))
+    Us, Ss, Vst = np.linalg.svd(S, full_matrices=False)
+    D = (Us * _poly(Ss / (np.sqrt(np.sum(Ss ** 2)) + 1e-7), WL.QUINTIC, iters)) @ Vst
+    expect = -(np.float32(eta) * D.astype(np.float32)).astype(np.float32)
+    np.testing.assert_allclose(out["W"][0], expect, rtol=3e-7, atol=0)
+    # the dense step moves W by eta * D, not by eta * vote: they differ
+    assert np.abs(out["W"][0] + np.float32(eta) * S.astype(np.float32)).max() > 1e-4
 
 
 def test_ns_flops_counts():
