@@ -49,6 +49,12 @@ typedef int32_t smuon_status;
 #define SMUON_F32  0
 #define SMUON_BF16 1
 #define SMUON_I8   2
+#define SMUON_BITS 3  /* the 1-bit message of a sign matrix (SignMuon summary, flow step 3, all-gather
+                         variant; communication efficiency: one bit per parameter): data holds uint32
+                         words, entry i of the row-major flattening (i = row*cols + col) at bit i % 32
+                         of word i / 32, ceil(rows*cols / 128) * 4 words (a 16-byte multiple) with the
+                         bits past the last entry zero; ld must equal cols and data be 16-byte aligned.
+                         A set bit is the sign +1 (u >= 0), a clear bit -1 */
 
 /* bits OR-ed into *d_status by device code */
 #define SMUON_DEV_NONFINITE_NORM 1  /* a Frobenius norm (or a spectral-norm estimate) was NaN or Inf */
@@ -106,7 +112,11 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
  *                 or I8: then only the entrywise sign of U is written, +1 for
  *                 u >= 0 (-0 included) and -1 otherwise (NaN included), taken on
  *                 the float32 value in the last step's epilogue (SignMuon
- *                 summary, flow step 2: the sign matrix without U in memory).
+ *                 summary, flow step 2: the sign matrix without U in memory),
+ *                 or BITS: the same signs as the worker's 1-bit message (flow
+ *                 step 3, all-gather variant), written by that epilogue, pad
+ *                 words zeroed by the call; needs cols % 32 == 0 and the
+ *                 tensor-core modes, not with SMUON_NS_EMIT_Q.
  *  G[n_mats]      nullable gradients (F32 or BF16), same shapes.
  *  beta           momentum coefficient (ignored when G == NULL).
  *  a, b, c        Newton-Schulz coefficients; c == 0 skips the A^2 product.
@@ -136,6 +146,23 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
                                       per matrix, on the device: at most 64 steps, each matrix stopped once
                                       the residual of its largest Ritz pair is below 1e-4 of it. Not with
                                       SMUON_NS_NO_NORMALIZE, SMUON_NS_EMIT_Q or SMUON_NS_GRAM_ONLY */
+#define SMUON_NS_PLAIN_LEAD(k) ((uint32_t)(k) << 12)  /* with SMUON_NS_SPLIT_BF16: the first k (0..7)
+                                      Newton-Schulz steps take plain BF16 operands (one MMA per product, the
+                                      lo parts still written for the later steps). While the normalised
+                                      singular values are small, the B X term of a step is small beside the
+                                      float32 a X term, so its operand rounding barely reaches the output;
+                                      from s_max(X_0) ~ 0.06 (Gaussian momenta of the workload shapes) two
+                                      plain steps keep five quintic steps within the split mode's accuracy.
+                                      A matrix with one dominant singular value has s_max near 1 from the
+                                      start: leave k = 0 there. Not with SMUON_NS_SPECTRAL (s_max = 1),
+                                      SMUON_NS_EMIT_Q or SMUON_NS_GRAM_ONLY */
+#define SMUON_NS_PLAIN_LEAD_MASK (7u << 12)
+#define SMUON_NS_TEST_WAIT_EXPIRY 0x8000u  /* failure-detection test, not for use: every tensor-core stage's
+                                      copy producers issue nothing and its pipeline waits are limited to
+                                      65536 SM clocks (about 2 s otherwise), so each stage's first waits run
+                                      out; the CTAs then record SMUON_DEV_WAIT_TIMEOUT in d_status, wait (with
+                                      the full budget) for anything they issued, free their tensor memory and
+                                      return. U is not written */
 #define SMUON_NS_GRAM_ONLY    32u  /* CacheMuon fresh solve iterated on the m x m Gram ("Gram
                                       Newton-Schulz", CacheMuon summary, method item 1): A_0 = X_0 X_0^T once,
                                       then per step P_k = aI + bA_k + cA_k^2, Q_{k+1} = P_k Q_k and
@@ -170,6 +197,9 @@ smuon_status smuon_ns(const smuon_mat* M_in, const smuon_mat* U_out, int32_t n_m
  *  - It calls no cudaMalloc, cudaFree or other allocating routine.
  *  - The first call on a device looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
+ *    The address is kept per device and context: a call from a new context
+ *    (after cudaDeviceReset, for instance) looks it up again, so make the
+ *    first call after such a reset outside stream capture too.
  *  - All calls share the one array and it keeps the last call's contents
  *    (nothing in it needs to start at zero: every call rewrites what it
  *    reads). Calls that may overlap on the GPU (other streams, other host
@@ -211,9 +241,13 @@ smuon_status smuon_sign_pack(const smuon_mat* U, int32_t M, uint32_t* packed, in
  * Ties (even M) give tie_value.
  *
  *  packed      [M][words] as written by smuon_sign_pack, or NULL
- *  signs_i8    [M][N] int8, or NULL (exactly one of the two)
+ *  signs_i8    [M][N] int8, or NULL (exactly one of the two). The vote is the
+ *              sign of the integer sum of the M rows, so a row may also hold a
+ *              partial sum of several workers' signs (e.g. the result of an
+ *              int8 SUM all-reduce, with M = 1); the per-entry total must stay
+ *              within -127..127.
  *  vote        device [N] int8 in {-1, 0, +1}
- * M in 1..64 (1..127 for int8 inputs is not needed: M <= 64 everywhere).
+ * M in 1..64.
  * ---------------------------------------------------------------------- */
 smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t M, int64_t N,
                         int8_t tie_value, int8_t* vote, void* stream);
@@ -229,7 +263,9 @@ smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t 
  * Exactly one source per call:
  *  U[n_layers*M]     (worker-minor) -> fused sign / vote / update in one pass;
  *                    F32, BF16, or I8 sign matrices (entry >= 0 counts as +1;
- *                    I8 takes no packed_out: pack with smuon_sign_pack);
+ *                    I8 takes no packed_out: pack with smuon_sign_pack), or
+ *                    BITS messages (a set bit counts as +1; the vote reads
+ *                    M/8 bytes per entry; no packed_out: they are the message);
  *                    vote_kind SMUON_VOTE_POPCOUNT (bit masks + popcount) or
  *                    SMUON_VOTE_INT8 (integer sum); both give the same vote.
  *                    Optional outputs: packed_out[l] ([M][words] message, the

@@ -19,10 +19,18 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsmuon.so")
 
-F32, BF16, I8 = 0, 1, 2
+F32, BF16, I8, BITS = 0, 1, 2, 3
 NS_FP32_REF, NS_SPLIT_BF16, NS_NO_NORMALIZE, NS_EMIT_Q, NS_SIMT_BF16 = 1, 2, 4, 8, 16
 NS_GRAM_ONLY = 32  # CacheMuon fresh solve iterated on the m x m Gram (with NS_EMIT_Q, one matrix)
 NS_SPECTRAL = 64  # spectral-norm normalisation X_0 = M / (||M||_2 + eps) (Lanczos estimate on the device)
+NS_TEST_WAIT_EXPIRY = 0x8000  # failure-detection test: the tensor-core stages' pipeline waits run out
+
+
+def ns_plain_lead(k: int) -> int:
+    """SMUON_NS_PLAIN_LEAD(k): with NS_SPLIT_BF16, the first k Newton-Schulz steps use plain BF16 operands."""
+    if not 0 <= k <= 7:
+        raise ValueError("k must be in 0..7")
+    return k << 12
 VOTE_POPCOUNT, VOTE_INT8 = 0, 1
 LION_MUON_VOTE = 0x100  # lionmuon_step ns_flags: Muon steps as Sign-Muon steps (per-worker NS + vote)
 DEV_NONFINITE_NORM, DEV_WAIT_TIMEOUT = 1, 2
@@ -122,8 +130,33 @@ def _check(code: int) -> None:
 _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.int8: I8}
 
 
-def mat(t: torch.Tensor) -> SmuonMat:
-    """Describes a 2-D row-major tensor (unit column stride)."""
+class Bits:
+    """The 1-bit message of a rows x cols sign matrix (SMUON_BITS): `words` is a
+    contiguous int32 tensor of packed_words(rows * cols) words, entry i of the
+    row-major flattening at bit i % 32 of word i // 32."""
+
+    def __init__(self, words: torch.Tensor, rows: int, cols: int):
+        if words.dtype != torch.int32 or not words.is_contiguous() or words.numel() < packed_words(rows * cols):
+            raise ValueError("words must be a contiguous int32 tensor of packed_words(rows * cols) words")
+        self.words, self.rows, self.cols = words, int(rows), int(cols)
+
+    @property
+    def shape(self):
+        return (self.rows, self.cols)
+
+    @property
+    def device(self):
+        return self.words.device
+
+    @staticmethod
+    def empty(rows: int, cols: int, device=None) -> "Bits":
+        return Bits(torch.zeros(packed_words(rows * cols), dtype=torch.int32, device=device or "cuda"), rows, cols)
+
+
+def mat(t) -> SmuonMat:
+    """Describes a 2-D row-major tensor (unit column stride), or a Bits message."""
+    if isinstance(t, Bits):
+        return SmuonMat(t.words.data_ptr(), t.rows, t.cols, t.cols, BITS)
     if t.dim() != 2 or (t.stride(1) != 1 and t.shape[1] > 1):
         raise ValueError("matrices must be 2-D with unit column stride")
     if t.dtype not in _DT:
@@ -322,11 +355,19 @@ class CacheMuon:
         self.fresh = NsPlan([M_t], [D_out], *coeffs, iters, flags=flags | NS_EMIT_Q, Q_out=[self.Q], eps=eps)
         self.steps = 0
 
-    def step(self, stream=None):
+    def probe(self, stream=None):
+        """The step's probe: D_hat = Q X_t into D, its residual and the accept flag (no cache on the first step)."""
         cachemuon_reuse_probe(self.Q if self.steps > 0 else None, self.M, self.D, self.gamma, self.err, self.accept,
                               self.cnt, eps=self.eps, ws=self.ws_probe, stream=stream)
+
+    def refresh(self, stream=None):
+        """The step's fresh solve (D and Q), whose kernels return at once when the probe accepted."""
         self.fresh.run(skip_if=self.accept, stream=stream)
         self.steps += 1
+
+    def step(self, stream=None):
+        self.probe(stream)
+        self.refresh(stream)
 
     def counters(self) -> dict:
         h, mi, pr, _ = self.cnt.tolist()

@@ -175,14 +175,20 @@ smuon_status encode_f32_3d(CUtensorMap* out, const void* ptr, int64_t inner, int
 int dtype_size(int32_t dt) { return dt == SMUON_F32 ? 4 : dt == SMUON_BF16 ? 2 : dt == SMUON_I8 ? 1 : 0; }
 
 smuon_status check_mat(const smuon_mat& m, const char* what, int i, bool allow_f32, bool allow_bf16,
-                       bool allow_i8) {
+                       bool allow_i8, bool allow_bits = false) {
   if (!m.data) return fail(SMUON_ERR_INVALID_ARG, "%s[%d].data is NULL", what, i);
   if (m.rows < 1 || m.cols < 1 || m.rows > 65536 || m.cols > 65536)
     return fail(SMUON_ERR_SHAPE, "%s[%d] has shape %dx%d (each side must be in 1..65536)", what, i, m.rows, m.cols);
   if (m.ld < m.cols) return fail(SMUON_ERR_SHAPE, "%s[%d].ld=%lld < cols=%d", what, i, (long long)m.ld, m.cols);
   const bool ok = (m.dtype == SMUON_F32 && allow_f32) || (m.dtype == SMUON_BF16 && allow_bf16) ||
-                  (m.dtype == SMUON_I8 && allow_i8);
+                  (m.dtype == SMUON_I8 && allow_i8) || (m.dtype == SMUON_BITS && allow_bits);
   if (!ok) return fail(SMUON_ERR_DTYPE, "%s[%d] has an unsupported dtype %d", what, i, m.dtype);
+  if (m.dtype == SMUON_BITS) {  // a packed message: flat words, no row stride
+    if (m.ld != m.cols) return fail(SMUON_ERR_SHAPE, "%s[%d] is a 1-bit message: ld must equal cols", what, i);
+    if (reinterpret_cast<uintptr_t>(m.data) % 16 != 0)
+      return fail(SMUON_ERR_INVALID_ARG, "%s[%d] is a 1-bit message: data must be 16-byte aligned", what, i);
+    return SMUON_OK;
+  }
   if (reinterpret_cast<uintptr_t>(m.data) % dtype_size(m.dtype) != 0)
     return fail(SMUON_ERR_INVALID_ARG, "%s[%d].data is not aligned to its element size", what, i);
   return SMUON_OK;
@@ -519,6 +525,10 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   h.flags = rq.flags;
   h.a = rq.a; h.b = rq.b; h.c = rq.c; h.eps = rq.eps; h.beta = rq.beta; h.gamma = rq.gamma;
   h.total_mom_tiles = mom_tiles;
+  // pipeline waits of the tensor-core stages: about 2 s of SM clock, or (failure-detection test) a
+  // budget that runs out while the producer issues nothing
+  h.wait_cycles = (rq.flags & SMUON_NS_TEST_WAIT_EXPIRY) ? (1ull << 16) : (1ull << 32);
+  h.starve_tc = (rq.flags & SMUON_NS_TEST_WAIT_EXPIRY) ? 1 : 0;
   h.tile_bm = BM; h.tile_bn = tc ? tc_tile_n(ST_AXPY, rq.flags) : kSimtBN;
   for (int st = 0; st < ST_COUNT; ++st) {
     h.total_tiles[st] = totals[st];
@@ -706,7 +716,8 @@ smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int it
        "k_gemm_tc_split.qx"}};
   if (h.mode == MODE_TC_BF16) {
     const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
-    Launch L(tc_names[split][st], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
+    const bool lead = split && plain_lead_stage(h.flags, st, iter);  // hi parts only: one product in three
+    Launch L(tc_names[split][st], SMUON_WORK_FLOPS, lead ? issued_flops / 3 : issued_flops, s, stage_flops);
     CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
   } else {
     const int grid = std::min(total, di.sms * 6);
@@ -725,7 +736,7 @@ smuon_status validate_ns(const NsRequest& rq) {
   if (rq.iters < 1 || rq.iters > 64) return fail(SMUON_ERR_INVALID_ARG, "iters=%d must be in 1..64", rq.iters);
   const uint32_t known =
       SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_SIMT_BF16 |
-      SMUON_NS_GRAM_ONLY | SMUON_NS_SPECTRAL;
+      SMUON_NS_GRAM_ONLY | SMUON_NS_SPECTRAL | SMUON_NS_PLAIN_LEAD_MASK | SMUON_NS_TEST_WAIT_EXPIRY;
   if (rq.flags & ~known) return fail(SMUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", rq.flags & ~known);
   const uint32_t modes = rq.flags & (SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_SIMT_BF16);
   if (modes & (modes - 1))
@@ -743,12 +754,28 @@ smuon_status validate_ns(const NsRequest& rq) {
   if ((rq.flags & SMUON_NS_SPECTRAL) && (rq.flags & (SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_GRAM_ONLY)))
     return fail(SMUON_ERR_UNSUPPORTED,
                 "SMUON_NS_SPECTRAL excludes SMUON_NS_NO_NORMALIZE, SMUON_NS_EMIT_Q and SMUON_NS_GRAM_ONLY");
+  if (rq.flags & SMUON_NS_PLAIN_LEAD_MASK) {
+    if (!(rq.flags & SMUON_NS_SPLIT_BF16))
+      return fail(SMUON_ERR_INVALID_ARG, "SMUON_NS_PLAIN_LEAD needs SMUON_NS_SPLIT_BF16");
+    if (rq.flags & (SMUON_NS_SPECTRAL | SMUON_NS_EMIT_Q | SMUON_NS_GRAM_ONLY))
+      return fail(SMUON_ERR_UNSUPPORTED,
+                  "SMUON_NS_PLAIN_LEAD excludes SMUON_NS_SPECTRAL, SMUON_NS_EMIT_Q and SMUON_NS_GRAM_ONLY");
+  }
   for (int i = 0; i < rq.n_mats; ++i) {
     smuon_status st;
     const bool has_g = rq.G != nullptr;
     if ((st = check_mat(rq.M_in[i], "M_in", i, true, !has_g, !has_g)) != SMUON_OK) return st;
-    if ((st = check_mat(rq.U_out[i], "U_out", i, true, true, true)) != SMUON_OK) return st;
+    if ((st = check_mat(rq.U_out[i], "U_out", i, true, true, true, true)) != SMUON_OK) return st;
     if (!same_shape(rq.M_in[i], rq.U_out[i])) return fail(SMUON_ERR_SHAPE, "U_out[%d] shape differs from M_in", i);
+    if (rq.U_out[i].dtype == SMUON_BITS) {
+      if (rq.flags & (SMUON_NS_FP32_REF | SMUON_NS_SIMT_BF16))
+        return fail(SMUON_ERR_UNSUPPORTED, "1-bit outputs need the tensor-core modes");
+      if (rq.flags & (SMUON_NS_EMIT_Q | SMUON_NS_GRAM_ONLY))
+        return fail(SMUON_ERR_UNSUPPORTED, "1-bit outputs are not written with SMUON_NS_EMIT_Q");
+      if (rq.U_out[i].cols % 32 != 0)
+        return fail(SMUON_ERR_SHAPE, "U_out[%d]: a 1-bit output needs cols %% 32 == 0 (cols=%d)", i,
+                    rq.U_out[i].cols);
+    }
     if (has_g) {
       if ((st = check_mat(rq.G[i], "G", i, true, true, false)) != SMUON_OK) return st;
       if (!same_shape(rq.M_in[i], rq.G[i])) return fail(SMUON_ERR_SHAPE, "G[%d] shape differs from M_in", i);
@@ -1122,14 +1149,17 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
     if (U) {
       for (int k = 0; k < M; ++k) {
         const smuon_mat& u = U[(int64_t)l * M + k];
-        if ((st = check_mat(u, "U", l * M + k, true, true, true)) != SMUON_OK) return st;
+        if ((st = check_mat(u, "U", l * M + k, true, true, true, true)) != SMUON_OK) return st;
         if (!same_shape(u, shape)) return fail(SMUON_ERR_SHAPE, "U[%d] shape differs from W[%d]", l * M + k, l);
         if (src_dtype >= 0 && u.dtype != src_dtype) return fail(SMUON_ERR_DTYPE, "all U must share one dtype");
         src_dtype = u.dtype;
-        if (!vec_ok(u.data, u.ld, u.cols, 1)) L.vec = 0;
+        // a 1-bit message is read word by word (16-byte aligned, checked above); W decides the fast path
+        if (u.dtype != SMUON_BITS && !vec_ok(u.data, u.ld, u.cols, 1)) L.vec = 0;
         srcs.push_back(EwSrc{u.data, u.ld});
       }
       if (packed_out && packed_out[l]) {
+        if (src_dtype == SMUON_BITS)
+          return fail(SMUON_ERR_INVALID_ARG, "packed_out with 1-bit message sources: they are the message");
         if (src_dtype == SMUON_I8)
           return fail(SMUON_ERR_UNSUPPORTED, "packed_out needs F32 or BF16 U (pack I8 signs with smuon_sign_pack)");
         if (reinterpret_cast<uintptr_t>(packed_out[l]) % 16)
@@ -1164,7 +1194,8 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
     double bytes = 0;
     for (int l = 0; l < tb.n_layers; ++l) {
       const EwLayer& Ly = tb.layers[l];
-      bytes += (double)Ly.n * (tb.M * dtype_size(src_dtype) + (Ly.w ? 2 * dtype_size(Ly.w_dtype) : 0));
+      const double src_bytes = src_dtype == SMUON_BITS ? tb.M / 8.0 : (double)tb.M * dtype_size(src_dtype);
+      bytes += (double)Ly.n * (src_bytes + (Ly.w ? 2 * dtype_size(Ly.w_dtype) : 0));
       if (Ly.packed_out) bytes += (double)Ly.n * tb.M / 8.0;
       if (Ly.vote_out) bytes += (double)Ly.n;
     }
@@ -1179,7 +1210,8 @@ smuon_status run_update(const UpdExec& ex, cudaStream_t s) {
     const EwTable& tb = ex.tables[i];
     const int grid = ew_grid(tb.total_chunks, ex.di);
     if (ex.source == 0) {
-      Launch L(ex.vote_kind == SMUON_VOTE_POPCOUNT ? "k_vote_update_popcount" : "k_vote_update_int8",
+      Launch L(tb.src_dtype == SMUON_BITS ? "k_vote_update_bits"
+               : ex.vote_kind == SMUON_VOTE_POPCOUNT ? "k_vote_update_popcount" : "k_vote_update_int8",
                SMUON_WORK_BYTES, ex.bytes[i], s);
       CUDA_TRY(launch_vote_update(tb, ex.vote_kind == SMUON_VOTE_POPCOUNT, grid, ex.di.sms, s));
     } else {
@@ -1550,20 +1582,43 @@ static __device__ __align__(256) unsigned char g_ns_static_scratch[SMUON_NS_STAT
 namespace {
 std::mutex g_static_mu;
 void* g_static_ptr[256] = {nullptr};
+CUcontext g_static_ctx[256] = {nullptr};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// the calling thread's current context (the device's primary context for runtime API callers)
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn) fn(&c);
+  return c;
+}
 
 // host code must not hand the symbol itself to a kernel: it is a host-side
-// stand-in, so the device address is looked up once per device
+// stand-in, so the device address is looked up once per device and context
+// (a context created anew, e.g. after cudaDeviceReset, may load the module at
+// another address, so a changed context handle looks it up again)
 smuon_status static_scratch(void** out) {
   int dev = 0;
   CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 256) return fail(SMUON_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  const CUcontext ctx = current_context();  // null before the runtime has made one current on this thread
   std::lock_guard<std::mutex> lk(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  if (!g_static_ptr[dev] || !ctx || g_static_ctx[dev] != ctx) {
     void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_ns_static_scratch);
+    cudaError_t e = cudaGetSymbolAddress(&p, g_ns_static_scratch);  // initialises the context if needed
     if (e != cudaSuccess || !p)
       return fail(SMUON_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
     g_static_ptr[dev] = p;
+    g_static_ctx[dev] = current_context();
   }
   *out = g_static_ptr[dev];
   return SMUON_OK;

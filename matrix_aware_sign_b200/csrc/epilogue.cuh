@@ -172,10 +172,48 @@ __device__ __forceinline__ void ld_user(const void* p, int64_t ld, int32_t dtype
   }
 }
 
+// 1-bit message of a wide-form row chunk (SMUON_BITS output): bit i % 32 of word i / 32 is set iff the
+// entry at flat user index i = user_row * cols + user_col is >= 0. cols (= ld) is a multiple of 32.
+//  - wide matrix: the lane's NV entries are consecutive user columns of one user row, starting at a
+//    multiple of NV: one 32-bit word (NV = 32) or one 16-bit half of a word (NV = 16) per lane.
+//  - tall matrix: the wide row is the user column, and the lanes of the warp hold 32 consecutive user
+//    columns (row & 31 is the lane) of the same user rows col0 + k: one ballot per k gives the word
+//    of user row col0 + k, stored by lane k. Rows and chunk bounds are warp-uniform here because the
+//    user's cols (the wide rows) are a multiple of 32, so every lane reaches the ballots.
+template <int NV>
+__device__ __forceinline__ void st_bits(void* p, int64_t ld, int tall, int row, int col0, int nvalid,
+                                        const float* v) {
+  if constexpr (NV % 16 == 0) {
+    if (!tall) {
+      uint32_t bits = 0;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) bits |= (uint32_t)(v[k] >= 0.f) << k;
+      const int64_t e = (int64_t)row * ld + col0;  // a multiple of NV
+      if (NV == 32) reinterpret_cast<uint32_t*>(p)[e >> 5] = bits;
+      else reinterpret_cast<uint16_t*>(p)[e >> 4] = (uint16_t)bits;
+    } else {
+      const int lane = threadIdx.x & 31;
+      const int64_t row_base = row & ~31;
+      uint32_t mine = 0;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        if (k >= nvalid) break;  // warp-uniform
+        const uint32_t b = __ballot_sync(0xffffffffu, v[k] >= 0.f);
+        if (lane == k) mine = b;
+      }
+      if (lane < nvalid) reinterpret_cast<uint32_t*>(p)[((int64_t)(col0 + lane) * ld + row_base) >> 5] = mine;
+    }
+  }
+}
+
 // user-orientation store of a wide-form row chunk (row i, cols j0..j0+NV-1)
 template <int NV>
 __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int tall, int vec, int row,
                                         int col0, int nvalid, const float* v) {
+  if (dtype == SMUON_BITS) {
+    st_bits<NV>(p, ld, tall, row, col0, nvalid, v);
+    return;
+  }
   if (!tall) {
     const int64_t base = (int64_t)row * ld + col0;
     if (vec && nvalid == NV) {

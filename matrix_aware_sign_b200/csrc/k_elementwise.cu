@@ -192,6 +192,11 @@ __global__ void k_norm_finalize(const Plan* plan, const int32_t* skip) {
     if (!isfinite(acc) && h.status) atomicOr(h.status, SMUON_DEV_NONFINITE_NORM);
     h.scale[mi] = s;
   }
+  if (md.u_dtype == SMUON_BITS) {  // the message's pad words (past the last entry's word) are zero
+    const int64_t n = (int64_t)md.rows * md.cols;  // a multiple of 32
+    const int64_t used = n >> 5, total = ((n + 127) >> 7) << 2;
+    if (used + lane < total) reinterpret_cast<uint32_t*>(md.u_ptr)[used + lane] = 0u;
+  }
 }
 
 // --------------------------------------------------------------------------
@@ -694,6 +699,107 @@ __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
   }
 }
 
+// Vote and update from the workers' 1-bit messages (SignMuon summary, flow steps 3-4, all-gather
+// variant): the message words of a Newton-Schulz call with a BITS output or of an all-gather. One
+// lane per packed word, i.e. 32 consecutive entries: the M words (M/8 bytes per entry) are added
+// bit-sliced -- plane p holds bit p of every entry's count of set bits -- by a ripple of half adders
+// per worker, and the counts are compared with h = floor(M/2) plane by plane from the top:
+// count > h is the +1 vote (2*count > M), count == h with M even the tie, the rest -1. Bits past a
+// layer's last entry are zero and are never applied. Layer chunk ranges are multiples of 16 chunks
+// (4 words), so global word g is chunk 4g.
+template <bool kHasW>
+__device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int M = tb.M;
+  const int h = M >> 1;
+  const uint32_t even = (M & 1) ? 0u : 0xffffffffu;
+  const int64_t total_words = tb.total_chunks >> 2;
+  for (int64_t wbase = warp_global * 32; wbase < total_words; wbase += warps_total * 32) {
+    const int64_t gw = wbase + lane;
+    const bool active = gw < total_words;
+    const int li = warp_layer(tb, 4 * wbase, active ? 4 * gw : tb.total_chunks - 1, lane);
+    const EwLayer& L = tb.layers[li];
+    const int64_t w = gw - (L.chunk_begin >> 2);
+    const int64_t e0 = 32 * w;
+    if (!(active && e0 < L.n)) continue;
+    uint32_t c[7] = {0u, 0u, 0u, 0u, 0u, 0u, 0u};  // counts up to 64 need 7 planes
+    for (int wk0 = 0; wk0 < M; wk0 += 8) {
+      uint32_t x[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        x[j] = (wk0 + j < M) ? reinterpret_cast<const uint32_t*>(tb.srcs[L.src_first + wk0 + j].ptr)[w] : 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t carry = x[j];
+#pragma unroll
+        for (int p = 0; p < 7; ++p) {
+          const uint32_t t = c[p] & carry;
+          c[p] ^= carry;
+          carry = t;
+        }
+      }
+    }
+    uint32_t gt = 0u, eq = 0xffffffffu;
+#pragma unroll
+    for (int p = 6; p >= 0; --p) {
+      if ((h >> p) & 1) {
+        eq &= c[p];
+      } else {
+        gt |= eq & c[p];
+        eq &= ~c[p];
+      }
+    }
+    const uint32_t pos = gt, tie = eq & even;
+    const float up = tb.eta, down = -tb.eta, tied = tb.eta * (float)tb.tie;
+    const int nent = (int)min((int64_t)32, L.n - e0);
+    if (L.vec && nent == 32) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float wv[8];
+        int8_t v8[8];
+        if (kHasW) load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int j = 8 * g + k;
+          const bool p1 = (pos >> j) & 1u, t1 = (tie >> j) & 1u;
+          v8[k] = (int8_t)(p1 ? 1 : (t1 ? tb.tie : -1));
+          wv[k] = __fsub_rn(wv[k], p1 ? up : (t1 ? tied : down));
+        }
+        if (kHasW) store8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
+        if (L.vote_out) {
+          int8_t* dst = L.vote_out + e0 + 8 * g;
+          if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
+            uint2 pk;
+            memcpy(&pk, v8, 8);
+            *reinterpret_cast<uint2*>(dst) = pk;
+          } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) dst[k] = v8[k];
+          }
+        }
+      }
+    } else {  // ragged last word or strided W: entry by entry
+      for (int j = 0; j < nent; ++j) {
+        const int64_t e = e0 + j;
+        const bool p1 = (pos >> j) & 1u, t1 = (tie >> j) & 1u;
+        const int8_t v = (int8_t)(p1 ? 1 : (t1 ? tb.tie : -1));
+        if (kHasW) {
+          const int64_t wi = ew_index(L, e, L.w_ld);
+          store_from_f32(L.w, wi, L.w_dtype, __fsub_rn(load_as_f32(L.w, wi, L.w_dtype), tb.eta * (float)v));
+        }
+        if (L.vote_out) L.vote_out[e] = v;
+      }
+    }
+  }
+}
+
+template <bool kHasW>
+__global__ void __launch_bounds__(256, 4) k_vote_update_bits(const __grid_constant__ EwTable tb) {
+  vote_update_bits<kHasW>(tb);
+}
+
 template <bool kPopcount, bool kBf16, typename MaskT>
 __global__ void __launch_bounds__(256) k_vote_update(const __grid_constant__ EwTable tb) {
   vote_update_body<kPopcount, kBf16, MaskT>(tb);
@@ -720,6 +826,13 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
   const int64_t want16 = (tb.total_chunks + 511) / 512;
   const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
   const bool has_w = tb.layers[0].w != nullptr;  // all layers or none (signs and votes only)
+  if (tb.src_dtype == SMUON_BITS) {  // one lane per packed word, four resident CTAs per SM, one wave
+    const int64_t want = (tb.total_chunks / 4 + 255) / 256;
+    const int gridb = (int)std::max<int64_t>(1, std::min<int64_t>(want, 4 * sms));
+    if (has_w) k_vote_update_bits<true><<<gridb, 256, 0, s>>>(tb);
+    else k_vote_update_bits<false><<<gridb, 256, 0, s>>>(tb);
+    return cudaGetLastError();
+  }
   if (tb.src_dtype == SMUON_I8) {  // sign matrices: both vote kinds count the same positives
     if (has_w) k_vote_update_i8src<true><<<grid16, 256, 0, s>>>(tb);
     else k_vote_update_i8src<false><<<grid16, 256, 0, s>>>(tb);
@@ -813,15 +926,16 @@ __global__ void __launch_bounds__(256) k_vote(const uint32_t* packed, const int8
         out[j] = threshold(2 * __popcll(mask) - M, tie);
       }
     } else {
+      int sum[32];  // rows may be partial sums (an all-reduced message): add in int
 #pragma unroll
-      for (int j = 0; j < 32; ++j) out[j] = 0;
+      for (int j = 0; j < 32; ++j) sum[j] = 0;
       for (int k = 0; k < M; ++k) {
         const int8_t* src = signs + (int64_t)k * N + e0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) if (j < nvalid) out[j] += src[j];
+        for (int j = 0; j < 32; ++j) if (j < nvalid) sum[j] += src[j];
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) out[j] = threshold(out[j], tie);
+      for (int j = 0; j < 32; ++j) out[j] = threshold(sum[j], tie);
     }
     if (nvalid == 32 && ((reinterpret_cast<uintptr_t>(vote + e0) & 15) == 0)) {
       uint4 a, b;

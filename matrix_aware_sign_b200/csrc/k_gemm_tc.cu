@@ -49,7 +49,7 @@ struct Cfg {
   static constexpr int SRC_RING = kSrc ? SRC_SLOTS * SRC_BYTES : 0;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SRC_RING + 1024 /*align*/ + 256 /*barriers*/;
 };
-constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz
+constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz: the exit drains' budget
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -72,15 +72,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// bounded wait: false when the budget ran out or another role aborted
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// bounded wait: false when the budget (SM clocks) ran out or another role aborted
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long budget) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) return false;
+      if (clock64() - t0 > budget) return false;
     }
   }
 }
@@ -250,6 +251,11 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // split mode: both parts of every operand, except in the plain leading steps (hi parts only); the
+  // producer and the MMA issuer take the same decision from the plan
+  const unsigned long long budget = h.wait_cycles;
+  const bool use_lo = kSplit && !plain_lead_stage(h.flags, stage, iter);
+  const int parts = use_lo ? PARTS : 1;
   // this CTA's tiles (host-balanced list; every role walks the same one)
   const int32_t* tiles = h.sched + h.sched_off[stage];
   const int t_begin = h.sched_begin[h.sched_boff[stage] + blockIdx.x];
@@ -261,7 +267,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
     uint32_t ph = 0;
     uint32_t armed = 0, last_par = 0;  // per-stage bit sets for the exit drain
     bool ok = true;
-    for (int i = t_begin; i < t_end && ok; ++i) {
+    for (int i = t_begin; i < t_end && ok && !h.starve_tc; ++i) {
       const int tile = tiles[i];
       int tm, tn;
       const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
@@ -271,14 +277,13 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         tensormap_acquire(o.mb);
         const int nk = (o.K + BK - 1) / BK;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(empty_bar + 8 * s, ph ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(empty_bar + 8 * s, ph ^ 1u, abort_flag, budget)) { ok = false; break; }
           const uint32_t fb = full_bar + 8 * s;
-          mbar_expect_tx(fb, STAGE_BYTES);
+          mbar_expect_tx(fb, parts * (A_BYTES + B_BYTES));
           armed |= 1u << s;
           last_par = (last_par & ~(1u << s)) | (ph << s);
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + PARTS * A_BYTES;
-#pragma unroll
-          for (int part = 0; part < PARTS; ++part) {
+          for (int part = 0; part < parts; ++part) {
             const int za = o.za + part * o.zlo, zb = o.zb + part * o.zlo;
             const uint32_t da = sa + part * A_BYTES, db = sb + part * B_BYTES;
             tma_load_3d(da, o.ma, kb * BK, tm * BM, za, fb);
@@ -321,12 +326,12 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
         const TcOps o = tc_ops(h, t, iter, kBN);
         const uint32_t idesc = make_idesc((uint32_t)o.b_mn, kBN);
-        if (!mbar_wait(tempty_bar + 8 * acc, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(tempty_bar + 8 * acc, acc_ph ^ 1u, abort_flag, budget)) { ok = false; break; }
         fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
         const int nk = (o.K + BK - 1) / BK;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(full_bar + 8 * s, ph, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(full_bar + 8 * s, ph, abort_flag, budget)) { ok = false; break; }
           fence_after();
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + PARTS * A_BYTES;
 #pragma unroll
@@ -334,7 +339,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
             const uint64_t ad = desc_sw128(sa + kk * 32, 16);
             const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, 8192) : desc_sw128(sb + kk * 32, 16);
             mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
-            if constexpr (kSplit) {
+            if (kSplit && use_lo) {
               const uint64_t adl = desc_sw128(sa + A_BYTES + kk * 32, 16);
               const uint32_t sbl = sb + B_BYTES;
               const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, 8192) : desc_sw128(sbl + kk * 32, 16);
@@ -365,7 +370,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       int k = 0;
       uint32_t armed = 0, last_par = 0;
       bool ok = true;
-      for (int i = t_begin; i < t_end && ok; ++i) {
+      for (int i = t_begin; i < t_end && ok && !h.starve_tc; ++i) {
         const int tile = tiles[i];
         int tm, tn;
         const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
@@ -376,7 +381,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         for (int c = 0; c < kBN / 32; ++c, ++k) {
           const int slot = k & 1;
           const uint32_t ph = (uint32_t)(k >> 1) & 1u;
-          if (!mbar_wait(sempty_bar + 8 * slot, ph ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(sempty_bar + 8 * slot, ph ^ 1u, abort_flag, budget)) { ok = false; break; }
           const uint32_t fb = sfull_bar + 8 * slot;
           mbar_expect_tx(fb, SRC_BYTES);
           armed |= 1u << slot;
@@ -414,12 +419,12 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       const int tile = tiles[i];
       int tm, tn;
       TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
-      if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag, budget)) { ok = false; break; }
       fence_after();
       const bool tall = iter == 0 && t.md->tall;
       for (int c = 0; c < kBN / 32; ++c, ++kc) {
         const int slot = kc & 1;
-        if (!mbar_wait(sfull_bar + 8 * slot, (uint32_t)(kc >> 1) & 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(sfull_bar + 8 * slot, (uint32_t)(kc >> 1) & 1u, abort_flag, budget)) { ok = false; break; }
         float v[16], x[16];
         tmem_ld16(tmem_base + (uint32_t)(acc * kBN + c * 32 + 16 * half) + ((uint32_t)(ew * 32) << 16), v);
         const float* sp = ring + slot * (SRC_BYTES / 4);
@@ -460,7 +465,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       const int tile = tiles[i];
       int tm, tn;
       TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
-      if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag)) {
+      if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag, budget)) {
         *abort_flag = 1;
         if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
         break;

@@ -42,6 +42,12 @@ __host__ __device__ inline bool wide_out_stage(int st) { return st == ST_AXPY ||
 // CacheMuon reuse and probe products, which read the cached bf16 transform)
 __host__ __device__ inline bool split_stage(int st) { return st != ST_REUSE && st != ST_PROBE; }
 
+// split mode with SMUON_NS_PLAIN_LEAD(k): the Newton-Schulz steps iter < k multiply only the hi parts
+// of their operands (one MMA per product); the lo parts are still written for the later steps
+__host__ __device__ inline bool plain_lead_stage(uint32_t flags, int st, int iter) {
+  return iter < (int)((flags >> 12) & 7u) && (st == ST_GRAM || st == ST_POLY || st == ST_AXPY);
+}
+
 enum Mode : int32_t { MODE_TC_BF16 = 0, MODE_SIMT_F32 = 1, MODE_SIMT_BF16 = 2 };
 
 // one user matrix (user orientation rows x cols); NS runs on the wide form
@@ -118,6 +124,8 @@ struct PlanHeader {
   int32_t sched_ctas[ST_COUNT];     // CTAs of each stage's launch
   int32_t max_k[ST_COUNT];          // longest K of each stage over the groups (picks the smem ring depth)
   int32_t axpy_tma;                 // the B X epilogue's X source is staged in shared memory by TMA
+  int32_t starve_tc;                // failure-detection test: the tensor-core stages' producers issue nothing
+  uint64_t wait_cycles;             // budget of one pipeline wait in the tensor-core stages (SM clocks)
   float* rscale;                    // spectral scaling: r per matrix (X_0 = s r M), or null
   float* lz;                        // Lanczos vectors of every matrix (kLanczosSteps + 2 vectors of m each)
   float* lz_ab;                     // [n_mats][2 kLanczosSteps] Lanczos alpha, beta

@@ -179,3 +179,58 @@ def test_size_limits_are_checked_on_the_host(L):
     assert L.smuon_ns(many, many, 4097, None, 0.9, 1.5, -0.5, 0.0, 1, 1e-7, 0, None, None, None, 0, None,
                       None) == -1
     assert b"n_mats" in L.smuon_last_error()
+
+
+def test_plain_lead_and_bits_outputs_are_checked_before_launch(L):
+    """SMUON_NS_PLAIN_LEAD needs the split mode and excludes spectral scaling and the
+    cached transform; a 1-bit output needs cols % 32 == 0, ld == cols, 16-byte
+    alignment and the tensor-core modes (no device is touched on these paths)."""
+    import matrix_aware_sign_b200 as S
+    args = (None, 0.9, 3.4445, -4.775, 2.0315, 5, 1e-7)
+    m = (S.SmuonMat * 1)(S.SmuonMat(4096, 64, 128, 128, S.F32))
+    u = (S.SmuonMat * 1)(S.SmuonMat(4096, 64, 128, 128, S.F32))
+
+    def call(M_in, U, flags, Q=None):
+        return L.smuon_ns(M_in, U, 1, *args, flags, Q, None, None, 0, None, None)
+
+    assert call(m, u, S.ns_plain_lead(2)) == -1                       # without the split mode
+    assert b"SPLIT" in L.smuon_last_error()
+    assert call(m, u, S.NS_SPLIT_BF16 | S.ns_plain_lead(2) | S.NS_SPECTRAL) == -4
+    assert call(m, u, S.NS_SPLIT_BF16 | S.ns_plain_lead(2) | S.NS_EMIT_Q, u) == -4
+    with pytest.raises(ValueError):
+        S.ns_plain_lead(8)
+    bits = (S.SmuonMat * 1)(S.SmuonMat(4096, 64, 128, 128, S.BITS))
+    assert call(m, bits, S.NS_FP32_REF) == -4                          # CUDA-core modes write no bits
+    assert call(m, bits, S.NS_SPLIT_BF16 | S.NS_EMIT_Q, u) == -4       # nor with the cached transform
+    m100 = (S.SmuonMat * 1)(S.SmuonMat(4096, 64, 100, 100, S.F32))
+    bits100 = (S.SmuonMat * 1)(S.SmuonMat(4096, 64, 100, 100, S.BITS))
+    assert call(m100, bits100, 0) == -2                                # cols % 32 != 0
+    assert b"cols % 32" in L.smuon_last_error()
+    strided = (S.SmuonMat * 1)(S.SmuonMat(4096, 64, 128, 160, S.BITS))
+    assert call(m, strided, 0) == -2                                   # a message has no row stride
+    unaligned = (S.SmuonMat * 1)(S.SmuonMat(4100, 64, 128, 128, S.BITS))
+    assert call(m, unaligned, 0) == -1
+
+
+def test_update_rejects_a_packed_output_for_message_sources(L):
+    import matrix_aware_sign_b200 as S
+    W = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 64, 64, S.F32))
+    U = (S.SmuonMat * 2)(S.SmuonMat(8192, 8, 64, 64, S.BITS), S.SmuonMat(12288, 8, 64, 64, S.BITS))
+    po = (ctypes.c_void_p * 1)(16384)
+    assert L.smuon_update(W, 1, U, None, None, 2, 0.01, 0, 0, po, None, None) == -1
+    assert b"message" in L.smuon_last_error()
+    mixed = (S.SmuonMat * 2)(S.SmuonMat(8192, 8, 64, 64, S.BITS), S.SmuonMat(12288, 8, 64, 64, S.I8))
+    assert L.smuon_update(W, 1, mixed, None, None, 2, 0.01, 0, 0, None, None, None) == -3
+
+
+def test_bits_wrapper_describes_a_message():
+    import torch
+
+    import matrix_aware_sign_b200 as S
+    b = S.Bits(torch.zeros(S.packed_words(96 * 40), dtype=torch.int32), 96, 40)
+    m = S.mat(b)
+    assert (m.rows, m.cols, m.ld, m.dtype) == (96, 40, 40, S.BITS)
+    with pytest.raises(ValueError):
+        S.Bits(torch.zeros(10, dtype=torch.int32), 96, 40)            # too few words
+    with pytest.raises(ValueError):
+        S.Bits(torch.zeros(S.packed_words(96 * 40), dtype=torch.int64), 96, 40)
