@@ -2,11 +2,13 @@
 outputs (the layers, matrices or entries the oracle can afford) and, where
 the oracle cannot follow, against properties that hold at any size.
 
-GPT-2-small set (48 matrices, 8 workers, five quintic steps, popcount vote,
-local polar step): accurate split-BF16 mode. CacheMuon large matrices:
-4096^2 fully checked, 8192^2 and 4096x16384 by properties. LionMuon on the
-GPT-2-Large set (144 matrices, 16 workers, P = 4): sign steps bit-exact on
-sampled entries, the Muon step on a sampled layer."""
+GPT-2-small set (48 matrices, 8 workers, five quintic steps, popcount vote):
+with the local polar step, and with the 1-bit messages written by the
+Newton-Schulz epilogue (the bench's form), in the split-BF16 mode. CacheMuon
+large matrices: 4096^2, 8192^2 and 4096x16384 fresh solves against the oracle
+(the two large ones marked slow), and the schedule by properties. LionMuon on
+the GPT-2-Large set (144 matrices, 16 workers, P = 4): sign steps bit-exact on
+sampled entries, the Muon step's direction on sampled layers."""
 import numpy as np
 import pytest
 import torch
@@ -74,7 +76,70 @@ def test_gpt2_small_set_one_step_sampled():
     assert n_dis <= 1e-4 * n_all
 
 
+def test_gpt2_small_set_one_step_messages():
+    """The GPT-2-small step as the bench runs it: five quintic steps with two
+    plain leading steps, the 1-bit messages written by the last epilogue, and
+    the fused vote / update from the messages. On one layer of each shape: the
+    messages' signs within the sign criterion of the oracle's, and W equal,
+    bit for bit, to the oracle's update wherever the vote agrees; the votes
+    differ at no more than 1e-4 of the entries."""
+    cfg = WL.SIGN_MUON_WORKLOADS["c3_gpt2s"]
+    M, shapes = cfg.workers, cfg.shapes
+    W = WL.weights(shapes, cfg.w_init, cfg.w_dtype)
+    grads = WL.GradientStreams(shapes, M, cfg.grad_sigma).next_step()
+    Md = [torch.zeros(s, device="cuda") for s in shapes for _ in range(M)]
+    Ub = [S.Bits.empty(*s) for s in shapes for _ in range(M)]
+    Gd = [dev(g) for layer in grads for g in layer]
+    Wd = [dev(w, torch.bfloat16) for w in W]
+    flags = S.NS_SPLIT_BF16 | S.ns_plain_lead(2)
+    S.smuon_ns(Md, Ub, *cfg.coeffs, cfg.iters, G=Gd, beta=cfg.beta, flags=flags)
+    S.smuon_update(Wd, cfg.eta, U=[Ub[l * M:(l + 1) * M] for l in range(len(shapes))], M=M,
+                   tie_value=cfg.tie_value)
+    torch.cuda.synchronize()
+    del Gd
+    n_flip, n_vote, n_all, worst = 0, 0, 0, 0.0
+    for l in (0, 1, 2, 3):
+        n = shapes[l][0] * shapes[l][1]
+        ref_u = [O.newton_schulz(grads[l][k].astype(np.float64), *cfg.coeffs, cfg.iters) for k in range(M)]
+        signs = [O.sign_extract(u).reshape(-1) for u in ref_u]
+        gpu = [O.unpack_bits(Ub[l * M + k].words.cpu().numpy().view(np.uint32), n) for k in range(M)]
+        for k in range(M):
+            dis = gpu[k] != signs[k]
+            n_flip += int(dis.sum())
+            if dis.any():
+                worst = max(worst, float(np.abs(ref_u[k].reshape(-1)[dis]).max() / np.abs(ref_u[k]).max()))
+        v_ref = O.vote_from_signs(signs, cfg.tie_value)
+        v_gpu = O.vote_from_signs(gpu, cfg.tie_value)
+        n_vote += int((v_gpu != v_ref).sum())
+        n_all += n
+        # given its own votes the update is exact: W follows the messages bit for bit
+        np.testing.assert_array_equal(host(Wd[l]), O.update_with_vote(W[l], v_gpu.reshape(shapes[l]), cfg.eta, "bf16"))
+        agree = (v_gpu == v_ref).reshape(shapes[l])
+        W_ref = O.update_with_vote(W[l], v_ref.reshape(shapes[l]), cfg.eta, "bf16")
+        np.testing.assert_array_equal(host(Wd[l])[agree], W_ref[agree])
+    assert n_flip <= 1e-4 * n_all * M and worst < 1e-3
+    assert n_vote <= 1e-4 * n_all
+
+
 # ------------------------------------------------------------------ CacheMuon
+@pytest.mark.slow
+@pytest.mark.parametrize("shape", [(8192, 8192), (4096, 16384)])
+def test_cachemuon_large_fresh_solve_against_oracle(shape):
+    """The two larger shapes of the CacheMuon sweep: the fresh solve's
+    direction D (split BF16, five quintic steps) and its cached transform Q
+    against the float64 oracle, in full."""
+    rng = np.random.default_rng(4242)
+    M = rng.standard_normal(shape, dtype=np.float32)
+    m = min(shape)
+    D = torch.zeros(shape, device="cuda")
+    Q = torch.zeros((m, m), dtype=torch.bfloat16, device="cuda")
+    S.smuon_ns([dev(M)], [D], *WL.QUINTIC, 5, flags=S.NS_SPLIT_BF16 | S.NS_EMIT_Q, Q_out=[Q])
+    torch.cuda.synchronize()
+    D_ref, Q_ref = O.newton_schulz_with_q(M.astype(np.float64), *WL.QUINTIC, 5)
+    check_ns_outputs([(host(D), D_ref)], 1e-2)
+    assert rel_fro(host(Q), Q_ref) < 1e-2
+
+
 def test_cachemuon_4096sq_against_oracle():
     shape = (4096, 4096)
     mom = list(WL.cachemuon_momenta(shape, 2, drift=0.01))
@@ -154,6 +219,8 @@ def test_lionmuon_gpt2_large_sampled():
             Wprev_layer1 = Wd[1].float().cpu().numpy()
             M_l1 = [m.cpu().numpy() for m in mom[1]]
             G_l1 = [g.cpu().numpy() for g in G[1]]
+            M_l3 = [m.cpu().numpy() for m in mom[3]]
+            G_l3 = [g.cpu().numpy() for g in G[3]]
         G_s = {l: [G[l][k].view(-1)[torch.from_numpy(idx).cuda()].cpu().numpy() for k in range(M)]
                for l, idx in samples.items()}
         S.lionmuon_step(opt, G, cfg.period, cfg.beta1, cfg.beta2, cfg.eta, *cfg.coeffs, cfg.iters,
@@ -174,11 +241,23 @@ def test_lionmuon_gpt2_large_sampled():
                                               M_s[l][k])
             W_s[l] = host(Wd[l]).reshape(-1)[idx]
     assert opt.t == 4
-    # the Muon step on layer 1 (1280 x 1280) against the oracle's direction
-    gh = [O.lion_interpolate(M_l1[k], G_l1[k], cfg.beta1) for k in range(M)]
-    D_ref = O.newton_schulz(np.mean(np.stack([g.astype(np.float64) for g in gh]), 0), *cfg.coeffs, cfg.iters)
-    W_ref = O.update_dense(Wprev_layer1, D_ref, cfg.eta, "bf16")
-    assert np.mean(host(Wd[1]) != W_ref) < 0.05
+    # the Muon step's direction on sampled layers (1280 x 1280 and the tall 5120 x 1280): the same step
+    # replayed from the same EMA and gradients on a float32 shadow whose weights start at zero, so the
+    # shadow holds -f32(f32(eta) D) exactly; D against the oracle's by the Newton-Schulz criteria
+    for l, (M_l, G_l) in ((1, (M_l1, G_l1)), (3, (M_l3, G_l3))):
+        shadow = [torch.zeros(shapes[l], device="cuda")]
+        smom = [[dev(x) for x in M_l]]
+        sopt = S.LionMuon(shadow, smom, t=3)
+        S.lionmuon_step(sopt, [[dev(g) for g in G_l]], cfg.period, cfg.beta1, cfg.beta2, cfg.eta, *cfg.coeffs,
+                        cfg.iters, tie_value=cfg.tie_value, ns_flags=S.NS_SPLIT_BF16)
+        torch.cuda.synchronize()
+        d_gpu = -host(shadow[0]).astype(np.float64) / np.float32(cfg.eta)
+        gh = [O.lion_interpolate(M_l[k], G_l[k], cfg.beta1) for k in range(M)]
+        D_ref = O.newton_schulz(np.mean(np.stack([g.astype(np.float64) for g in gh]), 0), *cfg.coeffs, cfg.iters)
+        check_ns_outputs([(d_gpu, D_ref)], 1e-2)
+        if l == 1:  # the bf16 weights moved by that same step: RN_bf16(W - f32(eta D)) = RN_bf16(W + shadow)
+            step = host(shadow[0]).astype(np.float32)
+            np.testing.assert_array_equal(host(Wd[1]), O.bf16_round(np.add(Wprev_layer1, step, dtype=np.float32)))
 
 
 # ------------------------------------------------------------------ LLaMA-style sets

@@ -501,3 +501,25 @@ def test_sign_muon_step_spectral_passes_the_scaling_through():
     v = O.vote_from_packed([O.pack_bits(O.sign_extract(u)) for u in out["U"][0]], M, 54).reshape(shape)
     np.testing.assert_array_equal(out["vote"][0], v)
     np.testing.assert_array_equal(out["W"][0], O.update_with_vote(W[0], v, 0.01, "f32"))
+
+
+@pytest.mark.parametrize("honest,bad", [(3, 1), (4, 1), (5, 2), (6, 3)])
+def test_vote_tolerates_a_minority_of_corrupted_workers(honest, bad):
+    """The robustness the SignMuon summary's significance section claims for
+    the majority vote, brute force: for every pattern of honest signs and every
+    pattern of corrupted ones, an entry whose honest margin |sum| exceeds the
+    number of corrupted workers keeps the honest vote."""
+    hp = np.array(list(itertools.product([-1, 1], repeat=honest)), np.int8)     # [2^h, h]
+    bp = np.array(list(itertools.product([-1, 1], repeat=bad)), np.int8)        # [2^b, b]
+    H = np.repeat(hp, len(bp), axis=0)
+    B = np.tile(bp, (len(hp), 1))
+    signs = [H[:, k] for k in range(honest)] + [B[:, k] for k in range(bad)]
+    v = O.vote_from_signs(signs, 0)
+    margin = H.astype(np.int64).sum(axis=1)
+    safe = np.abs(margin) > bad
+    assert safe.any()
+    np.testing.assert_array_equal(v[safe], np.sign(margin[safe]))
+    # and the bound is tight: at margin == bad some corruption reaches a tie or flips the vote
+    edge = np.abs(margin) == bad
+    if edge.any():
+        assert np.any(v[edge] != np.sign(margin[edge]))
