@@ -524,7 +524,8 @@ static cudaError_t launch_tc_variant(const Plan* d_plan, int stage, int iter, co
 template <bool kSplit, int kBN, bool kSrc>
 static cudaError_t launch_tc_src(const PlanHeader& h, const Plan* d_plan, int stage, int iter,
                                  const int32_t* skip, int grid, cudaStream_t s) {
-  if (h.max_k[stage] <= kShallowMaxK)
+  // split operands of 256-wide tiles take 96 KB per ring stage: only the deep ring holds two of them
+  if (h.max_k[stage] <= kShallowMaxK && !(kSplit && kBN == 256))
     return launch_tc_variant<kSplit, kBN, true, kSrc>(d_plan, stage, iter, skip, grid, s);
   return launch_tc_variant<kSplit, kBN, false, kSrc>(d_plan, stage, iter, skip, grid, s);
 }
@@ -542,7 +543,7 @@ static cudaError_t launch_tc_depth(const PlanHeader& h, const Plan* d_plan, int 
 
 int tc_tile_n(int stage, uint32_t flags) {
   (void)stage;
-  return (flags & SMUON_NS_SPLIT_BF16) ? 128 : 256;  // split mode needs the smem for its lo tiles
+  return (flags & SMUON_NS_SPLIT_BF16) ? kSplitBN : 256;  // split mode needs the smem for its lo tiles
 }
 
 cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter, const int32_t* skip,
@@ -551,7 +552,7 @@ cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, i
   const int grid = h.sched_ctas[stage];
   if (h.total_tiles[stage] == 0 || grid <= 0) return cudaSuccess;
   const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(stage);
-  if (split) return launch_tc_depth<true, 128>(h, d_plan, stage, iter, skip, grid, s);
+  if (split) return launch_tc_depth<true, kSplitBN>(h, d_plan, stage, iter, skip, grid, s);
   if (tc_tile_n(stage, h.flags) == 128) return launch_tc_depth<false, 128>(h, d_plan, stage, iter, skip, grid, s);
   return launch_tc_depth<false, 256>(h, d_plan, stage, iter, skip, grid, s);
 }

@@ -92,6 +92,10 @@ cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, i
                            const int32_t* skip, int num_sms, cudaStream_t s);
 constexpr int kProbeSlots = 8;  // residual partial sums per probe tile (one per epilogue warp)
 constexpr int kTcBM = 128;
+#ifndef SMUON_SPLIT_BN
+#define SMUON_SPLIT_BN 128
+#endif
+constexpr int kSplitBN = SMUON_SPLIT_BN;  // tile width of the split-BF16 stages (128: three ring stages of 64 KB)
 int tc_tile_n(int stage, uint32_t flags);  // 128 (symmetric stages, split mode) or 256
 constexpr int kSimtBM = 64;
 constexpr int kSimtBN = 64;
