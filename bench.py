@@ -97,6 +97,8 @@ def parse_args(argv=None):
     p.add_argument("--diagnose", action="store_true",
                    help="CacheMuon sweep: every step also runs a fresh solve and records the residual beside the "
                         "cached/fresh agreement")
+    p.add_argument("--drift", type=float, default=0.01,
+                   help="CacheMuon sweep: momentum drift per step, M_{t+1} = M_t + drift * N(0,1) (default 0.01)")
     p.add_argument("--cachemuon", nargs="*", metavar="RxC:GAMMA",
                    help="CacheMuon sweep instead of the Sign-Muon step, e.g. 4096x4096:2 8192x8192:15 "
                         "(no value: the three large shapes x gamma in {2, 15}); --steps sets the schedule length")
@@ -329,8 +331,8 @@ def cachemuon_saved(counts, hits, misses, probes, steps, gram_only):
     return 1.0 - cost / (steps * counts["muon"])
 
 
-def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagnose=False):
-    """M_0 ~ N(0,1); M_{t+1} = M_t + 0.01 N(0,1); every step probes the cached
+def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagnose=False, drift=0.01):
+    """M_0 ~ N(0,1); M_{t+1} = M_t + drift N(0,1); every step probes the cached
     transform on the device and runs the fresh solve only when the residual
     exceeds gamma. Reports the hit rate and the orthogonalisation flops saved
     against a fresh five-step quintic solve every step, on nominal and on
@@ -355,7 +357,7 @@ def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagn
     for t in range(steps):
         if t:
             noise.normal_(generator=gen)
-            M.add_(noise, alpha=0.01)
+            M.add_(noise, alpha=drift)
         if not diagnose:
             cm.step()
             continue
@@ -373,7 +375,7 @@ def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagn
     ms = e0.elapsed_time(e1)
     c = cm.counters()
     counts, sym = cachemuon_flop_counts(m, n, iters, gram_only)
-    out = {"workload": "cachemuon", "shape": list(shape), "gamma": gamma, "steps": steps,
+    out = {"workload": "cachemuon", "shape": list(shape), "gamma": gamma, "steps": steps, "drift": drift,
            "hits": c["hits"], "misses": c["misses"], "hit_rate": c["hits"] / steps,
            "orth_flops_saved_vs_fresh": cachemuon_saved(counts, c["hits"], c["misses"], c["probes"], steps, gram_only),
            "orth_flops_saved_vs_fresh_symmetric_aware": cachemuon_saved(sym, c["hits"], c["misses"], c["probes"],
@@ -1093,7 +1095,7 @@ def main():
             shp, gam = case.split(":")
             r, c = (int(x) for x in shp.split("x"))
             print(json.dumps(run_cachemuon(S, torch, (r, c), float(gam), args.steps, gram_only=args.gram_only,
-                                           diagnose=args.diagnose)), flush=True)
+                                           diagnose=args.diagnose, drift=args.drift)), flush=True)
         return
     if args.only_ns4096:
         flags = S.NS_SPLIT_BF16 if (args.ns_mode or "split") == "split" else 0

@@ -148,14 +148,16 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
                                       SMUON_NS_NO_NORMALIZE, SMUON_NS_EMIT_Q or SMUON_NS_GRAM_ONLY */
 #define SMUON_NS_PLAIN_LEAD(k) ((uint32_t)(k) << 12)  /* with SMUON_NS_SPLIT_BF16: the first k (0..7)
                                       Newton-Schulz steps take plain BF16 operands (one MMA per product, the
-                                      lo parts still written for the later steps). While the normalised
-                                      singular values are small, the B X term of a step is small beside the
-                                      float32 a X term, so its operand rounding barely reaches the output;
-                                      from s_max(X_0) ~ 0.06 (Gaussian momenta of the workload shapes) two
-                                      plain steps keep five quintic steps within the split mode's accuracy.
-                                      A matrix with one dominant singular value has s_max near 1 from the
-                                      start: leave k = 0 there. Not with SMUON_NS_SPECTRAL (s_max = 1),
-                                      SMUON_NS_EMIT_Q or SMUON_NS_GRAM_ONLY */
+                                      lo parts still written for the later steps) -- for matrices whose
+                                      smaller side is at least 512; smaller matrices take only their first
+                                      step plain. While the normalised singular values are small, the B X
+                                      term of a step is small beside the float32 a X term, so its operand
+                                      rounding barely reaches the output. On Gaussian momenta this keeps five
+                                      quintic steps within the split mode's accuracy for k <= 2; the top
+                                      normalised singular value starts near 1/sqrt(m) + 1/sqrt(n). A matrix
+                                      with one dominant singular value starts near 1: leave k = 0 there. Not
+                                      with SMUON_NS_SPECTRAL (s_max = 1), SMUON_NS_EMIT_Q or
+                                      SMUON_NS_GRAM_ONLY */
 #define SMUON_NS_PLAIN_LEAD_MASK (7u << 12)
 #define SMUON_NS_TEST_WAIT_EXPIRY 0x8000u  /* failure-detection test, not for use: every tensor-core stage's
                                       copy producers issue nothing and its pipeline waits are limited to

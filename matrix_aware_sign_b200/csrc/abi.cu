@@ -139,7 +139,8 @@ smuon_status get_encoder(EncodeTiledFn* fn) {
 
 // 3-D bf16 map over [count][rows][ld] with box {box0 (inner), box1, 1}, 128B swizzle
 smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, int64_t rows, int64_t count,
-                            int64_t ld, uint32_t box0, uint32_t box1) {
+                            int64_t ld, uint32_t box0, uint32_t box1,
+                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc;
   smuon_status st = get_encoder(&enc);
   if (st != SMUON_OK) return st;
@@ -148,7 +149,7 @@ smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, in
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return SMUON_OK;
@@ -581,28 +582,37 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   B->maps.assign(std::max(L.n_tmaps, 1), CUtensorMap{});
   for (auto& g : B->groups) {
     if (!tc) continue;
-    auto enc = [&](int32_t slot, const void* p, int64_t inner, int64_t rows, int64_t cnt, int64_t ld, uint32_t b0,
-                   uint32_t b1) -> smuon_status {
+    // K-major boxes {bk, rows}: 128-byte swizzled rows of 64 bf16, or (split stages with 32-deep k-blocks)
+    // 64-byte swizzled rows of 32; MN-major boxes {64, bk} with the 128-byte swizzle
+    const uint32_t bk = parts == 2 ? (uint32_t)kSplitBK : 64u;
+    const CUtensorMapSwizzle kswz = bk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    auto enc = [&](int32_t slot, const void* p, int64_t inner, int64_t rows, int64_t cnt, int64_t ld,
+                   uint32_t b1) -> smuon_status {  // K-major
       if (slot < 0) return SMUON_OK;
-      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, b0, b1);
+      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, bk, b1, kswz);
+    };
+    auto enc_mn = [&](int32_t slot, const void* p, int64_t inner, int64_t rows, int64_t cnt,
+                      int64_t ld) -> smuon_status {
+      if (slot < 0) return SMUON_OK;
+      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, 64, bk);
     };
     smuon_status st;
     const int64_t zc = (int64_t)g.count * parts;  // matrices in the map: hi parts, then lo parts
     for (int i = 0; i < 2; ++i) {
-      if ((st = enc(g.tm_x_k[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 128)) != SMUON_OK) return st;
-      if ((st = enc(g.tm_x_mn[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 64)) != SMUON_OK) return st;
-      if ((st = enc(g.tm_q_mn[i], g.qop[i], g.m, g.m, zc, g.ldm, 64, 64)) != SMUON_OK) return st;
-      if ((st = enc(g.tm_q_k[i], g.qop[i], g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
-      if ((st = enc(g.tm_x_kw[i], g.xop[i], g.n, g.m, zc, g.ldn, 64, 256)) != SMUON_OK) return st;
+      if ((st = enc(g.tm_x_k[i], g.xop[i], g.n, g.m, zc, g.ldn, 128)) != SMUON_OK) return st;
+      if ((st = enc_mn(g.tm_x_mn[i], g.xop[i], g.n, g.m, zc, g.ldn)) != SMUON_OK) return st;
+      if ((st = enc_mn(g.tm_q_mn[i], g.qop[i], g.m, g.m, zc, g.ldm)) != SMUON_OK) return st;
+      if ((st = enc(g.tm_q_k[i], g.qop[i], g.m, g.m, zc, g.ldm, 128)) != SMUON_OK) return st;
+      if ((st = enc(g.tm_x_kw[i], g.xop[i], g.n, g.m, zc, g.ldn, 256)) != SMUON_OK) return st;
     }
-    if ((st = enc(g.tm_a_kw, g.aop, g.m, g.m, zc, g.ldm, 64, 256)) != SMUON_OK) return st;
-    if ((st = enc(g.tm_t_k, g.aop2, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
-    if ((st = enc(g.tm_t_kw, g.aop2, g.m, g.m, zc, g.ldm, 64, 256)) != SMUON_OK) return st;
-    if ((st = enc(g.tm_a_k, g.aop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
-    if ((st = enc(g.tm_b_k, g.bop, g.m, g.m, zc, g.ldm, 64, 128)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_a_kw, g.aop, g.m, g.m, zc, g.ldm, 256)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_t_k, g.aop2, g.m, g.m, zc, g.ldm, 128)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_t_kw, g.aop2, g.m, g.m, zc, g.ldm, 256)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_a_k, g.aop, g.m, g.m, zc, g.ldm, 128)) != SMUON_OK) return st;
+    if ((st = enc(g.tm_b_k, g.bop, g.m, g.m, zc, g.ldm, 128)) != SMUON_OK) return st;
     if (g.tm_uq_k >= 0) {
       const MatDesc& d = B->mats[g.first_mat];
-      if ((st = enc(g.tm_uq_k, d.q_ptr, g.m, g.m, 1, d.q_ld, 64, 128)) != SMUON_OK) return st;
+      if ((st = encode_bf16_3d(&B->maps[g.tm_uq_k], d.q_ptr, g.m, g.m, 1, d.q_ld, 64, 128)) != SMUON_OK) return st;
     }
     for (int i = 0; i < 2; ++i)  // f32 masters [count][m][ldn], 32 x 128 boxes
       if (g.tm_xf[i] >= 0 &&
@@ -673,22 +683,24 @@ double stage_flops(const Builder& B, int st) {
 
 // flops the tensor cores (or CUDA cores) actually execute for a stage: tiles
 // x 2 * BM * BN * (K rounded up to the k-block), three products in split mode
-double stage_issued(const Builder& B, int st) {
+double stage_issued(const Builder& B, int st, int iter = 1 << 20) {
   const PlanHeader& h = B.h;
   const bool tc = h.mode == MODE_TC_BF16;
   const int BM = tc ? kTcBM : kSimtBM, BK = tc ? 64 : 16;
   const bool split = tc && (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
   double f = 0;
   for (const GroupDesc& g : B.groups) {
+    // split mode: three products per tile, one in a group's plain leading steps
+    const double parts = !split ? 1.0 : (plain_lead_stage(h.flags, st, iter, g.m) ? 1.0 : 3.0);
     const bool sym = sym_stage(st);
     const int BN = sym ? BM : (tc ? tc_tile_n(st, h.flags) : kSimtBN);
     const int T = g.tiles_m[st];
     const double tiles = (double)g.count * (sym ? T * (T + 1) / 2 : T * g.tiles_n[st]);
     const int K = (st == ST_GRAM || st == ST_PROBE) ? g.n : g.m;
     const double kpad = (double)((K + BK - 1) / BK) * BK;
-    f += tiles * 2.0 * BM * BN * kpad;
+    f += parts * tiles * 2.0 * BM * BN * kpad;
   }
-  return split ? 3 * f : f;
+  return f;
 }
 
 // algorithmic bytes of the momentum / normalisation prologue
@@ -716,8 +728,7 @@ smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int it
        "k_gemm_tc_split.qx"}};
   if (h.mode == MODE_TC_BF16) {
     const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
-    const bool lead = split && plain_lead_stage(h.flags, st, iter);  // hi parts only: one product in three
-    Launch L(tc_names[split][st], SMUON_WORK_FLOPS, lead ? issued_flops / 3 : issued_flops, s, stage_flops);
+    Launch L(tc_names[split][st], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
     CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
   } else {
     const int grid = std::min(total, di.sms * 6);
@@ -809,6 +820,7 @@ struct NsExec {
   double mom_bytes = 0;
   double sflops[ST_COUNT] = {0};
   double sissued[ST_COUNT] = {0};
+  double sissued_lead[8][ST_COUNT] = {{0}};  // issued flops of iteration k < 8 (plain leading steps)
   int64_t lz_rows = 0;          // spectral scaling: rows of all A_0 together
   double lz_matvec_bytes = 0;   // bytes of one A v product over the batch
 };
@@ -839,6 +851,7 @@ smuon_status prepare_ns(const NsRequest& rq, void* ws, size_t ws_bytes, int32_t*
   for (int k = 0; k < ST_COUNT; ++k) {
     ex->sflops[k] = stage_flops(B, k);
     ex->sissued[k] = stage_issued(B, k);
+    for (int it = 0; it < 8; ++it) ex->sissued_lead[it][k] = stage_issued(B, k, it);
   }
   return SMUON_OK;
 }
@@ -911,12 +924,13 @@ smuon_status run_ns(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
     }
     return run(ST_QX, ex.iters);
   }
+  auto issued = [&](int stg, int k) { return k < 8 ? ex.sissued_lead[k][stg] : ex.sissued[stg]; };
   for (int k = 0; k < ex.iters; ++k) {
-    if ((st = launch_gemm(ex.d_plan, h, ST_GRAM, k, skip, di, s, ex.sflops[ST_GRAM], ex.sissued[ST_GRAM])) != SMUON_OK) return st;
+    if ((st = launch_gemm(ex.d_plan, h, ST_GRAM, k, skip, di, s, ex.sflops[ST_GRAM], issued(ST_GRAM, k))) != SMUON_OK) return st;
     if (k == 0 && (ex.flags & SMUON_NS_SPECTRAL) && (st = run_lanczos(ex, skip, s)) != SMUON_OK) return st;
-    if (ex.c != 0.f && (st = launch_gemm(ex.d_plan, h, ST_POLY, k, skip, di, s, ex.sflops[ST_POLY], ex.sissued[ST_POLY])) != SMUON_OK)
+    if (ex.c != 0.f && (st = launch_gemm(ex.d_plan, h, ST_POLY, k, skip, di, s, ex.sflops[ST_POLY], issued(ST_POLY, k))) != SMUON_OK)
       return st;
-    if ((st = launch_gemm(ex.d_plan, h, ST_AXPY, k, skip, di, s, ex.sflops[ST_AXPY], ex.sissued[ST_AXPY])) != SMUON_OK) return st;
+    if ((st = launch_gemm(ex.d_plan, h, ST_AXPY, k, skip, di, s, ex.sflops[ST_AXPY], issued(ST_AXPY, k))) != SMUON_OK) return st;
     if (emit_q && k >= 1 &&
         (st = launch_gemm(ex.d_plan, h, ST_QAXPY, k, skip, di, s, ex.sflops[ST_QAXPY], ex.sissued[ST_QAXPY])) != SMUON_OK)
       return st;

@@ -24,8 +24,7 @@
 namespace smuon {
 namespace tc {
 
-constexpr int BM = kTcBM, BK = 64;
-constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x 64 k)
+constexpr int BM = kTcBM;
 constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps (+ one source warp for B X)
 constexpr int SRC_SLOTS = 2;                // B X epilogue source ring
 constexpr int SRC_BYTES = BM * 32 * 4;      // one 128 x 32 f32 chunk of X (or its transpose)
@@ -37,11 +36,16 @@ constexpr int SRC_BYTES = BM * 32 * 4;      // one 128 x 32 f32 chunk of X (or i
 // 192 KB of shared memory, or about 144 KB (kShallow) for stages whose K is
 // short: a tile then needs few k-blocks in flight, and the shared memory left
 // to the L1 cache serves the epilogue's row-per-lane global accesses.
+// k-block depth: 64 (128-byte swizzled K-major rows), or for the split stages kSplitBK (32: 64-byte
+// swizzled K-major rows, so that four ring stages of 128 x 256 split tiles fit)
 template <bool kSplit, int kBN, bool kShallow, bool kSrc>
 struct Cfg {
   static constexpr int PARTS = kSplit ? 2 : 1;
   static constexpr int BN = kBN;
+  static constexpr int BK = kSplit ? kSplitBK : 64;
+  static constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x BK)
   static constexpr int B_BYTES = kBN * BK * 2;
+  static constexpr int MN_BOX = 64 * BK * 2;     // one {64, BK} box of an MN-major B operand
   static constexpr int STAGE_BYTES = PARTS * (A_BYTES + B_BYTES);
   static constexpr int STAGES = ((kShallow ? 144 : 192) * 1024) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * kBN;
@@ -50,6 +54,9 @@ struct Cfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SRC_RING + 1024 /*align*/ + 256 /*barriers*/;
 };
 constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz: the exit drains' budget
+#ifndef SMUON_AXPY_PREFETCH
+#define SMUON_AXPY_PREFETCH 0
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -109,6 +116,22 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
   d |= (uint64_t)1 << 46;            // descriptor version for sm_100
   d |= (uint64_t)2 << 61;            // SWIZZLE_128B
   return d;
+}
+// K-major rows of 32 bf16 (64 bytes) with the 64-byte swizzle: 8-row groups of 512 bytes
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)(16 >> 4) << 16;
+  d |= (uint64_t)(512 >> 4) << 32;   // 8-row group stride
+  d |= (uint64_t)1 << 46;            // descriptor version for sm_100
+  d |= (uint64_t)4 << 61;            // SWIZZLE_64B
+  return d;
+}
+// K-major descriptor of a BK-deep tile at k-step kk (16 elements = 32 bytes into each row)
+template <int kBK>
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr, int kk) {
+  if constexpr (kBK == 64) return desc_sw128(saddr + kk * 32, 16);
+  else return desc_sw64(saddr + kk * 32);
 }
 
 // instruction descriptor: BF16 x BF16 -> F32, A K-major, B K- or MN-major, 128 x n
@@ -218,6 +241,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   constexpr int STAGE_BYTES = C::STAGE_BYTES;
   constexpr int PARTS = C::PARTS;
   constexpr int B_BYTES = C::B_BYTES;
+  constexpr int A_BYTES = C::A_BYTES;
+  constexpr int BK = C::BK;
   const PlanHeader& h = plan->h;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -252,10 +277,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // split mode: both parts of every operand, except in the plain leading steps (hi parts only); the
-  // producer and the MMA issuer take the same decision from the plan
+  // producer and the MMA issuer take the same decision, per tile, from the tile's group
   const unsigned long long budget = h.wait_cycles;
-  const bool use_lo = kSplit && !plain_lead_stage(h.flags, stage, iter);
-  const int parts = use_lo ? PARTS : 1;
   // this CTA's tiles (host-balanced list; every role walks the same one)
   const int32_t* tiles = h.sched + h.sched_off[stage];
   const int t_begin = h.sched_begin[h.sched_boff[stage] + blockIdx.x];
@@ -271,6 +294,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       const int tile = tiles[i];
       int tm, tn;
       const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+      const int parts = (kSplit && !plain_lead_stage(h.flags, stage, iter, t.g->m)) ? PARTS : 1;
       if (lane == 0) {
         const TcOps o = tc_ops(h, t, iter, kBN);
         tensormap_acquire(o.ma);
@@ -289,7 +313,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
             tma_load_3d(da, o.ma, kb * BK, tm * BM, za, fb);
             if (o.b_mn) {
 #pragma unroll
-              for (int q = 0; q < kBN / 64; ++q) tma_load_3d(db + q * 8192, o.mb, tn * kBN + 64 * q, kb * BK, zb, fb);
+              for (int q = 0; q < kBN / 64; ++q) tma_load_3d(db + q * C::MN_BOX, o.mb, tn * kBN + 64 * q, kb * BK, zb, fb);
             } else {
               tma_load_3d(db, o.mb, kb * BK, tn * kBN, zb, fb);
             }
@@ -326,6 +350,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
         const TcOps o = tc_ops(h, t, iter, kBN);
         const uint32_t idesc = make_idesc((uint32_t)o.b_mn, kBN);
+        const bool use_lo = kSplit && !plain_lead_stage(h.flags, stage, iter, t.g->m);
         if (!mbar_wait(tempty_bar + 8 * acc, acc_ph ^ 1u, abort_flag, budget)) { ok = false; break; }
         fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
@@ -336,13 +361,13 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + PARTS * A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = desc_sw128(sa + kk * 32, 16);
-            const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, 8192) : desc_sw128(sb + kk * 32, 16);
+            const uint64_t ad = desc_k<BK>(sa, kk);
+            const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, C::MN_BOX) : desc_k<BK>(sb, kk);
             mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
             if (kSplit && use_lo) {
-              const uint64_t adl = desc_sw128(sa + A_BYTES + kk * 32, 16);
+              const uint64_t adl = desc_k<BK>(sa + A_BYTES, kk);
               const uint32_t sbl = sb + B_BYTES;
-              const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, 8192) : desc_sw128(sbl + kk * 32, 16);
+              const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, C::MN_BOX) : desc_k<BK>(sbl, kk);
               mma_bf16(d_tmem, ad, bdl, idesc, 1u);   // A_hi * B_lo
               mma_bf16(d_tmem, adl, bd, idesc, 1u);   // A_lo * B_hi
             }
@@ -465,16 +490,33 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       const int tile = tiles[i];
       int tm, tn;
       TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+      const int row = tm * BM + ew * 32 + lane;
+#if SMUON_AXPY_PREFETCH
+      // the first step's B X epilogue reads its a X term row by row from the caller's f32 momentum: ask L1
+      // for each chunk's 128 bytes one chunk ahead, the first before the accumulator is ready
+      const bool pf = stage == ST_AXPY && iter == 0 && !t.md->tall && t.md->m_dtype == SMUON_F32 && row < t.Mo;
+      const float* pf_row = pf ? reinterpret_cast<const float*>(t.md->m_ptr) + (int64_t)row * t.md->m_ld : nullptr;
+      auto prefetch_chunk = [&](int ch) {
+        const int col = tn * kBN + ch * 32;
+        if (pf && col < t.No) {
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(pf_row + col));
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(pf_row + min(col + 31, t.No - 1)));
+        }
+      };
+      prefetch_chunk(half * CH);
+#endif
       if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag, budget)) {
         *abort_flag = 1;
         if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
         break;
       }
       fence_after();
-      const int row = tm * BM + ew * 32 + lane;
       float pacc = 0.f;
 #pragma unroll 1
       for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
+#if SMUON_AXPY_PREFETCH
+        if (ch + 1 < (half + 1) * CH) prefetch_chunk(ch + 1);
+#endif
         float v[32];
         tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
         epi_chunk<32>(t, row, tn * kBN + ch * 32, v, &pacc);

@@ -96,6 +96,10 @@ constexpr int kTcBM = 128;
 #define SMUON_SPLIT_BN 128
 #endif
 constexpr int kSplitBN = SMUON_SPLIT_BN;  // tile width of the split-BF16 stages (128: three ring stages of 64 KB)
+#ifndef SMUON_SPLIT_BK
+#define SMUON_SPLIT_BK 64
+#endif
+constexpr int kSplitBK = SMUON_SPLIT_BK;  // k-block depth of the split-BF16 stages (64, or 32 with 64-byte swizzle)
 int tc_tile_n(int stage, uint32_t flags);  // 128 (symmetric stages, split mode) or 256
 constexpr int kSimtBM = 64;
 constexpr int kSimtBN = 64;

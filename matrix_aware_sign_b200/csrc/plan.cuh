@@ -42,10 +42,15 @@ __host__ __device__ inline bool wide_out_stage(int st) { return st == ST_AXPY ||
 // CacheMuon reuse and probe products, which read the cached bf16 transform)
 __host__ __device__ inline bool split_stage(int st) { return st != ST_REUSE && st != ST_PROBE; }
 
-// split mode with SMUON_NS_PLAIN_LEAD(k): the Newton-Schulz steps iter < k multiply only the hi parts
-// of their operands (one MMA per product); the lo parts are still written for the later steps
-__host__ __device__ inline bool plain_lead_stage(uint32_t flags, int st, int iter) {
-  return iter < (int)((flags >> 12) & 7u) && (st == ST_GRAM || st == ST_POLY || st == ST_AXPY);
+// split mode with SMUON_NS_PLAIN_LEAD(k): the Newton-Schulz steps iter < k of a matrix group multiply only
+// the hi parts of their operands (one MMA per product; the lo parts are still written for the later
+// steps): every group's first step, and the later ones only where the smaller side m is at least
+// kPlainLeadMinM (below that the normalised singular values start near 1/sqrt(m), too large for a second
+// plain step)
+constexpr int kPlainLeadMinM = 512;
+__host__ __device__ inline bool plain_lead_stage(uint32_t flags, int st, int iter, int m) {
+  return iter < (int)((flags >> 12) & 7u) && (iter == 0 || m >= kPlainLeadMinM) &&
+         (st == ST_GRAM || st == ST_POLY || st == ST_AXPY);
 }
 
 enum Mode : int32_t { MODE_TC_BF16 = 0, MODE_SIMT_F32 = 1, MODE_SIMT_BF16 = 2 };

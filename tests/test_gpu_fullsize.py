@@ -161,11 +161,12 @@ def test_cachemuon_4096sq_against_oracle():
     assert cm.counters() == {"hits": 1, "misses": 1, "probes": 1}
 
 
-@pytest.mark.parametrize("shape", [(8192, 8192), (4096, 16384)])
-def test_cachemuon_large_properties(shape):
+@pytest.mark.parametrize("shape,drift", [((8192, 8192), 0.01), ((4096, 16384), 0.01), ((4096, 16384), 1.0)])
+def test_cachemuon_large_properties(shape, drift):
     """Beyond the oracle's reach: the residual the kernel reports is the
     residual of the candidate it returned, the decision follows it, the
-    counters follow the decisions, and a rejected step is a fresh solve."""
+    counters follow the decisions, and a rejected step is a fresh solve (with
+    a drift as large as the momentum, the cached transform goes stale)."""
     m = min(shape)
     gen = torch.Generator(device="cuda").manual_seed(4242)
     Md = torch.randn(shape, device="cuda", generator=gen)
@@ -174,7 +175,7 @@ def test_cachemuon_large_properties(shape):
     cm = S.CacheMuon(Md, D, 2.0, WL.QUINTIC, 5)
     for t in range(4):
         if t:
-            Md.add_(torch.randn(shape, device="cuda", generator=gen), alpha=0.01)
+            Md.add_(torch.randn(shape, device="cuda", generator=gen), alpha=drift)
         cm.step()
         torch.cuda.synchronize()
         acc = int(cm.accept.item())
@@ -185,10 +186,17 @@ def test_cachemuon_large_properties(shape):
             if acc:  # D is the candidate the probe measured
                 err = float(torch.linalg.norm(R) / m ** 0.5)
                 assert abs(cm.err.item() - err) <= 5e-3 * err + 1e-3
+            else:  # D is the fresh solve of this momentum
+                D_fresh = torch.empty_like(D)
+                S.smuon_ns([Md], [D_fresh], *WL.QUINTIC, 5, flags=S.NS_SPLIT_BF16)
+                torch.cuda.synchronize()
+                assert torch.equal(D, D_fresh)
             assert acc == int(cm.err.item() <= 2.0)
     c = cm.counters()
     assert decisions[0] == 0 and c["hits"] == sum(decisions) and c["misses"] == 4 - sum(decisions)
     assert c["probes"] == 3
+    if drift >= 1.0:  # the stale transform is refused at least once
+        assert sum(decisions[1:]) < 3
 
 
 # ------------------------------------------------------------------ LionMuon

@@ -73,3 +73,15 @@ def test_operand_precision_choices(shape):
     lead2 = _ns(M, [PLAIN] * 2 + [SPLIT] * 3)
     assert _passes(lead2, R) and _criteria(lead2, R)[0] < 1e-3
     assert not _passes(_ns(M, [PLAIN] * 3 + [SPLIT] * 2), R)
+
+
+@pytest.mark.parametrize("shape", [(96, 320), (200, 96)])
+def test_plain_leading_steps_on_small_matrices(shape):
+    """Small matrices start with larger normalised singular values (near
+    1/sqrt(m) + 1/sqrt(n)): one plain leading step still meets the criteria, two
+    do not. The library therefore runs later plain steps only where the smaller
+    side is at least 512."""
+    M = np.random.default_rng(shape[0] * 7 + shape[1]).standard_normal(shape)
+    R = O.newton_schulz(M, *WL.QUINTIC, 5)
+    assert _passes(_ns(M, [PLAIN] + [SPLIT] * 4), R)
+    assert not _passes(_ns(M, [PLAIN] * 2 + [SPLIT] * 3), R)
