@@ -139,8 +139,7 @@ smuon_status get_encoder(EncodeTiledFn* fn) {
 
 // 3-D bf16 map over [count][rows][ld] with box {box0 (inner), box1, 1}, 128B swizzle
 smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, int64_t rows, int64_t count,
-                            int64_t ld, uint32_t box0, uint32_t box1,
-                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+                            int64_t ld, uint32_t box0, uint32_t box1) {
   EncodeTiledFn enc;
   smuon_status st = get_encoder(&enc);
   if (st != SMUON_OK) return st;
@@ -149,7 +148,7 @@ smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, in
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return SMUON_OK;
@@ -582,19 +581,16 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   B->maps.assign(std::max(L.n_tmaps, 1), CUtensorMap{});
   for (auto& g : B->groups) {
     if (!tc) continue;
-    // K-major boxes {bk, rows}: 128-byte swizzled rows of 64 bf16, or (split stages with 32-deep k-blocks)
-    // 64-byte swizzled rows of 32; MN-major boxes {64, bk} with the 128-byte swizzle
-    const uint32_t bk = parts == 2 ? (uint32_t)kSplitBK : 64u;
-    const CUtensorMapSwizzle kswz = bk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    // K-major boxes {64, rows} and MN-major boxes {64, 64}, both with the 128-byte swizzle
     auto enc = [&](int32_t slot, const void* p, int64_t inner, int64_t rows, int64_t cnt, int64_t ld,
                    uint32_t b1) -> smuon_status {  // K-major
       if (slot < 0) return SMUON_OK;
-      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, bk, b1, kswz);
+      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, 64, b1);
     };
     auto enc_mn = [&](int32_t slot, const void* p, int64_t inner, int64_t rows, int64_t cnt,
                       int64_t ld) -> smuon_status {
       if (slot < 0) return SMUON_OK;
-      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, 64, bk);
+      return encode_bf16_3d(&B->maps[slot], p, inner, rows, cnt, ld, 64, 64);
     };
     smuon_status st;
     const int64_t zc = (int64_t)g.count * parts;  // matrices in the map: hi parts, then lo parts

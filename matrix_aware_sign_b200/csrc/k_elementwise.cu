@@ -699,6 +699,15 @@ __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
   }
 }
 
+__device__ __forceinline__ void unpack_bf16x8_ew(const uint4 w, float* o) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    o[2 * k] = __uint_as_float(u[k] << 16);
+    o[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+  }
+}
+
 // Vote and update from the workers' 1-bit messages (SignMuon summary, flow steps 3-4, all-gather
 // variant): the message words of a Newton-Schulz call with a BITS output or of an all-gather. One
 // lane per packed word, i.e. 32 consecutive entries: the M words (M/8 bytes per entry) are added
@@ -724,6 +733,17 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
     const int64_t w = gw - (L.chunk_begin >> 2);
     const int64_t e0 = 32 * w;
     if (!(active && e0 < L.n)) continue;
+    const int nent = (int)min((int64_t)32, L.n - e0);
+    const bool fast = L.vec && nent == 32;
+    const bool wbf = L.w_dtype == SMUON_BF16;
+    // bf16 W: its 32 entries (64 bytes) are requested first, raw, so that their latency overlaps the
+    // message words' instead of following it (f32 W is loaded after the count: fewer live registers)
+    uint4 wr[4];
+    if (kHasW && fast && wbf) {
+      const uint4* wp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(L.w) + e0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) wr[q] = wp[q];
+    }
     uint32_t c[7] = {0u, 0u, 0u, 0u, 0u, 0u, 0u};  // counts up to 64 need 7 planes
     for (int wk0 = 0; wk0 < M; wk0 += 8) {
       uint32_t x[8];
@@ -753,13 +773,15 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
     }
     const uint32_t pos = gt, tie = eq & even;
     const float up = tb.eta, down = -tb.eta, tied = tb.eta * (float)tb.tie;
-    const int nent = (int)min((int64_t)32, L.n - e0);
-    if (L.vec && nent == 32) {
+    if (fast) {
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         float wv[8];
         int8_t v8[8];
-        if (kHasW) load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
+        if (kHasW) {
+          if (wbf) unpack_bf16x8_ew(wr[g], wv);
+          else load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
+        }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int j = 8 * g + k;
@@ -796,7 +818,7 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
 }
 
 template <bool kHasW>
-__global__ void __launch_bounds__(256, 4) k_vote_update_bits(const __grid_constant__ EwTable tb) {
+__global__ void __launch_bounds__(256, 3) k_vote_update_bits(const __grid_constant__ EwTable tb) {
   vote_update_bits<kHasW>(tb);
 }
 
@@ -826,9 +848,9 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
   const int64_t want16 = (tb.total_chunks + 511) / 512;
   const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
   const bool has_w = tb.layers[0].w != nullptr;  // all layers or none (signs and votes only)
-  if (tb.src_dtype == SMUON_BITS) {  // one lane per packed word, four resident CTAs per SM, one wave
+  if (tb.src_dtype == SMUON_BITS) {  // one lane per packed word, three resident CTAs per SM, one wave
     const int64_t want = (tb.total_chunks / 4 + 255) / 256;
-    const int gridb = (int)std::max<int64_t>(1, std::min<int64_t>(want, 4 * sms));
+    const int gridb = (int)std::max<int64_t>(1, std::min<int64_t>(want, 3 * sms));
     if (has_w) k_vote_update_bits<true><<<gridb, 256, 0, s>>>(tb);
     else k_vote_update_bits<false><<<gridb, 256, 0, s>>>(tb);
     return cudaGetLastError();

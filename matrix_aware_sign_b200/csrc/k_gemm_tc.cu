@@ -6,11 +6,11 @@
 //   warp 0      TMA producer: 128B-swizzled tiles of A (K-major) and B
 //               (K-major, or MN-major for the X / Q right operand) into a
 //               shared-memory ring (full/empty mbarriers): 4 stages of
-//               128 x 64 + 256 x 64 bf16 in plain mode, 3 stages of hi and
-//               lo parts of 128 x 64 + 128 x 64 in split mode
+//               128 x 64 + 256 x 64 bf16 in plain mode, 2 stages of hi and
+//               lo parts of 128 x 64 + 256 x 64 in split mode
 //   warp 1      TMEM allocation and the single MMA-issuing thread:
 //               tcgen05.mma.cta_group::1.kind::f16, BF16 x BF16 -> FP32,
-//               M = 128, N = BN (256 plain, 128 split), K = 16 per
+//               M = 128, N = BN = 256, K = 16 per
 //               instruction (three per step in split mode: hi*hi, hi*lo,
 //               lo*hi), into one of two TMEM accumulators of BN columns
 //   warps 2-9   epilogue, two warps per TMEM lane group (one per half of the
@@ -31,18 +31,18 @@ constexpr int SRC_BYTES = BM * 32 * 4;      // one 128 x 32 f32 chunk of X (or i
 
 // plain BF16: one hi tile per operand; split BF16: hi and lo tiles per operand
 // (x = x_hi + x_lo, product ~ A_hi B_hi + A_hi B_lo + A_lo B_hi).
-// kBN = 128 in split mode, 256 in plain mode (the symmetric stages then use
-// 128 x 256 tiles over the triangle, the others a full grid). The ring takes
-// 192 KB of shared memory, or about 144 KB (kShallow) for stages whose K is
-// short: a tile then needs few k-blocks in flight, and the shared memory left
-// to the L1 cache serves the epilogue's row-per-lane global accesses.
-// k-block depth: 64 (128-byte swizzled K-major rows), or for the split stages kSplitBK (32: 64-byte
-// swizzled K-major rows, so that four ring stages of 128 x 256 split tiles fit)
+// Tiles are 128 x 256 (kBN = 256; the symmetric stages use them over the
+// triangle, the others a full grid). The ring takes 192 KB of shared memory,
+// or about 144 KB (kShallow, plain mode) for stages whose K is short: a tile
+// then needs few k-blocks in flight, and the shared memory left to the L1
+// cache serves the epilogue's row-per-lane global accesses. Split mode keeps
+// the 192 KB ring (two stages of 96 KB).
+// k-blocks are 64 deep: K-major rows of 64 bf16 (128 bytes) with the 128-byte swizzle
 template <bool kSplit, int kBN, bool kShallow, bool kSrc>
 struct Cfg {
   static constexpr int PARTS = kSplit ? 2 : 1;
   static constexpr int BN = kBN;
-  static constexpr int BK = kSplit ? kSplitBK : 64;
+  static constexpr int BK = 64;
   static constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x BK)
   static constexpr int B_BYTES = kBN * BK * 2;
   static constexpr int MN_BOX = 64 * BK * 2;     // one {64, BK} box of an MN-major B operand
@@ -54,9 +54,6 @@ struct Cfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SRC_RING + 1024 /*align*/ + 256 /*barriers*/;
 };
 constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz: the exit drains' budget
-#ifndef SMUON_AXPY_PREFETCH
-#define SMUON_AXPY_PREFETCH 0
-#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -117,22 +114,8 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
   d |= (uint64_t)2 << 61;            // SWIZZLE_128B
   return d;
 }
-// K-major rows of 32 bf16 (64 bytes) with the 64-byte swizzle: 8-row groups of 512 bytes
-__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-  d |= (uint64_t)(16 >> 4) << 16;
-  d |= (uint64_t)(512 >> 4) << 32;   // 8-row group stride
-  d |= (uint64_t)1 << 46;            // descriptor version for sm_100
-  d |= (uint64_t)4 << 61;            // SWIZZLE_64B
-  return d;
-}
-// K-major descriptor of a BK-deep tile at k-step kk (16 elements = 32 bytes into each row)
-template <int kBK>
-__device__ __forceinline__ uint64_t desc_k(uint32_t saddr, int kk) {
-  if constexpr (kBK == 64) return desc_sw128(saddr + kk * 32, 16);
-  else return desc_sw64(saddr + kk * 32);
-}
+// K-major descriptor of a 64-deep tile at k-step kk (16 elements = 32 bytes into each 128-byte row)
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr, int kk) { return desc_sw128(saddr + kk * 32, 16); }
 
 // instruction descriptor: BF16 x BF16 -> F32, A K-major, B K- or MN-major, 128 x n
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn, int n) {
@@ -361,13 +344,13 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + PARTS * A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = desc_k<BK>(sa, kk);
-            const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, C::MN_BOX) : desc_k<BK>(sb, kk);
+            const uint64_t ad = desc_k(sa, kk);
+            const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, C::MN_BOX) : desc_k(sb, kk);
             mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
             if (kSplit && use_lo) {
-              const uint64_t adl = desc_k<BK>(sa + A_BYTES, kk);
+              const uint64_t adl = desc_k(sa + A_BYTES, kk);
               const uint32_t sbl = sb + B_BYTES;
-              const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, C::MN_BOX) : desc_k<BK>(sbl, kk);
+              const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, C::MN_BOX) : desc_k(sbl, kk);
               mma_bf16(d_tmem, ad, bdl, idesc, 1u);   // A_hi * B_lo
               mma_bf16(d_tmem, adl, bd, idesc, 1u);   // A_lo * B_hi
             }
@@ -491,20 +474,6 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       int tm, tn;
       TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
       const int row = tm * BM + ew * 32 + lane;
-#if SMUON_AXPY_PREFETCH
-      // the first step's B X epilogue reads its a X term row by row from the caller's f32 momentum: ask L1
-      // for each chunk's 128 bytes one chunk ahead, the first before the accumulator is ready
-      const bool pf = stage == ST_AXPY && iter == 0 && !t.md->tall && t.md->m_dtype == SMUON_F32 && row < t.Mo;
-      const float* pf_row = pf ? reinterpret_cast<const float*>(t.md->m_ptr) + (int64_t)row * t.md->m_ld : nullptr;
-      auto prefetch_chunk = [&](int ch) {
-        const int col = tn * kBN + ch * 32;
-        if (pf && col < t.No) {
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(pf_row + col));
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(pf_row + min(col + 31, t.No - 1)));
-        }
-      };
-      prefetch_chunk(half * CH);
-#endif
       if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag, budget)) {
         *abort_flag = 1;
         if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
@@ -514,9 +483,6 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       float pacc = 0.f;
 #pragma unroll 1
       for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
-#if SMUON_AXPY_PREFETCH
-        if (ch + 1 < (half + 1) * CH) prefetch_chunk(ch + 1);
-#endif
         float v[32];
         tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
         epi_chunk<32>(t, row, tn * kBN + ch * 32, v, &pacc);

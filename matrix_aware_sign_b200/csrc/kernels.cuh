@@ -92,14 +92,9 @@ cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, i
                            const int32_t* skip, int num_sms, cudaStream_t s);
 constexpr int kProbeSlots = 8;  // residual partial sums per probe tile (one per epilogue warp)
 constexpr int kTcBM = 128;
-#ifndef SMUON_SPLIT_BN
-#define SMUON_SPLIT_BN 128
-#endif
-constexpr int kSplitBN = SMUON_SPLIT_BN;  // tile width of the split-BF16 stages (128: three ring stages of 64 KB)
-#ifndef SMUON_SPLIT_BK
-#define SMUON_SPLIT_BK 64
-#endif
-constexpr int kSplitBK = SMUON_SPLIT_BK;  // k-block depth of the split-BF16 stages (64, or 32 with 64-byte swizzle)
+// tile width of the split-BF16 stages: 128 x 256 tiles with two 96 KB ring stages (hi and lo parts of both
+// operands) beat 128 x 128 tiles with three of 64 KB (4096^2, five quintic steps: 3.69 against 4.24 ms)
+constexpr int kSplitBN = 256;
 int tc_tile_n(int stage, uint32_t flags);  // 128 (symmetric stages, split mode) or 256
 constexpr int kSimtBM = 64;
 constexpr int kSimtBN = 64;

@@ -213,8 +213,9 @@ def test_lionmuon_gpt2_large_sampled():
     Wd = [w.clone() for w in W0]
     mom = [[torch.zeros(s, device="cuda") for _ in range(M)] for s in shapes]
     G = [[torch.empty(s, device="cuda") for _ in range(M)] for s in shapes]
+    flags = S.NS_SPLIT_BF16 | S.ns_plain_lead(2)  # the bench's configuration
     opt = S.LionMuon(Wd, mom)
-    ws = S.workspace(opt.workspace_bytes(cfg.iters, S.NS_SPLIT_BF16))
+    ws = S.workspace(opt.workspace_bytes(cfg.iters, flags))
     rng = np.random.default_rng(0)
     samples = {l: rng.integers(0, shapes[l][0] * shapes[l][1], 2000) for l in (0, 1, 2, 3, 77, 143)}
     W_s = {l: host(W0[l]).reshape(-1)[idx] for l, idx in samples.items()}
@@ -233,7 +234,7 @@ def test_lionmuon_gpt2_large_sampled():
         G_s = {l: [G[l][k].view(-1)[torch.from_numpy(idx).cuda()].cpu().numpy() for k in range(M)]
                for l, idx in samples.items()}
         S.lionmuon_step(opt, G, cfg.period, cfg.beta1, cfg.beta2, cfg.eta, *cfg.coeffs, cfg.iters,
-                        tie_value=cfg.tie_value, ns_flags=S.NS_SPLIT_BF16, ws=ws)
+                        tie_value=cfg.tie_value, ns_flags=flags, ws=ws)
         torch.cuda.synchronize()
         muon = t % cfg.period == 0
         for l, idx in samples.items():
@@ -258,7 +259,7 @@ def test_lionmuon_gpt2_large_sampled():
         smom = [[dev(x) for x in M_l]]
         sopt = S.LionMuon(shadow, smom, t=3)
         S.lionmuon_step(sopt, [[dev(g) for g in G_l]], cfg.period, cfg.beta1, cfg.beta2, cfg.eta, *cfg.coeffs,
-                        cfg.iters, tie_value=cfg.tie_value, ns_flags=S.NS_SPLIT_BF16)
+                        cfg.iters, tie_value=cfg.tie_value, ns_flags=flags)
         torch.cuda.synchronize()
         d_gpu = -host(shadow[0]).astype(np.float64) / np.float32(cfg.eta)
         gh = [O.lion_interpolate(M_l[k], G_l[k], cfg.beta1) for k in range(M)]
