@@ -699,24 +699,16 @@ __device__ __forceinline__ void vote_update_body(const EwTable& tb) {
   }
 }
 
-__device__ __forceinline__ void unpack_bf16x8_ew(const uint4 w, float* o) {
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    o[2 * k] = __uint_as_float(u[k] << 16);
-    o[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
-  }
-}
-
 // Vote and update from the workers' 1-bit messages (SignMuon summary, flow steps 3-4, all-gather
 // variant): the message words of a Newton-Schulz call with a BITS output or of an all-gather. One
 // lane per packed word, i.e. 32 consecutive entries: the M words (M/8 bytes per entry) are added
-// bit-sliced -- plane p holds bit p of every entry's count of set bits -- by a ripple of half adders
-// per worker, and the counts are compared with h = floor(M/2) plane by plane from the top:
+// bit-sliced -- plane p holds bit p of every entry's count of set bits, as many planes as M needs --
+// by a ripple of half adders per worker, and the counts are compared with h = floor(M/2) plane by
+// plane from the top:
 // count > h is the +1 vote (2*count > M), count == h with M even the tie, the rest -1. Bits past a
 // layer's last entry are zero and are never applied. Layer chunk ranges are multiples of 16 chunks
 // (4 words), so global word g is chunk 4g.
-template <bool kHasW>
+template <bool kHasW, int kPlanes>
 __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -735,16 +727,9 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
     if (!(active && e0 < L.n)) continue;
     const int nent = (int)min((int64_t)32, L.n - e0);
     const bool fast = L.vec && nent == 32;
-    const bool wbf = L.w_dtype == SMUON_BF16;
-    // bf16 W: its 32 entries (64 bytes) are requested first, raw, so that their latency overlaps the
-    // message words' instead of following it (f32 W is loaded after the count: fewer live registers)
-    uint4 wr[4];
-    if (kHasW && fast && wbf) {
-      const uint4* wp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(L.w) + e0);
+    uint32_t c[kPlanes];  // counts up to M need kPlanes planes (4 for M <= 15, 7 for M <= 64)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) wr[q] = wp[q];
-    }
-    uint32_t c[7] = {0u, 0u, 0u, 0u, 0u, 0u, 0u};  // counts up to 64 need 7 planes
+    for (int p = 0; p < kPlanes; ++p) c[p] = 0u;
     for (int wk0 = 0; wk0 < M; wk0 += 8) {
       uint32_t x[8];
 #pragma unroll
@@ -754,7 +739,7 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
       for (int j = 0; j < 8; ++j) {
         uint32_t carry = x[j];
 #pragma unroll
-        for (int p = 0; p < 7; ++p) {
+        for (int p = 0; p < kPlanes; ++p) {
           const uint32_t t = c[p] & carry;
           c[p] ^= carry;
           carry = t;
@@ -763,7 +748,7 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
     }
     uint32_t gt = 0u, eq = 0xffffffffu;
 #pragma unroll
-    for (int p = 6; p >= 0; --p) {
+    for (int p = kPlanes - 1; p >= 0; --p) {
       if ((h >> p) & 1) {
         eq &= c[p];
       } else {
@@ -778,19 +763,17 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
       for (int g = 0; g < 4; ++g) {
         float wv[8];
         int8_t v8[8];
+        if (kHasW) load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
+        const uint32_t pb = pos >> (8 * g), tbits = tie >> (8 * g);
         if (kHasW) {
-          if (wbf) unpack_bf16x8_ew(wr[g], wv);
-          else load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
-        }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int j = 8 * g + k;
-          const bool p1 = (pos >> j) & 1u, t1 = (tie >> j) & 1u;
-          v8[k] = (int8_t)(p1 ? 1 : (t1 ? tb.tie : -1));
-          wv[k] = __fsub_rn(wv[k], p1 ? up : (t1 ? tied : down));
+          for (int k = 0; k < 8; ++k)
+            wv[k] = __fsub_rn(wv[k], ((pb >> k) & 1u) ? up : (((tbits >> k) & 1u) ? tied : down));
+          store8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
         }
-        if (kHasW) store8(L.w, L.w_ld, L.w_dtype, L, e0 + 8 * g, 1, wv);
         if (L.vote_out) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v8[k] = (int8_t)(((pb >> k) & 1u) ? 1 : (((tbits >> k) & 1u) ? tb.tie : -1));
           int8_t* dst = L.vote_out + e0 + 8 * g;
           if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
             uint2 pk;
@@ -817,9 +800,15 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
   }
 }
 
-template <bool kHasW>
-__global__ void __launch_bounds__(256, 3) k_vote_update_bits(const __grid_constant__ EwTable tb) {
-  vote_update_bits<kHasW>(tb);
+template <bool kHasW, int kPlanes>
+__global__ void __launch_bounds__(256, 4) k_vote_update_bits(const __grid_constant__ EwTable tb) {
+  vote_update_bits<kHasW, kPlanes>(tb);
+}
+
+template <int kPlanes>
+static void launch_bits(const EwTable& tb, bool has_w, int grid, cudaStream_t s) {
+  if (has_w) k_vote_update_bits<true, kPlanes><<<grid, 256, 0, s>>>(tb);
+  else k_vote_update_bits<false, kPlanes><<<grid, 256, 0, s>>>(tb);
 }
 
 template <bool kPopcount, bool kBf16, typename MaskT>
@@ -848,11 +837,12 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
   const int64_t want16 = (tb.total_chunks + 511) / 512;
   const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
   const bool has_w = tb.layers[0].w != nullptr;  // all layers or none (signs and votes only)
-  if (tb.src_dtype == SMUON_BITS) {  // one lane per packed word, three resident CTAs per SM, one wave
+  if (tb.src_dtype == SMUON_BITS) {  // one lane per packed word, four resident CTAs per SM, one wave
     const int64_t want = (tb.total_chunks / 4 + 255) / 256;
-    const int gridb = (int)std::max<int64_t>(1, std::min<int64_t>(want, 3 * sms));
-    if (has_w) k_vote_update_bits<true><<<gridb, 256, 0, s>>>(tb);
-    else k_vote_update_bits<false><<<gridb, 256, 0, s>>>(tb);
+    const int gridb = (int)std::max<int64_t>(1, std::min<int64_t>(want, 4 * sms));
+    if (tb.M <= 15) launch_bits<4>(tb, has_w, gridb, s);
+    else if (tb.M <= 31) launch_bits<5>(tb, has_w, gridb, s);
+    else launch_bits<7>(tb, has_w, gridb, s);
     return cudaGetLastError();
   }
   if (tb.src_dtype == SMUON_I8) {  // sign matrices: both vote kinds count the same positives

@@ -349,6 +349,20 @@ def test_ns_spectral_rank_two_closed_form():
         assert rel_fro(host(Uf[0]), want) > 0.02
 
 
+def test_ns_spectral_scaling_nearly_equal_top_pair():
+    """The two largest singular values 1 and 1 - 1e-5 over a spread tail: the
+    Lanczos run may settle on either of the pair, and either gives the SVD
+    scaling to within 1e-5, so the FP32 mode stays within its 1e-4."""
+    rng = np.random.default_rng(8)
+    m, n = 160, 480
+    Uo, _ = np.linalg.qr(rng.standard_normal((m, m)))
+    Vo, _ = np.linalg.qr(rng.standard_normal((n, m)))
+    sv = np.concatenate([[1.0, 1.0 - 1e-5], np.linspace(0.9, 0.05, m - 2)])
+    M = ((Uo * sv) @ Vo.T).astype(np.float32)
+    _, Ud = _ns_run([M], WL.QUINTIC, 1, S.NS_FP32_REF | S.NS_SPECTRAL)
+    check_ns_outputs([(host(Ud[0]), O.newton_schulz(M, *WL.QUINTIC, 1, spectral=True))], 1e-4)
+
+
 I8_OUT_CASES = [
     ((256, 1024), WL.QUINTIC, 1, 0),
     ((1024, 256), WL.QUINTIC, 1, 0),
