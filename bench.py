@@ -76,6 +76,10 @@ def parse_args(argv=None):
     p.add_argument("--plain-lead", type=int, default=None,
                    help="split mode: run this many leading Newton-Schulz steps with plain BF16 operands "
                         "(SMUON_NS_PLAIN_LEAD; default 2; matrices with a smaller side under 512 take one)")
+    p.add_argument("--one-sm", action="store_true",
+                   help="tensor-core stages on single-SM 128x256 tiles (SMUON_NS_ONE_SM) instead of the SM pairs "
+                        "(256x256 tiles over clusters of two CTAs) that batches of matrices with a smaller side "
+                        ">= 256 use by default")
     p.add_argument("--grad-source", choices=["hbm", "counter"], default="hbm",
                    help="LionMuon set: read a resident 45 GB gradient set (default), or draw the workers' "
                         "gradients inside the kernels from the counter-based streams (no gradient bytes, more ALU)")
@@ -883,6 +887,8 @@ def ns_flags_for(S, name, args):
         flags |= S.ns_plain_lead(lead)
     if args.spectral and name not in WL.LION_MUON_WORKLOADS:
         flags |= S.NS_SPECTRAL
+    if args.one_sm:
+        flags |= S.NS_ONE_SM
     return mode, flags, lead if mode == "split" else 0
 
 
@@ -1102,6 +1108,8 @@ def main():
         flags = S.NS_SPLIT_BF16 if (args.ns_mode or "split") == "split" else 0
         if flags and args.plain_lead:
             flags |= S.ns_plain_lead(args.plain_lead)
+        if args.one_sm:
+            flags |= S.NS_ONE_SM
         print(json.dumps({"ns_4096sq_quintic5": measure_ns_square(S, torch, peaks, 4096, 5, flags,
                                                                    reps=args.steps)}))
         return
@@ -1167,8 +1175,11 @@ def main():
             "split_bf16_plain_lead2": measure_ns_square(S, torch, peaks, 4096, 5,
                                                         S.NS_SPLIT_BF16 | S.ns_plain_lead(2)),
             "plain_bf16": measure_ns_square(S, torch, peaks, 4096, 5, 0),
+            "split_bf16_plain_lead2_one_sm": measure_ns_square(S, torch, peaks, 4096, 5,
+                                                               S.NS_SPLIT_BF16 | S.ns_plain_lead(2) | S.NS_ONE_SM),
             "note": "timed alone: compared with the burst peak; plain BF16 misses the sign criterion at five "
-                    "quintic steps, split BF16 (also with two plain leading steps) meets it"}
+                    "quintic steps, split BF16 (also with two plain leading steps) meets it; SM pairs "
+                    "(256x256 tiles) unless the key says one_sm (128x256 tiles on single SMs)"}
     sampler.stop()
 
     if rank == 0:

@@ -24,6 +24,7 @@ NS_FP32_REF, NS_SPLIT_BF16, NS_NO_NORMALIZE, NS_EMIT_Q, NS_SIMT_BF16 = 1, 2, 4, 
 NS_GRAM_ONLY = 32  # CacheMuon fresh solve iterated on the m x m Gram (with NS_EMIT_Q, one matrix)
 NS_SPECTRAL = 64  # spectral-norm normalisation X_0 = M / (||M||_2 + eps) (Lanczos estimate on the device)
 NS_TEST_WAIT_EXPIRY = 0x8000  # failure-detection test: the tensor-core stages' pipeline waits run out
+NS_ONE_SM = 0x80  # tensor-core stages on single-SM 128 x 256 tiles instead of SM pairs (256 x 256 tiles)
 
 
 def ns_plain_lead(k: int) -> int:

@@ -260,7 +260,7 @@ Mode pick_mode(uint32_t flags) {
 // epilogue-bound, so a count-balanced order does better than the cost model.
 bool lpt_stage(int st) { return st == ST_GRAM || st == ST_PROBE; }
 
-void schedule_stage(const std::vector<GroupDesc>& groups, int st, int total, int ctas, int bn, bool split,
+void schedule_stage(const std::vector<GroupDesc>& groups, int st, int total, int ctas, int bm, int bn, bool split,
                     int32_t* ids, int32_t* begin) {
   std::vector<std::vector<int32_t>> per(ctas);
   if (!lpt_stage(st)) {
@@ -269,12 +269,13 @@ void schedule_stage(const std::vector<GroupDesc>& groups, int st, int total, int
     std::vector<std::pair<double, int32_t>> cost_tile;  // (cost, tile)
     cost_tile.reserve(total);
     for (const GroupDesc& g : groups) {
-      const int tiles = sym_stage(st) ? sym_start(g.tiles_m[st], g.tiles_n[st], bn / kTcBM)
+      const int tiles = sym_stage(st) ? sym_start(g.tiles_m[st], g.tiles_n[st], bn / bm)
                                       : g.tiles_m[st] * g.tiles_n[st];
       const int K = (st == ST_GRAM || st == ST_PROBE) ? g.n : g.m;
       const int No = wide_out_stage(st) ? g.n : g.m;
+      // per SM: a pair's SMs each take a 128-row half of the 256 x 256 tile
       const double kb = (double)((K + 63) / 64) * (split && split_stage(st) ? 3 : 1) * bn / 256.0;
-      const double fill = (double)g.m * No / ((double)g.tiles_m[st] * kTcBM * g.tiles_n[st] * bn);
+      const double fill = (double)g.m * No / ((double)g.tiles_m[st] * bm * g.tiles_n[st] * bn);
       const double cost = kb + 8.0 * fill * bn / 256.0;
       for (int t = g.tile_begin[st]; t < g.tile_begin[st] + g.count * tiles; ++t) cost_tile.push_back({cost, t});
     }
@@ -375,19 +376,27 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     if (spectral) lz_floats += (int64_t)(kLanczosSteps + 2) * lz_stride(B->groups[d.group].m);
   }
 
+  // SM pairs (256 x 256 tiles over clusters of two CTAs) for the plain Newton-Schulz chain (Gram, A^2,
+  // B X) when no matrix is too small for a 256-row tile; decided from the flags and shapes alone, so the
+  // sizing pass and the filling pass lay the workspace out alike
+  bool pair = tc && !rq.probe && !emit_q && !gram_only && !(rq.flags & SMUON_NS_ONE_SM);
+  for (const auto& g : B->groups)
+    if (g.m < kPairMinM) pair = false;
+  const int TBM = pair ? 2 * kTcBM : BM;  // tile height of the tables
+
   // tile tables: for the symmetric stages the tiles that reach the diagonal or
-  // lie above it (BN = ratio * BM), a full grid of BM x BN tiles otherwise
+  // lie above it (BN = ratio * TBM), a full grid of TBM x BN tiles otherwise
   int totals[ST_COUNT] = {0};
   int ratios[ST_COUNT] = {0};
   for (int st = 0; st < ST_COUNT; ++st) {
     const int BN = tc ? tc_tile_n(st, rq.flags) : kSimtBN;
-    ratios[st] = BN / BM;
+    ratios[st] = BN / TBM;
   }
   for (auto& g : B->groups) {
-    const int tmm = ceil_div(g.m, BM);
+    const int tmm = ceil_div(g.m, TBM);
     for (int st = 0; st < ST_COUNT; ++st) {
       const bool sym = sym_stage(st);
-      const int BN = BM * ratios[st];
+      const int BN = TBM * ratios[st];
       const int No = wide_out_stage(st) ? g.n : g.m;
       g.tiles_m[st] = tmm;
       g.tiles_n[st] = ceil_div(No, BN);
@@ -440,7 +449,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     if (axpy_tma && bf && K >= 3) want_map(g.tm_xf[0]);
     g.tm_a_k = g.tm_b_k = g.tm_uq_k = g.tm_a_kw = g.tm_t_k = g.tm_t_kw = -1;
     if (!tc) continue;
-    const bool wide = tc_tile_n(ST_GRAM, rq.flags) == 256;
+    const bool wide = !pair && tc_tile_n(ST_GRAM, rq.flags) == 256;  // a pair's CTAs stage 128-row B halves
     if (!rq.probe) {
       want_map(g.tm_x_k[0]);
       want_map(g.tm_x_mn[0]);
@@ -529,7 +538,8 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   // budget that runs out while the producer issues nothing
   h.wait_cycles = (rq.flags & SMUON_NS_TEST_WAIT_EXPIRY) ? (1ull << 16) : (1ull << 32);
   h.starve_tc = (rq.flags & SMUON_NS_TEST_WAIT_EXPIRY) ? 1 : 0;
-  h.tile_bm = BM; h.tile_bn = tc ? tc_tile_n(ST_AXPY, rq.flags) : kSimtBN;
+  h.tile_bm = TBM; h.tile_bn = tc ? tc_tile_n(ST_AXPY, rq.flags) : kSimtBN;
+  h.pair = pair ? 1 : 0;
   for (int st = 0; st < ST_COUNT; ++st) {
     h.total_tiles[st] = totals[st];
     h.sym_ratio[st] = ratios[st];
@@ -568,12 +578,15 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     smuon_status dst = device_info(&di);
     if (dst != SMUON_OK) return dst;
     const bool split = (rq.flags & SMUON_NS_SPLIT_BF16) != 0 && parts == 2;
+    // one tile list per CTA, or per pair of SMs that the device holds at once
+    const int lists = pair ? tc_pair_clusters() : di.sms;
+    if (lists <= 0) return fail(SMUON_ERR_CUDA, "the device holds no cluster of the SM-pair GEMM kernel");
     for (int st = 0; st < ST_COUNT; ++st) {
       if (totals[st] == 0) continue;
-      const int ctas = std::min(std::min(totals[st], di.sms), kMaxSchedCtas);
+      const int ctas = std::min(std::min(totals[st], lists), kMaxSchedCtas);
       h.sched_ctas[st] = ctas;
-      schedule_stage(B->groups, st, totals[st], ctas, BM * ratios[st], split, B->sched.data() + sched_off[st],
-                     B->sched_begin.data() + sched_boff[st]);
+      schedule_stage(B->groups, st, totals[st], ctas, TBM, TBM * ratios[st], split,
+                     B->sched.data() + sched_off[st], B->sched_begin.data() + sched_boff[st]);
     }
   }
 
@@ -682,7 +695,7 @@ double stage_flops(const Builder& B, int st) {
 double stage_issued(const Builder& B, int st, int iter = 1 << 20) {
   const PlanHeader& h = B.h;
   const bool tc = h.mode == MODE_TC_BF16;
-  const int BM = tc ? kTcBM : kSimtBM, BK = tc ? 64 : 16;
+  const int BM = tc ? h.tile_bm : kSimtBM, BK = tc ? 64 : 16;
   const bool split = tc && (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
   double f = 0;
   for (const GroupDesc& g : B.groups) {
@@ -722,9 +735,13 @@ smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int it
       {"k_gemm_tc_split.gram", "k_gemm_tc_split.poly", "k_gemm_tc_split.axpy", "k_gemm_tc_split.qaxpy",
        "k_gemm_tc_split.reuse", "k_gemm_tc_split.probe", "k_gemm_tc_split.aa1", "k_gemm_tc_split.aa2",
        "k_gemm_tc_split.qx"}};
+  // SM pairs: only the plain Newton-Schulz chain's stages
+  static const char* tc2_names[2][3] = {{"k_gemm_tc2.gram", "k_gemm_tc2.poly", "k_gemm_tc2.axpy"},
+                                        {"k_gemm_tc2_split.gram", "k_gemm_tc2_split.poly", "k_gemm_tc2_split.axpy"}};
   if (h.mode == MODE_TC_BF16) {
     const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
-    Launch L(tc_names[split][st], SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
+    const char* name = (h.pair && st <= ST_AXPY) ? tc2_names[split][st] : tc_names[split][st];
+    Launch L(name, SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
     CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
   } else {
     const int grid = std::min(total, di.sms * 6);
@@ -743,7 +760,8 @@ smuon_status validate_ns(const NsRequest& rq) {
   if (rq.iters < 1 || rq.iters > 64) return fail(SMUON_ERR_INVALID_ARG, "iters=%d must be in 1..64", rq.iters);
   const uint32_t known =
       SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_NO_NORMALIZE | SMUON_NS_EMIT_Q | SMUON_NS_SIMT_BF16 |
-      SMUON_NS_GRAM_ONLY | SMUON_NS_SPECTRAL | SMUON_NS_PLAIN_LEAD_MASK | SMUON_NS_TEST_WAIT_EXPIRY;
+      SMUON_NS_GRAM_ONLY | SMUON_NS_SPECTRAL | SMUON_NS_PLAIN_LEAD_MASK | SMUON_NS_TEST_WAIT_EXPIRY |
+      SMUON_NS_ONE_SM;
   if (rq.flags & ~known) return fail(SMUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", rq.flags & ~known);
   const uint32_t modes = rq.flags & (SMUON_NS_FP32_REF | SMUON_NS_SPLIT_BF16 | SMUON_NS_SIMT_BF16);
   if (modes & (modes - 1))

@@ -19,6 +19,16 @@
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
 // i+1. Every mbarrier wait is bounded; on expiry the CTA records
 // SMUON_DEV_WAIT_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
+//
+// SM pairs (k_gemm_tc2, clusters of two CTAs): one 256 x 256 tile per pair,
+// tcgen05.mma.cta_group::2 with M = 256 issued by the even CTA. Each CTA
+// stages its own 128 rows of A and its own 128-row half of the B tile (by
+// TMA, the copies of both CTAs completing on the even CTA's full barrier) and
+// holds its 128 x 256 half of the accumulator in its own TMEM; the MMA
+// commits arrive on both CTAs' barriers, and both CTAs' epilogue warps
+// release an accumulator at the even CTA. Per SM this halves the shared-
+// memory operand traffic of a 256-wide tile (each SM reads A once and half of
+// B), the limit of the single-SM 128 x 256 form.
 #include "epilogue.cuh"
 
 namespace smuon {
@@ -38,13 +48,14 @@ constexpr int SRC_BYTES = BM * 32 * 4;      // one 128 x 32 f32 chunk of X (or i
 // cache serves the epilogue's row-per-lane global accesses. Split mode keeps
 // the 192 KB ring (two stages of 96 KB).
 // k-blocks are 64 deep: K-major rows of 64 bf16 (128 bytes) with the 128-byte swizzle
-template <bool kSplit, int kBN, bool kShallow, bool kSrc>
+template <bool kSplit, int kBN, bool kShallow, bool kSrc, bool kPair = false>
 struct Cfg {
   static constexpr int PARTS = kSplit ? 2 : 1;
   static constexpr int BN = kBN;
   static constexpr int BK = 64;
+  static constexpr int B_ROWS = kPair ? kBN / 2 : kBN;  // rows of the B tile this CTA stages
   static constexpr int A_BYTES = BM * BK * 2;   // one bf16 tile of A (128 rows x BK)
-  static constexpr int B_BYTES = kBN * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int MN_BOX = 64 * BK * 2;     // one {64, BK} box of an MN-major B operand
   static constexpr int STAGE_BYTES = PARTS * (A_BYTES + B_BYTES);
   static constexpr int STAGES = ((kShallow ? 144 : 192) * 1024) / STAGE_BYTES;
@@ -99,6 +110,35 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// SM-pair form: the copy lands in this CTA's shared memory and completes on the mbarrier at cluster
+// address bar_cluster (the even CTA's full barrier)
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar_cluster)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// cluster address of the same shared-memory location in the even CTA of the pair
+__device__ __forceinline__ uint32_t at_rank0(uint32_t saddr) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(saddr));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
 __device__ __forceinline__ void tensormap_acquire(const CUtensorMap* map) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(map))
                : "memory");
@@ -117,10 +157,11 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
 // K-major descriptor of a 64-deep tile at k-step kk (16 elements = 32 bytes into each 128-byte row)
 __device__ __forceinline__ uint64_t desc_k(uint32_t saddr, int kk) { return desc_sw128(saddr + kk * 32, 16); }
 
-// instruction descriptor: BF16 x BF16 -> F32, A K-major, B K- or MN-major, 128 x n
-__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn, int n) {
+// instruction descriptor: BF16 x BF16 -> F32, A K-major, B K- or MN-major, m x n (m = 128, or 256 for a
+// pair of SMs)
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn, int n, int m = BM) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(BM >> 4) << 24);
+         ((uint32_t)(m >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
@@ -133,6 +174,31 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
+}
+// SM pairs: the 256-row MMA (A rows and B columns from both CTAs, D in both TMEMs), and its commit,
+// which arrives on the barrier at the same offset in both CTAs
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  const uint16_t both = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      ::"r"(bar), "h"(both) : "memory");
+}
+template <bool kPair>
+__device__ __forceinline__ void mma_issue(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
+  if constexpr (kPair) mma_bf16_pair(d, a, b, idesc, accum);
+  else mma_bf16(d, a, b, idesc, accum);
+}
+template <bool kPair>
+__device__ __forceinline__ void commit_to(uint32_t bar) {
+  if constexpr (kPair) mma_commit_pair(bar);
+  else mma_commit(bar);
 }
 __device__ __forceinline__ void fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -179,12 +245,13 @@ struct TcOps {
   int b_mn;
 };
 
-__device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, int iter, int bn) {
+// brows: rows of the B tile one CTA stages (256 for a single-SM 128 x 256 tile, 128 for each CTA of a pair)
+__device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, int iter, int brows) {
   const GroupDesc& g = *t.g;
   TcOps o;
   o.za = o.zb = t.z;
   o.zlo = g.count;
-  const bool wide = bn == 256;  // K-major B tiles of 256 rows use the {64, 256} boxes
+  const bool wide = brows == 256;  // K-major B tiles of 256 rows use the {64, 256} boxes
   switch (t.stage) {
     case ST_GRAM:
       o.ma = &h.tmaps[g.tm_x_k[iter & 1]];
@@ -217,15 +284,16 @@ __device__ __forceinline__ TcOps tc_ops(const PlanHeader& h, const TileCtx& t, i
   return o;
 }
 
-template <bool kSplit, int kBN, bool kShallow, bool kSrc>
+template <bool kSplit, int kBN, bool kShallow, bool kSrc, bool kPair>
 __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int iter) {
-  using C = Cfg<kSplit, kBN, kShallow, kSrc>;
+  using C = Cfg<kSplit, kBN, kShallow, kSrc, kPair>;
   constexpr int STAGES = C::STAGES;
   constexpr int STAGE_BYTES = C::STAGE_BYTES;
   constexpr int PARTS = C::PARTS;
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int A_BYTES = C::A_BYTES;
   constexpr int BK = C::BK;
+  constexpr int B_ROWS = C::B_ROWS;
   const PlanHeader& h = plan->h;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -241,31 +309,53 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
 
+  // SM pairs: rank 0 issues the MMAs and owns the full and tempty barriers that count both CTAs
+  const uint32_t rank = kPair ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar + 8 * s, 1); mbar_init(empty_bar + 8 * s, 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar + 8 * a, 1); mbar_init(tempty_bar + 8 * a, 256); }
+    // tempty: every epilogue thread arrives (single SM), or one arrive per epilogue warp of both CTAs
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar + 8 * a, 1); mbar_init(tempty_bar + 8 * a, kPair ? 16 : 256); }
     mbar_init(done_bar, 1);
     for (int q = 0; q < SRC_SLOTS; ++q) { mbar_init(sfull_bar + 8 * q, 1); mbar_init(sempty_bar + 8 * q, 8); }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32((const void*)tmem_slot)),
-                 "r"(C::TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if constexpr (kPair) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32((const void*)tmem_slot)),
+                   "r"(C::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32((const void*)tmem_slot)),
+                   "r"(C::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   fence_before();
-  __syncthreads();
+  if constexpr (kPair) {
+    __syncwarp();
+    cluster_sync_all();  // both CTAs' barriers exist before either signals the other's
+  } else {
+    __syncthreads();
+  }
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // split mode: both parts of every operand, except in the plain leading steps (hi parts only); the
   // producer and the MMA issuer take the same decision, per tile, from the tile's group
   const unsigned long long budget = h.wait_cycles;
-  // this CTA's tiles (host-balanced list; every role walks the same one)
+  // this CTA's tiles (host-balanced list; every role walks the same one; both CTAs of a pair walk the
+  // pair's list, whose tiles are 256 rows high: this CTA takes rows 128 * (2 tm + rank) ...)
+  const int list = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int32_t* tiles = h.sched + h.sched_off[stage];
-  const int t_begin = h.sched_begin[h.sched_boff[stage] + blockIdx.x];
-  const int t_end = h.sched_begin[h.sched_boff[stage] + blockIdx.x + 1];
+  const int t_begin = h.sched_begin[h.sched_boff[stage] + list];
+  const int t_end = h.sched_begin[h.sched_boff[stage] + list + 1];
+  auto tile_at = [&](int i, int& tm, int& tn) {
+    const TileCtx t = make_ctx(h, stage, iter, tiles[i], tm, tn);
+    if (kPair) tm = 2 * tm + (int)rank;
+    return t;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer (lane 0)
@@ -274,31 +364,44 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
     uint32_t armed = 0, last_par = 0;  // per-stage bit sets for the exit drain
     bool ok = true;
     for (int i = t_begin; i < t_end && ok && !h.starve_tc; ++i) {
-      const int tile = tiles[i];
       int tm, tn;
-      const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+      const TileCtx t = tile_at(i, tm, tn);
       const int parts = (kSplit && !plain_lead_stage(h.flags, stage, iter, t.g->m)) ? PARTS : 1;
       if (lane == 0) {
-        const TcOps o = tc_ops(h, t, iter, kBN);
+        const TcOps o = tc_ops(h, t, iter, B_ROWS);
         tensormap_acquire(o.ma);
         tensormap_acquire(o.mb);
         const int nk = (o.K + BK - 1) / BK;
+        const int brow = tn * kBN + (int)rank * B_ROWS;  // first B row (K-major) or column (MN-major) staged here
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty_bar + 8 * s, ph ^ 1u, abort_flag, budget)) { ok = false; break; }
           const uint32_t fb = full_bar + 8 * s;
-          mbar_expect_tx(fb, parts * (A_BYTES + B_BYTES));
-          armed |= 1u << s;
-          last_par = (last_par & ~(1u << s)) | (ph << s);
+          const uint32_t fb_tx = kPair ? at_rank0(fb) : fb;
+          if (leader) {  // the pair's full barrier expects both CTAs' bytes
+            mbar_expect_tx(fb, (kPair ? 2 : 1) * parts * (A_BYTES + B_BYTES));
+            armed |= 1u << s;
+            last_par = (last_par & ~(1u << s)) | (ph << s);
+          }
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + PARTS * A_BYTES;
           for (int part = 0; part < parts; ++part) {
             const int za = o.za + part * o.zlo, zb = o.zb + part * o.zlo;
             const uint32_t da = sa + part * A_BYTES, db = sb + part * B_BYTES;
-            tma_load_3d(da, o.ma, kb * BK, tm * BM, za, fb);
-            if (o.b_mn) {
+            if constexpr (kPair) {
+              tma_load_3d_pair(da, o.ma, kb * BK, tm * BM, za, fb_tx);
+              if (o.b_mn) {
 #pragma unroll
-              for (int q = 0; q < kBN / 64; ++q) tma_load_3d(db + q * C::MN_BOX, o.mb, tn * kBN + 64 * q, kb * BK, zb, fb);
+                for (int q = 0; q < B_ROWS / 64; ++q) tma_load_3d_pair(db + q * C::MN_BOX, o.mb, brow + 64 * q, kb * BK, zb, fb_tx);
+              } else {
+                tma_load_3d_pair(db, o.mb, kb * BK, brow, zb, fb_tx);
+              }
             } else {
-              tma_load_3d(db, o.mb, kb * BK, tn * kBN, zb, fb);
+              tma_load_3d(da, o.ma, kb * BK, tm * BM, za, fb);
+              if (o.b_mn) {
+#pragma unroll
+                for (int q = 0; q < B_ROWS / 64; ++q) tma_load_3d(db + q * C::MN_BOX, o.mb, brow + 64 * q, kb * BK, zb, fb);
+              } else {
+                tma_load_3d(db, o.mb, kb * BK, brow, zb, fb);
+              }
             }
           }
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -311,7 +414,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         *abort_flag = 1;
         if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
       }
-      // drain: every armed stage's last phase must have landed before exit
+      // drain: every armed stage's last phase must have landed before exit (with SM pairs the even
+      // CTA's barriers count the copies of both CTAs, and the final cluster barrier holds the odd CTA)
       for (int q = 0; q < STAGES; ++q)
         if (armed & (1u << q)) {
           const uint32_t p = (last_par >> q) & 1u;
@@ -320,7 +424,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ---------------- MMA issuer
       int s = 0;
       uint32_t ph = 0;
@@ -328,11 +432,10 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       uint32_t acc_ph = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok; ++i) {
-        const int tile = tiles[i];
         int tm, tn;
-        const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
-        const TcOps o = tc_ops(h, t, iter, kBN);
-        const uint32_t idesc = make_idesc((uint32_t)o.b_mn, kBN);
+        const TileCtx t = tile_at(i, tm, tn);
+        const TcOps o = tc_ops(h, t, iter, B_ROWS);
+        const uint32_t idesc = make_idesc((uint32_t)o.b_mn, kBN, kPair ? 2 * BM : BM);
         const bool use_lo = kSplit && !plain_lead_stage(h.flags, stage, iter, t.g->m);
         if (!mbar_wait(tempty_bar + 8 * acc, acc_ph ^ 1u, abort_flag, budget)) { ok = false; break; }
         fence_after();
@@ -346,20 +449,20 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_k(sa, kk);
             const uint64_t bd = o.b_mn ? desc_sw128(sb + kk * 2048, C::MN_BOX) : desc_k(sb, kk);
-            mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            mma_issue<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0);
             if (kSplit && use_lo) {
               const uint64_t adl = desc_k(sa + A_BYTES, kk);
               const uint32_t sbl = sb + B_BYTES;
               const uint64_t bdl = o.b_mn ? desc_sw128(sbl + kk * 2048, C::MN_BOX) : desc_k(sbl, kk);
-              mma_bf16(d_tmem, ad, bdl, idesc, 1u);   // A_hi * B_lo
-              mma_bf16(d_tmem, adl, bd, idesc, 1u);   // A_lo * B_hi
+              mma_issue<kPair>(d_tmem, ad, bdl, idesc, 1u);   // A_hi * B_lo
+              mma_issue<kPair>(d_tmem, adl, bd, idesc, 1u);   // A_lo * B_hi
             }
           }
-          mma_commit(empty_bar + 8 * s);  // frees the smem slot once these MMAs have read it
+          commit_to<kPair>(empty_bar + 8 * s);  // frees the smem slot (of both CTAs) once these MMAs have read it
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(tfull_bar + 8 * acc);  // accumulator ready for the epilogue
+        commit_to<kPair>(tfull_bar + 8 * acc);  // accumulator ready for the epilogue(s)
         if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
       }
       if (!ok) {
@@ -367,7 +470,12 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
       }
       // all MMAs issued by this thread complete before TMEM is released
-      mma_commit(done_bar);
+      commit_to<kPair>(done_bar);
+      const unsigned long long t0 = clock64();
+      while (!mbar_try_wait(done_bar, 0) && clock64() - t0 < kWaitCycles) {}
+    } else if (kPair && lane == 0) {
+      // odd CTA of a pair: the even CTA's last commit also arrives here once its MMAs (which write this
+      // CTA's TMEM) are complete
       const unsigned long long t0 = clock64();
       while (!mbar_try_wait(done_bar, 0) && clock64() - t0 < kWaitCycles) {}
     }
@@ -379,9 +487,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       uint32_t armed = 0, last_par = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok && !h.starve_tc; ++i) {
-        const int tile = tiles[i];
         int tm, tn;
-        const TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+        const TileCtx t = tile_at(i, tm, tn);
         const bool first = iter == 0;
         const CUtensorMap* map = first ? &h.tmaps[t.md->tm_src] : &h.tmaps[t.g->tm_xf[iter & 1]];
         const bool tall = first && t.md->tall;
@@ -412,141 +519,155 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           while (!mbar_try_wait(sfull_bar + 8 * q, p) && clock64() - t0 < kWaitCycles) {}
         }
     }
-  } else if (kSrc) {
-    // ---------------- B X epilogue, warps 2..9: every warp takes each 32-column chunk in turn (its
-    // lane group's 32 rows, one 16-column half), with the X source from the shared-memory ring
-    const int ew = warp & 3;
+  } else if (warp >= 2 && warp < 10) {
+    // ---------------- epilogue warps 2..9: two warps per TMEM lane group (one per half of the columns)
+    const int ew = warp & 3;         // TMEM lane group this warp may access
     const int half = (warp - 2) >> 2;
-    const int lrow = ew * 32 + lane;   // row within the tile
-    const float* ring = reinterpret_cast<const float*>(base_ptr + STAGES * STAGE_BYTES);
+    const int lrow = ew * 32 + lane;  // row within the tile
     int acc = 0;
     uint32_t acc_ph = 0;
     int kc = 0;
     bool ok = true;
     for (int i = t_begin; i < t_end && ok; ++i) {
-      const int tile = tiles[i];
       int tm, tn;
-      TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
+      TileCtx t = tile_at(i, tm, tn);
       if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag, budget)) { ok = false; break; }
       fence_after();
-      const bool tall = iter == 0 && t.md->tall;
-      for (int c = 0; c < kBN / 32; ++c, ++kc) {
-        const int slot = kc & 1;
-        if (!mbar_wait(sfull_bar + 8 * slot, (uint32_t)(kc >> 1) & 1u, abort_flag, budget)) { ok = false; break; }
-        float v[16], x[16];
-        tmem_ld16(tmem_base + (uint32_t)(acc * kBN + c * 32 + 16 * half) + ((uint32_t)(ew * 32) << 16), v);
-        const float* sp = ring + slot * (SRC_BYTES / 4);
-        if (!tall) {
-          // [128 rows][32 f32] with the 128-byte swizzle: 16-byte unit u of row r sits at u ^ (r & 7)
-          const unsigned char* rp = reinterpret_cast<const unsigned char*>(sp) + lrow * 128;
+      float pacc = 0.f;
+      if constexpr (kSrc) {
+        // B X: every warp takes each 32-column chunk in turn (its lane group's 32 rows, one 16-column
+        // half), with the X source from the shared-memory ring
+        const float* ring = reinterpret_cast<const float*>(base_ptr + STAGES * STAGE_BYTES);
+        const bool tall = iter == 0 && t.md->tall;
+        for (int c = 0; c < kBN / 32; ++c, ++kc) {
+          const int slot = kc & 1;
+          if (!mbar_wait(sfull_bar + 8 * slot, (uint32_t)(kc >> 1) & 1u, abort_flag, budget)) { ok = false; break; }
+          float v[16], x[16];
+          tmem_ld16(tmem_base + (uint32_t)(acc * kBN + c * 32 + 16 * half) + ((uint32_t)(ew * 32) << 16), v);
+          const float* sp = ring + slot * (SRC_BYTES / 4);
+          if (!tall) {
+            // [128 rows][32 f32] with the 128-byte swizzle: 16-byte unit u of row r sits at u ^ (r & 7)
+            const unsigned char* rp = reinterpret_cast<const unsigned char*>(sp) + lrow * 128;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 f = *reinterpret_cast<const float4*>(rp + (((4 * half + q) ^ (lrow & 7)) << 4));
-            x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+            for (int q = 0; q < 4; ++q) {
+              const float4 f = *reinterpret_cast<const float4*>(rp + (((4 * half + q) ^ (lrow & 7)) << 4));
+              x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+            }
+          } else {
+            // [32 user rows = wide columns][128 f32 = wide rows], no swizzle: lanes read along a row
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[j] = sp[(16 * half + j) * BM + lrow];
           }
-        } else {
-          // [32 user rows = wide columns][128 f32 = wide rows], no swizzle: lanes read along a row
-#pragma unroll
-          for (int j = 0; j < 16; ++j) x[j] = sp[(16 * half + j) * BM + lrow];
+          epi_axpy_src<16>(t, tm * BM + lrow, tn * kBN + c * 32 + 16 * half, v, x);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sempty_bar + 8 * slot);
         }
-        epi_axpy_src<16>(t, tm * BM + lrow, tn * kBN + c * 32 + 16 * half, v, x);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sempty_bar + 8 * slot);
+        if (!ok) break;
+      } else {
+        constexpr int CH = kBN / 64;     // 32-column chunks per warp
+#pragma unroll 1
+        for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
+          float v[32];
+          tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
+          epi_chunk<32>(t, tm * BM + lrow, tn * kBN + ch * 32, v, &pacc);
+        }
       }
-      if (!ok) break;
       fence_before();
-      mbar_arrive(tempty_bar + 8 * acc);
+      if constexpr (kPair) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(at_rank0(tempty_bar + 8 * acc));
+      } else {
+        mbar_arrive(tempty_bar + 8 * acc);
+      }
+      if (!kSrc && stage == ST_PROBE) {  // one partial per epilogue warp: no barrier, fixed order later
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) pacc += __shfl_xor_sync(0xffffffffu, pacc, o2);
+        if (lane == 0) h.probe_partials[kProbeSlots * tiles[i] + (warp - 2)] = pacc;
+      }
       if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
     }
     if (!ok) {
       *abort_flag = 1;
       if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
     }
-  } else {
-    // ---------------- epilogue warps 2..9: two warps per TMEM lane group, one per half of the columns
-    const int ew = warp & 3;         // TMEM lane group this warp may access
-    const int half = (warp - 2) >> 2;
-    constexpr int CH = kBN / 64;     // 32-column chunks per warp
-    int acc = 0;
-    uint32_t acc_ph = 0;
-    for (int i = t_begin; i < t_end; ++i) {
-      const int tile = tiles[i];
-      int tm, tn;
-      TileCtx t = make_ctx(h, stage, iter, tile, tm, tn);
-      const int row = tm * BM + ew * 32 + lane;
-      if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag, budget)) {
-        *abort_flag = 1;
-        if (h.status) atomicOr(h.status, SMUON_DEV_WAIT_TIMEOUT);
-        break;
-      }
-      fence_after();
-      float pacc = 0.f;
-#pragma unroll 1
-      for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
-        float v[32];
-        tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
-        epi_chunk<32>(t, row, tn * kBN + ch * 32, v, &pacc);
-      }
-      fence_before();
-      mbar_arrive(tempty_bar + 8 * acc);
-      if (stage == ST_PROBE) {  // one partial per epilogue warp: no barrier, fixed order later
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) pacc += __shfl_xor_sync(0xffffffffu, pacc, o2);
-        if (lane == 0) h.probe_partials[kProbeSlots * tile + (warp - 2)] = pacc;
-      }
-      if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
-    }
   }
   fence_before();
-  __syncthreads();
+  if constexpr (kPair) {
+    __syncwarp();
+    cluster_sync_all();  // neither CTA leaves (or frees TMEM) while the other may still signal it
+  } else {
+    __syncthreads();
+  }
   fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+  if (warp == 1) {
+    if constexpr (kPair) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+    else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+  }
 }
 
 template <bool kSplit, int kBN, bool kShallow, bool kSrc>
 __global__ void __launch_bounds__(Cfg<kSplit, kBN, kShallow, kSrc>::NTHREADS, 1)
     k_gemm_tc(const Plan* plan, int stage, int iter, const int32_t* skip) {
   if (skip && *skip) return;
-  gemm_tc_body<kSplit, kBN, kShallow, kSrc>(plan, stage, iter);
+  gemm_tc_body<kSplit, kBN, kShallow, kSrc, false>(plan, stage, iter);
+}
+
+// SM pairs: 256 x 256 tiles, one cluster of two CTAs per pair of SMs
+template <bool kSplit, bool kShallow, bool kSrc>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kSplit, 256, kShallow, kSrc, true>::NTHREADS, 1)
+    k_gemm_tc2(const Plan* plan, int stage, int iter, const int32_t* skip) {
+  if (skip && *skip) return;  // read by both CTAs of a pair: both leave, or neither
+  gemm_tc_body<kSplit, 256, kShallow, kSrc, true>(plan, stage, iter);
 }
 
 }  // namespace tc
 
-template <bool kSplit, int kBN, bool kShallow, bool kSrc>
+template <bool kSplit, int kBN, bool kShallow, bool kSrc, bool kPair>
 static cudaError_t launch_tc_variant(const Plan* d_plan, int stage, int iter, const int32_t* skip, int grid,
                                      cudaStream_t s) {
-  using C = tc::Cfg<kSplit, kBN, kShallow, kSrc>;
+  using C = tc::Cfg<kSplit, kBN, kShallow, kSrc, kPair>;
   static bool attr_set[256] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 256 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc<kSplit, kBN, kShallow, kSrc>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+  if constexpr (kPair) {
+    if (dev < 256 && !attr_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc2<kSplit, kShallow, kSrc>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    // grid = the pairs' CTAs (a multiple of the cluster size)
+    tc::k_gemm_tc2<kSplit, kShallow, kSrc><<<2 * grid, C::NTHREADS, C::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
+  } else {
+    if (dev < 256 && !attr_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(tc::k_gemm_tc<kSplit, kBN, kShallow, kSrc>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    tc::k_gemm_tc<kSplit, kBN, kShallow, kSrc><<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
   }
-  tc::k_gemm_tc<kSplit, kBN, kShallow, kSrc><<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(d_plan, stage, iter, skip);
   return cudaGetLastError();
 }
 
-template <bool kSplit, int kBN, bool kSrc>
+template <bool kSplit, int kBN, bool kSrc, bool kPair>
 static cudaError_t launch_tc_src(const PlanHeader& h, const Plan* d_plan, int stage, int iter,
                                  const int32_t* skip, int grid, cudaStream_t s) {
-  // split operands of 256-wide tiles take 96 KB per ring stage: only the deep ring holds two of them
-  if (h.max_k[stage] <= kShallowMaxK && !(kSplit && kBN == 256))
-    return launch_tc_variant<kSplit, kBN, true, kSrc>(d_plan, stage, iter, skip, grid, s);
-  return launch_tc_variant<kSplit, kBN, false, kSrc>(d_plan, stage, iter, skip, grid, s);
+  // split operands of 256-wide single-SM tiles take 96 KB per ring stage: only the deep ring holds two
+  if (h.max_k[stage] <= kShallowMaxK && !(kSplit && kBN == 256 && !kPair))
+    return launch_tc_variant<kSplit, kBN, true, kSrc, kPair>(d_plan, stage, iter, skip, grid, s);
+  return launch_tc_variant<kSplit, kBN, false, kSrc, kPair>(d_plan, stage, iter, skip, grid, s);
 }
 
-template <bool kSplit, int kBN>
+template <bool kSplit, int kBN, bool kPair>
 static cudaError_t launch_tc_depth(const PlanHeader& h, const Plan* d_plan, int stage, int iter,
                                    const int32_t* skip, int grid, cudaStream_t s) {
   // the B X stage takes its X source through the shared-memory ring when the plan has the maps and
   // runs several steps (measured: with a single step the direct loads of the row-per-lane epilogue,
   // served by L1, were 4% faster on the ResNet-50 set; from two steps on the ring wins, 5-12%)
   if (stage == ST_AXPY && h.axpy_tma && h.iters >= 2)
-    return launch_tc_src<kSplit, kBN, true>(h, d_plan, stage, iter, skip, grid, s);
-  return launch_tc_src<kSplit, kBN, false>(h, d_plan, stage, iter, skip, grid, s);
+    return launch_tc_src<kSplit, kBN, true, kPair>(h, d_plan, stage, iter, skip, grid, s);
+  return launch_tc_src<kSplit, kBN, false, kPair>(h, d_plan, stage, iter, skip, grid, s);
 }
 
 int tc_tile_n(int stage, uint32_t flags) {
@@ -554,15 +675,44 @@ int tc_tile_n(int stage, uint32_t flags) {
   return (flags & SMUON_NS_SPLIT_BF16) ? kSplitBN : 256;  // split mode needs the smem for its lo tiles
 }
 
+int tc_pair_clusters() {
+  // pairs of SMs that can hold one cluster of the pair kernel each (its largest shared-memory form);
+  // the GPCs need not split evenly into pairs
+  static int cached[256] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 256 && cached[dev] > 0) return cached[dev];
+  using C = tc::Cfg<true, 256, false, true, true>;
+  auto fn = tc::k_gemm_tc2<true, false, true>;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) return 0;
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+  cfg.blockDim = dim3(C::NTHREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (const void*)fn, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev < 256) cached[dev] = n;
+  return n;
+}
+
 cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter, const int32_t* skip,
                            int num_sms, cudaStream_t s) {
-  (void)num_sms;  // the plan's schedule fixed the grid: one CTA per scheduled tile list
+  (void)num_sms;  // the plan's schedule fixed the grid: one CTA (or pair) per scheduled tile list
   const int grid = h.sched_ctas[stage];
   if (h.total_tiles[stage] == 0 || grid <= 0) return cudaSuccess;
   const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(stage);
-  if (split) return launch_tc_depth<true, kSplitBN>(h, d_plan, stage, iter, skip, grid, s);
-  if (tc_tile_n(stage, h.flags) == 128) return launch_tc_depth<false, 128>(h, d_plan, stage, iter, skip, grid, s);
-  return launch_tc_depth<false, 256>(h, d_plan, stage, iter, skip, grid, s);
+  if (h.pair) {
+    if (split) return launch_tc_depth<true, 256, true>(h, d_plan, stage, iter, skip, grid, s);
+    return launch_tc_depth<false, 256, true>(h, d_plan, stage, iter, skip, grid, s);
+  }
+  if (split) return launch_tc_depth<true, kSplitBN, false>(h, d_plan, stage, iter, skip, grid, s);
+  if (tc_tile_n(stage, h.flags) == 128) return launch_tc_depth<false, 128, false>(h, d_plan, stage, iter, skip, grid, s);
+  return launch_tc_depth<false, 256, false>(h, d_plan, stage, iter, skip, grid, s);
 }
 
 }  // namespace smuon

@@ -96,6 +96,9 @@ constexpr int kTcBM = 128;
 // operands) beat 128 x 128 tiles with three of 64 KB (4096^2, five quintic steps: 3.69 against 4.24 ms)
 constexpr int kSplitBN = 256;
 int tc_tile_n(int stage, uint32_t flags);  // 128 (symmetric stages, split mode) or 256
+int tc_pair_clusters();                    // clusters of the SM-pair GEMM kernel the device holds at once
+// a plan runs its tensor-core stages on SM pairs when every matrix's smaller side is at least this
+constexpr int kPairMinM = 256;
 constexpr int kSimtBM = 64;
 constexpr int kSimtBN = 64;
 

@@ -113,7 +113,9 @@ struct PlanHeader {
   float beta;
   float gamma;              // probe threshold
   int32_t total_mom_tiles;
-  int32_t tile_bm, tile_bn; // tile shape of the GEMM kernel the tables are built for
+  int32_t tile_bm, tile_bn; // tile shape of the GEMM kernel the tables are built for (256 x 256 for SM pairs)
+  int32_t pair;             // tensor-core stages on SM pairs (clusters of two CTAs, one 256 x 256 tile each)
+  int32_t pad_pair;
   int32_t total_tiles[ST_COUNT];
   int32_t sym_ratio[ST_COUNT];  // BN / BM of the symmetric stages' tiles (1 or 2)
   float* partials;          // [total_mom_tiles] sum of squares per momentum tile

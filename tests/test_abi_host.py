@@ -234,3 +234,24 @@ def test_bits_wrapper_describes_a_message():
         S.Bits(torch.zeros(10, dtype=torch.int32), 96, 40)            # too few words
     with pytest.raises(ValueError):
         S.Bits(torch.zeros(S.packed_words(96 * 40), dtype=torch.int64), 96, 40)
+
+
+def test_sm_pair_choice_is_a_valid_flag_and_sizes_the_tile_tables(L):
+    """SMUON_NS_ONE_SM is a known flag. The SM-pair choice is made from the flags
+    and the shapes alone (the host's sizing pass and the device's filling pass
+    agree): 256 x 256 pair tiles need fewer schedule entries than 128 x 256
+    single-SM tiles, so an eligible batch asks for no more workspace in the pair
+    form, and a batch with a matrix below 256 rows asks for the same in both."""
+    import matrix_aware_sign_b200 as S
+
+    def ws(shapes, flags):
+        arr = (S.SmuonMat * len(shapes))(*[S.SmuonMat(4096, r, c, c, S.F32) for r, c in shapes])
+        out = ctypes.c_size_t(0)
+        assert L.smuon_ns_workspace_bytes(arr, len(shapes), 5, flags, ctypes.byref(out)) == 0
+        return out.value
+
+    big = [(768, 2304), (4096, 4096)]
+    for fl in (0, S.NS_SPLIT_BF16):
+        assert ws(big, fl) <= ws(big, fl | S.NS_ONE_SM)
+        small = big + [(64, 147)]
+        assert ws(small, fl) == ws(small, fl | S.NS_ONE_SM)

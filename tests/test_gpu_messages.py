@@ -140,11 +140,13 @@ def test_plain_lead_two_steps_meets_the_criteria(shape):
     assert err < 1e-3
 
 
-def test_bounded_wait_runs_out_and_the_context_survives():
+@pytest.mark.parametrize("form", [0, S.NS_ONE_SM])
+def test_bounded_wait_runs_out_and_the_context_survives(form):
     """SMUON_NS_TEST_WAIT_EXPIRY: the tensor-core stages' producers issue nothing
     and their waits are limited to 65536 clocks, so every stage's waits run out.
     The call returns, SMUON_DEV_WAIT_TIMEOUT is set, and the next normal call
-    still matches the oracle."""
+    still matches the oracle. Both forms: 256 x 640 runs on SM pairs unless
+    SMUON_NS_ONE_SM asks for single-SM tiles."""
     rng = np.random.default_rng(3)
     Mx = rng.standard_normal((256, 640)).astype(np.float32)
     Md = dev(Mx)
@@ -152,11 +154,11 @@ def test_bounded_wait_runs_out_and_the_context_survives():
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     for flags in (S.NS_SPLIT_BF16 | S.NS_TEST_WAIT_EXPIRY, S.NS_TEST_WAIT_EXPIRY):
         status.zero_()
-        S.smuon_ns([Md], [U], *WL.QUINTIC, 2, flags=flags, status=status)
+        S.smuon_ns([Md], [U], *WL.QUINTIC, 2, flags=flags | form, status=status)
         torch.cuda.synchronize()
         assert int(status.item()) & S.DEV_WAIT_TIMEOUT
     status.zero_()
-    S.smuon_ns([Md], [U], *WL.QUINTIC, 2, flags=S.NS_SPLIT_BF16, status=status)
+    S.smuon_ns([Md], [U], *WL.QUINTIC, 2, flags=S.NS_SPLIT_BF16 | form, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     check_ns_outputs([(host(U), O.newton_schulz(Mx.astype(np.float64), *WL.QUINTIC, 2))], 1e-2)

@@ -1003,3 +1003,62 @@ def test_distributed_sign_muon_single_rank(exchange):
         assert opt.payload()["ratio_vs_f32"] == (32.0 if exchange == "allgather" else 4.0)
     finally:
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ SM pairs against single-SM tiles
+PAIR_SHAPES = [(256, 512), (1000, 384), (384, 640), (512, 300), (768, 2304), (2304, 768)]
+
+
+def _ns_out(Ms, shapes, M, out, iters, flags):
+    if out == "bits":
+        U = [S.Bits.empty(*s) for s in shapes for _ in range(M)]
+    else:
+        dt = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8}[out]
+        U = [torch.zeros(s, dtype=dt, device="cuda") for s in shapes for _ in range(M)]
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.trace_enable(True)
+    S.smuon_ns(Ms, U, *WL.QUINTIC, iters, flags=flags, status=st)
+    torch.cuda.synchronize()
+    names = {r["name"].split(".")[0] for r in S.trace_read() if r["name"].startswith("k_gemm")}
+    S.trace_enable(False)
+    assert int(st.item()) == 0
+    return [u.words if out == "bits" else u for u in U], names
+
+
+@pytest.mark.parametrize("out,iters,flags", [
+    ("f32", 1, 0),
+    ("f32", 5, S.NS_SPLIT_BF16),
+    ("bf16", 5, S.NS_SPLIT_BF16 | S.ns_plain_lead(2)),
+    ("i8", 3, S.NS_SPLIT_BF16),
+    ("bits", 5, S.NS_SPLIT_BF16 | S.ns_plain_lead(2)),
+    ("f32", 5, S.NS_SPLIT_BF16 | S.NS_SPECTRAL),
+])
+def test_sm_pairs_equal_single_sm_tiles(out, iters, flags):
+    """Matrices whose smaller side is at least 256 run the tensor-core stages on
+    pairs of SMs (256 x 256 tiles, one MMA over both SMs); both forms add the
+    same products in the same order, so their outputs agree bit for bit. The
+    shapes include pair rows whose second half lies partly or wholly beyond m
+    (m = 300, 384) and tall matrices read transposed."""
+    M = 2
+    shapes = [s for s in PAIR_SHAPES if out != "bits" or s[1] % 32 == 0]
+    rng = np.random.default_rng(iters * 7 + flags)
+    Mx = [rng.standard_normal(s).astype(np.float32) for s in shapes for _ in range(M)]
+    Ms = [dev(x) for x in Mx]
+    Up, names_p = _ns_out(Ms, shapes, M, out, iters, flags)
+    Us, names_s = _ns_out(Ms, shapes, M, out, iters, flags | S.NS_ONE_SM)
+    assert all(n.startswith("k_gemm_tc2") for n in names_p) and names_p
+    assert not any(n.startswith("k_gemm_tc2") for n in names_s) and names_s
+    for a, b in zip(Up, Us):
+        assert torch.equal(a, b)
+    if out == "f32" and not (flags & S.NS_SPECTRAL):
+        refs = [O.newton_schulz(x.astype(np.float64), *WL.QUINTIC, iters) for x in Mx]
+        check_ns_outputs([(host(u), r) for u, r in zip(Up, refs)], 1e-2)
+
+
+def test_small_matrices_stay_on_single_sm_tiles():
+    """A call with any matrix whose smaller side is below 256 keeps the whole
+    batch on single-SM 128 x 256 tiles (a pair's second half would be empty)."""
+    shapes = [(768, 2304), (64, 147)]
+    Ms = [dev(np.random.default_rng(i).standard_normal(s).astype(np.float32)) for i, s in enumerate(shapes)]
+    _, names = _ns_out(Ms, shapes, 1, "f32", 2, S.NS_SPLIT_BF16)
+    assert names and not any(n.startswith("k_gemm_tc2") for n in names)
