@@ -25,6 +25,20 @@ struct TileCtx {
   int32_t split;              // operands are stored as bf16 hi + lo parts
   int32_t sym;                // symmetric m x m stage (Gram, A^2, probe)
   int64_t xlo, mlo;           // element offset of the lo part of an X (m x n) / m x m buffer
+  // per-tile copies of the group's and the matrix's pointers and strides: they stay in registers across
+  // the epilogue's stores (reading them from the plan after a store would be a dependent load per chunk)
+  int64_t ldn, ldm;           // padded leading dims of the group's m x n and m x m buffers
+  float* af;                  // f32 A
+  void* aop;                  // A operand
+  void* bop;                  // B operand
+  const float* x_cur;         // B X, steps >= 1: this step's X (f32 master, or the FP32-mode operand)
+  float* xf_next;             // B X: f32 master of the next X (bf16 modes)
+  void* xop_next;             // B X: operand of the next X
+  const void* m_ptr;          // the user's momentum (the first B X step's source)
+  int64_t m_ld;
+  void* u_ptr;                // the user's output
+  int64_t u_ld;
+  int32_t m_dtype, u_dtype, tall, m_vec, u_vec;
 };
 
 // Gram, A^2 and the probe produce symmetric m x m results. Only tiles that
@@ -80,10 +94,66 @@ __device__ __forceinline__ void st_bf16_vec(__nv_bfloat16* p, const float* v) {
   }
 }
 
+// Workspace rows (256-byte aligned buffers, leading dims a multiple of 128 elements, chunks starting at a
+// multiple of 16 elements) take 256-bit accesses: a lane's 16 floats or 16 bf16 move as whole 32-byte
+// sectors, half the L2 requests of 128-bit accesses and no partial-sector writes. User buffers (16-byte
+// alignment at most) keep the 128-bit forms above.
+__device__ __forceinline__ void st_v8_f32(float* p, const float* v) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void st_v8_b32(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+__device__ __forceinline__ void ld_v8_f32(const float* p, float* v) {
+  asm volatile("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+               : "l"(p));
+}
+template <int NV>
+__device__ __forceinline__ void st_f32_ws(float* p, const float* v) {
+  if constexpr (NV % 8 == 0) {
+#pragma unroll
+    for (int q = 0; q < NV / 8; ++q) st_v8_f32(p + 8 * q, v + 8 * q);
+  } else {
+    st_f32_vec<NV>(p, v);
+  }
+}
+template <int NV>
+__device__ __forceinline__ void st_bf16_ws(__nv_bfloat16* p, const float* v) {
+  if constexpr (NV % 16 == 0) {
+#pragma unroll
+    for (int q = 0; q < NV / 16; ++q) {
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[k] = pack_bf16x2_rn(v[16 * q + 2 * k], v[16 * q + 2 * k + 1]);
+      st_v8_b32(p + 16 * q, w);
+    }
+  } else {
+    st_bf16_vec<NV>(p, v);
+  }
+}
+template <int NV>
+__device__ __forceinline__ void ld_f32_ws(const float* p, float* v) {
+  if constexpr (NV % 8 == 0) {
+#pragma unroll
+    for (int q = 0; q < NV / 8; ++q) ld_v8_f32(p + 8 * q, v + 8 * q);
+  } else {
+#pragma unroll
+    for (int q = 0; q < NV / 4; ++q) {
+      float4 t = reinterpret_cast<const float4*>(p)[q];
+      v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+    }
+  }
+}
+
 template <int NV>
 __device__ __forceinline__ void st_op(void* base, int64_t off, int bf, const float* v) {
-  if (bf) st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
-  else st_f32_vec<NV>(reinterpret_cast<float*>(base) + off, v);
+  if (bf) st_bf16_ws<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
+  else st_f32_ws<NV>(reinterpret_cast<float*>(base) + off, v);
 }
 
 // one operand element (same encodings as st_operand)
@@ -102,15 +172,15 @@ template <int NV>
 __device__ __forceinline__ void st_operand(const TileCtx& t, void* base, int64_t off, int64_t lo_off,
                                            const float* v) {
   if (!t.bf) {
-    st_f32_vec<NV>(reinterpret_cast<float*>(base) + off, v);
+    st_f32_ws<NV>(reinterpret_cast<float*>(base) + off, v);
     return;
   }
-  st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
+  st_bf16_ws<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
   if (t.split) {
     float lo[NV];
 #pragma unroll
     for (int k = 0; k < NV; ++k) lo[k] = v[k] - __bfloat162float(__float2bfloat16_rn(v[k]));
-    st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off + lo_off, lo);
+    st_bf16_ws<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off + lo_off, lo);
   }
 }
 
@@ -269,10 +339,10 @@ __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int 
 template <int NV>
 __device__ __forceinline__ void sym_store_f32(const TileCtx& t, float* base, int row, int col0, int nvalid,
                                               int ds, int ms, const float* v) {
-  const int64_t m = t.g->m, ld = t.g->ldm;
+  const int64_t m = t.Mo, ld = t.ldm;
   const int64_t off = ((int64_t)t.z * m + row) * ld + col0;
   if (ds == 0) {
-    st_f32_vec<NV>(base + off, v);
+    st_f32_ws<NV>(base + off, v);
   } else {
 #pragma unroll
     for (int k = 0; k < NV; ++k)
@@ -287,7 +357,7 @@ __device__ __forceinline__ void sym_store_f32(const TileCtx& t, float* base, int
 template <int NV>
 __device__ __forceinline__ void sym_store_operand(const TileCtx& t, void* base, int row, int col0, int nvalid,
                                                   int ds, int ms, const float* v) {
-  const int64_t m = t.g->m, ld = t.g->ldm;
+  const int64_t m = t.Mo, ld = t.ldm;
   const int64_t off = ((int64_t)t.z * m + row) * ld + col0;
   if (ds == 0) {
     st_operand<NV>(t, base, off, t.mlo, v);
@@ -336,50 +406,51 @@ __device__ __forceinline__ void emit_q1(const TileCtx& t, int row, int col0, int
   }
 }
 
-// v[] holds the raw accumulator of D = A_op * B_op at (row, col0..col0+NV-1)
-template <int NV>
+// v[] holds the raw accumulator of D = A_op * B_op at (row, col0..col0+NV-1). kStage is the stage when
+// the caller knows it at compile time (then only that stage's code and context stay live), else -1.
+template <int NV, int kStage = -1>
 __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, float* v,
                                           float* probe_acc) {
   if (row >= t.Mo || col0 >= t.No) return;
   const int nvalid = min(NV, t.No - col0);
   const GroupDesc& g = *t.g;
-  const int m = g.m;
+  const int m = t.Mo;
   // symmetric stages: elements k >= ds are on or above the diagonal, k >= ms strictly above
   const int ds = t.sym ? max(0, row - col0) : 0;
   const int ms = t.sym ? max(0, row - col0 + 1) : NV;
-  switch (t.stage) {
+  switch (kStage >= 0 ? kStage : t.stage) {
     case ST_GRAM: {
       if (ds >= nvalid) break;  // the chunk lies below the diagonal
       const float sc = (t.iter == 0 && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s * t.s : 1.f;
       if (t.c != 0.f) {
 #pragma unroll
         for (int k = 0; k < NV; ++k) v[k] *= sc;
-        sym_store_f32<NV>(t, g.af, row, col0, nvalid, ds, ms, v);
-        if (t.bf) sym_store_operand<NV>(t, g.aop, row, col0, nvalid, ds, ms, v);
+        sym_store_f32<NV>(t, t.af, row, col0, nvalid, ds, ms, v);
+        if (t.bf) sym_store_operand<NV>(t, t.aop, row, col0, nvalid, ds, ms, v);
       } else {
         if (t.flags & SMUON_NS_SPECTRAL) {  // f32 A_0 for the largest-eigenvalue estimate
           float a0[NV];
 #pragma unroll
           for (int k = 0; k < NV; ++k) a0[k] = sc * v[k];
-          sym_store_f32<NV>(t, g.af, row, col0, nvalid, ds, ms, a0);
+          sym_store_f32<NV>(t, t.af, row, col0, nvalid, ds, ms, a0);
         }
 #pragma unroll
         for (int k = 0; k < NV; ++k) v[k] = t.b * (sc * v[k]);
-        sym_store_operand<NV>(t, g.bop, row, col0, nvalid, ds, ms, v);
+        sym_store_operand<NV>(t, t.bop, row, col0, nvalid, ds, ms, v);
         if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, ds, ms, v);
       }
       break;
     }
     case ST_POLY: {
       if (ds >= nvalid) break;
-      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
+      const int64_t off = ((int64_t)t.z * m + row) * t.ldm + col0;
       float A[NV];
-      ld_f32_vec<NV>(g.af + off, A);
+      ld_f32_ws<NV>(t.af + off, A);
       // spectral scaling at the first step: A' = r^2 A, so B = b r^2 A + c r^4 A^2 (r = 1 otherwise)
       const float r2 = t.iter == 0 ? t.r * t.r : 1.f;
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] = t.b * (r2 * A[k]) + t.c * ((r2 * r2) * v[k]);
-      sym_store_operand<NV>(t, g.bop, row, col0, nvalid, ds, ms, v);
+      sym_store_operand<NV>(t, t.bop, row, col0, nvalid, ds, ms, v);
       if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, ds, ms, v);
       break;
     }
@@ -389,39 +460,36 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       // written before r was known, so its product takes the r^2 of A' = r^2 A here
       const float sc = (first && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s * t.r : 1.f;
       const float sv = (first && t.c == 0.f) ? sc * (t.r * t.r) : sc;
-      const int64_t off = ((int64_t)t.z * m + row) * g.ldn + col0;
+      const int64_t off = ((int64_t)t.z * m + row) * t.ldn + col0;
       float x[NV];
       if (first && t.bf) {
         // X_0 read from the user's momentum in its own dtype and orientation
-        const MatDesc& md = *t.md;
-        ld_user<NV>(md.m_ptr, md.m_ld, md.m_dtype, md.tall, md.vec & 1, row, col0, nvalid, x);
+        ld_user<NV>(t.m_ptr, t.m_ld, t.m_dtype, t.tall, t.m_vec, row, col0, nvalid, x);
       } else {
-        const float* src = t.bf ? g.xf[t.iter & 1] : reinterpret_cast<const float*>(g.xop[t.iter & 1]);
-        ld_f32_vec<NV>(src + off, x);
+        ld_f32_ws<NV>(t.x_cur + off, x);
       }
 #pragma unroll
       for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sv * v[k];
       if (t.iter != t.last) {
-        const int nb = (t.iter + 1) & 1;
-        if (t.bf) st_f32_vec<NV>(g.xf[nb] + off, x);
-        st_operand<NV>(t, g.xop[nb], off, t.xlo, x);
+        if (t.bf) st_f32_ws<NV>(t.xf_next + off, x);
+        st_operand<NV>(t, t.xop_next, off, t.xlo, x);
       } else {
-        st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, x);
+        st_user<NV>(t.u_ptr, t.u_ld, t.u_dtype, t.tall, t.u_vec, row, col0, nvalid, x);
       }
       break;
     }
     case ST_QAXPY: {
-      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
+      const int64_t off = ((int64_t)t.z * m + row) * t.ldm + col0;
       float q[NV];
       const float* src = t.bf ? g.qf[t.iter & 1] : reinterpret_cast<const float*>(g.qop[t.iter & 1]);
-      ld_f32_vec<NV>(src + off, q);
+      ld_f32_ws<NV>(src + off, q);
 #pragma unroll
       for (int k = 0; k < NV; ++k) q[k] = t.a * q[k] + v[k];
       if (t.iter == t.last)
         st_user<NV>(t.md->q_ptr, t.md->q_ld, SMUON_BF16, 0, (t.md->vec >> 2) & 1, row, col0, nvalid, q);
       if (t.iter != t.last || (t.flags & SMUON_NS_GRAM_ONLY)) {  // Q_K X_0 reads the workspace copy
         const int nb = (t.iter + 1) & 1;
-        if (t.bf) st_f32_vec<NV>(g.qf[nb] + off, q);
+        if (t.bf) st_f32_ws<NV>(g.qf[nb] + off, q);
         st_operand<NV>(t, g.qop[nb], off, t.mlo, q);
       }
       break;
@@ -429,14 +497,14 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
     case ST_QX: {  // Gram-only fresh solve: U = s Q_K X_0
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] *= t.s;
-      st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, v);
+      st_user<NV>(t.u_ptr, t.u_ld, t.u_dtype, t.tall, t.u_vec, row, col0, nvalid, v);
       break;
     }
     case ST_REUSE: {
-      const int64_t off = ((int64_t)t.z * m + row) * g.ldn + col0;
+      const int64_t off = ((int64_t)t.z * m + row) * t.ldn + col0;
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] *= t.s;
-      st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, v);
+      st_user<NV>(t.u_ptr, t.u_ld, t.u_dtype, t.tall, t.u_vec, row, col0, nvalid, v);
       if (!(t.flags & SMUON_NS_GRAM_ONLY)) st_op<NV>(g.xop[1], off, t.bf, v);  // the probe's operand
       break;
     }
@@ -446,9 +514,9 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       // (second); both are symmetric (polynomials in A_k), stored by the triangle rule
       if (ds >= nvalid) break;
       const bool first = t.stage == ST_AA1;
-      const int64_t off = ((int64_t)t.z * m + row) * g.ldm + col0;
+      const int64_t off = ((int64_t)t.z * m + row) * t.ldm + col0;
       float y[NV];
-      ld_f32_vec<NV>((first ? g.af : g.af2) + off, y);
+      ld_f32_ws<NV>((first ? g.af : g.af2) + off, y);
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] = t.a * y[k] + v[k];
       sym_store_f32<NV>(t, first ? g.af2 : g.af, row, col0, nvalid, ds, ms, v);
@@ -478,18 +546,16 @@ template <int NV>
 __device__ __forceinline__ void epi_axpy_src(const TileCtx& t, int row, int col0, const float* v, float* x) {
   if (row >= t.Mo || col0 >= t.No) return;
   const int nvalid = min(NV, t.No - col0);
-  const GroupDesc& g = *t.g;
   const float sc = (t.iter == 0 && !(t.flags & SMUON_NS_NO_NORMALIZE)) ? t.s * t.r : 1.f;
   const float sv = (t.iter == 0 && t.c == 0.f) ? sc * (t.r * t.r) : sc;
 #pragma unroll
   for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sv * v[k];
   if (t.iter != t.last) {
-    const int64_t off = ((int64_t)t.z * g.m + row) * g.ldn + col0;
-    const int nb = (t.iter + 1) & 1;
-    st_f32_vec<NV>(g.xf[nb] + off, x);
-    st_operand<NV>(t, g.xop[nb], off, t.xlo, x);
+    const int64_t off = ((int64_t)t.z * t.Mo + row) * t.ldn + col0;
+    st_f32_ws<NV>(t.xf_next + off, x);
+    st_operand<NV>(t, t.xop_next, off, t.xlo, x);
   } else {
-    st_user<NV>(t.md->u_ptr, t.md->u_ld, t.md->u_dtype, t.md->tall, (t.md->vec >> 1) & 1, row, col0, nvalid, x);
+    st_user<NV>(t.u_ptr, t.u_ld, t.u_dtype, t.tall, t.u_vec, row, col0, nvalid, x);
   }
 }
 
@@ -530,6 +596,24 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
   t.split = (h.flags & SMUON_NS_SPLIT_BF16) ? 1 : 0;
   t.xlo = (int64_t)g.count * g.m * g.ldn;
   t.mlo = (int64_t)g.count * g.m * g.ldm;
+  t.ldn = g.ldn;
+  t.ldm = g.ldm;
+  t.af = g.af;
+  t.aop = g.aop;
+  t.bop = g.bop;
+  t.x_cur = t.bf ? g.xf[iter & 1] : reinterpret_cast<const float*>(g.xop[iter & 1]);
+  t.xf_next = g.xf[(iter + 1) & 1];
+  t.xop_next = g.xop[(iter + 1) & 1];
+  const MatDesc& md = *t.md;
+  t.m_ptr = md.m_ptr;
+  t.m_ld = md.m_ld;
+  t.u_ptr = md.u_ptr;
+  t.u_ld = md.u_ld;
+  t.m_dtype = md.m_dtype;
+  t.u_dtype = md.u_dtype;
+  t.tall = md.tall;
+  t.m_vec = md.vec & 1;
+  t.u_vec = (md.vec >> 1) & 1;
   return t;
 }
 

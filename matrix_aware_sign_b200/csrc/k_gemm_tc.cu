@@ -65,6 +65,10 @@ struct Cfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SRC_RING + 1024 /*align*/ + 256 /*barriers*/;
 };
 constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz: the exit drains' budget
+template <int V>
+struct StageTag {
+  static constexpr int value = V;
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -135,8 +139,16 @@ __device__ __forceinline__ uint32_t at_rank0(uint32_t saddr) {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Relaxed arrives for the epilogue's releases of a source slot or an accumulator: what must precede them
+// is the warp's reads of that shared memory (whose values the warp has already used) or of that tensor
+// memory (completed by tcgen05.wait::ld and ordered by tcgen05.fence::before_thread_sync). A release arrive
+// would also wait for every global store the warp has issued, which the consumers of these barriers (the
+// source producer and the MMA issuer) never read.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 __device__ __forceinline__ void tensormap_acquire(const CUtensorMap* map) {
@@ -233,6 +245,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Split form of a 32-lane x 16-column accumulator load: issue now, wait later. The wait names the
+// destination registers as operands, so no use of them can be scheduled above it.
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
 }
 
 // operands of one tile: tensor maps, coordinates, K extent
@@ -536,14 +566,19 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       float pacc = 0.f;
       if constexpr (kSrc) {
         // B X: every warp takes each 32-column chunk in turn (its lane group's 32 rows, one 16-column
-        // half), with the X source from the shared-memory ring
+        // half), with the X source from the shared-memory ring. The accumulator load of the next chunk
+        // is in flight while this one is processed (two register sets, the loop unrolled by two).
         const float* ring = reinterpret_cast<const float*>(base_ptr + STAGES * STAGE_BYTES);
-        const bool tall = iter == 0 && t.md->tall;
-        for (int c = 0; c < kBN / 32; ++c, ++kc) {
+        const bool tall = iter == 0 && t.tall;
+        auto taddr = [&](int c) {
+          return tmem_base + (uint32_t)(acc * kBN + c * 32 + 16 * half) + ((uint32_t)(ew * 32) << 16);
+        };
+        auto process = [&](int c, const uint32_t (&r)[16]) -> bool {
           const int slot = kc & 1;
-          if (!mbar_wait(sfull_bar + 8 * slot, (uint32_t)(kc >> 1) & 1u, abort_flag, budget)) { ok = false; break; }
+          if (!mbar_wait(sfull_bar + 8 * slot, (uint32_t)(kc >> 1) & 1u, abort_flag, budget)) return false;
           float v[16], x[16];
-          tmem_ld16(tmem_base + (uint32_t)(acc * kBN + c * 32 + 16 * half) + ((uint32_t)(ew * 32) << 16), v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
           const float* sp = ring + slot * (SRC_BYTES / 4);
           if (!tall) {
             // [128 rows][32 f32] with the 128-byte swizzle: 16-byte unit u of row r sits at u ^ (r & 7)
@@ -560,16 +595,48 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           }
           epi_axpy_src<16>(t, tm * BM + lrow, tn * kBN + c * 32 + 16 * half, v, x);
           __syncwarp();
-          if (lane == 0) mbar_arrive(sempty_bar + 8 * slot);
+          if (lane == 0) mbar_arrive_relaxed(sempty_bar + 8 * slot);
+          ++kc;
+          return true;
+        };
+        static_assert((kBN / 32) % 2 == 0, "chunks are processed in pairs");
+        uint32_t ra[16], rb[16];
+        tmem_ld16_issue(taddr(0), ra);
+        for (int c = 0; c < kBN / 32 && ok; c += 2) {
+          tmem_ld_wait(ra);
+          tmem_ld16_issue(taddr(c + 1), rb);
+          if (!process(c, ra)) { ok = false; tmem_ld_wait(rb); break; }
+          tmem_ld_wait(rb);
+          if (c + 2 < kBN / 32) tmem_ld16_issue(taddr(c + 2), ra);
+          if (!process(c + 1, rb)) {
+            ok = false;
+            if (c + 2 < kBN / 32) tmem_ld_wait(ra);
+            break;
+          }
         }
         if (!ok) break;
       } else {
         constexpr int CH = kBN / 64;     // 32-column chunks per warp
+        // the stage as a compile-time constant: each instantiation keeps only its own context live
+        auto chunks = [&](auto tag) {
+          constexpr int kSt = decltype(tag)::value;
 #pragma unroll 1
-        for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
-          float v[32];
-          tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
-          epi_chunk<32>(t, tm * BM + lrow, tn * kBN + ch * 32, v, &pacc);
+          for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
+            float v[32];
+            tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
+            epi_chunk<32, kSt>(t, tm * BM + lrow, tn * kBN + ch * 32, v, &pacc);
+          }
+        };
+        switch (stage) {
+          case ST_GRAM: chunks(StageTag<ST_GRAM>{}); break;
+          case ST_POLY: chunks(StageTag<ST_POLY>{}); break;
+          case ST_AXPY: chunks(StageTag<ST_AXPY>{}); break;
+          case ST_QAXPY: chunks(StageTag<ST_QAXPY>{}); break;
+          case ST_REUSE: chunks(StageTag<ST_REUSE>{}); break;
+          case ST_PROBE: chunks(StageTag<ST_PROBE>{}); break;
+          case ST_AA1: chunks(StageTag<ST_AA1>{}); break;
+          case ST_AA2: chunks(StageTag<ST_AA2>{}); break;
+          default: chunks(StageTag<ST_QX>{}); break;
         }
       }
       fence_before();
@@ -577,7 +644,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(at_rank0(tempty_bar + 8 * acc));
       } else {
-        mbar_arrive(tempty_bar + 8 * acc);
+        mbar_arrive_relaxed(tempty_bar + 8 * acc);
       }
       if (!kSrc && stage == ST_PROBE) {  // one partial per epilogue warp: no barrier, fixed order later
 #pragma unroll
