@@ -837,9 +837,11 @@ def gemm_stage_bytes(shapes, workers, iters, c, split, u_bytes):
     """Algorithmic HBM bytes per launch of each Newton-Schulz GEMM stage
     (averaged over the iterations), from the shapes alone: every operand read
     once, the epilogue's source read and its outputs written once. X is the
-    wide m x n form; operands are bf16 (hi and lo parts in split mode), masters
-    and A are f32; the first step's X source is the f32 momentum, the last
-    step writes U (u_bytes per entry)."""
+    wide m x n form; operands are bf16 (hi and lo parts in split mode), A is
+    f32; between steps X is kept as an f32 master in plain mode and as its hi
+    and lo parts alone in split mode (4 bytes read back as the next step's
+    source either way); the first step's X source is the f32 momentum, the
+    last step writes U (u_bytes per entry)."""
     op = 4 if split else 2
     tot = {"gram": 0.0, "poly": 0.0, "axpy": 0.0}
     for r, cc in shapes:
@@ -849,7 +851,7 @@ def gemm_stage_bytes(shapes, workers, iters, c, split, u_bytes):
             tot["gram"] += workers * (op * m * n + (4 * m * m + op * m * m if c != 0 else op * m * m))
             if c != 0:
                 tot["poly"] += workers * (op * m * m + 4 * m * m + op * m * m)
-            out = u_bytes * m * n if last else (4 + op) * m * n
+            out = u_bytes * m * n if last else (op if split else 4 + op) * m * n
             tot["axpy"] += workers * (op * m * m + op * m * n + 4 * m * n + out)
     return {k: v / iters for k, v in tot.items()}
 

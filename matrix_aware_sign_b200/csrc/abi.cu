@@ -139,7 +139,8 @@ smuon_status get_encoder(EncodeTiledFn* fn) {
 
 // 3-D bf16 map over [count][rows][ld] with box {box0 (inner), box1, 1}, 128B swizzle
 smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, int64_t rows, int64_t count,
-                            int64_t ld, uint32_t box0, uint32_t box1) {
+                            int64_t ld, uint32_t box0, uint32_t box1,
+                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc;
   smuon_status st = get_encoder(&enc);
   if (st != SMUON_OK) return st;
@@ -148,7 +149,7 @@ smuon_status encode_bf16_3d(CUtensorMap* out, const void* ptr, int64_t inner, in
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return SMUON_OK;
@@ -507,8 +508,10 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
       g.aop2 = B->ptr_at<void>(B->take(nm * 2 * parts));
     }
     if (K >= 2 && !gram_only) g.xop[1] = B->ptr_at<void>(B->take(nx * esz * parts));
-    if (bf && K >= 2 && !gram_only) g.xf[1] = B->ptr_at<float>(B->take(nx * 4));
-    if (bf && K >= 3 && !gram_only) g.xf[0] = B->ptr_at<float>(B->take(nx * 4));
+    // f32 masters of X between steps: plain BF16 keeps one (its operand holds only bf16(X)); split mode
+    // carries X as its hi and lo operand parts, which the B X epilogue reads back as hi + lo
+    if (bf && parts == 1 && K >= 2 && !gram_only) g.xf[1] = B->ptr_at<float>(B->take(nx * 4));
+    if (bf && parts == 1 && K >= 3 && !gram_only) g.xf[0] = B->ptr_at<float>(B->take(nx * 4));
     if (rq.c != 0.f || spectral) g.af = B->ptr_at<float>(B->take(nm * 4));  // f32 A_0 (Lanczos input)
     if (rq.c != 0.f) g.aop = bf ? B->ptr_at<void>(B->take(nm * 2 * parts)) : (void*)g.af;
     g.bop = B->ptr_at<void>(B->take(nm * esz * parts));
@@ -623,10 +626,14 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
       const MatDesc& d = B->mats[g.first_mat];
       if ((st = encode_bf16_3d(&B->maps[g.tm_uq_k], d.q_ptr, g.m, g.m, 1, d.q_ld, 64, 128)) != SMUON_OK) return st;
     }
-    for (int i = 0; i < 2; ++i)  // f32 masters [count][m][ldn], 32 x 128 boxes
-      if (g.tm_xf[i] >= 0 &&
-          (st = encode_f32_3d(&B->maps[g.tm_xf[i]], g.xf[i], g.n, g.m, g.count, g.ldn, 32, 128)) != SMUON_OK)
-        return st;
+    for (int i = 0; i < 2; ++i) {  // the B X epilogue's source of X_i, 32 x 128 boxes
+      if (g.tm_xf[i] < 0) continue;
+      if (parts == 1)  // f32 master [count][m][ldn]
+        st = encode_f32_3d(&B->maps[g.tm_xf[i]], g.xf[i], g.n, g.m, g.count, g.ldn, 32, 128);
+      else  // bf16 hi parts then lo parts [2 count][m][ldn], 64-byte rows with the 64-byte swizzle
+        st = encode_bf16_3d(&B->maps[g.tm_xf[i]], g.xop[i], g.n, g.m, zc, g.ldn, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+      if (st != SMUON_OK) return st;
+    }
   }
   for (const MatDesc& d : B->mats) {  // the momentum as the first B X step's source
     if (d.tm_src < 0) continue;

@@ -32,6 +32,7 @@ struct TileCtx {
   void* aop;                  // A operand
   void* bop;                  // B operand
   const float* x_cur;         // B X, steps >= 1: this step's X (f32 master, or the FP32-mode operand)
+  const __nv_bfloat16* x_cur_op;  // split mode: this step's X as its hi parts (lo parts xlo further)
   float* xf_next;             // B X: f32 master of the next X (bf16 modes)
   void* xop_next;             // B X: operand of the next X
   const void* m_ptr;          // the user's momentum (the first B X step's source)
@@ -147,6 +148,28 @@ __device__ __forceinline__ void ld_f32_ws(const float* p, float* v) {
       float4 t = reinterpret_cast<const float4*>(p)[q];
       v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
     }
+  }
+}
+
+// x = hi + lo from the two bf16 parts of a workspace row chunk (split mode's X between steps)
+template <int NV>
+__device__ __forceinline__ void ld_hilo_ws(const __nv_bfloat16* hi, const __nv_bfloat16* lo, float* x) {
+  if constexpr (NV % 16 == 0) {
+#pragma unroll
+    for (int q = 0; q < NV / 16; ++q) {
+      float h[8], l[8];
+      ld_v8_f32(reinterpret_cast<const float*>(hi + 16 * q), h);  // 16 bf16 as 8 words
+      ld_v8_f32(reinterpret_cast<const float*>(lo + 16 * q), l);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t wh = __float_as_uint(h[k]), wl = __float_as_uint(l[k]);
+        x[16 * q + 2 * k] = __uint_as_float(wh << 16) + __uint_as_float(wl << 16);
+        x[16 * q + 2 * k + 1] = __uint_as_float(wh & 0xffff0000u) + __uint_as_float(wl & 0xffff0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) x[k] = __bfloat162float(hi[k]) + __bfloat162float(lo[k]);
   }
 }
 
@@ -465,13 +488,15 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       if (first && t.bf) {
         // X_0 read from the user's momentum in its own dtype and orientation
         ld_user<NV>(t.m_ptr, t.m_ld, t.m_dtype, t.tall, t.m_vec, row, col0, nvalid, x);
+      } else if (t.split) {
+        ld_hilo_ws<NV>(t.x_cur_op + off, t.x_cur_op + off + t.xlo, x);
       } else {
         ld_f32_ws<NV>(t.x_cur + off, x);
       }
 #pragma unroll
       for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sv * v[k];
       if (t.iter != t.last) {
-        if (t.bf) st_f32_ws<NV>(t.xf_next + off, x);
+        if (t.bf && !t.split) st_f32_ws<NV>(t.xf_next + off, x);
         st_operand<NV>(t, t.xop_next, off, t.xlo, x);
       } else {
         st_user<NV>(t.u_ptr, t.u_ld, t.u_dtype, t.tall, t.u_vec, row, col0, nvalid, x);
@@ -552,7 +577,7 @@ __device__ __forceinline__ void epi_axpy_src(const TileCtx& t, int row, int col0
   for (int k = 0; k < NV; ++k) x[k] = t.a * (sc * x[k]) + sv * v[k];
   if (t.iter != t.last) {
     const int64_t off = ((int64_t)t.z * t.Mo + row) * t.ldn + col0;
-    st_f32_ws<NV>(t.xf_next + off, x);
+    if (!t.split) st_f32_ws<NV>(t.xf_next + off, x);  // split mode: hi + lo is the next step's source
     st_operand<NV>(t, t.xop_next, off, t.xlo, x);
   } else {
     st_user<NV>(t.u_ptr, t.u_ld, t.u_dtype, t.tall, t.u_vec, row, col0, nvalid, x);
@@ -602,6 +627,7 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
   t.aop = g.aop;
   t.bop = g.bop;
   t.x_cur = t.bf ? g.xf[iter & 1] : reinterpret_cast<const float*>(g.xop[iter & 1]);
+  t.x_cur_op = reinterpret_cast<const __nv_bfloat16*>(g.xop[iter & 1]);
   t.xf_next = g.xf[(iter + 1) & 1];
   t.xop_next = g.xop[(iter + 1) & 1];
   const MatDesc& md = *t.md;

@@ -516,6 +516,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       int k = 0;
       uint32_t armed = 0, last_par = 0;
       bool ok = true;
+      const bool hilo = (h.flags & SMUON_NS_SPLIT_BF16) != 0;
       for (int i = t_begin; i < t_end && ok && !h.starve_tc; ++i) {
         int tm, tn;
         const TileCtx t = tile_at(i, tm, tn);
@@ -533,9 +534,16 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           last_par = (last_par & ~(1u << slot)) | (ph << slot);
           const uint32_t dst = src_base + slot * SRC_BYTES;
           const int col = tn * kBN + c * 32;  // wide-form column of the chunk
-          if (!first) tma_load_3d(dst, map, col, tm * BM, t.z, fb);
-          else if (!tall) tma_load_3d(dst, map, col, tm * BM, 0, fb);   // user rows = wide rows
-          else tma_load_3d(dst, map, tm * BM, col, 0, fb);              // user rows = wide columns
+          if (!first && hilo) {  // split mode: X as its bf16 hi part, then its lo part (matrix z + count)
+            tma_load_3d(dst, map, col, tm * BM, t.z, fb);
+            tma_load_3d(dst + SRC_BYTES / 2, map, col, tm * BM, t.z + t.g->count, fb);
+          } else if (!first) {
+            tma_load_3d(dst, map, col, tm * BM, t.z, fb);
+          } else if (!tall) {
+            tma_load_3d(dst, map, col, tm * BM, 0, fb);   // user rows = wide rows
+          } else {
+            tma_load_3d(dst, map, tm * BM, col, 0, fb);   // user rows = wide columns
+          }
         }
       }
       if (!ok) {
@@ -570,6 +578,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         // is in flight while this one is processed (two register sets, the loop unrolled by two).
         const float* ring = reinterpret_cast<const float*>(base_ptr + STAGES * STAGE_BYTES);
         const bool tall = iter == 0 && t.tall;
+        const bool hilo = iter > 0 && t.split;  // the source is X's hi and lo parts, not an f32 master
         auto taddr = [&](int c) {
           return tmem_base + (uint32_t)(acc * kBN + c * 32 + 16 * half) + ((uint32_t)(ew * 32) << 16);
         };
@@ -580,7 +589,24 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
           const float* sp = ring + slot * (SRC_BYTES / 4);
-          if (!tall) {
+          if (hilo) {
+            // split mode, steps >= 1: [128 rows][32 bf16] hi, then lo, with the 64-byte swizzle: 16-byte
+            // unit u of row r sits at u ^ ((r >> 1) & 3); this lane's 16 columns are units 2 half, 2 half + 1
+            const unsigned char* hp = reinterpret_cast<const unsigned char*>(sp) + lrow * 64;
+            const unsigned char* lp = hp + SRC_BYTES / 2;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int u = ((2 * half + q) ^ ((lrow >> 1) & 3)) << 4;
+              const uint4 wh = *reinterpret_cast<const uint4*>(hp + u);
+              const uint4 wl = *reinterpret_cast<const uint4*>(lp + u);
+              const uint32_t hw[4] = {wh.x, wh.y, wh.z, wh.w}, lw[4] = {wl.x, wl.y, wl.z, wl.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                x[8 * q + 2 * j] = __uint_as_float(hw[j] << 16) + __uint_as_float(lw[j] << 16);
+                x[8 * q + 2 * j + 1] = __uint_as_float(hw[j] & 0xffff0000u) + __uint_as_float(lw[j] & 0xffff0000u);
+              }
+            }
+          } else if (!tall) {
             // [128 rows][32 f32] with the 128-byte swizzle: 16-byte unit u of row r sits at u ^ (r & 7)
             const unsigned char* rp = reinterpret_cast<const unsigned char*>(sp) + lrow * 128;
 #pragma unroll

@@ -84,7 +84,7 @@ struct GroupDesc {
   int32_t m, n, count, first_mat;
   int64_t ldn, ldm;       // padded leading dims (elements), multiples of 128
   void* xop[2];           // X operand [count][m][ldn] (bf16, or f32 in FP32 mode)
-  float* xf[2];           // f32 master of X for iterations >= 1 (bf16 modes)
+  float* xf[2];           // f32 master of X for iterations >= 1 (plain BF16 mode; split mode keeps hi + lo)
   float* af;              // f32 A [count][m][ldm]
   void* aop;              // A operand (bf16 modes; == af in FP32 mode)
   void* bop;              // B operand [count][m][ldm]
@@ -101,7 +101,8 @@ struct GroupDesc {
   int32_t tm_x_kw[2];     // X K-major box {64,256}
   int32_t tm_t_k, tm_t_kw; // T K-major boxes {64,128} and {64,256}
   int32_t tm_q_k[2];      // Q K-major box {64,128} (left operand of Q_K X_0)
-  int32_t tm_xf[2];       // f32 masters, box {32,128}, 128B swizzle (B X epilogue source, steps >= 1)
+  int32_t tm_xf[2];       // B X epilogue source of X_i for steps >= 1: the f32 master, box {32,128}, 128B
+                          // swizzle (plain BF16), or the bf16 hi and lo parts, box {32,128}, 64B swizzle (split)
   int32_t tiles_m[ST_COUNT], tiles_n[ST_COUNT], tile_begin[ST_COUNT];
 };
 

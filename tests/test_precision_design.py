@@ -10,7 +10,11 @@ Gaussian momenta of the GPT-2 shapes, against the float64 oracle:
   per-product precision choice passes;
 * the split mode meets them; and with the first two steps plain it still does
   (the normalised singular values start near 1/sqrt(m), so the B X term of an
-  early step is small beside a X), while three plain steps do not.
+  early step is small beside a X), while three plain steps do not;
+* carrying X between steps as its bf16 hi and lo parts alone (x ~ hi + lo,
+  relative error near 2^-17, the operands the split products read anyway)
+  instead of a float32 master keeps the split mode within the criteria, with
+  and without the plain leading steps; the kernels' split mode does this.
 
 The GPU tests check the kernels' modes against the oracle directly."""
 import numpy as np
@@ -33,15 +37,19 @@ def _prod(A, B, split):
     return Ah @ Bh + Ah @ Bl + Al @ Bh
 
 
-def _ns(M, modes):
-    """modes[k] = (gram, poly, axpy) split flags of step k."""
+def _ns(M, modes, hilo_carry=False):
+    """modes[k] = (gram, poly, axpy) split flags of step k; hilo_carry: X is kept
+    between steps as bf16 hi + bf16 lo instead of float32."""
     a, b, c = WL.QUINTIC
     X = (M / (np.sqrt(np.sum(M.astype(np.float64) ** 2)) + 1e-7)).astype(np.float32)
     X = torch.from_numpy(X)
-    for g, p, x in modes:
+    for k, (g, p, x) in enumerate(modes):
         A = _prod(X, X.T.contiguous(), g)
         B = b * A + c * _prod(A, A, p)
         X = a * X + _prod(B, X, x)
+        if hilo_carry and k + 1 < len(modes):
+            hi = _bf(X)
+            X = hi + _bf(X - hi)
     return X.double().numpy()
 
 
@@ -73,6 +81,9 @@ def test_operand_precision_choices(shape):
     lead2 = _ns(M, [PLAIN] * 2 + [SPLIT] * 3)
     assert _passes(lead2, R) and _criteria(lead2, R)[0] < 1e-3
     assert not _passes(_ns(M, [PLAIN] * 3 + [SPLIT] * 2), R)
+    for lead in (0, 2):
+        carried = _ns(M, [PLAIN] * lead + [SPLIT] * (5 - lead), hilo_carry=True)
+        assert _passes(carried, R) and _criteria(carried, R)[0] < 1e-3
 
 
 @pytest.mark.parametrize("shape", [(96, 320), (200, 96)])
