@@ -724,9 +724,24 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
     const EwLayer& L = tb.layers[li];
     const int64_t w = gw - (L.chunk_begin >> 2);
     const int64_t e0 = 32 * w;
-    if (!(active && e0 < L.n)) continue;
-    const int nent = (int)min((int64_t)32, L.n - e0);
+    const bool lane_ok = active && e0 < L.n;
+    const int nent = lane_ok ? (int)min((int64_t)32, L.n - e0) : 0;
     const bool fast = L.vec && nent == 32;
+    // the warp's 32 words (1024 entries) whole and in one contiguous layer: W then moves in coalesced
+    // 512-byte rows (lane l holds entries 8 (32 q + l) .. + 7 of load q), requested before the message
+    // words, and each lane takes its vote bits from the lane that counted them
+    // (every lane executes both warp intrinsics: neither sits behind a lane-dependent condition)
+    const int li0 = __shfl_sync(0xffffffffu, li, 0);
+    const bool warp_fast = __all_sync(0xffffffffu, fast && li == li0);
+    const bool pre_w = kHasW && warp_fast && L.w_dtype == SMUON_BF16;  // warp-uniform
+    const int64_t ebase = e0 - 32 * lane;                                 // the warp's first entry
+    uint4 wq[4];
+    if (pre_w) {
+      const uint4* wp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(L.w) + ebase);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) wq[q] = wp[32 * q + lane];
+    }
+    if (!lane_ok) continue;  // never taken on the warp-wide path (every lane is whole there)
     uint32_t c[kPlanes];  // counts up to M need kPlanes planes (4 for M <= 15, 7 for M <= 64)
 #pragma unroll
     for (int p = 0; p < kPlanes; ++p) c[p] = 0u;
@@ -758,7 +773,48 @@ __device__ __forceinline__ void vote_update_bits(const EwTable& tb) {
     }
     const uint32_t pos = gt, tie = eq & even;
     const float up = tb.eta, down = -tb.eta, tied = tb.eta * (float)tb.tie;
-    if (fast) {
+    if (pre_w) {
+      __nv_bfloat16* wout = reinterpret_cast<__nv_bfloat16*>(L.w) + ebase;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        // entries 8 (32 q + lane) .. + 7: byte (lane & 3) of the word counted by lane 8 q + lane / 4
+        const int src = 8 * q + (lane >> 2), sh = 8 * (lane & 3);
+        const uint32_t pb = __shfl_sync(0xffffffffu, pos, src) >> sh;
+        const uint32_t tbits = __shfl_sync(0xffffffffu, tie, src) >> sh;
+        const uint32_t u[4] = {wq[q].x, wq[q].y, wq[q].z, wq[q].w};
+        float wv[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          wv[2 * k] = __uint_as_float(u[k] << 16);
+          wv[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          wv[k] = __fsub_rn(wv[k], ((pb >> k) & 1u) ? up : (((tbits >> k) & 1u) ? tied : down));
+        uint4 o;
+        o.x = pack_bf16x2_rn(wv[0], wv[1]); o.y = pack_bf16x2_rn(wv[2], wv[3]);
+        o.z = pack_bf16x2_rn(wv[4], wv[5]); o.w = pack_bf16x2_rn(wv[6], wv[7]);
+        reinterpret_cast<uint4*>(wout)[32 * q + lane] = o;
+      }
+      if (L.vote_out) {  // this lane's own 32 entries
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t pb = pos >> (8 * g), tbits = tie >> (8 * g);
+          int8_t v8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v8[k] = (int8_t)(((pb >> k) & 1u) ? 1 : (((tbits >> k) & 1u) ? tb.tie : -1));
+          int8_t* dst = L.vote_out + e0 + 8 * g;
+          if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
+            uint2 pk;
+            memcpy(&pk, v8, 8);
+            *reinterpret_cast<uint2*>(dst) = pk;
+          } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) dst[k] = v8[k];
+          }
+        }
+      }
+    } else if (fast) {
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         float wv[8];
@@ -837,7 +893,8 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
   const int64_t want16 = (tb.total_chunks + 511) / 512;
   const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
   const bool has_w = tb.layers[0].w != nullptr;  // all layers or none (signs and votes only)
-  if (tb.src_dtype == SMUON_BITS) {  // one lane per packed word, four resident CTAs per SM, one wave
+  if (tb.src_dtype == SMUON_BITS) {
+    // one lane per packed word, four resident CTAs per SM, one wave
     const int64_t want = (tb.total_chunks / 4 + 255) / 256;
     const int gridb = (int)std::max<int64_t>(1, std::min<int64_t>(want, 4 * sms));
     if (tb.M <= 15) launch_bits<4>(tb, has_w, gridb, s);
