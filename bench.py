@@ -837,18 +837,20 @@ def gemm_stage_bytes(shapes, workers, iters, c, split, u_bytes):
     """Algorithmic HBM bytes per launch of each Newton-Schulz GEMM stage
     (averaged over the iterations), from the shapes alone: every operand read
     once, the epilogue's source read and its outputs written once. X is the
-    wide m x n form; operands are bf16 (hi and lo parts in split mode), A is
-    f32; between steps X is kept as an f32 master in plain mode and as its hi
-    and lo parts alone in split mode (4 bytes read back as the next step's
-    source either way); the first step's X source is the f32 momentum, the
-    last step writes U (u_bytes per entry)."""
+    wide m x n form; operands are bf16 (hi and lo parts in split mode); A is
+    kept in f32 beside its operand in plain mode and as its hi and lo parts
+    alone in split mode, X likewise between steps (4 bytes read back as the
+    next step's source either way); the first step's X source is the f32
+    momentum, the last step writes U (u_bytes per entry). B's lo part, which a
+    plain leading step does not write, is counted as written."""
     op = 4 if split else 2
     tot = {"gram": 0.0, "poly": 0.0, "axpy": 0.0}
     for r, cc in shapes:
         m, n = min(r, cc), max(r, cc)
         for k in range(iters):
             last = k == iters - 1
-            tot["gram"] += workers * (op * m * n + (4 * m * m + op * m * m if c != 0 else op * m * m))
+            # A as f32 plus its operand (split mode: its hi + lo parts alone), or B = b A directly when c = 0
+            tot["gram"] += workers * (op * m * n + ((0 if split else 4 * m * m) + op * m * m if c != 0 else op * m * m))
             if c != 0:
                 tot["poly"] += workers * (op * m * m + 4 * m * m + op * m * m)
             out = u_bytes * m * n if last else (op if split else 4 + op) * m * n

@@ -40,6 +40,7 @@ struct TileCtx {
   void* u_ptr;                // the user's output
   int64_t u_ld;
   int32_t m_dtype, u_dtype, tall, m_vec, u_vec;
+  int32_t b_lo;               // write B's lo part: not in a plain leading step, whose B X multiplies hi parts only
 };
 
 // Gram, A^2 and the probe produce symmetric m x m results. Only tiles that
@@ -180,26 +181,27 @@ __device__ __forceinline__ void st_op(void* base, int64_t off, int bf, const flo
 }
 
 // one operand element (same encodings as st_operand)
-__device__ __forceinline__ void st_operand1(const TileCtx& t, void* base, int64_t off, int64_t lo_off, float v) {
+__device__ __forceinline__ void st_operand1(const TileCtx& t, void* base, int64_t off, int64_t lo_off, float v,
+                                            bool with_lo = true) {
   if (!t.bf) {
     reinterpret_cast<float*>(base)[off] = v;
     return;
   }
   const __nv_bfloat16 hi = __float2bfloat16_rn(v);
   reinterpret_cast<__nv_bfloat16*>(base)[off] = hi;
-  if (t.split) reinterpret_cast<__nv_bfloat16*>(base)[off + lo_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
+  if (t.split && with_lo) reinterpret_cast<__nv_bfloat16*>(base)[off + lo_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
 }
 
 // operand store: f32, bf16, or bf16 hi at off and lo = bf16(v - hi) at off + lo_off
 template <int NV>
 __device__ __forceinline__ void st_operand(const TileCtx& t, void* base, int64_t off, int64_t lo_off,
-                                           const float* v) {
+                                           const float* v, bool with_lo = true) {
   if (!t.bf) {
     st_f32_ws<NV>(reinterpret_cast<float*>(base) + off, v);
     return;
   }
   st_bf16_ws<NV>(reinterpret_cast<__nv_bfloat16*>(base) + off, v);
-  if (t.split) {
+  if (t.split && with_lo) {
     float lo[NV];
 #pragma unroll
     for (int k = 0; k < NV; ++k) lo[k] = v[k] - __bfloat162float(__float2bfloat16_rn(v[k]));
@@ -379,20 +381,20 @@ __device__ __forceinline__ void sym_store_f32(const TileCtx& t, float* base, int
 
 template <int NV>
 __device__ __forceinline__ void sym_store_operand(const TileCtx& t, void* base, int row, int col0, int nvalid,
-                                                  int ds, int ms, const float* v) {
+                                                  int ds, int ms, const float* v, bool with_lo = true) {
   const int64_t m = t.Mo, ld = t.ldm;
   const int64_t off = ((int64_t)t.z * m + row) * ld + col0;
   if (ds == 0) {
-    st_operand<NV>(t, base, off, t.mlo, v);
+    st_operand<NV>(t, base, off, t.mlo, v, with_lo);
   } else {
 #pragma unroll
     for (int k = 0; k < NV; ++k)
-      if (k >= ds && k < nvalid) st_operand1(t, base, off + k, t.mlo, v[k]);
+      if (k >= ds && k < nvalid) st_operand1(t, base, off + k, t.mlo, v[k], with_lo);
   }
   if (!t.sym) return;
 #pragma unroll
   for (int k = 0; k < NV; ++k)
-    if (k >= ms && k < nvalid) st_operand1(t, base, ((int64_t)t.z * m + col0 + k) * ld + row, t.mlo, v[k]);
+    if (k >= ms && k < nvalid) st_operand1(t, base, ((int64_t)t.z * m + col0 + k) * ld + row, t.mlo, v[k], with_lo);
 }
 
 // largest tm with sym_start(tm) <= r (binary search), then the column tile
@@ -448,7 +450,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       if (t.c != 0.f) {
 #pragma unroll
         for (int k = 0; k < NV; ++k) v[k] *= sc;
-        sym_store_f32<NV>(t, t.af, row, col0, nvalid, ds, ms, v);
+        if (t.af) sym_store_f32<NV>(t, t.af, row, col0, nvalid, ds, ms, v);  // split mode: A's hi + lo serve
         if (t.bf) sym_store_operand<NV>(t, t.aop, row, col0, nvalid, ds, ms, v);
       } else {
         if (t.flags & SMUON_NS_SPECTRAL) {  // f32 A_0 for the largest-eigenvalue estimate
@@ -459,7 +461,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
         }
 #pragma unroll
         for (int k = 0; k < NV; ++k) v[k] = t.b * (sc * v[k]);
-        sym_store_operand<NV>(t, t.bop, row, col0, nvalid, ds, ms, v);
+        sym_store_operand<NV>(t, t.bop, row, col0, nvalid, ds, ms, v, t.b_lo);
         if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, ds, ms, v);
       }
       break;
@@ -468,12 +470,17 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       if (ds >= nvalid) break;
       const int64_t off = ((int64_t)t.z * m + row) * t.ldm + col0;
       float A[NV];
-      ld_f32_ws<NV>(t.af + off, A);
+      if (t.af) {
+        ld_f32_ws<NV>(t.af + off, A);
+      } else {  // split mode: A = hi + lo
+        const __nv_bfloat16* ah = reinterpret_cast<const __nv_bfloat16*>(t.aop);
+        ld_hilo_ws<NV>(ah + off, ah + off + t.mlo, A);
+      }
       // spectral scaling at the first step: A' = r^2 A, so B = b r^2 A + c r^4 A^2 (r = 1 otherwise)
       const float r2 = t.iter == 0 ? t.r * t.r : 1.f;
 #pragma unroll
       for (int k = 0; k < NV; ++k) v[k] = t.b * (r2 * A[k]) + t.c * ((r2 * r2) * v[k]);
-      sym_store_operand<NV>(t, t.bop, row, col0, nvalid, ds, ms, v);
+      sym_store_operand<NV>(t, t.bop, row, col0, nvalid, ds, ms, v, t.b_lo);
       if ((t.flags & SMUON_NS_EMIT_Q) && t.iter == 0) emit_q1<NV>(t, row, col0, nvalid, ds, ms, v);
       break;
     }
@@ -640,6 +647,7 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
   t.tall = md.tall;
   t.m_vec = md.vec & 1;
   t.u_vec = (md.vec >> 1) & 1;
+  t.b_lo = !plain_lead_stage(h.flags, ST_AXPY, iter, g.m);
   return t;
 }
 

@@ -133,7 +133,8 @@ def test_gram_only_rejects_unsupported_requests(L):
 def test_spectral_flag_validation_and_workspace(L):
     """SMUON_NS_SPECTRAL excludes NO_NORMALIZE, EMIT_Q and GRAM_ONLY; its
     workspace adds the Lanczos vectors (66 vectors of m floats per matrix, the
-    tridiagonal coefficients and the f32 Gram matrix even for c = 0)."""
+    tridiagonal coefficients) and, in split mode (whose plain chain keeps A as
+    its hi and lo parts only), the f32 A that the Lanczos run reads."""
     import torch
     import matrix_aware_sign_b200 as S
     m = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 16, 16, S.F32))
@@ -148,7 +149,9 @@ def test_spectral_flag_validation_and_workspace(L):
         base = S.smuon_ns_workspace_bytes(mats, 5, flags)
         spec = S.smuon_ns_workspace_bytes(mats, 5, flags | sp)
         lz = 4 * 66 * (256 + 64 + 200) + 4 * 2 * 64 * 3  # at most 64 Lanczos steps: 65 vectors and w
-        assert base + lz <= spec <= base + lz + 4 * 256 * 4, (base, spec)
+        # f32 A per group [count][m][ldm], ldm = m rounded up to 128
+        af = 4 * (256 * 256 + 64 * 128 + 200 * 256) if flags == S.NS_SPLIT_BF16 else 0
+        assert base + lz + af <= spec <= base + lz + af + 4 * 256 * 4 + 3 * 256, (base, spec)
 
 
 def test_int8_sign_sources_reject_packed_message(L):

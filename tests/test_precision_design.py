@@ -13,8 +13,9 @@ Gaussian momenta of the GPT-2 shapes, against the float64 oracle:
   early step is small beside a X), while three plain steps do not;
 * carrying X between steps as its bf16 hi and lo parts alone (x ~ hi + lo,
   relative error near 2^-17, the operands the split products read anyway)
-  instead of a float32 master keeps the split mode within the criteria, with
-  and without the plain leading steps; the kernels' split mode does this.
+  instead of a float32 master, and taking the b A term from A's hi and lo
+  parts instead of a float32 A, keeps the split mode within the criteria, with
+  and without the plain leading steps; the kernels' split mode does both.
 
 The GPU tests check the kernels' modes against the oracle directly."""
 import numpy as np
@@ -37,19 +38,24 @@ def _prod(A, B, split):
     return Ah @ Bh + Ah @ Bl + Al @ Bh
 
 
+def _hilo(x):
+    hi = _bf(x)
+    return hi + _bf(x - hi)
+
+
 def _ns(M, modes, hilo_carry=False):
     """modes[k] = (gram, poly, axpy) split flags of step k; hilo_carry: X is kept
-    between steps as bf16 hi + bf16 lo instead of float32."""
+    between steps, and A read for the b A term, as bf16 hi + bf16 lo instead of
+    float32."""
     a, b, c = WL.QUINTIC
     X = (M / (np.sqrt(np.sum(M.astype(np.float64) ** 2)) + 1e-7)).astype(np.float32)
     X = torch.from_numpy(X)
     for k, (g, p, x) in enumerate(modes):
         A = _prod(X, X.T.contiguous(), g)
-        B = b * A + c * _prod(A, A, p)
+        B = b * (_hilo(A) if hilo_carry else A) + c * _prod(A, A, p)
         X = a * X + _prod(B, X, x)
         if hilo_carry and k + 1 < len(modes):
-            hi = _bf(X)
-            X = hi + _bf(X - hi)
+            X = _hilo(X)
     return X.double().numpy()
 
 
