@@ -41,7 +41,26 @@ struct TileCtx {
   int64_t u_ld;
   int32_t m_dtype, u_dtype, tall, m_vec, u_vec;
   int32_t b_lo;               // write B's lo part: not in a plain leading step, whose B X multiplies hi parts only
+  float* xs;                  // this warp's 32 x 33 float transpose buffer in shared memory, or null
 };
+
+// The mirrored half of a symmetric stage's 32 x 32 chunk as whole rows: only when the whole warp holds the
+// chunk (all 32 rows inside the matrix, all 32 columns valid, the chunk entirely above the diagonal), a test
+// that every lane evaluates alike, so no lane of the warp has left early and all take part in the transpose.
+__device__ __forceinline__ bool mirror_whole(const TileCtx& t, int row, int col0, int nvalid) {
+  const int row_base = row - (int)(threadIdx.x & 31);  // the warp's first row: lane = row within the chunk
+  return t.xs != nullptr && nvalid == 32 && row_base + 32 <= t.Mo && col0 >= row_base + 32;
+}
+// w[r] = the value at (row_base + r, col0 + lane): lane l then holds row col0 + l of the mirrored chunk
+__device__ __forceinline__ void xpose32(float* xs, const float* v, float* w) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();  // the buffer's previous readers are done
+#pragma unroll
+  for (int k = 0; k < 32; ++k) xs[lane * 33 + k] = v[k];
+  __syncwarp();
+#pragma unroll
+  for (int r = 0; r < 32; ++r) w[r] = xs[r * 33 + lane];
+}
 
 // Gram, A^2 and the probe produce symmetric m x m results. Only tiles that
 // reach the diagonal or lie above it are computed; in them an element
@@ -374,6 +393,15 @@ __device__ __forceinline__ void sym_store_f32(const TileCtx& t, float* base, int
       if (k >= ds && k < nvalid) base[off + k] = v[k];
   }
   if (!t.sym) return;
+  if constexpr (NV == 32) {
+    if (mirror_whole(t, row, col0, nvalid)) {
+      float w[32];
+      xpose32(t.xs, v, w);
+      const int lane = threadIdx.x & 31;
+      st_f32_ws<32>(base + ((int64_t)t.z * m + col0 + lane) * ld + (row - lane), w);
+      return;
+    }
+  }
 #pragma unroll
   for (int k = 0; k < NV; ++k)
     if (k >= ms && k < nvalid) base[((int64_t)t.z * m + col0 + k) * ld + row] = v[k];
@@ -392,6 +420,15 @@ __device__ __forceinline__ void sym_store_operand(const TileCtx& t, void* base, 
       if (k >= ds && k < nvalid) st_operand1(t, base, off + k, t.mlo, v[k], with_lo);
   }
   if (!t.sym) return;
+  if constexpr (NV == 32) {
+    if (mirror_whole(t, row, col0, nvalid)) {
+      float w[32];
+      xpose32(t.xs, v, w);
+      const int lane = threadIdx.x & 31;
+      st_operand<32>(t, base, ((int64_t)t.z * m + col0 + lane) * ld + (row - lane), t.mlo, w, with_lo);
+      return;
+    }
+  }
 #pragma unroll
   for (int k = 0; k < NV; ++k)
     if (k >= ms && k < nvalid) st_operand1(t, base, ((int64_t)t.z * m + col0 + k) * ld + row, t.mlo, v[k], with_lo);
@@ -648,6 +685,7 @@ __device__ __forceinline__ TileCtx make_ctx(const PlanHeader& h, int st, int ite
   t.m_vec = md.vec & 1;
   t.u_vec = (md.vec >> 1) & 1;
   t.b_lo = !plain_lead_stage(h.flags, ST_AXPY, iter, g.m);
+  t.xs = nullptr;
   return t;
 }
 

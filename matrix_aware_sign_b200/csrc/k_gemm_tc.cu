@@ -62,7 +62,9 @@ struct Cfg {
   static constexpr int TMEM_COLS = 2 * kBN;
   static constexpr int NTHREADS = THREADS + (kSrc ? 32 : 0);
   static constexpr int SRC_RING = kSrc ? SRC_SLOTS * SRC_BYTES : 0;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SRC_RING + 1024 /*align*/ + 256 /*barriers*/;
+  // the generic epilogue's transpose buffers (symmetric stages): 32 x 33 floats per epilogue warp
+  static constexpr int XPOSE = kSrc ? 0 : 8 * 32 * 33 * 4;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SRC_RING + 1024 /*align*/ + 256 /*barriers*/ + XPOSE;
 };
 constexpr unsigned long long kWaitCycles = 1ull << 32;  // ~2 s at 2 GHz: the exit drains' budget
 template <int V>
@@ -338,6 +340,9 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   unsigned char* misc = base_ptr + STAGES * STAGE_BYTES + C::SRC_RING + 8 * (2 * STAGES + 5 + 2 * SRC_SLOTS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  float* xpose = reinterpret_cast<float*>(base_ptr + STAGES * STAGE_BYTES + C::SRC_RING + 256);  // after the barriers
+  static_assert(8 * (2 * STAGES + 5 + 2 * SRC_SLOTS) + 8 <= 256, "barriers and flags fit their 256 bytes");
+  static_assert(C::SMEM_BYTES <= 232448, "shared memory per CTA");
 
   // SM pairs: rank 0 issues the MMAs and owns the full and tempty barriers that count both CTAs
   const uint32_t rank = kPair ? cluster_rank() : 0u;
@@ -644,6 +649,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       } else {
         constexpr int CH = kBN / 64;     // 32-column chunks per warp
         // the stage as a compile-time constant: each instantiation keeps only its own context live
+        t.xs = xpose + (warp - 2) * (32 * 33);
         auto chunks = [&](auto tag) {
           constexpr int kSt = decltype(tag)::value;
 #pragma unroll 1
