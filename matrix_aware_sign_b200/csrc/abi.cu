@@ -512,9 +512,10 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     // carries X as its hi and lo operand parts, which the B X epilogue reads back as hi + lo
     if (bf && parts == 1 && K >= 2 && !gram_only) g.xf[1] = B->ptr_at<float>(B->take(nx * 4));
     if (bf && parts == 1 && K >= 3 && !gram_only) g.xf[0] = B->ptr_at<float>(B->take(nx * 4));
-    // f32 A: the Lanczos input (spectral scaling), the Gram-only solve's A iterates and the CacheMuon stages
-    // read it; the plain chain's b A term reads A's hi + lo parts in split mode, the f32 A in the others
-    const bool af_needed = spectral || gram_only || emit_q || parts == 1;
+    // f32 A: the Lanczos input (spectral scaling) and the Gram-only solve's A iterates read it; the b A term of
+    // the A^2 stage reads A's hi + lo parts in split mode (so a CacheMuon fresh solve with the transform rounds
+    // exactly as the plain chain does), the f32 A in the other modes
+    const bool af_needed = spectral || gram_only || parts == 1;
     if ((rq.c != 0.f && af_needed) || spectral) g.af = B->ptr_at<float>(B->take(nm * 4));
     if (rq.c != 0.f) g.aop = bf ? B->ptr_at<void>(B->take(nm * 2 * parts)) : (void*)g.af;
     g.bop = B->ptr_at<void>(B->take(nm * esz * parts));

@@ -257,7 +257,14 @@ __device__ __forceinline__ void ld_user(const void* p, int64_t ld, int32_t dtype
     const int64_t base = (int64_t)row * ld + col0;
     if (vec && nvalid == NV) {
       if (dtype == SMUON_F32) {
-        ld_f32_vec<NV>(reinterpret_cast<const float*>(p) + base, out);
+        const float* q = reinterpret_cast<const float*>(p) + base;
+        if constexpr (NV % 8 == 0) {
+          if ((reinterpret_cast<uintptr_t>(q) & 31) == 0) {  // whole 32-byte sectors when the row piece allows
+            ld_f32_ws<NV>(q, out);
+            return;
+          }
+        }
+        ld_f32_vec<NV>(q, out);
         return;
       }
       if (dtype == SMUON_BF16 && NV % 8 == 0) {
@@ -332,7 +339,14 @@ __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int 
     const int64_t base = (int64_t)row * ld + col0;
     if (vec && nvalid == NV) {
       if (dtype == SMUON_F32) {
-        st_f32_vec<NV>(reinterpret_cast<float*>(p) + base, v);
+        float* q = reinterpret_cast<float*>(p) + base;
+        if constexpr (NV % 8 == 0) {
+          if ((reinterpret_cast<uintptr_t>(q) & 31) == 0) {
+            st_f32_ws<NV>(q, v);
+            return;
+          }
+        }
+        st_f32_vec<NV>(q, v);
         return;
       }
       if (dtype == SMUON_I8) {  // the signs only: four entries per 32-bit word
@@ -342,6 +356,13 @@ __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int 
           pk[k] = (uint32_t)(uint8_t)sign_i8(v[4 * k]) | ((uint32_t)(uint8_t)sign_i8(v[4 * k + 1]) << 8) |
                   ((uint32_t)(uint8_t)sign_i8(v[4 * k + 2]) << 16) | ((uint32_t)(uint8_t)sign_i8(v[4 * k + 3]) << 24);
         uint32_t* q = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(p) + base);
+        if constexpr (NV % 32 == 0) {
+          if ((reinterpret_cast<uintptr_t>(q) & 31) == 0) {  // 32 signs as one 32-byte sector
+#pragma unroll
+            for (int k = 0; k < NV / 32; ++k) st_v8_b32(q + 8 * k, pk + 8 * k);
+            return;
+          }
+        }
         if (NV % 16 == 0) {
 #pragma unroll
           for (int k = 0; k < NV / 16; ++k)
@@ -352,7 +373,14 @@ __device__ __forceinline__ void st_user(void* p, int64_t ld, int32_t dtype, int 
         }
         return;
       }
-      st_bf16_vec<NV>(reinterpret_cast<__nv_bfloat16*>(p) + base, v);
+      __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(p) + base;
+      if constexpr (NV % 16 == 0) {
+        if ((reinterpret_cast<uintptr_t>(qb) & 31) == 0) {
+          st_bf16_ws<NV>(qb, v);
+          return;
+        }
+      }
+      st_bf16_vec<NV>(qb, v);
       return;
     }
 #pragma unroll
