@@ -355,9 +355,21 @@ __device__ __forceinline__ uint32_t pos_halves_bf16(uint32_t w) {
   return (((~le & ~w) | ~nz) >> 15) & 0x00010001u;
 }
 
+// 256-bit accesses for a lane's 16 bf16 entries (32 bytes, whole sectors) where the address allows
+__device__ __forceinline__ void ld_v8_b32(const void* p, uint32_t* u) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void st_v8_b32(void* p, const uint32_t* u) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"l"(p), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+               : "memory");
+}
+
 // vote and update of 8 entries e0..e0+7 from their 4 packed count words, W
-// already loaded into w (when kHasW)
-template <bool kHasW>
+// already loaded into w (when kHasW); kStoreW false leaves the updated w to the caller's store
+template <bool kHasW, bool kStoreW = true>
 __device__ __forceinline__ void vote_apply8(const EwTable& tb, const EwLayer& L, int64_t e0, const uint32_t* cnt,
                                             float* w) {
   int8_t v8[8];
@@ -369,7 +381,7 @@ __device__ __forceinline__ void vote_apply8(const EwTable& tb, const EwLayer& L,
     v8[k] = (int8_t)(c2 > tb.M ? 1 : (c2 < tb.M ? -1 : tb.tie));
     w[k] = __fsub_rn(w[k], c2 > tb.M ? up : (c2 < tb.M ? down : tied));
   }
-  if (kHasW) store8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);  // no W: signs, message and vote only
+  if (kHasW && kStoreW) store8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);  // no W: signs, message and vote only
   if (L.vote_out) {
     int8_t* dst = L.vote_out + e0;
     if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
@@ -479,19 +491,29 @@ __device__ __forceinline__ void vote_update_i8src(const EwTable& tb) {
     if (L.vec && e0 + 16 <= L.n) {
       // W first: the int8 signs need few registers, so W's loads go out together with the workers'
       float w[16];
-      if (kHasW) {
+      __nv_bfloat16* wb = reinterpret_cast<__nv_bfloat16*>(L.w) + e0;
+      const bool w32 = kHasW && L.w_dtype == SMUON_BF16 && (reinterpret_cast<uintptr_t>(wb) & 31) == 0;
+      if (w32) {  // the lane's 16 bf16 as one 32-byte sector
+        uint32_t u[8];
+        ld_v8_b32(wb, u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          w[2 * k] = __uint_as_float(u[k] << 16);
+          w[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+        }
+      } else if (kHasW) {
         load8(L.w, L.w_ld, L.w_dtype, L, e0, 1, w);
         load8(L.w, L.w_ld, L.w_dtype, L, e0 + 8, 1, w + 8);
       }
       uint32_t b[4] = {0u, 0u, 0u, 0u};  // per byte: positive signs of entries e0 + 4i .. e0 + 4i + 3
-      for (int wk0 = 0; wk0 < M; wk0 += 8) {
-        uint4 u[8];
+      for (int wk0 = 0; wk0 < M; wk0 += 4) {  // four workers' 16-byte loads in flight (16 registers)
+        uint4 u[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
           if (wk0 + j < M) u[j] = *reinterpret_cast<const uint4*>(
                                reinterpret_cast<const int8_t*>(tb.srcs[L.src_first + wk0 + j].ptr) + e0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
           if (wk0 + j < M) {
             b[0] += (~u[j].x >> 7) & 0x01010101u;
             b[1] += (~u[j].y >> 7) & 0x01010101u;
@@ -505,8 +527,17 @@ __device__ __forceinline__ void vote_update_i8src(const EwTable& tb) {
         cnt[2 * i] = __byte_perm(b[i], 0u, 0x4140);      // entries 4i, 4i + 1 in the low and high halves
         cnt[2 * i + 1] = __byte_perm(b[i], 0u, 0x4342);  // entries 4i + 2, 4i + 3
       }
-      vote_apply8<kHasW>(tb, L, e0, cnt, w);
-      vote_apply8<kHasW>(tb, L, e0 + 8, cnt + 4, w + 8);
+      if (w32) {
+        vote_apply8<kHasW, false>(tb, L, e0, cnt, w);
+        vote_apply8<kHasW, false>(tb, L, e0 + 8, cnt + 4, w + 8);
+        uint32_t u[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) u[k] = pack_bf16x2_rn(w[2 * k], w[2 * k + 1]);
+        st_v8_b32(wb, u);
+      } else {
+        vote_apply8<kHasW>(tb, L, e0, cnt, w);
+        vote_apply8<kHasW>(tb, L, e0 + 8, cnt + 4, w + 8);
+      }
     } else {
       const int nent = (int)min((int64_t)16, L.n - e0);
       for (int k = 0; k < nent; ++k) {
