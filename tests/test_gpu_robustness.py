@@ -199,3 +199,29 @@ def test_cachemuon_resumes_bit_for_bit(tmp_path):
     torch.cuda.synchronize()
     assert torch.equal(Dc, Da) and torch.equal(resumed.Q, straight.Q)
     assert resumed.counters() == straight.counters()
+
+
+# ------------------------------------------------------------------ first use inside a CUDA graph capture
+def test_first_call_captured_in_a_cuda_graph():
+    """A process's first smuon_ns call may be made inside a CUDA graph capture:
+    building the plan (SM-pair occupancy query, attribute setting) enqueues
+    nothing, the plan upload is a captured kernel, and the replay gives the
+    eager result bit for bit. Run in a fresh process, so the call is the first."""
+    import subprocess
+    import sys
+    code = (
+        "import sys, torch\n"
+        "import matrix_aware_sign_b200 as S, workloads as WL\n"
+        "M=[torch.randn(768, 2304, device='cuda')]; U=[torch.empty(768, 2304, device='cuda')]\n"
+        "ws=S.workspace(S.smuon_ns_workspace_bytes(M, 5, S.NS_SPLIT_BF16), 'cuda')\n"
+        "g=torch.cuda.CUDAGraph(); side=torch.cuda.Stream(); torch.cuda.synchronize()\n"
+        "with torch.cuda.stream(side):\n"
+        "    with torch.cuda.graph(g, stream=side):\n"
+        "        S.smuon_ns(M, U, *WL.QUINTIC, 5, flags=S.NS_SPLIT_BF16, ws=ws)\n"
+        "g.replay(); torch.cuda.synchronize()\n"
+        "U2=[torch.empty(768, 2304, device='cuda')]\n"
+        "S.smuon_ns(M, U2, *WL.QUINTIC, 5, flags=S.NS_SPLIT_BF16); torch.cuda.synchronize()\n"
+        "sys.exit(0 if torch.equal(U[0], U2[0]) else 3)\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, timeout=240, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-2000:]
