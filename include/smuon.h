@@ -136,7 +136,10 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
  * ---------------------------------------------------------------------- */
 #define SMUON_NS_FP32_REF      1u  /* FP32 operands on CUDA cores (reference mode) */
 #define SMUON_NS_SPLIT_BF16    2u  /* accurate mode: every GEMM operand split into bf16 hi + lo
-                                      parts, three tcgen05 MMAs per product (3x tensor work) */
+                                      parts, three tcgen05 MMAs per product (3x tensor work). X between
+                                      steps and A for the b A term are kept as their hi + lo parts alone
+                                      (x ~ hi + lo to about 2^-17 relative); the a X and b A terms are
+                                      formed in float32 from them */
 #define SMUON_NS_NO_NORMALIZE  4u  /* skip the Frobenius normalisation (s = 1) */
 #define SMUON_NS_EMIT_Q        8u  /* also write the CacheMuon transform Q */
 #define SMUON_NS_SIMT_BF16    16u  /* diagnostic: BF16 operands on CUDA cores instead of tcgen05 */

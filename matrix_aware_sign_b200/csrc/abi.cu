@@ -430,7 +430,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   L.off_sched_begin = B->take(sizeof(int32_t) * std::max(begin_n, 1));
   L.off_lz_rows = B->take(sizeof(int32_t) * (B->mats.size() + 1));
   // the B X epilogue reads its X source through a TMA-fed shared-memory ring when every matrix's
-  // momentum is f32 with 16-byte aligned rows (later steps read the f32 masters, always aligned)
+  // momentum is f32 with 16-byte aligned rows (later steps read the workspace's copy of X, always aligned)
   bool axpy_tma = tc && !rq.probe && !gram_only;
   for (const MatDesc& d : B->mats)
     if (!(d.m_dtype == SMUON_F32 && reinterpret_cast<uintptr_t>(d.m_ptr) % 16 == 0 && (d.m_ld * 4) % 16 == 0))

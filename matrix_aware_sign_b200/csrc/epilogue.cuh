@@ -31,9 +31,9 @@ struct TileCtx {
   float* af;                  // f32 A
   void* aop;                  // A operand
   void* bop;                  // B operand
-  const float* x_cur;         // B X, steps >= 1: this step's X (f32 master, or the FP32-mode operand)
+  const float* x_cur;         // B X, steps >= 1: this step's X (plain BF16: f32 master; FP32 mode: the operand)
   const __nv_bfloat16* x_cur_op;  // split mode: this step's X as its hi parts (lo parts xlo further)
-  float* xf_next;             // B X: f32 master of the next X (bf16 modes)
+  float* xf_next;             // B X: f32 master of the next X (plain BF16 mode only)
   void* xop_next;             // B X: operand of the next X
   const void* m_ptr;          // the user's momentum (the first B X step's source)
   int64_t m_ld;
@@ -637,7 +637,7 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
 }
 
 // B X epilogue with its X source already read (x[]): X' = a s X + s B X (first
-// step) or a X + B X, written as the next step's f32 master and operand, or
+// step) or a X + B X, written as the next step's operand (and, in plain BF16, its f32 master), or
 // into the user's U after the last step
 template <int NV>
 __device__ __forceinline__ void epi_axpy_src(const TileCtx& t, int row, int col0, const float* v, float* x) {
