@@ -51,6 +51,14 @@ __device__ __forceinline__ bool mirror_whole(const TileCtx& t, int row, int col0
   const int row_base = row - (int)(threadIdx.x & 31);  // the warp's first row: lane = row within the chunk
   return t.xs != nullptr && nvalid == 32 && row_base + 32 <= t.Mo && col0 >= row_base + 32;
 }
+// A tall matrix's 32 x 32 chunk read or written as user rows through the warp's transpose buffer: only when
+// the whole warp holds it (all 32 wide rows inside the matrix, all 32 wide columns valid), a warp-uniform
+// test, so no lane has left early and all take part
+__device__ __forceinline__ bool tall_whole(const TileCtx& t, int row, int nvalid) {
+  const int row_base = row - (int)(threadIdx.x & 31);
+  return t.xs != nullptr && t.tall && nvalid == 32 && row_base + 32 <= t.Mo;
+}
+
 // w[r] = the value at (row_base + r, col0 + lane): lane l then holds row col0 + l of the mirrored chunk
 __device__ __forceinline__ void xpose32(float* xs, const float* v, float* w) {
   const int lane = threadIdx.x & 31;
@@ -557,7 +565,22 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       const float sv = (first && t.c == 0.f) ? sc * (t.r * t.r) : sc;
       const int64_t off = ((int64_t)t.z * m + row) * t.ldn + col0;
       float x[NV];
-      if (first && t.bf) {
+      bool whole_tall = false;
+      if constexpr (NV == 32) whole_tall = tall_whole(t, row, nvalid);
+      if (first && t.bf && whole_tall && t.m_dtype == SMUON_F32) {
+        // X_0 from a tall f32 momentum: lane l reads user row col0 + l (the wide rows row_base.. as 32
+        // contiguous floats), then the transpose gives each lane its wide row
+        if constexpr (NV == 32) {
+          const int lane = threadIdx.x & 31;
+          const float* urow = reinterpret_cast<const float*>(t.m_ptr) + (int64_t)(col0 + lane) * t.m_ld + (row - lane);
+          float y[32];
+          if (t.m_vec) ld_f32_vec<32>(urow, y);
+          else
+#pragma unroll
+            for (int k = 0; k < 32; ++k) y[k] = urow[k];
+          xpose32(t.xs, y, x);
+        }
+      } else if (first && t.bf) {
         // X_0 read from the user's momentum in its own dtype and orientation
         ld_user<NV>(t.m_ptr, t.m_ld, t.m_dtype, t.tall, t.m_vec, row, col0, nvalid, x);
       } else if (t.split) {
@@ -570,6 +593,14 @@ __device__ __forceinline__ void epi_chunk(const TileCtx& t, int row, int col0, f
       if (t.iter != t.last) {
         if (t.bf && !t.split) st_f32_ws<NV>(t.xf_next + off, x);
         st_operand<NV>(t, t.xop_next, off, t.xlo, x);
+      } else if (whole_tall && t.u_dtype != SMUON_BITS) {
+        // U of a tall matrix: the transpose gives lane l user row col0 + l, written as 32 contiguous entries
+        if constexpr (NV == 32) {
+          const int lane = threadIdx.x & 31;
+          float y[32];
+          xpose32(t.xs, x, y);
+          st_user<32>(t.u_ptr, t.u_ld, t.u_dtype, 0, t.u_vec, col0 + lane, row - lane, 32, y);
+        }
       } else {
         st_user<NV>(t.u_ptr, t.u_ld, t.u_dtype, t.tall, t.u_vec, row, col0, nvalid, x);
       }
