@@ -265,7 +265,14 @@ void schedule_stage(const std::vector<GroupDesc>& groups, int st, int total, int
                     int32_t* ids, int32_t* begin) {
   std::vector<std::vector<int32_t>> per(ctas);
   if (!lpt_stage(st)) {
-    for (int t = 0; t < total; ++t) per[t % ctas].push_back(t);
+    // a last partial wave of r tiles with 2r <= ctas goes out as 2r half tiles, one per list, so it takes half
+    // a tile's time instead of a whole one (B X only: its right operand is MN-major, cut along the columns)
+    const int r = total % ctas;
+    const int whole = (half_tile_stage(st) && r > 0 && 2 * r <= ctas) ? total - r : total;
+    for (int t = 0; t < whole; ++t) per[t % ctas].push_back(t);
+    for (int t = whole; t < total; ++t)
+      for (int side = 0; side < 2; ++side)
+        per[2 * (t - whole) + side].push_back(kHalfTileFlag | (side ? kHalfTileSide : 0) | t);
   } else {
     std::vector<std::pair<double, int32_t>> cost_tile;  // (cost, tile)
     cost_tile.reserve(total);
@@ -414,7 +421,8 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     sched_off[st] = sched_n;
     sched_boff[st] = begin_n;
     if (!tc) continue;
-    sched_n += totals[st];
+    // a B X stage may list up to one extra entry per list (a tile of its last wave cut in two halves)
+    sched_n += totals[st] + (half_tile_stage(st) ? std::min(totals[st], kMaxSchedCtas) : 0);
     begin_n += std::min(totals[st], kMaxSchedCtas) + 1;
   }
 

@@ -386,9 +386,15 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
   const int32_t* tiles = h.sched + h.sched_off[stage];
   const int t_begin = h.sched_begin[h.sched_boff[stage] + list];
   const int t_end = h.sched_begin[h.sched_boff[stage] + list + 1];
-  auto tile_at = [&](int i, int& tm, int& tn) {
-    const TileCtx t = make_ctx(h, stage, iter, tiles[i], tm, tn);
+  // tile i of the list: its tile coordinates, its first column and its width (kBN, or kBN / 2 for a half tile
+  // of a B X stage's last wave)
+  auto tile_at = [&](int i, int& tm, int& tn, int& cbase, int& bw) {
+    const int32_t e = tiles[i];
+    const bool halfw = (e & kHalfTileFlag) != 0;
+    const TileCtx t = make_ctx(h, stage, iter, e & (kHalfTileSide - 1), tm, tn);
     if (kPair) tm = 2 * tm + (int)rank;
+    bw = halfw ? kBN / 2 : kBN;
+    cbase = tn * kBN + ((halfw && (e & kHalfTileSide)) ? kBN / 2 : 0);
     return t;
   };
 
@@ -399,21 +405,23 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
     uint32_t armed = 0, last_par = 0;  // per-stage bit sets for the exit drain
     bool ok = true;
     for (int i = t_begin; i < t_end && ok && !h.starve_tc; ++i) {
-      int tm, tn;
-      const TileCtx t = tile_at(i, tm, tn);
+      int tm, tn, cbase, bw;
+      const TileCtx t = tile_at(i, tm, tn, cbase, bw);
       const int parts = (kSplit && !plain_lead_stage(h.flags, stage, iter, t.g->m)) ? PARTS : 1;
       if (lane == 0) {
         const TcOps o = tc_ops(h, t, iter, B_ROWS);
         tensormap_acquire(o.ma);
         tensormap_acquire(o.mb);
         const int nk = (o.K + BK - 1) / BK;
-        const int brow = tn * kBN + (int)rank * B_ROWS;  // first B row (K-major) or column (MN-major) staged here
+        const int brows = kPair ? bw / 2 : bw;           // B columns (MN-major) this CTA stages for the tile
+        const int brow = cbase + (int)rank * brows;      // first B row (K-major) or column (MN-major) staged here
+        const int b_bytes = brows * BK * 2;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty_bar + 8 * s, ph ^ 1u, abort_flag, budget)) { ok = false; break; }
           const uint32_t fb = full_bar + 8 * s;
           const uint32_t fb_tx = kPair ? at_rank0(fb) : fb;
           if (leader) {  // the pair's full barrier expects both CTAs' bytes
-            mbar_expect_tx(fb, (kPair ? 2 : 1) * parts * (A_BYTES + B_BYTES));
+            mbar_expect_tx(fb, (kPair ? 2 : 1) * parts * (A_BYTES + b_bytes));
             armed |= 1u << s;
             last_par = (last_par & ~(1u << s)) | (ph << s);
           }
@@ -425,7 +433,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
               tma_load_3d_pair(da, o.ma, kb * BK, tm * BM, za, fb_tx);
               if (o.b_mn) {
 #pragma unroll
-                for (int q = 0; q < B_ROWS / 64; ++q) tma_load_3d_pair(db + q * C::MN_BOX, o.mb, brow + 64 * q, kb * BK, zb, fb_tx);
+                for (int q = 0; q < B_ROWS / 64; ++q)
+                  if (q < brows / 64) tma_load_3d_pair(db + q * C::MN_BOX, o.mb, brow + 64 * q, kb * BK, zb, fb_tx);
               } else {
                 tma_load_3d_pair(db, o.mb, kb * BK, brow, zb, fb_tx);
               }
@@ -433,7 +442,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
               tma_load_3d(da, o.ma, kb * BK, tm * BM, za, fb);
               if (o.b_mn) {
 #pragma unroll
-                for (int q = 0; q < B_ROWS / 64; ++q) tma_load_3d(db + q * C::MN_BOX, o.mb, brow + 64 * q, kb * BK, zb, fb);
+                for (int q = 0; q < B_ROWS / 64; ++q)
+                  if (q < brows / 64) tma_load_3d(db + q * C::MN_BOX, o.mb, brow + 64 * q, kb * BK, zb, fb);
               } else {
                 tma_load_3d(db, o.mb, kb * BK, brow, zb, fb);
               }
@@ -467,10 +477,10 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       uint32_t acc_ph = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok; ++i) {
-        int tm, tn;
-        const TileCtx t = tile_at(i, tm, tn);
+        int tm, tn, cbase, bw;
+        const TileCtx t = tile_at(i, tm, tn, cbase, bw);
         const TcOps o = tc_ops(h, t, iter, B_ROWS);
-        const uint32_t idesc = make_idesc((uint32_t)o.b_mn, kBN, kPair ? 2 * BM : BM);
+        const uint32_t idesc = make_idesc((uint32_t)o.b_mn, bw, kPair ? 2 * BM : BM);
         const bool use_lo = kSplit && !plain_lead_stage(h.flags, stage, iter, t.g->m);
         if (!mbar_wait(tempty_bar + 8 * acc, acc_ph ^ 1u, abort_flag, budget)) { ok = false; break; }
         fence_after();
@@ -523,13 +533,13 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       bool ok = true;
       const bool hilo = (h.flags & SMUON_NS_SPLIT_BF16) != 0;
       for (int i = t_begin; i < t_end && ok && !h.starve_tc; ++i) {
-        int tm, tn;
-        const TileCtx t = tile_at(i, tm, tn);
+        int tm, tn, cbase, bw;
+        const TileCtx t = tile_at(i, tm, tn, cbase, bw);
         const bool first = iter == 0;
         const CUtensorMap* map = first ? &h.tmaps[t.md->tm_src] : &h.tmaps[t.g->tm_xf[iter & 1]];
         const bool tall = first && t.md->tall;
         tensormap_acquire(map);
-        for (int c = 0; c < kBN / 32; ++c, ++k) {
+        for (int c = 0; c < bw / 32; ++c, ++k) {
           const int slot = k & 1;
           const uint32_t ph = (uint32_t)(k >> 1) & 1u;
           if (!mbar_wait(sempty_bar + 8 * slot, ph ^ 1u, abort_flag, budget)) { ok = false; break; }
@@ -538,7 +548,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           armed |= 1u << slot;
           last_par = (last_par & ~(1u << slot)) | (ph << slot);
           const uint32_t dst = src_base + slot * SRC_BYTES;
-          const int col = tn * kBN + c * 32;  // wide-form column of the chunk
+          const int col = cbase + c * 32;  // wide-form column of the chunk
           if (!first && hilo) {  // split mode: X as its bf16 hi part, then its lo part (matrix z + count)
             tma_load_3d(dst, map, col, tm * BM, t.z, fb);
             tma_load_3d(dst + SRC_BYTES / 2, map, col, tm * BM, t.z + t.g->count, fb);
@@ -572,8 +582,8 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
     int kc = 0;
     bool ok = true;
     for (int i = t_begin; i < t_end && ok; ++i) {
-      int tm, tn;
-      TileCtx t = tile_at(i, tm, tn);
+      int tm, tn, cbase, bw;
+      TileCtx t = tile_at(i, tm, tn, cbase, bw);
       if (!mbar_wait(tfull_bar + 8 * acc, acc_ph, abort_flag, budget)) { ok = false; break; }
       fence_after();
       float pacc = 0.f;
@@ -624,7 +634,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
 #pragma unroll
             for (int j = 0; j < 16; ++j) x[j] = sp[(16 * half + j) * BM + lrow];
           }
-          epi_axpy_src<16>(t, tm * BM + lrow, tn * kBN + c * 32 + 16 * half, v, x);
+          epi_axpy_src<16>(t, tm * BM + lrow, cbase + c * 32 + 16 * half, v, x);
           __syncwarp();
           if (lane == 0) mbar_arrive_relaxed(sempty_bar + 8 * slot);
           ++kc;
@@ -633,21 +643,21 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
         static_assert((kBN / 32) % 2 == 0, "chunks are processed in pairs");
         uint32_t ra[16], rb[16];
         tmem_ld16_issue(taddr(0), ra);
-        for (int c = 0; c < kBN / 32 && ok; c += 2) {
+        for (int c = 0; c < bw / 32 && ok; c += 2) {
           tmem_ld_wait(ra);
           tmem_ld16_issue(taddr(c + 1), rb);
           if (!process(c, ra)) { ok = false; tmem_ld_wait(rb); break; }
           tmem_ld_wait(rb);
-          if (c + 2 < kBN / 32) tmem_ld16_issue(taddr(c + 2), ra);
+          if (c + 2 < bw / 32) tmem_ld16_issue(taddr(c + 2), ra);
           if (!process(c + 1, rb)) {
             ok = false;
-            if (c + 2 < kBN / 32) tmem_ld_wait(ra);
+            if (c + 2 < bw / 32) tmem_ld_wait(ra);
             break;
           }
         }
         if (!ok) break;
       } else {
-        constexpr int CH = kBN / 64;     // 32-column chunks per warp
+        const int CH = bw / 64;          // 32-column chunks per warp
         // the stage as a compile-time constant: each instantiation keeps only its own context live
         t.xs = xpose + (warp - 2) * (32 * 33);
         auto chunks = [&](auto tag) {
@@ -656,7 +666,7 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
           for (int ch = half * CH; ch < (half + 1) * CH; ++ch) {
             float v[32];
             tmem_ld32(tmem_base + (uint32_t)(acc * kBN + ch * 32) + ((uint32_t)(ew * 32) << 16), v);
-            epi_chunk<32, kSt>(t, tm * BM + lrow, tn * kBN + ch * 32, v, &pacc);
+            epi_chunk<32, kSt>(t, tm * BM + lrow, cbase + ch * 32, v, &pacc);
           }
         };
         switch (stage) {

@@ -55,6 +55,13 @@ __host__ __device__ inline bool plain_lead_stage(uint32_t flags, int st, int ite
 
 enum Mode : int32_t { MODE_TC_BF16 = 0, MODE_SIMT_F32 = 1, MODE_SIMT_BF16 = 2 };
 
+// Tile-list entries of the tensor-core stages: a tile id, or (B X stage only) half of a tile, the left or the
+// right half of its columns, flagged by bit 30 with the side in bit 29. The last partial wave of a B X stage
+// is split into half tiles when at most half the lists would take one (the wave then ends in half the time).
+constexpr int32_t kHalfTileFlag = 1 << 30;
+constexpr int32_t kHalfTileSide = 1 << 29;
+__host__ __device__ inline bool half_tile_stage(int st) { return st == ST_AXPY; }
+
 // one user matrix (user orientation rows x cols); NS runs on the wide form
 // m x n with m = min(rows, cols): a tall matrix is read transposed.
 struct MatDesc {

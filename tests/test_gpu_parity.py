@@ -1062,3 +1062,18 @@ def test_small_matrices_stay_on_single_sm_tiles():
     Ms = [dev(np.random.default_rng(i).standard_normal(s).astype(np.float32)) for i, s in enumerate(shapes)]
     _, names = _ns_out(Ms, shapes, 1, "f32", 2, S.NS_SPLIT_BF16)
     assert names and not any(n.startswith("k_gemm_tc2") for n in names)
+
+
+def test_last_wave_half_tiles_4096():
+    """A B X stage whose last wave would leave most tile lists idle cuts that wave's tiles into half-width
+    tiles (4096^2: 256 pair tiles over the pairs, 512 single-SM tiles over the SMs). Both forms agree bit for
+    bit and meet the criteria against the float64 oracle (split BF16, two plain leading steps)."""
+    rng = np.random.default_rng(4096)
+    Mx = rng.standard_normal((4096, 4096)).astype(np.float32)
+    Md = dev(Mx)
+    flags = S.NS_SPLIT_BF16 | S.ns_plain_lead(2)
+    Up, _ = _ns_out([Md], [(4096, 4096)], 1, "f32", 5, flags)
+    Us, _ = _ns_out([Md], [(4096, 4096)], 1, "f32", 5, flags | S.NS_ONE_SM)
+    assert torch.equal(Up[0], Us[0])
+    ref = O.newton_schulz(Mx.astype(np.float64), *WL.QUINTIC, 5)
+    check_ns_outputs([(host(Up[0]), ref)], 1e-2)
