@@ -336,7 +336,8 @@ def cachemuon_saved(counts, hits, misses, probes, steps, gram_only):
     return 1.0 - cost / (steps * counts["muon"])
 
 
-def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagnose=False, drift=0.01):
+def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagnose=False, drift=0.01,
+                  one_sm=False):
     """M_0 ~ N(0,1); M_{t+1} = M_t + drift N(0,1); every step probes the cached
     transform on the device and runs the fresh solve only when the residual
     exceeds gamma. Reports the hit rate and the orthogonalisation flops saved
@@ -348,7 +349,7 @@ def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagn
     gen = torch.Generator(device="cuda").manual_seed(4242)
     M = torch.randn(shape, device="cuda", generator=gen)
     D = torch.empty(shape, device="cuda")
-    flags = S.NS_SPLIT_BF16 | (S.NS_GRAM_ONLY if gram_only else 0)
+    flags = S.NS_SPLIT_BF16 | (S.NS_GRAM_ONLY if gram_only else 0) | (S.NS_ONE_SM if one_sm else 0)
     cm = S.CacheMuon(M, D, gamma, WL.QUINTIC, iters, flags=flags)
     noise = torch.empty_like(M)
     rows = []
@@ -386,6 +387,7 @@ def run_cachemuon(S, torch, shape, gamma, steps, iters=5, gram_only=False, diagn
            "orth_flops_saved_vs_fresh_symmetric_aware": cachemuon_saved(sym, c["hits"], c["misses"], c["probes"],
                                                                         steps, gram_only),
            "ms_per_step": ms / steps, "fresh_solve": "gram_only" if gram_only else "x_iteration",
+           "fresh_solve_tiles": "single_sm" if one_sm else "sm_pairs",
            "note": "momentum drift generated on the device inside the timed loop"}
     if diagnose:
         vals = torch.stack(rows).cpu().tolist() if rows else []
@@ -1106,7 +1108,8 @@ def main():
             shp, gam = case.split(":")
             r, c = (int(x) for x in shp.split("x"))
             print(json.dumps(run_cachemuon(S, torch, (r, c), float(gam), args.steps, gram_only=args.gram_only,
-                                           diagnose=args.diagnose, drift=args.drift)), flush=True)
+                                           diagnose=args.diagnose, drift=args.drift, one_sm=args.one_sm)),
+                  flush=True)
         return
     if args.only_ns4096:
         flags = S.NS_SPLIT_BF16 if (args.ns_mode or "split") == "split" else 0

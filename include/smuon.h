@@ -163,11 +163,12 @@ int32_t smuon_trace_read(smuon_trace_rec* out, int32_t max_recs);
                                       SMUON_NS_GRAM_ONLY */
 #define SMUON_NS_PLAIN_LEAD_MASK (7u << 12)
 #define SMUON_NS_ONE_SM     0x80u  /* tensor-core stages on single-SM 128 x 256 tiles. Without it, a call
-                                      whose tensor-core stages are the plain Newton-Schulz chain (no
-                                      SMUON_NS_EMIT_Q, SMUON_NS_GRAM_ONLY or probe) and whose matrices all
-                                      have a smaller side of at least 256 runs them on pairs of SMs: 256 x
-                                      256 tiles, clusters of two CTAs, tcgen05 MMAs over both SMs. The
-                                      results agree within the modes' rounding, not bit for bit */
+                                      whose matrices all have a smaller side of at least 256 runs them on
+                                      pairs of SMs: 256 x 256 tiles, clusters of two CTAs, tcgen05 MMAs over
+                                      both SMs. Each output element takes the same products in the same
+                                      order in both forms, so U and Q agree bit for bit. (The CacheMuon
+                                      probe, which takes no flags, always uses pairs when m >= 256; its
+                                      residual sums the same per-warp partials over another tiling.) */
 #define SMUON_NS_TEST_WAIT_EXPIRY 0x8000u  /* failure-detection test, not for use: every tensor-core stage's
                                       copy producers issue nothing and its pipeline waits are limited to
                                       65536 SM clocks (about 2 s otherwise), so each stage's first waits run

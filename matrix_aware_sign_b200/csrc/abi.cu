@@ -384,10 +384,10 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
     if (spectral) lz_floats += (int64_t)(kLanczosSteps + 2) * lz_stride(B->groups[d.group].m);
   }
 
-  // SM pairs (256 x 256 tiles over clusters of two CTAs) for the plain Newton-Schulz chain (Gram, A^2,
-  // B X) when no matrix is too small for a 256-row tile; decided from the flags and shapes alone, so the
-  // sizing pass and the filling pass lay the workspace out alike
-  bool pair = tc && !rq.probe && !emit_q && !gram_only && !(rq.flags & SMUON_NS_ONE_SM);
+  // SM pairs (256 x 256 tiles over clusters of two CTAs) for every tensor-core stage when no matrix is too
+  // small for a 256-row tile; decided from the flags and shapes alone, so the sizing pass and the filling
+  // pass lay the workspace out alike
+  bool pair = tc && !(rq.flags & SMUON_NS_ONE_SM);
   for (const auto& g : B->groups)
     if (g.m < kPairMinM) pair = false;
   const int TBM = pair ? 2 * kTcBM : BM;  // tile height of the tables
@@ -754,12 +754,15 @@ smuon_status launch_gemm(const Plan* d_plan, const PlanHeader& h, int st, int it
       {"k_gemm_tc_split.gram", "k_gemm_tc_split.poly", "k_gemm_tc_split.axpy", "k_gemm_tc_split.qaxpy",
        "k_gemm_tc_split.reuse", "k_gemm_tc_split.probe", "k_gemm_tc_split.aa1", "k_gemm_tc_split.aa2",
        "k_gemm_tc_split.qx"}};
-  // SM pairs: only the plain Newton-Schulz chain's stages
-  static const char* tc2_names[2][3] = {{"k_gemm_tc2.gram", "k_gemm_tc2.poly", "k_gemm_tc2.axpy"},
-                                        {"k_gemm_tc2_split.gram", "k_gemm_tc2_split.poly", "k_gemm_tc2_split.axpy"}};
+  static const char* tc2_names[2][ST_COUNT] = {
+      {"k_gemm_tc2.gram", "k_gemm_tc2.poly", "k_gemm_tc2.axpy", "k_gemm_tc2.qaxpy", "k_gemm_tc2.reuse",
+       "k_gemm_tc2.probe", "k_gemm_tc2.aa1", "k_gemm_tc2.aa2", "k_gemm_tc2.qx"},
+      {"k_gemm_tc2_split.gram", "k_gemm_tc2_split.poly", "k_gemm_tc2_split.axpy", "k_gemm_tc2_split.qaxpy",
+       "k_gemm_tc2_split.reuse", "k_gemm_tc2_split.probe", "k_gemm_tc2_split.aa1", "k_gemm_tc2_split.aa2",
+       "k_gemm_tc2_split.qx"}};
   if (h.mode == MODE_TC_BF16) {
     const bool split = (h.flags & SMUON_NS_SPLIT_BF16) && split_stage(st);
-    const char* name = (h.pair && st <= ST_AXPY) ? tc2_names[split][st] : tc_names[split][st];
+    const char* name = h.pair ? tc2_names[split][st] : tc_names[split][st];
     Launch L(name, SMUON_WORK_FLOPS, issued_flops, s, stage_flops);
     CUDA_TRY(launch_gemm_tc(d_plan, h, st, iter, skip, di.sms, s));
   } else {

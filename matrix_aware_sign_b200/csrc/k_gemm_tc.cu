@@ -691,7 +691,10 @@ __device__ __forceinline__ void gemm_tc_body(const Plan* plan, int stage, int it
       if (!kSrc && stage == ST_PROBE) {  // one partial per epilogue warp: no barrier, fixed order later
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) pacc += __shfl_xor_sync(0xffffffffu, pacc, o2);
-        if (lane == 0) h.probe_partials[kProbeSlots * tiles[i] + (warp - 2)] = pacc;
+        if (lane == 0) {  // slots 0..7: the even (or only) CTA's warps, 8..15: the odd CTA's (zero on one SM)
+          h.probe_partials[kProbeSlots * tiles[i] + (warp - 2) + 8 * (int)rank] = pacc;
+          if (!kPair) h.probe_partials[kProbeSlots * tiles[i] + (warp - 2) + 8] = 0.f;
+        }
       }
       if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
     }

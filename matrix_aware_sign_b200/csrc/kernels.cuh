@@ -90,7 +90,7 @@ __global__ void k_gemm_simt_bf16(const Plan* plan, int stage, int iter, const in
 // tcgen05 kernel entry (host-side launcher lives in k_gemm_tc.cu)
 cudaError_t launch_gemm_tc(const Plan* d_plan, const PlanHeader& h, int stage, int iter,
                            const int32_t* skip, int num_sms, cudaStream_t s);
-constexpr int kProbeSlots = 8;  // residual partial sums per probe tile (one per epilogue warp)
+constexpr int kProbeSlots = 16;  // residual partial sums per probe tile (one per epilogue warp of either SM of a pair)
 constexpr int kTcBM = 128;
 // tile width of the split-BF16 stages: 128 x 256 tiles with two 96 KB ring stages (hi and lo parts of both
 // operands) beat 128 x 128 tiles with three of 64 KB (4096^2, five quintic steps: 3.69 against 4.24 ms)

@@ -254,7 +254,10 @@ def test_sm_pair_choice_is_a_valid_flag_and_sizes_the_tile_tables(L):
         return out.value
 
     big = [(768, 2304), (4096, 4096)]
-    for fl in (0, S.NS_SPLIT_BF16):
+    for fl in (0, S.NS_SPLIT_BF16, S.NS_SPLIT_BF16 | S.NS_EMIT_Q):
         assert ws(big, fl) <= ws(big, fl | S.NS_ONE_SM)
         small = big + [(64, 147)]
         assert ws(small, fl) == ws(small, fl | S.NS_ONE_SM)
+    gram = S.NS_SPLIT_BF16 | S.NS_EMIT_Q | S.NS_GRAM_ONLY  # the CacheMuon stages take pairs too
+    assert ws([(768, 2304)], gram) <= ws([(768, 2304)], gram | S.NS_ONE_SM)
+    assert ws([(200, 700)], gram) == ws([(200, 700)], gram | S.NS_ONE_SM)

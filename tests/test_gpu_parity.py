@@ -1055,6 +1055,75 @@ def test_sm_pairs_equal_single_sm_tiles(out, iters, flags):
         check_ns_outputs([(host(u), r) for u, r in zip(Up, refs)], 1e-2)
 
 
+def _ns_q(M, iters, flags):
+    m = min(M.shape)
+    U = torch.zeros(M.shape, device="cuda")
+    Q = torch.zeros((m, m), dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.trace_enable(True)
+    S.smuon_ns([M], [U], *WL.QUINTIC, iters, flags=flags | S.NS_EMIT_Q, Q_out=[Q], status=st)
+    torch.cuda.synchronize()
+    names = {r["name"].split(".")[0] for r in S.trace_read() if r["name"].startswith("k_gemm")}
+    S.trace_enable(False)
+    assert int(st.item()) == 0
+    return U, Q, names
+
+
+@pytest.mark.parametrize("shape,iters,flags", [
+    ((768, 2304), 5, S.NS_SPLIT_BF16),
+    ((1000, 384), 3, S.NS_SPLIT_BF16),
+    ((512, 300), 2, 0),
+    ((384, 1536), 5, S.NS_SPLIT_BF16 | S.NS_GRAM_ONLY),
+    ((640, 256), 2, S.NS_SPLIT_BF16 | S.NS_GRAM_ONLY),
+])
+def test_cachemuon_stages_on_sm_pairs(shape, iters, flags):
+    """The CacheMuon stages run on pairs of SMs too: the fresh solve with its
+    transform Q (Q X stages beside the X chain, or the Gram-only solve with its
+    A-side stages and U = Q_K X_0) gives U and Q bit for bit as on single-SM
+    tiles, and the oracle's U and Q within the criteria."""
+    M = np.random.default_rng(shape[0] + iters).standard_normal(shape).astype(np.float32)
+    Md = dev(M)
+    Up, Qp, names_p = _ns_q(Md, iters, flags)
+    Us, Qs, names_s = _ns_q(Md, iters, flags | S.NS_ONE_SM)
+    assert names_p and all(n.startswith("k_gemm_tc2") for n in names_p)
+    assert names_s and not any(n.startswith("k_gemm_tc2") for n in names_s)
+    assert torch.equal(Up, Us) and torch.equal(Qp, Qs)
+    if flags & S.NS_SPLIT_BF16:  # plain BF16 operands do not meet the sign criteria (a design choice, not a parity claim)
+        D_ref, Q_ref = O.newton_schulz_with_q(M.astype(np.float64), *WL.QUINTIC, iters)
+        check_ns_outputs([(host(Up), D_ref)], 1e-2)
+        assert rel_fro(host(Qp), Q_ref) < 1e-2
+
+
+@pytest.mark.parametrize("shape", [(256, 640), (1000, 384)])
+def test_cachemuon_probe_on_sm_pairs(shape):
+    """The reuse and probe stages on pairs of SMs (every side at least 256):
+    the reuse output Q X_t and the orthogonality residual, summed from sixteen
+    partials per 256 x 256 tile, agree with the oracle; the accept decision
+    follows the residual on both sides of the threshold."""
+    mom = list(WL.cachemuon_momenta(shape, 2, drift=0.01, seed0=shape[0]))
+    m = min(shape)
+    _, Q_ref = O.newton_schulz_with_q(mom[0], *WL.QUINTIC, 5)
+    Qd = dev(Q_ref.astype(np.float32)).to(torch.bfloat16)
+    Q_used = host(Qd.float()).astype(np.float64)
+    err = torch.zeros(1, device="cuda")
+    acc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cnt = S.new_counters()
+    Dh = torch.zeros(shape, device="cuda")
+    S.trace_enable(True)
+    S.cachemuon_reuse_probe(Qd, dev(mom[1]), Dh, 1e9, err, acc, cnt)
+    torch.cuda.synchronize()
+    names = {r["name"].split(".")[0] for r in S.trace_read() if r["name"].startswith("k_gemm")}
+    S.trace_enable(False)
+    assert names and all(n.startswith("k_gemm_tc2") for n in names)
+    Dh_ref, err_ref = O.cachemuon_probe(Q_used, mom[1])
+    assert rel_fro(host(Dh), Dh_ref) < 1e-2
+    assert abs(err.item() - err_ref) <= 2e-2 * max(err_ref, 1e-3) + 1e-3
+    assert acc.item() == 1
+    S.cachemuon_reuse_probe(Qd, dev(mom[1]), Dh, err_ref / 4, err, acc, cnt)
+    torch.cuda.synchronize()
+    assert acc.item() == 0 and cnt.tolist()[:3] == [1, 1, 2]
+
+
 def test_small_matrices_stay_on_single_sm_tiles():
     """A call with any matrix whose smaller side is below 256 keeps the whole
     batch on single-SM 128 x 256 tiles (a pair's second half would be empty)."""
