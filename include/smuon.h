@@ -293,6 +293,18 @@ smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t 
  * ---------------------------------------------------------------------- */
 #define SMUON_VOTE_POPCOUNT 0u
 #define SMUON_VOTE_INT8     1u
+#define SMUON_VOTE_TEST_WAIT_EXPIRY 0x100u  /* failure-detection test, not for use (OR-ed into vote_kind):
+                                      the bulk-copy form of the 1-bit vote (below) issues no copy and its
+                                      waits are limited to 65536 SM clocks, so they run out: W is left as it
+                                      was and SMUON_DEV_WAIT_TIMEOUT goes to the update status word */
+
+/* The 1-bit vote of a call whose layers all have BF16 W (contiguous, 16-byte aligned, entry counts that
+ * are multiples of 8) and M <= 16 runs in its bulk-copy form: a ring of shared-memory slots, filled by
+ * the bulk-copy engine, holds W and the messages of 8192 entries per slot. Its pipeline waits are bounded
+ * (about 2 s of SM clock); one that runs out ORs SMUON_DEV_WAIT_TIMEOUT into a status word of the library
+ * (per device), and the update is then incomplete. smuon_update_device_status synchronizes the current
+ * device, copies that word to *out and, with clear != 0, resets it. */
+smuon_status smuon_update_device_status(int32_t* out, int32_t clear);
 
 smuon_status smuon_update(const smuon_mat* W, int32_t n_layers,
                           const smuon_mat* U, const smuon_mat* votes, const smuon_mat* dense,

@@ -33,6 +33,7 @@ def ns_plain_lead(k: int) -> int:
         raise ValueError("k must be in 0..7")
     return k << 12
 VOTE_POPCOUNT, VOTE_INT8 = 0, 1
+VOTE_TEST_WAIT_EXPIRY = 0x100  # failure-detection test: the bulk-copy 1-bit vote's waits run out, W unchanged
 LION_MUON_VOTE = 0x100  # lionmuon_step ns_flags: Muon steps as Sign-Muon steps (per-worker NS + vote)
 DEV_NONFINITE_NORM, DEV_WAIT_TIMEOUT = 1, 2
 
@@ -104,6 +105,7 @@ def lib() -> ctypes.CDLL:
             "smuon_update_plan_create": (c_int32, [M, c_int32, M, M, M, c_int32, c_float, c_int8, c_uint32,
                                                    POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p)]),
             "smuon_update_execute": (c_int32, [c_void_p, c_void_p]),
+            "smuon_update_device_status": (c_int32, [POINTER(c_int32), c_int32]),
             "smuon_plan_destroy": (None, [c_void_p]),
             "cachemuon_workspace_bytes": (c_int32, [M, POINTER(c_size_t)]),
             "cachemuon_reuse_probe": (c_int32, [M, M, M, c_float, c_float, c_void_p, c_void_p, c_void_p,
@@ -312,6 +314,13 @@ def smuon_update(W, eta: float, U=None, votes=None, dense=None, M: int = 1, tie_
     vo = None if vote_out is None else (c_void_p * n)(*[_ptr(v) for v in vote_out])
     _check(lib().smuon_update(_mats(W), n, _mats(Uflat), _mats(votes), _mats(dense), M, eta, tie_value,
                               vote_kind, po, vo, _stream(stream)))
+
+
+def update_device_status(clear: bool = True) -> int:
+    """SMUON_DEV_* bits recorded by the vote kernels' bounded waits (synchronizes the device)."""
+    out = c_int32(0)
+    _check(lib().smuon_update_device_status(ctypes.byref(out), 1 if clear else 0))
+    return out.value
 
 
 # ---------------------------------------------------------------- CacheMuon

@@ -1182,6 +1182,8 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
     return fail(SMUON_ERR_INVALID_ARG, "W may be NULL only with the U source and packed_out or vote_out");
   if (U && (M < 1 || M > kMaxWorkers)) return fail(SMUON_ERR_UNSUPPORTED, "M=%d must be in 1..%d", M, kMaxWorkers);
   if (tie_value < -1 || tie_value > 1) return fail(SMUON_ERR_INVALID_ARG, "tie_value must be -1, 0 or 1");
+  const bool test_starve = (vote_kind & SMUON_VOTE_TEST_WAIT_EXPIRY) != 0;
+  vote_kind &= ~SMUON_VOTE_TEST_WAIT_EXPIRY;
   if (vote_kind > SMUON_VOTE_INT8) return fail(SMUON_ERR_INVALID_ARG, "unknown vote_kind %u", vote_kind);
   if (!U && (packed_out || vote_out)) return fail(SMUON_ERR_INVALID_ARG, "packed_out/vote_out need the U source");
   int32_t src_dtype = -1;
@@ -1236,6 +1238,7 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
   proto.tie = tie_value;
   proto.src_dtype = src_dtype;
   proto.eta = eta;
+  proto.test_starve = test_starve ? 1 : 0;
   ex->source = U ? 0 : 1;
   ex->vote_kind = vote_kind;
   ex->tables.clear();
@@ -1260,7 +1263,7 @@ smuon_status run_update(const UpdExec& ex, cudaStream_t s) {
     const EwTable& tb = ex.tables[i];
     const int grid = ew_grid(tb.total_chunks, ex.di);
     if (ex.source == 0) {
-      Launch L(tb.src_dtype == SMUON_BITS ? "k_vote_update_bits"
+      Launch L(tb.src_dtype == SMUON_BITS ? (bits_tma_eligible(tb) ? "k_vote_update_bits_tma" : "k_vote_update_bits")
                : ex.vote_kind == SMUON_VOTE_POPCOUNT ? "k_vote_update_popcount" : "k_vote_update_int8",
                SMUON_WORK_BYTES, ex.bytes[i], s);
       CUDA_TRY(launch_vote_update(tb, ex.vote_kind == SMUON_VOTE_POPCOUNT, grid, ex.di.sms, s));
@@ -1283,6 +1286,13 @@ struct smuon_plan_s {
 };
 
 extern "C" {
+
+smuon_status smuon_update_device_status(int32_t* out, int32_t clear) {
+  if (!out) return fail(SMUON_ERR_INVALID_ARG, "out is NULL");
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(read_update_status(out, clear != 0));
+  return SMUON_OK;
+}
 
 smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
                           const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,

@@ -892,6 +892,333 @@ __global__ void __launch_bounds__(256, 4) k_vote_update_bits(const __grid_consta
   vote_update_bits<kHasW, kPlanes>(tb);
 }
 
+// ---- 1-bit vote and update with the operands staged by the bulk-copy engine
+// The same vote as vote_update_bits, for bf16 W: one elected lane streams each block's W rows (8192 entries,
+// 16 KB) and its M message rows (256 words each) into a ring of shared-memory slots with cp.async.bulk,
+// so the copies of the next slots are in flight while eight consumer warps count, vote and write W back
+// from the current one. Every wait is bounded: when one runs out the CTA records SMUON_DEV_WAIT_TIMEOUT in
+// the module's update status word, stops, waits (bounded) for the copies it issued and returns.
+namespace bitsq {
+constexpr int kWords = 256;               // packed words per block (one per consumer lane)
+constexpr int kEntries = 32 * kWords;     // 8192
+constexpr int kWBytes = 2 * kEntries;     // bf16 W of one block
+constexpr int kSlots = 3;
+constexpr int kConsumers = 8;             // warps
+constexpr int kThreads = 32 * (kConsumers + 1);
+constexpr int kMaxM = 16;
+constexpr unsigned long long kBudget = 1ull << 32;  // about 2 s of SM clock
+constexpr unsigned long long kTestBudget = 1ull << 16;
+__host__ __device__ constexpr int slot_bytes(int M) { return kWBytes + M * kWords * 4; }
+// the subtrahends of four entries for each (+1 bits, zero bits) pair, in eight copies: copy r serves the
+// lanes with lane % 8 == r, and entry i of copy r sits in 16-byte unit 8 i + r, so the eight lanes of a
+// quarter warp (one shared-memory wavefront of 16-byte loads) always read eight different bank groups
+constexpr int kLutBytes = 8 * 256 * 16;
+__host__ __device__ constexpr int smem_bytes(int M) {
+  return kSlots * slot_bytes(M) + kLutBytes + 16 * kSlots + 8 * (kEwMaxLayers + 1) + 16;
+}
+__device__ int32_t g_status;
+
+__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// bounded wait: false when the budget ran out or another role gave up
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned long long budget) {
+  if (bar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (bar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0 && (*abort_flag || clock64() - t0 > budget)) return false;
+  }
+}
+// full adder over bit planes: s = a ^ b ^ c, carry = majority(a, b, c) (one three-input logic op each)
+__device__ __forceinline__ void full_add(uint32_t a, uint32_t b, uint32_t c, uint32_t& s, uint32_t& carry) {
+  s = a ^ b ^ c;
+  carry = (a & b) | (c & (a ^ b));
+}
+// per bit position, the number of set bits among x[0..7] as planes q[0] (1) .. q[3] (8)
+__device__ __forceinline__ void csa_count8(const uint32_t (&x)[8], uint32_t (&q)[4]) {
+  uint32_t sa, ca, sb, cb, sc, cc, se, ce;
+  full_add(x[0], x[1], x[2], sa, ca);   // weight 1 -> 1, 2
+  full_add(x[3], x[4], x[5], sb, cb);
+  full_add(sa, sb, x[6], sc, cc);
+  q[0] = sc ^ x[7];
+  const uint32_t cd = sc & x[7];
+  full_add(ca, cb, cc, se, ce);         // weight 2 -> 2, 4
+  q[1] = se ^ cd;
+  const uint32_t cf = se & cd;
+  q[2] = ce ^ cf;                       // weight 4 -> 4, 8
+  q[3] = ce & cf;
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
+}
+}  // namespace bitsq
+
+template <int kPlanes>
+__global__ void __launch_bounds__(bitsq::kThreads) k_vote_update_bits_tma(const __grid_constant__ EwTable tb) {
+  using namespace bitsq;
+  extern __shared__ __align__(128) unsigned char sm[];
+  const int M = tb.M;
+  const int SB = slot_bytes(M);
+  unsigned char* ring = sm;
+  float4* lut = reinterpret_cast<float4*>(sm + kSlots * SB);
+  const uint32_t bars = saddr(sm + kSlots * SB + kLutBytes);  // full[kSlots], empty[kSlots]
+  int64_t* blk = reinterpret_cast<int64_t*>(sm + kSlots * SB + kLutBytes + 16 * kSlots);  // block prefix per layer
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(blk + kEwMaxLayers + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < kSlots; ++q) {
+      bar_init(bars + 8 * q, 1);
+      bar_init(bars + 8 * (kSlots + q), kConsumers);
+    }
+    int64_t acc = 0;
+    for (int l = 0; l < tb.n_layers; ++l) {
+      blk[l] = acc;
+      acc += (tb.layers[l].words + kWords - 1) / kWords;
+    }
+    blk[tb.n_layers] = acc;
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // lut[p | z << 4]: entry e of four (bit e of p: a +1 vote after the tie rule, bit e of z: a zero vote)
+  // subtracts eta, 0 or -eta
+  for (int t = threadIdx.x; t < 8 * 256; t += blockDim.x) {
+    const int i = t >> 3;
+    float d[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) d[e] = ((i >> (4 + e)) & 1) ? 0.f : (((i >> e) & 1) ? tb.eta : -tb.eta);
+    lut[t] = make_float4(d[0], d[1], d[2], d[3]);
+  }
+  __syncthreads();
+  const int64_t total = blk[tb.n_layers];
+  const unsigned long long budget = tb.test_starve ? kTestBudget : kBudget;
+  // block g: its layer (every role walks the blocks in increasing order, so the layer only moves forward)
+  // and the block's index within that layer
+  auto locate = [&](int64_t g, int& li, int64_t& b) {
+    while (li + 1 < tb.n_layers && blk[li + 1] <= g) ++li;
+    b = g - blk[li];
+  };
+  bool ok = true;
+  if (warp == kConsumers) {
+    // ---------------- producer (one lane)
+    if (lane == 0) {
+      int s = 0, li = 0;
+      uint32_t ph = 0, armed = 0, last_par = 0;
+      for (int64_t g = blockIdx.x; g < total && !tb.test_starve; g += gridDim.x) {
+        if (!bar_wait(bars + 8 * (kSlots + s), ph ^ 1u, abort_flag, budget)) { ok = false; break; }
+        int64_t b;
+        locate(g, li, b);
+        const EwLayer& L = tb.layers[li];
+        const int ne = (int)min((int64_t)kEntries, L.n - b * kEntries);      // a multiple of 8
+        const int nw = (int)min((int64_t)kWords, L.words - b * kWords);      // a multiple of 4
+        const uint32_t full = bars + 8 * s;
+        bar_expect_tx(full, (uint32_t)(2 * ne + M * 4 * nw));
+        armed |= 1u << s;
+        last_par = (last_par & ~(1u << s)) | (ph << s);
+        const uint32_t dst = saddr(ring + (size_t)s * SB);
+        bulk_load(dst, reinterpret_cast<const __nv_bfloat16*>(L.w) + b * kEntries, (uint32_t)(2 * ne), full);
+        for (int k = 0; k < M; ++k)
+          bulk_load(dst + kWBytes + k * kWords * 4,
+                    reinterpret_cast<const uint32_t*>(tb.srcs[L.src_first + k].ptr) + b * kWords,
+                    (uint32_t)(4 * nw), full);
+        if (++s == kSlots) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(&g_status, SMUON_DEV_WAIT_TIMEOUT);
+      }
+      // the copies this lane issued land before the CTA leaves
+      for (int q = 0; q < kSlots; ++q)
+        if (armed & (1u << q)) {
+          const unsigned long long t0 = clock64();
+          while (!bar_try_wait(bars + 8 * q, (last_par >> q) & 1u) && clock64() - t0 < kBudget) {}
+        }
+    }
+  } else {
+    // ---------------- consumers: lane = one packed word of the block (32 entries)
+    const int h = M >> 1;
+    const uint32_t even = (M & 1) ? 0u : 0xffffffffu;
+    // the tie rule folded into two masks per word: ties vote +1 with tie_value 1 (they join the +1 mask), -1
+    // with tie_value -1 (they stay out of it) and 0 with tie_value 0 (W unchanged: the zero mask, which only
+    // an even M can produce; a grid-uniform switch)
+    const bool zero_ties = tb.tie == 0 && !(M & 1);
+    const int j = warp * 32 + lane;
+    int s = 0, li = 0;
+    uint32_t ph = 0;
+    // the current layer's fields, read from the parameter table only when the layer changes
+    int64_t lb = 0, lnext = blk[1], Ln = tb.layers[0].n, Lwords = tb.layers[0].words;
+    __nv_bfloat16* Lw = reinterpret_cast<__nv_bfloat16*>(tb.layers[0].w);
+    int8_t* Lvote = tb.layers[0].vote_out;
+    for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+      if (!bar_wait(bars + 8 * s, ph, abort_flag, budget)) { ok = false; break; }
+      if (g >= lnext) {
+        while (li + 1 < tb.n_layers && blk[li + 1] <= g) ++li;
+        const EwLayer& L = tb.layers[li];
+        lb = blk[li]; lnext = blk[li + 1]; Ln = L.n; Lwords = L.words;
+        Lw = reinterpret_cast<__nv_bfloat16*>(L.w); Lvote = L.vote_out;
+      }
+      const int64_t b = g - lb;
+      const int ne = (int)min((int64_t)kEntries, Ln - b * kEntries);
+      const int nw = (int)min((int64_t)kWords, Lwords - b * kWords);
+      const unsigned char* slot = ring + (size_t)s * SB;
+      const uint32_t* msg = reinterpret_cast<const uint32_t*>(slot + kWBytes);
+      uint32_t c[kPlanes];
+#pragma unroll
+      for (int p = 0; p < kPlanes; ++p) c[p] = 0u;
+      if (j < nw) {
+        for (int k0 = 0; k0 < M; k0 += 8) {
+          uint32_t x[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = (k0 + i < M) ? msg[(k0 + i) * kWords + j] : 0u;
+          // the eight words' count per entry (0..8, four planes) by a carry-save tree of full adders
+          uint32_t q[4];
+          csa_count8(x, q);
+          // added into the running count, plane by plane with the carry rippling upward
+          uint32_t carry = 0u;
+#pragma unroll
+          for (int p = 0; p < kPlanes; ++p) {
+            const uint32_t a = c[p], bq = p < 4 ? q[p] : 0u;
+            c[p] = a ^ bq ^ carry;
+            carry = (a & bq) | (carry & (a ^ bq));
+          }
+        }
+      }
+      uint32_t gt = 0u, eq = 0xffffffffu;
+#pragma unroll
+      for (int p = kPlanes - 1; p >= 0; --p) {
+        if ((h >> p) & 1) {
+          eq &= c[p];
+        } else {
+          gt |= eq & c[p];
+          eq &= ~c[p];
+        }
+      }
+      const uint32_t pos = gt, tie = eq & even;
+      const uint32_t plus = tb.tie > 0 ? (pos | tie) : pos;
+      const uint32_t zero = zero_ties ? tie : 0u;
+      // this warp's 1024 entries of W as four 512-byte rows: lane l takes 16-byte unit 32 q + l (entries
+      // 8 (32 q + l) .. + 7), whose vote bits are byte (l & 3) of the word counted by lane 8 q + l / 4
+      const int wv = min(max(ne - 1024 * warp, 0), 1024);  // valid entries of the warp (a multiple of 8)
+      const uint4* ws = reinterpret_cast<const uint4*>(slot) + 128 * warp;
+      uint4* wg = reinterpret_cast<uint4*>(Lw + b * kEntries + 1024 * warp);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int src = 8 * q + (lane >> 2), sh = 8 * (lane & 3);
+        const uint32_t pb = __shfl_sync(0xffffffffu, plus, src) >> sh;
+        const uint32_t zb = (__shfl_sync(0xffffffffu, zero, src) >> sh) & 0xffu;
+        const int u = 32 * q + lane;
+        if (8 * u < wv) {
+          const uint4 wq = ws[u];
+          const uint32_t w4[4] = {wq.x, wq.y, wq.z, wq.w};
+          // the eight subtrahends from two table entries (entries 0-3 and 4-7 of the unit)
+          const float4 dl = lut[(((pb & 0xfu) | ((zb << 4) & 0xf0u)) << 3) | (lane & 7)];
+          const float4 dh = lut[((((pb >> 4) & 0xfu) | (zb & 0xf0u)) << 3) | (lane & 7)];
+          const float dv[8] = {dl.x, dl.y, dl.z, dl.w, dh.x, dh.y, dh.z, dh.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // entries 2 k (low half) and 2 k + 1 (high half)
+            const float d0 = dv[2 * k], d1 = dv[2 * k + 1];
+            float r0, r1;
+            // both entries' f32 W - d in one two-wide subtraction (round to nearest, per element)
+            asm("{\n .reg .b64 a, b, r;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n"
+                " sub.rn.f32x2 r, a, b;\n mov.b64 {%0, %1}, r;\n}"
+                : "=f"(r0), "=f"(r1)
+                : "f"(__uint_as_float(w4[k] << 16)), "f"(__uint_as_float(w4[k] & 0xffff0000u)), "f"(d0), "f"(d1));
+            o[k] = pack_bf16x2_rn(r0, r1);
+          }
+          wg[u] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      if (Lvote) {  // this lane's own 32 entries, in groups of 8
+        const int nent = min(max(ne - 32 * j, 0), 32);
+        for (int g8 = 0; g8 < nent / 8; ++g8) {
+          const uint32_t pb = pos >> (8 * g8), tbits = tie >> (8 * g8);
+          int8_t v8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v8[k] = (int8_t)(((pb >> k) & 1u) ? 1 : (((tbits >> k) & 1u) ? tb.tie : -1));
+          int8_t* dst = Lvote + b * kEntries + 32 * j + 8 * g8;
+          if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
+            uint2 pk;
+            memcpy(&pk, v8, 8);
+            *reinterpret_cast<uint2*>(dst) = pk;
+          } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) dst[k] = v8[k];
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) bar_arrive(bars + 8 * (kSlots + s));  // the warp's reads of the slot are done
+      if (++s == kSlots) { s = 0; ph ^= 1u; }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      atomicOr(&g_status, SMUON_DEV_WAIT_TIMEOUT);
+    }
+  }
+}
+
+// the TMA-staged form takes a launch whose layers all have bf16 W, contiguous and 16-byte aligned, with
+// entry counts that are multiples of 8 (whole 16-byte rows of W), and M <= 16
+bool bits_tma_eligible(const EwTable& tb) {
+  if (tb.src_dtype != SMUON_BITS || tb.M > bitsq::kMaxM || tb.M < 1 || tb.n_layers < 1) return false;
+  for (int l = 0; l < tb.n_layers; ++l) {
+    const EwLayer& L = tb.layers[l];
+    if (!L.w || L.w_dtype != SMUON_BF16 || !L.vec || L.n % 8 != 0 || L.packed_out) return false;
+    if (reinterpret_cast<uintptr_t>(L.w) % 16) return false;
+    for (int k = 0; k < tb.M; ++k)
+      if (reinterpret_cast<uintptr_t>(tb.srcs[L.src_first + k].ptr) % 16) return false;
+  }
+  return true;
+}
+
+template <int kPlanes>
+static cudaError_t launch_bits_tma(const EwTable& tb, int sms, cudaStream_t s) {
+  const int bytes = bitsq::smem_bytes(tb.M);
+  static bool attr_set[256] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 256 && !attr_set[dev]) {
+    // the largest form (M = 16) once per device
+    cudaError_t e = cudaFuncSetAttribute(k_vote_update_bits_tma<kPlanes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         bitsq::smem_bytes(bitsq::kMaxM));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  int64_t blocks = 0;
+  for (int l = 0; l < tb.n_layers; ++l) blocks += (tb.layers[l].words + bitsq::kWords - 1) / bitsq::kWords;
+  int per_sm = 1;  // as many CTAs as an SM holds with this M's ring
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_vote_update_bits_tma<kPlanes>, bitsq::kThreads, bytes) !=
+          cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks, (int64_t)per_sm * sms));
+  k_vote_update_bits_tma<kPlanes><<<grid, bitsq::kThreads, bytes, s>>>(tb);
+  return cudaGetLastError();
+}
+
+cudaError_t read_update_status(int32_t* out, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, bitsq::g_status, sizeof(int32_t));
+  if (e != cudaSuccess || !clear) return e;
+  const int32_t zero = 0;
+  return cudaMemcpyToSymbol(bitsq::g_status, &zero, sizeof(int32_t));
+}
+
 template <int kPlanes>
 static void launch_bits(const EwTable& tb, bool has_w, int grid, cudaStream_t s) {
   if (has_w) k_vote_update_bits<true, kPlanes><<<grid, 256, 0, s>>>(tb);
@@ -924,6 +1251,10 @@ cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int s
   const int64_t want16 = (tb.total_chunks + 511) / 512;
   const int grid16 = (int)std::max<int64_t>(1, std::min<int64_t>(want16, 3 * sms));
   const bool has_w = tb.layers[0].w != nullptr;  // all layers or none (signs and votes only)
+  if (tb.src_dtype == SMUON_BITS && bits_tma_eligible(tb)) {
+    if (tb.M <= 15) return launch_bits_tma<4>(tb, sms, s);
+    return launch_bits_tma<5>(tb, sms, s);
+  }
   if (tb.src_dtype == SMUON_BITS) {
     // one lane per packed word, four resident CTAs per SM, one wave
     const int64_t want = (tb.total_chunks / 4 + 255) / 256;

@@ -75,6 +75,78 @@ def test_fused_vote_update_from_messages(wdtype, M, tie):
     assert torch.all(Wbig[:, 50:] == 0)
 
 
+def _bits_update(shapes, M, tie, seed, wdtype="bf16", with_votes=True, kind=0):
+    """Random signs packed as messages, the fused update through the C ABI, and
+    the names of the vote kernels that ran."""
+    rng = np.random.default_rng(seed)
+    W = WL.weights(shapes, "normal002", wdtype)
+    tw = torch.bfloat16 if wdtype == "bf16" else torch.float32
+    Wd = [dev(w, tw) for w in W]
+    signs = [[np.where(rng.random(s) < 0.5, 1, -1).astype(np.int8) for _ in range(M)] for s in shapes]
+    msgs = [[S.Bits(dev(O.pack_bits(sg).view(np.int32), torch.int32), *s) for sg in layer]
+            for s, layer in zip(shapes, signs)]
+    votes = [torch.full((r * c,), 9, dtype=torch.int8, device="cuda") for r, c in shapes] if with_votes else None
+    S.trace_enable(True)
+    S.smuon_update(Wd, 0.02, U=msgs, M=M, tie_value=tie, vote_out=votes, vote_kind=kind)
+    torch.cuda.synchronize()
+    names = {r["name"] for r in S.trace_read() if r["name"].startswith("k_vote")}
+    S.trace_enable(False)
+    return W, Wd, signs, votes, names
+
+
+BULK_SHAPES = [(96, 320), (1024, 1032), (8, 1024), (1, 8), (24, 328), (768, 2304)]
+
+
+@pytest.mark.parametrize("M,tie", [(1, 0), (2, -1), (2, 1), (7, 0), (8, 0), (8, 1), (15, 0), (16, -1)])
+def test_bits_vote_bulk_copy_form(M, tie):
+    """Layers of bf16 W whose entry counts are multiples of 8 take the 1-bit vote
+    in its bulk-copy form (8192-entry blocks of W and the M message rows in a
+    shared-memory ring): W and the votes equal the oracle's bit for bit, on
+    layers of one block, of a ragged last block (96 x 320: 3.75 blocks; 24 x
+    328: a last word of 8 valid entries), of one 16-byte row (1 x 8) and of many
+    blocks, for odd and even M with each tie value."""
+    W, Wd, signs, votes, names = _bits_update(BULK_SHAPES, M, tie, seed=M * 10 + tie + 3)
+    assert names == {"k_vote_update_bits_tma"}
+    for i, s in enumerate(BULK_SHAPES):
+        v = O.vote_from_packed([O.pack_bits(sg) for sg in signs[i]], M, s[0] * s[1], tie).reshape(s)
+        np.testing.assert_array_equal(host(votes[i]).reshape(s), v)
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, 0.02, "bf16"))
+
+
+@pytest.mark.parametrize("case", ["m17", "f32", "ragged"])
+def test_bits_vote_other_layers_take_the_word_form(case):
+    """M = 17, f32 W, or a layer whose entry count is not a multiple of 8 keep
+    the whole launch on the word-per-lane kernel; the result is the oracle's."""
+    shapes = [(96, 320), (7, 13)] if case == "ragged" else [(96, 320), (64, 64)]
+    M = 17 if case == "m17" else 8
+    wdtype = "f32" if case == "f32" else "bf16"
+    W, Wd, signs, votes, names = _bits_update(shapes, M, 0, seed=len(case), wdtype=wdtype, with_votes=False)
+    assert names == {"k_vote_update_bits"}
+    for i, s in enumerate(shapes):
+        v = O.vote_from_packed([O.pack_bits(sg) for sg in signs[i]], M, s[0] * s[1], 0).reshape(s)
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, 0.02, wdtype))
+
+
+def test_bits_vote_bounded_wait_expiry():
+    """The bulk-copy vote's waits are bounded: with SMUON_VOTE_TEST_WAIT_EXPIRY
+    the producer issues no copy, every consumer wait runs out after 65536 SM
+    clocks, the call returns with SMUON_DEV_WAIT_TIMEOUT in the update status
+    word and W untouched; the next call is correct again."""
+    shapes = [(96, 320), (8, 1024)]
+    S.update_device_status(clear=True)
+    W, Wd, signs, votes, names = _bits_update(shapes, 8, 0, seed=99, kind=S.VOTE_TEST_WAIT_EXPIRY)
+    assert names == {"k_vote_update_bits_tma"}
+    assert S.update_device_status(clear=True) & S.DEV_WAIT_TIMEOUT
+    for i in range(len(shapes)):
+        np.testing.assert_array_equal(host(Wd[i]), W[i])
+    assert S.update_device_status(clear=True) == 0
+    W, Wd, signs, votes, names = _bits_update(shapes, 8, 0, seed=98)
+    assert S.update_device_status(clear=False) == 0
+    for i, s in enumerate(shapes):
+        v = O.vote_from_packed([O.pack_bits(sg) for sg in signs[i]], 8, s[0] * s[1], 0).reshape(s)
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, 0.02, "bf16"))
+
+
 def test_fused_vote_update_from_messages_many_layers():
     """More layers than one launch's table holds, W = NULL (votes only) and M = 2
     with ties."""
