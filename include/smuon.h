@@ -289,27 +289,28 @@ smuon_status smuon_vote(const uint32_t* packed, const int8_t* signs_i8, int32_t 
  *                    only writes the message and the votes (the input of the
  *                    local polar step, step 5; shapes are taken from U).
  * packed_out and vote_out are host arrays of n_layers device pointers
- * (entries may be NULL) or NULL. M in 1..64.
+ * (entries may be NULL) or NULL. M in 1..64. d_status: nullable device int32
+ * for SMUON_DEV_* bits, as in smuon_ns.
+ *
+ * The 1-bit vote of a call whose layers all have BF16 W (contiguous, 16-byte
+ * aligned, entry counts that are multiples of 8) and M <= 16 runs in its
+ * bulk-copy form: a ring of shared-memory slots, filled by the bulk-copy
+ * engine, holds W and the messages of 8192 entries per slot. Its pipeline
+ * waits are bounded (about 2 s of SM clock); one that runs out ORs
+ * SMUON_DEV_WAIT_TIMEOUT into *d_status, and the update is then incomplete.
  * ---------------------------------------------------------------------- */
 #define SMUON_VOTE_POPCOUNT 0u
 #define SMUON_VOTE_INT8     1u
 #define SMUON_VOTE_TEST_WAIT_EXPIRY 0x100u  /* failure-detection test, not for use (OR-ed into vote_kind):
-                                      the bulk-copy form of the 1-bit vote (below) issues no copy and its
-                                      waits are limited to 65536 SM clocks, so they run out: W is left as it
-                                      was and SMUON_DEV_WAIT_TIMEOUT goes to the update status word */
-
-/* The 1-bit vote of a call whose layers all have BF16 W (contiguous, 16-byte aligned, entry counts that
- * are multiples of 8) and M <= 16 runs in its bulk-copy form: a ring of shared-memory slots, filled by
- * the bulk-copy engine, holds W and the messages of 8192 entries per slot. Its pipeline waits are bounded
- * (about 2 s of SM clock); one that runs out ORs SMUON_DEV_WAIT_TIMEOUT into a status word of the library
- * (per device), and the update is then incomplete. smuon_update_device_status synchronizes the current
- * device, copies that word to *out and, with clear != 0, resets it. */
-smuon_status smuon_update_device_status(int32_t* out, int32_t clear);
+                                      the bulk-copy form of the 1-bit vote issues no copy and its waits
+                                      are limited to 65536 SM clocks, so they run out: W is left as it was
+                                      and SMUON_DEV_WAIT_TIMEOUT goes to d_status */
 
 smuon_status smuon_update(const smuon_mat* W, int32_t n_layers,
                           const smuon_mat* U, const smuon_mat* votes, const smuon_mat* dense,
                           int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
-                          uint32_t* const* packed_out, int8_t* const* vote_out, void* stream);
+                          uint32_t* const* packed_out, int8_t* const* vote_out, int32_t* d_status,
+                          void* stream);
 
 /* ------------------------------------------------------------------------
  * Plan handles: the same calls, prepared once and launched many times.
@@ -335,7 +336,7 @@ smuon_status smuon_update_plan_create(const smuon_mat* W, int32_t n_layers, cons
                                       const smuon_mat* votes, const smuon_mat* dense, int32_t M,
                                       float eta, int8_t tie_value, uint32_t vote_kind,
                                       uint32_t* const* packed_out, int8_t* const* vote_out,
-                                      smuon_plan* out);
+                                      int32_t* d_status, smuon_plan* out);
 smuon_status smuon_update_execute(smuon_plan plan, void* stream);
 void         smuon_plan_destroy(smuon_plan plan);
 

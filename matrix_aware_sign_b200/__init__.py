@@ -95,7 +95,7 @@ def lib() -> ctypes.CDLL:
             "smuon_sign_pack": (c_int32, [M, c_int32, c_void_p, c_void_p, c_void_p]),
             "smuon_vote": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int8, c_void_p, c_void_p]),
             "smuon_update": (c_int32, [M, c_int32, M, M, M, c_int32, c_float, c_int8, c_uint32,
-                                       POINTER(c_void_p), POINTER(c_void_p), c_void_p]),
+                                       POINTER(c_void_p), POINTER(c_void_p), c_void_p, c_void_p]),
             "smuon_ns_static": (c_int32, [M, M, c_int32, M, c_float, c_float, c_float, c_float, c_int32, c_float,
                                           c_uint32, M, c_void_p, c_void_p, c_void_p]),
             "smuon_ns_plan_create": (c_int32, [M, M, c_int32, M, c_float, c_float, c_float, c_float, c_int32,
@@ -103,9 +103,9 @@ def lib() -> ctypes.CDLL:
                                                POINTER(c_void_p)]),
             "smuon_ns_execute": (c_int32, [c_void_p, c_void_p, c_void_p]),
             "smuon_update_plan_create": (c_int32, [M, c_int32, M, M, M, c_int32, c_float, c_int8, c_uint32,
-                                                   POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p)]),
+                                                   POINTER(c_void_p), POINTER(c_void_p), c_void_p,
+                                                   POINTER(c_void_p)]),
             "smuon_update_execute": (c_int32, [c_void_p, c_void_p]),
-            "smuon_update_device_status": (c_int32, [POINTER(c_int32), c_int32]),
             "smuon_plan_destroy": (None, [c_void_p]),
             "cachemuon_workspace_bytes": (c_int32, [M, POINTER(c_size_t)]),
             "cachemuon_reuse_probe": (c_int32, [M, M, M, c_float, c_float, c_void_p, c_void_p, c_void_p,
@@ -270,15 +270,15 @@ class UpdatePlan:
     """smuon_update prepared once; run() enqueues only the kernels."""
 
     def __init__(self, W, eta, U=None, votes=None, dense=None, M=1, tie_value=0, vote_kind=VOTE_POPCOUNT,
-                 packed_out=None, vote_out=None):
+                 packed_out=None, vote_out=None, status=None):
         Uflat = None if U is None else [u for layer in U for u in layer]
-        self.tensors = (None if W is None else list(W), Uflat, votes, dense, packed_out, vote_out)
+        self.tensors = (None if W is None else list(W), Uflat, votes, dense, packed_out, vote_out, status)
         n = len(U) if W is None else len(W)  # W None: signs, message and votes only
         po = None if packed_out is None else (c_void_p * n)(*[_ptr(p) for p in packed_out])
         vo = None if vote_out is None else (c_void_p * n)(*[_ptr(v) for v in vote_out])
         h = c_void_p()
         _check(lib().smuon_update_plan_create(_mats(W), n, _mats(Uflat), _mats(votes), _mats(dense), M, eta,
-                                              tie_value, vote_kind, po, vo, ctypes.byref(h)))
+                                              tie_value, vote_kind, po, vo, _ptr(status), ctypes.byref(h)))
         self.handle = h
 
     def run(self, stream=None):
@@ -305,22 +305,16 @@ def smuon_vote(M: int, N: int, vote, packed=None, signs_i8=None, tie_value: int 
 
 
 def smuon_update(W, eta: float, U=None, votes=None, dense=None, M: int = 1, tie_value: int = 0,
-                 vote_kind: int = VOTE_POPCOUNT, packed_out=None, vote_out=None, stream=None):
+                 vote_kind: int = VOTE_POPCOUNT, packed_out=None, vote_out=None, status=None, stream=None):
     """U is a list over layers of lists over workers (flattened worker-minor).
-    W may be None with U and packed_out / vote_out: signs, message and votes only."""
+    W may be None with U and packed_out / vote_out: signs, message and votes only.
+    status: optional device int32 tensor for SMUON_DEV_* bits."""
     Uflat = None if U is None else [u for layer in U for u in layer]
     n = len(U) if W is None else len(W)
     po = None if packed_out is None else (c_void_p * n)(*[_ptr(p) for p in packed_out])
     vo = None if vote_out is None else (c_void_p * n)(*[_ptr(v) for v in vote_out])
     _check(lib().smuon_update(_mats(W), n, _mats(Uflat), _mats(votes), _mats(dense), M, eta, tie_value,
-                              vote_kind, po, vo, _stream(stream)))
-
-
-def update_device_status(clear: bool = True) -> int:
-    """SMUON_DEV_* bits recorded by the vote kernels' bounded waits (synchronizes the device)."""
-    out = c_int32(0)
-    _check(lib().smuon_update_device_status(ctypes.byref(out), 1 if clear else 0))
-    return out.value
+                              vote_kind, po, vo, _ptr(status), _stream(stream)))
 
 
 # ---------------------------------------------------------------- CacheMuon

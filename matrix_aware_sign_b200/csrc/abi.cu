@@ -1173,7 +1173,8 @@ struct UpdExec {
 
 smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
                             const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
-                            uint32_t* const* packed_out, int8_t* const* vote_out, UpdExec* ex) {
+                            uint32_t* const* packed_out, int8_t* const* vote_out, int32_t* d_status,
+                            UpdExec* ex) {
   if (n_layers < 1) return fail(SMUON_ERR_INVALID_ARG, "n_layers < 1");
   const int nsrc = (U != nullptr) + (votes != nullptr) + (dense != nullptr);
   if (nsrc != 1) return fail(SMUON_ERR_INVALID_ARG, "exactly one of U, votes, dense must be given");
@@ -1239,6 +1240,7 @@ smuon_status prepare_update(const smuon_mat* W, int32_t n_layers, const smuon_ma
   proto.src_dtype = src_dtype;
   proto.eta = eta;
   proto.test_starve = test_starve ? 1 : 0;
+  proto.status = d_status;
   ex->source = U ? 0 : 1;
   ex->vote_kind = vote_kind;
   ex->tables.clear();
@@ -1287,18 +1289,12 @@ struct smuon_plan_s {
 
 extern "C" {
 
-smuon_status smuon_update_device_status(int32_t* out, int32_t clear) {
-  if (!out) return fail(SMUON_ERR_INVALID_ARG, "out is NULL");
-  CUDA_TRY(cudaDeviceSynchronize());
-  CUDA_TRY(read_update_status(out, clear != 0));
-  return SMUON_OK;
-}
-
 smuon_status smuon_update(const smuon_mat* W, int32_t n_layers, const smuon_mat* U, const smuon_mat* votes,
                           const smuon_mat* dense, int32_t M, float eta, int8_t tie_value, uint32_t vote_kind,
-                          uint32_t* const* packed_out, int8_t* const* vote_out, void* stream) {
+                          uint32_t* const* packed_out, int8_t* const* vote_out, int32_t* d_status, void* stream) {
   UpdExec ex;
-  smuon_status st = prepare_update(W, n_layers, U, votes, dense, M, eta, tie_value, vote_kind, packed_out, vote_out, &ex);
+  smuon_status st =
+      prepare_update(W, n_layers, U, votes, dense, M, eta, tie_value, vote_kind, packed_out, vote_out, d_status, &ex);
   if (st != SMUON_OK) return st;
   return run_update(ex, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -1333,13 +1329,13 @@ smuon_status smuon_ns_execute(smuon_plan plan, const int32_t* d_skip_if, void* s
 smuon_status smuon_update_plan_create(const smuon_mat* W, int32_t n_layers, const smuon_mat* U,
                                       const smuon_mat* votes, const smuon_mat* dense, int32_t M, float eta,
                                       int8_t tie_value, uint32_t vote_kind, uint32_t* const* packed_out,
-                                      int8_t* const* vote_out, smuon_plan* out) {
+                                      int8_t* const* vote_out, int32_t* d_status, smuon_plan* out) {
   if (!out) return fail(SMUON_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   smuon_plan_s* p = new smuon_plan_s();
   p->kind = 1;
-  smuon_status st =
-      prepare_update(W, n_layers, U, votes, dense, M, eta, tie_value, vote_kind, packed_out, vote_out, &p->upd);
+  smuon_status st = prepare_update(W, n_layers, U, votes, dense, M, eta, tie_value, vote_kind, packed_out,
+                                   vote_out, d_status, &p->upd);
   if (st != SMUON_OK) {
     delete p;
     return st;
@@ -1622,9 +1618,10 @@ smuon_status lionmuon_step(lionmuon_state* st, int32_t P, float beta1, float bet
   if ((s = enqueue_ns(rq, base + ns_off, total - ns_off, d_status, nullptr, strm)) != SMUON_OK) return s;
   if (vote)  // Sign-Muon step on the orthogonalised G_hat: fused sign / popcount vote / update
     s = smuon_update(st->W, st->n_layers, dirs.data(), nullptr, nullptr, M, eta, tie_value, SMUON_VOTE_POPCOUNT,
-                     nullptr, nullptr, stream);
+                     nullptr, nullptr, d_status, stream);
   else
-    s = smuon_update(st->W, st->n_layers, nullptr, nullptr, dirs.data(), 1, eta, 0, 0, nullptr, nullptr, stream);
+    s = smuon_update(st->W, st->n_layers, nullptr, nullptr, dirs.data(), 1, eta, 0, 0, nullptr, nullptr, d_status,
+                     stream);
   if (s != SMUON_OK) return s;
   st->t = t_next;
   return SMUON_OK;

@@ -897,7 +897,7 @@ __global__ void __launch_bounds__(256, 4) k_vote_update_bits(const __grid_consta
 // 16 KB) and its M message rows (256 words each) into a ring of shared-memory slots with cp.async.bulk,
 // so the copies of the next slots are in flight while eight consumer warps count, vote and write W back
 // from the current one. Every wait is bounded: when one runs out the CTA records SMUON_DEV_WAIT_TIMEOUT in
-// the module's update status word, stops, waits (bounded) for the copies it issued and returns.
+// the caller's d_status, stops, waits (bounded) for the copies it issued and returns.
 namespace bitsq {
 constexpr int kWords = 256;               // packed words per block (one per consumer lane)
 constexpr int kEntries = 32 * kWords;     // 8192
@@ -916,7 +916,6 @@ constexpr int kLutBytes = 8 * 256 * 16;
 __host__ __device__ constexpr int smem_bytes(int M) {
   return kSlots * slot_bytes(M) + kLutBytes + 16 * kSlots + 8 * (kEwMaxLayers + 1) + 16;
 }
-__device__ int32_t g_status;
 
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
@@ -1041,7 +1040,7 @@ __global__ void __launch_bounds__(bitsq::kThreads) k_vote_update_bits_tma(const 
       }
       if (!ok) {
         *abort_flag = 1;
-        atomicOr(&g_status, SMUON_DEV_WAIT_TIMEOUT);
+        if (tb.status) atomicOr(tb.status, SMUON_DEV_WAIT_TIMEOUT);
       }
       // the copies this lane issued land before the CTA leaves
       for (int q = 0; q < kSlots; ++q)
@@ -1169,7 +1168,7 @@ __global__ void __launch_bounds__(bitsq::kThreads) k_vote_update_bits_tma(const 
     }
     if (!ok && lane == 0) {
       *abort_flag = 1;
-      atomicOr(&g_status, SMUON_DEV_WAIT_TIMEOUT);
+      if (tb.status) atomicOr(tb.status, SMUON_DEV_WAIT_TIMEOUT);
     }
   }
 }
@@ -1210,13 +1209,6 @@ static cudaError_t launch_bits_tma(const EwTable& tb, int sms, cudaStream_t s) {
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks, (int64_t)per_sm * sms));
   k_vote_update_bits_tma<kPlanes><<<grid, bitsq::kThreads, bytes, s>>>(tb);
   return cudaGetLastError();
-}
-
-cudaError_t read_update_status(int32_t* out, bool clear) {
-  cudaError_t e = cudaMemcpyFromSymbol(out, bitsq::g_status, sizeof(int32_t));
-  if (e != cudaSuccess || !clear) return e;
-  const int32_t zero = 0;
-  return cudaMemcpyToSymbol(bitsq::g_status, &zero, sizeof(int32_t));
 }
 
 template <int kPlanes>

@@ -44,6 +44,7 @@ struct EwTable {
   int32_t n_layers, M, tie, src_dtype;
   int32_t any_packed;
   int32_t test_starve;     // failure-detection test: the bulk-copy vote's producer issues nothing, short waits
+  int32_t* status;         // nullable: SMUON_DEV_* bits (the bulk-copy vote's bounded waits)
   float eta, beta1, beta2, c1, c2;
   int32_t gen_on;          // LionMuon: gradients drawn in-kernel instead of read (srcs hold no G)
   uint32_t gen_seed;       // key word 0 of worker k = gen_seed + k
@@ -65,7 +66,6 @@ __global__ void k_plan_upload(const __grid_constant__ UploadChunk c);
 __global__ void k_momentum(const Plan* plan, const int32_t* skip);
 __global__ void k_norm_finalize(const Plan* plan, const int32_t* skip);
 cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s);
-cudaError_t read_update_status(int32_t* out, bool clear);  // SMUON_DEV_* bits of the vote kernels
 bool bits_tma_eligible(const EwTable& tb);  // the 1-bit vote of this launch takes its bulk-copy form
 __global__ void k_sign_pack(const __grid_constant__ EwTable tb, uint32_t* packed, int8_t* signs);
 __global__ void k_vote(const uint32_t* packed, const int8_t* signs, int M, int64_t N, int64_t words,

@@ -85,12 +85,12 @@ def test_workspace_query_runs_on_the_host(L):
 def test_update_rejects_bad_source_combinations(L):
     import matrix_aware_sign_b200 as S
     W = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 8, 8, S.F32))
-    assert L.smuon_update(W, 1, None, None, None, 1, 0.01, 0, 0, None, None, None) == -1
-    assert L.smuon_update(W, 1, W, W, None, 1, 0.01, 0, 0, None, None, None) == -1
-    assert L.smuon_update(W, 1, W, None, None, 1, 0.01, 0, 7, None, None, None) == -1
+    assert L.smuon_update(W, 1, None, None, None, 1, 0.01, 0, 0, None, None, None, None) == -1
+    assert L.smuon_update(W, 1, W, W, None, 1, 0.01, 0, 0, None, None, None, None) == -1
+    assert L.smuon_update(W, 1, W, None, None, 1, 0.01, 0, 7, None, None, None, None) == -1
     # no W: only with the U source and an output to write
-    assert L.smuon_update(None, 1, W, None, None, 1, 0.01, 0, 0, None, None, None) == -1
-    assert L.smuon_update(None, 1, None, W, None, 1, 0.01, 0, 0, None, None, None) == -1
+    assert L.smuon_update(None, 1, W, None, None, 1, 0.01, 0, 0, None, None, None, None) == -1
+    assert L.smuon_update(None, 1, None, W, None, 1, 0.01, 0, 0, None, None, None, None) == -1
 
 
 def test_gradient_streams_reject_bad_arguments_before_launch(L):
@@ -162,7 +162,7 @@ def test_int8_sign_sources_reject_packed_message(L):
     W = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 32, 32, S.F32))
     U = (S.SmuonMat * 2)(S.SmuonMat(8192, 8, 32, 32, S.I8), S.SmuonMat(12288, 8, 32, 32, S.I8))
     packed = (ctypes.c_void_p * 1)(16384)
-    assert L.smuon_update(W, 1, U, None, None, 2, 0.01, 0, S.VOTE_INT8, packed, None, None) == -4
+    assert L.smuon_update(W, 1, U, None, None, 2, 0.01, 0, S.VOTE_INT8, packed, None, None, None) == -4
     assert b"packed_out needs F32 or BF16 U" in L.smuon_last_error()
 
 
@@ -220,10 +220,10 @@ def test_update_rejects_a_packed_output_for_message_sources(L):
     W = (S.SmuonMat * 1)(S.SmuonMat(4096, 8, 64, 64, S.F32))
     U = (S.SmuonMat * 2)(S.SmuonMat(8192, 8, 64, 64, S.BITS), S.SmuonMat(12288, 8, 64, 64, S.BITS))
     po = (ctypes.c_void_p * 1)(16384)
-    assert L.smuon_update(W, 1, U, None, None, 2, 0.01, 0, 0, po, None, None) == -1
+    assert L.smuon_update(W, 1, U, None, None, 2, 0.01, 0, 0, po, None, None, None) == -1
     assert b"message" in L.smuon_last_error()
     mixed = (S.SmuonMat * 2)(S.SmuonMat(8192, 8, 64, 64, S.BITS), S.SmuonMat(12288, 8, 64, 64, S.I8))
-    assert L.smuon_update(W, 1, mixed, None, None, 2, 0.01, 0, 0, None, None, None) == -3
+    assert L.smuon_update(W, 1, mixed, None, None, 2, 0.01, 0, 0, None, None, None, None) == -3
 
 
 def test_bits_wrapper_describes_a_message():

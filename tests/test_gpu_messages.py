@@ -75,7 +75,7 @@ def test_fused_vote_update_from_messages(wdtype, M, tie):
     assert torch.all(Wbig[:, 50:] == 0)
 
 
-def _bits_update(shapes, M, tie, seed, wdtype="bf16", with_votes=True, kind=0):
+def _bits_update(shapes, M, tie, seed, wdtype="bf16", with_votes=True, kind=0, status=None):
     """Random signs packed as messages, the fused update through the C ABI, and
     the names of the vote kernels that ran."""
     rng = np.random.default_rng(seed)
@@ -87,7 +87,7 @@ def _bits_update(shapes, M, tie, seed, wdtype="bf16", with_votes=True, kind=0):
             for s, layer in zip(shapes, signs)]
     votes = [torch.full((r * c,), 9, dtype=torch.int8, device="cuda") for r, c in shapes] if with_votes else None
     S.trace_enable(True)
-    S.smuon_update(Wd, 0.02, U=msgs, M=M, tie_value=tie, vote_out=votes, vote_kind=kind)
+    S.smuon_update(Wd, 0.02, U=msgs, M=M, tie_value=tie, vote_out=votes, vote_kind=kind, status=status)
     torch.cuda.synchronize()
     names = {r["name"] for r in S.trace_read() if r["name"].startswith("k_vote")}
     S.trace_enable(False)
@@ -130,18 +130,18 @@ def test_bits_vote_other_layers_take_the_word_form(case):
 def test_bits_vote_bounded_wait_expiry():
     """The bulk-copy vote's waits are bounded: with SMUON_VOTE_TEST_WAIT_EXPIRY
     the producer issues no copy, every consumer wait runs out after 65536 SM
-    clocks, the call returns with SMUON_DEV_WAIT_TIMEOUT in the update status
-    word and W untouched; the next call is correct again."""
+    clocks, the call returns with SMUON_DEV_WAIT_TIMEOUT in d_status and W
+    untouched; the next call is correct again and leaves its status clear."""
     shapes = [(96, 320), (8, 1024)]
-    S.update_device_status(clear=True)
-    W, Wd, signs, votes, names = _bits_update(shapes, 8, 0, seed=99, kind=S.VOTE_TEST_WAIT_EXPIRY)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    W, Wd, signs, votes, names = _bits_update(shapes, 8, 0, seed=99, kind=S.VOTE_TEST_WAIT_EXPIRY, status=st)
     assert names == {"k_vote_update_bits_tma"}
-    assert S.update_device_status(clear=True) & S.DEV_WAIT_TIMEOUT
+    assert int(st.item()) & S.DEV_WAIT_TIMEOUT
     for i in range(len(shapes)):
         np.testing.assert_array_equal(host(Wd[i]), W[i])
-    assert S.update_device_status(clear=True) == 0
-    W, Wd, signs, votes, names = _bits_update(shapes, 8, 0, seed=98)
-    assert S.update_device_status(clear=False) == 0
+    st.zero_()
+    W, Wd, signs, votes, names = _bits_update(shapes, 8, 0, seed=98, status=st)
+    assert int(st.item()) == 0
     for i, s in enumerate(shapes):
         v = O.vote_from_packed([O.pack_bits(sg) for sg in signs[i]], 8, s[0] * s[1], 0).reshape(s)
         np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, 0.02, "bf16"))
