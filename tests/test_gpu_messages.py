@@ -127,6 +127,57 @@ def test_bits_vote_other_layers_take_the_word_form(case):
         np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(W[i], v, 0.02, wdtype))
 
 
+def test_bits_vote_unaligned_w_takes_the_word_form():
+    """A bf16 W that starts 8 bytes past a 16-byte boundary cannot be staged by
+    the bulk-copy engine: the launch keeps the word-per-lane kernel and gives
+    the oracle's result."""
+    shapes, M = [(96, 320)], 8
+    W = WL.weights(shapes, "normal002", "bf16")
+    base = torch.zeros(96 * 320 + 4, dtype=torch.bfloat16, device="cuda")
+    Wv = base[4:].view(96, 320)
+    Wv.copy_(dev(W[0], torch.bfloat16))
+    rng = np.random.default_rng(17)
+    signs = [np.where(rng.random(shapes[0]) < 0.5, 1, -1).astype(np.int8) for _ in range(M)]
+    msgs = [[S.Bits(dev(O.pack_bits(sg).view(np.int32), torch.int32), *shapes[0]) for sg in signs]]
+    S.trace_enable(True)
+    S.smuon_update([Wv], 0.02, U=msgs, M=M)
+    torch.cuda.synchronize()
+    names = {r["name"] for r in S.trace_read() if r["name"].startswith("k_vote")}
+    S.trace_enable(False)
+    assert names == {"k_vote_update_bits"}
+    v = O.vote_from_packed([O.pack_bits(sg) for sg in signs], M, 96 * 320, 0).reshape(shapes[0])
+    np.testing.assert_array_equal(host(Wv), O.update_with_vote(W[0], v, 0.02, "bf16"))
+
+
+def test_bits_vote_plan_in_a_cuda_graph():
+    """A prepared update over 1-bit messages (the bulk-copy form) captured in a
+    CUDA graph and replayed twice equals two oracle updates."""
+    shapes, M = [(768, 2304), (3072, 768)], 8
+    W = WL.weights(shapes, "normal002", "bf16")
+    Wd = [dev(w, torch.bfloat16) for w in W]
+    rng = np.random.default_rng(23)
+    signs = [[np.where(rng.random(s) < 0.5, 1, -1).astype(np.int8) for _ in range(M)] for s in shapes]
+    msgs = [[S.Bits(dev(O.pack_bits(sg).view(np.int32), torch.int32), *s) for sg in layer]
+            for s, layer in zip(shapes, signs)]
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    plan = S.UpdatePlan(Wd, 0.02, U=msgs, M=M, status=st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g.capture_begin()
+        plan.run(stream=s)
+        g.capture_end()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for i, sh in enumerate(shapes):
+        v = O.vote_from_packed([O.pack_bits(sg) for sg in signs[i]], M, sh[0] * sh[1], 0).reshape(sh)
+        w1 = O.update_with_vote(W[i], v, 0.02, "bf16")
+        np.testing.assert_array_equal(host(Wd[i]), O.update_with_vote(w1, v, 0.02, "bf16"))
+
+
 def test_bits_vote_bounded_wait_expiry():
     """The bulk-copy vote's waits are bounded: with SMUON_VOTE_TEST_WAIT_EXPIRY
     the producer issues no copy, every consumer wait runs out after 65536 SM
