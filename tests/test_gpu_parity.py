@@ -1124,6 +1124,58 @@ def test_cachemuon_probe_on_sm_pairs(shape):
     assert acc.item() == 0 and cnt.tolist()[:3] == [1, 1, 2]
 
 
+@pytest.mark.parametrize("flags", [0, S.NS_SPLIT_BF16, S.NS_SPLIT_BF16 | S.ns_plain_lead(2),
+                                   S.NS_SPLIT_BF16 | S.NS_ONE_SM, S.NS_FP32_REF])
+def test_ns_zero_momentum(flags):
+    """All-zero momenta: ||M||_F = 0, X_0 = 0 and every Newton-Schulz product is
+    zero, so U is exactly zero in every mode and tile form, with a clean status;
+    the int8 and 1-bit outputs then hold the sign of zero, +1 (u >= 0), which
+    is also the oracle's."""
+    shapes = [(300, 700), (1000, 384), (64, 96)]
+    outs = ("f32", "i8") if flags & S.NS_FP32_REF else ("f32", "i8", "bits")  # messages need the tensor cores
+    for out in outs:
+        sh = [s for s in shapes if out != "bits" or s[1] % 32 == 0]
+        Ms = [torch.zeros(s, device="cuda") for s in sh]
+        U, _ = _ns_out(Ms, sh, 1, out, 5, flags)
+        for u, s in zip(U, sh):
+            if out == "f32":
+                assert torch.count_nonzero(u).item() == 0
+            elif out == "i8":
+                np.testing.assert_array_equal(host(u), O.sign_extract(np.zeros(s)))
+            else:
+                got = u.cpu().numpy().view(np.uint32)
+                np.testing.assert_array_equal(got, O.pack_bits(O.sign_extract(np.zeros(s))))
+
+
+@pytest.mark.parametrize("flags,iters,tol", [(S.NS_SPLIT_BF16, 5, 1e-2), (S.NS_SPLIT_BF16, 1, 1e-2),
+                                             (S.NS_SPLIT_BF16 | S.ns_plain_lead(2), 5, 1e-2),
+                                             (S.NS_FP32_REF, 5, 1e-3), (S.NS_FP32_REF, 1, 1e-4)])
+@pytest.mark.parametrize("shape", [(300, 700), (1000, 384)])
+def test_ns_rank_one_closed_form(shape, flags, iters, tol):
+    """A rank-one momentum u v^T has one singular value, which the Frobenius
+    scaling sets to s0 = ||M|| / (||M|| + eps); each quintic step maps it to
+    a s + b s^3 + c s^5, so after K steps U = s_K (u/|u|)(v/|v|)^T. Written
+    here from that closed form, not from the oracle. The float32 input is rank
+    one only up to its rounding, and the quintic's slope at zero (a = 3.44)
+    multiplies every such component by up to a^K (about 485 after five steps):
+    the FP32 mode is held to 1e-4 after one step and to 1e-3 after five (it
+    measured 1.5e-4), the split modes to the path's 1e-2."""
+    rng = np.random.default_rng(shape[0] + 3 * iters + flags)
+    u = rng.standard_normal(shape[0]).astype(np.float32)
+    v = rng.standard_normal(shape[1]).astype(np.float32)
+    M = np.outer(u, v).astype(np.float32)
+    Ms = [dev(M)]
+    U, _ = _ns_out(Ms, [shape], 1, "f32", iters, flags)
+    a, b, c = WL.QUINTIC
+    nrm = float(np.linalg.norm(M.astype(np.float64)))
+    sig = nrm / (nrm + 1e-7)
+    for _ in range(iters):
+        sig = a * sig + b * sig ** 3 + c * sig ** 5
+    u64, v64 = u.astype(np.float64), v.astype(np.float64)
+    ref = sig * np.outer(u64 / np.linalg.norm(u64), v64 / np.linalg.norm(v64))
+    check_ns_outputs([(host(U[0]), ref)], tol)
+
+
 def test_small_matrices_stay_on_single_sm_tiles():
     """A call with any matrix whose smaller side is below 256 keeps the whole
     batch on single-SM 128 x 256 tiles (a pair's second half would be empty)."""
