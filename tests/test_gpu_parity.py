@@ -520,6 +520,43 @@ def test_cachemuon_fresh_q_and_probe(shape):
     assert acc.item() == 0 and cnt.tolist()[:3] == [1, 1, 2]
 
 
+def test_cachemuon_schedule_against_the_oracle():
+    """A CacheMuon run on 512 x 1024 through a schedule with a rejection: small
+    drift (the cached transform is accepted), one large jump (rejected: a fresh
+    solve refreshes Q), small drift again (the new Q is accepted). The device's
+    decisions, counters and residuals follow the oracle's own schedule, each
+    step's direction is the oracle's (probe candidate or fresh solve), with gamma
+    placed between the oracle's accepted and rejected residuals."""
+    shape, K = (512, 1024), 5
+    rng = np.random.default_rng(2024)
+    mom = [rng.standard_normal(shape).astype(np.float32)]
+    for drift in (0.01, 0.01, 1.0, 0.01):
+        mom.append((mom[-1] + np.float32(drift) * rng.standard_normal(shape).astype(np.float32)).astype(np.float32))
+    ref, _ = O.cachemuon_run(mom, np.inf, WL.QUINTIC, K)  # every probe's residual against the first Q
+    errs_small, err_jump = [ref[t][2] for t in (1, 2)], ref[3][2]
+    gamma = float(np.sqrt(max(errs_small) * err_jump))
+    assert err_jump > 1.5 * max(errs_small)  # a clear gap, so rounding cannot move a decision
+    ref, _ = O.cachemuon_run(mom, gamma, WL.QUINTIC, K)
+    assert [r[1] for r in ref] == [False, True, True, False, True]
+    Md = dev(mom[0])
+    D = torch.zeros(shape, device="cuda")
+    cm = S.CacheMuon(Md, D, gamma, WL.QUINTIC, K, flags=S.NS_SPLIT_BF16)
+    for t in range(len(mom)):
+        if t:
+            Md.copy_(dev(mom[t]))
+        cm.step()
+        torch.cuda.synchronize()
+        D_ref, acc_ref, err_ref = ref[t]
+        assert bool(cm.accept.item()) == acc_ref
+        if t:
+            assert abs(cm.err.item() - err_ref) <= 2e-2 * err_ref + 1e-3
+        if acc_ref:
+            assert rel_fro(host(D), D_ref) < 1e-2
+        else:
+            check_ns_outputs([(host(D), D_ref)], 1e-2)
+    assert cm.counters() == {"hits": 3, "misses": 2, "probes": 4}
+
+
 def test_cachemuon_first_step_and_skip():
     shape = (128, 192)
     M = next(WL.cachemuon_momenta(shape, 1, seed0=5))
