@@ -493,7 +493,13 @@ def default_ns_mode(args):
 
 
 def plain_lead_of(args):
-    return args.plain_lead if args.plain_lead is not None else DEFAULT_PLAIN_LEAD
+    """Plain leading steps of the split mode: the default two, none with spectral scaling (its s_max = 1 start
+    leaves no step whose B X term is small), or --plain-lead as given."""
+    if args.plain_lead is not None:
+        if args.plain_lead and getattr(args, "spectral", False):
+            raise SystemExit("--plain-lead does not combine with --spectral")
+        return args.plain_lead
+    return 0 if getattr(args, "spectral", False) else DEFAULT_PLAIN_LEAD
 
 
 def describe(name, ns_mode, local_polar, spectral=False, plain_lead=0, sign_out="i8"):
@@ -791,11 +797,15 @@ def rollup(S, recs, peaks, t_peak):
     for r in recs:
         kname = r["name"].split(".")[0]  # stage-qualified names ("k_gemm_tc.axpy") roll up into their kernel
         for key, table in ((kname, by), (r["name"], stages)):
-            d = table.setdefault(key, {"ms": 0.0, "work": 0.0, "nominal": 0.0, "n": 0, "kind": r["kind"]})
+            d = table.setdefault(key, {"ms": 0.0, "work": 0.0, "nominal": 0.0, "n": 0, "kind": r["kind"],
+                                       "ms_known": 0.0, "n_known": 0})
             d["ms"] += max(r["ms"], 0.0)
             d["work"] += r["work"]
             d["nominal"] += r["nominal"]
             d["n"] += 1
+            if r["work"] > 0:  # launches whose work the library states (a later Lanczos step's is data-dependent)
+                d["ms_known"] += max(r["ms"], 0.0)
+                d["n_known"] += 1
     kernels = {}
     total_ms = sum(d["ms"] for d in by.values()) or 1.0
     for name, d in by.items():
@@ -807,7 +817,11 @@ def rollup(S, recs, peaks, t_peak):
             e["frac"] = e["achieved"] / t_peak
             e["frac_issued"] = e["achieved_issued"] / t_peak
         else:
-            e.update(achieved=d["work"] / secs / 1e9 if secs > 0 else 0.0, unit="GB/s")
+            rated = d["ms"]
+            if 0 < d["n_known"] < d["n"]:  # rate only the launches whose bytes are known
+                rated = d["ms_known"]
+                e["rated_launches"] = d["n_known"]
+            e.update(achieved=d["work"] / (rated / 1e3) / 1e9 if rated > 0 else 0.0, unit="GB/s")
             e["frac"] = e["achieved"] / peaks["hbm_gbs"]
         kernels[name] = e
     stage_detail = {k: {"launches": d["n"], "ms_per_launch": d["ms"] / max(d["n"], 1),

@@ -43,3 +43,33 @@ def test_committed_traffic_entries_name_existing_sources_and_profiles():
         # a stale hash makes the bench report null, never a number taken on other code
         got = bench.load_traffic(name)
         assert got in (None, e["bytes_per_launch"])
+
+
+def test_spectral_scaling_runs_without_plain_leading_steps():
+    """The split mode's default two plain leading steps assume the Frobenius start (normalised singular values
+    near 1/sqrt(m)); with spectral scaling the library rejects them, so the bench drops them by default and
+    refuses an explicit request."""
+    import pytest
+
+    assert bench.plain_lead_of(bench.parse_args([])) == bench.DEFAULT_PLAIN_LEAD
+    assert bench.plain_lead_of(bench.parse_args(["--spectral"])) == 0
+    assert bench.plain_lead_of(bench.parse_args(["--spectral", "--plain-lead", "0"])) == 0
+    with pytest.raises(SystemExit):
+        bench.plain_lead_of(bench.parse_args(["--spectral", "--plain-lead", "2"]))
+
+
+def test_rollup_rates_only_launches_with_known_bytes():
+    """A later Lanczos A·v launch reads only the matrices still iterating, so the library states no bytes
+    for it: the kernel's rate is the stated bytes over the stated launches' time, not over all of them."""
+    import types
+
+    S = types.SimpleNamespace(WORK_FLOPS=0, WORK_BYTES=1)  # the library's trace kinds
+    recs = [{"name": "k_lz_matvec", "kind": 1, "work": 1e9, "nominal": 0.0, "ms": 0.2},
+            {"name": "k_lz_matvec", "kind": 1, "work": 0.0, "nominal": 0.0, "ms": 0.1},
+            {"name": "k_lz_matvec", "kind": 1, "work": 0.0, "nominal": 0.0, "ms": 0.1},
+            {"name": "k_momentum", "kind": 1, "work": 2e9, "nominal": 0.0, "ms": 0.4}]
+    _, kernels, _ = bench.rollup(S, recs, {"hbm_gbs": 6650.0}, 1590.0)
+    lz = kernels["k_lz_matvec"]
+    assert lz["launches"] == 3 and lz["rated_launches"] == 1
+    assert abs(lz["achieved"] - 5000.0) < 1e-6  # 1 GB in 0.2 ms
+    assert abs(kernels["k_momentum"]["achieved"] - 5000.0) < 1e-6 and "rated_launches" not in kernels["k_momentum"]
