@@ -489,7 +489,7 @@ smuon_status build_plan(const NsRequest& rq, char* base, Builder* B) {
   }
   L.off_tmaps = B->take(sizeof(CUtensorMap) * std::max(L.n_tmaps, 1));
   L.plan_bytes = (size_t)round_up((int64_t)B->cursor, 256);
-  L.off_partials = B->take(sizeof(float) * std::max(mom_tiles, 1));
+  L.off_partials = B->take(sizeof(float) * kMomSlots * std::max(mom_tiles, 1));
   L.off_scale = B->take(sizeof(float) * B->mats.size());
   L.off_probe = B->take(sizeof(float) * kProbeSlots * std::max(totals[ST_PROBE], 1));
   L.off_rscale = B->take(sizeof(float) * B->mats.size());
@@ -936,7 +936,7 @@ smuon_status run_ns(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
       CUDA_TRY(cudaGetLastError());
     }
     const int warps_per_block = 8;
-    Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * h.total_mom_tiles, s);
+    Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * kMomSlots * h.total_mom_tiles, s);
     k_norm_finalize<<<(h.n_mats + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(ex.d_plan,
                                                                                                           skip);
     CUDA_TRY(cudaGetLastError());

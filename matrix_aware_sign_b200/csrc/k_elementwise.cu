@@ -69,8 +69,7 @@ __device__ __forceinline__ void put_x0_4(const GroupDesc& g, int bf, int split, 
 __global__ void __launch_bounds__(256, 4) k_momentum(const Plan* plan, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
-  __shared__ float tile[64][65];
-  __shared__ float red[8];
+  __shared__ float tile[64][65];  // the transpose of a tall matrix's tile
   const int bf = (h.mode != MODE_SIMT_F32);
   const int split = (h.flags & SMUON_NS_SPLIT_BF16) != 0;
   const int total = h.total_mom_tiles;
@@ -147,7 +146,7 @@ __global__ void __launch_bounds__(256, 4) k_momentum(const Plan* plan, const int
           if (!md.tall) put_x0(g, bf, split, ((int64_t)md.z * m + r) * g.ldn + c, val);
         }
         ss = fmaf(val, val, ss);
-        tile[rr][tx] = val;
+        if (md.tall) tile[rr][tx] = val;
       }
     }
     if (md.tall) {
@@ -158,19 +157,13 @@ __global__ void __launch_bounds__(256, 4) k_momentum(const Plan* plan, const int
         const int c = c0 + cc, r = r0 + tx;
         if (r < md.rows && c < md.cols) put_x0(g, bf, split, ((int64_t)md.z * m + c) * g.ldn + r, tile[tx][cc]);
       }
+      __syncthreads();  // every warp has read the tile before any writes the next one
     }
-    // deterministic block reduction of the tile's sum of squares
+    // the tile's sum of squares as one partial per warp (no block barrier), summed in a fixed order by
+    // k_norm_finalize
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float tot = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) tot += red[w];
-      partials[t] = tot;
-    }
-    __syncthreads();
+    if ((threadIdx.x & 31) == 0) partials[kMomSlots * t + (int)(threadIdx.x >> 5)] = ss;
   }
 }
 
@@ -183,7 +176,8 @@ __global__ void k_norm_finalize(const Plan* plan, const int32_t* skip) {
   if (mi >= h.n_mats) return;
   const MatDesc& md = h.mats[mi];
   float acc = 0.f;
-  for (int i = lane; i < md.mom_count; i += 32) acc += h.partials[md.mom_begin + i];
+  const float* part = h.partials + (int64_t)kMomSlots * md.mom_begin;
+  for (int i = lane; i < kMomSlots * md.mom_count; i += 32) acc += part[i];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) {

@@ -63,7 +63,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
 
 // ---- kernels
 __global__ void k_plan_upload(const __grid_constant__ UploadChunk c);
-__global__ void k_momentum(const Plan* plan, const int32_t* skip);
+__global__ void k_momentum(const Plan* plan, const int32_t* skip);  // 256 threads per CTA
+constexpr int kMomSlots = 8;  // sum-of-squares partials per 64x64 momentum tile (one per warp of k_momentum)
 __global__ void k_norm_finalize(const Plan* plan, const int32_t* skip);
 cudaError_t launch_vote_update(const EwTable& tb, bool popcount, int grid, int sms, cudaStream_t s);
 bool bits_tma_eligible(const EwTable& tb);  // the 1-bit vote of this launch takes its bulk-copy form

@@ -126,7 +126,7 @@ struct PlanHeader {
   int32_t pad_pair;
   int32_t total_tiles[ST_COUNT];
   int32_t sym_ratio[ST_COUNT];  // BN / BM of the symmetric stages' tiles (1 or 2)
-  float* partials;          // [total_mom_tiles] sum of squares per momentum tile
+  float* partials;          // [total_mom_tiles][8] sum of squares per momentum tile and warp
   float* scale;             // [n_mats] s = 1/(||M||_F + eps)
   float* probe_partials;    // [total PROBE tiles]
   const int32_t* mom_begin; // [n_mats + 1] first momentum tile of each matrix (compact, for the tile search)
