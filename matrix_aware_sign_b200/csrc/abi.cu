@@ -935,10 +935,8 @@ smuon_status run_ns(const NsExec& ex, const int32_t* skip, cudaStream_t s) {
       k_momentum<<<std::max(grid, 1), 256, 0, s>>>(ex.d_plan, skip);
       CUDA_TRY(cudaGetLastError());
     }
-    const int warps_per_block = 8;
     Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * kMomSlots * h.total_mom_tiles, s);
-    k_norm_finalize<<<(h.n_mats + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(ex.d_plan,
-                                                                                                          skip);
+    k_norm_finalize<<<std::max(h.n_mats, 1), 256, 0, s>>>(ex.d_plan, skip);
     CUDA_TRY(cudaGetLastError());
   }
   const bool emit_q = (ex.flags & SMUON_NS_EMIT_Q) != 0;
@@ -1403,8 +1401,8 @@ smuon_status cachemuon_reuse_probe(const smuon_mat* Q, const smuon_mat* M_t, con
     CUDA_TRY(cudaGetLastError());
   }
   {
-    Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * B.h.total_mom_tiles, s);
-    k_norm_finalize<<<1, 32, 0, s>>>(d_plan, nullptr);
+    Launch L("k_norm_finalize", SMUON_WORK_BYTES, 4.0 * kMomSlots * B.h.total_mom_tiles, s);
+    k_norm_finalize<<<std::max(B.h.n_mats, 1), 256, 0, s>>>(d_plan, nullptr);
     CUDA_TRY(cudaGetLastError());
   }
   if ((st = launch_gemm(d_plan, B.h, ST_REUSE, 0, nullptr, di, s, stage_flops(B, ST_REUSE),

@@ -167,28 +167,36 @@ __global__ void __launch_bounds__(256, 4) k_momentum(const Plan* plan, const int
   }
 }
 
-// s = 1 / (||M||_F + eps) (reading R4); one warp per matrix, fixed order.
-__global__ void k_norm_finalize(const Plan* plan, const int32_t* skip) {
+// s = 1 / (||M||_F + eps) (reading R4): one 256-thread CTA per matrix sums that matrix's per-warp tile
+// partials, each thread a fixed strided share, then a fixed-order block reduction (deterministic).
+__global__ void __launch_bounds__(256) k_norm_finalize(const Plan* plan, const int32_t* skip) {
   if (skip && *skip) return;
   const PlanHeader& h = plan->h;
-  const int mi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (mi >= h.n_mats) return;
+  const int mi = blockIdx.x;
+  if (mi >= h.n_mats) return;  // uniform over the CTA
+  __shared__ float red[8];
   const MatDesc& md = h.mats[mi];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float acc = 0.f;
   const float* part = h.partials + (int64_t)kMomSlots * md.mom_begin;
-  for (int i = lane; i < kMomSlots * md.mom_count; i += 32) acc += part[i];
+  const int n = kMomSlots * md.mom_count;
+  for (int i = threadIdx.x; i < n; i += 256) acc += part[i];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) {
-    float s = 1.f;
-    if (!(h.flags & SMUON_NS_NO_NORMALIZE)) s = 1.f / (sqrtf(acc) + h.eps);
-    if (!isfinite(acc) && h.status) atomicOr(h.status, SMUON_DEV_NONFINITE_NORM);
-    h.scale[mi] = s;
+  if (lane == 0) red[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    float sc = 1.f;
+    if (!(h.flags & SMUON_NS_NO_NORMALIZE)) sc = 1.f / (sqrtf(tot) + h.eps);
+    if (!isfinite(tot) && h.status) atomicOr(h.status, SMUON_DEV_NONFINITE_NORM);
+    h.scale[mi] = sc;
   }
-  if (md.u_dtype == SMUON_BITS) {  // the message's pad words (past the last entry's word) are zero
-    const int64_t n = (int64_t)md.rows * md.cols;  // a multiple of 32
-    const int64_t used = n >> 5, total = ((n + 127) >> 7) << 2;
+  if (warp == 0 && md.u_dtype == SMUON_BITS) {  // the message's pad words (past the last entry's word) are zero
+    const int64_t nn = (int64_t)md.rows * md.cols;  // a multiple of 32
+    const int64_t used = nn >> 5, total = ((nn + 127) >> 7) << 2;
     if (used + lane < total) reinterpret_cast<uint32_t*>(md.u_ptr)[used + lane] = 0u;
   }
 }
